@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200: prefill tokens/s and decode steps/s, with roofline.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+One step = one kda_chunk_fwd call over the prefill workload (B=1, H=32, T=8192, d=128; inputs
+resident in HBM).  The decode row (kda_decode_step over 256 sequences x 64 heads, 128x128 fp32
+states, 512 steps) is timed in the same run and reported under "decode".  Every rank runs its own
+independent batch (weak scaling, no collective on the data path); timing is on the device with
+CUDA events, max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this build) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s and decode steps/s on 1 B200; % of roofline"
+CHUNK = 64
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# DRAM traffic of the dominant kernel per launch, from an ncu capture (profiles/); it is
+# reported only while the kernel sources still hash to the value they had when captured.
+NCU_TRAFFIC = {}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="kda", choices=["kda", "reference"])
+    p.add_argument("--workload", default="prefill_B1_H32_T8192_d128")
+    p.add_argument("--decode-steps", type=int, default=512)
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---- algorithmic work (per (token, head) unless stated) -----------------------------------------
+
+def prefill_bytes(w) -> int:
+    per_th = 2 * (3 * w.d_k + w.d_v) + (2 * w.d_v if w.gate else 0) + 4 + 2 * w.d_v
+    states = w.num_seqs * w.H * w.d_k * w.d_v * 4
+    n_states = (1 if w.init_state != "none" else 0) + (1 if w.final_state else 0)
+    return w.total_tokens * w.H * per_th + n_states * states
+
+
+def prefill_flops(w) -> float:
+    C, dk, dv = CHUNK, w.d_k, w.d_v
+    per_th = 2.0 * (3 * dk * dv + (C + 1) / 2.0 * (3 * dk + 2 * dv) - dk + C * C / 6.0)
+    return w.total_tokens * w.H * per_th
+
+
+def decode_bytes(dw) -> int:
+    per_unit = 2 * dw.d_k * dw.d_v * 4 + 2 * (3 * dw.d_k + 2 * dw.d_v) + 4 + 2 * dw.d_v
+    return dw.N * dw.H * per_unit
+
+
+def decode_flops(dw) -> float:
+    return dw.N * dw.H * 7.0 * dw.d_k * dw.d_v
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        m = json.load(open(path))
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), float(m.get("bf16_tflops_sustained", m["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kda_chunkwise_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ---- clocks sampled during the timed regions (NVML, read-only) -----------------------------------
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._active = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return
+        self._t = threading.Thread(target=self._run, args=(period_s,), daemon=True)
+        self._t.start()
+
+    def _run(self, period):
+        while not self._stop.is_set():
+            if self._active.is_set():
+                try:
+                    self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                    self.reasons |= int(self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+                except Exception:
+                    pass
+            time.sleep(period)
+
+    def active(self, on: bool):
+        (self._active.set if on else self._active.clear)()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self._stop.set()
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---- the reference arm: the fp64 oracle on the host cores -------------------------------------
+
+def host_inputs_f64(inp, heads):
+    import numpy as np
+    h = lambda t: None if t is None else t[:, heads].detach().cpu().double().numpy()
+    S0 = inp["initial_state"]
+    return dict(q=h(inp["q"]), k=h(inp["k"]), v=h(inp["v"]), a=h(inp["a"]), beta=h(inp["beta"]),
+                gate=h(inp["gate"]), A_log=inp["A_log"][heads].cpu().double().numpy(),
+                cu=inp["cu_seqlens"].cpu().numpy().astype(np.int64),
+                S0=None if S0 is None else S0[:, heads].cpu().double().numpy())
+
+
+def oracle_step(x, threads):
+    import oracle
+    oracle.kda_fwd(x["q"], x["k"], x["v"], x["a"], x["beta"], x["A_log"], x["cu"], gate=x["gate"],
+                   S0=x["S0"], n_threads=threads)
+
+
+def oracle_sample(inp, w, target_s: float, threads: int):
+    """Pick how many heads (full sequences) one oracle pass covers so it takes about target_s."""
+    one = host_inputs_f64(inp, [0])
+    t0 = time.perf_counter()
+    oracle_step(one, 1)
+    per_head = max(time.perf_counter() - t0, 1e-6)
+    waves_budget = max(1, int(target_s / per_head))
+    heads = max(1, min(w.H, waves_budget * max(1, threads)))
+    return list(range(heads)), per_head
+
+
+def cpu_baseline(inp, w, target_s=15.0):
+    threads = len(os.sched_getaffinity(0))
+    heads, _ = oracle_sample(inp, w, target_s, threads)
+    x = host_inputs_f64(inp, heads)
+    used = min(threads, len(heads) * w.num_seqs)
+    t0 = time.perf_counter()
+    oracle_step(x, used)
+    dt = time.perf_counter() - t0
+    tokens = w.total_tokens * len(heads) / w.H
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{len(heads)} of {w.H} heads x all {w.total_tokens} tokens of {w.name} "
+                      f"(fp64 token-by-token recurrence, {dt:.2f} s wall)"}
+
+
+def run_reference(args):
+    import torch
+
+    import kda_inputs as KI
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = KI.WORKLOADS[args.workload]
+    inp = KI.make_inputs(w, "cpu")
+    threads = len(os.sched_getaffinity(0))
+    heads, per_head = oracle_sample(inp, w, target_s=2.0, threads=threads)
+    x = host_inputs_f64(inp, heads)
+    used = min(threads, len(heads) * w.num_seqs)
+    for _ in range(args.warmup):
+        oracle_step(x, used)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(x, used)
+    dt = (time.perf_counter() - t0) / args.steps
+    tokens = w.total_tokens * len(heads) / w.H
+    value = tokens / dt
+    sample = (f"{len(heads)} of {w.H} heads x all {w.total_tokens} tokens of {w.name} per step "
+              f"(fp64 oracle; throughput scaled to whole tokens of all heads)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.num_seqs, "H": w.H, "T": w.total_tokens,
+                   "d_k": w.d_k, "d_v": w.d_v},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+    return 0
+
+
+# ---- the CUDA arm ------------------------------------------------------------------------------
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    import kda_chunkwise_b200 as kda
+    import kda_inputs as KI
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = KI.WORKLOADS[args.workload].replace(seed=KI.WORKLOADS[args.workload].seed + rank)
+    inp = KI.make_inputs(w, dev)
+    max_seqlen = max(w.seqlens)
+    ws_bytes = kda.kda_chunk_fwd_workspace_size(w.total_tokens, w.num_seqs, max_seqlen, w.H,
+                                                w.d_k, w.d_v)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((w.total_tokens, w.H, w.d_v), dtype=torch.bfloat16, device=dev)
+    S_final = torch.empty((w.num_seqs, w.H, w.d_k, w.d_v), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"],
+                          inp["cu_seqlens"], gate=inp["gate"], initial_state=inp["initial_state"],
+                          out=out, final_state=S_final, max_seqlen=max_seqlen,
+                          workspace=workspace, stream=stream)
+
+    clocks = ClockSampler(dev)
+    for _ in range(args.warmup):
+        step()
+    kda.kda_sync_check()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = kda.kda_launch_count()
+    clocks.active(True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.active(False)
+    launches = kda.kda_launch_count() - launches0
+    barrier()
+    kda.kda_sync_check()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    value = w.total_tokens * world / (ms * 1e-3)
+
+    hbm, tf, tf_sus, peak_src = peaks()
+    bytes_step = prefill_bytes(w)
+    flops_step = prefill_flops(w)
+    achieved = bytes_step / (ms * 1e-3) / 1e9
+    src_hash = kernel_source_hash()
+    traffic = NCU_TRAFFIC.get(w.name)
+    traffic_val = traffic["bytes_per_launch"] if traffic and traffic.get("src") == src_hash else None
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic_val,
+                "peak_source": f"hbm_gbs of {peak_src}",
+                "scope": "one kda_chunk_fwd call (all kernels of the prefill path)",
+                "algorithmic_bytes": bytes_step, "algorithmic_flops": flops_step,
+                "tensor_frac_of_bf16_peak": flops_step / (ms * 1e-3) / 1e12 / tf}
+
+    # decode row: 512 back-to-back steps over fixed states (each step reads and writes 1.07 GB)
+    decode = None
+    if not args.no_decode:
+        dw = dataclasses.replace(KI.DECODE, seed=KI.DECODE.seed + rank, steps=args.decode_steps)
+        d = KI.make_decode_inputs(dw, dev)
+        state = d["state"].clone()
+        dout = torch.empty((dw.N, dw.H, dw.d_v), dtype=torch.bfloat16, device=dev)
+
+        def dstep(t):
+            kda.kda_decode_step(d["q"][t], d["k"][t], d["v"][t], d["a"][t], d["beta"][t],
+                                d["A_log"], state, gate=d["gate"][t], out=dout, stream=stream)
+
+        for t in range(max(3, args.warmup)):
+            dstep(t % dw.steps)
+        state.copy_(d["state"])
+        barrier()
+        clocks.active(True)
+        e0.record(stream)
+        for t in range(dw.steps):
+            dstep(t)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.active(False)
+        barrier()
+        kda.kda_sync_check()
+        dms = max_over_ranks(e0.elapsed_time(e1) / dw.steps)
+        dbytes = decode_bytes(dw)
+        dach = dbytes / (dms * 1e-3) / 1e9
+        decode = {"value": world / (dms * 1e-3), "unit": "steps/s", "ms_per_step": dms,
+                  "workload": dw.name, "tokens_per_s": world * dw.N / (dms * 1e-3),
+                  "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
+                               "frac": dach / hbm, "traffic": None,
+                               "peak_source": f"hbm_gbs of {peak_src}",
+                               "algorithmic_bytes": dbytes}}
+        del d, state, dout
+        torch.cuda.empty_cache()
+
+    # end to end through the public API: pinned host inputs -> device -> kda_chunk_fwd -> host
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k", "v", "a", "beta", "gate", "A_log", "cu_seqlens", "initial_state"]
+        host_in = {n: inp[n].cpu().pin_memory() for n in names if inp[n] is not None}
+        dev_in = {n: torch.empty_like(inp[n]) for n in host_in}
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        S_h = torch.empty(S_final.shape, dtype=S_final.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = out_h.numel() * out_h.element_size() + S_h.numel() * S_h.element_size()
+
+        def e2e_step():
+            for n, t in host_in.items():
+                dev_in[n].copy_(t, non_blocking=True)
+            kda.kda_chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["a"], dev_in["beta"],
+                              dev_in["A_log"], dev_in["cu_seqlens"], gate=dev_in.get("gate"),
+                              initial_state=dev_in.get("initial_state"), out=out,
+                              final_state=S_final, max_seqlen=max_seqlen, workspace=workspace,
+                              stream=stream)
+            out_h.copy_(out, non_blocking=True)
+            S_h.copy_(S_final, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        e2e = {"value": w.total_tokens * world / (ems * 1e-3), "unit": "tokens/s",
+               "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, w)
+
+    clk = clocks.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.num_seqs, "H": w.H, "T": w.total_tokens,
+                       "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "tile": 16,
+                       "parallelism": f"independent batch per rank x{world}",
+                       "l2": f"inputs larger than L2 ({bytes_step / 1e6:.0f} MB per step > 126 MB); no flush"},
+            "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": launches, "clocks": clk, "kernel_src": src_hash,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

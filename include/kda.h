@@ -1,0 +1,130 @@
+/*
+ * kda.h — C ABI of libkda, the B200 (sm_100a) implementation of the Kimi Delta Attention (KDA)
+ * gated delta-rule recurrence.
+ *
+ * The recurrence, per (sequence, head), with state S in R^{d_k x d_v} (row = key channel,
+ * column = value channel), for each token t:
+ *   g_t   = -5 * sigmoid(exp(A_h) * a_t)          per-key-channel log-decay in [-5, 0]
+ *   S     = Diag(exp(g_t)) S                      fade
+ *   S     = S + beta_t k_t (v_t - S^T k_t)^T      erase what k_t retrieves, write v_t
+ *   o_t   = S^T (scale * q_t)                     read (after the token's own write)
+ *   out_t = sigmoid(gate_t) (.) o_t               full-rank output gate
+ * Sources: "Review A · Sequence and depth", Free recall (fade, erase, write, then the read S^T q);
+ * "Kimi K3 · Lesson 3 of 14" (chunkwise form, 16-token tiles, g_min = -5 scaled-sigmoid decay of
+ * §2.1.1 eq. 5, full-rank output gate); "K3 Architecture Illustrated", §"Combining KDA and MLA",
+ * FIG 21 (retention first, then the delta update, then the query read).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, 16-byte aligned,
+ *     densely packed (row-major, innermost dimension last).  bf16 is IEEE bfloat16 stored as
+ *     uint16_t.  The caller owns every buffer; the library allocates nothing and keeps no state
+ *     between calls except one per-device error word (see kda_sync_check).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are asynchronous:
+ *     a KDA_OK return means the work was validated and enqueued.
+ *   - Argument errors are detected on the host before anything is enqueued and return
+ *     KDA_ERR_INVALID_ARG or KDA_ERR_UNSUPPORTED.  A launch failure returns KDA_ERR_CUDA.
+ *     Errors that can only be seen on the device (malformed cu_seqlens, a max_seqlen smaller
+ *     than a sequence) are recorded in the per-device error word and reported by
+ *     kda_sync_check; the affected outputs are then unspecified.  Kernels never trap.
+ *   - Supported head sizes: d_k, d_v in {64, 128}.  g_min = -5, chunk = 64 tokens and
+ *     tile = 16 tokens are compile-time constants.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* NULL required pointer, bad size, misaligned pointer, small workspace */
+    KDA_ERR_UNSUPPORTED = 2, /* d_k or d_v outside {64, 128} */
+    KDA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (reported by kda_sync_check) */
+} kda_status;
+
+/*
+ * kda_chunk_fwd — prefill over packed variable-length sequences, in the chunkwise form
+ * ("Kimi K3 · Lesson 3 of 14", CHUNKWISE diagram: O = (Gamma (.) Q) S + A V~, state carried
+ * sequentially between 64-token chunks, every 16-token tile a dense product thanks to the
+ * g_min = -5 bound).
+ *
+ * Layout: token-major, packed.  Sequence n owns tokens [cu_seqlens[n], cu_seqlens[n+1]).
+ *   q, k, a     bf16  [total_tokens, H, d_k]   query, key, decay logits
+ *   v           bf16  [total_tokens, H, d_v]
+ *   beta        fp32  [total_tokens, H]        write strength
+ *   gate        bf16  [total_tokens, H, d_v]   output-gate logits, or NULL for no gate
+ *   A_log       fp32  [H]                      per-head log-scale A_h of the decay mapping
+ *   cu_seqlens  int32 [num_seqs + 1]           device; 0 = cu[0] <= ... <= cu[num_seqs] = total_tokens
+ *   initial_state fp32 [num_seqs, H, d_k, d_v] or NULL (zeros)
+ *   final_state   fp32 [num_seqs, H, d_k, d_v] or NULL (not written); may alias initial_state
+ *   out         bf16  [total_tokens, H, d_v]
+ * max_seqlen: an upper bound on every sequence length (0 = use total_tokens).  It sizes the launch;
+ *   a sequence longer than it is reported through the error word.
+ * scale multiplies q.  workspace: device scratch of at least
+ *   kda_chunk_fwd_workspace_min(...) bytes, 256-byte aligned; a larger workspace (up to
+ *   kda_chunk_fwd_workspace_size(...)) lets the library process more chunks per launch.
+ * A zero-length sequence copies its initial state (or zeros) to final_state.
+ * total_tokens == 0 or num_seqs == 0 is valid and only writes final_state.
+ */
+KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *a,
+                         const float *beta, const void *gate, const float *A_log,
+                         const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                         int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                         const float *initial_state, float *final_state, void *out,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* Recommended workspace for kda_chunk_fwd (host-only; 0 on invalid sizes). */
+KDA_API size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
+                                    int32_t H, int32_t d_k, int32_t d_v);
+
+/* Smallest workspace kda_chunk_fwd accepts for these sizes (host-only; 0 on invalid sizes). */
+KDA_API size_t kda_chunk_fwd_workspace_min(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
+                                   int32_t H, int32_t d_k, int32_t d_v);
+
+/*
+ * kda_decode_step — one recurrent step for N independent sequences, state updated in place
+ * (the fixed-size decode state of "K3 Architecture Illustrated", FIG 22: the state's shape does
+ * not grow with the context).
+ *   q, k, a     bf16 [N, H, d_k]      v, gate bf16 [N, H, d_v] (gate may be NULL)
+ *   beta        fp32 [N, H]           A_log fp32 [H]
+ *   state       fp32 [N, H, d_k, d_v] read and overwritten with the new state
+ *   out         bf16 [N, H, d_v]
+ */
+KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *a,
+                           const float *beta, const void *gate, const float *A_log, float *state,
+                           void *out, int32_t N, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                           void *stream);
+
+/* Static description of a status code. */
+KDA_API const char *kda_status_string(kda_status status);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error word.  Returns
+ * KDA_ERR_CUDA if the stream reported a CUDA error, KDA_ERR_INVALID_ARG if a kernel found
+ * malformed cu_seqlens or a sequence longer than max_seqlen, KDA_ERR_TIMEOUT if a bounded wait
+ * gave up, else KDA_OK.
+ */
+KDA_API kda_status kda_sync_check(void *stream);
+
+/* Text of the most recent error seen by this thread's calls (never NULL; "" when none). */
+KDA_API const char *kda_last_error(void);
+
+/* Number of CUDA kernels this process has launched through libkda so far (all devices). */
+KDA_API uint64_t kda_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,188 @@
+"""kda_chunkwise_b200 — Python binding of libkda (the KDA gated delta-rule recurrence on B200).
+
+Argument marshalling only: every step of the recurrence runs in the CUDA kernels of libkda.so,
+reached through its C ABI (include/kda.h).  PyTorch provides device memory and streams.  There is
+no CPU or PyTorch fallback: importing this package without the built library raises ImportError.
+
+Entry points (same names as the C ABI):
+  kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, ...)  prefill, chunkwise form
+  kda_decode_step(q, k, v, a, beta, A_log, state, ...)      one recurrent step, state in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
+           "kda_chunk_fwd_workspace_min", "kda_sync_check", "kda_status_string", "KDAError",
+           "kda_launch_count",
+           "LIB_PATH", "lib"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {kda_status_string(status)}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkda.so is not built ({LIB_PATH}); run `python -m "
+                          "kda_chunkwise_b200.build` (nvcc 12.9, sm_100a) first")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, fp, i32, i64, sz, f32 = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                 ctypes.c_int64, ctypes.c_size_t, ctypes.c_float)
+    L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, fp, vp, fp, vp, i32, i64, i32, i32, i32, i32, f32,
+                                fp, fp, vp, vp, sz, vp]
+    L.kda_chunk_fwd.restype = ctypes.c_int
+    L.kda_chunk_fwd_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+    L.kda_chunk_fwd_workspace_size.restype = sz
+    L.kda_chunk_fwd_workspace_min.argtypes = [i64, i32, i32, i32, i32, i32]
+    L.kda_chunk_fwd_workspace_min.restype = sz
+    L.kda_decode_step.argtypes = [vp, vp, vp, vp, fp, vp, fp, fp, vp, i32, i32, i32, i32, f32, vp]
+    L.kda_decode_step.restype = ctypes.c_int
+    L.kda_status_string.argtypes = [ctypes.c_int]
+    L.kda_status_string.restype = ctypes.c_char_p
+    L.kda_sync_check.argtypes = [vp]
+    L.kda_sync_check.restype = ctypes.c_int
+    L.kda_last_error.argtypes = []
+    L.kda_last_error.restype = ctypes.c_char_p
+    L.kda_launch_count.argtypes = []
+    L.kda_launch_count.restype = ctypes.c_uint64
+    return L
+
+
+lib = _load()
+
+
+def kda_status_string(status: int) -> str:
+    return lib.kda_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != KDA_OK:
+        raise KDAError(status, where, lib.kda_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, shape, device):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def kda_chunk_fwd_workspace_size(total_tokens, num_seqs, max_seqlen, H, d_k, d_v) -> int:
+    return int(lib.kda_chunk_fwd_workspace_size(total_tokens, num_seqs, max_seqlen, H, d_k, d_v))
+
+
+def kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v) -> int:
+    return int(lib.kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v))
+
+
+def kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None,
+                  output_final_state: bool = True, scale: float = 1.0, max_seqlen: int | None = None,
+                  out=None, final_state=None, workspace=None, stream=None):
+    """Chunkwise prefill over packed sequences (see include/kda.h for the full contract).
+
+    q, k, a [T, H, d_k] bf16; v, gate [T, H, d_v] bf16; beta [T, H] fp32; A_log [H] fp32;
+    cu_seqlens [N+1] int32 (device); initial_state [N, H, d_k, d_v] fp32 or None.
+    max_seqlen: longest sequence (None: computed from cu_seqlens with one device->host copy).
+    Returns (out [T, H, d_v] bf16, final_state [N, H, d_k, d_v] fp32 or None).
+    """
+    dev = q.device
+    T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    bf = torch.bfloat16
+    for name, t, shp in (("q", q, (T, H, d_k)), ("k", k, (T, H, d_k)), ("a", a, (T, H, d_k)),
+                         ("v", v, (T, H, d_v))):
+        _need(t, name, bf, shp, dev)
+    _need(beta, "beta", torch.float32, (T, H), dev)
+    _need(A_log, "A_log", torch.float32, (H,), dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+    if gate is not None:
+        _need(gate, "gate", bf, (T, H, d_v), dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, (N, H, d_k, d_v), dev)
+    if out is None:
+        out = torch.empty((T, H, d_v), dtype=bf, device=dev)
+    _need(out, "out", bf, (T, H, d_v), dev)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, (N, H, d_k, d_v), dev)
+    if max_seqlen is None:
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if N > 0 else 0
+    if workspace is None:
+        nbytes = kda_chunk_fwd_workspace_size(T, N, max_seqlen, H, d_k, d_v)
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate),
+                           _ptr(A_log), _ptr(cu_seqlens), N, T, int(max_seqlen), H, d_k, d_v,
+                           float(scale), _ptr(initial_state), _ptr(final_state), _ptr(out),
+                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                           _stream_handle(stream, dev))
+    _check(st, "kda_chunk_fwd")
+    return out, final_state
+
+
+def kda_decode_step(q, k, v, a, beta, A_log, state, gate=None, scale: float = 1.0, out=None,
+                    stream=None):
+    """One recurrent step for N sequences; ``state`` [N, H, d_k, d_v] fp32 is updated in place.
+
+    q, k, a [N, H, d_k] bf16; v, gate [N, H, d_v] bf16; beta [N, H] fp32; A_log [H] fp32.
+    Returns out [N, H, d_v] bf16.
+    """
+    dev = q.device
+    N, H, d_k = q.shape
+    d_v = v.shape[-1]
+    bf = torch.bfloat16
+    for name, t, shp in (("q", q, (N, H, d_k)), ("k", k, (N, H, d_k)), ("a", a, (N, H, d_k)),
+                         ("v", v, (N, H, d_v))):
+        _need(t, name, bf, shp, dev)
+    _need(beta, "beta", torch.float32, (N, H), dev)
+    _need(A_log, "A_log", torch.float32, (H,), dev)
+    _need(state, "state", torch.float32, (N, H, d_k, d_v), dev)
+    if gate is not None:
+        _need(gate, "gate", bf, (N, H, d_v), dev)
+    if out is None:
+        out = torch.empty((N, H, d_v), dtype=bf, device=dev)
+    _need(out, "out", bf, (N, H, d_v), dev)
+    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate),
+                             _ptr(A_log), _ptr(state), _ptr(out), N, H, d_k, d_v, float(scale),
+                             _stream_handle(stream, dev))
+    _check(st, "kda_decode_step")
+    return out
+
+
+def kda_launch_count() -> int:
+    """Kernels launched through libkda by this process so far."""
+    return int(lib.kda_launch_count())
+
+
+def kda_sync_check(stream=None, device=None) -> None:
+    """Synchronise the stream and raise KDAError if a kernel recorded a device-side error."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _check(lib.kda_sync_check(_stream_handle(stream, dev)), "kda_sync_check")

@@ -1,0 +1,97 @@
+"""The C ABI library: it builds, loads, exports every symbol that include/kda.h declares, and
+rejects bad arguments on the host before touching a GPU.  CPU only (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+from kda_chunkwise_b200 import build as kbuild  # noqa: E402
+
+kbuild.build()
+import kda_chunkwise_b200 as kda  # noqa: E402
+
+lib = kda.lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for must in ("kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
+                 "kda_chunk_fwd_workspace_min", "kda_status_string", "kda_sync_check",
+                 "kda_last_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    raw = ctypes.CDLL(kda.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), f"libkda.so does not export {name}"
+
+
+def test_status_strings():
+    for code in range(5):
+        assert kda.kda_status_string(code)
+    assert kda.kda_status_string(0) == "ok"
+
+
+def test_workspace_sizes():
+    mn = kda.kda_chunk_fwd_workspace_min(8192, 1, 8192, 32, 128, 128)
+    rec = kda.kda_chunk_fwd_workspace_size(8192, 1, 8192, 32, 128, 128)
+    assert 0 < mn <= rec
+    assert rec % 256 == 0 and mn % 256 == 0
+    assert kda.kda_chunk_fwd_workspace_size(8192, 1, 8192, 32, 96, 128) == 0   # unsupported d_k
+    assert kda.kda_chunk_fwd_workspace_size(-1, 1, 0, 32, 128, 128) == 0
+    # a short batch never asks for more than its own chunks
+    small = kda.kda_chunk_fwd_workspace_size(64, 1, 64, 2, 64, 64)
+    assert small == kda.kda_chunk_fwd_workspace_min(64, 1, 64, 2, 64, 64)
+
+
+def _fwd(**over):
+    base = dict(q=16, k=16, v=16, a=16, beta=16, gate=None, A_log=16, cu=16, N=1, T=64,
+                max_seqlen=64, H=2, dk=64, dv=64, scale=1.0, S0=None, SF=None, out=16,
+                ws=256, ws_bytes=1 << 30, stream=None)
+    base.update(over)
+    b = base
+    return lib.kda_chunk_fwd(b["q"], b["k"], b["v"], b["a"], b["beta"], b["gate"], b["A_log"],
+                             b["cu"], b["N"], b["T"], b["max_seqlen"], b["H"], b["dk"], b["dv"],
+                             b["scale"], b["S0"], b["SF"], b["out"], b["ws"], b["ws_bytes"],
+                             b["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dv=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(cu=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=24), kda.KDA_ERR_INVALID_ARG),          # misaligned
+    (dict(ws=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(ws=16 + 256), kda.KDA_ERR_INVALID_ARG),   # workspace must be 256-byte aligned
+    (dict(ws_bytes=1024), kda.KDA_ERR_INVALID_ARG),  # too small
+    (dict(N=0, T=5), kda.KDA_ERR_INVALID_ARG),
+])
+def test_chunk_fwd_rejects_bad_arguments(over, code):
+    assert _fwd(**over) == code
+    assert lib.kda_last_error().decode()
+
+
+def test_chunk_fwd_empty_batch_is_ok():
+    assert _fwd(N=0, T=0) == kda.KDA_OK
+
+
+def test_decode_rejects_bad_arguments():
+    f = lib.kda_decode_step
+    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 4, 0, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 4, 2, 128, 80, 1.0, None) == kda.KDA_ERR_UNSUPPORTED
+    assert f(None, 16, 16, 16, 16, None, 16, 16, 16, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, 8, 16, 16, 16, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 0, 2, 128, 128, 1.0, None) == kda.KDA_OK
