@@ -34,8 +34,8 @@ class KDAError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libkda.so is not built ({LIB_PATH}); run `python -m "
-                          "kda_chunkwise_b200.build` (nvcc 12.9, sm_100a) first")
+        raise ImportError(f"libkda.so is not built ({LIB_PATH}); run `python "
+                          "kda_chunkwise_b200/csrc/build.py` (nvcc 12.9, sm_100a) first")
     L = ctypes.CDLL(LIB_PATH)
     vp, fp, i32, i64, sz, f32 = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                  ctypes.c_int64, ctypes.c_size_t, ctypes.c_float)

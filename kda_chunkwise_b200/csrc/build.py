@@ -1,6 +1,8 @@
 """Build libkda.so (sm_100a) in-tree with nvcc.
 
-    python -m kda_chunkwise_b200.build [--verbose]
+    python kda_chunkwise_b200/csrc/build.py [--verbose]
+
+This script is run by path (it does not import the package, which loads the built library).
 
 The library is one CUDA translation unit (csrc/kda_lib.cu) plus headers; it links the CUDA
 runtime statically so it loads without any other CUDA library on the search path.
@@ -13,9 +15,9 @@ import shutil
 import subprocess
 import sys
 
-PKG = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.dirname(os.path.abspath(__file__))
+PKG = os.path.dirname(CSRC)
 ROOT = os.path.dirname(PKG)
-CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libkda.so")
 
@@ -32,6 +34,8 @@ def nvcc_path() -> str:
 def sources() -> list:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
                   [os.path.join(INCLUDE, "kda.h")])
+
+
 
 
 def needs_build() -> bool:

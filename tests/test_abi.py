@@ -9,9 +9,9 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "kda.h")
 
-from kda_chunkwise_b200 import build as kbuild  # noqa: E402
+import __graft_entry__  # noqa: E402
 
-kbuild.build()
+__graft_entry__._builder().build()
 import kda_chunkwise_b200 as kda  # noqa: E402
 
 lib = kda.lib
