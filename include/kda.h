@@ -15,9 +15,10 @@
  * FIG 21 (retention first, then the delta update, then the query read).
  *
  * Conventions for every entry point:
- *   - All tensor pointers are DEVICE pointers on the current CUDA device, 16-byte aligned,
- *     densely packed (row-major, innermost dimension last).  bf16 is IEEE bfloat16 stored as
- *     uint16_t.  The caller owns every buffer; the library allocates nothing and keeps no state
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, densely packed
+ *     (row-major, innermost dimension last).  Per-channel tensors (q, k, v, a, gate, out, states)
+ *     must be 16-byte aligned; beta, A_log and cu_seqlens 4-byte aligned.  bf16 is IEEE bfloat16
+ *     stored as uint16_t.  The caller owns every buffer; the library allocates nothing and keeps no state
  *     between calls except one per-device error word (see kda_sync_check).
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are asynchronous:
  *     a KDA_OK return means the work was validated and enqueued.
@@ -53,6 +54,12 @@ typedef enum kda_status {
     KDA_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (reported by kda_sync_check) */
 } kda_status;
 
+/* Storage type of the output o.  The recurrence itself is computed in fp32 either way. */
+typedef enum kda_dtype {
+    KDA_DTYPE_BF16 = 0,
+    KDA_DTYPE_F32 = 1
+} kda_dtype;
+
 /*
  * kda_chunk_fwd — prefill over packed variable-length sequences, in the chunkwise form
  * ("Kimi K3 · Lesson 3 of 14", CHUNKWISE diagram: O = (Gamma (.) Q) S + A V~, state carried
@@ -68,7 +75,7 @@ typedef enum kda_status {
  *   cu_seqlens  int32 [num_seqs + 1]           device; 0 = cu[0] <= ... <= cu[num_seqs] = total_tokens
  *   initial_state fp32 [num_seqs, H, d_k, d_v] or NULL (zeros)
  *   final_state   fp32 [num_seqs, H, d_k, d_v] or NULL (not written); may alias initial_state
- *   out         bf16  [total_tokens, H, d_v]
+ *   out         [total_tokens, H, d_v] of out_dtype (bf16 or fp32)
  * max_seqlen: an upper bound on every sequence length (0 = use total_tokens).  It sizes the launch;
  *   a sequence longer than it is reported through the error word.
  * scale multiplies q.  workspace: device scratch of at least
@@ -82,7 +89,8 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, co
                          const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                          int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v, float scale,
                          const float *initial_state, float *final_state, void *out,
-                         void *workspace, size_t workspace_bytes, void *stream);
+                         kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                         void *stream);
 
 /* Recommended workspace for kda_chunk_fwd (host-only; 0 on invalid sizes). */
 KDA_API size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
@@ -99,12 +107,12 @@ KDA_API size_t kda_chunk_fwd_workspace_min(int64_t total_tokens, int32_t num_seq
  *   q, k, a     bf16 [N, H, d_k]      v, gate bf16 [N, H, d_v] (gate may be NULL)
  *   beta        fp32 [N, H]           A_log fp32 [H]
  *   state       fp32 [N, H, d_k, d_v] read and overwritten with the new state
- *   out         bf16 [N, H, d_v]
+ *   out         [N, H, d_v] of out_dtype (bf16 or fp32)
  */
 KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *a,
                            const float *beta, const void *gate, const float *A_log, float *state,
-                           void *out, int32_t N, int32_t H, int32_t d_k, int32_t d_v, float scale,
-                           void *stream);
+                           void *out, kda_dtype out_dtype, int32_t N, int32_t H, int32_t d_k,
+                           int32_t d_v, float scale, void *stream);
 
 /* Static description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);

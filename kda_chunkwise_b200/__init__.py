@@ -23,6 +23,8 @@ __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_DTYPE_BF16, KDA_DTYPE_F32 = 0, 1
+_OUT_DTYPES = {torch.bfloat16: KDA_DTYPE_BF16, torch.float32: KDA_DTYPE_F32}
 
 
 class KDAError(RuntimeError):
@@ -40,13 +42,14 @@ def _load() -> ctypes.CDLL:
     vp, fp, i32, i64, sz, f32 = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                  ctypes.c_int64, ctypes.c_size_t, ctypes.c_float)
     L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, fp, vp, fp, vp, i32, i64, i32, i32, i32, i32, f32,
-                                fp, fp, vp, vp, sz, vp]
+                                fp, fp, vp, ctypes.c_int, vp, sz, vp]
     L.kda_chunk_fwd.restype = ctypes.c_int
     L.kda_chunk_fwd_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
     L.kda_chunk_fwd_workspace_size.restype = sz
     L.kda_chunk_fwd_workspace_min.argtypes = [i64, i32, i32, i32, i32, i32]
     L.kda_chunk_fwd_workspace_min.restype = sz
-    L.kda_decode_step.argtypes = [vp, vp, vp, vp, fp, vp, fp, fp, vp, i32, i32, i32, i32, f32, vp]
+    L.kda_decode_step.argtypes = [vp, vp, vp, vp, fp, vp, fp, fp, vp, ctypes.c_int, i32, i32, i32,
+                                  i32, f32, vp]
     L.kda_decode_step.restype = ctypes.c_int
     L.kda_status_string.argtypes = [ctypes.c_int]
     L.kda_status_string.restype = ctypes.c_char_p
@@ -104,13 +107,15 @@ def kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v)
 
 def kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None,
                   output_final_state: bool = True, scale: float = 1.0, max_seqlen: int | None = None,
-                  out=None, final_state=None, workspace=None, stream=None):
+                  out=None, final_state=None, workspace=None, stream=None,
+                  out_dtype=torch.bfloat16):
     """Chunkwise prefill over packed sequences (see include/kda.h for the full contract).
 
     q, k, a [T, H, d_k] bf16; v, gate [T, H, d_v] bf16; beta [T, H] fp32; A_log [H] fp32;
     cu_seqlens [N+1] int32 (device); initial_state [N, H, d_k, d_v] fp32 or None.
     max_seqlen: longest sequence (None: computed from cu_seqlens with one device->host copy).
-    Returns (out [T, H, d_v] bf16, final_state [N, H, d_k, d_v] fp32 or None).
+    out_dtype: storage of the output, torch.bfloat16 or torch.float32 (taken from ``out`` if given).
+    Returns (out [T, H, d_v], final_state [N, H, d_k, d_v] fp32 or None).
     """
     dev = q.device
     T, H, d_k = q.shape
@@ -128,8 +133,10 @@ def kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=
     if initial_state is not None:
         _need(initial_state, "initial_state", torch.float32, (N, H, d_k, d_v), dev)
     if out is None:
-        out = torch.empty((T, H, d_v), dtype=bf, device=dev)
-    _need(out, "out", bf, (T, H, d_v), dev)
+        out = torch.empty((T, H, d_v), dtype=out_dtype, device=dev)
+    if out.dtype not in _OUT_DTYPES:
+        raise TypeError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, (T, H, d_v), dev)
     if output_final_state and final_state is None:
         final_state = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=dev)
     if final_state is not None:
@@ -142,18 +149,18 @@ def kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=
     st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate),
                            _ptr(A_log), _ptr(cu_seqlens), N, T, int(max_seqlen), H, d_k, d_v,
                            float(scale), _ptr(initial_state), _ptr(final_state), _ptr(out),
-                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                           _OUT_DTYPES[out.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream_handle(stream, dev))
     _check(st, "kda_chunk_fwd")
     return out, final_state
 
 
 def kda_decode_step(q, k, v, a, beta, A_log, state, gate=None, scale: float = 1.0, out=None,
-                    stream=None):
+                    stream=None, out_dtype=torch.bfloat16):
     """One recurrent step for N sequences; ``state`` [N, H, d_k, d_v] fp32 is updated in place.
 
     q, k, a [N, H, d_k] bf16; v, gate [N, H, d_v] bf16; beta [N, H] fp32; A_log [H] fp32.
-    Returns out [N, H, d_v] bf16.
+    Returns out [N, H, d_v] (bfloat16 or float32, see kda_chunk_fwd).
     """
     dev = q.device
     N, H, d_k = q.shape
@@ -168,10 +175,13 @@ def kda_decode_step(q, k, v, a, beta, A_log, state, gate=None, scale: float = 1.
     if gate is not None:
         _need(gate, "gate", bf, (N, H, d_v), dev)
     if out is None:
-        out = torch.empty((N, H, d_v), dtype=bf, device=dev)
-    _need(out, "out", bf, (N, H, d_v), dev)
+        out = torch.empty((N, H, d_v), dtype=out_dtype, device=dev)
+    if out.dtype not in _OUT_DTYPES:
+        raise TypeError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, (N, H, d_v), dev)
     st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate),
-                             _ptr(A_log), _ptr(state), _ptr(out), N, H, d_k, d_v, float(scale),
+                             _ptr(A_log), _ptr(state), _ptr(out), _OUT_DTYPES[out.dtype], N, H,
+                             d_k, d_v, float(scale),
                              _stream_handle(stream, dev))
     _check(st, "kda_decode_step")
     return out

@@ -40,6 +40,12 @@ __device__ __forceinline__ uint16_t f32_to_bf16(float x) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
+// Stores one output element in the caller's storage type (fp32 or bf16).
+__device__ __forceinline__ void store_out(void *out, int64_t off, bool f32, float x) {
+    if (f32) static_cast<float *>(out)[off] = x;
+    else static_cast<uint16_t *>(out)[off] = f32_to_bf16(x);
+}
+
 // sigmoid with the fast exponential; saturates cleanly (no NaN) for |x| -> inf.
 __device__ __forceinline__ float sigmoid_fast(float x) { return 1.0f / (1.0f + __expf(-x)); }
 

@@ -21,8 +21,9 @@ struct DecodeParams {
     const uint16_t *q, *k, *v, *a, *gate;
     const float *beta, *A_log;
     float *state;
-    uint16_t *out;
+    void *out;
     int H;
+    bool out_f32;
     float scale;
 };
 
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const DecodeParams p) 
         s_u[tid] = u;
         float o = fmaf(s_kq, u, pp);
         if (p.gate) o *= sigmoid_fast(bf16_to_f32(p.gate[off]));
-        p.out[off] = f32_to_bf16(o);
+        store_out(p.out, off, p.out_f32, o);
     }
     __syncthreads();
 

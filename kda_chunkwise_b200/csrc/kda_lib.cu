@@ -27,7 +27,7 @@ kda_status cuda_fail(cudaError_t e, const char *where) {
     return fail(KDA_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 bool supported_dim(int d) { return d == 64 || d == 128; }
 
@@ -136,7 +136,8 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
                          const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                          int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v, float scale,
                          const float *initial_state, float *final_state, void *out,
-                         void *workspace, size_t workspace_bytes, void *stream) {
+                         kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                         void *stream) {
     if (!sizes_ok(total_tokens, num_seqs, max_seqlen, H))
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: negative size or H <= 0");
     if (!supported_dim(d_k) || !supported_dim(d_v))
@@ -148,9 +149,14 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     if (!cu_seqlens || !A_log) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: NULL cu_seqlens or A_log");
     if (total_tokens > 0 && (!q || !k || !v || !a || !beta || !out))
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: NULL q/k/v/a/beta/out");
-    const void *ptrs[] = {q, k, v, a, beta, gate, A_log, cu_seqlens, initial_state, final_state, out, workspace};
+    if (out_dtype != KDA_DTYPE_BF16 && out_dtype != KDA_DTYPE_F32)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: out_dtype must be KDA_DTYPE_BF16 or KDA_DTYPE_F32");
+    const void *ptrs[] = {q, k, v, a, gate, initial_state, final_state, out, workspace};
     for (const void *ptr : ptrs)
-        if (ptr && !aligned16(ptr)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: pointer not 16-byte aligned");
+        if (ptr && !aligned(ptr, 16)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: tensor pointer not 16-byte aligned");
+    const void *ptrs4[] = {beta, A_log, cu_seqlens};
+    for (const void *ptr : ptrs4)
+        if (ptr && !aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: beta/A_log/cu_seqlens not 4-byte aligned");
     if (!workspace) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: NULL workspace");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: workspace not 256-byte aligned");
@@ -186,7 +192,8 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     kda::StateParams sp{};
     sp.rec = pp.rec;
     sp.gate = static_cast<const uint16_t *>(gate);
-    sp.out = static_cast<uint16_t *>(out);
+    sp.out = out;
+    sp.out_f32 = out_dtype == KDA_DTYPE_F32;
     sp.cu = cu_seqlens;
     sp.S_in = initial_state;
     sp.S_out = run;
@@ -204,17 +211,22 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *a,
                            const float *beta, const void *gate, const float *A_log, float *state,
-                           void *out, int32_t N, int32_t H, int32_t d_k, int32_t d_v, float scale,
-                           void *stream) {
+                           void *out, kda_dtype out_dtype, int32_t N, int32_t H, int32_t d_k,
+                           int32_t d_v, float scale, void *stream) {
     if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: N < 0 or H <= 0");
     if (!supported_dim(d_k) || !supported_dim(d_v))
         return fail(KDA_ERR_UNSUPPORTED, "kda_decode_step: d_k and d_v must be 64 or 128");
     if (N == 0) return KDA_OK;
     if (!q || !k || !v || !a || !beta || !A_log || !state || !out)
         return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: NULL required pointer");
-    const void *ptrs[] = {q, k, v, a, beta, gate, A_log, state, out};
+    if (out_dtype != KDA_DTYPE_BF16 && out_dtype != KDA_DTYPE_F32)
+        return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: out_dtype must be KDA_DTYPE_BF16 or KDA_DTYPE_F32");
+    const void *ptrs[] = {q, k, v, a, gate, state, out};
     for (const void *ptr : ptrs)
-        if (ptr && !aligned16(ptr)) return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: pointer not 16-byte aligned");
+        if (ptr && !aligned(ptr, 16)) return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: tensor pointer not 16-byte aligned");
+    const void *ptrs4[] = {beta, A_log};
+    for (const void *ptr : ptrs4)
+        if (ptr && !aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: beta/A_log not 4-byte aligned");
     const int64_t units = (int64_t)N * H;
     if (units > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_decode_step: N*H too large");
     kda::DecodeParams p{};
@@ -226,7 +238,8 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     p.beta = beta;
     p.A_log = A_log;
     p.state = state;
-    p.out = static_cast<uint16_t *>(out);
+    p.out = out;
+    p.out_f32 = out_dtype == KDA_DTYPE_F32;
     p.H = H;
     p.scale = scale;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -174,12 +174,13 @@ __global__ void __launch_bounds__(256) prep_simt_kernel(const PrepParams p) {
 struct StateParams {
     const float *rec;
     const uint16_t *gate;
-    uint16_t *out;
+    void *out;
     const int32_t *cu;
     const float *S_in;
     float *S_out;
     int64_t total_tokens;
     int num_seqs, H, chunk0, Wc, max_chunks, first_window;
+    bool out_f32;
 };
 
 constexpr int kSlab = 32;  // d_v columns per state CTA
@@ -265,7 +266,7 @@ __global__ void __launch_bounds__(256) state_simt_kernel(const StateParams p) {
             if (i < L) {
                 const int64_t off = ((t0 + i) * H + h) * DV + col0 + j;
                 if (p.gate) acc *= sigmoid_fast(bf16_to_f32(p.gate[off]));
-                p.out[off] = f32_to_bf16(acc);
+                store_out(p.out, off, p.out_f32, acc);
             }
         }
         __syncthreads();

@@ -57,13 +57,13 @@ def test_workspace_sizes():
 def _fwd(**over):
     base = dict(q=16, k=16, v=16, a=16, beta=16, gate=None, A_log=16, cu=16, N=1, T=64,
                 max_seqlen=64, H=2, dk=64, dv=64, scale=1.0, S0=None, SF=None, out=16,
-                ws=256, ws_bytes=1 << 30, stream=None)
+                out_dtype=0, ws=256, ws_bytes=1 << 30, stream=None)
     base.update(over)
     b = base
     return lib.kda_chunk_fwd(b["q"], b["k"], b["v"], b["a"], b["beta"], b["gate"], b["A_log"],
                              b["cu"], b["N"], b["T"], b["max_seqlen"], b["H"], b["dk"], b["dv"],
-                             b["scale"], b["S0"], b["SF"], b["out"], b["ws"], b["ws_bytes"],
-                             b["stream"])
+                             b["scale"], b["S0"], b["SF"], b["out"], b["out_dtype"], b["ws"],
+                             b["ws_bytes"], b["stream"])
 
 
 @pytest.mark.parametrize("over,code", [
@@ -74,6 +74,8 @@ def _fwd(**over):
     (dict(q=None), kda.KDA_ERR_INVALID_ARG),
     (dict(cu=None), kda.KDA_ERR_INVALID_ARG),
     (dict(q=24), kda.KDA_ERR_INVALID_ARG),          # misaligned
+    (dict(beta=18), kda.KDA_ERR_INVALID_ARG),       # beta needs 4-byte alignment
+    (dict(out_dtype=7), kda.KDA_ERR_INVALID_ARG),
     (dict(ws=None), kda.KDA_ERR_INVALID_ARG),
     (dict(ws=16 + 256), kda.KDA_ERR_INVALID_ARG),   # workspace must be 256-byte aligned
     (dict(ws_bytes=1024), kda.KDA_ERR_INVALID_ARG),  # too small
@@ -86,12 +88,14 @@ def test_chunk_fwd_rejects_bad_arguments(over, code):
 
 def test_chunk_fwd_empty_batch_is_ok():
     assert _fwd(N=0, T=0) == kda.KDA_OK
+    assert _fwd(N=0, T=0, beta=20) == kda.KDA_OK   # 4-byte aligned beta is enough
 
 
 def test_decode_rejects_bad_arguments():
     f = lib.kda_decode_step
-    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 4, 0, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
-    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 4, 2, 128, 80, 1.0, None) == kda.KDA_ERR_UNSUPPORTED
-    assert f(None, 16, 16, 16, 16, None, 16, 16, 16, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
-    assert f(16, 16, 16, 16, 16, 8, 16, 16, 16, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
-    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 0, 2, 128, 128, 1.0, None) == kda.KDA_OK
+    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 0, 4, 0, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 0, 4, 2, 128, 80, 1.0, None) == kda.KDA_ERR_UNSUPPORTED
+    assert f(None, 16, 16, 16, 16, None, 16, 16, 16, 0, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, 8, 16, 16, 16, 0, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 5, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 0, 0, 2, 128, 128, 1.0, None) == kda.KDA_OK
