@@ -92,6 +92,33 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, co
                          kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
                          void *stream);
 
+/*
+ * kda_chunk_fwd_noalloc — kda_chunk_fwd for callers that cannot allocate device memory.
+ * (No counterpart in the pages: this is a deployment convenience, not part of the method.)
+ *
+ * Some callers cannot hand the library a workspace: their device memory belongs to someone else
+ * (a serving engine's pre-reserved pool, a runtime plugin whose enqueue path must not allocate),
+ * or they cannot afford the implicit synchronisation of cudaMalloc on a latency-critical path.
+ * This entry point takes the same arguments as kda_chunk_fwd minus the workspace and instead uses
+ * scratch memory built into the library: a 32 MiB device array that every GPU which loads
+ * libkda holds until the process exits.  It calls no cudaMalloc or cudaFree.
+ *   - The first call on a device looks up that array's device address (with that device current)
+ *     and caches it; make that first call before any stream capture.
+ *   - Sizes whose scratch need (kda_chunk_fwd_workspace_min) exceeds 32 MiB are rejected with
+ *     KDA_ERR_INVALID_ARG and a message in kda_last_error.  With d_k = d_v = 128 that allows
+ *     roughly 150 (sequence, head) units per call; longer sequences only take more launches.
+ *   - Every call on a device shares the one array and nothing in it needs to start at zero, but
+ *     calls that overlap on the GPU (different streams, or other threads) race on it: serialise
+ *     them, for example by issuing them all on one stream.
+ */
+KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *a,
+                                         const float *beta, const void *gate, const float *A_log,
+                                         const int32_t *cu_seqlens, int32_t num_seqs,
+                                         int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                                         int32_t d_k, int32_t d_v, float scale,
+                                         const float *initial_state, float *final_state, void *out,
+                                         kda_dtype out_dtype, void *stream);
+
 /* Recommended workspace for kda_chunk_fwd (host-only; 0 on invalid sizes). */
 KDA_API size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
                                     int32_t H, int32_t d_k, int32_t d_v);

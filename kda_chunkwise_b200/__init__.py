@@ -17,7 +17,7 @@ import torch
 
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_chunk_fwd_workspace_min", "kda_sync_check", "kda_status_string", "KDAError",
-           "kda_launch_count",
+           "kda_launch_count", "kda_chunk_fwd_noalloc",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -44,6 +44,9 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, fp, vp, fp, vp, i32, i64, i32, i32, i32, i32, f32,
                                 fp, fp, vp, ctypes.c_int, vp, sz, vp]
     L.kda_chunk_fwd.restype = ctypes.c_int
+    L.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, fp, vp, fp, vp, i32, i64, i32, i32, i32,
+                                        i32, f32, fp, fp, vp, ctypes.c_int, vp]
+    L.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     L.kda_chunk_fwd_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
     L.kda_chunk_fwd_workspace_size.restype = sz
     L.kda_chunk_fwd_workspace_min.argtypes = [i64, i32, i32, i32, i32, i32]
@@ -152,6 +155,44 @@ def kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=
                            _OUT_DTYPES[out.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream_handle(stream, dev))
     _check(st, "kda_chunk_fwd")
+    return out, final_state
+
+
+def kda_chunk_fwd_noalloc(q, k, v, a, beta, A_log, cu_seqlens, max_seqlen: int, gate=None,
+                          initial_state=None, scale: float = 1.0, out=None, final_state=None,
+                          stream=None):
+    """kda_chunk_fwd on the library's built-in 32 MiB scratch instead of a workspace.
+
+    For callers that cannot allocate device memory on this path: it allocates nothing (the
+    caller passes ``out`` and ``final_state`` if it wants them; ``out`` is required and its dtype,
+    bfloat16 or float32, selects the output storage).  Calls on one device share the scratch:
+    keep them on one stream.  max_seqlen must be given (no device-to-host read is made).
+    """
+    dev = q.device
+    T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    bf = torch.bfloat16
+    for name, t, shp in (("q", q, (T, H, d_k)), ("k", k, (T, H, d_k)), ("a", a, (T, H, d_k)),
+                         ("v", v, (T, H, d_v))):
+        _need(t, name, bf, shp, dev)
+    _need(beta, "beta", torch.float32, (T, H), dev)
+    _need(A_log, "A_log", torch.float32, (H,), dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+    if gate is not None:
+        _need(gate, "gate", bf, (T, H, d_v), dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, (N, H, d_k, d_v), dev)
+    if out is None or out.dtype not in _OUT_DTYPES:
+        raise ValueError("out (bfloat16 or float32, [T, H, d_v]) is required")
+    _need(out, "out", out.dtype, (T, H, d_v), dev)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, (N, H, d_k, d_v), dev)
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate),
+                                   _ptr(A_log), _ptr(cu_seqlens), N, T, int(max_seqlen), H, d_k,
+                                   d_v, float(scale), _ptr(initial_state), _ptr(final_state),
+                                   _ptr(out), _OUT_DTYPES[out.dtype], _stream_handle(stream, dev))
+    _check(st, "kda_chunk_fwd_noalloc")
     return out, final_state
 
 

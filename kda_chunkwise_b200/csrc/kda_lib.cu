@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
+#include <mutex>
 #include <cstring>
 #include <string>
 
@@ -92,6 +93,37 @@ kda_status launch_decode(const kda::DecodeParams &p, int64_t units, cudaStream_t
     g_launches.fetch_add(1, std::memory_order_relaxed);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "decode_step launch");
+}
+
+// Built-in scratch for kda_chunk_fwd_noalloc (callers that cannot allocate).  Host code must not
+// use this name as an address: it is a host-side stand-in; the device address comes from
+// cudaGetSymbolAddress, looked up once per device below.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_kda_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+kda_status static_scratch_address(void **ptr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_noalloc: device ordinal out of range");
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_kda_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetSymbolAddress");
+        g_scratch_ptr[dev] = p;
+    }
+    *ptr = g_scratch_ptr[dev];
+    return KDA_OK;
 }
 
 }  // namespace
@@ -207,6 +239,26 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     if (d_k == 128 && d_v == 64) return launch_chunk_fwd<128, 64>(pp, sp, windows, st);
     if (d_k == 64 && d_v == 128) return launch_chunk_fwd<64, 128>(pp, sp, windows, st);
     return launch_chunk_fwd<64, 64>(pp, sp, windows, st);
+}
+
+kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *a,
+                                 const float *beta, const void *gate, const float *A_log,
+                                 const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                 int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v,
+                                 float scale, const float *initial_state, float *final_state,
+                                 void *out, kda_dtype out_dtype, void *stream) {
+    const size_t need = kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
+    if (need > kStaticScratchBytes)
+        return fail(KDA_ERR_INVALID_ARG,
+                    "kda_chunk_fwd_noalloc: these sizes need " + std::to_string(need) +
+                        " bytes of scratch, more than the " + std::to_string(kStaticScratchBytes) +
+                        " built into the library; call kda_chunk_fwd with a workspace instead");
+    void *scratch = nullptr;
+    const kda_status st = static_scratch_address(&scratch);
+    if (st != KDA_OK) return st;
+    return kda_chunk_fwd(q, k, v, a, beta, gate, A_log, cu_seqlens, num_seqs, total_tokens,
+                         max_seqlen, H, d_k, d_v, scale, initial_state, final_state, out,
+                         out_dtype, scratch, kStaticScratchBytes, stream);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *a,
