@@ -76,11 +76,11 @@ typedef enum kda_dtype {
  *   initial_state fp32 [num_seqs, H, d_k, d_v] or NULL (zeros)
  *   final_state   fp32 [num_seqs, H, d_k, d_v] or NULL (not written); may alias initial_state
  *   out         [total_tokens, H, d_v] of out_dtype (bf16 or fp32)
- * max_seqlen: an upper bound on every sequence length (0 = use total_tokens).  It sizes the launch;
- *   a sequence longer than it is reported through the error word.
- * scale multiplies q.  workspace: device scratch of at least
- *   kda_chunk_fwd_workspace_min(...) bytes, 256-byte aligned; a larger workspace (up to
- *   kda_chunk_fwd_workspace_size(...)) lets the library process more chunks per launch.
+ * max_seqlen: an upper bound on every sequence length, or 0 for none.  A sequence longer than a
+ *   non-zero bound is reported through the error word (the result is still computed in full).
+ * scale multiplies q.  workspace: device scratch of at least kda_chunk_fwd_workspace_min(...)
+ *   bytes (equal to kda_chunk_fwd_workspace_size(...)), 256-byte aligned; it holds per-unit rings
+ *   of chunk records (about 0.55 MiB per (sequence, head) at d = 128) and is reused across calls.
  * A zero-length sequence copies its initial state (or zeros) to final_state.
  * total_tokens == 0 or num_seqs == 0 is valid and only writes final_state.
  */
@@ -106,7 +106,7 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, co
  *     and caches it; make that first call before any stream capture.
  *   - Sizes whose scratch need (kda_chunk_fwd_workspace_min) exceeds 32 MiB are rejected with
  *     KDA_ERR_INVALID_ARG and a message in kda_last_error.  With d_k = d_v = 128 that allows
- *     roughly 150 (sequence, head) units per call; longer sequences only take more launches.
+ *     58 (sequence, head) units per call, of any length.
  *   - Every call on a device shares the one array and nothing in it needs to start at zero, but
  *     calls that overlap on the GPU (different streams, or other threads) race on it: serialise
  *     them, for example by issuing them all on one stream.
@@ -119,11 +119,11 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const voi
                                          const float *initial_state, float *final_state, void *out,
                                          kda_dtype out_dtype, void *stream);
 
-/* Recommended workspace for kda_chunk_fwd (host-only; 0 on invalid sizes). */
+/* Workspace kda_chunk_fwd needs for these sizes (host-only; 0 on invalid sizes). */
 KDA_API size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
                                     int32_t H, int32_t d_k, int32_t d_v);
 
-/* Smallest workspace kda_chunk_fwd accepts for these sizes (host-only; 0 on invalid sizes). */
+/* Same value as kda_chunk_fwd_workspace_size (kept so callers can ask for the minimum by name). */
 KDA_API size_t kda_chunk_fwd_workspace_min(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
                                    int32_t H, int32_t d_k, int32_t d_v);
 

@@ -12,7 +12,7 @@
 #include "kda.h"
 #include "common.cuh"
 #include "decode.cuh"
-#include "prefill_simt.cuh"
+#include "prefill_fused.cuh"
 
 namespace {
 
@@ -34,56 +34,52 @@ bool supported_dim(int d) { return d == 64 || d == 128; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace of the chunkwise path: [running state | chunk records of one window].
-size_t record_bytes(int d_k, int d_v) {
-    const size_t floats = (size_t)kda::kChunk * (3 * d_k + d_v) + kda::kChunk * kda::kChunk + d_k;
-    return round_up(floats * 4, 256);
+// Workspace of the chunkwise path: [per-unit ring flags | per-unit rings of chunk records].
+size_t ring_slot_bytes(int d_k, int d_v) {
+    if (d_k == 128 && d_v == 128) return kda::RingLayout<128, 128>::kBytes;
+    if (d_k == 128 && d_v == 64) return kda::RingLayout<128, 64>::kBytes;
+    if (d_k == 64 && d_v == 128) return kda::RingLayout<64, 128>::kBytes;
+    return kda::RingLayout<64, 64>::kBytes;
 }
 
-size_t state_bytes(int32_t num_seqs, int32_t H, int d_k, int d_v) {
-    return round_up((size_t)num_seqs * H * d_k * d_v * 4, 256);
-}
+int ring_slots(int d_v) { return 2 * (d_v / kda::kSlab); }
 
-int64_t max_chunks_of(int64_t total_tokens, int32_t max_seqlen) {
-    const int64_t L = max_seqlen > 0 ? std::min<int64_t>(max_seqlen, total_tokens) : total_tokens;
-    return (L + kda::kChunk - 1) / kda::kChunk;
+size_t flag_bytes(int64_t units, int d_v) { return round_up((size_t)units * ring_slots(d_v) * 2 * 4, 256); }
+
+size_t ring_bytes(int64_t units, int d_k, int d_v) {
+    return (size_t)units * ring_slots(d_v) * ring_slot_bytes(d_k, d_v);
 }
 
 bool sizes_ok(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen, int32_t H) {
     return total_tokens >= 0 && num_seqs >= 0 && max_seqlen >= 0 && H > 0;
 }
 
-constexpr size_t kDefaultWindowBudget = size_t(1) << 30;  // bytes of chunk records per window
+constexpr unsigned long long kWaitNs = 4000000000ull;   // bound of every device-side wait (4 s)
 
 template <int DK, int DV>
-kda_status launch_chunk_fwd(const kda::PrepParams &pp0, const kda::StateParams &sp0,
-                            int64_t windows, cudaStream_t stream) {
-    const int prep_smem = kda::prep_smem_bytes<DK, DV>();
-    const int state_smem = kda::state_smem_bytes<DK, DV>();
-    cudaError_t e = cudaFuncSetAttribute(kda::prep_simt_kernel<DK, DV>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, prep_smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prep)");
-    e = cudaFuncSetAttribute(kda::state_simt_kernel<DK, DV>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, state_smem);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(state)");
-    const int num_seqs = sp0.num_seqs;
-    for (int64_t w = 0; w < windows; ++w) {
-        kda::PrepParams pp = pp0;
-        kda::StateParams sp = sp0;
-        pp.chunk0 = sp.chunk0 = static_cast<int>(w * pp0.Wc);
-        sp.first_window = w == 0;
-        if (w > 0) sp.S_in = sp.S_out;
-        if (sp0.max_chunks > 0) {
-            dim3 grid((unsigned)(num_seqs * pp.Wc), (unsigned)pp.H);
-            kda::prep_simt_kernel<DK, DV><<<grid, 256, prep_smem, stream>>>(pp);
-            g_launches.fetch_add(1, std::memory_order_relaxed);
-        }
-        dim3 sgrid((unsigned)num_seqs, (unsigned)sp.H, DV / kda::kSlab);
-        kda::state_simt_kernel<DK, DV><<<sgrid, 256, state_smem, stream>>>(sp);
-        g_launches.fetch_add(1, std::memory_order_relaxed);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "chunk_fwd launch");
-    }
+kda_status launch_prefill(const kda::FusedParams &p, int64_t units, cudaStream_t stream) {
+    constexpr int G = DV / kda::kSlab;
+    const int smem = kda::FusedSmem<DK, DV>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kda::kda_prefill_fused_kernel<DK, DV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
+    e = cudaMemsetAsync(p.flags, 0, flag_bytes(units, DV), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(ring flags)");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units * G));
+    cfg.blockDim = dim3(kda::kFusedThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kda::kda_prefill_fused_kernel<DK, DV>, p);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
     return KDA_OK;
 }
 
@@ -149,18 +145,13 @@ size_t kda_chunk_fwd_workspace_min(int64_t total_tokens, int32_t num_seqs, int32
                                    int32_t H, int32_t d_k, int32_t d_v) {
     if (!sizes_ok(total_tokens, num_seqs, max_seqlen, H) || !supported_dim(d_k) || !supported_dim(d_v))
         return 0;
-    return state_bytes(num_seqs, H, d_k, d_v) + (size_t)num_seqs * H * record_bytes(d_k, d_v);
+    const int64_t units = (int64_t)num_seqs * H;
+    return flag_bytes(units, d_v) + ring_bytes(units, d_k, d_v);
 }
 
 size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
                                     int32_t H, int32_t d_k, int32_t d_v) {
-    if (!sizes_ok(total_tokens, num_seqs, max_seqlen, H) || !supported_dim(d_k) || !supported_dim(d_v))
-        return 0;
-    const size_t per_row = (size_t)num_seqs * H * record_bytes(d_k, d_v);
-    const int64_t max_chunks = std::max<int64_t>(1, max_chunks_of(total_tokens, max_seqlen));
-    int64_t wc = per_row ? (int64_t)(kDefaultWindowBudget / per_row) : 1;
-    wc = std::max<int64_t>(1, std::min<int64_t>(wc, max_chunks));
-    return state_bytes(num_seqs, H, d_k, d_v) + per_row * (size_t)wc;
+    return kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
 }
 
 kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *a,
@@ -197,48 +188,36 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: workspace too small (need " +
                                              std::to_string(need) + " bytes)");
 
-    const int64_t max_chunks = max_chunks_of(total_tokens, max_seqlen);
-    const size_t sbytes = state_bytes(num_seqs, H, d_k, d_v);
-    const size_t per_row = (size_t)num_seqs * H * record_bytes(d_k, d_v);
-    int64_t wc = (int64_t)((workspace_bytes - sbytes) / per_row);
-    wc = std::max<int64_t>(1, std::min<int64_t>(wc, std::max<int64_t>(1, max_chunks)));
-    wc = std::min<int64_t>(wc, (int64_t)(0x7fffffff / num_seqs));
-    const int64_t windows = std::max<int64_t>(1, (max_chunks + wc - 1) / wc);
-
+    const int64_t units = (int64_t)num_seqs * H;
+    if (units * (d_v / kda::kSlab) > 0x7fffffffLL)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: num_seqs * H too large");
     char *ws = static_cast<char *>(workspace);
-    float *run = final_state ? final_state : reinterpret_cast<float *>(ws);
-    kda::PrepParams pp{};
-    pp.q = static_cast<const uint16_t *>(q);
-    pp.k = static_cast<const uint16_t *>(k);
-    pp.v = static_cast<const uint16_t *>(v);
-    pp.a = static_cast<const uint16_t *>(a);
-    pp.beta = beta;
-    pp.A_log = A_log;
-    pp.cu = cu_seqlens;
-    pp.rec = reinterpret_cast<float *>(ws + sbytes);
-    pp.total_tokens = total_tokens;
-    pp.num_seqs = num_seqs;
-    pp.H = H;
-    pp.Wc = (int)wc;
-    pp.scale = scale;
-    kda::StateParams sp{};
-    sp.rec = pp.rec;
-    sp.gate = static_cast<const uint16_t *>(gate);
-    sp.out = out;
-    sp.out_f32 = out_dtype == KDA_DTYPE_F32;
-    sp.cu = cu_seqlens;
-    sp.S_in = initial_state;
-    sp.S_out = run;
-    sp.total_tokens = total_tokens;
-    sp.num_seqs = num_seqs;
-    sp.H = H;
-    sp.Wc = (int)wc;
-    sp.max_chunks = (int)std::min<int64_t>(max_chunks, 0x7fffffff);
+    kda::FusedParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.a = static_cast<const uint16_t *>(a);
+    p.gate = static_cast<const uint16_t *>(gate);
+    p.beta = beta;
+    p.A_log = A_log;
+    p.cu = cu_seqlens;
+    p.S_in = initial_state;
+    p.S_out = final_state;
+    p.out = out;
+    p.flags = reinterpret_cast<int *>(ws);
+    p.ring = ws + flag_bytes(units, d_v);
+    p.total_tokens = total_tokens;
+    p.num_seqs = num_seqs;
+    p.H = H;
+    p.max_seqlen = max_seqlen;
+    p.scale = scale;
+    p.out_f32 = out_dtype == KDA_DTYPE_F32;
+    p.wait_ns = kWaitNs;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d_k == 128 && d_v == 128) return launch_chunk_fwd<128, 128>(pp, sp, windows, st);
-    if (d_k == 128 && d_v == 64) return launch_chunk_fwd<128, 64>(pp, sp, windows, st);
-    if (d_k == 64 && d_v == 128) return launch_chunk_fwd<64, 128>(pp, sp, windows, st);
-    return launch_chunk_fwd<64, 64>(pp, sp, windows, st);
+    if (d_k == 128 && d_v == 128) return launch_prefill<128, 128>(p, units, st);
+    if (d_k == 128 && d_v == 64) return launch_prefill<128, 64>(p, units, st);
+    if (d_k == 64 && d_v == 128) return launch_prefill<64, 128>(p, units, st);
+    return launch_prefill<64, 64>(p, units, st);
 }
 
 kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *a,
