@@ -46,8 +46,9 @@ __device__ __forceinline__ void store_out(void *out, int64_t off, bool f32, floa
     else static_cast<uint16_t *>(out)[off] = f32_to_bf16(x);
 }
 
-// sigmoid with the fast exponential; saturates cleanly (no NaN) for |x| -> inf.
-__device__ __forceinline__ float sigmoid_fast(float x) { return 1.0f / (1.0f + __expf(-x)); }
+// sigmoid with the fast exponential and a round-to-nearest reciprocal (no IEEE division);
+// saturates cleanly (no NaN) for |x| -> inf.
+__device__ __forceinline__ float sigmoid_fast(float x) { return __frcp_rn(1.0f + __expf(-x)); }
 
 // Log-decay g = g_min * sigmoid(exp(A_h) * a), with e^{A_h} precomputed by the caller.
 __device__ __forceinline__ float log_decay(float a, float expA) {

@@ -79,12 +79,15 @@ struct FusedSmem {
     static constexpr int kKr = kV + 64 * DV * 2;      // bf16 [64][DK] a, then k e^{b - r}
     static constexpr int kKh = kKr + 64 * DK * 2;     // fp16 [64][DK] K^
     static constexpr int kKb = kKh + 64 * DK * 2;     // fp16 [64][DK] K-
-    static constexpr int kKt = kKb + 64 * DK * 2;     // fp32 [64][DK] K~ = k e^{r_q - b}
-    static constexpr int kB = kKt + 64 * DK * 4;      // fp32 [64][DK] b; later L, T fp32 [64][65]
-    static constexpr int kBBytes = (64 * DK * 4 > 2 * 64 * 65 * 4) ? 64 * DK * 4 : 2 * 64 * 65 * 4;
-    static constexpr int kTb = kB + kBBytes;          // fp16 [64][64] T'
-    static constexpr int kTmp = kTb + 64 * 64 * 2;    // fp32 [3][16][17] solve scratch
-    static constexpr int kBeta = kTmp + 3 * 16 * 17 * 4;  // fp32 [64]
+    static constexpr int kKt = kKb + 64 * DK * 2;     // fp32 [64][DK] K~; later fp16 X [64][DK+DV]
+    static constexpr int kKtBytes = (64 * DK * 4 > 64 * (DK + DV) * 2) ? 64 * DK * 4 : 64 * (DK + DV) * 2;
+    static constexpr int kB = kKt + kKtBytes;         // fp32 [64][DK] b; later Ld and LD
+    static constexpr int kLd = kB;                    //   fp32 [4][16][17] diagonal blocks of L
+    static constexpr int kLD = kB + 4 * 16 * 17 * 4;  //   fp16 [64][64]: -L below the diagonal blocks,
+                                                      //   (I + L_pp)^-1 on them
+    static constexpr int kBBytes = (64 * DK * 4 > 4 * 16 * 17 * 4 + 64 * 64 * 2)
+                                       ? 64 * DK * 4 : 4 * 16 * 17 * 4 + 64 * 64 * 2;
+    static constexpr int kBeta = kB + kBBytes;        // fp32 [64]
     static constexpr int kTot = kBeta + 64 * 4;       // fp32 [4][DK] cumsum part totals
     static constexpr int kRef = kTot + 4 * DK * 4;    // fp32 [4][DK] r_p
     static constexpr int kEP = kRef + 4 * DK * 4;     // fp32 [4][DK] e^{r_p}
@@ -134,18 +137,6 @@ __device__ __forceinline__ bool wait_at_least(const int *flag, int target, unsig
     }
 }
 
-// Role-wide bounded wait: thread 0 of the role spins, the role's barrier publishes the outcome.
-__device__ __forceinline__ bool role_wait(const int *flag, int target, int role_tid, int bar_id,
-                                          volatile int *abort_flag, unsigned long long wait_ns) {
-    if (role_tid == 0) {
-        const bool ok = wait_at_least(flag, target, wait_ns);
-        if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
-        *abort_flag = ok ? 0 : 1;
-    }
-    named_bar(bar_id, kRoleThreads);
-    return *abort_flag == 0;
-}
-
 __device__ __forceinline__ float2 unpack_f16(uint32_t v) {
     const __half2 h = *reinterpret_cast<const __half2 *>(&v);
     return __half22float2(h);
@@ -161,19 +152,18 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
     using RL = RingLayout<DK, DV>;
     using SM = FusedSmem<DK, DV>;
     constexpr int G = RL::G, R = RL::R, KT = RL::KT;
-    constexpr int RB = DK * 2;   // row bytes of the [64][DK] 16-bit operands
+    constexpr int RB = DK * 2;            // row bytes of the [64][DK] 16-bit operands
     constexpr int RBV = DV * 2;
+    constexpr int RBX = (DK + DV) * 2;    // row bytes of X = [W | U~]
     const int tid = threadIdx.x - kRoleThreads;
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
 
     unsigned char *const sQhi = sm + SM::kQhi, *const sQlo = sm + SM::kQlo, *const sK = sm + SM::kK;
     unsigned char *const sKr = sm + SM::kKr, *const sKh = sm + SM::kKh, *const sKb = sm + SM::kKb;
-    unsigned char *const sKt = sm + SM::kKt, *const sTb = sm + SM::kTb;
-    unsigned char *const sBb = sm + SM::kB;
-    float *const sL = reinterpret_cast<float *>(sm + SM::kB);   // [64][65] once b is dead
-    float *const sT = sL + 64 * 65;                             // [64][65]
-    float *const sTmp = reinterpret_cast<float *>(sm + SM::kTmp);
+    unsigned char *const sKt = sm + SM::kKt, *const sX = sm + SM::kKt, *const sV = sm + SM::kV;
+    unsigned char *const sBb = sm + SM::kB, *const sLD = sm + SM::kLD;
+    float *const sLd = reinterpret_cast<float *>(sm + SM::kLd);
     float *const sbeta = reinterpret_cast<float *>(sm + SM::kBeta);
     float *const stot = reinterpret_cast<float *>(sm + SM::kTot);
     float *const sref = reinterpret_cast<float *>(sm + SM::kRef);
@@ -191,18 +181,25 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
     int *const flags = p.flags + (size_t)unit * R * 2;
     char *const ring = p.ring + (size_t)unit * R * RL::kBytes;
     const uint32_t aQhi = smem_u32(sQhi), aQlo = smem_u32(sQlo), aK = smem_u32(sK);
-    const uint32_t aV = smem_u32(sm + SM::kV), aKr = smem_u32(sKr), aKh = smem_u32(sKh);
-    const uint32_t aKb = smem_u32(sKb), aTb = smem_u32(sTb);
+    const uint32_t aV = smem_u32(sV), aKr = smem_u32(sKr), aKh = smem_u32(sKh);
+    const uint32_t aKb = smem_u32(sKb), aX = smem_u32(sX), aLD = smem_u32(sLD);
 
     for (int c = rank; c < nchunks; c += G) {
         const int slot = c % R;
         const int64_t t0 = s0 + (int64_t)c * kChunk;
         const int L = static_cast<int>(min64(kChunk, s1 - t0));
+        // the slot's release counter, read early so its latency overlaps the loads
+        const int empty_target = G * (c / R);
+        int empty_seen = 0;
+        if (tid == 0 && c >= R) empty_seen = ld_acquire_gpu(flags + slot * 2 + 1);
 
-        // 1. q, k, a, v rows of the chunk into shared memory (rows >= L zero-filled), and beta
+        // 1. q, k, a, v rows of the chunk into shared memory (rows >= L zero-filled), and beta;
+        //    then an L2 prefetch of the rows of this producer's next chunk
         {
             constexpr int CPR = DK / 8;  // 16-byte chunks per row
-            for (int e = tid; e < 64 * CPR; e += kRoleThreads) {
+#pragma unroll
+            for (int it = 0; it < 64 * CPR / kRoleThreads; ++it) {
+                const int e = tid + it * kRoleThreads;
                 const int row = e / CPR, ch = e % CPR;
                 const bool in = row < L;
                 const int64_t off = ((t0 + (in ? row : 0)) * H + h) * DK + ch * 8;
@@ -212,35 +209,69 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                 cp_async_16(aKr + dst, p.a + off, in ? 16 : 0);
             }
             constexpr int CPRV = DV / 8;
-            for (int e = tid; e < 64 * CPRV; e += kRoleThreads) {
+#pragma unroll
+            for (int it = 0; it < 64 * CPRV / kRoleThreads; ++it) {
+                const int e = tid + it * kRoleThreads;
                 const int row = e / CPRV, ch = e % CPRV;
                 const bool in = row < L;
                 const int64_t off = ((t0 + (in ? row : 0)) * H + h) * DV + ch * 8;
                 cp_async_16(aV + swz<RBV>(row, ch), p.v + off, in ? 16 : 0);
             }
             if (tid < 64) sbeta[tid] = tid < L ? p.beta[(t0 + tid) * H + h] : 0.f;
+            const int cn = c + G;
+            if (cn < nchunks) {
+                const int64_t tn = s0 + (int64_t)cn * kChunk;
+                const int Ln = static_cast<int>(min64(kChunk, s1 - tn));
+                const int row = tid & 63, which = tid >> 6;   // 4 tensors x 64 rows
+                if (row < Ln) {
+                    const uint16_t *base = which == 0 ? p.q : which == 1 ? p.k : which == 2 ? p.a : p.v;
+                    const int d = which == 3 ? DV : DK;
+                    prefetch_l2_bulk(base + ((tn + row) * H + h) * d, d * 2);
+                }
+            }
             cp_async_wait_all();
             named_bar(kBarProducer, kRoleThreads);
         }
 
-        // 2. log-decay g and its chunk-local inclusive cumsum b (rows >= L carry g = 0)
+        // 2. log-decay g for every element (independent), then the chunk-local inclusive
+        //    cumsum b per channel (rows >= L carry g = 0)
+        {
+            constexpr int NIT = 64 * DK / kRoleThreads;
+            float gv[NIT];
+#pragma unroll
+            for (int it = 0; it < NIT; ++it) {   // all loads first, then the math, then the stores
+                const int e = tid + it * kRoleThreads;
+                gv[it] = bf16_to_f32(*reinterpret_cast<const uint16_t *>(sKr + swz_elem<RB>(e / DK, e % DK)));
+            }
+#pragma unroll
+            for (int it = 0; it < NIT; ++it) {
+                const int e = tid + it * kRoleThreads;
+                gv[it] = e / DK < L ? log_decay(gv[it], expA) : 0.f;
+            }
+#pragma unroll
+            for (int it = 0; it < NIT; ++it) {
+                const int e = tid + it * kRoleThreads;
+                bval(e / DK, e % DK) = gv[it];
+            }
+        }
+        named_bar(kBarProducer, kRoleThreads);
         {
             constexpr int PARTS = kRoleThreads / DK;   // 2 for d_k = 128, 4 for 64
             constexpr int TPP = 64 / PARTS;
             const int ch = tid % DK, part = tid / DK;
             float acc = 0.f;
-#pragma unroll 4
+#pragma unroll 8
             for (int i = 0; i < TPP; ++i) {
-                const int t = part * TPP + i;
-                const uint16_t raw = *reinterpret_cast<const uint16_t *>(sKr + swz_elem<RB>(t, ch));
-                acc += t < L ? log_decay(bf16_to_f32(raw), expA) : 0.f;
-                bval(t, ch) = acc;
+                float &x = bval(part * TPP + i, ch);
+                acc += x;
+                x = acc;
             }
             stot[part * DK + ch] = acc;
             named_bar(kBarProducer, kRoleThreads);
             if (part > 0) {
                 float off = 0.f;
                 for (int pp = 0; pp < part; ++pp) off += stot[pp * DK + ch];
+#pragma unroll 8
                 for (int i = 0; i < TPP; ++i) bval(part * TPP + i, ch) += off;
             }
             named_bar(kBarProducer, kRoleThreads);
@@ -266,20 +297,23 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                     sD[pair_index(pp, qq) * DK + ch] = ex2((r[pp] - r[qq]) * kLog2e);
             }
         }
-        named_bar(kBarProducer, kRoleThreads);
-
         // the slot must be free (chunk c - R consumed by all G consumers) before any ring write
-        if (c >= R) {
-            if (!role_wait(flags + slot * 2 + 1, G * (c / R), tid, kBarProducer, abort_flag,
-                           p.wait_ns))
-                return;
+        if (tid == 0) {
+            bool ok = true;
+            if (c >= R && empty_seen < empty_target) {
+                ok = wait_at_least(flags + slot * 2 + 1, empty_target, p.wait_ns);
+                if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
+            }
+            *abort_flag = ok ? 0 : 1;
         }
+        named_bar(kBarProducer, kRoleThreads);
+        if (*abort_flag) return;
         char *const slotp = ring + (size_t)slot * RL::kBytes;
 
         // 3. operands.  Each thread owns the A-fragment positions of KT/2 tiles of [64][DK]
         //    (rows 16m + g, +8; columns 16kd + 2t4, +1, +8, +9) and writes its Q^ fragments
         //    straight to the ring.
-#pragma unroll 1
+#pragma unroll
         for (int j = 0; j < KT / 2; ++j) {
             const int idx = warp * (KT / 2) + j;
             const int m = idx / KT, kd = idx % KT, pt = m;   // token tile = 16-token tile
@@ -327,8 +361,9 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             const int qb = blk - pb * (pb + 1) / 2;
             const int jrow = 16 * qb + 8 * nt + g;   // column index j of this lane's B element
             const float *dcol = pb > qb ? sD + pair_index(pb, qb) * DK : nullptr;
-            float aqk[4] = {0.f, 0.f, 0.f, 0.f}, akk[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
+            float ahh[4] = {0.f, 0.f, 0.f, 0.f}, ahl[4] = {0.f, 0.f, 0.f, 0.f};
+            float alh[4] = {0.f, 0.f, 0.f, 0.f}, akk[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
             for (int ks = 0; ks < KT; ++ks) {
                 uint32_t ahi[4], alo[4], ak[4];
                 ldsm_x4(ahi, ldsm_addr_a<RB>(aQhi, 16 * pb, 16 * ks, lane));
@@ -345,25 +380,35 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                 uint32_t bh0, bl0, bh1, bl1;
                 split_bf16(k0.x, k0.y, bh0, bl0);
                 split_bf16(k1.x, k1.y, bh1, bl1);
-                mma_bf16(aqk, ahi, bh0, bh1);
-                mma_bf16(aqk, ahi, bl0, bl1);
-                mma_bf16(aqk, alo, bh0, bh1);
+                mma_bf16(ahh, ahi, bh0, bh1);
+                mma_bf16(ahl, ahi, bl0, bl1);
+                mma_bf16(alh, alo, bh0, bh1);
                 mma_bf16(akk, ak, bh0, bh1);
             }
             const int i0 = 16 * pb + g, i1 = i0 + 8;
             const int jc = 16 * qb + 8 * nt + 2 * t4;
             const bool diag = pb == qb;
+            float aq[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) aq[e] = ahh[e] + (ahl[e] + alh[e]);
             // A fragment half (columns 8 nt .. 8 nt + 7 of the 16x16 tile), fp16
-            const float a0 = !diag || jc <= i0 ? aqk[0] : 0.f;
-            const float a1 = !diag || jc + 1 <= i0 ? aqk[1] : 0.f;
-            const float a2 = !diag || jc <= i1 ? aqk[2] : 0.f;
-            const float a3 = !diag || jc + 1 <= i1 ? aqk[3] : 0.f;
+            const float a0 = !diag || jc <= i0 ? aq[0] : 0.f;
+            const float a1 = !diag || jc + 1 <= i0 ? aq[1] : 0.f;
+            const float a2 = !diag || jc <= i1 ? aq[2] : 0.f;
+            const float a3 = !diag || jc + 1 <= i1 ? aq[3] : 0.f;
             stg_v2(slotp + RL::kA + blk * 512 + lane * 16 + nt * 8, pack_f16(a0, a1), pack_f16(a2, a3));
             const float b0 = sbeta[i0], b1 = sbeta[i1];
-            sL[i0 * 65 + jc] = !diag || jc < i0 ? b0 * akk[0] : 0.f;
-            sL[i0 * 65 + jc + 1] = !diag || jc + 1 < i0 ? b0 * akk[1] : 0.f;
-            sL[i1 * 65 + jc] = !diag || jc < i1 ? b1 * akk[2] : 0.f;
-            sL[i1 * 65 + jc + 1] = !diag || jc + 1 < i1 ? b1 * akk[3] : 0.f;
+            if (diag) {   // fp32 diagonal block for the 16x16 inverses
+                const int li = g, lj = 8 * nt + 2 * t4;
+                float *Ld = sLd + pb * 16 * 17;
+                Ld[li * 17 + lj] = lj < li ? b0 * akk[0] : 0.f;
+                Ld[li * 17 + lj + 1] = lj + 1 < li ? b0 * akk[1] : 0.f;
+                Ld[(li + 8) * 17 + lj] = lj < li + 8 ? b1 * akk[2] : 0.f;
+                Ld[(li + 8) * 17 + lj + 1] = lj + 1 < li + 8 ? b1 * akk[3] : 0.f;
+            } else {      // -L below the diagonal blocks, fp16, as the A operand of the solve
+                *reinterpret_cast<uint32_t *>(sLD + swz_elem<128>(i0, jc)) = pack_f16(-b0 * akk[0], -b0 * akk[1]);
+                *reinterpret_cast<uint32_t *>(sLD + swz_elem<128>(i1, jc)) = pack_f16(-b1 * akk[2], -b1 * akk[3]);
+            }
         }
         // 4b. K-^T fragments and Gamma_C
         for (int idx = warp; idx < 4 * KT; idx += 8) {
@@ -376,115 +421,99 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             reinterpret_cast<float *>(slotp + RL::kGam)[tid] = sEP[3 * DK + tid] * sTT[3 * DK + tid];
         named_bar(kBarProducer, kRoleThreads);
 
-        // 5. T = (I + L)^-1, blocked: diagonal 16x16 inverses, then off-diagonal blocks by level
+        // 5. diagonal blocks D_p = (I + L_pp)^-1 by forward substitution (fp32), one column per lane
         if (warp < 4 && lane < 16) {
-            const int pb = warp, m = lane, o = 16 * pb;
+            const int pb = warp, mcol = lane;
+            const float *Ld = sLd + pb * 16 * 17;
             float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                float v = i == m ? 1.f : 0.f;
+                float v = i == mcol ? 1.f : 0.f;
 #pragma unroll
-                for (int j = 0; j < i; ++j) v = fmaf(-sL[(o + i) * 65 + o + j], x[j], v);
-                x[i] = i >= m ? v : 0.f;
+                for (int j = 0; j < i; ++j) v = fmaf(-Ld[i * 17 + j], x[j], v);
+                x[i] = i >= mcol ? v : 0.f;
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sT[(o + i) * 65 + o + m] = x[i];
-        }
-        named_bar(kBarProducer, kRoleThreads);
-        {
-            const int ii = tid >> 4, jj = tid & 15;
-#pragma unroll 1
-            for (int d = 1; d < 4; ++d) {
-                // M = sum_{m=q}^{p-1} L_pm T_mq for every block (p, q = p - d)
-                for (int bq = 0; bq + d < 4; ++bq) {
-                    const int pb = bq + d;
-                    float acc = 0.f;
-                    for (int mb = bq; mb < pb; ++mb)
-#pragma unroll
-                        for (int x = 0; x < 16; ++x)
-                            acc = fmaf(sL[(16 * pb + ii) * 65 + 16 * mb + x],
-                                       sT[(16 * mb + x) * 65 + 16 * bq + jj], acc);
-                    sTmp[(bq * 16 + ii) * 17 + jj] = acc;
-                }
-                named_bar(kBarProducer, kRoleThreads);
-                // T_pq = -D_p M
-                for (int bq = 0; bq + d < 4; ++bq) {
-                    const int pb = bq + d;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int x = 0; x < 16; ++x)
-                        acc = fmaf(sT[(16 * pb + ii) * 65 + 16 * pb + x], sTmp[(bq * 16 + x) * 17 + jj],
-                                   acc);
-                    sT[(16 * pb + ii) * 65 + 16 * bq + jj] = -acc;
-                }
-                named_bar(kBarProducer, kRoleThreads);
-            }
-        }
-        // T' = T diag(beta) as fp16 (lower triangle incl. diagonal; zero above)
-        for (int e = tid; e < 64 * 32; e += kRoleThreads) {
-            const int i = e >> 5, j = (e & 31) * 2;
-            const float v0 = j <= i ? sT[i * 65 + j] * sbeta[j] : 0.f;
-            const float v1 = j + 1 <= i ? sT[i * 65 + j + 1] * sbeta[j + 1] : 0.f;
-            *reinterpret_cast<uint32_t *>(sTb + swz_elem<128>(i, j)) = pack_f16(v0, v1);
+            for (int i = 0; i < 16; ++i)
+                *reinterpret_cast<__half *>(sLD + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = __float2half_rn(x[i]);
         }
         named_bar(kBarProducer, kRoleThreads);
 
-        // 6. W = T' K^ and U~ = T' V: warp -> token tile m, column half hf
+        // 6. [W | U~] = (I + L)^-1 diag(beta) [K^ | V], blocked forward substitution per 16-row block:
+        //    X_p = D_p (B_p - sum_{m<p} L_pm X_m).  Each warp owns 16-column units of X, so the
+        //    whole solve is warp-local; X_p (fp16) is kept in shared memory for later blocks.
         {
-            const int m = warp & 3, hf = warp >> 2;
-            constexpr int WN = DK / 2, UN = DV / 2;   // columns per half
-            float accW[WN / 8][4], accU[UN / 8][4];
+            constexpr int UW = DK / 16, UT = (DK + DV) / 16;
+#pragma unroll 1
+            for (int u = warp; u < UT; u += 8) {
+                const bool isW = u < UW;
+                const int xc = 16 * u;                          // column in X
+                const int vc = isW ? xc : xc - DK;              // column in K^ or V
+#pragma unroll 1
+                for (int pb = 0; pb < 4; ++pb) {
+                    const int r0 = 16 * pb + g, r1 = r0 + 8;
+                    const float b0 = sbeta[r0], b1 = sbeta[r1];
+                    float acc[2][4];
 #pragma unroll
-            for (int i = 0; i < WN / 8; ++i) accW[i][0] = accW[i][1] = accW[i][2] = accW[i][3] = 0.f;
-#pragma unroll
-            for (int i = 0; i < UN / 8; ++i) accU[i][0] = accU[i][1] = accU[i][2] = accU[i][3] = 0.f;
-#pragma unroll
-            for (int kt = 0; kt < 4; ++kt) {
-                if (kt <= m) {
-                    uint32_t af[4];
-                    ldsm_x4(af, ldsm_addr_a<128>(aTb, 16 * m, 16 * kt, lane));
-#pragma unroll
-                    for (int np = 0; np < WN / 16; ++np) {
-                        uint32_t bf[4];
-                        ldsm_x4_t(bf, ldsm_addr_bt<RB>(aKh, 16 * kt, hf * WN + 16 * np, lane));
-                        mma_f16(accW[2 * np], af, bf[0], bf[1]);
-                        mma_f16(accW[2 * np + 1], af, bf[2], bf[3]);
+                    for (int j = 0; j < 2; ++j) {
+                        const int cc = vc + 8 * j + 2 * t4;
+                        float2 x0, x1;
+                        if (isW) {
+                            x0 = unpack_f16(*reinterpret_cast<const uint32_t *>(sKh + swz_elem<RB>(r0, cc)));
+                            x1 = unpack_f16(*reinterpret_cast<const uint32_t *>(sKh + swz_elem<RB>(r1, cc)));
+                        } else {
+                            x0 = unpack_bf16(*reinterpret_cast<const uint32_t *>(sV + swz_elem<RBV>(r0, cc)));
+                            x1 = unpack_bf16(*reinterpret_cast<const uint32_t *>(sV + swz_elem<RBV>(r1, cc)));
+                        }
+                        acc[j][0] = b0 * x0.x; acc[j][1] = b0 * x0.y;
+                        acc[j][2] = b1 * x1.x; acc[j][3] = b1 * x1.y;
                     }
 #pragma unroll
-                    for (int np = 0; np < UN / 16; ++np) {
-                        uint32_t bf[4];
-                        ldsm_x4_t(bf, ldsm_addr_bt<RBV>(aV, 16 * kt, hf * UN + 16 * np, lane));
-                        mma_f16(accU[2 * np], af, bf16x2_to_f16x2(bf[0]), bf16x2_to_f16x2(bf[1]));
-                        mma_f16(accU[2 * np + 1], af, bf16x2_to_f16x2(bf[2]), bf16x2_to_f16x2(bf[3]));
+                    for (int mb = 0; mb < 3; ++mb) {
+                        if (mb >= pb) break;
+                        uint32_t af[4], bf[4];
+                        ldsm_x4(af, ldsm_addr_a<128>(aLD, 16 * pb, 16 * mb, lane));   // -L_pm
+                        ldsm_x4_t(bf, ldsm_addr_bt<RBX>(aX, 16 * mb, xc, lane));      // X_m
+                        mma_f16(acc[0], af, bf[0], bf[1]);
+                        mma_f16(acc[1], af, bf[2], bf[3]);
+                    }
+                    // R_p -> shared memory (this warp's columns), then X_p = D_p R_p
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int cc = xc + 8 * j + 2 * t4;
+                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r0, cc)) = pack_f16(acc[j][0], acc[j][1]);
+                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r1, cc)) = pack_f16(acc[j][2], acc[j][3]);
+                    }
+                    __syncwarp();
+                    float xp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                    {
+                        uint32_t af[4], bf[4];
+                        ldsm_x4(af, ldsm_addr_a<128>(aLD, 16 * pb, 16 * pb, lane));   // D_p
+                        ldsm_x4_t(bf, ldsm_addr_bt<RBX>(aX, 16 * pb, xc, lane));      // R_p
+                        mma_f16(xp[0], af, bf[0], bf[1]);
+                        mma_f16(xp[1], af, bf[2], bf[3]);
+                    }
+                    __syncwarp();
+                    uint32_t fr[4];
+                    fr[0] = pack_f16(xp[0][0], xp[0][1]);
+                    fr[1] = pack_f16(xp[0][2], xp[0][3]);
+                    fr[2] = pack_f16(xp[1][0], xp[1][1]);
+                    fr[3] = pack_f16(xp[1][2], xp[1][3]);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int cc = xc + 8 * j + 2 * t4;
+                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r0, cc)) = fr[2 * j];
+                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r1, cc)) = fr[2 * j + 1];
+                    }
+                    __syncwarp();
+                    if (isW) {   // W tile (token tile pb, d_k tile u): an A fragment
+                        stg_v4(slotp + RL::kW + (pb * KT + u) * 512 + lane * 16, make_uint4(fr[0], fr[1], fr[2], fr[3]));
+                    } else {     // U~: half (vc / 16) % 2 of slab vc / 32
+                        const int sl = vc / kSlab, half = (vc / 16) & 1;
+                        stg_v4(slotp + RL::kU + ((pb * G + sl) * 32 + lane) * 32 + half * 16,
+                               make_uint4(fr[0], fr[1], fr[2], fr[3]));
                     }
                 }
-            }
-#pragma unroll
-            for (int np = 0; np < WN / 16; ++np) {
-                const int kd = hf * (WN / 16) + np;
-                uint4 fr;
-                fr.x = pack_f16(accW[2 * np][0], accW[2 * np][1]);
-                fr.y = pack_f16(accW[2 * np][2], accW[2 * np][3]);
-                fr.z = pack_f16(accW[2 * np + 1][0], accW[2 * np + 1][1]);
-                fr.w = pack_f16(accW[2 * np + 1][2], accW[2 * np + 1][3]);
-                stg_v4(slotp + RL::kW + (m * KT + kd) * 512 + lane * 16, fr);
-            }
-#pragma unroll
-            for (int sl = 0; sl < UN / kSlab; ++sl) {
-                const int s = hf * (UN / kSlab) + sl;
-                const float(*u)[4] = accU + 4 * sl;
-                uint4 lo, hi;
-                lo.x = pack_f16(u[0][0], u[0][1]);
-                lo.y = pack_f16(u[0][2], u[0][3]);
-                lo.z = pack_f16(u[1][0], u[1][1]);
-                lo.w = pack_f16(u[1][2], u[1][3]);
-                hi.x = pack_f16(u[2][0], u[2][1]);
-                hi.y = pack_f16(u[2][2], u[2][3]);
-                hi.z = pack_f16(u[3][0], u[3][1]);
-                hi.w = pack_f16(u[3][2], u[3][3]);
-                char *dst = slotp + RL::kU + ((m * G + s) * 32 + lane) * 32;
-                stg_v4(dst, lo);
-                stg_v4(dst + 16, hi);
             }
         }
         named_bar(kBarProducer, kRoleThreads);
@@ -538,6 +567,26 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     // output tile of this warp: token rows 16 m + (g, g+8), slab columns 16 ch + 8 j + 2 t4 (+1)
     const int m = warp & 3, ch = warp >> 2;
 
+    const int i0 = 16 * m + g, i1 = i0 + 8;
+    // gate logits of the next chunk, loaded a chunk ahead (they come from HBM)
+    auto load_gate = [&](int cg, uint32_t (&gt)[2][2]) {
+        gt[0][0] = gt[0][1] = gt[1][0] = gt[1][1] = 0u;
+        if (!p.gate || cg >= nchunks) return;
+        const int64_t tg = s0 + (int64_t)cg * kChunk;
+        const int Lg = static_cast<int>(min64(kChunk, s1 - tg));
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int cc = col0 + 16 * ch + 8 * j + 2 * t4;
+            if (i0 < Lg) gt[j][0] = __ldg(reinterpret_cast<const unsigned int *>(p.gate + ((tg + i0) * H + h) * DV + cc));
+            if (i1 < Lg) gt[j][1] = __ldg(reinterpret_cast<const unsigned int *>(p.gate + ((tg + i1) * H + h) * DV + cc));
+        }
+    };
+    uint32_t gt[2][2];
+    load_gate(0, gt);
+    // the next chunk's `full` counter, read early so its latency overlaps the current chunk
+    int full_seen = 0;
+    if (tid == 0 && nchunks > 0) full_seen = ld_acquire_gpu(flags);
+
     for (int c = 0; c < nchunks; ++c) {
         // fp16 copy of the state: the B operand of W S and Q^ S
 #pragma unroll
@@ -547,7 +596,16 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             *reinterpret_cast<uint32_t *>(sS + swz_elem<64>(r1, cc)) = pack_f16(S[j][2], S[j][3]);
         }
         const int slot = c % R;
-        if (!role_wait(flags + slot * 2, c + 1, tid, kBarConsumer, abort_flag, p.wait_ns)) return;
+        if (tid == 0) {
+            bool ok = true;
+            if (full_seen < c + 1) {
+                ok = wait_at_least(flags + slot * 2, c + 1, p.wait_ns);
+                if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
+            }
+            *abort_flag = ok ? 0 : 1;
+        }
+        named_bar(kBarConsumer, kRoleThreads);
+        if (*abort_flag) return;
         const char *const slotp = ring + (size_t)slot * RL::kBytes;
         const int64_t t0 = s0 + (int64_t)c * kChunk;
         const int L = static_cast<int>(min64(kChunk, s1 - t0));
@@ -564,22 +622,31 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         const uint4 Uf = ldg_cg_v4(slotp + RL::kU + ((m * G + rank) * 32 + lane) * 32 + ch * 16);
         const float gam0 = __ldcg(reinterpret_cast<const float *>(slotp + RL::kGam) + r0);
         const float gam1 = __ldcg(reinterpret_cast<const float *>(slotp + RL::kGam) + r1);
-        const int i0 = 16 * m + g, i1 = i0 + 8;
 
-        // U = U~ - W S  (the chain), then O = Q^ S
-        float accU[2][4], accO[2][4];
+        // U = U~ - W S  (the chain; two independent partial sums halve the dependent MMAs),
+        // then O = Q^ S
+        float accU[2][4], accV[2][4], accO[2][4];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) accU[j][e] = accO[j][e] = 0.f;
+            for (int e = 0; e < 4; ++e) accU[j][e] = accV[j][e] = accO[j][e] = 0.f;
 #pragma unroll
         for (int kd = 0; kd < KT; ++kd) {
             uint32_t bf[4];
             ldsm_x4_t(bf, ldsm_addr_bt<64>(aS, 16 * kd, 16 * ch, lane));
             const uint32_t wa[4] = {Wf[kd].x, Wf[kd].y, Wf[kd].z, Wf[kd].w};
-            mma_f16(accU[0], wa, bf[0], bf[1]);
-            mma_f16(accU[1], wa, bf[2], bf[3]);
+            if (kd & 1) {
+                mma_f16(accV[0], wa, bf[0], bf[1]);
+                mma_f16(accV[1], wa, bf[2], bf[3]);
+            } else {
+                mma_f16(accU[0], wa, bf[0], bf[1]);
+                mma_f16(accU[1], wa, bf[2], bf[3]);
+            }
         }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) accU[j][e] += accV[j][e];
         {
             const uint32_t uw[4] = {Uf.x, Uf.y, Uf.z, Uf.w};
 #pragma unroll
@@ -603,15 +670,9 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             mma_f16(accO[0], qa, bf[0], bf[1]);
             mma_f16(accO[1], qa, bf[2], bf[3]);
         }
-        uint32_t gt[2][2] = {{0u, 0u}, {0u, 0u}};
-        if (p.gate) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int cc = col0 + 16 * ch + 8 * j + 2 * t4;
-                if (i0 < L) gt[j][0] = *reinterpret_cast<const uint32_t *>(p.gate + ((t0 + i0) * H + h) * DV + cc);
-                if (i1 < L) gt[j][1] = *reinterpret_cast<const uint32_t *>(p.gate + ((t0 + i1) * H + h) * DV + cc);
-            }
-        }
+        uint32_t gtn[2][2];
+        load_gate(c + 1, gtn);
+        if (tid == 0 && c + 1 < nchunks) full_seen = ld_acquire_gpu(flags + ((c + 1) % R) * 2);
         named_bar(kBarConsumer, kRoleThreads);   // U complete in shared memory
 
         // S = Diag(Gamma_C) S + K-^T U   (the chain)
@@ -619,16 +680,26 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         for (int j = 0; j < SNT; ++j) {
             S[j][0] *= gam0; S[j][1] *= gam0; S[j][2] *= gam1; S[j][3] *= gam1;
         }
+        {
+            float Sx[SNT][4];   // odd token tiles accumulate separately (two short chains)
 #pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            const uint32_t ka[4] = {Kf[kt].x, Kf[kt].y, Kf[kt].z, Kf[kt].w};
+            for (int j = 0; j < SNT; ++j) Sx[j][0] = Sx[j][1] = Sx[j][2] = Sx[j][3] = 0.f;
 #pragma unroll
-            for (int np = 0; np < SNT / 2; ++np) {
-                uint32_t bf[4];
-                ldsm_x4_t(bf, ldsm_addr_bt<64>(aU, 16 * kt, 8 * sn0 + 16 * np, lane));
-                mma_f16(S[2 * np], ka, bf[0], bf[1]);
-                mma_f16(S[2 * np + 1], ka, bf[2], bf[3]);
+            for (int kt = 0; kt < 4; ++kt) {
+                const uint32_t ka[4] = {Kf[kt].x, Kf[kt].y, Kf[kt].z, Kf[kt].w};
+#pragma unroll
+                for (int np = 0; np < SNT / 2; ++np) {
+                    uint32_t bf[4];
+                    ldsm_x4_t(bf, ldsm_addr_bt<64>(aU, 16 * kt, 8 * sn0 + 16 * np, lane));
+                    float(*dst)[4] = (kt & 1) ? Sx : S;
+                    mma_f16(dst[2 * np], ka, bf[0], bf[1]);
+                    mma_f16(dst[2 * np + 1], ka, bf[2], bf[3]);
+                }
             }
+#pragma unroll
+            for (int j = 0; j < SNT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) S[j][e] += Sx[j][e];
         }
         // O += A U, gate, store
 #pragma unroll
@@ -661,6 +732,7 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                 else *reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(p.out) + off) = pack_bf16(o2, o3);
             }
         }
+        gt[0][0] = gtn[0][0]; gt[0][1] = gtn[0][1]; gt[1][0] = gtn[1][0]; gt[1][1] = gtn[1][1];
         // every warp is done with this slot and with sS / sU before they are rewritten
         named_bar(kBarConsumer, kRoleThreads);
         if (tid == 0) red_release_add_gpu(flags + slot * 2 + 1, 1);
