@@ -46,9 +46,23 @@ __device__ __forceinline__ void store_out(void *out, int64_t off, bool f32, floa
     else static_cast<uint16_t *>(out)[off] = f32_to_bf16(x);
 }
 
-// sigmoid with the fast exponential and a round-to-nearest reciprocal (no IEEE division);
-// saturates cleanly (no NaN) for |x| -> inf.
-__device__ __forceinline__ float sigmoid_fast(float x) { return __frcp_rn(1.0f + __expf(-x)); }
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// sigmoid from the hardware exp2 and reciprocal approximations (about 2 ulp); saturates cleanly
+// (1 / inf = 0, no NaN) for |x| -> inf.
+__device__ __forceinline__ float sigmoid_fast(float x) {
+    return rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * x));
+}
 
 // Log-decay g = g_min * sigmoid(exp(A_h) * a), with e^{A_h} precomputed by the caller.
 __device__ __forceinline__ float log_decay(float a, float expA) {

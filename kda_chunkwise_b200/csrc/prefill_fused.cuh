@@ -66,27 +66,33 @@ struct RingLayout {
 // Shared memory of one CTA (bytes).
 template <int DK, int DV>
 struct FusedSmem {
+    using RL = RingLayout<DK, DV>;
     // consumer
     static constexpr int kS = 0;                      // fp16 [DK][32] state operand
     static constexpr int kU = kS + DK * kSlab * 2;    // fp16 [64][32] U operand
-    static constexpr int kCFlag = kU + 64 * kSlab * 2;  // int abort flag
+    static constexpr int kPW = kU + 64 * kSlab * 2;   // prefetched W tiles of the next chunk
+    static constexpr int kPK = kPW + 4 * RL::KT * 512;   // prefetched K-^T tiles
+    static constexpr int kPU = kPK + 4 * RL::KT * 512;   // prefetched U~ of this slab [4][32][32 B]
+    static constexpr int kPG = kPU + 4 * 32 * 32;     // prefetched Gamma_C fp32 [DK]
+    static constexpr int kCFlag = kPG + DK * 4;       // int abort flag
     static constexpr int kProd = (kCFlag + 16 + 1023) / 1024 * 1024;
     // producer (all [64][*] operand tiles are swizzled row-major)
     static constexpr int kQhi = kProd;                // bf16 [64][DK] q, then hi of q e^{b - r}
     static constexpr int kQlo = kQhi + 64 * DK * 2;   // bf16 [64][DK] lo of q e^{b - r}
-    static constexpr int kK = kQlo + 64 * DK * 2;     // bf16 [64][DK] k
+    static constexpr int kK = kQlo + 64 * DK * 2;     // bf16 [64][DK] k, then fp16 K-
     static constexpr int kV = kK + 64 * DK * 2;       // bf16 [64][DV] v
     static constexpr int kKr = kV + 64 * DV * 2;      // bf16 [64][DK] a, then k e^{b - r}
     static constexpr int kKh = kKr + 64 * DK * 2;     // fp16 [64][DK] K^
-    static constexpr int kKb = kKh + 64 * DK * 2;     // fp16 [64][DK] K-
-    static constexpr int kKt = kKb + 64 * DK * 2;     // fp32 [64][DK] K~; later fp16 X [64][DK+DV]
-    static constexpr int kKtBytes = (64 * DK * 4 > 64 * (DK + DV) * 2) ? 64 * DK * 4 : 64 * (DK + DV) * 2;
-    static constexpr int kB = kKt + kKtBytes;         // fp32 [64][DK] b; later Ld and LD
+    static constexpr int kKt = kKh + 64 * DK * 2;     // fp32 [64][DK] K~; later fp16 T' [64][64]
+    static constexpr int kKtBytes = (64 * DK * 4 > 64 * 64 * 2) ? 64 * DK * 4 : 64 * 64 * 2;
+    static constexpr int kB = kKt + kKtBytes;         // fp32 [64][DK] b; later:
     static constexpr int kLd = kB;                    //   fp32 [4][16][17] diagonal blocks of L
-    static constexpr int kLD = kB + 4 * 16 * 17 * 4;  //   fp16 [64][64]: -L below the diagonal blocks,
-                                                      //   (I + L_pp)^-1 on them
-    static constexpr int kBBytes = (64 * DK * 4 > 4 * 16 * 17 * 4 + 64 * 64 * 2)
-                                       ? 64 * DK * 4 : 4 * 16 * 17 * 4 + 64 * 64 * 2;
+    static constexpr int kLD = kLd + 4 * 16 * 17 * 4;   //   fp16 [64][64]: -L below the diagonal
+                                                      //   blocks, (I + L_pp)^-1 on them
+    static constexpr int kT = kLD + 64 * 64 * 2;      //   fp16 [64][64] T = (I + L)^-1
+    static constexpr int kM = kT + 64 * 64 * 2;       //   fp16 [3][16][32] block-product scratch
+    static constexpr int kBNeed = kM + 3 * 16 * 64 - kB;
+    static constexpr int kBBytes = (64 * DK * 4 > kBNeed) ? 64 * DK * 4 : kBNeed;
     static constexpr int kBeta = kB + kBBytes;        // fp32 [64]
     static constexpr int kTot = kBeta + 64 * 4;       // fp32 [4][DK] cumsum part totals
     static constexpr int kRef = kTot + 4 * DK * 4;    // fp32 [4][DK] r_p
@@ -154,15 +160,15 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
     constexpr int G = RL::G, R = RL::R, KT = RL::KT;
     constexpr int RB = DK * 2;            // row bytes of the [64][DK] 16-bit operands
     constexpr int RBV = DV * 2;
-    constexpr int RBX = (DK + DV) * 2;    // row bytes of X = [W | U~]
     const int tid = threadIdx.x - kRoleThreads;
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
 
     unsigned char *const sQhi = sm + SM::kQhi, *const sQlo = sm + SM::kQlo, *const sK = sm + SM::kK;
-    unsigned char *const sKr = sm + SM::kKr, *const sKh = sm + SM::kKh, *const sKb = sm + SM::kKb;
-    unsigned char *const sKt = sm + SM::kKt, *const sX = sm + SM::kKt, *const sV = sm + SM::kV;
-    unsigned char *const sBb = sm + SM::kB, *const sLD = sm + SM::kLD;
+    unsigned char *const sKr = sm + SM::kKr, *const sKh = sm + SM::kKh, *const sKb = sm + SM::kK;
+    unsigned char *const sKt = sm + SM::kKt, *const sTp = sm + SM::kKt, *const sV = sm + SM::kV;
+    unsigned char *const sBb = sm + SM::kB, *const sLD = sm + SM::kLD, *const sT = sm + SM::kT;
+    unsigned char *const sM = sm + SM::kM;
     float *const sLd = reinterpret_cast<float *>(sm + SM::kLd);
     float *const sbeta = reinterpret_cast<float *>(sm + SM::kBeta);
     float *const stot = reinterpret_cast<float *>(sm + SM::kTot);
@@ -182,7 +188,41 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
     char *const ring = p.ring + (size_t)unit * R * RL::kBytes;
     const uint32_t aQhi = smem_u32(sQhi), aQlo = smem_u32(sQlo), aK = smem_u32(sK);
     const uint32_t aV = smem_u32(sV), aKr = smem_u32(sKr), aKh = smem_u32(sKh);
-    const uint32_t aKb = smem_u32(sKb), aX = smem_u32(sX), aLD = smem_u32(sLD);
+    const uint32_t aKb = smem_u32(sKb), aTp = smem_u32(sTp), aLD = smem_u32(sLD);
+    const uint32_t aT = smem_u32(sT), aM = smem_u32(sM);
+
+    // asynchronous input copies of one chunk: q, k, a as one commit group, v as another
+    auto load_qka = [&](int cl) {
+        const int64_t tl = s0 + (int64_t)cl * kChunk;
+        const int Ll = static_cast<int>(min64(kChunk, s1 - tl));
+        constexpr int CPR = DK / 8;  // 16-byte chunks per row
+#pragma unroll
+        for (int it = 0; it < 64 * CPR / kRoleThreads; ++it) {
+            const int e = tid + it * kRoleThreads;
+            const int row = e / CPR, ch = e % CPR;
+            const bool in = row < Ll;
+            const int64_t off = ((tl + (in ? row : 0)) * H + h) * DK + ch * 8;
+            const uint32_t dst = swz<RB>(row, ch);
+            cp_async_16(aQhi + dst, p.q + off, in ? 16 : 0);
+            cp_async_16(aK + dst, p.k + off, in ? 16 : 0);
+            cp_async_16(aKr + dst, p.a + off, in ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+    auto load_v = [&](int cl) {
+        const int64_t tl = s0 + (int64_t)cl * kChunk;
+        const int Ll = static_cast<int>(min64(kChunk, s1 - tl));
+        constexpr int CPRV = DV / 8;
+#pragma unroll
+        for (int it = 0; it < 64 * CPRV / kRoleThreads; ++it) {
+            const int e = tid + it * kRoleThreads;
+            const int row = e / CPRV, ch = e % CPRV;
+            const bool in = row < Ll;
+            const int64_t off = ((tl + (in ? row : 0)) * H + h) * DV + ch * 8;
+            cp_async_16(aV + swz<RBV>(row, ch), p.v + off, in ? 16 : 0);
+        }
+        cp_async_commit();
+    };
 
     for (int c = rank; c < nchunks; c += G) {
         const int slot = c % R;
@@ -191,31 +231,16 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         // the slot's release counter, read early so its latency overlaps the loads
         const int empty_target = G * (c / R);
         int empty_seen = 0;
-        if (tid == 0 && c >= R) empty_seen = ld_acquire_gpu(flags + slot * 2 + 1);
+        if (tid == 0 && c >= R) empty_seen = ld_relaxed_gpu(flags + slot * 2 + 1);
 
-        // 1. q, k, a, v rows of the chunk into shared memory (rows >= L zero-filled), and beta;
-        //    then an L2 prefetch of the rows of this producer's next chunk
+        // 1. this chunk's q, k, a rows were requested at the end of the previous chunk's Gram
+        //    phase and its v rows at the end of the previous chunk (the very first chunk
+        //    requests them here); rows >= L are zero-filled.  Then an L2 prefetch of the rows of
+        //    this producer's next chunk.
         {
-            constexpr int CPR = DK / 8;  // 16-byte chunks per row
-#pragma unroll
-            for (int it = 0; it < 64 * CPR / kRoleThreads; ++it) {
-                const int e = tid + it * kRoleThreads;
-                const int row = e / CPR, ch = e % CPR;
-                const bool in = row < L;
-                const int64_t off = ((t0 + (in ? row : 0)) * H + h) * DK + ch * 8;
-                const uint32_t dst = swz<RB>(row, ch);
-                cp_async_16(aQhi + dst, p.q + off, in ? 16 : 0);
-                cp_async_16(aK + dst, p.k + off, in ? 16 : 0);
-                cp_async_16(aKr + dst, p.a + off, in ? 16 : 0);
-            }
-            constexpr int CPRV = DV / 8;
-#pragma unroll
-            for (int it = 0; it < 64 * CPRV / kRoleThreads; ++it) {
-                const int e = tid + it * kRoleThreads;
-                const int row = e / CPRV, ch = e % CPRV;
-                const bool in = row < L;
-                const int64_t off = ((t0 + (in ? row : 0)) * H + h) * DV + ch * 8;
-                cp_async_16(aV + swz<RBV>(row, ch), p.v + off, in ? 16 : 0);
+            if (c == rank) {
+                load_qka(c);
+                load_v(c);
             }
             if (tid < 64) sbeta[tid] = tid < L ? p.beta[(t0 + tid) * H + h] : 0.f;
             const int cn = c + G;
@@ -229,51 +254,31 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                     prefetch_l2_bulk(base + ((tn + row) * H + h) * d, d * 2);
                 }
             }
-            cp_async_wait_all();
+            cp_async_wait_group<1>();   // q, k, a of this chunk (v may still be in flight)
             named_bar(kBarProducer, kRoleThreads);
         }
 
-        // 2. log-decay g for every element (independent), then the chunk-local inclusive
-        //    cumsum b per channel (rows >= L carry g = 0)
-        {
-            constexpr int NIT = 64 * DK / kRoleThreads;
-            float gv[NIT];
-#pragma unroll
-            for (int it = 0; it < NIT; ++it) {   // all loads first, then the math, then the stores
-                const int e = tid + it * kRoleThreads;
-                gv[it] = bf16_to_f32(*reinterpret_cast<const uint16_t *>(sKr + swz_elem<RB>(e / DK, e % DK)));
-            }
-#pragma unroll
-            for (int it = 0; it < NIT; ++it) {
-                const int e = tid + it * kRoleThreads;
-                gv[it] = e / DK < L ? log_decay(gv[it], expA) : 0.f;
-            }
-#pragma unroll
-            for (int it = 0; it < NIT; ++it) {
-                const int e = tid + it * kRoleThreads;
-                bval(e / DK, e % DK) = gv[it];
-            }
-        }
-        named_bar(kBarProducer, kRoleThreads);
+        // 2. log-decay g and its chunk-local inclusive cumsum b (rows >= L carry g = 0).  Each
+        //    thread takes one channel and a contiguous run of tokens: the loads and the
+        //    exponentials are independent, only the running sum is sequential.
         {
             constexpr int PARTS = kRoleThreads / DK;   // 2 for d_k = 128, 4 for 64
             constexpr int TPP = 64 / PARTS;
             const int ch = tid % DK, part = tid / DK;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < TPP; ++i) {
-                float &x = bval(part * TPP + i, ch);
-                acc += x;
-                x = acc;
-            }
-            stot[part * DK + ch] = acc;
+            float gv[TPP];
+#pragma unroll
+            for (int i = 0; i < TPP; ++i)
+                gv[i] = bf16_to_f32(*reinterpret_cast<const uint16_t *>(sKr + swz_elem<RB>(part * TPP + i, ch)));
+#pragma unroll
+            for (int i = 0; i < TPP; ++i) gv[i] = part * TPP + i < L ? log_decay(gv[i], expA) : 0.f;
+#pragma unroll
+            for (int i = 1; i < TPP; ++i) gv[i] += gv[i - 1];
+            stot[part * DK + ch] = gv[TPP - 1];
             named_bar(kBarProducer, kRoleThreads);
-            if (part > 0) {
-                float off = 0.f;
-                for (int pp = 0; pp < part; ++pp) off += stot[pp * DK + ch];
-#pragma unroll 8
-                for (int i = 0; i < TPP; ++i) bval(part * TPP + i, ch) += off;
-            }
+            float off = 0.f;
+            for (int pp = 0; pp < part; ++pp) off += stot[pp * DK + ch];
+#pragma unroll
+            for (int i = 0; i < TPP; ++i) bval(part * TPP + i, ch) = gv[i] + off;
             named_bar(kBarProducer, kRoleThreads);
         }
 
@@ -300,9 +305,13 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         // the slot must be free (chunk c - R consumed by all G consumers) before any ring write
         if (tid == 0) {
             bool ok = true;
-            if (c >= R && empty_seen < empty_target) {
-                ok = wait_at_least(flags + slot * 2 + 1, empty_target, p.wait_ns);
-                if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
+            if (c >= R) {
+                if (empty_seen >= empty_target) {
+                    fence_acquire_gpu();   // the early relaxed read already showed the release
+                } else {
+                    ok = wait_at_least(flags + slot * 2 + 1, empty_target, p.wait_ns);
+                    if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
+                }
             }
             *abort_flag = ok ? 0 : 1;
         }
@@ -342,7 +351,8 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                 *reinterpret_cast<uint32_t *>(sKr + off) = pack_bf16(kv.x * rf0, kv.y * rf1);
                 *reinterpret_cast<float2 *>(sKt + swz_f32<DK>(t, ch)) = make_float2(kv.x * iv0, kv.y * iv1);
                 *reinterpret_cast<uint32_t *>(sKh + off) = pack_f16(kv.x * ep.x * rf0, kv.y * ep.y * rf1);
-                // K- = k e^{b_C - b} = k (e^{b_C - r_{p+1}}) (e^{r_{p+1} - r_p} e^{r_p - b}), each <= 1
+                // K- = k e^{b_C - b} = k (e^{b_C - r_{p+1}}) (e^{r_{p+1} - r_p} e^{r_p - b}), each
+                // <= 1; it overwrites k at the same element, which this thread has already read
                 *reinterpret_cast<uint32_t *>(sKb + off) =
                     pack_f16(kv.x * ab.x * (tt.x * iv0), kv.y * ab.y * (tt.y * iv1));
                 qfrag[e] = pack_f16(qv.x * ep.x * rf0, qv.y * ep.y * rf1);   // Q^ = q e^{b}
@@ -351,18 +361,19 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         }
         named_bar(kBarProducer, kRoleThreads);
 
-        // 4a. Gram blocks (p, q <= p), one n8 half per job: A = mask(Q K^T) (split bf16) and
-        //     L = beta * strict(K K^T) (bf16).  Column fragments are built in registers from K~
-        //     times e^{r_p - r_q} and split into bf16 hi + lo.
+        // 4a. Gram blocks (p, q <= p), one block per job (both n8 halves share the A fragments):
+        //     A = mask(Q K^T) (split bf16) and L = beta * strict(K K^T) (bf16).  Column fragments
+        //     are built in registers from K~ times e^{r_p - r_q} and split into bf16 hi + lo.
 #pragma unroll 1
-        for (int job = warp; job < 20; job += 8) {
-            const int blk = job >> 1, nt = job & 1;
+        for (int blk = warp; blk < 10; blk += 8) {
             const int pb = blk >= 6 ? 3 : blk >= 3 ? 2 : blk >= 1 ? 1 : 0;
             const int qb = blk - pb * (pb + 1) / 2;
-            const int jrow = 16 * qb + 8 * nt + g;   // column index j of this lane's B element
             const float *dcol = pb > qb ? sD + pair_index(pb, qb) * DK : nullptr;
-            float ahh[4] = {0.f, 0.f, 0.f, 0.f}, ahl[4] = {0.f, 0.f, 0.f, 0.f};
-            float alh[4] = {0.f, 0.f, 0.f, 0.f}, akk[4] = {0.f, 0.f, 0.f, 0.f};
+            float ahh[2][4], ahl[2][4], alh[2][4], akk[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ahh[nt][e] = ahl[nt][e] = alh[nt][e] = akk[nt][e] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < KT; ++ks) {
                 uint32_t ahi[4], alo[4], ak[4];
@@ -370,45 +381,51 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                 ldsm_x4(alo, ldsm_addr_a<RB>(aQlo, 16 * pb, 16 * ks, lane));
                 ldsm_x4(ak, ldsm_addr_a<RB>(aKr, 16 * pb, 16 * ks, lane));
                 const int c0 = 16 * ks + 2 * t4;
-                float2 k0 = *reinterpret_cast<const float2 *>(sKt + swz_f32<DK>(jrow, c0));
-                float2 k1 = *reinterpret_cast<const float2 *>(sKt + swz_f32<DK>(jrow, c0 + 8));
+                float2 d0 = make_float2(1.f, 1.f), d1 = d0;
                 if (dcol) {
-                    const float2 d0 = *reinterpret_cast<const float2 *>(dcol + c0);
-                    const float2 d1 = *reinterpret_cast<const float2 *>(dcol + c0 + 8);
-                    k0.x *= d0.x; k0.y *= d0.y; k1.x *= d1.x; k1.y *= d1.y;
+                    d0 = *reinterpret_cast<const float2 *>(dcol + c0);
+                    d1 = *reinterpret_cast<const float2 *>(dcol + c0 + 8);
                 }
-                uint32_t bh0, bl0, bh1, bl1;
-                split_bf16(k0.x, k0.y, bh0, bl0);
-                split_bf16(k1.x, k1.y, bh1, bl1);
-                mma_bf16(ahh, ahi, bh0, bh1);
-                mma_bf16(ahl, ahi, bl0, bl1);
-                mma_bf16(alh, alo, bh0, bh1);
-                mma_bf16(akk, ak, bh0, bh1);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int jrow = 16 * qb + 8 * nt + g;   // column j of this lane's B element
+                    float2 k0 = *reinterpret_cast<const float2 *>(sKt + swz_f32<DK>(jrow, c0));
+                    float2 k1 = *reinterpret_cast<const float2 *>(sKt + swz_f32<DK>(jrow, c0 + 8));
+                    k0.x *= d0.x; k0.y *= d0.y; k1.x *= d1.x; k1.y *= d1.y;
+                    uint32_t bh0, bl0, bh1, bl1;
+                    split_bf16(k0.x, k0.y, bh0, bl0);
+                    split_bf16(k1.x, k1.y, bh1, bl1);
+                    mma_bf16(ahh[nt], ahi, bh0, bh1);
+                    mma_bf16(ahl[nt], ahi, bl0, bl1);
+                    mma_bf16(alh[nt], alo, bh0, bh1);
+                    mma_bf16(akk[nt], ak, bh0, bh1);
+                }
             }
             const int i0 = 16 * pb + g, i1 = i0 + 8;
-            const int jc = 16 * qb + 8 * nt + 2 * t4;
             const bool diag = pb == qb;
-            float aq[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) aq[e] = ahh[e] + (ahl[e] + alh[e]);
-            // A fragment half (columns 8 nt .. 8 nt + 7 of the 16x16 tile), fp16
-            const float a0 = !diag || jc <= i0 ? aq[0] : 0.f;
-            const float a1 = !diag || jc + 1 <= i0 ? aq[1] : 0.f;
-            const float a2 = !diag || jc <= i1 ? aq[2] : 0.f;
-            const float a3 = !diag || jc + 1 <= i1 ? aq[3] : 0.f;
-            stg_v2(slotp + RL::kA + blk * 512 + lane * 16 + nt * 8, pack_f16(a0, a1), pack_f16(a2, a3));
             const float b0 = sbeta[i0], b1 = sbeta[i1];
-            if (diag) {   // fp32 diagonal block for the 16x16 inverses
-                const int li = g, lj = 8 * nt + 2 * t4;
-                float *Ld = sLd + pb * 16 * 17;
-                Ld[li * 17 + lj] = lj < li ? b0 * akk[0] : 0.f;
-                Ld[li * 17 + lj + 1] = lj + 1 < li ? b0 * akk[1] : 0.f;
-                Ld[(li + 8) * 17 + lj] = lj < li + 8 ? b1 * akk[2] : 0.f;
-                Ld[(li + 8) * 17 + lj + 1] = lj + 1 < li + 8 ? b1 * akk[3] : 0.f;
-            } else {      // -L below the diagonal blocks, fp16, as the A operand of the solve
-                *reinterpret_cast<uint32_t *>(sLD + swz_elem<128>(i0, jc)) = pack_f16(-b0 * akk[0], -b0 * akk[1]);
-                *reinterpret_cast<uint32_t *>(sLD + swz_elem<128>(i1, jc)) = pack_f16(-b1 * akk[2], -b1 * akk[3]);
+            uint32_t afr[4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int jc = 16 * qb + 8 * nt + 2 * t4;
+                float aq[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) aq[e] = ahh[nt][e] + (ahl[nt][e] + alh[nt][e]);
+                afr[2 * nt] = pack_f16(!diag || jc <= i0 ? aq[0] : 0.f, !diag || jc + 1 <= i0 ? aq[1] : 0.f);
+                afr[2 * nt + 1] = pack_f16(!diag || jc <= i1 ? aq[2] : 0.f, !diag || jc + 1 <= i1 ? aq[3] : 0.f);
+                if (diag) {   // fp32 diagonal block for the 16x16 inverses
+                    const int li = g, lj = 8 * nt + 2 * t4;
+                    float *Ld = sLd + pb * 16 * 17;
+                    Ld[li * 17 + lj] = lj < li ? b0 * akk[nt][0] : 0.f;
+                    Ld[li * 17 + lj + 1] = lj + 1 < li ? b0 * akk[nt][1] : 0.f;
+                    Ld[(li + 8) * 17 + lj] = lj < li + 8 ? b1 * akk[nt][2] : 0.f;
+                    Ld[(li + 8) * 17 + lj + 1] = lj + 1 < li + 8 ? b1 * akk[nt][3] : 0.f;
+                } else {      // -L below the diagonal blocks, fp16 A operand of the block products
+                    *reinterpret_cast<uint32_t *>(sLD + swz_elem<128>(i0, jc)) = pack_f16(-b0 * akk[nt][0], -b0 * akk[nt][1]);
+                    *reinterpret_cast<uint32_t *>(sLD + swz_elem<128>(i1, jc)) = pack_f16(-b1 * akk[nt][2], -b1 * akk[nt][3]);
+                }
             }
+            stg_v4(slotp + RL::kA + blk * 512 + lane * 16, make_uint4(afr[0], afr[1], afr[2], afr[3]));
         }
         // 4b. K-^T fragments and Gamma_C
         for (int idx = warp; idx < 4 * KT; idx += 8) {
@@ -420,8 +437,11 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         if (tid < DK)   // e^{b_C} = e^{r_3} e^{b_C - r_3}
             reinterpret_cast<float *>(slotp + RL::kGam)[tid] = sEP[3 * DK + tid] * sTT[3 * DK + tid];
         named_bar(kBarProducer, kRoleThreads);
+        // the q, k (now K-) and a (now K r) buffers are no longer read: request the next chunk's
+        if (c + G < nchunks) load_qka(c + G);
 
-        // 5. diagonal blocks D_p = (I + L_pp)^-1 by forward substitution (fp32), one column per lane
+        // 5. diagonal blocks D_p = (I + L_pp)^-1 by forward substitution (fp32), one column per lane;
+        //    written as fp16 into the diagonal blocks of both LD and T
         if (warp < 4 && lane < 16) {
             const int pb = warp, mcol = lane;
             const float *Ld = sLd + pb * 16 * 17;
@@ -434,84 +454,104 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                 x[i] = i >= mcol ? v : 0.f;
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                *reinterpret_cast<__half *>(sLD + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = __float2half_rn(x[i]);
+            for (int i = 0; i < 16; ++i) {
+                const __half hv = __float2half_rn(x[i]);
+                *reinterpret_cast<__half *>(sLD + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = hv;
+                *reinterpret_cast<__half *>(sT + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = hv;
+            }
         }
         named_bar(kBarProducer, kRoleThreads);
 
-        // 6. [W | U~] = (I + L)^-1 diag(beta) [K^ | V], blocked forward substitution per 16-row block:
-        //    X_p = D_p (B_p - sum_{m<p} L_pm X_m).  Each warp owns 16-column units of X, so the
-        //    whole solve is warp-local; X_p (fp16) is kept in shared memory for later blocks.
+        // 5b. off-diagonal blocks of T = (I + L)^-1 by level d = p - q:
+        //     T_pq = D_p M,  M = sum_{m=q}^{p-1} (-L_pm) T_mq   (16x16 tensor-core products)
+#pragma unroll 1
+        for (int d = 1; d < 4; ++d) {
+            if (warp < 4 - d) {
+                const int qb = warp, pb = warp + d;
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                for (int mb = qb; mb < pb; ++mb) {
+                    uint32_t af[4], bf[4];
+                    ldsm_x4(af, ldsm_addr_a<128>(aLD, 16 * pb, 16 * mb, lane));   // -L_pm
+                    ldsm_x4_t(bf, ldsm_addr_bt<128>(aT, 16 * mb, 16 * qb, lane));  // T_mq
+                    mma_f16(acc[0], af, bf[0], bf[1]);
+                    mma_f16(acc[1], af, bf[2], bf[3]);
+                }
+                const uint32_t aMw = aM + warp * 16 * 64;
+                unsigned char *const sMw = sM + warp * 16 * 64;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int cc = 8 * j + 2 * t4;
+                    *reinterpret_cast<uint32_t *>(sMw + swz_elem<64>(g, cc)) = pack_f16(acc[j][0], acc[j][1]);
+                    *reinterpret_cast<uint32_t *>(sMw + swz_elem<64>(g + 8, cc)) = pack_f16(acc[j][2], acc[j][3]);
+                }
+                __syncwarp();
+                float tq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                {
+                    uint32_t af[4], bf[4];
+                    ldsm_x4(af, ldsm_addr_a<128>(aLD, 16 * pb, 16 * pb, lane));   // D_p
+                    ldsm_x4_t(bf, ldsm_addr_bt<64>(aMw, 0, 0, lane));              // M
+                    mma_f16(tq[0], af, bf[0], bf[1]);
+                    mma_f16(tq[1], af, bf[2], bf[3]);
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int cc = 16 * qb + 8 * j + 2 * t4;
+                    *reinterpret_cast<uint32_t *>(sT + swz_elem<128>(16 * pb + g, cc)) = pack_f16(tq[j][0], tq[j][1]);
+                    *reinterpret_cast<uint32_t *>(sT + swz_elem<128>(16 * pb + g + 8, cc)) = pack_f16(tq[j][2], tq[j][3]);
+                }
+            }
+            named_bar(kBarProducer, kRoleThreads);
+        }
+        // T' = T diag(beta), lower triangle (blocks above the diagonal are never read)
+        for (int e = tid; e < 64 * 32; e += kRoleThreads) {
+            const int i = e >> 5, j = (e & 31) * 2;
+            if ((j >> 4) <= (i >> 4)) {
+                const float2 tv = unpack_f16(*reinterpret_cast<const uint32_t *>(sT + swz_elem<128>(i, j)));
+                *reinterpret_cast<uint32_t *>(sTp + swz_elem<128>(i, j)) = pack_f16(tv.x * sbeta[j], tv.y * sbeta[j + 1]);
+            }
+        }
+        named_bar(kBarProducer, kRoleThreads);
+
+        // v of this chunk (its group is older than the next chunk's q, k, a group)
+        if (c + G < nchunks) cp_async_wait_group<1>();
+        else cp_async_wait_group<0>();
+        named_bar(kBarProducer, kRoleThreads);
+
+        // 6. [W | U~] = T' [K^ | V].  Warp w owns 16-column units w and w + 8 of [W | U~]; the B
+        //    fragments of a unit are loaded once per token tile and reused for every row tile.
         {
             constexpr int UW = DK / 16, UT = (DK + DV) / 16;
 #pragma unroll 1
             for (int u = warp; u < UT; u += 8) {
                 const bool isW = u < UW;
-                const int xc = 16 * u;                          // column in X
-                const int vc = isW ? xc : xc - DK;              // column in K^ or V
-#pragma unroll 1
-                for (int pb = 0; pb < 4; ++pb) {
-                    const int r0 = 16 * pb + g, r1 = r0 + 8;
-                    const float b0 = sbeta[r0], b1 = sbeta[r1];
-                    float acc[2][4];
+                const int vc = isW ? 16 * u : 16 * u - DK;    // column in K^ or V
+                uint32_t bfr[4][4];
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int cc = vc + 8 * j + 2 * t4;
-                        float2 x0, x1;
-                        if (isW) {
-                            x0 = unpack_f16(*reinterpret_cast<const uint32_t *>(sKh + swz_elem<RB>(r0, cc)));
-                            x1 = unpack_f16(*reinterpret_cast<const uint32_t *>(sKh + swz_elem<RB>(r1, cc)));
-                        } else {
-                            x0 = unpack_bf16(*reinterpret_cast<const uint32_t *>(sV + swz_elem<RBV>(r0, cc)));
-                            x1 = unpack_bf16(*reinterpret_cast<const uint32_t *>(sV + swz_elem<RBV>(r1, cc)));
-                        }
-                        acc[j][0] = b0 * x0.x; acc[j][1] = b0 * x0.y;
-                        acc[j][2] = b1 * x1.x; acc[j][3] = b1 * x1.y;
-                    }
+                for (int kt = 0; kt < 4; ++kt) {
+                    if (isW) {
+                        ldsm_x4_t(bfr[kt], ldsm_addr_bt<RB>(aKh, 16 * kt, vc, lane));
+                    } else {
+                        ldsm_x4_t(bfr[kt], ldsm_addr_bt<RBV>(aV, 16 * kt, vc, lane));
 #pragma unroll
-                    for (int mb = 0; mb < 3; ++mb) {
-                        if (mb >= pb) break;
-                        uint32_t af[4], bf[4];
-                        ldsm_x4(af, ldsm_addr_a<128>(aLD, 16 * pb, 16 * mb, lane));   // -L_pm
-                        ldsm_x4_t(bf, ldsm_addr_bt<RBX>(aX, 16 * mb, xc, lane));      // X_m
-                        mma_f16(acc[0], af, bf[0], bf[1]);
-                        mma_f16(acc[1], af, bf[2], bf[3]);
+                        for (int e = 0; e < 4; ++e) bfr[kt][e] = bf16x2_to_f16x2(bfr[kt][e]);
                     }
-                    // R_p -> shared memory (this warp's columns), then X_p = D_p R_p
+                }
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int cc = xc + 8 * j + 2 * t4;
-                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r0, cc)) = pack_f16(acc[j][0], acc[j][1]);
-                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r1, cc)) = pack_f16(acc[j][2], acc[j][3]);
-                    }
-                    __syncwarp();
-                    float xp[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                    {
-                        uint32_t af[4], bf[4];
-                        ldsm_x4(af, ldsm_addr_a<128>(aLD, 16 * pb, 16 * pb, lane));   // D_p
-                        ldsm_x4_t(bf, ldsm_addr_bt<RBX>(aX, 16 * pb, xc, lane));      // R_p
-                        mma_f16(xp[0], af, bf[0], bf[1]);
-                        mma_f16(xp[1], af, bf[2], bf[3]);
-                    }
-                    __syncwarp();
-                    uint32_t fr[4];
-                    fr[0] = pack_f16(xp[0][0], xp[0][1]);
-                    fr[1] = pack_f16(xp[0][2], xp[0][3]);
-                    fr[2] = pack_f16(xp[1][0], xp[1][1]);
-                    fr[3] = pack_f16(xp[1][2], xp[1][3]);
+                for (int m = 0; m < 4; ++m) {
+                    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int cc = xc + 8 * j + 2 * t4;
-                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r0, cc)) = fr[2 * j];
-                        *reinterpret_cast<uint32_t *>(sX + swz_elem<RBX>(r1, cc)) = fr[2 * j + 1];
+                    for (int kt = 0; kt <= m; ++kt) {
+                        uint32_t af[4];
+                        ldsm_x4(af, ldsm_addr_a<128>(aTp, 16 * m, 16 * kt, lane));
+                        mma_f16(acc[0], af, bfr[kt][0], bfr[kt][1]);
+                        mma_f16(acc[1], af, bfr[kt][2], bfr[kt][3]);
                     }
-                    __syncwarp();
-                    if (isW) {   // W tile (token tile pb, d_k tile u): an A fragment
-                        stg_v4(slotp + RL::kW + (pb * KT + u) * 512 + lane * 16, make_uint4(fr[0], fr[1], fr[2], fr[3]));
+                    const uint4 fr = make_uint4(pack_f16(acc[0][0], acc[0][1]), pack_f16(acc[0][2], acc[0][3]),
+                                                pack_f16(acc[1][0], acc[1][1]), pack_f16(acc[1][2], acc[1][3]));
+                    if (isW) {   // W tile (token tile m, d_k tile u): an A fragment
+                        stg_v4(slotp + RL::kW + (m * KT + u) * 512 + lane * 16, fr);
                     } else {     // U~: half (vc / 16) % 2 of slab vc / 32
-                        const int sl = vc / kSlab, half = (vc / 16) & 1;
-                        stg_v4(slotp + RL::kU + ((pb * G + sl) * 32 + lane) * 32 + half * 16,
-                               make_uint4(fr[0], fr[1], fr[2], fr[3]));
+                        stg_v4(slotp + RL::kU + ((m * G + vc / kSlab) * 32 + lane) * 32 + ((vc >> 4) & 1) * 16, fr);
                     }
                 }
             }
@@ -521,11 +561,19 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             __threadfence();
             st_release_gpu(flags + slot * 2, c + 1);
         }
+        if (c + G < nchunks) load_v(c + G);   // the v buffer is free now
     }
 }
 
 // ---------------------------------------------------------------------------------------------
 // Consumer: the sequential state pass for slab `rank` (32 columns of d_v) of one unit.
+//
+// Per chunk c, with the state S_c (fp32 registers; fp16 copy in shared memory as the B operand):
+//   U = U~ - W S_c  ->  shared memory;   S_{c+1} = Diag(Gamma_C) S_c + K-^T U;
+//   O = Q^ S_c + A U, gated and stored.
+// The chain operands (W, U~ and K-^T, Gamma_C) of chunk c + 1 are copied from the ring into
+// shared memory while chunk c runs: W and U~ as soon as chunk c has read them, K-^T and Gamma_C
+// at the end of chunk c.  Q^ and A go to registers at the start of their chunk (off the chain).
 // ---------------------------------------------------------------------------------------------
 template <int DK, int DV>
 __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned char *sm, int unit,
@@ -538,14 +586,55 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
-    unsigned char *const sS = sm + SM::kS;
-    unsigned char *const sU = sm + SM::kU;
+    unsigned char *const sS = sm + SM::kS, *const sU = sm + SM::kU;
+    unsigned char *const sPW = sm + SM::kPW, *const sPK = sm + SM::kPK, *const sPU = sm + SM::kPU;
+    const float *const sPG = reinterpret_cast<const float *>(sm + SM::kPG);
     const uint32_t aS = smem_u32(sS), aU = smem_u32(sU);
+    const uint32_t aPW = smem_u32(sPW), aPK = smem_u32(sPK), aPU = smem_u32(sPU), aPG = smem_u32(sm + SM::kPG);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(sm + SM::kCFlag);
     const int64_t H = p.H;
     const int col0 = rank * kSlab;
     int *const flags = p.flags + (size_t)unit * R * 2;
     const char *const ring = p.ring + (size_t)unit * R * RL::kBytes;
+    auto slot_of = [&](int c) { return ring + (size_t)(c % R) * RL::kBytes; };
+
+    // ring -> shared memory copies of the chain operands (16-byte cp.async, L2 only)
+    auto prefetch_wu = [&](int c) {   // W tiles and this slab's U~
+        const char *sp = slot_of(c);
+#pragma unroll
+        for (int it = 0; it < 4 * KT * 32 / kRoleThreads; ++it) {
+            const int e = tid + it * kRoleThreads;   // 16-byte piece of the W tiles
+            cp_async_16(aPW + e * 16, sp + RL::kW + e * 16, 16);
+        }
+        {   // U~ of slab `rank`: 4 token tiles x 1 KB
+            const int m = tid >> 6, piece = tid & 63;
+            cp_async_16(aPU + m * 1024 + piece * 16, sp + RL::kU + (m * G + rank) * 1024 + piece * 16, 16);
+        }
+        cp_async_commit();
+    };
+    auto prefetch_kg = [&](int c) {   // K-^T tiles and Gamma_C
+        const char *sp = slot_of(c);
+#pragma unroll
+        for (int it = 0; it < 4 * KT * 32 / kRoleThreads; ++it) {
+            const int e = tid + it * kRoleThreads;
+            cp_async_16(aPK + e * 16, sp + RL::kKbT + e * 16, 16);
+        }
+        if (tid < DK / 4) cp_async_16(aPG + tid * 16, sp + RL::kGam + tid * 16, 16);
+        cp_async_commit();
+    };
+    // thread 0 waits for chunk c to be published; the role's barrier publishes the outcome
+    auto wait_full = [&](int c, int seen) {
+        if (tid == 0) {
+            bool ok = true;
+            if (seen >= c + 1) {
+                fence_acquire_gpu();   // the early relaxed read already showed the publication
+            } else {
+                ok = wait_at_least(flags + (c % R) * 2, c + 1, p.wait_ns);
+                if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
+            }
+            *abort_flag = ok ? 0 : 1;
+        }
+    };
 
     // state tile of this warp: d_k rows 16 md + (g, g+8), slab columns 8 (sn0 + j) + 2 t4 (+1)
     const int md = DK == 128 ? warp : (warp & 3);
@@ -566,9 +655,8 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     }
     // output tile of this warp: token rows 16 m + (g, g+8), slab columns 16 ch + 8 j + 2 t4 (+1)
     const int m = warp & 3, ch = warp >> 2;
-
     const int i0 = 16 * m + g, i1 = i0 + 8;
-    // gate logits of the next chunk, loaded a chunk ahead (they come from HBM)
+    // gate logits of a chunk, loaded a chunk ahead (they come from HBM)
     auto load_gate = [&](int cg, uint32_t (&gt)[2][2]) {
         gt[0][0] = gt[0][1] = gt[1][0] = gt[1][1] = 0u;
         if (!p.gate || cg >= nchunks) return;
@@ -583,48 +671,43 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     };
     uint32_t gt[2][2];
     load_gate(0, gt);
-    // the next chunk's `full` counter, read early so its latency overlaps the current chunk
-    int full_seen = 0;
-    if (tid == 0 && nchunks > 0) full_seen = ld_acquire_gpu(flags);
+
+    if (nchunks > 0) {
+        wait_full(0, 0);
+        named_bar(kBarConsumer, kRoleThreads);
+        if (*abort_flag) return;
+        prefetch_wu(0);
+        prefetch_kg(0);
+    }
 
     for (int c = 0; c < nchunks; ++c) {
-        // fp16 copy of the state: the B operand of W S and Q^ S
+        const char *const slotp = slot_of(c);
+        const int64_t t0 = s0 + (int64_t)c * kChunk;
+        const int L = static_cast<int>(min64(kChunk, s1 - t0));
+        const bool has_next = c + 1 < nchunks;
+        // 1. fp16 copy of S_c (B operand of W S and Q^ S); early read of chunk c+1's counter;
+        //    Q^ and A of chunk c and the next chunk's gate into registers
 #pragma unroll
         for (int j = 0; j < SNT; ++j) {
             const int cc = 8 * (sn0 + j) + 2 * t4;
             *reinterpret_cast<uint32_t *>(sS + swz_elem<64>(r0, cc)) = pack_f16(S[j][0], S[j][1]);
             *reinterpret_cast<uint32_t *>(sS + swz_elem<64>(r1, cc)) = pack_f16(S[j][2], S[j][3]);
         }
-        const int slot = c % R;
-        if (tid == 0) {
-            bool ok = true;
-            if (full_seen < c + 1) {
-                ok = wait_at_least(flags + slot * 2, c + 1, p.wait_ns);
-                if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
-            }
-            *abort_flag = ok ? 0 : 1;
-        }
-        named_bar(kBarConsumer, kRoleThreads);
-        if (*abort_flag) return;
-        const char *const slotp = ring + (size_t)slot * RL::kBytes;
-        const int64_t t0 = s0 + (int64_t)c * kChunk;
-        const int L = static_cast<int>(min64(kChunk, s1 - t0));
-
-        uint4 Wf[KT], Af[4], Kf[4];
+        int full_seen = 0;
+        if (tid == 0 && has_next) full_seen = ld_relaxed_gpu(flags + ((c + 1) % R) * 2);
+        uint4 Qf[KT], Af[4];
 #pragma unroll
-        for (int kd = 0; kd < KT; ++kd) Wf[kd] = ldg_cg_v4(slotp + RL::kW + (m * KT + kd) * 512 + lane * 16);
+        for (int kd = 0; kd < KT; ++kd) Qf[kd] = ldg_cg_v4(slotp + RL::kQ + (m * KT + kd) * 512 + lane * 16);
 #pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
+        for (int kt = 0; kt < 4; ++kt)
             Af[kt] = kt <= m ? ldg_cg_v4(slotp + RL::kA + (m * (m + 1) / 2 + kt) * 512 + lane * 16)
                              : make_uint4(0, 0, 0, 0);
-            Kf[kt] = ldg_cg_v4(slotp + RL::kKbT + (md * 4 + kt) * 512 + lane * 16);
-        }
-        const uint4 Uf = ldg_cg_v4(slotp + RL::kU + ((m * G + rank) * 32 + lane) * 32 + ch * 16);
-        const float gam0 = __ldcg(reinterpret_cast<const float *>(slotp + RL::kGam) + r0);
-        const float gam1 = __ldcg(reinterpret_cast<const float *>(slotp + RL::kGam) + r1);
+        uint32_t gtn[2][2];
+        load_gate(c + 1, gtn);
+        cp_async_wait_group<1>();                  // this thread's W, U~ copies of chunk c
+        named_bar(kBarConsumer, kRoleThreads);     // all copies and sS visible
 
-        // U = U~ - W S  (the chain; two independent partial sums halve the dependent MMAs),
-        // then O = Q^ S
+        // 2. U = U~ - W S_c  (the chain; two independent partial sums halve the dependent MMAs)
         float accU[2][4], accV[2][4], accO[2][4];
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -634,7 +717,8 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         for (int kd = 0; kd < KT; ++kd) {
             uint32_t bf[4];
             ldsm_x4_t(bf, ldsm_addr_bt<64>(aS, 16 * kd, 16 * ch, lane));
-            const uint32_t wa[4] = {Wf[kd].x, Wf[kd].y, Wf[kd].z, Wf[kd].w};
+            const uint4 w4 = *reinterpret_cast<const uint4 *>(sPW + (m * KT + kd) * 512 + lane * 16);
+            const uint32_t wa[4] = {w4.x, w4.y, w4.z, w4.w};
             if (kd & 1) {
                 mma_f16(accV[0], wa, bf[0], bf[1]);
                 mma_f16(accV[1], wa, bf[2], bf[3]);
@@ -643,50 +727,50 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                 mma_f16(accU[1], wa, bf[2], bf[3]);
             }
         }
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) accU[j][e] += accV[j][e];
         {
-            const uint32_t uw[4] = {Uf.x, Uf.y, Uf.z, Uf.w};
+            const uint4 u4 = *reinterpret_cast<const uint4 *>(sPU + m * 1024 + lane * 32 + ch * 16);
+            const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const float2 ut0 = unpack_f16(uw[2 * j]), ut1 = unpack_f16(uw[2 * j + 1]);
-                accU[j][0] = ut0.x - accU[j][0];
-                accU[j][1] = ut0.y - accU[j][1];
-                accU[j][2] = ut1.x - accU[j][2];
-                accU[j][3] = ut1.y - accU[j][3];
+                const float u0 = ut0.x - (accU[j][0] + accV[j][0]), u1 = ut0.y - (accU[j][1] + accV[j][1]);
+                const float u2 = ut1.x - (accU[j][2] + accV[j][2]), u3 = ut1.y - (accU[j][3] + accV[j][3]);
                 const int cc = 16 * ch + 8 * j + 2 * t4;
-                *reinterpret_cast<uint32_t *>(sU + swz_elem<64>(i0, cc)) = pack_f16(accU[j][0], accU[j][1]);
-                *reinterpret_cast<uint32_t *>(sU + swz_elem<64>(i1, cc)) = pack_f16(accU[j][2], accU[j][3]);
+                *reinterpret_cast<uint32_t *>(sU + swz_elem<64>(i0, cc)) = pack_f16(u0, u1);
+                *reinterpret_cast<uint32_t *>(sU + swz_elem<64>(i1, cc)) = pack_f16(u2, u3);
             }
         }
+        // 3. chunk c+1 must be published before its W and U~ are copied
+        if (has_next) wait_full(c + 1, full_seen);
+        cp_async_wait_group<0>();                  // this thread's K-^T, Gamma_C copies of chunk c
+        named_bar(kBarConsumer, kRoleThreads);     // U complete; W, U~ buffers free; K-^T visible
+        if (has_next && *abort_flag) return;
+        if (has_next) prefetch_wu(c + 1);
+
+        // 4. O = Q^ S_c (off the chain)
 #pragma unroll
         for (int kd = 0; kd < KT; ++kd) {
             uint32_t bf[4];
             ldsm_x4_t(bf, ldsm_addr_bt<64>(aS, 16 * kd, 16 * ch, lane));
-            const uint4 q4 = ldg_cg_v4(slotp + RL::kQ + (m * KT + kd) * 512 + lane * 16);
-            const uint32_t qa[4] = {q4.x, q4.y, q4.z, q4.w};
+            const uint32_t qa[4] = {Qf[kd].x, Qf[kd].y, Qf[kd].z, Qf[kd].w};
             mma_f16(accO[0], qa, bf[0], bf[1]);
             mma_f16(accO[1], qa, bf[2], bf[3]);
         }
-        uint32_t gtn[2][2];
-        load_gate(c + 1, gtn);
-        if (tid == 0 && c + 1 < nchunks) full_seen = ld_acquire_gpu(flags + ((c + 1) % R) * 2);
-        named_bar(kBarConsumer, kRoleThreads);   // U complete in shared memory
 
-        // S = Diag(Gamma_C) S + K-^T U   (the chain)
-#pragma unroll
-        for (int j = 0; j < SNT; ++j) {
-            S[j][0] *= gam0; S[j][1] *= gam0; S[j][2] *= gam1; S[j][3] *= gam1;
-        }
+        // 5. S_{c+1} = Diag(Gamma_C) S_c + K-^T U   (the chain)
         {
+            const float gam0 = sPG[r0], gam1 = sPG[r1];
+#pragma unroll
+            for (int j = 0; j < SNT; ++j) {
+                S[j][0] *= gam0; S[j][1] *= gam0; S[j][2] *= gam1; S[j][3] *= gam1;
+            }
             float Sx[SNT][4];   // odd token tiles accumulate separately (two short chains)
 #pragma unroll
             for (int j = 0; j < SNT; ++j) Sx[j][0] = Sx[j][1] = Sx[j][2] = Sx[j][3] = 0.f;
 #pragma unroll
             for (int kt = 0; kt < 4; ++kt) {
-                const uint32_t ka[4] = {Kf[kt].x, Kf[kt].y, Kf[kt].z, Kf[kt].w};
+                const uint4 k4 = *reinterpret_cast<const uint4 *>(sPK + (md * 4 + kt) * 512 + lane * 16);
+                const uint32_t ka[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                 for (int np = 0; np < SNT / 2; ++np) {
                     uint32_t bf[4];
@@ -701,7 +785,8 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
 #pragma unroll
                 for (int e = 0; e < 4; ++e) S[j][e] += Sx[j][e];
         }
-        // O += A U, gate, store
+
+        // 6. O += A U, gate, store
 #pragma unroll
         for (int kt = 0; kt < 4; ++kt) {
             if (kt <= m) {
@@ -733,9 +818,10 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             }
         }
         gt[0][0] = gtn[0][0]; gt[0][1] = gtn[0][1]; gt[1][0] = gtn[1][0]; gt[1][1] = gtn[1][1];
-        // every warp is done with this slot and with sS / sU before they are rewritten
+        // 7. every warp is done with this slot, sS, sU and the K-^T buffer
         named_bar(kBarConsumer, kRoleThreads);
-        if (tid == 0) red_release_add_gpu(flags + slot * 2 + 1, 1);
+        if (tid == 0) red_release_add_gpu(flags + (c % R) * 2 + 1, 1);
+        if (has_next) prefetch_kg(c + 1);
     }
     if (p.S_out) {
 #pragma unroll
