@@ -95,6 +95,29 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+# ---- multi-rank plumbing (no data-path collective: every rank runs its own batch) --------------
+
+def rank_workload(w, rank: int):
+    """Weak scaling: rank r runs an independent batch of the same workload (seed + r)."""
+    return w.replace(seed=w.seed + rank)
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (the job finishes when the slowest rank does)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
 # ---- clocks sampled during the timed regions (NVML, read-only) -----------------------------------
 
 class ClockSampler:
@@ -255,14 +278,7 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    w = KI.WORKLOADS[args.workload].replace(seed=KI.WORKLOADS[args.workload].seed + rank)
+    w = rank_workload(KI.WORKLOADS[args.workload], rank)
     inp = KI.make_inputs(w, dev)
     max_seqlen = max(w.seqlens)
     ws_bytes = kda.kda_chunk_fwd_workspace_size(w.total_tokens, w.num_seqs, max_seqlen, w.H,
@@ -295,8 +311,8 @@ def main():
     launches = kda.kda_launch_count() - launches0
     barrier()
     kda.kda_sync_check()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    value = w.total_tokens * world / (ms * 1e-3)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    value = whole_job_rate(w.total_tokens, world, ms)
 
     hbm, tf, tf_sus, peak_src = peaks()
     bytes_step = prefill_bytes(w)
@@ -337,11 +353,11 @@ def main():
         clocks.active(False)
         barrier()
         kda.kda_sync_check()
-        dms = max_over_ranks(e0.elapsed_time(e1) / dw.steps)
+        dms = max_over_ranks(e0.elapsed_time(e1) / dw.steps, world, dev)
         dbytes = decode_bytes(dw)
         dach = dbytes / (dms * 1e-3) / 1e9
-        decode = {"value": world / (dms * 1e-3), "unit": "steps/s", "ms_per_step": dms,
-                  "workload": dw.name, "tokens_per_s": world * dw.N / (dms * 1e-3),
+        decode = {"value": whole_job_rate(1, world, dms), "unit": "steps/s", "ms_per_step": dms,
+                  "workload": dw.name, "tokens_per_s": whole_job_rate(dw.N, world, dms),
                   "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
                                "frac": dach / hbm, "traffic": None,
                                "peak_source": f"hbm_gbs of {peak_src}",
@@ -380,8 +396,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-        e2e = {"value": w.total_tokens * world / (ems * 1e-3), "unit": "tokens/s",
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+        e2e = {"value": whole_job_rate(w.total_tokens, world, ems), "unit": "tokens/s",
                "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None

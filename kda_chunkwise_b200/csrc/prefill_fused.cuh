@@ -224,6 +224,14 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         cp_async_commit();
     };
 
+    // beta of a chunk (64 scattered floats), loaded a chunk ahead into registers
+    auto load_beta = [&](int cl) -> float {
+        if (tid >= 64 || cl >= nchunks) return 0.f;
+        const int64_t tl = s0 + (int64_t)cl * kChunk;
+        return tid < min64(kChunk, s1 - tl) ? __ldg(p.beta + (tl + tid) * H + h) : 0.f;
+    };
+    float beta_next = load_beta(rank);
+
     for (int c = rank; c < nchunks; c += G) {
         const int slot = c % R;
         const int64_t t0 = s0 + (int64_t)c * kChunk;
@@ -242,7 +250,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                 load_qka(c);
                 load_v(c);
             }
-            if (tid < 64) sbeta[tid] = tid < L ? p.beta[(t0 + tid) * H + h] : 0.f;
+            if (tid < 64) sbeta[tid] = beta_next;   // loaded one chunk ahead
             const int cn = c + G;
             if (cn < nchunks) {
                 const int64_t tn = s0 + (int64_t)cn * kChunk;
@@ -257,6 +265,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             cp_async_wait_group<1>();   // q, k, a of this chunk (v may still be in flight)
             named_bar(kBarProducer, kRoleThreads);
         }
+        beta_next = load_beta(c + G);
 
         // 2. log-decay g and its chunk-local inclusive cumsum b (rows >= L carry g = 0).  Each
         //    thread takes one channel and a contiguous run of tokens: the loads and the
@@ -818,9 +827,10 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             }
         }
         gt[0][0] = gtn[0][0]; gt[0][1] = gtn[0][1]; gt[1][0] = gtn[1][0]; gt[1][1] = gtn[1][1];
-        // 7. every warp is done with this slot, sS, sU and the K-^T buffer
+        // 7. every warp is done with this slot, sS, sU and the K-^T buffer.  Every value read from
+        //    the slot has already been consumed, so returning it needs no release ordering.
         named_bar(kBarConsumer, kRoleThreads);
-        if (tid == 0) red_release_add_gpu(flags + (c % R) * 2 + 1, 1);
+        if (tid == 0) red_relaxed_add_gpu(flags + (c % R) * 2 + 1, 1);
         if (has_next) prefetch_kg(c + 1);
     }
     if (p.S_out) {
