@@ -80,7 +80,8 @@ typedef enum kda_dtype {
  *   non-zero bound is reported through the error word (the result is still computed in full).
  * scale multiplies q.  workspace: device scratch of at least kda_chunk_fwd_workspace_min(...)
  *   bytes (equal to kda_chunk_fwd_workspace_size(...)), 256-byte aligned; it holds per-unit rings
- *   of chunk records (about 0.55 MiB per (sequence, head) at d = 128) and is reused across calls.
+ *   of chunk records (about 0.55 MiB per (sequence, head) at d = 128); its contents need no
+ *   initialisation and it may be reused across calls on one stream.
  * A zero-length sequence copies its initial state (or zeros) to final_state.
  * total_tokens == 0 or num_seqs == 0 is valid and only writes final_state.
  */
@@ -157,6 +158,21 @@ KDA_API const char *kda_last_error(void);
 
 /* Number of CUDA kernels this process has launched through libkda so far (all devices). */
 KDA_API uint64_t kda_launch_count(void);
+
+/*
+ * kda_inject_stall — failure injection for tests of the bounded waits.  (No counterpart in the
+ * pages: the method has no inter-CTA waits; this exercises the library's own failure handling.)
+ *
+ * enable != 0: every later prefill launch in this process (kda_chunk_fwd, kda_chunk_fwd_noalloc)
+ *   withholds the publication of chunk 0 of every (sequence, head) unit, so the waits on it can
+ *   never be satisfied, and every device-side wait gives up after wait_limit_ns nanoseconds
+ *   (1e6 <= wait_limit_ns <= 4e9, else KDA_ERR_INVALID_ARG).  Such a call still returns KDA_OK;
+ *   its outputs are undefined, and the following kda_sync_check returns KDA_ERR_TIMEOUT.  The
+ *   CUDA context stays usable.
+ * enable == 0: back to normal operation (wait_limit_ns is ignored; the bound returns to 4 s).
+ * Process-wide; not synchronised with launches in flight on other threads.
+ */
+KDA_API kda_status kda_inject_stall(int32_t enable, uint64_t wait_limit_ns);
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,7 @@ import torch
 
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_chunk_fwd_workspace_min", "kda_sync_check", "kda_status_string", "KDAError",
-           "kda_launch_count", "kda_chunk_fwd_noalloc",
+           "kda_launch_count", "kda_chunk_fwd_noalloc", "kda_inject_stall",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -62,6 +62,8 @@ def _load() -> ctypes.CDLL:
     L.kda_last_error.restype = ctypes.c_char_p
     L.kda_launch_count.argtypes = []
     L.kda_launch_count.restype = ctypes.c_uint64
+    L.kda_inject_stall.argtypes = [i32, ctypes.c_uint64]
+    L.kda_inject_stall.restype = ctypes.c_int
     return L
 
 
@@ -231,6 +233,12 @@ def kda_decode_step(q, k, v, a, beta, A_log, state, gate=None, scale: float = 1.
 def kda_launch_count() -> int:
     """Kernels launched through libkda by this process so far."""
     return int(lib.kda_launch_count())
+
+
+def kda_inject_stall(enable: bool, wait_limit_ns: int = 0) -> None:
+    """Failure injection for tests: while enabled, prefill launches withhold chunk 0 and every
+    device-side wait gives up after wait_limit_ns (the next kda_sync_check raises a timeout)."""
+    _check(lib.kda_inject_stall(1 if enable else 0, int(wait_limit_ns)), "kda_inject_stall")
 
 
 def kda_sync_check(stream=None, device=None) -> None:

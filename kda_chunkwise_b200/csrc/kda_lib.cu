@@ -32,9 +32,7 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool supported_dim(int d) { return d == 64 || d == 128; }
 
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-// Workspace of the chunkwise path: [per-unit ring flags | per-unit rings of chunk records].
+// Workspace of the chunkwise path: per-unit rings of chunk records.
 size_t ring_slot_bytes(int d_k, int d_v) {
     if (d_k == 128 && d_v == 128) return kda::RingLayout<128, 128>::kBytes;
     if (d_k == 128 && d_v == 64) return kda::RingLayout<128, 64>::kBytes;
@@ -43,8 +41,6 @@ size_t ring_slot_bytes(int d_k, int d_v) {
 }
 
 int ring_slots(int d_v) { return 2 * (d_v / kda::kSlab); }
-
-size_t flag_bytes(int64_t units, int d_v) { return round_up((size_t)units * ring_slots(d_v) * 2 * 4, 256); }
 
 size_t ring_bytes(int64_t units, int d_k, int d_v) {
     return (size_t)units * ring_slots(d_v) * ring_slot_bytes(d_k, d_v);
@@ -56,6 +52,10 @@ bool sizes_ok(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen, int32_
 
 constexpr unsigned long long kWaitNs = 4000000000ull;   // bound of every device-side wait (4 s)
 
+// failure injection (kda_inject_stall): withhold chunk 0, shorten the wait bound
+std::atomic<int> g_inject_stall{0};
+std::atomic<unsigned long long> g_inject_wait_ns{kWaitNs};
+
 template <int DK, int DV>
 kda_status launch_prefill(const kda::FusedParams &p, int64_t units, cudaStream_t stream) {
     constexpr int G = DV / kda::kSlab;
@@ -63,8 +63,6 @@ kda_status launch_prefill(const kda::FusedParams &p, int64_t units, cudaStream_t
     cudaError_t e = cudaFuncSetAttribute(kda::kda_prefill_fused_kernel<DK, DV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
-    e = cudaMemsetAsync(p.flags, 0, flag_bytes(units, DV), stream);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(ring flags)");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(units * G));
     cfg.blockDim = dim3(kda::kFusedThreads);
@@ -146,7 +144,7 @@ size_t kda_chunk_fwd_workspace_min(int64_t total_tokens, int32_t num_seqs, int32
     if (!sizes_ok(total_tokens, num_seqs, max_seqlen, H) || !supported_dim(d_k) || !supported_dim(d_v))
         return 0;
     const int64_t units = (int64_t)num_seqs * H;
-    return flag_bytes(units, d_v) + ring_bytes(units, d_k, d_v);
+    return ring_bytes(units, d_k, d_v);
 }
 
 size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
@@ -204,15 +202,15 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     p.S_in = initial_state;
     p.S_out = final_state;
     p.out = out;
-    p.flags = reinterpret_cast<int *>(ws);
-    p.ring = ws + flag_bytes(units, d_v);
+    p.ring = ws;
     p.total_tokens = total_tokens;
     p.num_seqs = num_seqs;
     p.H = H;
     p.max_seqlen = max_seqlen;
     p.scale = scale;
     p.out_f32 = out_dtype == KDA_DTYPE_F32;
-    p.wait_ns = kWaitNs;
+    p.stall_first_chunk = g_inject_stall.load(std::memory_order_relaxed);
+    p.wait_ns = p.stall_first_chunk ? g_inject_wait_ns.load(std::memory_order_relaxed) : kWaitNs;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d_k == 128 && d_v == 128) return launch_prefill<128, 128>(p, units, st);
     if (d_k == 128 && d_v == 64) return launch_prefill<128, 64>(p, units, st);
@@ -278,6 +276,18 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     if (d_k == 128 && d_v == 64) return launch_decode<128, 64>(p, units, st);
     if (d_k == 64 && d_v == 128) return launch_decode<64, 128>(p, units, st);
     return launch_decode<64, 64>(p, units, st);
+}
+
+kda_status kda_inject_stall(int32_t enable, uint64_t wait_limit_ns) {
+    if (!enable) {
+        g_inject_stall.store(0);
+        return KDA_OK;
+    }
+    if (wait_limit_ns < 1000000ull || wait_limit_ns > kWaitNs)
+        return fail(KDA_ERR_INVALID_ARG, "kda_inject_stall: wait_limit_ns must be in [1e6, 4e9]");
+    g_inject_wait_ns.store(wait_limit_ns);
+    g_inject_stall.store(1);
+    return KDA_OK;
 }
 
 kda_status kda_sync_check(void *stream) {

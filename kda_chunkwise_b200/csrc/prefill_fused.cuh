@@ -32,8 +32,13 @@
 //   producer warps 8-15: the chunk-parallel work for chunks rank, rank + G, rank + 2G, ...,
 //                        written as ready-to-use mma fragments into the unit's ring.
 // The ring (2G slots per unit, in the workspace, small enough to stay in L2) carries chunk c in
-// slot c % 2G; `full` and `empty` counters per slot order the hand-off (release/acquire at gpu
-// scope).  Every wait is bounded: on timeout the waiting role records kErrTimeout and returns.
+// slot c % 2G.  Shared-memory mbarriers order the hand-off at cluster scope: every CTA has a
+// `full` barrier per slot, on which the producing CTA arrives (remotely) once the chunk is in the
+// ring; the producing CTA's `empty` barrier of the slot collects one arrival from each of the G
+// consumers once they have read it.  Slot s is always produced by CTA s % G, so phase u of a
+// slot's barriers belongs to chunk s + u 2G.  Every wait is bounded: on timeout the waiting role
+// records kErrTimeout and returns; all threads then meet at a cluster barrier before exit, so no
+// CTA leaves while another may still arrive on its barriers.
 #pragma once
 
 #include "common.cuh"
@@ -74,7 +79,10 @@ struct FusedSmem {
     static constexpr int kPK = kPW + 4 * RL::KT * 512;   // prefetched K-^T tiles
     static constexpr int kPU = kPK + 4 * RL::KT * 512;   // prefetched U~ of this slab [4][32][32 B]
     static constexpr int kPG = kPU + 4 * 32 * 32;     // prefetched Gamma_C fp32 [DK]
-    static constexpr int kCFlag = kPG + DK * 4;       // int abort flag
+    static constexpr int kFull = kPG + DK * 4;        // u64 mbarrier [R]: chunk published
+    static constexpr int kEmpty = kFull + 8 * RL::R;  // u64 mbarrier [R]: chunk consumed (the
+                                                      //   producing CTA's copy is the one used)
+    static constexpr int kCFlag = kEmpty + 8 * RL::R; // int abort flag
     static constexpr int kProd = (kCFlag + 16 + 1023) / 1024 * 1024;
     // producer (all [64][*] operand tiles are swizzled row-major)
     static constexpr int kQhi = kProd;                // bf16 [64][DK] q, then hi of q e^{b - r}
@@ -102,6 +110,7 @@ struct FusedSmem {
     static constexpr int kD = kAbc + 4 * DK * 4;      // fp32 [6][DK] e^{r_p - r_q}, q < p
     static constexpr int kPFlag = kD + 6 * DK * 4;    // int abort flag
     static constexpr int kBytes = kPFlag + 16;
+    static_assert(kFull % 8 == 0, "mbarriers need 8-byte alignment");
 };
 
 // index of the pair (p, q < p) in the 6-entry decay table
@@ -114,13 +123,13 @@ struct FusedParams {
     const float *S_in;
     float *S_out;
     void *out;
-    int *flags;         // [units][R][2]: full, empty
     char *ring;         // [units][R][slot bytes]
     int64_t total_tokens;
     int num_seqs, H;
     int max_seqlen;              // 0: no bound to check
     float scale;
     bool out_f32;
+    int stall_first_chunk;       // failure injection: never publish chunk 0
     unsigned long long wait_ns;  // bound of every wait
 };
 
@@ -130,14 +139,16 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
     return t;
 }
 
-// Spin (one thread) until *flag >= target, at most wait_ns.  Returns false on timeout.
-__device__ __forceinline__ bool wait_at_least(const int *flag, int target, unsigned long long wait_ns) {
-    if (ld_acquire_gpu(flag) >= target) return true;
+// Spin (one thread) until the phase with parity `parity` of a local mbarrier completes, at most
+// wait_ns.  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity,
+                                                  unsigned long long wait_ns) {
+    if (mbar_test(addr, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     unsigned ns = 32;
     while (true) {
         __nanosleep(ns);
-        if (ld_acquire_gpu(flag) >= target) return true;
+        if (mbar_test(addr, parity)) return true;
         if (ns < 256) ns <<= 1;
         if (globaltimer_ns() - t0 > wait_ns) return false;
     }
@@ -184,8 +195,8 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
 
     const int64_t H = p.H;
     const float expA = expf(p.A_log[h]);
-    int *const flags = p.flags + (size_t)unit * R * 2;
     char *const ring = p.ring + (size_t)unit * R * RL::kBytes;
+    const uint32_t aFull = smem_u32(sm + SM::kFull), aEmpty = smem_u32(sm + SM::kEmpty);
     const uint32_t aQhi = smem_u32(sQhi), aQlo = smem_u32(sQlo), aK = smem_u32(sK);
     const uint32_t aV = smem_u32(sV), aKr = smem_u32(sKr), aKh = smem_u32(sKh);
     const uint32_t aKb = smem_u32(sKb), aTp = smem_u32(sTp), aLD = smem_u32(sLD);
@@ -236,11 +247,6 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         const int slot = c % R;
         const int64_t t0 = s0 + (int64_t)c * kChunk;
         const int L = static_cast<int>(min64(kChunk, s1 - t0));
-        // the slot's release counter, read early so its latency overlaps the loads
-        const int empty_target = G * (c / R);
-        int empty_seen = 0;
-        if (tid == 0 && c >= R) empty_seen = ld_relaxed_gpu(flags + slot * 2 + 1);
-
         // 1. this chunk's q, k, a rows were requested at the end of the previous chunk's Gram
         //    phase and its v rows at the end of the previous chunk (the very first chunk
         //    requests them here); rows >= L are zero-filled.  Then an L2 prefetch of the rows of
@@ -314,13 +320,9 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         // the slot must be free (chunk c - R consumed by all G consumers) before any ring write
         if (tid == 0) {
             bool ok = true;
-            if (c >= R) {
-                if (empty_seen >= empty_target) {
-                    fence_acquire_gpu();   // the early relaxed read already showed the release
-                } else {
-                    ok = wait_at_least(flags + slot * 2 + 1, empty_target, p.wait_ns);
-                    if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
-                }
+            if (c >= R) {   // phase c / R - 1 of the slot's empty barrier: chunk c - R consumed
+                ok = mbar_wait_bounded(aEmpty + 8 * slot, ((c / R) - 1) & 1, p.wait_ns);
+                if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
             }
             *abort_flag = ok ? 0 : 1;
         }
@@ -566,10 +568,8 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             }
         }
         named_bar(kBarProducer, kRoleThreads);
-        if (tid == 0) {
-            __threadfence();
-            st_release_gpu(flags + slot * 2, c + 1);
-        }
+        if (tid < G && !(c == 0 && p.stall_first_chunk))
+            mbar_arrive_cluster(mapa_shared(aFull + 8 * slot, tid));   // publish to CTA tid
         if (c + G < nchunks) load_v(c + G);   // the v buffer is free now
     }
 }
@@ -603,8 +603,8 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(sm + SM::kCFlag);
     const int64_t H = p.H;
     const int col0 = rank * kSlab;
-    int *const flags = p.flags + (size_t)unit * R * 2;
     const char *const ring = p.ring + (size_t)unit * R * RL::kBytes;
+    const uint32_t aFull = smem_u32(sm + SM::kFull), aEmpty = smem_u32(sm + SM::kEmpty);
     auto slot_of = [&](int c) { return ring + (size_t)(c % R) * RL::kBytes; };
 
     // ring -> shared memory copies of the chain operands (16-byte cp.async, L2 only)
@@ -632,15 +632,10 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         cp_async_commit();
     };
     // thread 0 waits for chunk c to be published; the role's barrier publishes the outcome
-    auto wait_full = [&](int c, int seen) {
+    auto wait_full = [&](int c) {
         if (tid == 0) {
-            bool ok = true;
-            if (seen >= c + 1) {
-                fence_acquire_gpu();   // the early relaxed read already showed the publication
-            } else {
-                ok = wait_at_least(flags + (c % R) * 2, c + 1, p.wait_ns);
-                if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
-            }
+            const bool ok = mbar_wait_bounded(aFull + 8 * (c % R), (c / R) & 1, p.wait_ns);
+            if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
             *abort_flag = ok ? 0 : 1;
         }
     };
@@ -682,7 +677,7 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     load_gate(0, gt);
 
     if (nchunks > 0) {
-        wait_full(0, 0);
+        wait_full(0);
         named_bar(kBarConsumer, kRoleThreads);
         if (*abort_flag) return;
         prefetch_wu(0);
@@ -694,16 +689,14 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         const int64_t t0 = s0 + (int64_t)c * kChunk;
         const int L = static_cast<int>(min64(kChunk, s1 - t0));
         const bool has_next = c + 1 < nchunks;
-        // 1. fp16 copy of S_c (B operand of W S and Q^ S); early read of chunk c+1's counter;
-        //    Q^ and A of chunk c and the next chunk's gate into registers
+        // 1. fp16 copy of S_c (B operand of W S and Q^ S); Q^ and A of chunk c and the next
+        //    chunk's gate into registers
 #pragma unroll
         for (int j = 0; j < SNT; ++j) {
             const int cc = 8 * (sn0 + j) + 2 * t4;
             *reinterpret_cast<uint32_t *>(sS + swz_elem<64>(r0, cc)) = pack_f16(S[j][0], S[j][1]);
             *reinterpret_cast<uint32_t *>(sS + swz_elem<64>(r1, cc)) = pack_f16(S[j][2], S[j][3]);
         }
-        int full_seen = 0;
-        if (tid == 0 && has_next) full_seen = ld_relaxed_gpu(flags + ((c + 1) % R) * 2);
         uint4 Qf[KT], Af[4];
 #pragma unroll
         for (int kd = 0; kd < KT; ++kd) Qf[kd] = ldg_cg_v4(slotp + RL::kQ + (m * KT + kd) * 512 + lane * 16);
@@ -750,7 +743,7 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             }
         }
         // 3. chunk c+1 must be published before its W and U~ are copied
-        if (has_next) wait_full(c + 1, full_seen);
+        if (has_next) wait_full(c + 1);
         cp_async_wait_group<0>();                  // this thread's K-^T, Gamma_C copies of chunk c
         named_bar(kBarConsumer, kRoleThreads);     // U complete; W, U~ buffers free; K-^T visible
         if (has_next && *abort_flag) return;
@@ -827,10 +820,10 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             }
         }
         gt[0][0] = gtn[0][0]; gt[0][1] = gtn[0][1]; gt[1][0] = gtn[1][0]; gt[1][1] = gtn[1][1];
-        // 7. every warp is done with this slot, sS, sU and the K-^T buffer.  Every value read from
-        //    the slot has already been consumed, so returning it needs no release ordering.
+        // 7. every warp is done with this slot, sS, sU and the K-^T buffer: return the slot to the
+        //    CTA that produces it
         named_bar(kBarConsumer, kRoleThreads);
-        if (tid == 0) red_relaxed_add_gpu(flags + (c % R) * 2 + 1, 1);
+        if (tid == 0) mbar_arrive_cluster(mapa_shared(aEmpty + 8 * (c % R), (c % R) % G));
         if (has_next) prefetch_kg(c + 1);
     }
     if (p.S_out) {
@@ -856,10 +849,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1) kda_prefill_fused_kernel(con
         if (p.max_seqlen > 0 && s1 - s0 > p.max_seqlen) atomicOr(&g_kda_error_word, kErrSeqTooLong);
     }
     const int nchunks = static_cast<int>((s1 - s0 + kChunk - 1) / kChunk);
+    // The cluster is G CTAs along x, so `rank` is this CTA's rank in it.
+    if (threadIdx.x < RingLayout<DK, DV>::R) {
+        using SM = FusedSmem<DK, DV>;
+        mbar_init(smem_u32(fsmem + SM::kFull) + 8 * threadIdx.x, 1);
+        mbar_init(smem_u32(fsmem + SM::kEmpty) + 8 * threadIdx.x, G);
+    }
+    cluster_sync_after_init();
     if (threadIdx.x < kRoleThreads)
         fused_consumer<DK, DV>(p, fsmem, unit, n, h, rank, s0, s1, nchunks);
     else
         fused_producer<DK, DV>(p, fsmem, unit, h, rank, s0, s1, nchunks);
+    cp_async_wait_all();
+    cluster_sync();   // no CTA exits while a peer may still arrive on its barriers
 }
 
 }  // namespace kda

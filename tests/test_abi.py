@@ -99,3 +99,11 @@ def test_decode_rejects_bad_arguments():
     assert f(16, 16, 16, 16, 16, 8, 16, 16, 16, 0, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
     assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 5, 4, 2, 128, 128, 1.0, None) == kda.KDA_ERR_INVALID_ARG
     assert f(16, 16, 16, 16, 16, None, 16, 16, 16, 0, 0, 2, 128, 128, 1.0, None) == kda.KDA_OK
+
+
+def test_inject_stall_validates_its_limit_on_the_host():
+    assert lib.kda_inject_stall(1, 10) == kda.KDA_ERR_INVALID_ARG          # below 1 ms
+    assert lib.kda_inject_stall(1, 5_000_000_000) == kda.KDA_ERR_INVALID_ARG   # above 4 s
+    assert lib.kda_inject_stall(0, 0) == kda.KDA_OK
+    with pytest.raises(kda.KDAError):
+        kda.kda_inject_stall(True, 0)

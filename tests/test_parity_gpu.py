@@ -171,6 +171,27 @@ def test_device_reports_bad_seqlens(kda):
     kda.kda_sync_check()
 
 
+def test_bounded_wait_gives_up_and_context_survives(kda):
+    """Failure injection on the host side of the boundary: chunk 0 of every unit is never
+    published, so the consumers' waits (and, past the ring's 2G slots, the producers' waits) can
+    only end by their bound, here 20 ms.  The launch must end, kda_sync_check must report
+    KDA_ERR_TIMEOUT, and the next call on the same context must be correct."""
+    w = KI.Workload("stall", (1100, 130), 2, 64, 128, seed=11)
+    inp = KI.make_inputs(w, "cuda")
+    kda.kda_inject_stall(True, 20_000_000)
+    try:
+        run(kda, inp, max_seqlen=1100)
+        with pytest.raises(kda.KDAError) as err:
+            kda.kda_sync_check()
+        assert err.value.status == 4   # KDA_ERR_TIMEOUT
+    finally:
+        kda.kda_inject_stall(False)
+    kda.kda_sync_check()
+    out, S = run(kda, inp, max_seqlen=1100)
+    kda.kda_sync_check()
+    check_units(inp, out, S, all_units(w))
+
+
 # ---- decode ------------------------------------------------------------------------------------
 
 def decode_run(kda, inp, steps, scale=1.0, out_dtype=BF16):
