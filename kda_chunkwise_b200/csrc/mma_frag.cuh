@@ -208,11 +208,6 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, int s
                  : "memory");
 }
 
-// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *p, int bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // ---- mbarriers and the cluster ------------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
@@ -240,6 +235,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 // Arrive (release, cluster scope) on an mbarrier that may live in another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+}
+
+// Arrive (relaxed, cluster scope): for a hand-back after which nothing written needs ordering.
+__device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
 }
 
 // One non-blocking test (acquire, cluster scope) of whether the phase with parity `parity` of a

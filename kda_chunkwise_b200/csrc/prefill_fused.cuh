@@ -93,21 +93,19 @@ struct FusedSmem {
     static constexpr int kKh = kKr + 64 * DK * 2;     // fp16 [64][DK] K^
     static constexpr int kKt = kKh + 64 * DK * 2;     // fp32 [64][DK] K~; later fp16 T' [64][64]
     static constexpr int kKtBytes = (64 * DK * 4 > 64 * 64 * 2) ? 64 * DK * 4 : 64 * 64 * 2;
-    static constexpr int kB = kKt + kKtBytes;         // fp32 [64][DK] b; later:
+    static constexpr int kB = kKt + kKtBytes;         // scratch of the later phases:
     static constexpr int kLd = kB;                    //   fp32 [4][16][17] diagonal blocks of L
     static constexpr int kLD = kLd + 4 * 16 * 17 * 4;   //   fp16 [64][64]: -L below the diagonal
                                                       //   blocks, (I + L_pp)^-1 on them
     static constexpr int kT = kLD + 64 * 64 * 2;      //   fp16 [64][64] T = (I + L)^-1
     static constexpr int kM = kT + 64 * 64 * 2;       //   fp16 [3][16][32] block-product scratch
-    static constexpr int kBNeed = kM + 3 * 16 * 64 - kB;
-    static constexpr int kBBytes = (64 * DK * 4 > kBNeed) ? 64 * DK * 4 : kBNeed;
+    static constexpr int kQh = kT;                    //   fp16 [64][DK] Q^, copied to the ring
+                                                      //   before T and M are written
+    static constexpr int kBNeed = (kM + 3 * 16 * 64 > kQh + 64 * DK * 2 ? kM + 3 * 16 * 64 : kQh + 64 * DK * 2) - kB;
+    static constexpr int kBBytes = (kBNeed + 15) / 16 * 16;
     static constexpr int kBeta = kB + kBBytes;        // fp32 [64]
-    static constexpr int kTot = kBeta + 64 * 4;       // fp32 [4][DK] cumsum part totals
-    static constexpr int kRef = kTot + 4 * DK * 4;    // fp32 [4][DK] r_p
-    static constexpr int kEP = kRef + 4 * DK * 4;     // fp32 [4][DK] e^{r_p}
-    static constexpr int kTT = kEP + 4 * DK * 4;      // fp32 [4][DK] e^{r_{p+1} - r_p}
-    static constexpr int kAbc = kTT + 4 * DK * 4;     // fp32 [4][DK] e^{b_C - r_{p+1}}
-    static constexpr int kD = kAbc + 4 * DK * 4;      // fp32 [6][DK] e^{r_p - r_q}, q < p
+    static constexpr int kTot = kBeta + 64 * 4;       // fp32 [2 * threads]: run totals of the decay sums
+    static constexpr int kD = kTot + 2 * kRoleThreads * 4;   // fp32 [6][DK] e^{r_p - r_q}, q < p
     static constexpr int kPFlag = kD + 6 * DK * 4;    // int abort flag
     static constexpr int kBytes = kPFlag + 16;
     static_assert(kFull % 8 == 0, "mbarriers need 8-byte alignment");
@@ -178,20 +176,13 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
     unsigned char *const sQhi = sm + SM::kQhi, *const sQlo = sm + SM::kQlo, *const sK = sm + SM::kK;
     unsigned char *const sKr = sm + SM::kKr, *const sKh = sm + SM::kKh, *const sKb = sm + SM::kK;
     unsigned char *const sKt = sm + SM::kKt, *const sTp = sm + SM::kKt, *const sV = sm + SM::kV;
-    unsigned char *const sBb = sm + SM::kB, *const sLD = sm + SM::kLD, *const sT = sm + SM::kT;
+    unsigned char *const sQh = sm + SM::kQh, *const sLD = sm + SM::kLD, *const sT = sm + SM::kT;
     unsigned char *const sM = sm + SM::kM;
     float *const sLd = reinterpret_cast<float *>(sm + SM::kLd);
     float *const sbeta = reinterpret_cast<float *>(sm + SM::kBeta);
     float *const stot = reinterpret_cast<float *>(sm + SM::kTot);
-    float *const sref = reinterpret_cast<float *>(sm + SM::kRef);
-    float *const sEP = reinterpret_cast<float *>(sm + SM::kEP);
-    float *const sTT = reinterpret_cast<float *>(sm + SM::kTT);
-    float *const sAbc = reinterpret_cast<float *>(sm + SM::kAbc);
     float *const sD = reinterpret_cast<float *>(sm + SM::kD);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(sm + SM::kPFlag);
-    auto bval = [&](int t, int c) -> float & {   // b in the swizzled fp32 layout
-        return *reinterpret_cast<float *>(sBb + swz_f32<DK>(t, c & ~1) + ((c & 1) << 2));
-    };
 
     const int64_t H = p.H;
     const float expA = expf(p.A_log[h]);
@@ -200,7 +191,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
     const uint32_t aQhi = smem_u32(sQhi), aQlo = smem_u32(sQlo), aK = smem_u32(sK);
     const uint32_t aV = smem_u32(sV), aKr = smem_u32(sKr), aKh = smem_u32(sKh);
     const uint32_t aKb = smem_u32(sKb), aTp = smem_u32(sTp), aLD = smem_u32(sLD);
-    const uint32_t aT = smem_u32(sT), aM = smem_u32(sM);
+    const uint32_t aT = smem_u32(sT), aM = smem_u32(sM), aQh = smem_u32(sQh);
 
     // asynchronous input copies of one chunk: q, k, a as one commit group, v as another
     auto load_qka = [&](int cl) {
@@ -249,73 +240,39 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         const int L = static_cast<int>(min64(kChunk, s1 - t0));
         // 1. this chunk's q, k, a rows were requested at the end of the previous chunk's Gram
         //    phase and its v rows at the end of the previous chunk (the very first chunk
-        //    requests them here); rows >= L are zero-filled.  Then an L2 prefetch of the rows of
-        //    this producer's next chunk.
+        //    requests them here), several microseconds ahead of use; rows >= L are zero-filled.
         {
             if (c == rank) {
                 load_qka(c);
                 load_v(c);
             }
             if (tid < 64) sbeta[tid] = beta_next;   // loaded one chunk ahead
-            const int cn = c + G;
-            if (cn < nchunks) {
-                const int64_t tn = s0 + (int64_t)cn * kChunk;
-                const int Ln = static_cast<int>(min64(kChunk, s1 - tn));
-                const int row = tid & 63, which = tid >> 6;   // 4 tensors x 64 rows
-                if (row < Ln) {
-                    const uint16_t *base = which == 0 ? p.q : which == 1 ? p.k : which == 2 ? p.a : p.v;
-                    const int d = which == 3 ? DV : DK;
-                    prefetch_l2_bulk(base + ((tn + row) * H + h) * d, d * 2);
-                }
-            }
             cp_async_wait_group<1>();   // q, k, a of this chunk (v may still be in flight)
             named_bar(kBarProducer, kRoleThreads);
         }
         beta_next = load_beta(c + G);
 
-        // 2. log-decay g and its chunk-local inclusive cumsum b (rows >= L carry g = 0).  Each
-        //    thread takes one channel and a contiguous run of tokens: the loads and the
-        //    exponentials are independent, only the running sum is sequential.
+        // 2. log-decay g (in log2 units) and its running sum over each thread's run of tokens.
+        //    Thread (part, channel pair cp) takes TPP consecutive tokens of channels 2cp, 2cp + 1:
+        //    a whole 16-token tile (d_k = 128) or half of one (d_k = 64).  Rows >= L carry g = 0.
+        constexpr int CP = DK / 2;                   // channel pairs
+        constexpr int PARTS = kRoleThreads / CP;     // 4 (d_k = 128) or 8 (d_k = 64)
+        constexpr int TPP = 64 / PARTS;              // tokens per run: 16 or 8
+        constexpr int PPT = 16 / TPP;                // runs per 16-token tile: 1 or 2
+        const int cp = tid % CP, part = tid / CP, ch = 2 * cp;
+        const int pt = part / PPT;                   // tile of this run
+        float2 l[TPP];
         {
-            constexpr int PARTS = kRoleThreads / DK;   // 2 for d_k = 128, 4 for 64
-            constexpr int TPP = 64 / PARTS;
-            const int ch = tid % DK, part = tid / DK;
-            float gv[TPP];
+            constexpr float kG2 = kGMin * kLog2e;
 #pragma unroll
-            for (int i = 0; i < TPP; ++i)
-                gv[i] = bf16_to_f32(*reinterpret_cast<const uint16_t *>(sKr + swz_elem<RB>(part * TPP + i, ch)));
-#pragma unroll
-            for (int i = 0; i < TPP; ++i) gv[i] = part * TPP + i < L ? log_decay(gv[i], expA) : 0.f;
-#pragma unroll
-            for (int i = 1; i < TPP; ++i) gv[i] += gv[i - 1];
-            stot[part * DK + ch] = gv[TPP - 1];
-            named_bar(kBarProducer, kRoleThreads);
-            float off = 0.f;
-            for (int pp = 0; pp < part; ++pp) off += stot[pp * DK + ch];
-#pragma unroll
-            for (int i = 0; i < TPP; ++i) bval(part * TPP + i, ch) = gv[i] + off;
-            named_bar(kBarProducer, kRoleThreads);
-        }
-
-        // 2b. per-channel tile constants
-        if (tid < DK) {
-            const int ch = tid;
-            float r[5];
-            r[0] = 0.f;
-            r[1] = bval(15, ch);
-            r[2] = bval(31, ch);
-            r[3] = bval(47, ch);
-            r[4] = bval(63, ch);   // b_C
-#pragma unroll
-            for (int pp = 0; pp < 4; ++pp) {
-                sref[pp * DK + ch] = r[pp];
-                sEP[pp * DK + ch] = ex2(r[pp] * kLog2e);
-                sTT[pp * DK + ch] = ex2((r[pp + 1] - r[pp]) * kLog2e);
-                sAbc[pp * DK + ch] = ex2((r[4] - r[pp + 1]) * kLog2e);
-#pragma unroll
-                for (int qq = 0; qq < pp; ++qq)
-                    sD[pair_index(pp, qq) * DK + ch] = ex2((r[pp] - r[qq]) * kLog2e);
+            for (int i = 0; i < TPP; ++i) {
+                const int t = part * TPP + i;
+                const float2 av = unpack_bf16(*reinterpret_cast<const uint32_t *>(sKr + swz_elem<RB>(t, ch)));
+                float2 gg = make_float2(kG2 * sigmoid_fast(expA * av.x), kG2 * sigmoid_fast(expA * av.y));
+                if (t >= L) gg = make_float2(0.f, 0.f);
+                l[i] = i == 0 ? gg : make_float2(l[i - 1].x + gg.x, l[i - 1].y + gg.y);
             }
+            *reinterpret_cast<float2 *>(stot + part * DK + ch) = l[TPP - 1];
         }
         // the slot must be free (chunk c - R consumed by all G consumers) before any ring write
         if (tid == 0) {
@@ -326,49 +283,71 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             }
             *abort_flag = ok ? 0 : 1;
         }
-        named_bar(kBarProducer, kRoleThreads);
+        named_bar(kBarProducer, kRoleThreads);   // run totals visible
         if (*abort_flag) return;
         char *const slotp = ring + (size_t)slot * RL::kBytes;
 
-        // 3. operands.  Each thread owns the A-fragment positions of KT/2 tiles of [64][DK]
-        //    (rows 16m + g, +8; columns 16kd + 2t4, +1, +8, +9) and writes its Q^ fragments
-        //    straight to the ring.
+        // 3. operands of every token of the run.  In log2 units, r_p = b before tile p, lo = the
+        //    part of tile pt before this run; then per token
+        //      e^{b - r_p} = 2^(l + lo) <= 1,   e^{r_p - b} = 2^-(l + lo) in [1, e^80],
+        //    and Q r = scale q e^{b - r_p} (split bf16 hi + lo), K r = k e^{b - r_p} (bf16),
+        //    K~ = k e^{r_p - b} (fp32), K^ = k e^{r_p} e^{b - r_p}, Q^ = scale q e^{r_p} e^{b - r_p},
+        //    K- = k e^{b_C - r_{p+1}} (e^{r_{p+1} - r_p} e^{r_p - b}) (fp16; each factor <= 1).
+        {
+            float2 rp = make_float2(0.f, 0.f), lo = rp, tile = rp, bc = rp;
 #pragma unroll
-        for (int j = 0; j < KT / 2; ++j) {
-            const int idx = warp * (KT / 2) + j;
-            const int m = idx / KT, kd = idx % KT, pt = m;   // token tile = 16-token tile
-            uint32_t qfrag[4];
+            for (int pp = 0; pp < PARTS; ++pp) {
+                const float2 tv = *reinterpret_cast<const float2 *>(stot + pp * DK + ch);
+                bc.x += tv.x; bc.y += tv.y;
+                if (pp / PPT < pt) { rp.x += tv.x; rp.y += tv.y; }
+                if (pp / PPT == pt) {
+                    tile.x += tv.x; tile.y += tv.y;
+                    if (pp < part) { lo.x += tv.x; lo.y += tv.y; }
+                }
+            }
+            const float2 ep = make_float2(ex2(rp.x), ex2(rp.y));                    // e^{r_p}
+            const float2 tt = make_float2(ex2(tile.x), ex2(tile.y));                // e^{r_{p+1} - r_p}
+            const float2 ab = make_float2(ex2(bc.x - rp.x - tile.x), ex2(bc.y - rp.y - tile.y));   // e^{b_C - r_{p+1}}
+            const float2 eps = make_float2(ep.x * p.scale, ep.y * p.scale);
+            if (part == 0) {   // inter-tile decays e^{r_p - r_q} (q < p) and Gamma_C = e^{b_C}
+                float2 r[4];
+                r[0] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = 16 * m + g + 8 * (e & 1);
-                const int ch = 16 * kd + 2 * t4 + 8 * (e >> 1);
+                for (int pp = 1; pp < 4; ++pp) {
+                    r[pp] = r[pp - 1];
+#pragma unroll
+                    for (int q2 = 0; q2 < PPT; ++q2) {
+                        const float2 tv = *reinterpret_cast<const float2 *>(stot + ((pp - 1) * PPT + q2) * DK + ch);
+                        r[pp].x += tv.x; r[pp].y += tv.y;
+                    }
+                }
+#pragma unroll
+                for (int pp = 1; pp < 4; ++pp)
+#pragma unroll
+                    for (int qq = 0; qq < pp; ++qq)
+                        *reinterpret_cast<float2 *>(sD + pair_index(pp, qq) * DK + ch) =
+                            make_float2(ex2(r[pp].x - r[qq].x), ex2(r[pp].y - r[qq].y));
+                *reinterpret_cast<float2 *>(slotp + RL::kGam + ch * 4) = make_float2(ex2(bc.x), ex2(bc.y));
+            }
+#pragma unroll
+            for (int i = 0; i < TPP; ++i) {
+                const int t = part * TPP + i;
                 const uint32_t off = swz_elem<RB>(t, ch);
-                const float2 bb = *reinterpret_cast<const float2 *>(sBb + swz_f32<DK>(t, ch));
-                const float2 rr = *reinterpret_cast<const float2 *>(sref + pt * DK + ch);
-                const float x0 = (bb.x - rr.x) * kLog2e, x1 = (bb.y - rr.y) * kLog2e;
-                const float rf0 = ex2(x0), rf1 = ex2(x1);      // e^{b - r_p} in [e^-80, 1]
-                const float iv0 = ex2(-x0), iv1 = ex2(-x1);    // e^{r_p - b} in [1, e^80]
-                float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(sQhi + off));
+                const float x0 = l[i].x + lo.x, x1 = l[i].y + lo.y;
+                const float rf0 = ex2(x0), rf1 = ex2(x1);      // e^{b - r_p}
+                const float iv0 = ex2(-x0), iv1 = ex2(-x1);    // e^{r_p - b}
+                const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t *>(sQhi + off));
                 const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t *>(sK + off));
-                qv.x *= p.scale;
-                qv.y *= p.scale;
-                const float2 ep = *reinterpret_cast<const float2 *>(sEP + pt * DK + ch);
-                const float2 tt = *reinterpret_cast<const float2 *>(sTT + pt * DK + ch);
-                const float2 ab = *reinterpret_cast<const float2 *>(sAbc + pt * DK + ch);
-                uint32_t hi, lo;
-                split_bf16(qv.x * rf0, qv.y * rf1, hi, lo);
+                uint32_t hi, lo2;
+                split_bf16(qv.x * p.scale * rf0, qv.y * p.scale * rf1, hi, lo2);
                 *reinterpret_cast<uint32_t *>(sQhi + off) = hi;
-                *reinterpret_cast<uint32_t *>(sQlo + off) = lo;
+                *reinterpret_cast<uint32_t *>(sQlo + off) = lo2;
                 *reinterpret_cast<uint32_t *>(sKr + off) = pack_bf16(kv.x * rf0, kv.y * rf1);
                 *reinterpret_cast<float2 *>(sKt + swz_f32<DK>(t, ch)) = make_float2(kv.x * iv0, kv.y * iv1);
                 *reinterpret_cast<uint32_t *>(sKh + off) = pack_f16(kv.x * ep.x * rf0, kv.y * ep.y * rf1);
-                // K- = k e^{b_C - b} = k (e^{b_C - r_{p+1}}) (e^{r_{p+1} - r_p} e^{r_p - b}), each
-                // <= 1; it overwrites k at the same element, which this thread has already read
-                *reinterpret_cast<uint32_t *>(sKb + off) =
-                    pack_f16(kv.x * ab.x * (tt.x * iv0), kv.y * ab.y * (tt.y * iv1));
-                qfrag[e] = pack_f16(qv.x * ep.x * rf0, qv.y * ep.y * rf1);   // Q^ = q e^{b}
+                *reinterpret_cast<uint32_t *>(sKb + off) = pack_f16(kv.x * ab.x * (tt.x * iv0), kv.y * ab.y * (tt.y * iv1));
+                *reinterpret_cast<uint32_t *>(sQh + off) = pack_f16(qv.x * eps.x * rf0, qv.y * eps.y * rf1);
             }
-            stg_v4(slotp + RL::kQ + idx * 512 + lane * 16, make_uint4(qfrag[0], qfrag[1], qfrag[2], qfrag[3]));
         }
         named_bar(kBarProducer, kRoleThreads);
 
@@ -438,15 +417,16 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             }
             stg_v4(slotp + RL::kA + blk * 512 + lane * 16, make_uint4(afr[0], afr[1], afr[2], afr[3]));
         }
-        // 4b. K-^T fragments and Gamma_C
+        // 4b. K-^T and Q^ fragments to the ring
         for (int idx = warp; idx < 4 * KT; idx += 8) {
             uint32_t fr[4];
             const int md = idx / 4, kt = idx % 4;   // K-^T tile (d_k tile md, token tile kt)
             ldsm_x4_t(fr, ldsm_addr_bn<RB>(aKb, 16 * kt, 16 * md, lane));
             stg_v4(slotp + RL::kKbT + idx * 512 + lane * 16, make_uint4(fr[0], fr[1], fr[2], fr[3]));
+            const int m = idx / KT, kd = idx % KT;  // Q^ tile (token tile m, d_k tile kd)
+            ldsm_x4(fr, ldsm_addr_a<RB>(aQh, 16 * m, 16 * kd, lane));
+            stg_v4(slotp + RL::kQ + idx * 512 + lane * 16, make_uint4(fr[0], fr[1], fr[2], fr[3]));
         }
-        if (tid < DK)   // e^{b_C} = e^{r_3} e^{b_C - r_3}
-            reinterpret_cast<float *>(slotp + RL::kGam)[tid] = sEP[3 * DK + tid] * sTT[3 * DK + tid];
         named_bar(kBarProducer, kRoleThreads);
         // the q, k (now K-) and a (now K r) buffers are no longer read: request the next chunk's
         if (c + G < nchunks) load_qka(c + G);
@@ -821,9 +801,11 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         }
         gt[0][0] = gtn[0][0]; gt[0][1] = gtn[0][1]; gt[1][0] = gtn[1][0]; gt[1][1] = gtn[1][1];
         // 7. every warp is done with this slot, sS, sU and the K-^T buffer: return the slot to the
-        //    CTA that produces it
+        //    CTA that produces it.  Every value read from the slot has already arrived in registers
+        //    or shared memory, so the hand-back needs no release ordering (a release would wait for
+        //    this chunk's output stores).
         named_bar(kBarConsumer, kRoleThreads);
-        if (tid == 0) mbar_arrive_cluster(mapa_shared(aEmpty + 8 * (c % R), (c % R) % G));
+        if (tid == 0) mbar_arrive_relaxed_cluster(mapa_shared(aEmpty + 8 * (c % R), (c % R) % G));
         if (has_next) prefetch_kg(c + 1);
     }
     if (p.S_out) {
