@@ -431,19 +431,19 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         // the q, k (now K-) and a (now K r) buffers are no longer read: request the next chunk's
         if (c + G < nchunks) load_qka(c + G);
 
-        // 5. diagonal blocks D_p = (I + L_pp)^-1 by forward substitution (fp32), one column per lane;
-        //    written as fp16 into the diagonal blocks of both LD and T
+        // 5. diagonal blocks D_p = (I + L_pp)^-1 by forward substitution (fp32), one column per lane,
+        //    column-oriented: once x_j is final it is eliminated from every later row, so the
+        //    dependent chain is 15 steps long; written as fp16 into the diagonal blocks of LD and T
         if (warp < 4 && lane < 16) {
             const int pb = warp, mcol = lane;
             const float *Ld = sLd + pb * 16 * 17;
             float x[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float v = i == mcol ? 1.f : 0.f;
+            for (int i = 0; i < 16; ++i) x[i] = i == mcol ? 1.f : 0.f;
 #pragma unroll
-                for (int j = 0; j < i; ++j) v = fmaf(-Ld[i * 17 + j], x[j], v);
-                x[i] = i >= mcol ? v : 0.f;
-            }
+            for (int j = 0; j < 15; ++j)
+#pragma unroll
+                for (int i = j + 1; i < 16; ++i) x[i] = fmaf(-Ld[i * 17 + j], x[j], x[i]);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const __half hv = __float2half_rn(x[i]);
@@ -548,9 +548,9 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             }
         }
         named_bar(kBarProducer, kRoleThreads);
+        if (c + G < nchunks) load_v(c + G);   // the v buffer is free now
         if (tid < G && !(c == 0 && p.stall_first_chunk))
             mbar_arrive_cluster(mapa_shared(aFull + 8 * slot, tid));   // publish to CTA tid
-        if (c + G < nchunks) load_v(c + G);   // the v buffer is free now
     }
 }
 
