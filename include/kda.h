@@ -80,7 +80,7 @@ typedef enum kda_dtype {
  *   non-zero bound is reported through the error word (the result is still computed in full).
  * scale multiplies q.  workspace: device scratch of at least kda_chunk_fwd_workspace_min(...)
  *   bytes (equal to kda_chunk_fwd_workspace_size(...)), 256-byte aligned; it holds per-unit rings
- *   of chunk records (about 0.55 MiB per (sequence, head) at d = 128); its contents need no
+ *   of chunk records (about 0.57 MiB per (sequence, head) at d = 128); its contents need no
  *   initialisation and it may be reused across calls on one stream.
  * A zero-length sequence copies its initial state (or zeros) to final_state.
  * total_tokens == 0 or num_seqs == 0 is valid and only writes final_state.
@@ -107,7 +107,7 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, co
  *     and caches it; make that first call before any stream capture.
  *   - Sizes whose scratch need (kda_chunk_fwd_workspace_min) exceeds 32 MiB are rejected with
  *     KDA_ERR_INVALID_ARG and a message in kda_last_error.  With d_k = d_v = 128 that allows
- *     58 (sequence, head) units per call, of any length.
+ *     56 (sequence, head) units per call, of any length.
  *   - Every call on a device shares the one array and nothing in it needs to start at zero, but
  *     calls that overlap on the GPU (different streams, or other threads) race on it: serialise
  *     them, for example by issuing them all on one stream.

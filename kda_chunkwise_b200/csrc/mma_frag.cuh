@@ -163,6 +163,10 @@ __device__ __forceinline__ uint4 ldg_cg_v4(const void *p) {
     return __ldcg(reinterpret_cast<const uint4 *>(p));
 }
 
+__device__ __forceinline__ void st_u32(void *p, uint32_t x) {
+    asm volatile("st.global.u32 [%0], %1;\n" ::"l"(p), "r"(x) : "memory");
+}
+
 __device__ __forceinline__ void stg_v2(void *p, uint32_t x, uint32_t y) {
     asm volatile("st.global.v2.u32 [%0], {%1,%2};\n" ::"l"(p), "r"(x), "r"(y) : "memory");
 }

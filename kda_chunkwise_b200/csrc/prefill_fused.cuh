@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "mma_frag.cuh"
+#include "umma.cuh"
 
 namespace kda {
 
@@ -52,19 +53,21 @@ constexpr int kFusedThreads = 2 * kRoleThreads;
 constexpr int kBarConsumer = 1, kBarProducer = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Ring slot layout.  "Tile" = one 16x16 fp16 A-operand tile stored fragment-major: lane l's four
-// 32-bit registers at byte 16 l, so a warp loads or stores a tile with one 16-byte access per lane.
+// Ring slot layout.  The consumer moves the tensor-core A operands of a chunk into tensor memory
+// (TMEM), so the producer writes them as "TMEM images": [16-byte chunk j][TMEM lane][16 bytes],
+// where chunk j of a lane holds its 32-bit columns 4j .. 4j + 3 and column c holds the fp16 pair
+// (row, 2c), (row, 2c + 1).  A warp then reads 512 contiguous bytes per load, one 16-byte piece
+// per lane.
 template <int DK, int DV>
 struct RingLayout {
     static constexpr int G = DV / kSlab;          // slabs = consumers = producers per unit
     static constexpr int R = 2 * G;               // slots per unit
     static constexpr int KT = DK / 16;            // d_k tiles
-    static constexpr int kW = 0;                  // W tiles   (token tile m, d_k tile k): m*KT + k
-    static constexpr int kQ = kW + 4 * KT * 512;  // Q^ tiles  (m, k): m*KT + k
-    static constexpr int kKbT = kQ + 4 * KT * 512;  // K-^T tiles (d_k tile m, token tile k): m*4 + k
-    static constexpr int kA = kKbT + KT * 4 * 512;  // A tiles (m, k <= m): m(m+1)/2 + k
-    static constexpr int kU = kA + 10 * 512;      // U~: [token tile][slab][lane][16 fp16]
-    static constexpr int kGam = kU + 4 * G * 32 * 32;  // Gamma_C fp32 [DK]
+    static constexpr int kA1 = 0;                 // [W ; Q^]: lanes 0-63 W, 64-127 Q^ (K = d_k)
+    static constexpr int kA2 = kA1 + DK / 8 * 128 * 16;  // K-^T: lanes = d_k rows (K = tokens)
+    static constexpr int kA3 = kA2 + 8 * DK * 16;        // A: lanes 64-127 = token rows (K = tokens)
+    static constexpr int kU = kA3 + 8 * 64 * 16;  // U~: [slab][half][chunk 2][row 64][8 fp16]
+    static constexpr int kGam = kU + G * 2 * 2 * 64 * 16;  // Gamma_C fp32 [DK]
     static constexpr int kBytes = ((kGam + DK * 4) + 1023) / 1024 * 1024;
 };
 
@@ -72,17 +75,16 @@ struct RingLayout {
 template <int DK, int DV>
 struct FusedSmem {
     using RL = RingLayout<DK, DV>;
-    // consumer
-    static constexpr int kS = 0;                      // fp16 [DK][32] state operand
-    static constexpr int kU = kS + DK * kSlab * 2;    // fp16 [64][32] U operand
-    static constexpr int kPW = kU + 64 * kSlab * 2;   // prefetched W tiles of the next chunk
-    static constexpr int kPK = kPW + 4 * RL::KT * 512;   // prefetched K-^T tiles
-    static constexpr int kPU = kPK + 4 * RL::KT * 512;   // prefetched U~ of this slab [4][32][32 B]
-    static constexpr int kPG = kPU + 4 * 32 * 32;     // prefetched Gamma_C fp32 [DK]
-    static constexpr int kFull = kPG + DK * 4;        // u64 mbarrier [R]: chunk published
+    // consumer (B operands of the tensor-core products: 8 x 8 fp16 core matrices, MN-major)
+    static constexpr int kB1 = 0;                     // S_c: K = d_k rows, N = 32 columns
+    static constexpr int kB2 = kB1 + DK * kSlab * 2;  // U:   K = 64 tokens, N = 32 columns
+    static constexpr int kFull = kB2 + 64 * kSlab * 2;  // u64 mbarrier [R]: chunk published
     static constexpr int kEmpty = kFull + 8 * RL::R;  // u64 mbarrier [R]: chunk consumed (the
                                                       //   producing CTA's copy is the one used)
-    static constexpr int kCFlag = kEmpty + 8 * RL::R; // int abort flag
+    static constexpr int kM1 = kEmpty + 8 * RL::R;    // u64 mbarrier: [W; Q^] S complete
+    static constexpr int kM2 = kM1 + 8;               // u64 mbarrier: K-^T U and A U complete
+    static constexpr int kTmem = kM2 + 8;             // u32 TMEM base address
+    static constexpr int kCFlag = kTmem + 8;          // int abort flag
     static constexpr int kProd = (kCFlag + 16 + 1023) / 1024 * 1024;
     // producer (all [64][*] operand tiles are swizzled row-major)
     static constexpr int kQhi = kProd;                // bf16 [64][DK] q, then hi of q e^{b - r}
@@ -415,17 +417,34 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                     *reinterpret_cast<uint32_t *>(sLD + swz_elem<128>(i1, jc)) = pack_f16(-b1 * akk[nt][2], -b1 * akk[nt][3]);
                 }
             }
-            stg_v4(slotp + RL::kA + blk * 512 + lane * 16, make_uint4(afr[0], afr[1], afr[2], afr[3]));
+            // A rows i0, i1 = lanes of the A image; columns 8qb + 4nt + t4 = chunk 2qb + nt
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                char *const b = slotp + RL::kA3 + ((2 * qb + nt) * 64 + i0) * 16 + t4 * 4;
+                st_u32(b, afr[2 * nt]);
+                st_u32(b + 8 * 16, afr[2 * nt + 1]);
+            }
         }
-        // 4b. K-^T and Q^ fragments to the ring
+        if (warp >= 2) {   // zero blocks above the diagonal (the A image is read whole): one per warp
+            const int ub = warp - 2;   // (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+            const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
+            stg_v4(slotp + RL::kA3 + ((2 * qb + (lane >> 4)) * 64 + 16 * pb + (lane & 15)) * 16, make_uint4(0, 0, 0, 0));
+        }
+        // 4b. K-^T and Q^ to the ring.  K-^T tile (d_k tile md, token tile kt) as an A fragment:
+        //     register e of a lane is row 16md + g (+8 for e odd), columns 8kt + t4 (+4 for e >= 2).
         for (int idx = warp; idx < 4 * KT; idx += 8) {
             uint32_t fr[4];
-            const int md = idx / 4, kt = idx % 4;   // K-^T tile (d_k tile md, token tile kt)
+            const int md = idx / 4, kt = idx % 4;
             ldsm_x4_t(fr, ldsm_addr_bn<RB>(aKb, 16 * kt, 16 * md, lane));
-            stg_v4(slotp + RL::kKbT + idx * 512 + lane * 16, make_uint4(fr[0], fr[1], fr[2], fr[3]));
-            const int m = idx / KT, kd = idx % KT;  // Q^ tile (token tile m, d_k tile kd)
-            ldsm_x4(fr, ldsm_addr_a<RB>(aQh, 16 * m, 16 * kd, lane));
-            stg_v4(slotp + RL::kQ + idx * 512 + lane * 16, make_uint4(fr[0], fr[1], fr[2], fr[3]));
+            char *const b = slotp + RL::kA2 + ((2 * kt) * DK + 16 * md + g) * 16 + t4 * 4;
+            st_u32(b, fr[0]);
+            st_u32(b + 8 * 16, fr[1]);
+            st_u32(b + DK * 16, fr[2]);
+            st_u32(b + DK * 16 + 8 * 16, fr[3]);
+        }
+        for (int e = tid; e < 64 * (DK / 8); e += kRoleThreads) {   // Q^ row t -> lane 64 + t
+            const int t = e & 63, j = e >> 6;
+            stg_v4(slotp + RL::kA1 + (j * 128 + 64 + t) * 16, *reinterpret_cast<const uint4 *>(sQh + swz<RB>(t, j)));
         }
         named_bar(kBarProducer, kRoleThreads);
         // the q, k (now K-) and a (now K r) buffers are no longer read: request the next chunk's
@@ -537,13 +556,20 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                         mma_f16(acc[0], af, bfr[kt][0], bfr[kt][1]);
                         mma_f16(acc[1], af, bfr[kt][2], bfr[kt][3]);
                     }
-                    const uint4 fr = make_uint4(pack_f16(acc[0][0], acc[0][1]), pack_f16(acc[0][2], acc[0][3]),
-                                                pack_f16(acc[1][0], acc[1][1]), pack_f16(acc[1][2], acc[1][3]));
-                    if (isW) {   // W tile (token tile m, d_k tile u): an A fragment
-                        stg_v4(slotp + RL::kW + (m * KT + u) * 512 + lane * 16, fr);
-                    } else {     // U~: half (vc / 16) % 2 of slab vc / 32
-                        stg_v4(slotp + RL::kU + ((m * G + vc / kSlab) * 32 + lane) * 32 + ((vc >> 4) & 1) * 16, fr);
+                    // rows 16m + g (+8); columns vc + 2t4 (+1) and vc + 8 + 2t4 (+1)
+                    char *b;
+                    int chunk_step;
+                    if (isW) {   // [W; Q^] lanes 16m + g, columns 8u + t4 (chunk 2u) and + 4 (chunk 2u + 1)
+                        b = slotp + RL::kA1 + ((2 * u) * 128 + 16 * m + g) * 16 + t4 * 4;
+                        chunk_step = 128 * 16;
+                    } else {     // U~ of slab vc / 32, half (vc / 16) % 2, chunks 0 and 1
+                        b = slotp + RL::kU + ((((vc / kSlab) * 2 + ((vc >> 4) & 1)) * 2) * 64 + 16 * m + g) * 16 + t4 * 4;
+                        chunk_step = 64 * 16;
                     }
+                    st_u32(b, pack_f16(acc[0][0], acc[0][1]));
+                    st_u32(b + 8 * 16, pack_f16(acc[0][2], acc[0][3]));
+                    st_u32(b + chunk_step, pack_f16(acc[1][0], acc[1][1]));
+                    st_u32(b + chunk_step + 8 * 16, pack_f16(acc[1][2], acc[1][3]));
                 }
             }
         }
@@ -555,272 +581,276 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
 }
 
 // ---------------------------------------------------------------------------------------------
-// Consumer: the sequential state pass for slab `rank` (32 columns of d_v) of one unit.
+// Consumer: the sequential state pass for slab `rank` (32 columns of d_v) of one unit, on the
+// 5th-generation tensor cores.
 //
-// Per chunk c, with the state S_c (fp32 registers; fp16 copy in shared memory as the B operand):
-//   U = U~ - W S_c  ->  shared memory;   S_{c+1} = Diag(Gamma_C) S_c + K-^T U;
-//   O = Q^ S_c + A U, gated and stored.
-// The chain operands (W, U~ and K-^T, Gamma_C) of chunk c + 1 are copied from the ring into
-// shared memory while chunk c runs: W and U~ as soon as chunk c has read them, K-^T and Gamma_C
-// at the end of chunk c.  Q^ and A go to registers at the start of their chunk (off the chain).
+// Per chunk c, with S_c (fp32, in registers: thread (lane quadrant q, half) holds row 32q + lane,
+// columns 16 half .. + 15; an fp16 copy in shared memory is the B operand):
+//   D  = [W ; Q^] S_c            (M = 128: rows 0-63 W S_c, rows 64-127 Q^ S_c)     TMEM
+//   U  = U~ - D[0:64]  -> shared memory (fp16, B operand)
+//   D3 = K-^T U,   D[64:128] += A U                                                  TMEM
+//   S_{c+1} = Diag(Gamma_C) S_c + D3;   out = sigmoid(gate) D[64:128]
+// The A operands ([W; Q^], K-^T, A) of chunk c + 1 are copied from the ring into the other of two
+// TMEM buffers while chunk c's products run; the ring slot is handed back as soon as that copy
+// is done.  One thread issues the MMAs; every wait is bounded.
 // ---------------------------------------------------------------------------------------------
 template <int DK, int DV>
-__device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned char *sm, int unit,
-                                               int n, int h, int rank, int64_t s0, int64_t s1,
-                                               int nchunks) {
+__device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned char *sm, uint32_t tmem, int unit,
+                                               int n, int h, int rank, int64_t s0, int64_t s1, int nchunks) {
     using RL = RingLayout<DK, DV>;
     using SM = FusedSmem<DK, DV>;
-    constexpr int G = RL::G, R = RL::R, KT = RL::KT;
-    constexpr int SNT = DK / 32;   // n8 tiles of the state per warp
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t4 = lane & 3;
-    unsigned char *const sS = sm + SM::kS, *const sU = sm + SM::kU;
-    unsigned char *const sPW = sm + SM::kPW, *const sPK = sm + SM::kPK, *const sPU = sm + SM::kPU;
-    const float *const sPG = reinterpret_cast<const float *>(sm + SM::kPG);
-    const uint32_t aS = smem_u32(sS), aU = smem_u32(sU);
-    const uint32_t aPW = smem_u32(sPW), aPK = smem_u32(sPK), aPU = smem_u32(sPU), aPG = smem_u32(sm + SM::kPG);
+    constexpr int G = RL::G, R = RL::R;
+    constexpr int A1C = DK / 2;                        // TMEM columns of one [W; Q^] buffer
+    constexpr uint32_t cD = 0, cD3 = 32, cA1 = 64, cA2 = cA1 + 2 * A1C, cA3 = cA2 + 64;
+    constexpr uint32_t kIdesc = umma_idesc_f16(128, kSlab);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, half = warp >> 2;
+    const int row = 32 * q + lane;                     // this thread's TMEM lane
+    const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+    const bool has_s = row < DK, has_u = row < 64, has_o = row >= 64;
+    unsigned char *const sB1 = sm + SM::kB1, *const sB2 = sm + SM::kB2;
+    const uint32_t aB1 = smem_u32(sB1), aB2 = smem_u32(sB2);
+    const uint32_t aFull = smem_u32(sm + SM::kFull), aEmpty = smem_u32(sm + SM::kEmpty);
+    const uint32_t aM1 = smem_u32(sm + SM::kM1), aM2 = smem_u32(sm + SM::kM2);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(sm + SM::kCFlag);
     const int64_t H = p.H;
-    const int col0 = rank * kSlab;
+    const int col0 = rank * kSlab + 16 * half;         // this thread's first d_v column
     const char *const ring = p.ring + (size_t)unit * R * RL::kBytes;
-    const uint32_t aFull = smem_u32(sm + SM::kFull), aEmpty = smem_u32(sm + SM::kEmpty);
     auto slot_of = [&](int c) { return ring + (size_t)(c % R) * RL::kBytes; };
+    auto wait_bar = [&](uint32_t bar, uint32_t parity) {
+        if (!mbar_wait_bounded(bar, parity, p.wait_ns)) {
+            atomicOr(&g_kda_error_word, kErrTimeout);
+            *abort_flag = 1;
+        }
+        __syncwarp();   // the warp-wide tcgen05 loads and stores that follow need a converged warp
+    };
+    // fp16 copy of 16 values of row k (columns 16 half ..) into a B operand (MN-major core matrices)
+    auto store_b = [&](unsigned char *base, int k, const float (&x)[16]) {
+#pragma unroll
+        for (int g8 = 0; g8 < 2; ++g8) {
+            const uint4 v = make_uint4(pack_f16(x[8 * g8 + 0], x[8 * g8 + 1]), pack_f16(x[8 * g8 + 2], x[8 * g8 + 3]),
+                                       pack_f16(x[8 * g8 + 4], x[8 * g8 + 5]), pack_f16(x[8 * g8 + 6], x[8 * g8 + 7]));
+            *reinterpret_cast<uint4 *>(base + (((k >> 3) * 4 + 2 * half + g8) * 64 + (k & 7) * 8) * 2) = v;
+        }
+    };
+    // chunk cl's A operands into TMEM buffer b (each warp: its lane quadrant, its half of the columns)
+    auto load_a1 = [&](int cl, int b) {
+        const char *sp = slot_of(cl) + RL::kA1;
+        constexpr int NJ = A1C / 8;                    // 16-byte chunks per thread
+        uint4 x[NJ];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) x[j] = ldg_cg_v4(sp + ((half * NJ + j) * 128 + row) * 16);
+#pragma unroll
+        for (int part = 0; part < NJ / 4; ++part) {
+            const uint32_t v[16] = {x[4 * part].x, x[4 * part].y, x[4 * part].z, x[4 * part].w,
+                                    x[4 * part + 1].x, x[4 * part + 1].y, x[4 * part + 1].z, x[4 * part + 1].w,
+                                    x[4 * part + 2].x, x[4 * part + 2].y, x[4 * part + 2].z, x[4 * part + 2].w,
+                                    x[4 * part + 3].x, x[4 * part + 3].y, x[4 * part + 3].z, x[4 * part + 3].w};
+            tmem_st16(tq + cA1 + b * A1C + half * (A1C / 2) + 16 * part, v);
+        }
+    };
+    auto load_a23 = [&](int cl, int b) {
+        const char *sp = slot_of(cl);
+        if (has_s) {   // K-^T: lanes = d_k rows
+            uint4 x[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[j] = ldg_cg_v4(sp + RL::kA2 + ((half * 4 + j) * DK + row) * 16);
+            const uint32_t v[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
+                                    x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
+            tmem_st16(tq + cA2 + b * 32 + 16 * half, v);
+        }
+        if (has_o) {   // A: lanes 64-127 = token rows
+            uint4 x[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[j] = ldg_cg_v4(sp + RL::kA3 + ((half * 4 + j) * 64 + row - 64) * 16);
+            const uint32_t v[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
+                                    x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
+            tmem_st16(tq + cA3 + b * 32 + 16 * half, v);
+        }
+    };
+    // per-thread operands of chunk cl kept in registers: U~ (rows 0-63), Gamma_C (state rows),
+    // gate logits (output rows)
+    uint4 ut[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)}, gt[2] = {ut[0], ut[1]};
+    float gam = 0.f;
+    auto load_regs = [&](int cl, uint4 (&u_)[2], float &gam_, uint4 (&g_)[2]) {
+        const char *sp = slot_of(cl);
+        if (has_u) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) u_[j] = ldg_cg_v4(sp + RL::kU + ((((rank * 2 + half) * 2 + j) * 64) + row) * 16);
+        }
+        if (has_s) gam_ = __ldcg(reinterpret_cast<const float *>(sp + RL::kGam) + row);
+        g_[0] = g_[1] = make_uint4(0, 0, 0, 0);
+        if (has_o && p.gate) {
+            const int64_t tg = s0 + (int64_t)cl * kChunk + (row - 64);
+            if (tg < s1) {
+                const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + (tg * H + h) * DV + col0);
+                g_[0] = __ldg(gp);
+                g_[1] = __ldg(gp + 1);
+            }
+        }
+    };
 
-    // ring -> shared memory copies of the chain operands (16-byte cp.async, L2 only)
-    auto prefetch_wu = [&](int c) {   // W tiles and this slab's U~
-        const char *sp = slot_of(c);
+    // initial state; its fp16 copy is the first B operand
+    const size_t st_base = ((size_t)n * H + h) * DK * DV;
+    float S[16];
 #pragma unroll
-        for (int it = 0; it < 4 * KT * 32 / kRoleThreads; ++it) {
-            const int e = tid + it * kRoleThreads;   // 16-byte piece of the W tiles
-            cp_async_16(aPW + e * 16, sp + RL::kW + e * 16, 16);
-        }
-        {   // U~ of slab `rank`: 4 token tiles x 1 KB
-            const int m = tid >> 6, piece = tid & 63;
-            cp_async_16(aPU + m * 1024 + piece * 16, sp + RL::kU + (m * G + rank) * 1024 + piece * 16, 16);
-        }
-        cp_async_commit();
-    };
-    auto prefetch_kg = [&](int c) {   // K-^T tiles and Gamma_C
-        const char *sp = slot_of(c);
+    for (int j = 0; j < 16; ++j) S[j] = 0.f;
+    if (has_s && p.S_in) {
+        const float4 *sp = reinterpret_cast<const float4 *>(p.S_in + st_base + (size_t)row * DV + col0);
 #pragma unroll
-        for (int it = 0; it < 4 * KT * 32 / kRoleThreads; ++it) {
-            const int e = tid + it * kRoleThreads;
-            cp_async_16(aPK + e * 16, sp + RL::kKbT + e * 16, 16);
-        }
-        if (tid < DK / 4) cp_async_16(aPG + tid * 16, sp + RL::kGam + tid * 16, 16);
-        cp_async_commit();
-    };
-    // thread 0 waits for chunk c to be published; the role's barrier publishes the outcome
-    auto wait_full = [&](int c) {
-        if (tid == 0) {
-            const bool ok = mbar_wait_bounded(aFull + 8 * (c % R), (c / R) & 1, p.wait_ns);
-            if (!ok) atomicOr(&g_kda_error_word, kErrTimeout);
-            *abort_flag = ok ? 0 : 1;
-        }
-    };
-
-    // state tile of this warp: d_k rows 16 md + (g, g+8), slab columns 8 (sn0 + j) + 2 t4 (+1)
-    const int md = DK == 128 ? warp : (warp & 3);
-    const int sn0 = DK == 128 ? 0 : 2 * (warp >> 2);
-    const int r0 = 16 * md + g, r1 = r0 + 8;
-    const size_t st_base = ((size_t)n * H + h) * DK * DV + col0;
-    float S[SNT][4];
-#pragma unroll
-    for (int j = 0; j < SNT; ++j) {
-        const int cc = 8 * (sn0 + j) + 2 * t4;
-        if (p.S_in) {
-            const float2 x0 = *reinterpret_cast<const float2 *>(p.S_in + st_base + (size_t)r0 * DV + cc);
-            const float2 x1 = *reinterpret_cast<const float2 *>(p.S_in + st_base + (size_t)r1 * DV + cc);
-            S[j][0] = x0.x; S[j][1] = x0.y; S[j][2] = x1.x; S[j][3] = x1.y;
-        } else {
-            S[j][0] = S[j][1] = S[j][2] = S[j][3] = 0.f;
+        for (int j = 0; j < 4; ++j) {
+            const float4 x = sp[j];
+            S[4 * j] = x.x; S[4 * j + 1] = x.y; S[4 * j + 2] = x.z; S[4 * j + 3] = x.w;
         }
     }
-    // output tile of this warp: token rows 16 m + (g, g+8), slab columns 16 ch + 8 j + 2 t4 (+1)
-    const int m = warp & 3, ch = warp >> 2;
-    const int i0 = 16 * m + g, i1 = i0 + 8;
-    // gate logits of a chunk, loaded a chunk ahead (they come from HBM)
-    auto load_gate = [&](int cg, uint32_t (&gt)[2][2]) {
-        gt[0][0] = gt[0][1] = gt[1][0] = gt[1][1] = 0u;
-        if (!p.gate || cg >= nchunks) return;
-        const int64_t tg = s0 + (int64_t)cg * kChunk;
-        const int Lg = static_cast<int>(min64(kChunk, s1 - tg));
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int cc = col0 + 16 * ch + 8 * j + 2 * t4;
-            if (i0 < Lg) gt[j][0] = __ldg(reinterpret_cast<const unsigned int *>(p.gate + ((tg + i0) * H + h) * DV + cc));
-            if (i1 < Lg) gt[j][1] = __ldg(reinterpret_cast<const unsigned int *>(p.gate + ((tg + i1) * H + h) * DV + cc));
-        }
-    };
-    uint32_t gt[2][2];
-    load_gate(0, gt);
+    if (has_s) store_b(sB1, row, S);
 
-    if (nchunks > 0) {
-        wait_full(0);
-        named_bar(kBarConsumer, kRoleThreads);
-        if (*abort_flag) return;
-        prefetch_wu(0);
-        prefetch_kg(0);
+    if (nchunks > 0) {   // chunk 0's operands
+        wait_bar(aFull + 8 * 0, 0);
+        load_a1(0, 0);
+        load_a23(0, 0);
+        load_regs(0, ut, gam, gt);
     }
+    fence_async_smem();
+    tmem_wait_st();
+    tc_fence_before();
+    named_bar(kBarConsumer, kRoleThreads);
+    tc_fence_after();
+    if (*abort_flag) return;
+    if (nchunks > 0 && tid == 0) mbar_arrive_relaxed_cluster(mapa_shared(aEmpty, 0));   // slot 0 copied
 
     for (int c = 0; c < nchunks; ++c) {
-        const char *const slotp = slot_of(c);
+        const int buf = c & 1;
+        const bool has_next = c + 1 < nchunks;
         const int64_t t0 = s0 + (int64_t)c * kChunk;
         const int L = static_cast<int>(min64(kChunk, s1 - t0));
-        const bool has_next = c + 1 < nchunks;
-        // 1. fp16 copy of S_c (B operand of W S and Q^ S); Q^ and A of chunk c and the next
-        //    chunk's gate into registers
+        // 1. D = [W; Q^] S_c
+        if (tid == 0) {
 #pragma unroll
-        for (int j = 0; j < SNT; ++j) {
-            const int cc = 8 * (sn0 + j) + 2 * t4;
-            *reinterpret_cast<uint32_t *>(sS + swz_elem<64>(r0, cc)) = pack_f16(S[j][0], S[j][1]);
-            *reinterpret_cast<uint32_t *>(sS + swz_elem<64>(r1, cc)) = pack_f16(S[j][2], S[j][3]);
+            for (int k = 0; k < DK / 16; ++k)
+                umma_f16_ts(tmem + cD, tmem + cA1 + buf * A1C + 8 * k, umma_desc(aB1 + 1024 * k, 512, 128), kIdesc, k > 0);
+            umma_commit(aM1);
         }
-        uint4 Qf[KT], Af[4];
-#pragma unroll
-        for (int kd = 0; kd < KT; ++kd) Qf[kd] = ldg_cg_v4(slotp + RL::kQ + (m * KT + kd) * 512 + lane * 16);
-#pragma unroll
-        for (int kt = 0; kt < 4; ++kt)
-            Af[kt] = kt <= m ? ldg_cg_v4(slotp + RL::kA + (m * (m + 1) / 2 + kt) * 512 + lane * 16)
-                             : make_uint4(0, 0, 0, 0);
-        uint32_t gtn[2][2];
-        load_gate(c + 1, gtn);
-        cp_async_wait_group<1>();                  // this thread's W, U~ copies of chunk c
-        named_bar(kBarConsumer, kRoleThreads);     // all copies and sS visible
-
-        // 2. U = U~ - W S_c  (the chain; two independent partial sums halve the dependent MMAs)
-        float accU[2][4], accV[2][4], accO[2][4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) accU[j][e] = accV[j][e] = accO[j][e] = 0.f;
-#pragma unroll
-        for (int kd = 0; kd < KT; ++kd) {
-            uint32_t bf[4];
-            ldsm_x4_t(bf, ldsm_addr_bt<64>(aS, 16 * kd, 16 * ch, lane));
-            const uint4 w4 = *reinterpret_cast<const uint4 *>(sPW + (m * KT + kd) * 512 + lane * 16);
-            const uint32_t wa[4] = {w4.x, w4.y, w4.z, w4.w};
-            if (kd & 1) {
-                mma_f16(accV[0], wa, bf[0], bf[1]);
-                mma_f16(accV[1], wa, bf[2], bf[3]);
-            } else {
-                mma_f16(accU[0], wa, bf[0], bf[1]);
-                mma_f16(accU[1], wa, bf[2], bf[3]);
-            }
+        // 2. chunk c+1's [W; Q^] into the other buffer (its previous user, chunk c-1, is done)
+        if (has_next) {
+            wait_bar(aFull + 8 * ((c + 1) % R), ((c + 1) / R) & 1);
+            load_a1(c + 1, buf ^ 1);
         }
-        {
-            const uint4 u4 = *reinterpret_cast<const uint4 *>(sPU + m * 1024 + lane * 32 + ch * 16);
-            const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
+        // 3. U = U~ - W S_c  (rows 0-63) -> B operand of the next products
+        wait_bar(aM1, c & 1);
+        tc_fence_after();
+        if (has_u) {
+            uint32_t d[16];
+            tmem_ld16(tq + cD + 16 * half, d);
+            tmem_wait_ld();
+            float u[16];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const float2 ut0 = unpack_f16(uw[2 * j]), ut1 = unpack_f16(uw[2 * j + 1]);
-                const float u0 = ut0.x - (accU[j][0] + accV[j][0]), u1 = ut0.y - (accU[j][1] + accV[j][1]);
-                const float u2 = ut1.x - (accU[j][2] + accV[j][2]), u3 = ut1.y - (accU[j][3] + accV[j][3]);
-                const int cc = 16 * ch + 8 * j + 2 * t4;
-                *reinterpret_cast<uint32_t *>(sU + swz_elem<64>(i0, cc)) = pack_f16(u0, u1);
-                *reinterpret_cast<uint32_t *>(sU + swz_elem<64>(i1, cc)) = pack_f16(u2, u3);
-            }
-        }
-        // 3. chunk c+1 must be published before its W and U~ are copied
-        if (has_next) wait_full(c + 1);
-        cp_async_wait_group<0>();                  // this thread's K-^T, Gamma_C copies of chunk c
-        named_bar(kBarConsumer, kRoleThreads);     // U complete; W, U~ buffers free; K-^T visible
-        if (has_next && *abort_flag) return;
-        if (has_next) prefetch_wu(c + 1);
-
-        // 4. O = Q^ S_c (off the chain)
+                const uint32_t w4[4] = {ut[j].x, ut[j].y, ut[j].z, ut[j].w};
 #pragma unroll
-        for (int kd = 0; kd < KT; ++kd) {
-            uint32_t bf[4];
-            ldsm_x4_t(bf, ldsm_addr_bt<64>(aS, 16 * kd, 16 * ch, lane));
-            const uint32_t qa[4] = {Qf[kd].x, Qf[kd].y, Qf[kd].z, Qf[kd].w};
-            mma_f16(accO[0], qa, bf[0], bf[1]);
-            mma_f16(accO[1], qa, bf[2], bf[3]);
-        }
-
-        // 5. S_{c+1} = Diag(Gamma_C) S_c + K-^T U   (the chain)
-        {
-            const float gam0 = sPG[r0], gam1 = sPG[r1];
-#pragma unroll
-            for (int j = 0; j < SNT; ++j) {
-                S[j][0] *= gam0; S[j][1] *= gam0; S[j][2] *= gam1; S[j][3] *= gam1;
-            }
-            float Sx[SNT][4];   // odd token tiles accumulate separately (two short chains)
-#pragma unroll
-            for (int j = 0; j < SNT; ++j) Sx[j][0] = Sx[j][1] = Sx[j][2] = Sx[j][3] = 0.f;
-#pragma unroll
-            for (int kt = 0; kt < 4; ++kt) {
-                const uint4 k4 = *reinterpret_cast<const uint4 *>(sPK + (md * 4 + kt) * 512 + lane * 16);
-                const uint32_t ka[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-                for (int np = 0; np < SNT / 2; ++np) {
-                    uint32_t bf[4];
-                    ldsm_x4_t(bf, ldsm_addr_bt<64>(aU, 16 * kt, 8 * sn0 + 16 * np, lane));
-                    float(*dst)[4] = (kt & 1) ? Sx : S;
-                    mma_f16(dst[2 * np], ka, bf[0], bf[1]);
-                    mma_f16(dst[2 * np + 1], ka, bf[2], bf[3]);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 t = unpack_f16(w4[e]);
+                    u[8 * j + 2 * e] = t.x - __uint_as_float(d[8 * j + 2 * e]);
+                    u[8 * j + 2 * e + 1] = t.y - __uint_as_float(d[8 * j + 2 * e + 1]);
                 }
             }
-#pragma unroll
-            for (int j = 0; j < SNT; ++j)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) S[j][e] += Sx[j][e];
+            store_b(sB2, row, u);
         }
-
-        // 6. O += A U, gate, store
-#pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            if (kt <= m) {
-                uint32_t bf[4];
-                ldsm_x4_t(bf, ldsm_addr_bt<64>(aU, 16 * kt, 16 * ch, lane));
-                const uint32_t aa[4] = {Af[kt].x, Af[kt].y, Af[kt].z, Af[kt].w};
-                mma_f16(accO[0], aa, bf[0], bf[1]);
-                mma_f16(accO[1], aa, bf[2], bf[3]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int cc = col0 + 16 * ch + 8 * j + 2 * t4;
-            float o0 = accO[j][0], o1 = accO[j][1], o2 = accO[j][2], o3 = accO[j][3];
-            if (p.gate) {
-                const float2 ga = unpack_bf16(gt[j][0]), gb = unpack_bf16(gt[j][1]);
-                o0 *= sigmoid_fast(ga.x); o1 *= sigmoid_fast(ga.y);
-                o2 *= sigmoid_fast(gb.x); o3 *= sigmoid_fast(gb.y);
-            }
-            if (i0 < L) {
-                const int64_t off = ((t0 + i0) * H + h) * DV + cc;
-                if (p.out_f32) *reinterpret_cast<float2 *>(static_cast<float *>(p.out) + off) = make_float2(o0, o1);
-                else *reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(p.out) + off) = pack_bf16(o0, o1);
-            }
-            if (i1 < L) {
-                const int64_t off = ((t0 + i1) * H + h) * DV + cc;
-                if (p.out_f32) *reinterpret_cast<float2 *>(static_cast<float *>(p.out) + off) = make_float2(o2, o3);
-                else *reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(p.out) + off) = pack_bf16(o2, o3);
-            }
-        }
-        gt[0][0] = gtn[0][0]; gt[0][1] = gtn[0][1]; gt[1][0] = gtn[1][0]; gt[1][1] = gtn[1][1];
-        // 7. every warp is done with this slot, sS, sU and the K-^T buffer: return the slot to the
-        //    CTA that produces it.  Every value read from the slot has already arrived in registers
-        //    or shared memory, so the hand-back needs no release ordering (a release would wait for
-        //    this chunk's output stores).
+        fence_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
         named_bar(kBarConsumer, kRoleThreads);
-        if (tid == 0) mbar_arrive_relaxed_cluster(mapa_shared(aEmpty + 8 * (c % R), (c % R) % G));
-        if (has_next) prefetch_kg(c + 1);
-    }
-    if (p.S_out) {
+        tc_fence_after();
+        if (*abort_flag) return;
+        // 4. D3 = K-^T U;  D[64:128] += A U
+        if (tid == 0) {
 #pragma unroll
-        for (int j = 0; j < SNT; ++j) {
-            const int cc = 8 * (sn0 + j) + 2 * t4;
-            *reinterpret_cast<float2 *>(p.S_out + st_base + (size_t)r0 * DV + cc) = make_float2(S[j][0], S[j][1]);
-            *reinterpret_cast<float2 *>(p.S_out + st_base + (size_t)r1 * DV + cc) = make_float2(S[j][2], S[j][3]);
+            for (int k = 0; k < 4; ++k)
+                umma_f16_ts(tmem + cD3, tmem + cA2 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, k > 0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                umma_f16_ts(tmem + cD, tmem + cA3 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, 1);
+            umma_commit(aM2);
         }
+        // 5. the rest of chunk c+1's operands
+        uint4 utn[2] = {ut[0], ut[1]}, gtn[2] = {gt[0], gt[1]};
+        float gamn = gam;
+        if (has_next) {
+            load_a23(c + 1, buf ^ 1);
+            load_regs(c + 1, utn, gamn, gtn);
+        }
+        // 6. S_{c+1} = Diag(Gamma_C) S_c + D3;  gated output rows
+        wait_bar(aM2, c & 1);
+        tc_fence_after();
+        if (has_s) {
+            uint32_t d[16];
+            tmem_ld16(tq + cD3 + 16 * half, d);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(gam, S[j], __uint_as_float(d[j]));
+            store_b(sB1, row, S);
+        }
+        if (has_o) {
+            uint32_t d[16];
+            tmem_ld16(tq + cD + 16 * half, d);
+            tmem_wait_ld();
+            const int i = row - 64;
+            if (i < L) {
+                float o[16];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t g4[4] = {gt[j].x, gt[j].y, gt[j].z, gt[j].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float o0 = __uint_as_float(d[8 * j + 2 * e]), o1 = __uint_as_float(d[8 * j + 2 * e + 1]);
+                        if (p.gate) {
+                            const float2 ga = unpack_bf16(g4[e]);
+                            o0 *= sigmoid_fast(ga.x);
+                            o1 *= sigmoid_fast(ga.y);
+                        }
+                        o[8 * j + 2 * e] = o0;
+                        o[8 * j + 2 * e + 1] = o1;
+                    }
+                }
+                const int64_t off = ((t0 + i) * H + h) * DV + col0;
+                if (p.out_f32) {
+                    float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) op[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                } else {
+                    uint4 *op = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + off);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+                        op[j] = make_uint4(pack_bf16(o[8 * j], o[8 * j + 1]), pack_bf16(o[8 * j + 2], o[8 * j + 3]),
+                                           pack_bf16(o[8 * j + 4], o[8 * j + 5]), pack_bf16(o[8 * j + 6], o[8 * j + 7]));
+                }
+            }
+        }
+        fence_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        named_bar(kBarConsumer, kRoleThreads);
+        tc_fence_after();
+        if (*abort_flag) return;
+        // 7. chunk c+1 now lives in TMEM and registers: hand its slot back to the producing CTA.
+        //    Every value read from it has arrived, so no release ordering is needed.
+        if (has_next && tid == 0)
+            mbar_arrive_relaxed_cluster(mapa_shared(aEmpty + 8 * ((c + 1) % R), ((c + 1) % R) % G));
+        ut[0] = utn[0]; ut[1] = utn[1]; gt[0] = gtn[0]; gt[1] = gtn[1];
+        gam = gamn;
+    }
+    if (has_s && p.S_out) {
+        float4 *sp = reinterpret_cast<float4 *>(p.S_out + st_base + (size_t)row * DV + col0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sp[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
     }
 }
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kFusedThreads, 1) kda_prefill_fused_kernel(const FusedParams p) {
+    using SM = FusedSmem<DK, DV>;
     constexpr int G = DV / kSlab;
+    constexpr uint32_t kTmemCols = DK == 128 ? 512 : 256;   // see the column map of the consumer
     extern __shared__ __align__(1024) unsigned char fsmem[];
     const int unit = blockIdx.x / G, rank = blockIdx.x % G;
     const int n = unit / p.H, h = unit % p.H;
@@ -833,17 +863,32 @@ __global__ void __launch_bounds__(kFusedThreads, 1) kda_prefill_fused_kernel(con
     const int nchunks = static_cast<int>((s1 - s0 + kChunk - 1) / kChunk);
     // The cluster is G CTAs along x, so `rank` is this CTA's rank in it.
     if (threadIdx.x < RingLayout<DK, DV>::R) {
-        using SM = FusedSmem<DK, DV>;
         mbar_init(smem_u32(fsmem + SM::kFull) + 8 * threadIdx.x, 1);
         mbar_init(smem_u32(fsmem + SM::kEmpty) + 8 * threadIdx.x, G);
     }
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(fsmem + SM::kM1), 1);
+        mbar_init(smem_u32(fsmem + SM::kM2), 1);
+        *reinterpret_cast<volatile int *>(fsmem + SM::kCFlag) = 0;
+        *reinterpret_cast<volatile int *>(fsmem + SM::kPFlag) = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(smem_u32(fsmem + SM::kTmem), kTmemCols);
+    tc_fence_before();
     cluster_sync_after_init();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(fsmem + SM::kTmem);
     if (threadIdx.x < kRoleThreads)
-        fused_consumer<DK, DV>(p, fsmem, unit, n, h, rank, s0, s1, nchunks);
+        fused_consumer<DK, DV>(p, fsmem, tmem, unit, n, h, rank, s0, s1, nchunks);
     else
         fused_producer<DK, DV>(p, fsmem, unit, h, rank, s0, s1, nchunks);
     cp_async_wait_all();
+    tc_fence_before();
     cluster_sync();   // no CTA exits while a peer may still arrive on its barriers
+    tc_fence_after();
+    if (threadIdx.x < 32) {
+        __syncwarp();
+        tmem_dealloc(tmem, kTmemCols);
+    }
 }
 
 }  // namespace kda
