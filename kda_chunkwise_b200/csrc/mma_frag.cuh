@@ -259,6 +259,20 @@ __device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
     return ok != 0;
 }
 
+// Wait (acquire, cluster scope) for the phase with parity `parity` of a local mbarrier, letting the
+// hardware suspend the thread for a bounded, implementation-defined time; true once the phase has
+// completed, false if the suspension ended first.
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 
 template <int N>

@@ -26,11 +26,14 @@
 // for unit keys and bounded values.  The state itself stays fp32 in registers.
 //
 // Work decomposition.  A unit is one (sequence, head).  Its d_v columns are split into G slabs
-// of 32; the unit runs on a cluster of G CTAs (the cluster only guarantees the G CTAs run at the
-// same time).  Every CTA has 16 warps:
-//   consumer warps 0-7:  the sequential state pass for slab `rank` of the unit.
-//   producer warps 8-15: the chunk-parallel work for chunks rank, rank + G, rank + 2G, ...,
-//                        written as ready-to-use mma fragments into the unit's ring.
+// of 32; the unit runs on a cluster of G CTAs (the cluster guarantees the G CTAs run at the same
+// time and gives them each other's shared-memory barriers).  Every CTA has 16 warps:
+//   consumer warps 0-7:  the sequential state pass for slab `rank` of the unit, on tcgen05: the
+//                        chunk's A operands in tensor memory, S and U as fp16 B operands in
+//                        shared memory, fp32 accumulators in tensor memory.
+//   producer warps 8-15: the chunk-parallel work for chunks rank, rank + G, rank + 2G, ...
+//                        (mma.sync tiles of 16), written into the unit's ring in the layout the
+//                        consumer copies straight into tensor memory.
 // The ring (2G slots per unit, in the workspace, small enough to stay in L2) carries chunk c in
 // slot c % 2G.  Shared-memory mbarriers order the hand-off at cluster scope: every CTA has a
 // `full` barrier per slot, on which the producing CTA arrives (remotely) once the chunk is in the
@@ -93,13 +96,12 @@ struct FusedSmem {
     static constexpr int kV = kK + 64 * DK * 2;       // bf16 [64][DV] v
     static constexpr int kKr = kV + 64 * DV * 2;      // bf16 [64][DK] a, then k e^{b - r}
     static constexpr int kKh = kKr + 64 * DK * 2;     // fp16 [64][DK] K^
-    static constexpr int kKt = kKh + 64 * DK * 2;     // fp32 [64][DK] K~; later fp16 T' [64][64]
-    static constexpr int kKtBytes = (64 * DK * 4 > 64 * 64 * 2) ? 64 * DK * 4 : 64 * 64 * 2;
-    static constexpr int kB = kKt + kKtBytes;         // scratch of the later phases:
+    static constexpr int kKt = kKh + 64 * DK * 2;     // fp32 [64][DK] K~
+    static constexpr int kB = kKt + 64 * DK * 4;      // scratch of the later phases:
     static constexpr int kLd = kB;                    //   fp32 [4][16][17] diagonal blocks of L
     static constexpr int kLD = kLd + 4 * 16 * 17 * 4;   //   fp16 [64][64]: -L below the diagonal
                                                       //   blocks, (I + L_pp)^-1 on them
-    static constexpr int kT = kLD + 64 * 64 * 2;      //   fp16 [64][64] T = (I + L)^-1
+    static constexpr int kT = kLD + 64 * 64 * 2;      //   fp16 [64][64] T' = (I + L)^-1 diag(beta)
     static constexpr int kM = kT + 64 * 64 * 2;       //   fp16 [3][16][32] block-product scratch
     static constexpr int kQh = kT;                    //   fp16 [64][DK] Q^, copied to the ring
                                                       //   before T and M are written
@@ -139,19 +141,15 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
     return t;
 }
 
-// Spin (one thread) until the phase with parity `parity` of a local mbarrier completes, at most
-// wait_ns.  Returns false on timeout.
+// Wait until the phase with parity `parity` of a local mbarrier completes, at most wait_ns
+// (hardware-suspended polls, %globaltimer bound).  Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity,
                                                   unsigned long long wait_ns) {
-    if (mbar_test(addr, parity)) return true;
+    if (mbar_try(addr, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
-    unsigned ns = 32;
-    while (true) {
-        __nanosleep(ns);
-        if (mbar_test(addr, parity)) return true;
-        if (ns < 256) ns <<= 1;
+    while (!mbar_try(addr, parity))
         if (globaltimer_ns() - t0 > wait_ns) return false;
-    }
+    return true;
 }
 
 __device__ __forceinline__ float2 unpack_f16(uint32_t v) {
@@ -177,7 +175,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
 
     unsigned char *const sQhi = sm + SM::kQhi, *const sQlo = sm + SM::kQlo, *const sK = sm + SM::kK;
     unsigned char *const sKr = sm + SM::kKr, *const sKh = sm + SM::kKh, *const sKb = sm + SM::kK;
-    unsigned char *const sKt = sm + SM::kKt, *const sTp = sm + SM::kKt, *const sV = sm + SM::kV;
+    unsigned char *const sKt = sm + SM::kKt, *const sV = sm + SM::kV;
     unsigned char *const sQh = sm + SM::kQh, *const sLD = sm + SM::kLD, *const sT = sm + SM::kT;
     unsigned char *const sM = sm + SM::kM;
     float *const sLd = reinterpret_cast<float *>(sm + SM::kLd);
@@ -192,7 +190,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
     const uint32_t aFull = smem_u32(sm + SM::kFull), aEmpty = smem_u32(sm + SM::kEmpty);
     const uint32_t aQhi = smem_u32(sQhi), aQlo = smem_u32(sQlo), aK = smem_u32(sK);
     const uint32_t aV = smem_u32(sV), aKr = smem_u32(sKr), aKh = smem_u32(sKh);
-    const uint32_t aKb = smem_u32(sKb), aTp = smem_u32(sTp), aLD = smem_u32(sLD);
+    const uint32_t aKb = smem_u32(sKb), aLD = smem_u32(sLD);
     const uint32_t aT = smem_u32(sT), aM = smem_u32(sM), aQh = smem_u32(sQh);
 
     // asynchronous input copies of one chunk: q, k, a as one commit group, v as another
@@ -430,9 +428,10 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
             stg_v4(slotp + RL::kA3 + ((2 * qb + (lane >> 4)) * 64 + 16 * pb + (lane & 15)) * 16, make_uint4(0, 0, 0, 0));
         }
-        // 4b. K-^T and Q^ to the ring.  K-^T tile (d_k tile md, token tile kt) as an A fragment:
-        //     register e of a lane is row 16md + g (+8 for e odd), columns 8kt + t4 (+4 for e >= 2).
-        for (int idx = warp; idx < 4 * KT; idx += 8) {
+        // 4b. K-^T and Q^ to the ring, by warps 2-7 (warps 0 and 1 take two Gram blocks each).
+        //     K-^T tile (d_k tile md, token tile kt) as an A fragment: register e of a lane is row
+        //     16md + g (+8 for e odd), columns 8kt + t4 (+4 for e >= 2).
+        for (int idx = warp - 2; idx >= 0 && idx < 4 * KT; idx += 6) {
             uint32_t fr[4];
             const int md = idx / 4, kt = idx % 4;
             ldsm_x4_t(fr, ldsm_addr_bn<RB>(aKb, 16 * kt, 16 * md, lane));
@@ -442,7 +441,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             st_u32(b + DK * 16, fr[2]);
             st_u32(b + DK * 16 + 8 * 16, fr[3]);
         }
-        for (int e = tid; e < 64 * (DK / 8); e += kRoleThreads) {   // Q^ row t -> lane 64 + t
+        for (int e = tid - 64; e >= 0 && e < 64 * (DK / 8); e += kRoleThreads - 64) {   // Q^ row t -> lane 64 + t
             const int t = e & 63, j = e >> 6;
             stg_v4(slotp + RL::kA1 + (j * 128 + 64 + t) * 16, *reinterpret_cast<const uint4 *>(sQh + swz<RB>(t, j)));
         }
@@ -463,17 +462,22 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             for (int j = 0; j < 15; ++j)
 #pragma unroll
                 for (int i = j + 1; i < 16; ++i) x[i] = fmaf(-Ld[i * 17 + j], x[j], x[i]);
+            const float bcol = sbeta[16 * pb + mcol];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const __half hv = __float2half_rn(x[i]);
-                *reinterpret_cast<__half *>(sLD + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = hv;
-                *reinterpret_cast<__half *>(sT + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = hv;
+                *reinterpret_cast<__half *>(sLD + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = __float2half_rn(x[i]);
+                *reinterpret_cast<__half *>(sT + swz_elem<128>(16 * pb + i, 16 * pb + mcol)) = __float2half_rn(x[i] * bcol);
             }
         }
+        // this chunk's v rows (their group is older than the next chunk's q, k, a group)
+        if (c + G < nchunks) cp_async_wait_group<1>();
+        else cp_async_wait_group<0>();
         named_bar(kBarProducer, kRoleThreads);
 
-        // 5b. off-diagonal blocks of T = (I + L)^-1 by level d = p - q:
-        //     T_pq = D_p M,  M = sum_{m=q}^{p-1} (-L_pm) T_mq   (16x16 tensor-core products)
+        // 5b. off-diagonal blocks of T' = (I + L)^-1 diag(beta) by level d = p - q:
+        //     T'_pq = D_p M,  M = sum_{m=q}^{p-1} (-L_pm) T'_mq   (16x16 tensor-core products);
+        //     the recursion is linear in the columns of block column q, so starting it from the
+        //     diagonal blocks D_q diag(beta_q) yields T' directly.
 #pragma unroll 1
         for (int d = 1; d < 4; ++d) {
             if (warp < 4 - d) {
@@ -512,21 +516,6 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             }
             named_bar(kBarProducer, kRoleThreads);
         }
-        // T' = T diag(beta), lower triangle (blocks above the diagonal are never read)
-        for (int e = tid; e < 64 * 32; e += kRoleThreads) {
-            const int i = e >> 5, j = (e & 31) * 2;
-            if ((j >> 4) <= (i >> 4)) {
-                const float2 tv = unpack_f16(*reinterpret_cast<const uint32_t *>(sT + swz_elem<128>(i, j)));
-                *reinterpret_cast<uint32_t *>(sTp + swz_elem<128>(i, j)) = pack_f16(tv.x * sbeta[j], tv.y * sbeta[j + 1]);
-            }
-        }
-        named_bar(kBarProducer, kRoleThreads);
-
-        // v of this chunk (its group is older than the next chunk's q, k, a group)
-        if (c + G < nchunks) cp_async_wait_group<1>();
-        else cp_async_wait_group<0>();
-        named_bar(kBarProducer, kRoleThreads);
-
         // 6. [W | U~] = T' [K^ | V].  Warp w owns 16-column units w and w + 8 of [W | U~]; the B
         //    fragments of a unit are loaded once per token tile and reused for every row tile.
         {
@@ -552,7 +541,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
 #pragma unroll
                     for (int kt = 0; kt <= m; ++kt) {
                         uint32_t af[4];
-                        ldsm_x4(af, ldsm_addr_a<128>(aTp, 16 * m, 16 * kt, lane));
+                        ldsm_x4(af, ldsm_addr_a<128>(aT, 16 * m, 16 * kt, lane));
                         mma_f16(acc[0], af, bfr[kt][0], bfr[kt][1]);
                         mma_f16(acc[1], af, bfr[kt][2], bfr[kt][3]);
                     }
@@ -590,9 +579,9 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
 //   U  = U~ - D[0:64]  -> shared memory (fp16, B operand)
 //   D3 = K-^T U,   D[64:128] += A U                                                  TMEM
 //   S_{c+1} = Diag(Gamma_C) S_c + D3;   out = sigmoid(gate) D[64:128]
-// The A operands ([W; Q^], K-^T, A) of chunk c + 1 are copied from the ring into the other of two
-// TMEM buffers while chunk c's products run; the ring slot is handed back as soon as that copy
-// is done.  One thread issues the MMAs; every wait is bounded.
+// The A operands ([W; Q^], K-^T, A) of chunk c + 1 are fetched from the ring into registers while
+// chunk c's products run and then stored into the other of two TMEM buffers; the ring slot is
+// handed back as soon as that copy is done.  One thread issues the MMAs; every wait is bounded.
 // ---------------------------------------------------------------------------------------------
 template <int DK, int DV>
 __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned char *sm, uint32_t tmem, int unit,
@@ -633,59 +622,52 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             *reinterpret_cast<uint4 *>(base + (((k >> 3) * 4 + 2 * half + g8) * 64 + (k & 7) * 8) * 2) = v;
         }
     };
-    // chunk cl's A operands into TMEM buffer b (each warp: its lane quadrant, its half of the columns)
-    auto load_a1 = [&](int cl, int b) {
-        const char *sp = slot_of(cl) + RL::kA1;
-        constexpr int NJ = A1C / 8;                    // 16-byte chunks per thread
-        uint4 x[NJ];
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) x[j] = ldg_cg_v4(sp + ((half * NJ + j) * 128 + row) * 16);
-#pragma unroll
-        for (int part = 0; part < NJ / 4; ++part) {
-            const uint32_t v[16] = {x[4 * part].x, x[4 * part].y, x[4 * part].z, x[4 * part].w,
-                                    x[4 * part + 1].x, x[4 * part + 1].y, x[4 * part + 1].z, x[4 * part + 1].w,
-                                    x[4 * part + 2].x, x[4 * part + 2].y, x[4 * part + 2].z, x[4 * part + 2].w,
-                                    x[4 * part + 3].x, x[4 * part + 3].y, x[4 * part + 3].z, x[4 * part + 3].w};
-            tmem_st16(tq + cA1 + b * A1C + half * (A1C / 2) + 16 * part, v);
-        }
-    };
-    auto load_a23 = [&](int cl, int b) {
+    // chunk cl's A operands: fetched from the ring into registers, then stored into TMEM buffer b
+    // (each warp: its lane quadrant, its half of the columns)
+    constexpr int NJ = A1C / 8;                        // 16-byte pieces of [W; Q^] per thread
+    auto fetch_a12 = [&](int cl, uint4 (&x1)[NJ], uint4 (&x2)[4]) {
         const char *sp = slot_of(cl);
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) x1[j] = ldg_cg_v4(sp + RL::kA1 + ((half * NJ + j) * 128 + row) * 16);
         if (has_s) {   // K-^T: lanes = d_k rows
-            uint4 x[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) x[j] = ldg_cg_v4(sp + RL::kA2 + ((half * 4 + j) * DK + row) * 16);
-            const uint32_t v[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
-                                    x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
-            tmem_st16(tq + cA2 + b * 32 + 16 * half, v);
-        }
-        if (has_o) {   // A: lanes 64-127 = token rows
-            uint4 x[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) x[j] = ldg_cg_v4(sp + RL::kA3 + ((half * 4 + j) * 64 + row - 64) * 16);
-            const uint32_t v[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
-                                    x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
-            tmem_st16(tq + cA3 + b * 32 + 16 * half, v);
+            for (int j = 0; j < 4; ++j) x2[j] = ldg_cg_v4(sp + RL::kA2 + ((half * 4 + j) * DK + row) * 16);
         }
     };
-    // per-thread operands of chunk cl kept in registers: U~ (rows 0-63), Gamma_C (state rows),
-    // gate logits (output rows)
+    auto fetch_a3 = [&](int cl, uint4 (&x3)[4]) {   // A: lanes 64-127 = token rows (has_o threads)
+        const char *sp = slot_of(cl);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x3[j] = ldg_cg_v4(sp + RL::kA3 + ((half * 4 + j) * 64 + row - 64) * 16);
+    };
+    auto st4 = [&](uint32_t taddr, const uint4 *x) {
+        const uint32_t v[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
+                                x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
+        tmem_st16(taddr, v);
+    };
+    auto put_a = [&](int b, const uint4 (&x1)[NJ], const uint4 (&x2)[4], const uint4 (&x3)[4]) {
+#pragma unroll
+        for (int part = 0; part < NJ / 4; ++part) st4(tq + cA1 + b * A1C + half * (A1C / 2) + 16 * part, x1 + 4 * part);
+        if (has_s) st4(tq + cA2 + b * 32 + 16 * half, x2);
+        if (has_o) st4(tq + cA3 + b * 32 + 16 * half, x3);
+    };
+    // per-thread operands kept in registers: U~ (rows 0-63), Gamma_C (state rows), gate logits
+    // (output rows); each is reloaded for the next chunk right after its last use
     uint4 ut[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)}, gt[2] = {ut[0], ut[1]};
     float gam = 0.f;
-    auto load_regs = [&](int cl, uint4 (&u_)[2], float &gam_, uint4 (&g_)[2]) {
+    auto load_ut = [&](int cl) {
         const char *sp = slot_of(cl);
-        if (has_u) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) u_[j] = ldg_cg_v4(sp + RL::kU + ((((rank * 2 + half) * 2 + j) * 64) + row) * 16);
-        }
-        if (has_s) gam_ = __ldcg(reinterpret_cast<const float *>(sp + RL::kGam) + row);
-        g_[0] = g_[1] = make_uint4(0, 0, 0, 0);
-        if (has_o && p.gate) {
+        for (int j = 0; j < 2; ++j) ut[j] = ldg_cg_v4(sp + RL::kU + ((((rank * 2 + half) * 2 + j) * 64) + row) * 16);
+    };
+    auto load_gam = [&](int cl) { return __ldcg(reinterpret_cast<const float *>(slot_of(cl) + RL::kGam) + row); };
+    auto load_gate = [&](int cl) {
+        gt[0] = gt[1] = make_uint4(0, 0, 0, 0);
+        if (p.gate) {
             const int64_t tg = s0 + (int64_t)cl * kChunk + (row - 64);
             if (tg < s1) {
                 const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + (tg * H + h) * DV + col0);
-                g_[0] = __ldg(gp);
-                g_[1] = __ldg(gp + 1);
+                gt[0] = __ldg(gp);
+                gt[1] = __ldg(gp + 1);
             }
         }
     };
@@ -705,11 +687,17 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     }
     if (has_s) store_b(sB1, row, S);
 
+    uint4 x1[NJ], x2[4], x3[4];
     if (nchunks > 0) {   // chunk 0's operands
         wait_bar(aFull + 8 * 0, 0);
-        load_a1(0, 0);
-        load_a23(0, 0);
-        load_regs(0, ut, gam, gt);
+        fetch_a12(0, x1, x2);
+        if (has_o) fetch_a3(0, x3);
+        if (has_u) load_ut(0);
+        if (has_s) gam = load_gam(0);
+        if (has_o) load_gate(0);
+        put_a(0, x1, x2, x3);
+        if (has_u) asm volatile("" ::"r"(ut[0].x), "r"(ut[1].x));   // arrived before slot 0 is handed back
+        if (has_s) asm volatile("" ::"f"(gam));
     }
     fence_async_smem();
     tmem_wait_st();
@@ -731,10 +719,12 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                 umma_f16_ts(tmem + cD, tmem + cA1 + buf * A1C + 8 * k, umma_desc(aB1 + 1024 * k, 512, 128), kIdesc, k > 0);
             umma_commit(aM1);
         }
-        // 2. chunk c+1's [W; Q^] into the other buffer (its previous user, chunk c-1, is done)
+        // 2. chunk c+1's operands into registers; their L2 latency overlaps this chunk's products
+        float gamn = 0.f;
         if (has_next) {
             wait_bar(aFull + 8 * ((c + 1) % R), ((c + 1) / R) & 1);
-            load_a1(c + 1, buf ^ 1);
+            fetch_a12(c + 1, x1, x2);
+            if (has_s) gamn = load_gam(c + 1);
         }
         // 3. U = U~ - W S_c  (rows 0-63) -> B operand of the next products
         wait_bar(aM1, c & 1);
@@ -755,6 +745,9 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                 }
             }
             store_b(sB2, row, u);
+            if (has_next) load_ut(c + 1);
+        } else if (has_next) {
+            fetch_a3(c + 1, x3);
         }
         fence_async_smem();
         tmem_wait_st();
@@ -772,13 +765,8 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                 umma_f16_ts(tmem + cD, tmem + cA3 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, 1);
             umma_commit(aM2);
         }
-        // 5. the rest of chunk c+1's operands
-        uint4 utn[2] = {ut[0], ut[1]}, gtn[2] = {gt[0], gt[1]};
-        float gamn = gam;
-        if (has_next) {
-            load_a23(c + 1, buf ^ 1);
-            load_regs(c + 1, utn, gamn, gtn);
-        }
+        // 5. chunk c+1's A operands into the other TMEM buffer (its last user, chunk c-1, is done)
+        if (has_next) put_a(buf ^ 1, x1, x2, x3);
         // 6. S_{c+1} = Diag(Gamma_C) S_c + D3;  gated output rows
         wait_bar(aM2, c & 1);
         tc_fence_after();
@@ -825,6 +813,12 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                                            pack_bf16(o[8 * j + 4], o[8 * j + 5]), pack_bf16(o[8 * j + 6], o[8 * j + 7]));
                 }
             }
+            if (has_next) load_gate(c + 1);
+        }
+        // every value read from slot c+1 must have arrived before the slot is handed back
+        if (has_next) {
+            if (has_u) asm volatile("" ::"r"(ut[0].x), "r"(ut[1].x));
+            if (has_s) asm volatile("" ::"f"(gamn));
         }
         fence_async_smem();
         tmem_wait_st();
@@ -836,7 +830,6 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         //    Every value read from it has arrived, so no release ordering is needed.
         if (has_next && tid == 0)
             mbar_arrive_relaxed_cluster(mapa_shared(aEmpty + 8 * ((c + 1) % R), ((c + 1) % R) % G));
-        ut[0] = utn[0]; ut[1] = utn[1]; gt[0] = gtn[0]; gt[1] = gtn[1];
         gam = gamn;
     }
     if (has_s && p.S_out) {
