@@ -73,6 +73,20 @@ def decode_bytes(dw) -> int:
     return dw.N * dw.H * per_unit
 
 
+def spec_bytes(sw, accepted) -> int:
+    """Algorithmic bytes of one verify + commit round: verify reads every state and the K tokens'
+    inputs and writes the outputs and write vectors; commit reads and writes the states of the
+    sequences that accepted at least one token, plus those tokens' k, a and write vectors."""
+    units = sw.N * sw.H
+    state = sw.d_k * sw.d_v * 4
+    per_tok_in = 2 * (3 * sw.d_k + 2 * sw.d_v) + 4
+    verify = units * (state + sw.K * (per_tok_in + 2 * sw.d_v + 4 * sw.d_v))
+    acc = [int(x) for x in accepted.cpu().tolist()]
+    moved = sum(1 for x in acc if x > 0) * sw.H
+    commit = moved * 2 * state + sum(acc) * sw.H * (2 * 2 * sw.d_k + 4 * sw.d_v)
+    return verify + commit
+
+
 def decode_flops(dw) -> float:
     return dw.N * dw.H * 7.0 * dw.d_k * dw.d_v
 
@@ -365,6 +379,48 @@ def main():
         del d, state, dout
         torch.cuda.empty_cache()
 
+    # speculative decode row: rounds of verify (K proposed tokens) + commit (accepted prefixes)
+    spec = None
+    if not args.no_decode:
+        sw = dataclasses.replace(KI.SPEC, seed=KI.SPEC.seed + rank)
+        d = KI.make_spec_inputs(sw, dev)
+        state = d["state"].clone()
+        sout = torch.empty((sw.N, sw.K, sw.H, sw.d_v), dtype=torch.bfloat16, device=dev)
+        su = torch.empty((sw.N, sw.H, sw.K, sw.d_v), dtype=torch.float32, device=dev)
+
+        def sround(r):
+            kda.kda_decode_verify(d["q"][r], d["k"][r], d["v"][r], d["a"][r], d["beta"][r], d["A_log"],
+                                  state, gate=d["gate"][r], u=su, out=sout, stream=stream)
+            kda.kda_decode_commit(d["k"][r], d["a"][r], d["A_log"], d["accepted"][r], su, state,
+                                  stream=stream)
+
+        for r in range(max(3, args.warmup)):
+            sround(r % sw.rounds)
+        state.copy_(d["state"])
+        barrier()
+        clocks.active(True)
+        e0.record(stream)
+        for r in range(sw.rounds):
+            sround(r)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.active(False)
+        barrier()
+        kda.kda_sync_check()
+        sms = max_over_ranks(e0.elapsed_time(e1) / sw.rounds, world, dev)
+        sbytes = sum(spec_bytes(sw, d["accepted"][r]) for r in range(sw.rounds)) / sw.rounds
+        accepted_per_round = float(d["accepted"].to(torch.float64).sum()) / sw.rounds   # tokens, all heads
+        sach = sbytes / (sms * 1e-3) / 1e9
+        spec = {"value": whole_job_rate(accepted_per_round, world, sms), "unit": "accepted tokens/s",
+                "ms_per_round": sms, "workload": sw.name, "proposed_per_round": sw.N * sw.K,
+                "accepted_per_round": accepted_per_round,
+                "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s",
+                             "frac": sach / hbm, "traffic": None, "peak_source": f"hbm_gbs of {peak_src}",
+                             "algorithmic_bytes": int(sbytes),
+                             "scope": "one round = kda_decode_verify + kda_decode_commit"}}
+        del d, state, sout, su
+        torch.cuda.empty_cache()
+
     # end to end through the public API: pinned host inputs -> device -> kda_chunk_fwd -> host
     e2e = None
     if not args.no_e2e:
@@ -415,7 +471,7 @@ def main():
                        "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "tile": 16,
                        "parallelism": f"independent batch per rank x{world}",
                        "l2": f"inputs larger than L2 ({bytes_step / 1e6:.0f} MB per step > 126 MB); no flush"},
-            "roofline": roofline, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roofline, "decode": decode, "speculative": spec, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": launches, "clocks": clk, "kernel_src": src_hash,
         }
         print(json.dumps(line))

@@ -142,14 +142,48 @@ KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v, 
                            void *out, kda_dtype out_dtype, int32_t N, int32_t H, int32_t d_k,
                            int32_t d_v, float scale, void *stream);
 
+/*
+ * Multi-token decode with rollback (speculative decoding).  The pages state only that KDA's
+ * recurrent state needs rollback handling after rejected proposals ("K3 Architecture
+ * Illustrated", "Speculative decoding changes the value of extra computation"); these two calls
+ * are the plainest reading: verify K proposed tokens, then keep the state of the accepted prefix.
+ *
+ * kda_decode_verify — runs tokens 1..K of each of N sequences from its current state, exactly as K
+ * calls of kda_decode_step would, but does not write the state.  For every token it writes the
+ * output and the write vector u_t = beta_t (v_t - (Diag(alpha_t) S_{t-1})^T k_t).
+ *   q, k, a     bf16 [N, K, H, d_k]      v, gate bf16 [N, K, H, d_v] (gate may be NULL)
+ *   beta        fp32 [N, K, H]           A_log fp32 [H]
+ *   state       fp32 [N, H, d_k, d_v]    read only
+ *   u           fp32 [N, H, K, d_v]      written (consumed by kda_decode_commit)
+ *   out         [N, K, H, d_v] of out_dtype
+ * 1 <= K <= 16.  The caller owns every buffer.
+ */
+KDA_API kda_status kda_decode_verify(const void *q, const void *k, const void *v, const void *a,
+                                     const float *beta, const void *gate, const float *A_log,
+                                     const float *state, float *u, void *out, kda_dtype out_dtype,
+                                     int32_t N, int32_t K, int32_t H, int32_t d_k, int32_t d_v,
+                                     float scale, void *stream);
+
+/*
+ * kda_decode_commit — advances state n by its first accepted[n] verified tokens:
+ *   S <- Diag(alpha_t) S + k_t u_t^T  for t = 1 .. accepted[n]
+ * with the same k, a, A_log and K as the verify call and its u.  accepted (int32 [N], device)
+ * must lie in [0, K]; 0 leaves a state untouched.  A count outside [0, K] is clamped and reported
+ * through the error word (kda_sync_check returns KDA_ERR_INVALID_ARG).
+ */
+KDA_API kda_status kda_decode_commit(const void *k, const void *a, const float *A_log,
+                                     const int32_t *accepted, const float *u, float *state,
+                                     int32_t N, int32_t K, int32_t H, int32_t d_k, int32_t d_v,
+                                     void *stream);
+
 /* Static description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error word.  Returns
  * KDA_ERR_CUDA if the stream reported a CUDA error, KDA_ERR_INVALID_ARG if a kernel found
- * malformed cu_seqlens or a sequence longer than max_seqlen, KDA_ERR_TIMEOUT if a bounded wait
- * gave up, else KDA_OK.
+ * malformed cu_seqlens, a sequence longer than max_seqlen or an accepted count outside [0, K],
+ * KDA_ERR_TIMEOUT if a bounded wait gave up, else KDA_OK.
  */
 KDA_API kda_status kda_sync_check(void *stream);
 

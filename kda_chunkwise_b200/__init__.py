@@ -7,6 +7,7 @@ no CPU or PyTorch fallback: importing this package without the built library rai
 Entry points (same names as the C ABI):
   kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, ...)  prefill, chunkwise form
   kda_decode_step(q, k, v, a, beta, A_log, state, ...)      one recurrent step, state in place
+  kda_decode_verify / kda_decode_commit                     K proposed tokens, then the accepted prefix
 """
 from __future__ import annotations
 
@@ -18,6 +19,7 @@ import torch
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_chunk_fwd_workspace_min", "kda_sync_check", "kda_status_string", "KDAError",
            "kda_launch_count", "kda_chunk_fwd_noalloc", "kda_inject_stall",
+           "kda_decode_verify", "kda_decode_commit",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -62,6 +64,11 @@ def _load() -> ctypes.CDLL:
     L.kda_last_error.restype = ctypes.c_char_p
     L.kda_launch_count.argtypes = []
     L.kda_launch_count.restype = ctypes.c_uint64
+    L.kda_decode_verify.argtypes = [vp, vp, vp, vp, fp, vp, fp, fp, fp, vp, ctypes.c_int, i32, i32, i32,
+                                    i32, i32, f32, vp]
+    L.kda_decode_verify.restype = ctypes.c_int
+    L.kda_decode_commit.argtypes = [vp, vp, fp, vp, fp, fp, i32, i32, i32, i32, i32, vp]
+    L.kda_decode_commit.restype = ctypes.c_int
     L.kda_inject_stall.argtypes = [i32, ctypes.c_uint64]
     L.kda_inject_stall.restype = ctypes.c_int
     return L
@@ -228,6 +235,58 @@ def kda_decode_step(q, k, v, a, beta, A_log, state, gate=None, scale: float = 1.
                              _stream_handle(stream, dev))
     _check(st, "kda_decode_step")
     return out
+
+
+def kda_decode_verify(q, k, v, a, beta, A_log, state, gate=None, scale: float = 1.0, u=None, out=None,
+                      stream=None, out_dtype=torch.bfloat16):
+    """Run K proposed tokens of N sequences from ``state`` without changing it.
+
+    q, k, a [N, K, H, d_k] bf16; v, gate [N, K, H, d_v] bf16; beta [N, K, H] fp32; A_log [H];
+    state [N, H, d_k, d_v] fp32 (read only).  Returns (out [N, K, H, d_v], u [N, H, K, d_v] fp32);
+    pass u to kda_decode_commit.
+    """
+    dev = q.device
+    N, K, H, d_k = q.shape
+    d_v = v.shape[-1]
+    bf = torch.bfloat16
+    for name, t, shp in (("q", q, (N, K, H, d_k)), ("k", k, (N, K, H, d_k)), ("a", a, (N, K, H, d_k)),
+                         ("v", v, (N, K, H, d_v))):
+        _need(t, name, bf, shp, dev)
+    _need(beta, "beta", torch.float32, (N, K, H), dev)
+    _need(A_log, "A_log", torch.float32, (H,), dev)
+    _need(state, "state", torch.float32, (N, H, d_k, d_v), dev)
+    if gate is not None:
+        _need(gate, "gate", bf, (N, K, H, d_v), dev)
+    if u is None:
+        u = torch.empty((N, H, K, d_v), dtype=torch.float32, device=dev)
+    _need(u, "u", torch.float32, (N, H, K, d_v), dev)
+    if out is None:
+        out = torch.empty((N, K, H, d_v), dtype=out_dtype, device=dev)
+    if out.dtype not in _OUT_DTYPES:
+        raise TypeError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, (N, K, H, d_v), dev)
+    st = lib.kda_decode_verify(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate), _ptr(A_log),
+                               _ptr(state), _ptr(u), _ptr(out), _OUT_DTYPES[out.dtype], N, K, H, d_k, d_v,
+                               float(scale), _stream_handle(stream, dev))
+    _check(st, "kda_decode_verify")
+    return out, u
+
+
+def kda_decode_commit(k, a, A_log, accepted, u, state, stream=None):
+    """Advance each state by its accepted[n] verified tokens (int32 [N] on the device); in place."""
+    dev = k.device
+    N, K, H, d_k = k.shape
+    d_v = u.shape[-1]
+    _need(k, "k", torch.bfloat16, (N, K, H, d_k), dev)
+    _need(a, "a", torch.bfloat16, (N, K, H, d_k), dev)
+    _need(A_log, "A_log", torch.float32, (H,), dev)
+    _need(accepted, "accepted", torch.int32, (N,), dev)
+    _need(u, "u", torch.float32, (N, H, K, d_v), dev)
+    _need(state, "state", torch.float32, (N, H, d_k, d_v), dev)
+    st = lib.kda_decode_commit(_ptr(k), _ptr(a), _ptr(A_log), _ptr(accepted), _ptr(u), _ptr(state),
+                               N, K, H, d_k, d_v, _stream_handle(stream, dev))
+    _check(st, "kda_decode_commit")
+    return state
 
 
 def kda_launch_count() -> int:

@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_fused.cuh"
+#include "speculative.cuh"
 
 namespace {
 
@@ -87,6 +88,22 @@ kda_status launch_decode(const kda::DecodeParams &p, int64_t units, cudaStream_t
     g_launches.fetch_add(1, std::memory_order_relaxed);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "decode_step launch");
+}
+
+template <int DK, int DV>
+kda_status launch_spec(const kda::SpecParams &p, int64_t units, bool commit, cudaStream_t stream) {
+    if (commit) kda::spec_commit_kernel<DK, DV><<<(unsigned)units, 256, 0, stream>>>(p);
+    else kda::spec_verify_kernel<DK, DV><<<(unsigned)units, 256, 0, stream>>>(p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, commit ? "decode_commit launch" : "decode_verify launch");
+}
+
+kda_status dispatch_spec(const kda::SpecParams &p, int64_t units, int d_k, int d_v, bool commit, cudaStream_t st) {
+    if (d_k == 128 && d_v == 128) return launch_spec<128, 128>(p, units, commit, st);
+    if (d_k == 128 && d_v == 64) return launch_spec<128, 64>(p, units, commit, st);
+    if (d_k == 64 && d_v == 128) return launch_spec<64, 128>(p, units, commit, st);
+    return launch_spec<64, 64>(p, units, commit, st);
 }
 
 // Built-in scratch for kda_chunk_fwd_noalloc (callers that cannot allocate).  Host code must not
@@ -290,6 +307,76 @@ kda_status kda_inject_stall(int32_t enable, uint64_t wait_limit_ns) {
     return KDA_OK;
 }
 
+kda_status kda_decode_verify(const void *q, const void *k, const void *v, const void *a, const float *beta,
+                             const void *gate, const float *A_log, const float *state, float *u, void *out,
+                             kda_dtype out_dtype, int32_t N, int32_t K, int32_t H, int32_t d_k, int32_t d_v,
+                             float scale, void *stream) {
+    if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_decode_verify: N < 0 or H <= 0");
+    if (K < 1 || K > kda::kSpecMaxTokens)
+        return fail(KDA_ERR_INVALID_ARG, "kda_decode_verify: K must be in [1, 16]");
+    if (!supported_dim(d_k) || !supported_dim(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_decode_verify: d_k and d_v must be 64 or 128");
+    if (N == 0) return KDA_OK;
+    if (!q || !k || !v || !a || !beta || !A_log || !state || !u || !out)
+        return fail(KDA_ERR_INVALID_ARG, "kda_decode_verify: NULL required pointer");
+    if (out_dtype != KDA_DTYPE_BF16 && out_dtype != KDA_DTYPE_F32)
+        return fail(KDA_ERR_INVALID_ARG, "kda_decode_verify: out_dtype must be KDA_DTYPE_BF16 or KDA_DTYPE_F32");
+    const void *ptrs[] = {q, k, v, a, gate, state, u, out};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned(ptr, 16)) return fail(KDA_ERR_INVALID_ARG, "kda_decode_verify: tensor pointer not 16-byte aligned");
+    const void *ptrs4[] = {beta, A_log};
+    for (const void *ptr : ptrs4)
+        if (!aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_decode_verify: beta/A_log not 4-byte aligned");
+    const int64_t units = (int64_t)N * H;
+    if (units > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_decode_verify: N*H too large");
+    kda::SpecParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.a = static_cast<const uint16_t *>(a);
+    p.gate = static_cast<const uint16_t *>(gate);
+    p.beta = beta;
+    p.A_log = A_log;
+    p.state = const_cast<float *>(state);   // read only by the verify kernel
+    p.u = u;
+    p.out = out;
+    p.H = H;
+    p.K = K;
+    p.out_f32 = out_dtype == KDA_DTYPE_F32;
+    p.scale = scale;
+    return dispatch_spec(p, units, d_k, d_v, false, static_cast<cudaStream_t>(stream));
+}
+
+kda_status kda_decode_commit(const void *k, const void *a, const float *A_log, const int32_t *accepted,
+                             const float *u, float *state, int32_t N, int32_t K, int32_t H, int32_t d_k,
+                             int32_t d_v, void *stream) {
+    if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_decode_commit: N < 0 or H <= 0");
+    if (K < 1 || K > kda::kSpecMaxTokens)
+        return fail(KDA_ERR_INVALID_ARG, "kda_decode_commit: K must be in [1, 16]");
+    if (!supported_dim(d_k) || !supported_dim(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_decode_commit: d_k and d_v must be 64 or 128");
+    if (N == 0) return KDA_OK;
+    if (!k || !a || !A_log || !accepted || !u || !state)
+        return fail(KDA_ERR_INVALID_ARG, "kda_decode_commit: NULL required pointer");
+    const void *ptrs[] = {k, a, u, state};
+    for (const void *ptr : ptrs)
+        if (!aligned(ptr, 16)) return fail(KDA_ERR_INVALID_ARG, "kda_decode_commit: tensor pointer not 16-byte aligned");
+    if (!aligned(A_log, 4) || !aligned(accepted, 4))
+        return fail(KDA_ERR_INVALID_ARG, "kda_decode_commit: A_log/accepted not 4-byte aligned");
+    const int64_t units = (int64_t)N * H;
+    if (units > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_decode_commit: N*H too large");
+    kda::SpecParams p{};
+    p.k = static_cast<const uint16_t *>(k);
+    p.a = static_cast<const uint16_t *>(a);
+    p.A_log = A_log;
+    p.accepted = accepted;
+    p.u = const_cast<float *>(u);   // read only by the commit kernel
+    p.state = state;
+    p.H = H;
+    p.K = K;
+    return dispatch_spec(p, units, d_k, d_v, true, static_cast<cudaStream_t>(stream));
+}
+
 kda_status kda_sync_check(void *stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kda_sync_check: stream");
@@ -306,6 +393,8 @@ kda_status kda_sync_check(void *stream) {
         return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not monotone from 0 to total_tokens");
     if (word & kda::kErrSeqTooLong)
         return fail(KDA_ERR_INVALID_ARG, "a sequence is longer than max_seqlen");
+    if (word & kda::kErrBadAccepted)
+        return fail(KDA_ERR_INVALID_ARG, "an accepted count is outside [0, K] (it was clamped)");
     return KDA_OK;
 }
 

@@ -87,6 +87,26 @@ class DecodeWorkload:
 DECODE = DecodeWorkload()
 
 
+@dataclasses.dataclass(frozen=True)
+class SpecWorkload:
+    """Speculative decode: K proposed tokens per sequence per round, then an accepted prefix.
+
+    The shapes are the decode configuration's (256 sequences x 64 heads, 128 x 128 states); K = 4
+    proposals per round, and each sequence accepts a prefix of length ~ U{0..K} (the pages give no
+    acceptance rate; uniform is the plainest stand-in)."""
+    name: str = "spec_N256_H64_d128_K4"
+    N: int = 256
+    H: int = 64
+    d_k: int = 128
+    d_v: int = 128
+    K: int = 4
+    rounds: int = 64
+    seed: int = 0
+
+
+SPEC = SpecWorkload()
+
+
 def _gen(device, seed):
     return torch.Generator(device=torch.device(device)).manual_seed(int(seed))
 
@@ -166,3 +186,23 @@ def make_decode_inputs(w: DecodeWorkload, device="cpu", steps: int | None = None
     gate = _normal_rows(steps * N, H, w.d_v, g, device).view(steps, N, H, w.d_v)
     A_log = torch.zeros((H,), device=device)
     return dict(q=q, k=k, v=v, a=a, beta=beta, gate=gate, A_log=A_log, state=state, workload=w)
+
+
+def make_spec_inputs(w: SpecWorkload, device="cpu", rounds: int | None = None) -> dict:
+    """Per-round inputs [rounds, N, K, H, d], accepted counts [rounds, N] (int32, U{0..K}) and the
+    starting states [N, H, d_k, d_v]; inputs follow the decode recipe."""
+    rounds = w.rounds if rounds is None else rounds
+    g = _gen(device, w.seed)
+    N, H, K = w.N, w.H, w.K
+    rows = rounds * N * K
+    state = torch.randn((N, H, w.d_k, w.d_v), generator=g, device=device) * 0.02
+    q = _unit_rows(rows, H, w.d_k, g, device).view(rounds, N, K, H, w.d_k)
+    k = _unit_rows(rows, H, w.d_k, g, device).view(rounds, N, K, H, w.d_k)
+    v = _normal_rows(rows, H, w.d_v, g, device).view(rounds, N, K, H, w.d_v)
+    a = _normal_rows(rows, H, w.d_k, g, device).view(rounds, N, K, H, w.d_k)
+    beta = _beta(rows, H, "sigmoid_normal", g, device).view(rounds, N, K, H)
+    gate = _normal_rows(rows, H, w.d_v, g, device).view(rounds, N, K, H, w.d_v)
+    accepted = torch.randint(0, K + 1, (rounds, N), generator=g, device=device, dtype=torch.int32)
+    A_log = torch.zeros((H,), device=device)
+    return dict(q=q, k=k, v=v, a=a, beta=beta, gate=gate, A_log=A_log, state=state, accepted=accepted,
+                workload=w)

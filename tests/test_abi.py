@@ -107,3 +107,26 @@ def test_inject_stall_validates_its_limit_on_the_host():
     assert lib.kda_inject_stall(0, 0) == kda.KDA_OK
     with pytest.raises(kda.KDAError):
         kda.kda_inject_stall(True, 0)
+
+
+def test_verify_and_commit_reject_bad_arguments():
+    V, C = lib.kda_decode_verify, lib.kda_decode_commit
+    ok = dict(q=16, k=16, v=16, a=16, beta=16, gate=None, A_log=16, state=16, u=16, out=16, dt=0, N=2, K=4,
+              H=2, dk=128, dv=128)
+
+    def ver(**o):
+        a = dict(ok, **o)
+        return V(a["q"], a["k"], a["v"], a["a"], a["beta"], a["gate"], a["A_log"], a["state"], a["u"], a["out"],
+                 a["dt"], a["N"], a["K"], a["H"], a["dk"], a["dv"], 1.0, None)
+
+    assert ver(K=0) == kda.KDA_ERR_INVALID_ARG
+    assert ver(K=17) == kda.KDA_ERR_INVALID_ARG
+    assert ver(dv=96) == kda.KDA_ERR_UNSUPPORTED
+    assert ver(u=None) == kda.KDA_ERR_INVALID_ARG
+    assert ver(q=8) == kda.KDA_ERR_INVALID_ARG          # misaligned
+    assert ver(dt=5) == kda.KDA_ERR_INVALID_ARG
+    assert ver(N=0) == kda.KDA_OK
+    assert C(16, 16, 16, 16, 16, 16, 2, 0, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG       # K = 0
+    assert C(16, 16, 16, None, 16, 16, 2, 4, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG     # accepted
+    assert C(16, 16, 16, 18, 16, 16, 2, 4, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG       # alignment
+    assert C(16, 16, 16, 16, 16, 16, 0, 4, 2, 128, 128, None) == kda.KDA_OK
