@@ -47,6 +47,7 @@ def parse_args():
     p.add_argument("--impl", default="kda", choices=["kda", "reference"])
     p.add_argument("--workload", default="prefill_B1_H32_T8192_d128")
     p.add_argument("--decode-steps", type=int, default=512)
+    p.add_argument("--spec-rounds", type=int, default=64)
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -382,7 +383,7 @@ def main():
     # speculative decode row: rounds of verify (K proposed tokens) + commit (accepted prefixes)
     spec = None
     if not args.no_decode:
-        sw = dataclasses.replace(KI.SPEC, seed=KI.SPEC.seed + rank)
+        sw = dataclasses.replace(KI.SPEC, seed=KI.SPEC.seed + rank, rounds=args.spec_rounds)
         d = KI.make_spec_inputs(sw, dev)
         state = d["state"].clone()
         sout = torch.empty((sw.N, sw.K, sw.H, sw.d_v), dtype=torch.bfloat16, device=dev)

@@ -35,9 +35,11 @@ __device__ __forceinline__ float4 f4_fma(float s, float4 x, float4 acc) {
     return acc;
 }
 
+constexpr int kDecodeThreads = 256;
+
 template <int DK, int DV>
-__global__ void __launch_bounds__(256) decode_step_kernel(const DecodeParams p) {
-    constexpr int kThreads = 256;
+__global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const DecodeParams p) {
+    constexpr int kThreads = kDecodeThreads;
     constexpr int LPR = DV / 4;          // threads per state row, one float4 each
     constexpr int RPP = kThreads / LPR;  // rows covered by the block in one pass
     constexpr int NR = DK / RPP;         // rows held per thread

@@ -84,7 +84,7 @@ kda_status launch_prefill(const kda::FusedParams &p, int64_t units, cudaStream_t
 
 template <int DK, int DV>
 kda_status launch_decode(const kda::DecodeParams &p, int64_t units, cudaStream_t stream) {
-    kda::decode_step_kernel<DK, DV><<<(unsigned)units, 256, 0, stream>>>(p);
+    kda::decode_step_kernel<DK, DV><<<(unsigned)units, kda::kDecodeThreads, 0, stream>>>(p);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "decode_step launch");
@@ -92,8 +92,8 @@ kda_status launch_decode(const kda::DecodeParams &p, int64_t units, cudaStream_t
 
 template <int DK, int DV>
 kda_status launch_spec(const kda::SpecParams &p, int64_t units, bool commit, cudaStream_t stream) {
-    if (commit) kda::spec_commit_kernel<DK, DV><<<(unsigned)units, 256, 0, stream>>>(p);
-    else kda::spec_verify_kernel<DK, DV><<<(unsigned)units, 256, 0, stream>>>(p);
+    if (commit) kda::spec_commit_kernel<DK, DV><<<(unsigned)units, kda::kSpecThreads, 0, stream>>>(p);
+    else kda::spec_verify_kernel<DK, DV><<<(unsigned)units, kda::kSpecThreads, 0, stream>>>(p);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, commit ? "decode_commit launch" : "decode_verify launch");
