@@ -36,7 +36,16 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 # DRAM traffic of the dominant kernel per launch, from an ncu capture (profiles/); it is
 # reported only while the kernel sources still hash to the value they had when captured.
-NCU_TRAFFIC = {}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture of each
+# kernel (profiles/ gives the commands), keyed by workload, with the hash of the kernel's sources at
+# capture time.  Reported only while the sources are unchanged.
+NCU_TRAFFIC = {
+    "prefill_B1_H32_T8192_d128": {"bytes_per_launch": 396773376, "src": "ca3932fc27f6ad64"},
+    "decode_N256_H64_d128_512steps": {"bytes_per_launch": 2114315008, "src": "1c3a7d12c8610c04"},
+    # one verify launch plus one commit launch (round 4 of the captured run; commit's bytes depend on
+    # how many sequences accepted at least one token)
+    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1182260224 + 1765504000, "src": "089cfaaf3b46dbfe"},
+}
 
 
 def parse_args():
@@ -101,13 +110,29 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+# source files each kernel is built from (a DRAM traffic figure is reported only while they are
+# unchanged since the ncu capture it came from)
+KERNEL_SOURCES = {
+    "prefill": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh"),
+    "decode": ("common.cuh", "decode.cuh"),
+    "speculative": ("common.cuh", "decode.cuh", "speculative.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str | None = None) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kda_chunkwise_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES[kernel] if kernel else sorted(os.listdir(csrc))
+    for name in names:
         if name.endswith((".cu", ".cuh")):
             h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
+
+
+def ncu_traffic(key: str, kernel: str):
+    """DRAM bytes (read + write) per launch from the committed ncu capture, if still current."""
+    t = NCU_TRAFFIC.get(key)
+    return t["bytes_per_launch"] if t and t.get("src") == kernel_source_hash(kernel) else None
 
 
 # ---- multi-rank plumbing (no data-path collective: every rank runs its own batch) --------------
@@ -334,8 +359,7 @@ def main():
     flops_step = prefill_flops(w)
     achieved = bytes_step / (ms * 1e-3) / 1e9
     src_hash = kernel_source_hash()
-    traffic = NCU_TRAFFIC.get(w.name)
-    traffic_val = traffic["bytes_per_launch"] if traffic and traffic.get("src") == src_hash else None
+    traffic_val = ncu_traffic(w.name, "prefill")
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic_val,
                 "peak_source": f"hbm_gbs of {peak_src}",
@@ -374,7 +398,7 @@ def main():
         decode = {"value": whole_job_rate(1, world, dms), "unit": "steps/s", "ms_per_step": dms,
                   "workload": dw.name, "tokens_per_s": whole_job_rate(dw.N, world, dms),
                   "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
-                               "frac": dach / hbm, "traffic": None,
+                               "frac": dach / hbm, "traffic": ncu_traffic(dw.name, "decode"),
                                "peak_source": f"hbm_gbs of {peak_src}",
                                "algorithmic_bytes": dbytes}}
         del d, state, dout
@@ -416,7 +440,8 @@ def main():
                 "ms_per_round": sms, "workload": sw.name, "proposed_per_round": sw.N * sw.K,
                 "accepted_per_round": accepted_per_round,
                 "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s",
-                             "frac": sach / hbm, "traffic": None, "peak_source": f"hbm_gbs of {peak_src}",
+                             "frac": sach / hbm, "traffic": ncu_traffic(sw.name, "speculative"),
+                             "peak_source": f"hbm_gbs of {peak_src}",
                              "algorithmic_bytes": int(sbytes),
                              "scope": "one round = kda_decode_verify + kda_decode_commit"}}
         del d, state, sout, su
