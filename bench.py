@@ -491,7 +491,10 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            # tensor-core operands are bf16 (Gram blocks, split hi + lo for Q K^T) and fp16 (value
+            # path); accumulation, the decay arithmetic and the carried state are fp32
+            "dtype": "bf16/fp16 mma, f32 accumulate",
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.num_seqs, "H": w.H, "T": w.total_tokens,
                        "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "tile": 16,
