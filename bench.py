@@ -5,7 +5,9 @@
 
 One step = one kda_chunk_fwd call over the prefill workload (B=1, H=32, T=8192, d=128; inputs
 resident in HBM).  The decode row (kda_decode_step over 256 sequences x 64 heads, 128x128 fp32
-states, 512 steps) is timed in the same run and reported under "decode".  Every rank runs its own
+states, 512 steps) is timed in the same run and reported under "decode", and rounds of speculative
+decode (kda_decode_verify of 4 proposed tokens + kda_decode_commit of the accepted prefix, same
+states) under "speculative".  Every rank runs its own
 independent batch (weak scaling, no collective on the data path); timing is on the device with
 CUDA events, max over ranks.  Rank 0 prints one JSON line.
 
@@ -34,8 +36,6 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM traffic of the dominant kernel per launch, from an ncu capture (profiles/); it is
-# reported only while the kernel sources still hash to the value they had when captured.
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture of each
 # kernel (profiles/ gives the commands), keyed by workload, with the hash of the kernel's sources at
 # capture time.  Reported only while the sources are unchanged.
