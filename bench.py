@@ -40,7 +40,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # kernel (profiles/ gives the commands), keyed by workload, with the hash of the kernel's sources at
 # capture time.  Reported only while the sources are unchanged.
 NCU_TRAFFIC = {
-    "prefill_B1_H32_T8192_d128": {"bytes_per_launch": 396773376, "src": "ca3932fc27f6ad64"},
+    "prefill_B1_H32_T8192_d128": {"bytes_per_launch": 396773376, "src": "ce2389bee8082413"},
     "decode_N256_H64_d128_512steps": {"bytes_per_launch": 2114315008, "src": "1c3a7d12c8610c04"},
     # one verify launch plus one commit launch (round 4 of the captured run; commit's bytes depend on
     # how many sequences accepted at least one token)

@@ -69,25 +69,6 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], u
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// tf32 MMA m16n8k8, fp32 accumulate.  Fragments (g = lane / 4, t = lane % 4):
-//   A (16x8): a[0] = (g, t)  a[1] = (g+8, t)  a[2] = (g, t+4)  a[3] = (g+8, t+4)
-//   B (8x8):  b[0] = (k t, n g)  b[1] = (k t+4, n g)
-// ldmatrix.x4 on an fp32 matrix viewed as 16-bit pairs yields exactly the A fragment.
-__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// fp32 -> tf32 (10 explicit mantissa bits), round to nearest, ties away from zero
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t y;
-    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(y) : "f"(x));
-    return y;
-}
-
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -167,42 +148,10 @@ __device__ __forceinline__ void st_u32(void *p, uint32_t x) {
     asm volatile("st.global.u32 [%0], %1;\n" ::"l"(p), "r"(x) : "memory");
 }
 
-__device__ __forceinline__ void stg_v2(void *p, uint32_t x, uint32_t y) {
-    asm volatile("st.global.v2.u32 [%0], {%1,%2};\n" ::"l"(p), "r"(x), "r"(y) : "memory");
-}
-
 __device__ __forceinline__ void stg_v4(void *p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                  "r"(v.w)
                  : "memory");
-}
-
-__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Relaxed read (no ordering); pair with fence_acquire_gpu() once the value is known to suffice.
-__device__ __forceinline__ int ld_relaxed_gpu(const int *p) {
-    int v;
-    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
-
-__device__ __forceinline__ void st_release_gpu(int *p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
-}
-
-// Relaxed add: used to return a ring slot once every value read from it has been consumed.
-__device__ __forceinline__ void red_relaxed_add_gpu(int *p, int v) {
-    asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void red_release_add_gpu(int *p, int v) {
-    asm volatile("red.release.gpu.global.add.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
 }
 
 // 16-byte asynchronous global->shared copy; bytes beyond src_bytes (0 or 16) are zero-filled.
@@ -244,19 +193,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 // Arrive (relaxed, cluster scope): for a hand-back after which nothing written needs ordering.
 __device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
-}
-
-// One non-blocking test (acquire, cluster scope) of whether the phase with parity `parity` of a
-// local mbarrier has completed.
-__device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-        "selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    return ok != 0;
 }
 
 // Wait (acquire, cluster scope) for the phase with parity `parity` of a local mbarrier, letting the
