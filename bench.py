@@ -367,6 +367,44 @@ def main():
                 "algorithmic_bytes": bytes_step, "algorithmic_flops": flops_step,
                 "tensor_frac_of_bf16_peak": flops_step / (ms * 1e-3) / 1e12 / tf}
 
+    # module row: the short convolution of q, k, v (q, k L2-normalised) and the pre-gate
+    # normalisation + gate of one fp32 output, on the prefill workload's tensors
+    module = None
+    if not args.no_decode:
+        gm = torch.Generator(device=dev).manual_seed(101 + rank)
+        cw = torch.randn((w.H, w.d_k, 4), generator=gm, device=dev) * 0.5
+        nw = torch.rand((w.d_v,), generator=gm, device=dev) + 0.5
+        o32 = torch.randn((w.total_tokens, w.H, w.d_v), generator=gm, device=dev)
+        yq, yk, yv = (torch.empty_like(inp[key]) for key in ("q", "k", "v"))
+
+        def mstep():
+            kda.kda_short_conv(inp["q"], cw, inp["cu_seqlens"], l2norm=True, out=yq, stream=stream)
+            kda.kda_short_conv(inp["k"], cw, inp["cu_seqlens"], l2norm=True, out=yk, stream=stream)
+            kda.kda_short_conv(inp["v"], cw, inp["cu_seqlens"], l2norm=False, out=yv, stream=stream)
+            kda.kda_output_norm_gate(o32, inp["gate"], nw, out=out, stream=stream)
+
+        for _ in range(max(3, args.warmup)):
+            mstep()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            mstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        kda.kda_sync_check()
+        mms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+        th = w.total_tokens * w.H
+        mbytes = 3 * 2 * th * w.d_k * 2 + th * w.d_v * (4 + 2 + 2)   # conv read + write x3; o, gate, out
+        mach = mbytes / (mms * 1e-3) / 1e9
+        module = {"value": whole_job_rate(w.total_tokens, world, mms), "unit": "tokens/s", "ms_per_step": mms,
+                  "workload": w.name, "scope": "3 kda_short_conv (width 4) + 1 kda_output_norm_gate",
+                  "roofline": {"bound": "hbm", "achieved": mach, "peak": hbm, "unit": "GB/s",
+                               "frac": mach / hbm, "traffic": None, "peak_source": f"hbm_gbs of {peak_src}",
+                               "algorithmic_bytes": mbytes}}
+        del o32, yq, yk, yv
+        torch.cuda.empty_cache()
+
     # decode row: 512 back-to-back steps over fixed states (each step reads and writes 1.07 GB)
     decode = None
     if not args.no_decode:
@@ -500,7 +538,7 @@ def main():
                        "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "tile": 16,
                        "parallelism": f"independent batch per rank x{world}",
                        "l2": f"inputs larger than L2 ({bytes_step / 1e6:.0f} MB per step > 126 MB); no flush"},
-            "roofline": roofline, "decode": decode, "speculative": spec, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roofline, "module": module, "decode": decode, "speculative": spec, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": launches, "clocks": clk, "kernel_src": src_hash,
         }
         print(json.dumps(line))

@@ -176,6 +176,36 @@ KDA_API kda_status kda_decode_commit(const void *k, const void *a, const float *
                                      int32_t N, int32_t K, int32_t H, int32_t d_k, int32_t d_v,
                                      void *stream);
 
+/*
+ * The module pieces around the recurrence.  The pages say only that the actual KDA module also has
+ * short convolution, normalisation and output gating ("K3 Architecture Illustrated", FIG 21) and
+ * that short convolution depends on input order (§"Why can K3's MLA use NoPE?"); the forms below
+ * are the plainest readings.
+ *
+ * kda_short_conv — causal depthwise convolution over time, per sequence of the packed batch:
+ *   y_t[h][c] = sum_{j < width} w[h][c][j] * x_{t-(width-1)+j}[h][c]     (x before a sequence = 0)
+ * optionally followed (l2norm != 0) by y_t[h] <- y_t[h] / sqrt(|y_t[h]|^2 + 1e-12).
+ *   x, y  bf16 [total_tokens, H, d] (d = 64 or 128; y may not alias x)
+ *   w     fp32 [H, d, width], 1 <= width <= 4
+ *   cu_seqlens int32 [num_seqs + 1] (device), as for kda_chunk_fwd.  At most 2,097,120 tokens.
+ * Malformed cu_seqlens are reported through the error word.
+ */
+KDA_API kda_status kda_short_conv(const void *x, const float *w, const int32_t *cu_seqlens, int32_t num_seqs,
+                                  int64_t total_tokens, int32_t H, int32_t d, int32_t width, int32_t l2norm,
+                                  void *y, void *stream);
+
+/*
+ * kda_output_norm_gate — pre-gate RMS normalisation of every (token, head) output row, then the
+ * sigmoid output gate:  out = sigmoid(gate) * o / sqrt(mean_c(o^2) + eps) * w.
+ *   o     fp32 [total_tokens, H, d_v] (e.g. kda_chunk_fwd with gate = NULL and fp32 output)
+ *   gate  bf16 [total_tokens, H, d_v] or NULL (no gate)
+ *   w     fp32 [d_v] per-channel gain, shared by the heads
+ *   out   [total_tokens, H, d_v] of out_dtype
+ */
+KDA_API kda_status kda_output_norm_gate(const float *o, const void *gate, const float *w, int64_t total_tokens,
+                                        int32_t H, int32_t d_v, float eps, void *out, kda_dtype out_dtype,
+                                        void *stream);
+
 /* Static description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);
 

@@ -8,6 +8,8 @@ Entry points (same names as the C ABI):
   kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, ...)  prefill, chunkwise form
   kda_decode_step(q, k, v, a, beta, A_log, state, ...)      one recurrent step, state in place
   kda_decode_verify / kda_decode_commit                     K proposed tokens, then the accepted prefix
+  kda_short_conv, kda_output_norm_gate                      the module's short convolution and
+                                                            pre-gate normalisation + output gate
 """
 from __future__ import annotations
 
@@ -19,7 +21,7 @@ import torch
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_chunk_fwd_workspace_min", "kda_sync_check", "kda_status_string", "KDAError",
            "kda_launch_count", "kda_chunk_fwd_noalloc", "kda_inject_stall",
-           "kda_decode_verify", "kda_decode_commit",
+           "kda_decode_verify", "kda_decode_commit", "kda_short_conv", "kda_output_norm_gate",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -69,6 +71,10 @@ def _load() -> ctypes.CDLL:
     L.kda_decode_verify.restype = ctypes.c_int
     L.kda_decode_commit.argtypes = [vp, vp, fp, vp, fp, fp, i32, i32, i32, i32, i32, vp]
     L.kda_decode_commit.restype = ctypes.c_int
+    L.kda_short_conv.argtypes = [vp, fp, vp, i32, i64, i32, i32, i32, i32, vp, vp]
+    L.kda_short_conv.restype = ctypes.c_int
+    L.kda_output_norm_gate.argtypes = [fp, vp, fp, i64, i32, i32, f32, vp, ctypes.c_int, vp]
+    L.kda_output_norm_gate.restype = ctypes.c_int
     L.kda_inject_stall.argtypes = [i32, ctypes.c_uint64]
     L.kda_inject_stall.restype = ctypes.c_int
     return L
@@ -287,6 +293,45 @@ def kda_decode_commit(k, a, A_log, accepted, u, state, stream=None):
                                N, K, H, d_k, d_v, _stream_handle(stream, dev))
     _check(st, "kda_decode_commit")
     return state
+
+
+def kda_short_conv(x, w, cu_seqlens, l2norm: bool = False, out=None, stream=None):
+    """Causal depthwise convolution over time per packed sequence (bf16 [T, H, d] in and out),
+    optionally L2-normalising every (token, head) row.  w: fp32 [H, d, width], width <= 4."""
+    dev = x.device
+    T, H, d = x.shape
+    width = w.shape[-1]
+    _need(x, "x", torch.bfloat16, (T, H, d), dev)
+    _need(w, "w", torch.float32, (H, d, width), dev)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev or cu_seqlens.dim() != 1:
+        raise TypeError("cu_seqlens must be int32 [num_seqs + 1] on the device")
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", torch.bfloat16, (T, H, d), dev)
+    st = lib.kda_short_conv(_ptr(x), _ptr(w), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, H, d, width,
+                            1 if l2norm else 0, _ptr(out), _stream_handle(stream, dev))
+    _check(st, "kda_short_conv")
+    return out
+
+
+def kda_output_norm_gate(o, gate, w, eps: float = 1e-6, out=None, stream=None, out_dtype=torch.bfloat16):
+    """out = sigmoid(gate) * RMSNorm(o) * w per (token, head) row; o fp32 [T, H, d_v], gate bf16 or
+    None, w fp32 [d_v]."""
+    dev = o.device
+    T, H, d_v = o.shape
+    _need(o, "o", torch.float32, (T, H, d_v), dev)
+    _need(w, "w", torch.float32, (d_v,), dev)
+    if gate is not None:
+        _need(gate, "gate", torch.bfloat16, (T, H, d_v), dev)
+    if out is None:
+        out = torch.empty((T, H, d_v), dtype=out_dtype, device=dev)
+    if out.dtype not in _OUT_DTYPES:
+        raise TypeError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, (T, H, d_v), dev)
+    st = lib.kda_output_norm_gate(_ptr(o), _ptr(gate), _ptr(w), T, H, d_v, float(eps), _ptr(out),
+                                  _OUT_DTYPES[out.dtype], _stream_handle(stream, dev))
+    _check(st, "kda_output_norm_gate")
+    return out
 
 
 def kda_launch_count() -> int:

@@ -14,6 +14,7 @@
 #include "decode.cuh"
 #include "prefill_fused.cuh"
 #include "speculative.cuh"
+#include "preprocess.cuh"
 
 namespace {
 
@@ -375,6 +376,70 @@ kda_status kda_decode_commit(const void *k, const void *a, const float *A_log, c
     p.H = H;
     p.K = K;
     return dispatch_spec(p, units, d_k, d_v, true, static_cast<cudaStream_t>(stream));
+}
+
+kda_status kda_short_conv(const void *x, const float *w, const int32_t *cu_seqlens, int32_t num_seqs,
+                          int64_t total_tokens, int32_t H, int32_t d, int32_t width, int32_t l2norm, void *y,
+                          void *stream) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0)
+        return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: negative size or H <= 0");
+    if (!supported_dim(d)) return fail(KDA_ERR_UNSUPPORTED, "kda_short_conv: d must be 64 or 128");
+    if (width < 1 || width > kda::kConvMaxWidth) return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: width must be in [1, 4]");
+    if (total_tokens == 0) return KDA_OK;
+    if (num_seqs == 0) return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: tokens without sequences");
+    if (!x || !w || !cu_seqlens || !y) return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: NULL required pointer");
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(w, 4) || !aligned(cu_seqlens, 4))
+        return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: misaligned pointer");
+    kda::ConvParams p{};
+    p.x = static_cast<const uint16_t *>(x);
+    p.w = w;
+    p.cu = cu_seqlens;
+    p.y = static_cast<uint16_t *>(y);
+    p.total_tokens = total_tokens;
+    p.num_seqs = num_seqs;
+    p.H = H;
+    p.width = width;
+    p.l2norm = l2norm != 0;
+    const int64_t runs = (total_tokens + kda::kConvRun - 1) / kda::kConvRun;
+    if (runs > 65535) return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: more than 2,097,120 tokens per call");
+    const int64_t groups = (int64_t)H * (d / 8);
+    const dim3 grid((unsigned)((groups + kda::kPrepThreads - 1) / kda::kPrepThreads), (unsigned)runs);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 128) kda::short_conv_kernel<128><<<grid, kda::kPrepThreads, 0, st>>>(p);
+    else kda::short_conv_kernel<64><<<grid, kda::kPrepThreads, 0, st>>>(p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "short_conv launch");
+}
+
+kda_status kda_output_norm_gate(const float *o, const void *gate, const float *w, int64_t total_tokens, int32_t H,
+                                int32_t d_v, float eps, void *out, kda_dtype out_dtype, void *stream) {
+    if (total_tokens < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_output_norm_gate: negative size or H <= 0");
+    if (!supported_dim(d_v)) return fail(KDA_ERR_UNSUPPORTED, "kda_output_norm_gate: d_v must be 64 or 128");
+    if (!(eps >= 0.f)) return fail(KDA_ERR_INVALID_ARG, "kda_output_norm_gate: eps must be >= 0");
+    if (out_dtype != KDA_DTYPE_BF16 && out_dtype != KDA_DTYPE_F32)
+        return fail(KDA_ERR_INVALID_ARG, "kda_output_norm_gate: out_dtype must be KDA_DTYPE_BF16 or KDA_DTYPE_F32");
+    if (total_tokens == 0) return KDA_OK;
+    if (!o || !w || !out) return fail(KDA_ERR_INVALID_ARG, "kda_output_norm_gate: NULL required pointer");
+    if (!aligned(o, 16) || !aligned(out, 16) || (gate && !aligned(gate, 16)) || !aligned(w, 4))
+        return fail(KDA_ERR_INVALID_ARG, "kda_output_norm_gate: misaligned pointer");
+    kda::NormGateParams p{};
+    p.o = o;
+    p.gate = static_cast<const uint16_t *>(gate);
+    p.w = w;
+    p.out = out;
+    p.rows = total_tokens * H;
+    p.eps = eps;
+    p.out_f32 = out_dtype == KDA_DTYPE_F32;
+    const int64_t threads = p.rows * (d_v / 8);
+    const int64_t blocks = (threads + kda::kPrepThreads - 1) / kda::kPrepThreads;
+    if (blocks > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_output_norm_gate: too many rows");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d_v == 128) kda::norm_gate_kernel<128><<<(unsigned)blocks, kda::kPrepThreads, 0, st>>>(p);
+    else kda::norm_gate_kernel<64><<<(unsigned)blocks, kda::kPrepThreads, 0, st>>>(p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "norm_gate launch");
 }
 
 kda_status kda_sync_check(void *stream) {

@@ -1,0 +1,204 @@
+// The two pieces of the KDA module around the recurrence that the pages name without giving their
+// form ("K3 Architecture Illustrated", FIG 21: the actual module also has short convolution,
+// normalisation and output gating; §"Why can K3's MLA use NoPE?": short convolution depends on
+// input order).  Plainest readings:
+//   short convolution: causal depthwise convolution over time within each sequence,
+//       y_t[c] = sum_{j < W} w[h][c][j] x_{t - (W-1) + j}[c]      (x before the sequence start = 0)
+//     with W <= 4 taps per channel, optionally followed by L2 normalisation of each (token, head)
+//     row (the recurrence expects unit q and k);
+//   pre-gate normalisation: RMS normalisation of each (token, head) output row with a per-channel
+//     gain, then the sigmoid output gate:  out = sigmoid(gate) (.) o / sqrt(mean(o^2) + eps) (.) w.
+// Both are HBM-bound streaming kernels: each thread owns 8 consecutive channels (a 16-byte piece of
+// a row), and the row reductions are shuffles among the d/8 lanes that hold one (token, head).
+#pragma once
+
+#include "common.cuh"
+
+namespace kda {
+
+constexpr int kConvMaxWidth = 4;
+constexpr int kConvRun = 32;          // tokens per thread (history rows are re-read once per run)
+constexpr int kConvBatch = 4;         // rows loaded together
+constexpr int kPrepThreads = 256;
+
+struct ConvParams {
+    const uint16_t *x;        // [T, H, d] bf16
+    const float *w;           // [H, d, W]
+    const int32_t *cu;        // [num_seqs + 1]
+    uint16_t *y;              // [T, H, d] bf16
+    int64_t total_tokens;
+    int num_seqs, H, width;
+    bool l2norm;
+};
+
+// first token of the sequence containing token t (cu_seqlens searched once per run)
+__device__ __forceinline__ int seq_of(const int32_t *cu, int num_seqs, int64_t t) {
+    int lo = 0, hi = num_seqs;   // invariant: cu[lo] <= t < cu[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cu[mid] <= t) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ void load8(const uint16_t *p, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = bf16_to_f32(static_cast<uint16_t>(w4[i] & 0xFFFFu));
+        v[2 * i + 1] = bf16_to_f32(static_cast<uint16_t>(w4[i] >> 16));
+    }
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w4[i] = (uint32_t)f32_to_bf16(v[2 * i]) | ((uint32_t)f32_to_bf16(v[2 * i + 1]) << 16);
+    return make_uint4(w4[0], w4[1], w4[2], w4[3]);
+}
+
+// grid: x = column groups of 8 channels (H d / 8 per row) / kPrepThreads, y = runs of kConvRun
+// tokens.  A thread keeps its 8 channels' taps in registers for the whole run and slides a window
+// of the last W - 1 input rows; the run's rows are loaded kConvBatch at a time so that several
+// loads are in flight.
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads) short_conv_kernel(const ConvParams p) {
+    constexpr int LPH = D / 8;                        // lanes per (token, head) row
+    const int64_t groups = (int64_t)p.H * LPH;        // 8-channel groups per token row
+    const int64_t g = (int64_t)blockIdx.x * kPrepThreads + threadIdx.x;
+    const bool active = g < groups;                   // whole (token, head) rows share a warp
+    const int h = static_cast<int>(g / LPH);
+    const int c0 = static_cast<int>(g % LPH) * 8;
+    const int64_t t_begin = (int64_t)blockIdx.y * kConvRun;
+    if (t_begin >= p.total_tokens) return;
+    const int64_t t_end = min64(t_begin + kConvRun, p.total_tokens);
+    const int W = p.width;
+
+    // taps on the history (zero beyond W - 1) and the tap on the current token
+    float wt[8][kConvMaxWidth - 1], wcur[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const float *wc = p.w + ((int64_t)h * D + c0 + c) * W;
+#pragma unroll
+        for (int j = 0; j < kConvMaxWidth - 1; ++j) wt[c][j] = (active && j < W - 1) ? wc[j] : 0.f;
+        wcur[c] = active ? wc[W - 1] : 0.f;
+    }
+
+    int s = seq_of(p.cu, p.num_seqs, t_begin);
+    int64_t s_start = p.cu[s], s_end = p.cu[s + 1];
+    // history window: hist[j] = x_{t - (W-1) + j} for j < W - 1 (zero before the sequence start)
+    float hist[kConvMaxWidth - 1][8];
+#pragma unroll
+    for (int j = 0; j < kConvMaxWidth - 1; ++j) {
+        const int64_t tj = t_begin - (W - 1) + j;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) hist[j][c] = 0.f;
+        if (active && j < W - 1 && tj >= s_start) load8(p.x + (tj * p.H + h) * D + c0, hist[j]);
+    }
+    for (int64_t tb = t_begin; tb < t_end; tb += kConvBatch) {
+        float xs[kConvBatch][8];
+#pragma unroll
+        for (int u = 0; u < kConvBatch; ++u) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) xs[u][c] = 0.f;
+            if (active && tb + u < t_end) load8(p.x + ((tb + u) * p.H + h) * D + c0, xs[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kConvBatch; ++u) {
+            const int64_t t = tb + u;
+            if (t >= t_end) break;   // the same for the whole block
+            if (t >= s_end) {        // a new sequence starts here: its history is zero
+                while (t >= s_end && s + 1 < p.num_seqs) { ++s; s_start = p.cu[s]; s_end = p.cu[s + 1]; }
+                if (t >= s_end && threadIdx.x == 0) atomicOr(&g_kda_error_word, kErrBadSeqlens);
+#pragma unroll
+                for (int j = 0; j < kConvMaxWidth - 1; ++j)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) hist[j][c] = 0.f;
+            }
+            float y[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float acc = wcur[c] * xs[u][c];
+#pragma unroll
+                for (int j = 0; j < kConvMaxWidth - 1; ++j) acc = fmaf(wt[c][j], hist[j][c], acc);
+                y[c] = acc;
+            }
+            if (p.l2norm) {
+                float ss = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) ss = fmaf(y[c], y[c], ss);
+#pragma unroll
+                for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                const float inv = rsqrtf(ss + 1e-12f);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) y[c] *= inv;
+            }
+            if (active) *reinterpret_cast<uint4 *>(p.y + (t * p.H + h) * D + c0) = pack8_bf16(y);
+            // slide the window: hist[j] <- hist[j + 1], newest = x_t
+#pragma unroll
+            for (int j = 0; j < kConvMaxWidth - 2; ++j)
+                if (j < W - 2)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) hist[j][c] = hist[j + 1][c];
+            if (W >= 2) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (W == 2) hist[0][c] = xs[u][c];
+                    else if (W == 3) hist[1][c] = xs[u][c];
+                    else hist[2][c] = xs[u][c];
+                }
+            }
+        }
+    }
+}
+
+struct NormGateParams {
+    const float *o;           // [T, H, d] fp32
+    const uint16_t *gate;     // [T, H, d] bf16 or null
+    const float *w;           // [d]
+    void *out;                // [T, H, d] bf16 or fp32
+    int64_t rows;             // T * H
+    float eps;
+    bool out_f32;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads) norm_gate_kernel(const NormGateParams p) {
+    constexpr int LPH = D / 8;
+    const int64_t g = (int64_t)blockIdx.x * kPrepThreads + threadIdx.x;
+    const int64_t row = g / LPH;
+    const int c0 = static_cast<int>(g % LPH) * 8;
+    const bool active = row < p.rows;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) {
+        const float4 *src = reinterpret_cast<const float4 *>(p.o + row * D + c0);
+        const float4 a = __ldcs(src), b = __ldcs(src + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) ss = fmaf(v[c], v[c], ss);
+#pragma unroll
+    for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = rsqrtf(ss / D + p.eps);
+    if (!active) return;
+    float gt[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (p.gate) load8(p.gate + row * D + c0, gt);
+    float y[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        y[c] = v[c] * inv * __ldg(p.w + c0 + c);
+        if (p.gate) y[c] *= sigmoid_fast(gt[c]);
+    }
+    if (p.out_f32) {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + row * D + c0);
+        dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+        dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+    } else {
+        *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + row * D + c0) = pack8_bf16(y);
+    }
+}
+
+}  // namespace kda

@@ -130,3 +130,19 @@ def test_verify_and_commit_reject_bad_arguments():
     assert C(16, 16, 16, None, 16, 16, 2, 4, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG     # accepted
     assert C(16, 16, 16, 18, 16, 16, 2, 4, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG       # alignment
     assert C(16, 16, 16, 16, 16, 16, 0, 4, 2, 128, 128, None) == kda.KDA_OK
+
+
+def test_short_conv_and_norm_gate_reject_bad_arguments():
+    SC, NG = lib.kda_short_conv, lib.kda_output_norm_gate
+    assert SC(16, 16, 16, 2, 64, 2, 128, 0, 1, 32, None) == kda.KDA_ERR_INVALID_ARG      # width 0
+    assert SC(16, 16, 16, 2, 64, 2, 128, 5, 1, 32, None) == kda.KDA_ERR_INVALID_ARG      # width 5
+    assert SC(16, 16, 16, 2, 64, 2, 80, 4, 1, 32, None) == kda.KDA_ERR_UNSUPPORTED       # d
+    assert SC(16, 16, None, 2, 64, 2, 128, 4, 1, 32, None) == kda.KDA_ERR_INVALID_ARG    # cu_seqlens
+    assert SC(8, 16, 16, 2, 64, 2, 128, 4, 1, 32, None) == kda.KDA_ERR_INVALID_ARG       # misaligned x
+    assert SC(16, 16, 16, 0, 64, 2, 128, 4, 1, 32, None) == kda.KDA_ERR_INVALID_ARG      # tokens, no sequences
+    assert SC(16, 16, 16, 2, 0, 2, 128, 4, 1, 32, None) == kda.KDA_OK                    # nothing to do
+    assert NG(16, None, 16, 64, 2, 96, 1e-6, 32, 0, None) == kda.KDA_ERR_UNSUPPORTED
+    assert NG(16, None, 16, 64, 2, 128, -1.0, 32, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert NG(16, None, None, 64, 2, 128, 1e-6, 32, 0, None) == kda.KDA_ERR_INVALID_ARG
+    assert NG(16, None, 16, 64, 2, 128, 1e-6, 32, 7, None) == kda.KDA_ERR_INVALID_ARG
+    assert NG(16, None, 16, 0, 2, 128, 1e-6, 32, 0, None) == kda.KDA_OK
