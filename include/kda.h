@@ -206,6 +206,19 @@ KDA_API kda_status kda_output_norm_gate(const float *o, const void *gate, const 
                                         int32_t H, int32_t d_v, float eps, void *out, kda_dtype out_dtype,
                                         void *stream);
 
+/*
+ * kda_state_combine — one affine state map per (sequence, head) unit, for context-parallel prefill
+ * (a sequence split into segments held by different GPUs):
+ *   S_out[u] = M[u] S_in[u] + B[u]
+ *   M fp32 [units, d_k, d_k]; S_in, B, S_out fp32 [units, d_k, d_v]; S_out may alias B, not S_in.
+ * Over a segment, the recurrence maps its incoming state S to M S + B, where B is the state it
+ * reaches from S = 0 and M the state the homogeneous recurrence (v = 0) reaches from S = I; both
+ * come from kda_chunk_fwd (the pages carry the state sequentially from chunk to chunk: "Kimi K3 ·
+ * Lesson 3 of 14", CHUNKWISE diagram).  At most 65535 units per call.
+ */
+KDA_API kda_status kda_state_combine(const float *M, const float *S_in, const float *B, float *S_out,
+                                     int32_t units, int32_t d_k, int32_t d_v, void *stream);
+
 /* Static description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);
 

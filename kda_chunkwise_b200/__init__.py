@@ -10,11 +10,15 @@ Entry points (same names as the C ABI):
   kda_decode_verify / kda_decode_commit                     K proposed tokens, then the accepted prefix
   kda_short_conv, kda_output_norm_gate                      the module's short convolution and
                                                             pre-gate normalisation + output gate
+  kda_segment_maps, kda_state_combine,                      context-parallel prefill: a sequence split
+  kda_context_parallel_fwd                                  into segments over the ranks of a group
 """
 from __future__ import annotations
 
 import ctypes
 import os
+
+import numpy as np
 
 import torch
 
@@ -22,6 +26,7 @@ __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_chunk_fwd_workspace_min", "kda_sync_check", "kda_status_string", "KDAError",
            "kda_launch_count", "kda_chunk_fwd_noalloc", "kda_inject_stall",
            "kda_decode_verify", "kda_decode_commit", "kda_short_conv", "kda_output_norm_gate",
+           "kda_state_combine", "kda_segment_maps", "context_parallel_states", "kda_context_parallel_fwd",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -75,6 +80,8 @@ def _load() -> ctypes.CDLL:
     L.kda_short_conv.restype = ctypes.c_int
     L.kda_output_norm_gate.argtypes = [fp, vp, fp, i64, i32, i32, f32, vp, ctypes.c_int, vp]
     L.kda_output_norm_gate.restype = ctypes.c_int
+    L.kda_state_combine.argtypes = [fp, fp, fp, fp, i32, i32, i32, vp]
+    L.kda_state_combine.restype = ctypes.c_int
     L.kda_inject_stall.argtypes = [i32, ctypes.c_uint64]
     L.kda_inject_stall.restype = ctypes.c_int
     return L
@@ -332,6 +339,77 @@ def kda_output_norm_gate(o, gate, w, eps: float = 1e-6, out=None, stream=None, o
                                   _OUT_DTYPES[out.dtype], _stream_handle(stream, dev))
     _check(st, "kda_output_norm_gate")
     return out
+
+
+def kda_state_combine(M, S_in, B, out=None, stream=None):
+    """S_out = M S_in + B per (sequence, head): M fp32 [..., d_k, d_k], S_in and B [..., d_k, d_v]."""
+    dev = M.device
+    d_k, d_v = B.shape[-2], B.shape[-1]
+    lead = tuple(B.shape[:-2])
+    units = int(np.prod(lead)) if lead else 1
+    _need(M, "M", torch.float32, lead + (d_k, d_k), dev)
+    _need(S_in, "S_in", torch.float32, lead + (d_k, d_v), dev)
+    _need(B, "B", torch.float32, lead + (d_k, d_v), dev)
+    if out is None:
+        out = torch.empty_like(B)
+    _need(out, "out", torch.float32, lead + (d_k, d_v), dev)
+    st = lib.kda_state_combine(_ptr(M), _ptr(S_in), _ptr(B), _ptr(out), units, d_k, d_v,
+                               _stream_handle(stream, dev))
+    _check(st, "kda_state_combine")
+    return out
+
+
+def kda_segment_maps(q, k, v, a, beta, A_log, cu_seqlens, scale: float = 1.0, max_seqlen=None, stream=None):
+    """The affine map S -> M S + B of each (sequence, head) over the tokens given: B is the final
+    state from S = 0, M the final state of the homogeneous recurrence (v = 0) from S = I.  Two
+    kda_chunk_fwd calls; returns (M [N, H, d_k, d_k], B [N, H, d_k, d_v])."""
+    N = cu_seqlens.numel() - 1
+    T, H, d_k = q.shape
+    _, B = kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None, scale=scale,
+                         max_seqlen=max_seqlen, stream=stream, out_dtype=torch.bfloat16)
+    v0 = torch.zeros((T, H, d_k), dtype=torch.bfloat16, device=q.device)
+    eye = torch.eye(d_k, dtype=torch.float32, device=q.device).expand(N, H, d_k, d_k).contiguous()
+    _, M = kda_chunk_fwd(q, k, v0, a, beta, A_log, cu_seqlens, gate=None, initial_state=eye, scale=scale,
+                         max_seqlen=max_seqlen, stream=stream, out_dtype=torch.bfloat16)
+    return M, B
+
+
+def context_parallel_states(M, B, S0, group=None, combine=None):
+    """Incoming state of this rank's segments: gather every rank's (M, B) over the process group and
+    fold the maps of the ranks before this one, in rank order, starting from S0.  ``combine(M, S, B)``
+    applies one map (kda_state_combine unless given)."""
+    import torch.distributed as dist
+    combine = combine or (lambda m, s, b: kda_state_combine(m, s, b))
+    world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+    S = S0.clone() if S0 is not None else torch.zeros_like(B)
+    if world == 1:
+        return S
+    rank = dist.get_rank(group)
+
+    def gather(x):   # every rank's x, stacked in rank order
+        x = x.contiguous()
+        flat = torch.empty((world * x.shape[0],) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
+        dist.all_gather_into_tensor(flat, x, group=group)
+        return flat.view((world,) + tuple(x.shape))
+
+    Ms, Bs = gather(M), gather(B)
+    for r in range(rank):
+        S = combine(Ms[r], S, Bs[r])
+    return S
+
+
+def kda_context_parallel_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None,
+                             scale: float = 1.0, group=None, max_seqlen=None, stream=None,
+                             out_dtype=torch.bfloat16):
+    """Prefill of sequences split along time over the ranks of ``group``: this rank holds segment
+    `rank` of every sequence (the same sequences, in the same order, on every rank; segments in
+    rank order).  ``initial_state`` is the sequences' initial state (the same on every rank).
+    Returns (out of this segment, state after this segment): on the last rank, the final states."""
+    M, B = kda_segment_maps(q, k, v, a, beta, A_log, cu_seqlens, scale=scale, max_seqlen=max_seqlen,
+                            stream=stream)
+    S_in = context_parallel_states(M, B, initial_state, group=group)
+    return kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=gate, initial_state=S_in, scale=scale,
+                         max_seqlen=max_seqlen, stream=stream, out_dtype=out_dtype)
 
 
 def kda_launch_count() -> int:

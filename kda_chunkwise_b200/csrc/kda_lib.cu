@@ -15,6 +15,7 @@
 #include "prefill_fused.cuh"
 #include "speculative.cuh"
 #include "preprocess.cuh"
+#include "state_map.cuh"
 
 namespace {
 
@@ -440,6 +441,32 @@ kda_status kda_output_norm_gate(const float *o, const void *gate, const float *w
     g_launches.fetch_add(1, std::memory_order_relaxed);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "norm_gate launch");
+}
+
+kda_status kda_state_combine(const float *M, const float *S_in, const float *B, float *S_out, int32_t units,
+                             int32_t d_k, int32_t d_v, void *stream) {
+    if (units < 0) return fail(KDA_ERR_INVALID_ARG, "kda_state_combine: units < 0");
+    if (!supported_dim(d_k) || !supported_dim(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_state_combine: d_k and d_v must be 64 or 128");
+    if (units == 0) return KDA_OK;
+    if (!M || !S_in || !B || !S_out) return fail(KDA_ERR_INVALID_ARG, "kda_state_combine: NULL pointer");
+    if (!aligned(M, 16) || !aligned(S_in, 16) || !aligned(B, 16) || !aligned(S_out, 16))
+        return fail(KDA_ERR_INVALID_ARG, "kda_state_combine: pointer not 16-byte aligned");
+    const size_t state_bytes = (size_t)units * d_k * d_v * 4;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(S_in), b0 = reinterpret_cast<uintptr_t>(S_out);
+    if (a0 < b0 + state_bytes && b0 < a0 + state_bytes)
+        return fail(KDA_ERR_INVALID_ARG, "kda_state_combine: S_out overlaps S_in");
+    if (units > 65535) return fail(KDA_ERR_INVALID_ARG, "kda_state_combine: more than 65535 units per call");
+    kda::CombineParams p{M, S_in, B, S_out};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)(d_k / kda::kCombineRows), (unsigned)units);
+    if (d_k == 128 && d_v == 128) kda::state_combine_kernel<128, 128><<<grid, 256, 0, st>>>(p);
+    else if (d_k == 128 && d_v == 64) kda::state_combine_kernel<128, 64><<<grid, 256, 0, st>>>(p);
+    else if (d_k == 64 && d_v == 128) kda::state_combine_kernel<64, 128><<<grid, 256, 0, st>>>(p);
+    else kda::state_combine_kernel<64, 64><<<grid, 256, 0, st>>>(p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "state_combine launch");
 }
 
 kda_status kda_sync_check(void *stream) {
