@@ -219,6 +219,35 @@ KDA_API kda_status kda_output_norm_gate(const float *o, const void *gate, const 
 KDA_API kda_status kda_state_combine(const float *M, const float *S_in, const float *B, float *S_out,
                                      int32_t units, int32_t d_k, int32_t d_v, void *stream);
 
+/*
+ * kda_chunk_bwd — gradients of the prefill (kda_chunk_fwd with the same inputs) with respect to
+ * q, k, v, the decay logits a, beta, the gate logits, A_log and the initial state, given dout (the
+ * gradient of the outputs) and optionally dfinal_state (the gradient of the final states).  The
+ * pages describe only the forward recurrence; this is its reverse-mode derivative, token by token
+ * ("Review A · Sequence and depth", Free recall; "Kimi K3 · Lesson 3 of 14", eq. 5 passage).
+ *   inputs      as kda_chunk_fwd (bf16 q, k, a, v, gate; fp32 beta, A_log; cu_seqlens on the device)
+ *   dout        fp32 [total_tokens, H, d_v]        dfinal_state fp32 [num_seqs, H, d_k, d_v] or NULL
+ *   dq, dk, da  fp32 [total_tokens, H, d_k]        dv, dgate fp32 [total_tokens, H, d_v]
+ *   dbeta       fp32 [total_tokens, H]             dA_log fp32 [H] (overwritten: summed over sequences)
+ *   dinitial_state fp32 [num_seqs, H, d_k, d_v] or NULL
+ *   dgate must be given when gate is; workspace of kda_chunk_bwd_workspace_size(...) bytes, 16-byte
+ *   aligned: the state at the start of every 64-token chunk plus a 64-state scratch per unit.
+ * Runs one CTA per (sequence, head) over the tokens in order, then in reverse: its time is the
+ * latency of the sequence's token steps.
+ */
+KDA_API kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, const float *beta,
+                                 const void *gate, const float *A_log, const int32_t *cu_seqlens,
+                                 int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v,
+                                 float scale, const float *initial_state, const float *dout,
+                                 const float *dfinal_state, float *dq, float *dk, float *dv, float *da,
+                                 float *dbeta, float *dgate, float *dA_log, float *dinitial_state,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace kda_chunk_bwd needs (host-only; 0 on invalid sizes):
+ * ((total_tokens / 64 + num_seqs) * H + num_seqs * H * 64) * d_k * d_v * 4 bytes. */
+KDA_API size_t kda_chunk_bwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k,
+                                            int32_t d_v);
+
 /* Static description of a status code. */
 KDA_API const char *kda_status_string(kda_status status);
 

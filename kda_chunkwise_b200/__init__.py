@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
                                                             pre-gate normalisation + output gate
   kda_segment_maps, kda_state_combine,                      context-parallel prefill: a sequence split
   kda_context_parallel_fwd                                  into segments over the ranks of a group
+  kda_chunk_bwd                                             gradients of the prefill
 """
 from __future__ import annotations
 
@@ -27,6 +28,7 @@ __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_launch_count", "kda_chunk_fwd_noalloc", "kda_inject_stall",
            "kda_decode_verify", "kda_decode_commit", "kda_short_conv", "kda_output_norm_gate",
            "kda_state_combine", "kda_segment_maps", "context_parallel_states", "kda_context_parallel_fwd",
+           "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -82,6 +84,11 @@ def _load() -> ctypes.CDLL:
     L.kda_output_norm_gate.restype = ctypes.c_int
     L.kda_state_combine.argtypes = [fp, fp, fp, fp, i32, i32, i32, vp]
     L.kda_state_combine.restype = ctypes.c_int
+    L.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, fp, vp, fp, vp, i32, i64, i32, i32, i32, f32, fp, fp, fp,
+                                fp, fp, fp, fp, fp, fp, fp, fp, vp, sz, vp]
+    L.kda_chunk_bwd.restype = ctypes.c_int
+    L.kda_chunk_bwd_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+    L.kda_chunk_bwd_workspace_size.restype = sz
     L.kda_inject_stall.argtypes = [i32, ctypes.c_uint64]
     L.kda_inject_stall.restype = ctypes.c_int
     return L
@@ -410,6 +417,52 @@ def kda_context_parallel_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, ini
     S_in = context_parallel_states(M, B, initial_state, group=group)
     return kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=gate, initial_state=S_in, scale=scale,
                          max_seqlen=max_seqlen, stream=stream, out_dtype=out_dtype)
+
+
+def kda_chunk_bwd_workspace_size(total_tokens, num_seqs, H, d_k, d_v) -> int:
+    return int(lib.kda_chunk_bwd_workspace_size(total_tokens, num_seqs, H, d_k, d_v))
+
+
+def kda_chunk_bwd(q, k, v, a, beta, A_log, cu_seqlens, dout, gate=None, initial_state=None,
+                  dfinal_state=None, scale: float = 1.0, workspace=None, stream=None):
+    """Gradients of kda_chunk_fwd's outputs (and final states) with respect to its inputs.
+
+    dout fp32 [T, H, d_v]; dfinal_state fp32 [N, H, d_k, d_v] or None.  Returns a dict of fp32
+    tensors: dq, dk, da [T, H, d_k]; dv, dgate [T, H, d_v] (dgate None without a gate); dbeta
+    [T, H]; dA_log [H]; dinitial_state [N, H, d_k, d_v] (None without an initial state).
+    """
+    dev = q.device
+    T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    bf, f32 = torch.bfloat16, torch.float32
+    for name, t, shp in (("q", q, (T, H, d_k)), ("k", k, (T, H, d_k)), ("a", a, (T, H, d_k)),
+                         ("v", v, (T, H, d_v))):
+        _need(t, name, bf, shp, dev)
+    _need(beta, "beta", f32, (T, H), dev)
+    _need(A_log, "A_log", f32, (H,), dev)
+    _need(dout, "dout", f32, (T, H, d_v), dev)
+    if gate is not None:
+        _need(gate, "gate", bf, (T, H, d_v), dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", f32, (N, H, d_k, d_v), dev)
+    if dfinal_state is not None:
+        _need(dfinal_state, "dfinal_state", f32, (N, H, d_k, d_v), dev)
+    g = dict(dq=torch.empty((T, H, d_k), dtype=f32, device=dev), dk=torch.empty((T, H, d_k), dtype=f32, device=dev),
+             da=torch.empty((T, H, d_k), dtype=f32, device=dev), dv=torch.empty((T, H, d_v), dtype=f32, device=dev),
+             dbeta=torch.empty((T, H), dtype=f32, device=dev), dA_log=torch.empty((H,), dtype=f32, device=dev),
+             dgate=None if gate is None else torch.empty((T, H, d_v), dtype=f32, device=dev),
+             dinitial_state=None if initial_state is None else torch.empty((N, H, d_k, d_v), dtype=f32, device=dev))
+    need = kda_chunk_bwd_workspace_size(T, N, H, d_k, d_v)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate), _ptr(A_log),
+                           _ptr(cu_seqlens), N, T, H, d_k, d_v, float(scale), _ptr(initial_state), _ptr(dout),
+                           _ptr(dfinal_state), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]),
+                           _ptr(g["dbeta"]), _ptr(g["dgate"]), _ptr(g["dA_log"]), _ptr(g["dinitial_state"]),
+                           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream, dev))
+    _check(st, "kda_chunk_bwd")
+    return g
 
 
 def kda_launch_count() -> int:

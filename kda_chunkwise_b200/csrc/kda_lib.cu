@@ -16,6 +16,7 @@
 #include "speculative.cuh"
 #include "preprocess.cuh"
 #include "state_map.cuh"
+#include "backward.cuh"
 
 namespace {
 
@@ -467,6 +468,77 @@ kda_status kda_state_combine(const float *M, const float *S_in, const float *B, 
     g_launches.fetch_add(1, std::memory_order_relaxed);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "state_combine launch");
+}
+
+size_t kda_chunk_bwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || !supported_dim(d_k) || !supported_dim(d_v)) return 0;
+    const size_t state = (size_t)d_k * d_v * 4;
+    const size_t ckpts = (size_t)(total_tokens / kda::kBwdChunk + num_seqs) * H;   // >= sum ceil(len / 64)
+    const size_t scratch = (size_t)num_seqs * H * kda::kBwdChunk;
+    return (ckpts + scratch) * state;
+}
+
+kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, const float *beta,
+                         const void *gate, const float *A_log, const int32_t *cu_seqlens, int32_t num_seqs,
+                         int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                         const float *initial_state, const float *dout, const float *dfinal_state, float *dq,
+                         float *dk, float *dv, float *da, float *dbeta, float *dgate, float *dA_log,
+                         float *dinitial_state, void *workspace, size_t workspace_bytes, void *stream) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: negative size or H <= 0");
+    if (!supported_dim(d_k) || !supported_dim(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_bwd: d_k and d_v must be 64 or 128");
+    if (num_seqs == 0) {
+        if (total_tokens != 0) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: tokens without sequences");
+        return KDA_OK;
+    }
+    if (!cu_seqlens || !A_log || !dA_log) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: NULL cu_seqlens, A_log or dA_log");
+    if (total_tokens > 0 && (!q || !k || !v || !a || !beta || !dout || !dq || !dk || !dv || !da || !dbeta))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: NULL input or gradient pointer");
+    if (gate && !dgate) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: gate given without dgate");
+    const void *ptrs[] = {q, k, v, a, gate, initial_state, dout, dfinal_state, dq, dk, dv, da, dgate,
+                          dinitial_state, workspace};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned(ptr, 16)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: tensor pointer not 16-byte aligned");
+    const void *ptrs4[] = {beta, A_log, cu_seqlens, dbeta, dA_log};
+    for (const void *ptr : ptrs4)
+        if (ptr && !aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: scalar array not 4-byte aligned");
+    const size_t need = kda_chunk_bwd_workspace_size(total_tokens, num_seqs, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: workspace missing or too small (need " + std::to_string(need) + " bytes)");
+    const int64_t units = (int64_t)num_seqs * H;
+    if (units > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: num_seqs * H too large");
+    kda::BwdParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.a = static_cast<const uint16_t *>(a);
+    p.gate = static_cast<const uint16_t *>(gate);
+    p.beta = beta;
+    p.A_log = A_log;
+    p.cu = cu_seqlens;
+    p.S0 = initial_state;
+    p.dout = dout;
+    p.dS_T = dfinal_state;
+    p.dq = dq; p.dk = dk; p.dv = dv; p.da = da; p.dbeta = dbeta; p.dgate = dgate;
+    p.dA_log = dA_log;
+    p.dS0 = dinitial_state;
+    const size_t state = (size_t)d_k * d_v;
+    p.ckpt = static_cast<float *>(workspace);
+    p.scratch = p.ckpt + (size_t)(total_tokens / kda::kBwdChunk + num_seqs) * H * state;
+    p.total_tokens = total_tokens;
+    p.num_seqs = num_seqs;
+    p.H = H;
+    p.scale = scale;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(dA_log, 0, sizeof(float) * H, st);   // the kernel accumulates into it
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dA_log)");
+    if (d_k == 128 && d_v == 128) kda::kda_bwd_kernel<128, 128><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
+    else if (d_k == 128 && d_v == 64) kda::kda_bwd_kernel<128, 64><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
+    else if (d_k == 64 && d_v == 128) kda::kda_bwd_kernel<64, 128><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
+    else kda::kda_bwd_kernel<64, 64><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "chunk_bwd launch");
 }
 
 kda_status kda_sync_check(void *stream) {

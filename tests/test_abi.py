@@ -146,3 +146,24 @@ def test_short_conv_and_norm_gate_reject_bad_arguments():
     assert NG(16, None, None, 64, 2, 128, 1e-6, 32, 0, None) == kda.KDA_ERR_INVALID_ARG
     assert NG(16, None, 16, 64, 2, 128, 1e-6, 32, 7, None) == kda.KDA_ERR_INVALID_ARG
     assert NG(16, None, 16, 0, 2, 128, 1e-6, 32, 0, None) == kda.KDA_OK
+
+
+def test_chunk_bwd_rejects_bad_arguments():
+    B = lib.kda_chunk_bwd
+    ok = dict(q=16, k=16, v=16, a=16, beta=16, gate=None, A_log=16, cu=16, N=1, T=64, H=2, dk=128, dv=128,
+              S0=None, dout=16, dST=None, dq=16, dkk=16, dvv=16, da=16, db=16, dg=None, dA=16, dS0=None,
+              ws=256, wsb=1 << 30)
+
+    def bwd(**o):
+        a = dict(ok, **o)
+        return B(a["q"], a["k"], a["v"], a["a"], a["beta"], a["gate"], a["A_log"], a["cu"], a["N"], a["T"], a["H"],
+                 a["dk"], a["dv"], 1.0, a["S0"], a["dout"], a["dST"], a["dq"], a["dkk"], a["dvv"], a["da"], a["db"],
+                 a["dg"], a["dA"], a["dS0"], a["ws"], a["wsb"], None)
+
+    assert bwd(dv=96) == kda.KDA_ERR_UNSUPPORTED
+    assert bwd(dout=None) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(gate=16, dg=None) == kda.KDA_ERR_INVALID_ARG      # a gate needs its gradient
+    assert bwd(wsb=10) == kda.KDA_ERR_INVALID_ARG                 # workspace too small
+    assert bwd(q=8) == kda.KDA_ERR_INVALID_ARG                    # misaligned
+    assert bwd(N=0, T=0) == kda.KDA_OK
+    assert kda.kda_chunk_bwd_workspace_size(8192, 1, 32, 128, 128) == (8192 // 64 + 1 + 64) * 32 * 128 * 128 * 4

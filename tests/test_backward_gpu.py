@@ -1,0 +1,91 @@
+"""GPU parity of the backward pass (kda_chunk_bwd) against the oracle's reverse-mode derivative of
+the token-by-token recurrence (oracle/backward.py, itself pinned by finite differences).
+
+Tolerances as for the forward outputs, applied to every gradient of every (sequence, head) unit:
+relative L2 error <= 5e-3 and max |error| <= 2e-2 * rms(oracle gradient)."""
+import numpy as np
+import pytest
+import torch
+
+import kda_inputs as KI
+from oracle.backward import recurrence_bwd
+from parity import host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kda():
+    import kda_chunkwise_b200 as m
+    return m
+
+
+def _close(got, ref, label):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    nrm = np.linalg.norm(ref)
+    if nrm == 0:
+        assert np.abs(got).max() <= 1e-6, label
+        return
+    rel = np.linalg.norm(got - ref) / nrm
+    rms = np.sqrt(np.mean(ref ** 2))
+    assert rel <= 5e-3, f"{label}: rel L2 {rel:.2e}"
+    assert np.abs(got - ref).max() <= 2e-2 * rms + 1e-30, f"{label}: max err {np.abs(got - ref).max():.2e} rms {rms:.2e}"
+
+
+def _check(kda, inp, dout, dST, g, units, scale=1.0):
+    cu = inp["cu_seqlens"].cpu().tolist()
+    dA_ref = {}
+    for n, h in units:
+        s, e = cu[n], cu[n + 1]
+        gate = inp["gate"]
+        S0 = inp["initial_state"]
+        ref = recurrence_bwd(host(inp["q"][s:e, h]), host(inp["k"][s:e, h]), host(inp["v"][s:e, h]),
+                             host(inp["a"][s:e, h]), host(inp["beta"][s:e, h]), float(inp["A_log"][h]),
+                             host(dout[s:e, h]), gate=None if gate is None else host(gate[s:e, h]),
+                             S0=None if S0 is None else host(S0[n, h]),
+                             dS_T=None if dST is None else host(dST[n, h]), scale=scale)
+        lab = f"unit ({n},{h})"
+        if e > s:
+            for key in ("dq", "dk", "dv", "da"):
+                _close(host(g[key][s:e, h]), ref[key], f"{lab} {key}")
+            _close(host(g["dbeta"][s:e, h]), ref["dbeta"], f"{lab} dbeta")
+            if gate is not None:
+                _close(host(g["dgate"][s:e, h]), ref["dgate"], f"{lab} dgate")
+        if S0 is not None:
+            _close(host(g["dinitial_state"][n, h]), ref["dS0"], f"{lab} dS0")
+        dA_ref[h] = dA_ref.get(h, 0.0) + ref["dA_log"]
+    return dA_ref
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("with_gate,with_state", [(True, True), (False, False)])
+def test_backward_matches_oracle(kda, dk, dv, with_gate, with_state):
+    w = KI.Workload("bwd", (70, 1, 130, 0, 64), 2, dk, dv, A_log="uniform", gate=with_gate,
+                    init_state="normal_0.02" if with_state else "none", seed=31)
+    inp = KI.make_inputs(w, "cuda")
+    g_ = torch.Generator(device="cuda").manual_seed(32)
+    dout = torch.randn((w.total_tokens, w.H, dv), generator=g_, device="cuda")
+    dST = torch.randn((w.num_seqs, w.H, dk, dv), generator=g_, device="cuda") if with_state else None
+    g = kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
+                          dout, gate=inp["gate"], initial_state=inp["initial_state"], dfinal_state=dST,
+                          scale=0.9)
+    kda.kda_sync_check()
+    units = [(n, h) for n in range(w.num_seqs) for h in range(w.H)]
+    dA_ref = _check(kda, inp, dout, dST, g, units, scale=0.9)
+    for h, ref in dA_ref.items():   # dA_log sums over every sequence
+        assert abs(float(g["dA_log"][h]) - ref) <= 5e-3 * max(abs(ref), 1e-6), f"dA_log[{h}]"
+
+
+def test_backward_full_size_sampled(kda):
+    # the prefill workload (B=1, H=32, T=8192, d=128), three heads checked over all 8192 tokens
+    w = KI.WORKLOADS["prefill_B1_H32_T8192_d128"]
+    inp = KI.make_inputs(w, "cuda")
+    g_ = torch.Generator(device="cuda").manual_seed(33)
+    dout = torch.randn((w.total_tokens, w.H, w.d_v), generator=g_, device="cuda") * 0.1
+    dST = torch.randn((w.num_seqs, w.H, w.d_k, w.d_v), generator=g_, device="cuda") * 0.1
+    g = kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
+                          dout, gate=inp["gate"], initial_state=inp["initial_state"], dfinal_state=dST)
+    kda.kda_sync_check()
+    dA_ref = _check(kda, inp, dout, dST, g, [(0, 0), (0, 13), (0, 31)])
+    for h, ref in dA_ref.items():
+        assert abs(float(g["dA_log"][h]) - ref) <= 5e-3 * max(abs(ref), 1e-6), f"dA_log[{h}]"
