@@ -367,6 +367,45 @@ def main():
                 "algorithmic_bytes": bytes_step, "algorithmic_flops": flops_step,
                 "tensor_frac_of_bf16_peak": flops_step / (ms * 1e-3) / 1e12 / tf}
 
+    # backward row: kda_chunk_bwd on the prefill workload (gradients of every input)
+    backward = None
+    if not args.no_decode:
+        gb = torch.Generator(device=dev).manual_seed(201 + rank)
+        dout = torch.randn((w.total_tokens, w.H, w.d_v), generator=gb, device=dev) * 0.1
+        dST = torch.randn((w.num_seqs, w.H, w.d_k, w.d_v), generator=gb, device=dev) * 0.1
+        bws = torch.empty(kda.kda_chunk_bwd_workspace_size(w.total_tokens, w.num_seqs, w.H, w.d_k, w.d_v),
+                          dtype=torch.uint8, device=dev)
+
+        def bstep():
+            return kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"],
+                                     inp["cu_seqlens"], dout, gate=inp["gate"], initial_state=inp["initial_state"],
+                                     dfinal_state=dST, workspace=bws, stream=stream)
+
+        bstep()
+        barrier()
+        reps = 3
+        e0.record(stream)
+        for _ in range(reps):
+            bstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        kda.kda_sync_check()
+        bms = max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
+        th = w.total_tokens * w.H
+        # inputs (as the forward) + dout (fp32) read; dq, dk, da, dv, dgate (fp32), dbeta written;
+        # initial state and its gradient, final-state gradient
+        bbytes = th * (2 * (3 * w.d_k + 2 * w.d_v) + 4 + 4 * w.d_v + 4 * (3 * w.d_k + 2 * w.d_v) + 4) + \
+            3 * w.num_seqs * w.H * w.d_k * w.d_v * 4
+        bach = bbytes / (bms * 1e-3) / 1e9
+        backward = {"value": whole_job_rate(w.total_tokens, world, bms), "unit": "tokens/s", "ms_per_step": bms,
+                    "workload": w.name, "scope": "one kda_chunk_bwd call",
+                    "roofline": {"bound": "latency (sequential token steps per unit)", "achieved": bach,
+                                 "peak": hbm, "unit": "GB/s", "frac": bach / hbm, "traffic": None,
+                                 "peak_source": f"hbm_gbs of {peak_src}", "algorithmic_bytes": bbytes}}
+        del dout, dST, bws
+        torch.cuda.empty_cache()
+
     # module row: the short convolution of q, k, v (q, k L2-normalised) and the pre-gate
     # normalisation + gate of one fp32 output, on the prefill workload's tensors
     module = None
@@ -538,7 +577,7 @@ def main():
                        "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "tile": 16,
                        "parallelism": f"independent batch per rank x{world}",
                        "l2": f"inputs larger than L2 ({bytes_step / 1e6:.0f} MB per step > 126 MB); no flush"},
-            "roofline": roofline, "module": module, "decode": decode, "speculative": spec, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roofline, "backward": backward, "module": module, "decode": decode, "speculative": spec, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": launches, "clocks": clk, "kernel_src": src_hash,
         }
         print(json.dumps(line))
