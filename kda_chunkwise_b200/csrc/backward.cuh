@@ -27,6 +27,19 @@ namespace kda {
 constexpr int kBwdThreads = 512;
 constexpr int kBwdChunk = 64;
 
+// dynamic shared memory: one chunk's inputs, staged with coalesced loads before its token steps
+template <int DK, int DV>
+struct BwdStage {
+    static constexpr int kQ = 0;                            // bf16 [64][DK]
+    static constexpr int kK = kQ + kBwdChunk * DK * 2;
+    static constexpr int kA = kK + kBwdChunk * DK * 2;
+    static constexpr int kV = kA + kBwdChunk * DK * 2;      // bf16 [64][DV]
+    static constexpr int kG = kV + kBwdChunk * DV * 2;
+    static constexpr int kD = kG + kBwdChunk * DV * 2;      // fp32 [64][DV] dout
+    static constexpr int kB = kD + kBwdChunk * DV * 4;      // fp32 [64] beta
+    static constexpr int kBytes = kB + kBwdChunk * 4;
+};
+
 struct BwdParams {
     const uint16_t *q, *k, *v, *a, *gate;   // packed [T, H, d], bf16
     const float *beta, *A_log;              // [T, H], [H]
@@ -53,6 +66,15 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
     __shared__ float s_beta, s_dx_dot;
     __shared__ float s_db[DV / 32];
 
+    using ST = BwdStage<DK, DV>;
+    extern __shared__ __align__(16) unsigned char bsm[];
+    const uint16_t *sq = reinterpret_cast<const uint16_t *>(bsm + ST::kQ);
+    const uint16_t *sk = reinterpret_cast<const uint16_t *>(bsm + ST::kK);
+    const uint16_t *sa = reinterpret_cast<const uint16_t *>(bsm + ST::kA);
+    const uint16_t *sv = reinterpret_cast<const uint16_t *>(bsm + ST::kV);
+    const uint16_t *sg = reinterpret_cast<const uint16_t *>(bsm + ST::kG);
+    const float *sd = reinterpret_cast<const float *>(bsm + ST::kD);
+    const float *sb = reinterpret_cast<const float *>(bsm + ST::kB);
     const int64_t unit = blockIdx.x;
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
     const int tid = threadIdx.x, cq = tid % LPR, rg = tid / LPR;
@@ -74,17 +96,38 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
     float4 *scratch = reinterpret_cast<float4 *>(p.scratch + (size_t)unit * kBwdChunk * SZ);
     auto ck_ptr = [&](int c) { return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(ckbase + c) * H + h) * SZ); };
 
-    // per-token inputs into shared memory; alpha and x per key channel
-    auto load_tok = [&](int64_t t) {
-        for (int i = tid; i < DK; i += kBwdThreads) {
-            const int64_t off = (t * H + h) * DK + i;
-            const float x = expA * bf16_to_f32(p.a[off]);
-            s_x[i] = x;
-            s_al[i] = __expf(kGMin * sigmoid_fast(x));
-            s_k[i] = bf16_to_f32(p.k[off]);
-            s_q[i] = p.scale * bf16_to_f32(p.q[off]);
+    // a chunk's inputs (tokens tc .. tc + L - 1) into shared memory, 16 bytes per load
+    auto stage = [&](int64_t tc, int L, bool grads) {
+        auto copy_rows = [&](const void *src, int off, int row_bytes) {
+            const int pieces = row_bytes / 16;
+            for (int e = tid; e < L * pieces; e += kBwdThreads) {
+                const int i = e / pieces, j = e % pieces;
+                const uint4 *g = reinterpret_cast<const uint4 *>(static_cast<const char *>(src) +
+                                                                 ((tc + i) * H + h) * (int64_t)row_bytes) + j;
+                *reinterpret_cast<uint4 *>(bsm + off + i * row_bytes + j * 16) = __ldg(g);
+            }
+        };
+        copy_rows(p.q, ST::kQ, DK * 2);
+        copy_rows(p.k, ST::kK, DK * 2);
+        copy_rows(p.a, ST::kA, DK * 2);
+        copy_rows(p.v, ST::kV, DV * 2);
+        if (grads) {
+            if (p.gate) copy_rows(p.gate, ST::kG, DV * 2);
+            copy_rows(p.dout, ST::kD, DV * 4);
         }
-        if (tid == 0) s_beta = p.beta[t * H + h];
+        for (int i = tid; i < L; i += kBwdThreads)
+            reinterpret_cast<float *>(bsm + ST::kB)[i] = p.beta[(tc + i) * H + h];
+    };
+    // token i of the staged chunk: alpha and x per key channel, k, scale q, beta
+    auto load_tok = [&](int i) {
+        for (int c = tid; c < DK; c += kBwdThreads) {
+            const float x = expA * bf16_to_f32(sa[i * DK + c]);
+            s_x[c] = x;
+            s_al[c] = __expf(kGMin * sigmoid_fast(x));
+            s_k[c] = bf16_to_f32(sk[i * DK + c]);
+            s_q[c] = p.scale * bf16_to_f32(sq[i * DK + c]);
+        }
+        if (tid == 0) s_beta = sb[i];
     };
     // column sums over the rows of two per-thread partial vectors (through shared memory)
     auto col_sums = [&](float4 a0, float4 a1, float &c0, float &c1) {
@@ -104,7 +147,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
     };
     // forward step S <- Diag(alpha) S + k u^T, with u = beta (v - (Diag(alpha) S)^T k); the token's
     // inputs are in shared memory; u goes to s_vec[0] and v - r to s_vec[1]
-    auto fwd_step = [&](float4 (&S)[NR], int64_t t) {
+    auto fwd_step = [&](float4 (&S)[NR], int i) {
         float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int m = 0; m < NR; ++m) {
@@ -116,7 +159,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
         float rc, unused;
         col_sums(r, r, rc, unused);
         if (tid < DV) {
-            const float vmr = bf16_to_f32(p.v[(t * H + h) * DV + tid]) - rc;
+            const float vmr = bf16_to_f32(sv[i * DV + tid]) - rc;
             s_vec[1][tid] = vmr;
             s_vec[0][tid] = s_beta * vmr;
         }
@@ -135,16 +178,20 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
     const float4 *S0p = p.S0 ? reinterpret_cast<const float4 *>(p.S0 + (size_t)unit * SZ) : nullptr;
 #pragma unroll
     for (int m = 0; m < NR; ++m) S[m] = S0p ? S0p[(rg + m * RPP) * LPR + cq] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int64_t t = s0; t < s1; ++t) {
-        if ((t - s0) % kBwdChunk == 0) {
-            float4 *ck = ck_ptr(static_cast<int>((t - s0) / kBwdChunk));
+    for (int c = 0; c < nck; ++c) {
+        const int64_t tc = s0 + (int64_t)c * kBwdChunk;
+        const int L = static_cast<int>(min64(kBwdChunk, s1 - tc));
+        float4 *ck = ck_ptr(c);
 #pragma unroll
-            for (int m = 0; m < NR; ++m) ck[(rg + m * RPP) * LPR + cq] = S[m];
+        for (int m = 0; m < NR; ++m) ck[(rg + m * RPP) * LPR + cq] = S[m];
+        stage(tc, L, false);
+        __syncthreads();
+        for (int i = 0; i < L; ++i) {
+            load_tok(i);
+            __syncthreads();
+            fwd_step(S, i);
+            __syncthreads();
         }
-        load_tok(t);
-        __syncthreads();
-        fwd_step(S, t);
-        __syncthreads();
     }
 
     // ---- backward, chunk by chunk in reverse ----------------------------------------------------
@@ -160,13 +207,15 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
         const float4 *ck = ck_ptr(c);
 #pragma unroll
         for (int m = 0; m < NR; ++m) S[m] = ck[(rg + m * RPP) * LPR + cq];
+        stage(tc, L, true);
+        __syncthreads();
         for (int i = 0; i < L; ++i) {
 #pragma unroll
             for (int m = 0; m < NR; ++m) scratch[(size_t)i * (SZ / 4) + (rg + m * RPP) * LPR + cq] = S[m];
             if (i + 1 == L) break;   // the state after the last token is not needed
-            load_tok(tc + i);
+            load_tok(i);
             __syncthreads();
-            fwd_step(S, tc + i);
+            fwd_step(S, i);
             __syncthreads();
         }
         // undo the chunk's tokens in reverse order
@@ -176,7 +225,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
             float4 Sp[NR];   // S' = Diag(alpha) S_{t-1}
 #pragma unroll
             for (int m = 0; m < NR; ++m) Sp[m] = scratch[(size_t)i * (SZ / 4) + (rg + m * RPP) * LPR + cq];
-            load_tok(t);
+            load_tok(i);
             __syncthreads();
             float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -189,7 +238,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
             float rc, unused;
             col_sums(r, r, rc, unused);
             if (tid < DV) {
-                const float vmr = bf16_to_f32(p.v[tv + tid]) - rc;
+                const float vmr = bf16_to_f32(sv[i * DV + tid]) - rc;
                 s_vec[1][tid] = vmr;
                 s_vec[0][tid] = s_beta * vmr;
             }
@@ -209,12 +258,12 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
             float oc;
             col_sums(pq, pq, oc, unused);
             if (tid < DV) {
-                const float dout = p.dout[tv + tid];
+                const float dout = sd[i * DV + tid];
                 float dov = dout;
                 if (p.gate) {
-                    const float sg = sigmoid_fast(bf16_to_f32(p.gate[tv + tid]));
-                    p.dgate[tv + tid] = dout * oc * sg * (1.f - sg);
-                    dov = dout * sg;
+                    const float sgv = sigmoid_fast(bf16_to_f32(sg[i * DV + tid]));
+                    p.dgate[tv + tid] = dout * oc * sgv * (1.f - sgv);
+                    dov = dout * sgv;
                 }
                 s_vec[2][tid] = dov;
             }

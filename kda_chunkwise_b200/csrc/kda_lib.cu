@@ -109,6 +109,17 @@ kda_status dispatch_spec(const kda::SpecParams &p, int64_t units, int d_k, int d
     return launch_spec<64, 64>(p, units, commit, st);
 }
 
+template <int DK, int DV>
+kda_status launch_bwd(const kda::BwdParams &p, int64_t units, cudaStream_t stream) {
+    const int smem = kda::BwdStage<DK, DV>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kda::kda_bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chunk_bwd)");
+    kda::kda_bwd_kernel<DK, DV><<<(unsigned)units, kda::kBwdThreads, smem, stream>>>(p);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "chunk_bwd launch");
+}
+
 // Built-in scratch for kda_chunk_fwd_noalloc (callers that cannot allocate).  Host code must not
 // use this name as an address: it is a host-side stand-in; the device address comes from
 // cudaGetSymbolAddress, looked up once per device below.
@@ -532,13 +543,10 @@ kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(dA_log, 0, sizeof(float) * H, st);   // the kernel accumulates into it
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dA_log)");
-    if (d_k == 128 && d_v == 128) kda::kda_bwd_kernel<128, 128><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
-    else if (d_k == 128 && d_v == 64) kda::kda_bwd_kernel<128, 64><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
-    else if (d_k == 64 && d_v == 128) kda::kda_bwd_kernel<64, 128><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
-    else kda::kda_bwd_kernel<64, 64><<<(unsigned)units, kda::kBwdThreads, 0, st>>>(p);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    e = cudaGetLastError();
-    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "chunk_bwd launch");
+    if (d_k == 128 && d_v == 128) return launch_bwd<128, 128>(p, units, st);
+    if (d_k == 128 && d_v == 64) return launch_bwd<128, 64>(p, units, st);
+    if (d_k == 64 && d_v == 128) return launch_bwd<64, 128>(p, units, st);
+    return launch_bwd<64, 64>(p, units, st);
 }
 
 kda_status kda_sync_check(void *stream) {
