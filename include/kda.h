@@ -231,9 +231,10 @@ KDA_API kda_status kda_state_combine(const float *M, const float *S_in, const fl
  *   dbeta       fp32 [total_tokens, H]             dA_log fp32 [H] (overwritten: summed over sequences)
  *   dinitial_state fp32 [num_seqs, H, d_k, d_v] or NULL
  *   dgate must be given when gate is; workspace of kda_chunk_bwd_workspace_size(...) bytes, 16-byte
- *   aligned: the state at the start of every 64-token chunk plus a 64-state scratch per unit.
- * Runs one CTA per (sequence, head) over the tokens in order, then in reverse: its time is the
- * latency of the sequence's token steps.
+ *   aligned: the state at the start of every 32-token chunk plus a 32-state scratch per unit.
+ * Runs a cluster of d_v / 32 CTAs per (sequence, head) (one per 32 value columns) over the tokens
+ * in order, then in reverse: its time is the latency of the sequence's token steps.  Deterministic
+ * except dA_log, which is summed with atomics over sequences and column slices.
  */
 KDA_API kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *a, const float *beta,
                                  const void *gate, const float *A_log, const int32_t *cu_seqlens,
@@ -244,7 +245,7 @@ KDA_API kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, co
                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /* Workspace kda_chunk_bwd needs (host-only; 0 on invalid sizes):
- * ((total_tokens / 64 + num_seqs) * H + num_seqs * H * 64) * d_k * d_v * 4 bytes. */
+ * ((total_tokens / 32 + num_seqs) * H + num_seqs * H * 32) * d_k * d_v * 4 bytes. */
 KDA_API size_t kda_chunk_bwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k,
                                             int32_t d_v);
 

@@ -11,33 +11,46 @@
 //   dk = dS u + S' dr;  dalpha_i = sum_j dS'_ij S_ij;  dS_{t-1} = Diag(alpha) dS'
 //   dx = dalpha alpha (-5) sigmoid(x)(1 - sigmoid(x));  da = e^A dx;  dA_log += dx . x
 //
-// Execution: one CTA per (sequence, head), the state and its gradient in registers, the layout of
-// the decode step (a warp holds whole 512-byte rows, so row sums are warp shuffles and column sums
-// go through shared memory).  A forward pass stores the state at the start of every 64-token chunk
-// (workspace); then, chunk by chunk in reverse, the chunk's 64 states are recomputed into a
-// per-unit scratch (workspace) and the tokens are undone in reverse order.  The recurrence is
+// Every one of these steps acts on the value columns j of S and dS independently, except the row
+// sums (dq, dk, dalpha) and the dot product of dbeta, which add up over the columns.  So a unit
+// (sequence, head) runs on a cluster of d_v / 32 CTAs, each holding a d_k x 32 column slice of S and
+// dS in registers; the row sums are kept per CTA for a whole 32-token chunk in shared memory and
+// added over the cluster through distributed shared memory once per chunk (in a fixed order: the
+// result does not depend on timing).  Per token a CTA needs the column sums over d_k rows only:
+// warp shuffles plus one block barrier.  A forward pass stores the state at the start of every
+// chunk (workspace); then, chunk by chunk in reverse, the chunk's states are recomputed into a
+// per-CTA scratch (workspace) and the tokens are undone in reverse order.  The recurrence is
 // sequential in time, so this runs at the latency of its token steps.
 #pragma once
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "mma_frag.cuh"
 
 namespace kda {
 
-constexpr int kBwdThreads = 512;
-constexpr int kBwdChunk = 64;
+constexpr int kBwdThreads = 256;
+constexpr int kBwdChunk = 32;   // tokens per checkpoint / recompute chunk
+constexpr int kBwdCols = 32;    // value columns per CTA
 
-// dynamic shared memory: one chunk's inputs, staged with coalesced loads before its token steps
-template <int DK, int DV>
-struct BwdStage {
-    static constexpr int kQ = 0;                            // bf16 [64][DK]
-    static constexpr int kK = kQ + kBwdChunk * DK * 2;
-    static constexpr int kA = kK + kBwdChunk * DK * 2;
-    static constexpr int kV = kA + kBwdChunk * DK * 2;      // bf16 [64][DV]
-    static constexpr int kG = kV + kBwdChunk * DV * 2;
-    static constexpr int kD = kG + kBwdChunk * DV * 2;      // fp32 [64][DV] dout
-    static constexpr int kB = kD + kBwdChunk * DV * 4;      // fp32 [64] beta
-    static constexpr int kBytes = kB + kBwdChunk * 4;
+// Dynamic shared memory of one CTA: a chunk's inputs (and values derived from them), the chunk's
+// per-CTA row sums, and the per-warp column sums of the current token (two buffers).
+template <int DK>
+struct BwdSmem {
+    static constexpr int C = kBwdChunk, DC = kBwdCols;
+    static constexpr int kQ = 0;                          // bf16 [C][DK] q, then k, then a
+    static constexpr int kK = kQ + C * DK * 2;
+    static constexpr int kA = kK + C * DK * 2;
+    static constexpr int kAl = kA + C * DK * 2;           // f32 [C][DK] alpha
+    static constexpr int kV = kAl + C * DK * 4;           // f32 [C][DC] v (this CTA's columns)
+    static constexpr int kDo = kV + C * DC * 4;           // f32 [C][DC] dout sigmoid(gate)
+    static constexpr int kDg = kDo + C * DC * 4;          // f32 [C][DC] dout sigmoid'(gate)
+    static constexpr int kB = kDg + C * DC * 4;           // f32 [C] beta
+    static constexpr int kQK = kB + C * 4;                // f32 [C] scale q . k
+    static constexpr int kP = kQK + C * 4;                // f32 [C][3][DK] row sums: S_t do, dk, dg
+    static constexpr int kPB = kP + C * 3 * DK * 4;       // f32 [C] dbeta (this CTA's columns)
+    static constexpr int kRed = kPB + C * 4;              // f32 [2][3][8 warps][DC]
+    static constexpr int kBytes = kRed + 2 * 3 * 8 * DC * 4;
 };
 
 struct BwdParams {
@@ -48,304 +61,387 @@ struct BwdParams {
     const float *dout;                      // [T, H, d_v] fp32
     const float *dS_T;                      // [N, H, d_k, d_v] or null
     float *dq, *dk, *dv, *da, *dbeta, *dgate, *dA_log, *dS0;
-    float *ckpt;                            // [sum_n ceil(len_n / 64)][H][d_k][d_v]
-    float *scratch;                         // [N H][64][d_k][d_v]
+    float *ckpt;                            // [sum_n ceil(len_n / 32)][H][d_v / 32][d_k x 32 slice]
+    float *scratch;                         // [N H][d_v / 32][32 tokens][d_k x 32 slice]
     int64_t total_tokens;
     int num_seqs, H;
     float scale;
 };
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];\n"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float f4_dot(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
+
+__device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+// sum over the 4 row groups of a warp (lanes l, l ^ 8, l ^ 16, l ^ 24 share a column quad)
+__device__ __forceinline__ float4 warp_rows_sum(float4 x) {
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) {
+        x.x += __shfl_xor_sync(0xffffffffu, x.x, o);
+        x.y += __shfl_xor_sync(0xffffffffu, x.y, o);
+        x.z += __shfl_xor_sync(0xffffffffu, x.z, o);
+        x.w += __shfl_xor_sync(0xffffffffu, x.w, o);
+    }
+    return x;
+}
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p) {
-    constexpr int LPR = DV / 4;                // threads per state row (float4 each)
-    constexpr int RPP = kBwdThreads / LPR;     // rows per pass
-    constexpr int NR = DK / RPP;               // rows per thread
-    __shared__ float s_k[DK], s_q[DK], s_al[DK], s_x[DK];
-    __shared__ float s_vec[4][DV];             // u, v - r, do, du
-    __shared__ float4 s_red[2][RPP][LPR];
-    __shared__ float s_beta, s_dx_dot;
-    __shared__ float s_db[DV / 32];
-
-    using ST = BwdStage<DK, DV>;
+    constexpr int C = kBwdChunk, DC = kBwdCols, G = DV / DC;
+    constexpr int NR = DK / 32;                 // rows per thread: rg + 32 m
+    constexpr int NT = kBwdThreads;
+    static_assert(NR == 2 || NR == 4, "d_k must be 64 or 128");
+    using SM = BwdSmem<DK>;
     extern __shared__ __align__(16) unsigned char bsm[];
-    const uint16_t *sq = reinterpret_cast<const uint16_t *>(bsm + ST::kQ);
-    const uint16_t *sk = reinterpret_cast<const uint16_t *>(bsm + ST::kK);
-    const uint16_t *sa = reinterpret_cast<const uint16_t *>(bsm + ST::kA);
-    const uint16_t *sv = reinterpret_cast<const uint16_t *>(bsm + ST::kV);
-    const uint16_t *sg = reinterpret_cast<const uint16_t *>(bsm + ST::kG);
-    const float *sd = reinterpret_cast<const float *>(bsm + ST::kD);
-    const float *sb = reinterpret_cast<const float *>(bsm + ST::kB);
-    const int64_t unit = blockIdx.x;
+    const uint16_t *sQ = reinterpret_cast<const uint16_t *>(bsm + SM::kQ);
+    const uint16_t *sK = reinterpret_cast<const uint16_t *>(bsm + SM::kK);
+    const uint16_t *sA = reinterpret_cast<const uint16_t *>(bsm + SM::kA);
+    float *sAl = reinterpret_cast<float *>(bsm + SM::kAl);
+    float *sV = reinterpret_cast<float *>(bsm + SM::kV);
+    float *sDo = reinterpret_cast<float *>(bsm + SM::kDo);
+    float *sDg = reinterpret_cast<float *>(bsm + SM::kDg);
+    float *sB = reinterpret_cast<float *>(bsm + SM::kB);
+    float *sQK = reinterpret_cast<float *>(bsm + SM::kQK);
+    float *sP = reinterpret_cast<float *>(bsm + SM::kP);
+    float *sPB = reinterpret_cast<float *>(bsm + SM::kPB);
+    float *sRed = reinterpret_cast<float *>(bsm + SM::kRed);
+
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int64_t unit = blockIdx.x / G;
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
-    const int tid = threadIdx.x, cq = tid % LPR, rg = tid / LPR;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, cq = tid & 7, rg = tid >> 3;
     int64_t s0, s1;
     if (!seq_span(p.cu, n, p.num_seqs, p.total_tokens, s0, s1)) {
-        if (tid == 0) atomicOr(&g_kda_error_word, kErrBadSeqlens);
+        if (tid == 0 && rank == 0) atomicOr(&g_kda_error_word, kErrBadSeqlens);
     }
     const int64_t len = s1 - s0;
-    const int nck = static_cast<int>((len + kBwdChunk - 1) / kBwdChunk);
+    const int nck = static_cast<int>((len + C - 1) / C);
     int64_t ckbase = 0;   // checkpoints of the sequences before this one
     for (int m = 0; m < n; ++m) {
         int64_t a0, a1;
         seq_span(p.cu, m, p.num_seqs, p.total_tokens, a0, a1);
-        ckbase += (a1 - a0 + kBwdChunk - 1) / kBwdChunk;
+        ckbase += (a1 - a0 + C - 1) / C;
     }
     const int64_t H = p.H;
     const float expA = expf(p.A_log[h]);
-    const size_t SZ = (size_t)DK * DV;
-    float4 *scratch = reinterpret_cast<float4 *>(p.scratch + (size_t)unit * kBwdChunk * SZ);
-    auto ck_ptr = [&](int c) { return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(ckbase + c) * H + h) * SZ); };
+    const size_t SZ = (size_t)DK * DV, SL = (size_t)DK * DC;
+    const int col0 = rank * DC + 4 * cq;   // first of this thread's four value columns
+    float4 *scratch = reinterpret_cast<float4 *>(p.scratch + (size_t)unit * C * SZ + (size_t)rank * C * SL);
+    auto ck_ptr = [&](int c) {
+        return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(ckbase + c) * H + h) * SZ + (size_t)rank * SL);
+    };
 
-    // a chunk's inputs (tokens tc .. tc + L - 1) into shared memory, 16 bytes per load
+    // a chunk's inputs (tokens tc .. tc + L - 1) into shared memory, then alpha (and with the
+    // gradients: dout sigmoid(gate), dout sigmoid'(gate), scale q . k)
     auto stage = [&](int64_t tc, int L, bool grads) {
-        auto copy_rows = [&](const void *src, int off, int row_bytes) {
-            const int pieces = row_bytes / 16;
-            for (int e = tid; e < L * pieces; e += kBwdThreads) {
-                const int i = e / pieces, j = e % pieces;
-                const uint4 *g = reinterpret_cast<const uint4 *>(static_cast<const char *>(src) +
-                                                                 ((tc + i) * H + h) * (int64_t)row_bytes) + j;
-                *reinterpret_cast<uint4 *>(bsm + off + i * row_bytes + j * 16) = __ldg(g);
-            }
-        };
-        copy_rows(p.q, ST::kQ, DK * 2);
-        copy_rows(p.k, ST::kK, DK * 2);
-        copy_rows(p.a, ST::kA, DK * 2);
-        copy_rows(p.v, ST::kV, DV * 2);
+        __syncthreads();   // the previous chunk's readers are done
+        constexpr int PR = DK * 2 / 16;
+        for (int e = tid; e < 3 * L * PR; e += NT) {
+            const int which = e / (L * PR), r = e % (L * PR), i = r / PR, j = r % PR;
+            const uint16_t *src = which == 0 ? p.q : (which == 1 ? p.k : p.a);
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + ((tc + i) * H + h) * DK) + j);
+            *reinterpret_cast<uint4 *>(bsm + SM::kQ + which * (C * DK * 2) + i * (DK * 2) + j * 16) = x;
+        }
+        for (int e = tid; e < L * (DC / 8); e += NT) {
+            const int i = e / (DC / 8), j = e % (DC / 8);
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(p.v + ((tc + i) * H + h) * DV + rank * DC) + j);
+            float4 *d = reinterpret_cast<float4 *>(sV + i * DC + j * 8);
+            d[0] = make_float4(bf16_to_f32(x.x & 0xffff), bf16_to_f32(x.x >> 16), bf16_to_f32(x.y & 0xffff),
+                               bf16_to_f32(x.y >> 16));
+            d[1] = make_float4(bf16_to_f32(x.z & 0xffff), bf16_to_f32(x.z >> 16), bf16_to_f32(x.w & 0xffff),
+                               bf16_to_f32(x.w >> 16));
+        }
+        for (int i = tid; i < L; i += NT) sB[i] = p.beta[(tc + i) * H + h];
         if (grads) {
-            if (p.gate) copy_rows(p.gate, ST::kG, DV * 2);
-            copy_rows(p.dout, ST::kD, DV * 4);
-        }
-        for (int i = tid; i < L; i += kBwdThreads)
-            reinterpret_cast<float *>(bsm + ST::kB)[i] = p.beta[(tc + i) * H + h];
-    };
-    // token i of the staged chunk: alpha and x per key channel, k, scale q, beta
-    auto load_tok = [&](int i) {
-        for (int c = tid; c < DK; c += kBwdThreads) {
-            const float x = expA * bf16_to_f32(sa[i * DK + c]);
-            s_x[c] = x;
-            s_al[c] = __expf(kGMin * sigmoid_fast(x));
-            s_k[c] = bf16_to_f32(sk[i * DK + c]);
-            s_q[c] = p.scale * bf16_to_f32(sq[i * DK + c]);
-        }
-        if (tid == 0) s_beta = sb[i];
-    };
-    // column sums over the rows of two per-thread partial vectors (through shared memory)
-    auto col_sums = [&](float4 a0, float4 a1, float &c0, float &c1) {
-        s_red[0][rg][cq] = a0;
-        s_red[1][rg][cq] = a1;
-        __syncthreads();
-        c0 = c1 = 0.f;
-        if (tid < DV) {
-            const float *r0 = reinterpret_cast<const float *>(&s_red[0][0][0]);
-            const float *r1 = reinterpret_cast<const float *>(&s_red[1][0][0]);
-#pragma unroll 4
-            for (int g = 0; g < RPP; ++g) {
-                c0 += r0[g * DV + tid];
-                c1 += r1[g * DV + tid];
+            for (int e = tid; e < L * (DC / 4); e += NT) {
+                const int i = e / (DC / 4), j = e % (DC / 4);
+                const int64_t off = ((tc + i) * H + h) * DV + rank * DC + 4 * j;
+                float4 d = __ldg(reinterpret_cast<const float4 *>(p.dout + off));
+                float4 dg = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p.gate) {
+                    const uint2 gr = __ldg(reinterpret_cast<const uint2 *>(p.gate + off));
+                    const float g0 = sigmoid_fast(bf16_to_f32(gr.x & 0xffff)), g1 = sigmoid_fast(bf16_to_f32(gr.x >> 16));
+                    const float g2 = sigmoid_fast(bf16_to_f32(gr.y & 0xffff)), g3 = sigmoid_fast(bf16_to_f32(gr.y >> 16));
+                    dg = make_float4(d.x * g0 * (1.f - g0), d.y * g1 * (1.f - g1), d.z * g2 * (1.f - g2),
+                                     d.w * g3 * (1.f - g3));
+                    d = make_float4(d.x * g0, d.y * g1, d.z * g2, d.w * g3);
+                }
+                reinterpret_cast<float4 *>(sDo + i * DC)[j] = d;
+                reinterpret_cast<float4 *>(sDg + i * DC)[j] = dg;
             }
         }
+        __syncthreads();
+        for (int e = tid; e < L * DK; e += NT) sAl[e] = __expf(kGMin * sigmoid_fast(expA * bf16_to_f32(sA[e])));
+        if (grads) {
+            for (int i = warp; i < L; i += NT / 32) {
+                float s = 0.f;
+                for (int c = lane; c < DK; c += 32) s += bf16_to_f32(sQ[i * DK + c]) * bf16_to_f32(sK[i * DK + c]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane == 0) sQK[i] = p.scale * s;
+            }
+        }
+        __syncthreads();
     };
-    // forward step S <- Diag(alpha) S + k u^T, with u = beta (v - (Diag(alpha) S)^T k); the token's
-    // inputs are in shared memory; u goes to s_vec[0] and v - r to s_vec[1]
-    auto fwd_step = [&](float4 (&S)[NR], int i) {
+
+    int buf = 0;   // which of the two column-sum buffers the next token uses
+    // forward step of token i: S <- S' + k u^T, S' = Diag(alpha) S, u = beta (v - S'^T k); S' is
+    // stored to `save` when given
+    auto fwd_tok = [&](float4 (&S)[NR], int i, float4 *save) {
+        float kk[NR];
         float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int m = 0; m < NR; ++m) {
-            const int row = rg + m * RPP;
-            const float al = s_al[row];
+            const int row = rg + 32 * m;
+            const float al = sAl[i * DK + row];
+            kk[m] = bf16_to_f32(sK[i * DK + row]);
             S[m].x *= al; S[m].y *= al; S[m].z *= al; S[m].w *= al;
-            r = f4_fma(s_k[row], S[m], r);
+            if (save) save[m * NT + tid] = S[m];
+            r = f4_fma(kk[m], S[m], r);
         }
-        float rc, unused;
-        col_sums(r, r, rc, unused);
-        if (tid < DV) {
-            const float vmr = bf16_to_f32(sv[i * DV + tid]) - rc;
-            s_vec[1][tid] = vmr;
-            s_vec[0][tid] = s_beta * vmr;
-        }
+        r = warp_rows_sum(r);
+        float *red = sRed + buf * (3 * 8 * DC);
+        if (lane < 8) reinterpret_cast<float4 *>(red + warp * DC)[cq] = r;
         __syncthreads();
-        const float4 u4 = reinterpret_cast<const float4 *>(s_vec[0])[cq];
+        float4 rt = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int m = 0; m < NR; ++m) {
-            const float kk = s_k[rg + m * RPP];
-            S[m].x = fmaf(kk, u4.x, S[m].x); S[m].y = fmaf(kk, u4.y, S[m].y);
-            S[m].z = fmaf(kk, u4.z, S[m].z); S[m].w = fmaf(kk, u4.w, S[m].w);
-        }
+        for (int w = 0; w < 8; ++w) rt = f4_add(rt, reinterpret_cast<const float4 *>(red + w * DC)[cq]);
+        buf ^= 1;
+        const float b = sB[i];
+        const float4 v = reinterpret_cast<const float4 *>(sV + i * DC)[cq];
+        const float4 u = make_float4(b * (v.x - rt.x), b * (v.y - rt.y), b * (v.z - rt.z), b * (v.w - rt.w));
+#pragma unroll
+        for (int m = 0; m < NR; ++m) S[m] = f4_fma(kk[m], u, S[m]);
     };
 
     // ---- forward pass: the state at the start of every chunk ---------------------------------
     float4 S[NR];
-    const float4 *S0p = p.S0 ? reinterpret_cast<const float4 *>(p.S0 + (size_t)unit * SZ) : nullptr;
+    {
+        const float *S0p = p.S0 ? p.S0 + (size_t)unit * SZ : nullptr;
 #pragma unroll
-    for (int m = 0; m < NR; ++m) S[m] = S0p ? S0p[(rg + m * RPP) * LPR + cq] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = 0; m < NR; ++m)
+            S[m] = S0p ? *reinterpret_cast<const float4 *>(S0p + (size_t)(rg + 32 * m) * DV + col0)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     for (int c = 0; c < nck; ++c) {
-        const int64_t tc = s0 + (int64_t)c * kBwdChunk;
-        const int L = static_cast<int>(min64(kBwdChunk, s1 - tc));
         float4 *ck = ck_ptr(c);
 #pragma unroll
-        for (int m = 0; m < NR; ++m) ck[(rg + m * RPP) * LPR + cq] = S[m];
-        stage(tc, L, false);
-        __syncthreads();
-        for (int i = 0; i < L; ++i) {
-            load_tok(i);
-            __syncthreads();
-            fwd_step(S, i);
-            __syncthreads();
-        }
+        for (int m = 0; m < NR; ++m) ck[m * NT + tid] = S[m];
+        if (c + 1 == nck) break;   // the state after the last chunk is not needed
+        const int64_t tc = s0 + (int64_t)c * C;
+        stage(tc, C, false);
+        for (int i = 0; i < C; ++i) fwd_tok(S, i, nullptr);
     }
 
     // ---- backward, chunk by chunk in reverse ----------------------------------------------------
     float4 dS[NR];
-    const float4 *dST = p.dS_T ? reinterpret_cast<const float4 *>(p.dS_T + (size_t)unit * SZ) : nullptr;
+    {
+        const float *dTp = p.dS_T ? p.dS_T + (size_t)unit * SZ : nullptr;
 #pragma unroll
-    for (int m = 0; m < NR; ++m) dS[m] = dST ? dST[(rg + m * RPP) * LPR + cq] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = 0; m < NR; ++m)
+            dS[m] = dTp ? *reinterpret_cast<const float4 *>(dTp + (size_t)(rg + 32 * m) * DV + col0)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float dA_acc = 0.f;
+    const uint32_t pBase = smem_u32(sP), pbBase = smem_u32(sPB);
     for (int c = nck - 1; c >= 0; --c) {
-        const int64_t tc = s0 + (int64_t)c * kBwdChunk;
-        const int L = static_cast<int>(min64(kBwdChunk, s1 - tc));
-        // recompute the chunk's states: scratch[i] = state before token tc + i
+        const int64_t tc = s0 + (int64_t)c * C;
+        const int L = static_cast<int>(min64(C, s1 - tc));
         const float4 *ck = ck_ptr(c);
 #pragma unroll
-        for (int m = 0; m < NR; ++m) S[m] = ck[(rg + m * RPP) * LPR + cq];
+        for (int m = 0; m < NR; ++m) S[m] = ck[m * NT + tid];
         stage(tc, L, true);
-        __syncthreads();
-        for (int i = 0; i < L; ++i) {
+        // recompute the chunk: scratch[i] = S' of token tc + i (this thread's part; read back by it)
+        for (int i = 0; i + 1 < L; ++i) fwd_tok(S, i, scratch + (size_t)i * NR * NT);
 #pragma unroll
-            for (int m = 0; m < NR; ++m) scratch[(size_t)i * (SZ / 4) + (rg + m * RPP) * LPR + cq] = S[m];
-            if (i + 1 == L) break;   // the state after the last token is not needed
-            load_tok(i);
-            __syncthreads();
-            fwd_step(S, i);
-            __syncthreads();
+        for (int m = 0; m < NR; ++m) {
+            const float al = sAl[(L - 1) * DK + rg + 32 * m];
+            scratch[(size_t)((L - 1) * NR + m) * NT + tid] =
+                make_float4(al * S[m].x, al * S[m].y, al * S[m].z, al * S[m].w);
         }
         // undo the chunk's tokens in reverse order
+        float4 Spn[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) Spn[m] = scratch[(size_t)((L - 1) * NR + m) * NT + tid];
         for (int i = L - 1; i >= 0; --i) {
-            const int64_t t = tc + i;
-            const int64_t tv = (t * H + h) * DV;
-            float4 Sp[NR];   // S' = Diag(alpha) S_{t-1}
+            float4 Sp[NR];
 #pragma unroll
-            for (int m = 0; m < NR; ++m) Sp[m] = scratch[(size_t)i * (SZ / 4) + (rg + m * RPP) * LPR + cq];
-            load_tok(i);
-            __syncthreads();
-            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int m = 0; m < NR; ++m) Sp[m] = Spn[m];
+            if (i > 0) {
 #pragma unroll
-            for (int m = 0; m < NR; ++m) {
-                const int row = rg + m * RPP;
-                const float al = s_al[row];
-                Sp[m].x *= al; Sp[m].y *= al; Sp[m].z *= al; Sp[m].w *= al;
-                r = f4_fma(s_k[row], Sp[m], r);
+                for (int m = 0; m < NR; ++m) Spn[m] = scratch[(size_t)((i - 1) * NR + m) * NT + tid];
             }
-            float rc, unused;
-            col_sums(r, r, rc, unused);
-            if (tid < DV) {
-                const float vmr = bf16_to_f32(sv[i * DV + tid]) - rc;
-                s_vec[1][tid] = vmr;
-                s_vec[0][tid] = s_beta * vmr;
-            }
-            __syncthreads();
-            // o = S_t^T (scale q) with S_t = S' + k u^T:  o = S'^T (scale q) + (k . scale q) u
-            const float4 u4 = reinterpret_cast<const float4 *>(s_vec[0])[cq];
-            float4 pq = make_float4(0.f, 0.f, 0.f, 0.f), du = pq;
+            float kk[NR], qq[NR], al[NR];
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f), pq = r, dko = r;
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
-                const int row = rg + m * RPP;
-                const float kk = s_k[row], qq = s_q[row];
-                float4 St = Sp[m];
-                St.x = fmaf(kk, u4.x, St.x); St.y = fmaf(kk, u4.y, St.y);
-                St.z = fmaf(kk, u4.z, St.z); St.w = fmaf(kk, u4.w, St.w);
-                pq = f4_fma(qq, St, pq);
+                const int row = rg + 32 * m;
+                kk[m] = bf16_to_f32(sK[i * DK + row]);
+                qq[m] = p.scale * bf16_to_f32(sQ[i * DK + row]);
+                al[m] = sAl[i * DK + row];
+                r = f4_fma(kk[m], Sp[m], r);
+                pq = f4_fma(qq[m], Sp[m], pq);
+                dko = f4_fma(kk[m], dS[m], dko);
             }
-            float oc;
-            col_sums(pq, pq, oc, unused);
-            if (tid < DV) {
-                const float dout = sd[i * DV + tid];
-                float dov = dout;
-                if (p.gate) {
-                    const float sgv = sigmoid_fast(bf16_to_f32(sg[i * DV + tid]));
-                    p.dgate[tv + tid] = dout * oc * sgv * (1.f - sgv);
-                    dov = dout * sgv;
+            r = warp_rows_sum(r);
+            pq = warp_rows_sum(pq);
+            dko = warp_rows_sum(dko);
+            float *red = sRed + buf * (3 * 8 * DC);
+            if (lane < 8) {
+                reinterpret_cast<float4 *>(red + warp * DC)[cq] = r;
+                reinterpret_cast<float4 *>(red + (8 + warp) * DC)[cq] = pq;
+                reinterpret_cast<float4 *>(red + (16 + warp) * DC)[cq] = dko;
+            }
+            __syncthreads();
+            float4 rt = make_float4(0.f, 0.f, 0.f, 0.f), pqt = rt, dkt = rt;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                rt = f4_add(rt, reinterpret_cast<const float4 *>(red + w * DC)[cq]);
+                pqt = f4_add(pqt, reinterpret_cast<const float4 *>(red + (8 + w) * DC)[cq]);
+                dkt = f4_add(dkt, reinterpret_cast<const float4 *>(red + (16 + w) * DC)[cq]);
+            }
+            buf ^= 1;
+            const float b = sB[i], qk = sQK[i];
+            const float4 v = reinterpret_cast<const float4 *>(sV + i * DC)[cq];
+            const float4 do4 = reinterpret_cast<const float4 *>(sDo + i * DC)[cq];
+            const float4 vmr = make_float4(v.x - rt.x, v.y - rt.y, v.z - rt.z, v.w - rt.w);
+            const float4 u = make_float4(b * vmr.x, b * vmr.y, b * vmr.z, b * vmr.w);
+            // du = (dS + scale q do^T)^T k = dS^T k + (scale q . k) do
+            const float4 du = f4_fma(qk, do4, dkt);
+            if (tid < 8) {   // row group 0 of warp 0 holds every column of the CTA once
+                const int64_t ov = ((tc + i) * H + h) * DV + col0;
+                *reinterpret_cast<float4 *>(p.dv + ov) = make_float4(b * du.x, b * du.y, b * du.z, b * du.w);
+                if (p.gate) {   // o = S_t^T (scale q) = S'^T (scale q) + (scale q . k) u
+                    const float4 o = f4_fma(qk, u, pqt);
+                    const float4 dg = reinterpret_cast<const float4 *>(sDg + i * DC)[cq];
+                    *reinterpret_cast<float4 *>(p.dgate + ov) = make_float4(dg.x * o.x, dg.y * o.y, dg.z * o.z, dg.w * o.w);
                 }
-                s_vec[2][tid] = dov;
             }
-            __syncthreads();
-            // dS += (scale q) do^T; then du = dS^T k
-            const float4 do4 = reinterpret_cast<const float4 *>(s_vec[2])[cq];
+            if (warp == 0) {   // dbeta over this CTA's columns
+                float db = f4_dot(du, vmr);
+                db += __shfl_xor_sync(0xffffffffu, db, 1);
+                db += __shfl_xor_sync(0xffffffffu, db, 2);
+                db += __shfl_xor_sync(0xffffffffu, db, 4);
+                if (lane == 0) sPB[i] = db;
+            }
+            const float udo = f4_dot(u, do4);
+            float vals[3 * NR];
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
-                const int row = rg + m * RPP;
-                const float qq = s_q[row];
-                dS[m].x = fmaf(qq, do4.x, dS[m].x); dS[m].y = fmaf(qq, do4.y, dS[m].y);
-                dS[m].z = fmaf(qq, do4.z, dS[m].z); dS[m].w = fmaf(qq, do4.w, dS[m].w);
-                du = f4_fma(s_k[row], dS[m], du);
+                const float4 dSn = f4_fma(qq[m], do4, dS[m]);
+                const float sdu = f4_dot(Sp[m], du);
+                vals[3 * m + 0] = f4_dot(Sp[m], do4) + kk[m] * udo;         // (S_t do)_row
+                vals[3 * m + 1] = f4_dot(dSn, u) - b * sdu;                 // dk_row
+                vals[3 * m + 2] = f4_dot(dSn, Sp[m]) - b * kk[m] * sdu;     // dalpha_row alpha_row
+                const float4 dSp = f4_fma(-b * kk[m], du, dSn);
+                dS[m] = make_float4(al[m] * dSp.x, al[m] * dSp.y, al[m] * dSp.z, al[m] * dSp.w);
             }
-            float duc;
-            col_sums(du, du, duc, unused);
-            if (tid < DV) {
-                s_vec[3][tid] = duc;
-                p.dv[tv + tid] = s_beta * duc;
+            // sum the row values over the 8 lanes of a row (lanes differ in bits 0..2), leaving each
+            // lane pair (quad for NR = 2) with the three sums of one row
+            const int b4 = (lane >> 2) & 1;
+            float w1[3 * NR / 2];
+#pragma unroll
+            for (int k2 = 0; k2 < 3 * NR / 2; ++k2) {
+                const float send = b4 ? vals[k2] : vals[k2 + 3 * NR / 2];
+                const float keep = b4 ? vals[k2 + 3 * NR / 2] : vals[k2];
+                w1[k2] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
             }
-            if (tid == 0) s_dx_dot = 0.f;
-            __syncthreads();
-            // row sums: dq = S_t do, dk = dS u + S' dr (dr = -beta du), dalpha = rowsum(dS' (.) S_{t-1});
-            // then dS <- Diag(alpha) (dS + k dr^T)
-            const float4 du4 = reinterpret_cast<const float4 *>(s_vec[3])[cq];
-            const float bt = s_beta;
-            float dbeta_part = 0.f;
-            if (tid < DV) dbeta_part = s_vec[3][tid] * s_vec[1][tid];
+            if constexpr (NR == 4) {
+                const int b2 = (lane >> 1) & 1;
+                float w2[3];
 #pragma unroll
-            for (int m = 0; m < NR; ++m) {
-                const int row = rg + m * RPP;
-                const float kk = s_k[row], al = s_al[row];
-                float4 St = Sp[m];
-                St.x = fmaf(kk, u4.x, St.x); St.y = fmaf(kk, u4.y, St.y);
-                St.z = fmaf(kk, u4.z, St.z); St.w = fmaf(kk, u4.w, St.w);
-                float dqp = St.x * do4.x + St.y * do4.y + St.z * do4.z + St.w * do4.w;
-                float dkp = dS[m].x * u4.x + dS[m].y * u4.y + dS[m].z * u4.z + dS[m].w * u4.w
-                          - bt * (Sp[m].x * du4.x + Sp[m].y * du4.y + Sp[m].z * du4.z + Sp[m].w * du4.w);
-                float4 dSp = dS[m];
-                dSp.x -= bt * kk * du4.x; dSp.y -= bt * kk * du4.y;
-                dSp.z -= bt * kk * du4.z; dSp.w -= bt * kk * du4.w;
-                // dalpha_i = sum_j dS'_ij S_{t-1,ij} = sum_j dS'_ij S'_ij / alpha_i
-                float dap = dSp.x * Sp[m].x + dSp.y * Sp[m].y + dSp.z * Sp[m].z + dSp.w * Sp[m].w;
-#pragma unroll
-                for (int o = LPR / 2; o > 0; o >>= 1) {
-                    dqp += __shfl_xor_sync(0xffffffffu, dqp, o);
-                    dkp += __shfl_xor_sync(0xffffffffu, dkp, o);
-                    dap += __shfl_xor_sync(0xffffffffu, dap, o);
+                for (int k2 = 0; k2 < 3; ++k2) {
+                    const float send = b2 ? w1[k2] : w1[k2 + 3];
+                    const float keep = b2 ? w1[k2 + 3] : w1[k2];
+                    w2[k2] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    w2[k2] += __shfl_xor_sync(0xffffffffu, w2[k2], 1);
                 }
-                if (cq == 0) {
-                    const int64_t tk = (t * H + h) * DK + row;
-                    p.dq[tk] = p.scale * dqp;
-                    p.dk[tk] = dkp;
-                    const float x = s_x[row];
-                    const float sx = sigmoid_fast(x);
-                    // dalpha = dap / alpha; dg = dalpha alpha = dap
-                    const float dx = dap * kGMin * sx * (1.f - sx);
-                    p.da[tk] = dx * expA;
-                    atomicAdd(&s_dx_dot, dx * x);
+                if ((lane & 1) == 0) {
+                    const int row = rg + 32 * (2 * b4 + b2);
+#pragma unroll
+                    for (int q3 = 0; q3 < 3; ++q3) sP[(i * 3 + q3) * DK + row] = w2[q3];
                 }
-                dS[m].x = al * dSp.x; dS[m].y = al * dSp.y; dS[m].z = al * dSp.z; dS[m].w = al * dSp.w;
-            }
-            // dbeta = du . (v - r)
+            } else {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) dbeta_part += __shfl_xor_sync(0xffffffffu, dbeta_part, o);
-            if (tid < DV && (tid & 31) == 0) s_db[tid >> 5] = dbeta_part;
-            __syncthreads();
-            if (tid == 0) {
-                float db = 0.f;
+                for (int k2 = 0; k2 < 3; ++k2) {
+                    w1[k2] += __shfl_xor_sync(0xffffffffu, w1[k2], 2);
+                    w1[k2] += __shfl_xor_sync(0xffffffffu, w1[k2], 1);
+                }
+                if ((lane & 3) == 0) {
+                    const int row = rg + 32 * b4;
 #pragma unroll
-                for (int w = 0; w < DV / 32; ++w) db += s_db[w];
-                p.dbeta[t * H + h] = db;
-                dA_acc += s_dx_dot;
+                    for (int q3 = 0; q3 < 3; ++q3) sP[(i * 3 + q3) * DK + row] = w1[q3];
+                }
             }
-            __syncthreads();
         }
-    }
-    if (tid == 0) atomicAdd(p.dA_log + h, dA_acc);
-    if (p.dS0) {
-        float4 *d0 = reinterpret_cast<float4 *>(p.dS0 + (size_t)unit * SZ);
+        // add the row sums over the cluster: this CTA finishes tokens i = rank (mod G)
+        cluster_sync();
+        const int mine = (L - rank + G - 1) / G;
+        for (int e = tid; e < mine * (DK / 4); e += NT) {
+            const int i = rank + G * (e / (DK / 4)), c4 = 4 * (e % (DK / 4));
+            float4 acc[3];
 #pragma unroll
-        for (int m = 0; m < NR; ++m) d0[(rg + m * RPP) * LPR + cq] = dS[m];
+            for (int q3 = 0; q3 < 3; ++q3) acc[q3] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+#pragma unroll
+                for (int q3 = 0; q3 < 3; ++q3)
+                    acc[q3] = f4_add(acc[q3], ld_cluster_f4(mapa_shared(pBase + ((i * 3 + q3) * DK + c4) * 4, g)));
+            }
+            const int64_t ok = ((tc + i) * H + h) * DK + c4;
+            *reinterpret_cast<float4 *>(p.dq + ok) =
+                make_float4(p.scale * acc[0].x, p.scale * acc[0].y, p.scale * acc[0].z, p.scale * acc[0].w);
+            *reinterpret_cast<float4 *>(p.dk + ok) = acc[1];
+            const float dg[4] = {acc[2].x, acc[2].y, acc[2].z, acc[2].w};
+            float da[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float x = expA * bf16_to_f32(sA[i * DK + c4 + j]);
+                const float sx = sigmoid_fast(x);
+                const float dx = dg[j] * kGMin * sx * (1.f - sx);
+                da[j] = dx * expA;
+                dA_acc = fmaf(dx, x, dA_acc);
+            }
+            *reinterpret_cast<float4 *>(p.da + ok) = make_float4(da[0], da[1], da[2], da[3]);
+        }
+        if (tid < mine) {
+            const int i = rank + G * tid;
+            float db = 0.f;
+#pragma unroll
+            for (int g = 0; g < G; ++g) db += ld_cluster_f32(mapa_shared(pbBase + i * 4, g));
+            p.dbeta[(tc + i) * H + h] = db;
+        }
+        cluster_sync();   // every CTA is done reading the row sums before they are overwritten
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dA_acc += __shfl_xor_sync(0xffffffffu, dA_acc, o);
+    if (lane == 0 && dA_acc != 0.f) atomicAdd(p.dA_log + h, dA_acc);
+    if (p.dS0) {
+        float *d0 = p.dS0 + (size_t)unit * SZ;
+#pragma unroll
+        for (int m = 0; m < NR; ++m) *reinterpret_cast<float4 *>(d0 + (size_t)(rg + 32 * m) * DV + col0) = dS[m];
     }
 }
 

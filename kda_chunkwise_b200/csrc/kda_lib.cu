@@ -111,13 +111,26 @@ kda_status dispatch_spec(const kda::SpecParams &p, int64_t units, int d_k, int d
 
 template <int DK, int DV>
 kda_status launch_bwd(const kda::BwdParams &p, int64_t units, cudaStream_t stream) {
-    const int smem = kda::BwdStage<DK, DV>::kBytes;
+    constexpr int G = DV / kda::kBwdCols;   // CTAs per unit: one per 32 value columns
+    const int smem = kda::BwdSmem<DK>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kda::kda_bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chunk_bwd)");
-    kda::kda_bwd_kernel<DK, DV><<<(unsigned)units, kda::kBwdThreads, smem, stream>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units * G));
+    cfg.blockDim = dim3(kda::kBwdThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kda::kda_bwd_kernel<DK, DV>, p);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_bwd launch");
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    e = cudaGetLastError();
-    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "chunk_bwd launch");
+    return KDA_OK;
 }
 
 // Built-in scratch for kda_chunk_fwd_noalloc (callers that cannot allocate).  Host code must not
@@ -484,7 +497,7 @@ kda_status kda_state_combine(const float *M, const float *S_in, const float *B, 
 size_t kda_chunk_bwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v) {
     if (total_tokens < 0 || num_seqs < 0 || H <= 0 || !supported_dim(d_k) || !supported_dim(d_v)) return 0;
     const size_t state = (size_t)d_k * d_v * 4;
-    const size_t ckpts = (size_t)(total_tokens / kda::kBwdChunk + num_seqs) * H;   // >= sum ceil(len / 64)
+    const size_t ckpts = (size_t)(total_tokens / kda::kBwdChunk + num_seqs) * H;   // >= sum ceil(len / 32)
     const size_t scratch = (size_t)num_seqs * H * kda::kBwdChunk;
     return (ckpts + scratch) * state;
 }
@@ -517,7 +530,7 @@ kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void
     if (!workspace || workspace_bytes < need)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: workspace missing or too small (need " + std::to_string(need) + " bytes)");
     const int64_t units = (int64_t)num_seqs * H;
-    if (units > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: num_seqs * H too large");
+    if (units * (d_v / kda::kBwdCols) > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: num_seqs * H too large");
     kda::BwdParams p{};
     p.q = static_cast<const uint16_t *>(q);
     p.k = static_cast<const uint16_t *>(k);

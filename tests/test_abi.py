@@ -166,4 +166,4 @@ def test_chunk_bwd_rejects_bad_arguments():
     assert bwd(wsb=10) == kda.KDA_ERR_INVALID_ARG                 # workspace too small
     assert bwd(q=8) == kda.KDA_ERR_INVALID_ARG                    # misaligned
     assert bwd(N=0, T=0) == kda.KDA_OK
-    assert kda.kda_chunk_bwd_workspace_size(8192, 1, 32, 128, 128) == (8192 // 64 + 1 + 64) * 32 * 128 * 128 * 4
+    assert kda.kda_chunk_bwd_workspace_size(8192, 1, 32, 128, 128) == (8192 // 32 + 1 + 32) * 32 * 128 * 128 * 4
