@@ -33,20 +33,27 @@ constexpr int kBwdThreads = 256;
 constexpr int kBwdChunk = 32;   // tokens per checkpoint / recompute chunk
 constexpr int kBwdCols = 32;    // value columns per CTA
 
-// Dynamic shared memory of one CTA: a chunk's inputs (and values derived from them), the chunk's
-// per-CTA row sums, and the per-warp column sums of the current token (two buffers).
+// Dynamic shared memory of one CTA: two buffers of a chunk's raw inputs (the next chunk's are
+// copied in asynchronously while the current one runs), values derived from the current chunk, the
+// chunk's per-CTA row sums, and the per-warp column sums of the current token (two buffers).
 template <int DK>
 struct BwdSmem {
     static constexpr int C = kBwdChunk, DC = kBwdCols;
-    static constexpr int kQ = 0;                          // bf16 [C][DK] q, then k, then a
-    static constexpr int kK = kQ + C * DK * 2;
-    static constexpr int kA = kK + C * DK * 2;
-    static constexpr int kAl = kA + C * DK * 2;           // f32 [C][DK] alpha
-    static constexpr int kV = kAl + C * DK * 4;           // f32 [C][DC] v (this CTA's columns)
+    // raw buffer (offsets within one buffer)
+    static constexpr int kRQ = 0;                         // bf16 [C][DK] q, then k, then a
+    static constexpr int kRK = kRQ + C * DK * 2;
+    static constexpr int kRA = kRK + C * DK * 2;
+    static constexpr int kRV = kRA + C * DK * 2;          // bf16 [C][DC] v (this CTA's columns)
+    static constexpr int kRG = kRV + C * DC * 2;          // bf16 [C][DC] gate logits
+    static constexpr int kRD = kRG + C * DC * 2;          // f32 [C][DC] dout
+    static constexpr int kRB = kRD + C * DC * 4;          // f32 [C] beta
+    static constexpr int kRaw = kRB + C * 4;
+    // derived values and sums
+    static constexpr int kAl = 2 * kRaw;                  // f32 [C][DK] alpha
+    static constexpr int kV = kAl + C * DK * 4;           // f32 [C][DC] v
     static constexpr int kDo = kV + C * DC * 4;           // f32 [C][DC] dout sigmoid(gate)
     static constexpr int kDg = kDo + C * DC * 4;          // f32 [C][DC] dout sigmoid'(gate)
-    static constexpr int kB = kDg + C * DC * 4;           // f32 [C] beta
-    static constexpr int kQK = kB + C * 4;                // f32 [C] scale q . k
+    static constexpr int kQK = kDg + C * DC * 4;          // f32 [C] scale q . k
     static constexpr int kP = kQK + C * 4;                // f32 [C][3][DK] row sums: S_t do, dk, dg
     static constexpr int kPB = kP + C * 3 * DK * 4;       // f32 [C] dbeta (this CTA's columns)
     static constexpr int kRed = kPB + C * 4;              // f32 [2][3][8 warps][DC]
@@ -89,6 +96,14 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
     return v;
 }
 
+// 4-byte asynchronous global->shared copy
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+}
+
+// streaming (evict-first) store of a gradient that is never read again here
+__device__ __forceinline__ void st_stream(float *p, float4 v) { __stcs(reinterpret_cast<float4 *>(p), v); }
+
 __device__ __forceinline__ float f4_dot(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
 
 __device__ __forceinline__ float4 f4_add(float4 a, float4 b) {
@@ -115,14 +130,10 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
     static_assert(NR == 2 || NR == 4, "d_k must be 64 or 128");
     using SM = BwdSmem<DK>;
     extern __shared__ __align__(16) unsigned char bsm[];
-    const uint16_t *sQ = reinterpret_cast<const uint16_t *>(bsm + SM::kQ);
-    const uint16_t *sK = reinterpret_cast<const uint16_t *>(bsm + SM::kK);
-    const uint16_t *sA = reinterpret_cast<const uint16_t *>(bsm + SM::kA);
     float *sAl = reinterpret_cast<float *>(bsm + SM::kAl);
     float *sV = reinterpret_cast<float *>(bsm + SM::kV);
     float *sDo = reinterpret_cast<float *>(bsm + SM::kDo);
     float *sDg = reinterpret_cast<float *>(bsm + SM::kDg);
-    float *sB = reinterpret_cast<float *>(bsm + SM::kB);
     float *sQK = reinterpret_cast<float *>(bsm + SM::kQK);
     float *sP = reinterpret_cast<float *>(bsm + SM::kP);
     float *sPB = reinterpret_cast<float *>(bsm + SM::kPB);
@@ -153,51 +164,66 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
         return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(ckbase + c) * H + h) * SZ + (size_t)rank * SL);
     };
 
-    // a chunk's inputs (tokens tc .. tc + L - 1) into shared memory, then alpha (and with the
-    // gradients: dout sigmoid(gate), dout sigmoid'(gate), scale q . k)
-    auto stage = [&](int64_t tc, int L, bool grads) {
-        __syncthreads();   // the previous chunk's readers are done
+    // The work is a list of jobs: the forward pass over chunks 0 .. nck - 2, then the backward over
+    // chunks nck - 1 .. 0.  The raw inputs of job j + 1 are copied in while job j runs.
+    const int nfwd = nck > 0 ? nck - 1 : 0, njobs = nfwd + nck;
+    auto job_chunk = [&](int j) { return j < nfwd ? j : nck - 1 - (j - nfwd); };
+    auto issue = [&](int j, int rb) {   // asynchronous copy of job j's raw inputs into buffer rb
+        const bool grads = j >= nfwd;
+        const int64_t tc = s0 + (int64_t)job_chunk(j) * C;
+        const int L = static_cast<int>(min64(C, s1 - tc));
+        const uint32_t raw = smem_u32(bsm + rb * SM::kRaw);
         constexpr int PR = DK * 2 / 16;
         for (int e = tid; e < 3 * L * PR; e += NT) {
-            const int which = e / (L * PR), r = e % (L * PR), i = r / PR, j = r % PR;
+            const int which = e / (L * PR), r = e % (L * PR), i = r / PR, j16 = r % PR;
             const uint16_t *src = which == 0 ? p.q : (which == 1 ? p.k : p.a);
-            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + ((tc + i) * H + h) * DK) + j);
-            *reinterpret_cast<uint4 *>(bsm + SM::kQ + which * (C * DK * 2) + i * (DK * 2) + j * 16) = x;
+            cp_async_16(raw + SM::kRQ + which * (C * DK * 2) + i * (DK * 2) + j16 * 16,
+                        src + ((tc + i) * H + h) * DK + j16 * 8, 16);
         }
         for (int e = tid; e < L * (DC / 8); e += NT) {
-            const int i = e / (DC / 8), j = e % (DC / 8);
-            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(p.v + ((tc + i) * H + h) * DV + rank * DC) + j);
-            float4 *d = reinterpret_cast<float4 *>(sV + i * DC + j * 8);
-            d[0] = make_float4(bf16_to_f32(x.x & 0xffff), bf16_to_f32(x.x >> 16), bf16_to_f32(x.y & 0xffff),
-                               bf16_to_f32(x.y >> 16));
-            d[1] = make_float4(bf16_to_f32(x.z & 0xffff), bf16_to_f32(x.z >> 16), bf16_to_f32(x.w & 0xffff),
-                               bf16_to_f32(x.w >> 16));
+            const int i = e / (DC / 8), j16 = e % (DC / 8);
+            cp_async_16(raw + SM::kRV + i * (DC * 2) + j16 * 16, p.v + ((tc + i) * H + h) * DV + rank * DC + j16 * 8, 16);
+            if (grads && p.gate)
+                cp_async_16(raw + SM::kRG + i * (DC * 2) + j16 * 16,
+                            p.gate + ((tc + i) * H + h) * DV + rank * DC + j16 * 8, 16);
         }
-        for (int i = tid; i < L; i += NT) sB[i] = p.beta[(tc + i) * H + h];
         if (grads) {
             for (int e = tid; e < L * (DC / 4); e += NT) {
-                const int i = e / (DC / 4), j = e % (DC / 4);
-                const int64_t off = ((tc + i) * H + h) * DV + rank * DC + 4 * j;
-                float4 d = __ldg(reinterpret_cast<const float4 *>(p.dout + off));
-                float4 dg = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (p.gate) {
-                    const uint2 gr = __ldg(reinterpret_cast<const uint2 *>(p.gate + off));
-                    const float g0 = sigmoid_fast(bf16_to_f32(gr.x & 0xffff)), g1 = sigmoid_fast(bf16_to_f32(gr.x >> 16));
-                    const float g2 = sigmoid_fast(bf16_to_f32(gr.y & 0xffff)), g3 = sigmoid_fast(bf16_to_f32(gr.y >> 16));
-                    dg = make_float4(d.x * g0 * (1.f - g0), d.y * g1 * (1.f - g1), d.z * g2 * (1.f - g2),
-                                     d.w * g3 * (1.f - g3));
-                    d = make_float4(d.x * g0, d.y * g1, d.z * g2, d.w * g3);
-                }
-                reinterpret_cast<float4 *>(sDo + i * DC)[j] = d;
-                reinterpret_cast<float4 *>(sDg + i * DC)[j] = dg;
+                const int i = e / (DC / 4), j16 = e % (DC / 4);
+                cp_async_16(raw + SM::kRD + i * (DC * 4) + j16 * 16, p.dout + ((tc + i) * H + h) * DV + rank * DC + j16 * 4, 16);
             }
         }
-        __syncthreads();
-        for (int e = tid; e < L * DK; e += NT) sAl[e] = __expf(kGMin * sigmoid_fast(expA * bf16_to_f32(sA[e])));
+        for (int i = tid; i < L; i += NT) cp_async_4(raw + SM::kRB + i * 4, p.beta + (tc + i) * H + h);
+        cp_async_commit();
+    };
+    // job j's raw inputs have landed in buffer rb: alpha, v in fp32 (and with the gradients: dout
+    // sigmoid(gate), dout sigmoid'(gate), scale q . k)
+    auto derive = [&](int L, bool grads, int rb) {
+        cp_async_wait_all();
+        __syncthreads();   // every thread's copies have landed; the previous job's readers are done
+        const unsigned char *raw = bsm + rb * SM::kRaw;
+        const uint16_t *rq = reinterpret_cast<const uint16_t *>(raw + SM::kRQ);
+        const uint16_t *rk = reinterpret_cast<const uint16_t *>(raw + SM::kRK);
+        const uint16_t *ra = reinterpret_cast<const uint16_t *>(raw + SM::kRA);
+        for (int e = tid; e < L * DK; e += NT) sAl[e] = __expf(kGMin * sigmoid_fast(expA * bf16_to_f32(ra[e])));
+        const uint16_t *rv = reinterpret_cast<const uint16_t *>(raw + SM::kRV);
+        for (int e = tid; e < L * DC; e += NT) sV[e] = bf16_to_f32(rv[e]);
         if (grads) {
+            const float *rd = reinterpret_cast<const float *>(raw + SM::kRD);
+            const uint16_t *rgt = reinterpret_cast<const uint16_t *>(raw + SM::kRG);
+            for (int e = tid; e < L * DC; e += NT) {
+                const float d = rd[e];
+                if (p.gate) {
+                    const float sg = sigmoid_fast(bf16_to_f32(rgt[e]));
+                    sDo[e] = d * sg;
+                    sDg[e] = d * sg * (1.f - sg);
+                } else {
+                    sDo[e] = d;
+                }
+            }
             for (int i = warp; i < L; i += NT / 32) {
                 float s = 0.f;
-                for (int c = lane; c < DK; c += 32) s += bf16_to_f32(sQ[i * DK + c]) * bf16_to_f32(sK[i * DK + c]);
+                for (int c = lane; c < DK; c += 32) s += bf16_to_f32(rq[i * DK + c]) * bf16_to_f32(rk[i * DK + c]);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
                 if (lane == 0) sQK[i] = p.scale * s;
@@ -207,9 +233,18 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
     };
 
     int buf = 0;   // which of the two column-sum buffers the next token uses
+    // sum of the 8 warps' float4 partials of column quad cq (pairwise)
+    auto red_sum = [&](const float *red) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(red);
+        const float4 a0 = f4_add(r4[0 * DC / 4 + cq], r4[1 * DC / 4 + cq]);
+        const float4 a1 = f4_add(r4[2 * DC / 4 + cq], r4[3 * DC / 4 + cq]);
+        const float4 a2 = f4_add(r4[4 * DC / 4 + cq], r4[5 * DC / 4 + cq]);
+        const float4 a3 = f4_add(r4[6 * DC / 4 + cq], r4[7 * DC / 4 + cq]);
+        return f4_add(f4_add(a0, a1), f4_add(a2, a3));
+    };
     // forward step of token i: S <- S' + k u^T, S' = Diag(alpha) S, u = beta (v - S'^T k); S' is
     // stored to `save` when given
-    auto fwd_tok = [&](float4 (&S)[NR], int i, float4 *save) {
+    auto fwd_tok = [&](float4 (&S)[NR], const uint16_t *sK, const float *sB, int i, float4 *save) {
         float kk[NR];
         float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -225,9 +260,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
         float *red = sRed + buf * (3 * 8 * DC);
         if (lane < 8) reinterpret_cast<float4 *>(red + warp * DC)[cq] = r;
         __syncthreads();
-        float4 rt = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int w = 0; w < 8; ++w) rt = f4_add(rt, reinterpret_cast<const float4 *>(red + w * DC)[cq]);
+        const float4 rt = red_sum(red);
         buf ^= 1;
         const float b = sB[i];
         const float4 v = reinterpret_cast<const float4 *>(sV + i * DC)[cq];
@@ -236,71 +269,84 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
         for (int m = 0; m < NR; ++m) S[m] = f4_fma(kk[m], u, S[m]);
     };
 
-    // ---- forward pass: the state at the start of every chunk ---------------------------------
-    float4 S[NR];
+    float4 S[NR], dS[NR];
     {
         const float *S0p = p.S0 ? p.S0 + (size_t)unit * SZ : nullptr;
-#pragma unroll
-        for (int m = 0; m < NR; ++m)
-            S[m] = S0p ? *reinterpret_cast<const float4 *>(S0p + (size_t)(rg + 32 * m) * DV + col0)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int c = 0; c < nck; ++c) {
-        float4 *ck = ck_ptr(c);
-#pragma unroll
-        for (int m = 0; m < NR; ++m) ck[m * NT + tid] = S[m];
-        if (c + 1 == nck) break;   // the state after the last chunk is not needed
-        const int64_t tc = s0 + (int64_t)c * C;
-        stage(tc, C, false);
-        for (int i = 0; i < C; ++i) fwd_tok(S, i, nullptr);
-    }
-
-    // ---- backward, chunk by chunk in reverse ----------------------------------------------------
-    float4 dS[NR];
-    {
         const float *dTp = p.dS_T ? p.dS_T + (size_t)unit * SZ : nullptr;
 #pragma unroll
-        for (int m = 0; m < NR; ++m)
-            dS[m] = dTp ? *reinterpret_cast<const float4 *>(dTp + (size_t)(rg + 32 * m) * DV + col0)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = 0; m < NR; ++m) {
+            const size_t o = (size_t)(rg + 32 * m) * DV + col0;
+            S[m] = S0p ? *reinterpret_cast<const float4 *>(S0p + o) : make_float4(0.f, 0.f, 0.f, 0.f);
+            dS[m] = dTp ? *reinterpret_cast<const float4 *>(dTp + o) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
     float dA_acc = 0.f;
     const uint32_t pBase = smem_u32(sP), pbBase = smem_u32(sPB);
-    for (int c = nck - 1; c >= 0; --c) {
+    if (njobs > 0) issue(0, 0);
+    for (int j = 0; j < njobs; ++j) {
+        const int rb = j & 1;
+        const int c = job_chunk(j);
+        const bool bwd = j >= nfwd;
         const int64_t tc = s0 + (int64_t)c * C;
         const int L = static_cast<int>(min64(C, s1 - tc));
-        const float4 *ck = ck_ptr(c);
+        const unsigned char *raw = bsm + rb * SM::kRaw;
+        const uint16_t *sQ = reinterpret_cast<const uint16_t *>(raw + SM::kRQ);
+        const uint16_t *sK = reinterpret_cast<const uint16_t *>(raw + SM::kRK);
+        const uint16_t *sA = reinterpret_cast<const uint16_t *>(raw + SM::kRA);
+        const float *sB = reinterpret_cast<const float *>(raw + SM::kRB);
+        if (!bwd) {   // forward: the state at the start of the chunk, then its tokens
+            float4 *ck = ck_ptr(c);
 #pragma unroll
-        for (int m = 0; m < NR; ++m) S[m] = ck[m * NT + tid];
-        stage(tc, L, true);
+            for (int m = 0; m < NR; ++m) ck[m * NT + tid] = S[m];
+        } else if (c + 1 < nck) {
+            const float4 *ck = ck_ptr(c);
+#pragma unroll
+            for (int m = 0; m < NR; ++m) S[m] = ck[m * NT + tid];
+        }   // (the backward of the last chunk starts from the forward's state)
+        derive(L, bwd, rb);
+        if (j + 1 < njobs) issue(j + 1, rb ^ 1);
+        if (!bwd) {
+            for (int i = 0; i < C; ++i) fwd_tok(S, sK, sB, i, nullptr);
+            continue;
+        }
         // recompute the chunk: scratch[i] = S' of token tc + i (this thread's part; read back by it)
-        for (int i = 0; i + 1 < L; ++i) fwd_tok(S, i, scratch + (size_t)i * NR * NT);
+        for (int i = 0; i + 1 < L; ++i) fwd_tok(S, sK, sB, i, scratch + (size_t)i * NR * NT);
 #pragma unroll
         for (int m = 0; m < NR; ++m) {
             const float al = sAl[(L - 1) * DK + rg + 32 * m];
             scratch[(size_t)((L - 1) * NR + m) * NT + tid] =
                 make_float4(al * S[m].x, al * S[m].y, al * S[m].z, al * S[m].w);
         }
-        // undo the chunk's tokens in reverse order
+        // undo the chunk's tokens in reverse order; S' and the row inputs of token i - 1 are fetched
+        // while token i runs
         float4 Spn[NR];
+        float kkn[NR], qqn[NR], aln[NR];
 #pragma unroll
-        for (int m = 0; m < NR; ++m) Spn[m] = scratch[(size_t)((L - 1) * NR + m) * NT + tid];
+        for (int m = 0; m < NR; ++m) {
+            const int row = rg + 32 * m;
+            Spn[m] = scratch[(size_t)((L - 1) * NR + m) * NT + tid];
+            kkn[m] = bf16_to_f32(sK[(L - 1) * DK + row]);
+            qqn[m] = p.scale * bf16_to_f32(sQ[(L - 1) * DK + row]);
+            aln[m] = sAl[(L - 1) * DK + row];
+        }
         for (int i = L - 1; i >= 0; --i) {
             float4 Sp[NR];
+            float kk[NR], qq[NR], al[NR];
 #pragma unroll
-            for (int m = 0; m < NR; ++m) Sp[m] = Spn[m];
+            for (int m = 0; m < NR; ++m) { Sp[m] = Spn[m]; kk[m] = kkn[m]; qq[m] = qqn[m]; al[m] = aln[m]; }
             if (i > 0) {
 #pragma unroll
-                for (int m = 0; m < NR; ++m) Spn[m] = scratch[(size_t)((i - 1) * NR + m) * NT + tid];
+                for (int m = 0; m < NR; ++m) {
+                    const int row = rg + 32 * m;
+                    Spn[m] = scratch[(size_t)((i - 1) * NR + m) * NT + tid];
+                    kkn[m] = bf16_to_f32(sK[(i - 1) * DK + row]);
+                    qqn[m] = p.scale * bf16_to_f32(sQ[(i - 1) * DK + row]);
+                    aln[m] = sAl[(i - 1) * DK + row];
+                }
             }
-            float kk[NR], qq[NR], al[NR];
             float4 r = make_float4(0.f, 0.f, 0.f, 0.f), pq = r, dko = r;
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
-                const int row = rg + 32 * m;
-                kk[m] = bf16_to_f32(sK[i * DK + row]);
-                qq[m] = p.scale * bf16_to_f32(sQ[i * DK + row]);
-                al[m] = sAl[i * DK + row];
                 r = f4_fma(kk[m], Sp[m], r);
                 pq = f4_fma(qq[m], Sp[m], pq);
                 dko = f4_fma(kk[m], dS[m], dko);
@@ -315,13 +361,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
                 reinterpret_cast<float4 *>(red + (16 + warp) * DC)[cq] = dko;
             }
             __syncthreads();
-            float4 rt = make_float4(0.f, 0.f, 0.f, 0.f), pqt = rt, dkt = rt;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                rt = f4_add(rt, reinterpret_cast<const float4 *>(red + w * DC)[cq]);
-                pqt = f4_add(pqt, reinterpret_cast<const float4 *>(red + (8 + w) * DC)[cq]);
-                dkt = f4_add(dkt, reinterpret_cast<const float4 *>(red + (16 + w) * DC)[cq]);
-            }
+            const float4 rt = red_sum(red), pqt = red_sum(red + 8 * DC), dkt = red_sum(red + 16 * DC);
             buf ^= 1;
             const float b = sB[i], qk = sQK[i];
             const float4 v = reinterpret_cast<const float4 *>(sV + i * DC)[cq];
@@ -332,11 +372,11 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
             const float4 du = f4_fma(qk, do4, dkt);
             if (tid < 8) {   // row group 0 of warp 0 holds every column of the CTA once
                 const int64_t ov = ((tc + i) * H + h) * DV + col0;
-                *reinterpret_cast<float4 *>(p.dv + ov) = make_float4(b * du.x, b * du.y, b * du.z, b * du.w);
+                st_stream(p.dv + ov, make_float4(b * du.x, b * du.y, b * du.z, b * du.w));
                 if (p.gate) {   // o = S_t^T (scale q) = S'^T (scale q) + (scale q . k) u
                     const float4 o = f4_fma(qk, u, pqt);
                     const float4 dg = reinterpret_cast<const float4 *>(sDg + i * DC)[cq];
-                    *reinterpret_cast<float4 *>(p.dgate + ov) = make_float4(dg.x * o.x, dg.y * o.y, dg.z * o.z, dg.w * o.w);
+                    st_stream(p.dgate + ov, make_float4(dg.x * o.x, dg.y * o.y, dg.z * o.z, dg.w * o.w));
                 }
             }
             if (warp == 0) {   // dbeta over this CTA's columns
@@ -411,20 +451,19 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
                     acc[q3] = f4_add(acc[q3], ld_cluster_f4(mapa_shared(pBase + ((i * 3 + q3) * DK + c4) * 4, g)));
             }
             const int64_t ok = ((tc + i) * H + h) * DK + c4;
-            *reinterpret_cast<float4 *>(p.dq + ok) =
-                make_float4(p.scale * acc[0].x, p.scale * acc[0].y, p.scale * acc[0].z, p.scale * acc[0].w);
-            *reinterpret_cast<float4 *>(p.dk + ok) = acc[1];
+            st_stream(p.dq + ok, make_float4(p.scale * acc[0].x, p.scale * acc[0].y, p.scale * acc[0].z, p.scale * acc[0].w));
+            st_stream(p.dk + ok, acc[1]);
             const float dg[4] = {acc[2].x, acc[2].y, acc[2].z, acc[2].w};
             float da[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float x = expA * bf16_to_f32(sA[i * DK + c4 + j]);
+            for (int jj = 0; jj < 4; ++jj) {
+                const float x = expA * bf16_to_f32(sA[i * DK + c4 + jj]);
                 const float sx = sigmoid_fast(x);
-                const float dx = dg[j] * kGMin * sx * (1.f - sx);
-                da[j] = dx * expA;
+                const float dx = dg[jj] * kGMin * sx * (1.f - sx);
+                da[jj] = dx * expA;
                 dA_acc = fmaf(dx, x, dA_acc);
             }
-            *reinterpret_cast<float4 *>(p.da + ok) = make_float4(da[0], da[1], da[2], da[3]);
+            st_stream(p.da + ok, make_float4(da[0], da[1], da[2], da[3]));
         }
         if (tid < mine) {
             const int i = rank + G * tid;
