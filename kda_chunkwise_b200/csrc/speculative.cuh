@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "mma_frag.cuh"
 
 namespace kda {
 
@@ -40,98 +41,140 @@ struct SpecParams {
     float scale;
 };
 
+// Dynamic shared memory of the verify kernel: the next state (fp32, its global layout), the next
+// unit's raw inputs (bf16 a, k, q [K][DK], v, gate [K][DV]; fp32 beta [K]) and the current unit's
+// derived inputs (alpha, k, scale q [K][DK], v, sigmoid(gate) [K][DV], beta [K], k . scale q [K],
+// fp32).
 template <int DK, int DV>
-__global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecParams p) {
+struct SpecVerifySmem {
+    __host__ __device__ static size_t raw_off() { return (size_t)DK * DV * 4; }
+    __host__ __device__ static size_t beta_off(int K) { return raw_off() + (size_t)K * (3 * DK + 2 * DV) * 2; }
+    __host__ __device__ static size_t derived_off(int K) { return beta_off(K) + (size_t)((K + 3) & ~3) * 4; }
+    __host__ __device__ static size_t bytes(int K) { return derived_off(K) + (size_t)K * (3 * DK + 2 * DV + 2) * 4; }
+};
+
+// Persistent: a CTA takes units blockIdx.x, blockIdx.x + gridDim.x, ...; while it runs the K token
+// steps of one unit, the next unit's state and inputs are copied into shared memory asynchronously,
+// so the loads of HBM overlap the dependent token steps.
+template <int DK, int DV>
+__global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecParams p, int64_t units) {
     constexpr int kThreads = kSpecThreads;
     constexpr int LPR = DV / 4;          // threads per state row, one float4 each
     constexpr int RPP = kThreads / LPR;  // rows covered by the block in one pass
     constexpr int NR = DK / RPP;         // rows held per thread
+    using SL = SpecVerifySmem<DK, DV>;
 
-    __shared__ float s_alpha[kSpecMaxTokens][DK], s_k[kSpecMaxTokens][DK], s_q[kSpecMaxTokens][DK];
-    __shared__ float s_v[kSpecMaxTokens][DV], s_beta[kSpecMaxTokens];
-    __shared__ uint16_t s_g[kSpecMaxTokens][DV];   // gate logits (bf16)
-    __shared__ float4 s_red[2][RPP][LPR];
-    __shared__ __align__(16) float s_u[DV];
-    __shared__ float s_kq;
+    extern __shared__ __align__(16) unsigned char spec_dyn[];
+    const int K = p.K;
+    const float4 *sS = reinterpret_cast<const float4 *>(spec_dyn);
+    const uint16_t *r_a = reinterpret_cast<const uint16_t *>(spec_dyn + SL::raw_off());
+    const uint16_t *r_k = r_a + K * DK, *r_q = r_k + K * DK, *r_v = r_q + K * DK, *r_g = r_v + K * DV;
+    const float *r_beta = reinterpret_cast<const float *>(spec_dyn + SL::beta_off(K));
+    float *s_alpha = reinterpret_cast<float *>(spec_dyn + SL::derived_off(K));
+    float *s_k = s_alpha + K * DK, *s_q = s_k + K * DK, *s_v = s_q + K * DK, *s_sg = s_v + K * DV;
+    float *s_b = s_sg + K * DV, *s_kqt = s_b + K;
+    __shared__ float4 s_red[2][2][RPP][LPR];   // two buffers: consecutive tokens alternate
 
-    const int64_t nh = blockIdx.x;
-    const int64_t n = nh / p.H;
-    const int h = static_cast<int>(nh % p.H);
     const int tid = threadIdx.x;
     const int cq = tid % LPR, rg = tid / LPR;
+    auto issue = [&](int64_t nh) {   // asynchronous copy of unit nh's state and inputs
+        const int64_t n = nh / p.H;
+        const int h = static_cast<int>(nh % p.H);
+        const uint32_t base = smem_u32(spec_dyn);
+        const float *St = p.state + nh * (int64_t)(DK * DV);
+        for (int e = tid; e < DK * DV / 4; e += kThreads) cp_async_16(base + e * 16, St + e * 4, 16);
+        const uint32_t raw = base + (uint32_t)SL::raw_off();
+        for (int e = tid; e < K * (3 * DK / 8); e += kThreads) {   // a, k, q rows: 16 bytes = 8 values
+            const int which = e / (K * DK / 8), r = e % (K * DK / 8), t = r / (DK / 8), j = r % (DK / 8);
+            const uint16_t *src = which == 0 ? p.a : (which == 1 ? p.k : p.q);
+            cp_async_16(raw + ((which * K + t) * DK + j * 8) * 2, src + ((n * K + t) * p.H + h) * DK + j * 8, 16);
+        }
+        for (int e = tid; e < K * (DV / 8); e += kThreads) {
+            const int t = e / (DV / 8), j = e % (DV / 8);
+            const int64_t off = ((n * K + t) * p.H + h) * DV + j * 8;
+            cp_async_16(raw + (3 * K * DK + t * DV + j * 8) * 2, p.v + off, 16);
+            if (p.gate) cp_async_16(raw + (3 * K * DK + (K + t) * DV + j * 8) * 2, p.gate + off, 16);
+        }
+        const uint32_t rb = base + (uint32_t)SL::beta_off(K);
+        for (int t = tid; t < K; t += kThreads) cp_async_4(rb + t * 4, p.beta + (n * K + t) * p.H + h);
+        cp_async_commit();
+    };
 
-    const float4 *St = reinterpret_cast<const float4 *>(p.state + nh * (int64_t)(DK * DV));
-    float4 S[NR];
+    int64_t nh = blockIdx.x;
+    if (nh < units) issue(nh);
+    for (; nh < units; nh += gridDim.x) {
+        const int64_t n = nh / p.H;
+        const int h = static_cast<int>(nh % p.H);
+        cp_async_wait_all();
+        __syncthreads();   // this unit's copies have landed (every thread's)
+        float4 S[NR];
 #pragma unroll
-    for (int m = 0; m < NR; ++m) S[m] = __ldcs(St + (rg + m * RPP) * LPR + cq);
-    const float expA = expf(p.A_log[h]);
-    for (int e = tid; e < p.K * DK; e += kThreads) {   // all K tokens' inputs, once
-        const int t = e / DK, i = e % DK;
-        const int64_t tok = (n * p.K + t) * p.H + h;   // row of token t of this sequence, head h
-        s_alpha[t][i] = __expf(log_decay(bf16_to_f32(p.a[tok * DK + i]), expA));
-        s_k[t][i] = bf16_to_f32(p.k[tok * DK + i]);
-        s_q[t][i] = p.scale * bf16_to_f32(p.q[tok * DK + i]);
-    }
-    for (int e = tid; e < p.K * DV; e += kThreads) {
-        const int t = e / DV, i = e % DV;
-        const int64_t off = ((n * p.K + t) * p.H + h) * DV + i;
-        s_v[t][i] = bf16_to_f32(p.v[off]);
-        if (p.gate) s_g[t][i] = p.gate[off];
-    }
-    if (tid < p.K) s_beta[tid] = p.beta[(n * p.K + tid) * p.H + h];
-    __syncthreads();
-
-    for (int t = 0; t < p.K; ++t) {
-        const int64_t tok = (n * p.K + t) * p.H + h;
-        if (tid < 32) {
+        for (int m = 0; m < NR; ++m) S[m] = sS[(rg + m * RPP) * LPR + cq];
+        const float expA = expf(p.A_log[h]);
+        for (int e = tid; e < K * DK; e += kThreads) {
+            s_alpha[e] = __expf(log_decay(bf16_to_f32(r_a[e]), expA));
+            s_k[e] = bf16_to_f32(r_k[e]);
+            s_q[e] = p.scale * bf16_to_f32(r_q[e]);
+        }
+        for (int e = tid; e < K * DV; e += kThreads) {
+            s_v[e] = bf16_to_f32(r_v[e]);
+            if (p.gate) s_sg[e] = sigmoid_fast(bf16_to_f32(r_g[e]));
+        }
+        for (int t = tid; t < K; t += kThreads) s_b[t] = r_beta[t];
+        __syncthreads();
+        for (int t = tid >> 5; t < K; t += kThreads / 32) {   // k . scale q per token, as the decode step
+            const int lane = tid & 31;
             float acc = 0.f;
-            for (int i = tid; i < DK; i += 32) acc = fmaf(s_k[t][i], s_q[t][i], acc);
+            for (int i = lane; i < DK; i += 32) acc = fmaf(s_k[t * DK + i], s_q[t * DK + i], acc);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (tid == 0) s_kq = acc;
-        }
-        float4 r = make_float4(0.f, 0.f, 0.f, 0.f), pq = r;
+            if (lane == 0) s_kqt[t] = acc;
+        }   // the state and raw buffers are free for the next unit
+        if (nh + gridDim.x < units) issue(nh + gridDim.x);
+
+        for (int t = 0; t < K; ++t) {
+            const int64_t tok = (n * K + t) * p.H + h;
+            float4 r = make_float4(0.f, 0.f, 0.f, 0.f), pq = r;
 #pragma unroll
-        for (int m = 0; m < NR; ++m) {
-            const int row = rg + m * RPP;
-            const float al = s_alpha[t][row];
-            S[m].x *= al; S[m].y *= al; S[m].z *= al; S[m].w *= al;
-            r = f4_fma(s_k[t][row], S[m], r);
-            pq = f4_fma(s_q[t][row], S[m], pq);
-        }
-        s_red[0][rg][cq] = r;
-        s_red[1][rg][cq] = pq;
-        __syncthreads();
-        if (tid < DV) {
-            const float *red_r = reinterpret_cast<const float *>(&s_red[0][0][0]);
-            const float *red_p = reinterpret_cast<const float *>(&s_red[1][0][0]);
-            float rr = 0.f, pp = 0.f;
-#pragma unroll 8
-            for (int g = 0; g < RPP; ++g) {
-                rr += red_r[g * DV + tid];
-                pp += red_p[g * DV + tid];
+            for (int m = 0; m < NR; ++m) {
+                const int row = rg + m * RPP;
+                const float al = s_alpha[t * DK + row];
+                S[m].x *= al; S[m].y *= al; S[m].z *= al; S[m].w *= al;
+                r = f4_fma(s_k[t * DK + row], S[m], r);
+                pq = f4_fma(s_q[t * DK + row], S[m], pq);
             }
-            const int64_t off = tok * DV + tid;
-            const float u = s_beta[t] * (s_v[t][tid] - rr);
-            s_u[tid] = u;
-            p.u[(nh * p.K + t) * DV + tid] = u;
-            float o = fmaf(s_kq, u, pp);
-            if (p.gate) o *= sigmoid_fast(bf16_to_f32(s_g[t][tid]));
-            store_out(p.out, off, p.out_f32, o);
-        }
-        __syncthreads();
-        const float4 u4 = reinterpret_cast<const float4 *>(s_u)[cq];
+            float4 (&red)[2][RPP][LPR] = s_red[t & 1];
+            red[0][rg][cq] = r;
+            red[1][rg][cq] = pq;
+            __syncthreads();   // (the k . q of every token is ready too)
+            float4 rr, pp;
+            quad_col_sums<RPP, LPR>(red, cq, rr, pp);
+            const float bt = s_b[t];
+            const float4 v4 = reinterpret_cast<const float4 *>(s_v + t * DV)[cq];
+            const float4 u4 = make_float4(bt * (v4.x - rr.x), bt * (v4.y - rr.y), bt * (v4.z - rr.z), bt * (v4.w - rr.w));
+            if (rg == 0) {   // the first row group holds every column once
+                reinterpret_cast<float4 *>(p.u + (nh * K + t) * DV)[cq] = u4;
+                const float kq = s_kqt[t];
+                float o[4] = {fmaf(kq, u4.x, pp.x), fmaf(kq, u4.y, pp.y), fmaf(kq, u4.z, pp.z), fmaf(kq, u4.w, pp.w)};
+                if (p.gate) {
+                    const float4 sg = reinterpret_cast<const float4 *>(s_sg + t * DV)[cq];
+                    o[0] *= sg.x; o[1] *= sg.y; o[2] *= sg.z; o[3] *= sg.w;
+                }
 #pragma unroll
-        for (int m = 0; m < NR; ++m) {
-            const float kk = s_k[t][rg + m * RPP];
-            S[m].x = fmaf(kk, u4.x, S[m].x);
-            S[m].y = fmaf(kk, u4.y, S[m].y);
-            S[m].z = fmaf(kk, u4.z, S[m].z);
-            S[m].w = fmaf(kk, u4.w, S[m].w);
+                for (int c = 0; c < 4; ++c) store_out(p.out, tok * DV + 4 * cq + c, p.out_f32, o[c]);
+            }
+#pragma unroll
+            for (int m = 0; m < NR; ++m) {
+                const float kk = s_k[t * DK + rg + m * RPP];
+                S[m].x = fmaf(kk, u4.x, S[m].x);
+                S[m].y = fmaf(kk, u4.y, S[m].y);
+                S[m].z = fmaf(kk, u4.z, S[m].z);
+                S[m].w = fmaf(kk, u4.w, S[m].w);
+            }
         }
-        // the next token overwrites s_u and s_red only after every thread is done here
-        __syncthreads();
+        __syncthreads();   // the derived inputs are read by every thread before the next unit's
     }
+    cp_async_wait_all();   // nothing is left in flight at exit
 }
 
 template <int DK, int DV>
@@ -157,6 +200,11 @@ __global__ void __launch_bounds__(kSpecThreads) spec_commit_kernel(const SpecPar
     }
     if (j == 0) return;   // nothing accepted: the state stays as it is
 
+    // the state's loads are issued first so that they overlap the staging of the small inputs
+    float4 *St = reinterpret_cast<float4 *>(p.state + nh * (int64_t)(DK * DV));
+    float4 S[NR];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) S[m] = __ldcs(St + (rg + m * RPP) * LPR + cq);
     const float expA = expf(p.A_log[h]);
     for (int e = tid; e < j * DK; e += kThreads) {
         const int t = e / DK, i = e % DK;
@@ -166,11 +214,6 @@ __global__ void __launch_bounds__(kSpecThreads) spec_commit_kernel(const SpecPar
     }
     for (int e = tid; e < j * DV; e += kThreads) s_uw[e / DV][e % DV] = __ldcs(p.u + (nh * p.K + e / DV) * DV + e % DV);
     __syncthreads();
-
-    float4 *St = reinterpret_cast<float4 *>(p.state + nh * (int64_t)(DK * DV));
-    float4 S[NR];
-#pragma unroll
-    for (int m = 0; m < NR; ++m) S[m] = __ldcs(St + (rg + m * RPP) * LPR + cq);
     for (int t = 0; t < j; ++t) {
         const float4 u4 = reinterpret_cast<const float4 *>(s_uw[t])[cq];
 #pragma unroll
