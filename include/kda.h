@@ -120,6 +120,39 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const voi
                                          const float *initial_state, float *final_state, void *out,
                                          kda_dtype out_dtype, void *stream);
 
+/*
+ * kda_chunk_fwd_host — kda_chunk_fwd with every input and output in HOST memory (page-locked for
+ * the copies to overlap): the end-to-end prefill of a batch that lives on the host.
+ * (No counterpart in the pages: this is the runtime around the method.)
+ *   q, k, v, a, beta, gate, out, initial_state, final_state: host pointers, layouts and types as
+ *     kda_chunk_fwd; A_log fp32 [H] and cu_seqlens int32 [num_seqs + 1] are HOST arrays here (read
+ *     by this call; cu_seqlens must run monotonically from 0 to total_tokens).
+ *   piece_tokens: tokens per piece (0 = 2048; at least 64).
+ *   device_buffer: caller-owned device memory, 256-byte aligned, of
+ *     kda_chunk_fwd_host_buffer_size(...) bytes: two staging slots, the prefill workspace and the
+ *     states.
+ * The batch is cut into pieces along the packed token axis; a cut inside a sequence falls on a
+ * 64-token chunk boundary of that sequence, so every piece runs the chunks the whole call would,
+ * and a sequence that continues into the next piece hands its state over on the device.  The
+ * host-to-device copy of piece i+1, the prefill of piece i (on `stream`) and the device-to-host
+ * copy of piece i-1 run on three streams at once.  Asynchronous with respect to the host: the
+ * host buffers must stay valid, and `out` / `final_state` hold the results, once `stream` has
+ * reached the end of the call.
+ */
+KDA_API kda_status kda_chunk_fwd_host(const void *q, const void *k, const void *v, const void *a,
+                                      const float *beta, const void *gate, const float *A_log,
+                                      const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                      int32_t H, int32_t d_k, int32_t d_v, float scale,
+                                      const float *initial_state, float *final_state, void *out,
+                                      kda_dtype out_dtype, int64_t piece_tokens, void *device_buffer,
+                                      size_t device_buffer_bytes, void *stream);
+
+/* Device buffer kda_chunk_fwd_host needs (host-only; reads the host cu_seqlens; 0 on invalid
+ * arguments). */
+KDA_API size_t kda_chunk_fwd_host_buffer_size(const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                              int32_t H, int32_t d_k, int32_t d_v, kda_dtype out_dtype,
+                                              int64_t piece_tokens);
+
 /* Workspace kda_chunk_fwd needs for these sizes (host-only; 0 on invalid sizes). */
 KDA_API size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t max_seqlen,
                                     int32_t H, int32_t d_k, int32_t d_v);

@@ -6,6 +6,8 @@ no CPU or PyTorch fallback: importing this package without the built library rai
 
 Entry points (same names as the C ABI):
   kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, ...)  prefill, chunkwise form
+  kda_chunk_fwd_host(...)                                   the same prefill on host tensors, the copies
+                                                            overlapped with the compute piece by piece
   kda_decode_step(q, k, v, a, beta, A_log, state, ...)      one recurrent step, state in place
   kda_decode_verify / kda_decode_commit                     K proposed tokens, then the accepted prefix
   kda_short_conv, kda_output_norm_gate                      the module's short convolution and
@@ -28,7 +30,8 @@ __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_launch_count", "kda_chunk_fwd_noalloc", "kda_inject_stall",
            "kda_decode_verify", "kda_decode_commit", "kda_short_conv", "kda_output_norm_gate",
            "kda_state_combine", "kda_segment_maps", "context_parallel_states", "kda_context_parallel_fwd",
-           "kda_chunk_bwd", "kda_chunk_bwd_workspace_size",
+           "kda_chunk_bwd", "kda_chunk_bwd_workspace_size", "kda_chunk_fwd_host",
+           "kda_chunk_fwd_host_buffer_size",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -89,6 +92,11 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_bwd.restype = ctypes.c_int
     L.kda_chunk_bwd_workspace_size.argtypes = [i64, i32, i32, i32, i32]
     L.kda_chunk_bwd_workspace_size.restype = sz
+    L.kda_chunk_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, f32, vp, vp, vp,
+                                     ctypes.c_int, i64, vp, sz, vp]
+    L.kda_chunk_fwd_host.restype = ctypes.c_int
+    L.kda_chunk_fwd_host_buffer_size.argtypes = [vp, i32, i64, i32, i32, i32, ctypes.c_int, i64]
+    L.kda_chunk_fwd_host_buffer_size.restype = sz
     L.kda_inject_stall.argtypes = [i32, ctypes.c_uint64]
     L.kda_inject_stall.restype = ctypes.c_int
     return L
@@ -184,6 +192,62 @@ def kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=
                            _OUT_DTYPES[out.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
                            _stream_handle(stream, dev))
     _check(st, "kda_chunk_fwd")
+    return out, final_state
+
+
+def kda_chunk_fwd_host_buffer_size(cu_seqlens, H, d_k, d_v, out_dtype=torch.bfloat16, piece_tokens: int = 0) -> int:
+    """Device bytes kda_chunk_fwd_host needs; cu_seqlens is a host int32 tensor."""
+    N = cu_seqlens.numel() - 1
+    T = int(cu_seqlens[-1]) if N >= 0 else 0
+    return int(lib.kda_chunk_fwd_host_buffer_size(_ptr(cu_seqlens), N, T, H, d_k, d_v, _OUT_DTYPES[out_dtype],
+                                                  int(piece_tokens)))
+
+
+def kda_chunk_fwd_host(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None, out=None,
+                       final_state=None, out_dtype=torch.bfloat16, scale: float = 1.0, piece_tokens: int = 0,
+                       device_buffer=None, device=None, stream=None):
+    """Prefill of a batch held in host memory (see include/kda.h): every tensor, A_log and cu_seqlens
+    included, is on the CPU (page-locked tensors let the copies overlap the compute).  The outputs
+    ``out`` and ``final_state`` (host tensors; allocated page-locked when not given) hold the result
+    once ``stream`` has reached the end of the call.  device_buffer: a CUDA uint8 tensor of
+    kda_chunk_fwd_host_buffer_size(...) bytes (allocated when not given).
+    Returns (out, final_state)."""
+    cpu = torch.device("cpu")
+    T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    bf = torch.bfloat16
+    for name, t, shp in (("q", q, (T, H, d_k)), ("k", k, (T, H, d_k)), ("a", a, (T, H, d_k)),
+                         ("v", v, (T, H, d_v))):
+        _need(t, name, bf, shp, cpu)
+    _need(beta, "beta", torch.float32, (T, H), cpu)
+    _need(A_log, "A_log", torch.float32, (H,), cpu)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), cpu)
+    if gate is not None:
+        _need(gate, "gate", bf, (T, H, d_v), cpu)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32, (N, H, d_k, d_v), cpu)
+    for name, t in (("q", q), ("k", k), ("a", a), ("v", v), ("beta", beta), ("gate", gate),
+                    ("initial_state", initial_state), ("A_log", A_log), ("cu_seqlens", cu_seqlens)):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if out is None:
+        out = torch.empty((T, H, d_v), dtype=out_dtype, pin_memory=True)
+    if out.dtype not in _OUT_DTYPES:
+        raise TypeError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, (T, H, d_v), cpu)
+    if final_state is None:
+        final_state = torch.empty((N, H, d_k, d_v), dtype=torch.float32, pin_memory=True)
+    _need(final_state, "final_state", torch.float32, (N, H, d_k, d_v), cpu)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if device_buffer is None:
+        nbytes = kda_chunk_fwd_host_buffer_size(cu_seqlens, H, d_k, d_v, out.dtype, piece_tokens)
+        device_buffer = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    st = lib.kda_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate), _ptr(A_log),
+                                _ptr(cu_seqlens), N, T, H, d_k, d_v, float(scale), _ptr(initial_state),
+                                _ptr(final_state), _ptr(out), _OUT_DTYPES[out.dtype], int(piece_tokens),
+                                _ptr(device_buffer), device_buffer.numel(), _stream_handle(stream, dev))
+    _check(st, "kda_chunk_fwd_host")
     return out, final_state
 
 

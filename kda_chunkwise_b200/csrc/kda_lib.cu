@@ -8,6 +8,7 @@
 #include <mutex>
 #include <cstring>
 #include <string>
+#include <vector>
 
 #include "kda.h"
 #include "common.cuh"
@@ -599,3 +600,237 @@ kda_status kda_sync_check(void *stream) {
 }
 
 }  // extern "C"
+
+// ---- prefill with host buffers: pieces along the token axis, copies overlapped with compute ------
+
+namespace {
+
+constexpr int kHostSlots = 2;             // staging slots: piece p uses slot p % 2
+constexpr int64_t kHostPieceDefault = 2048;
+
+struct HostPiece {
+    int64_t a, e;       // packed tokens [a, e)
+    int32_t n_lo, n_hi; // sequences taking part (inclusive)
+    bool carry;         // sequence n_hi continues into the next piece
+};
+
+// Cuts the packed batch into pieces of about `piece` tokens.  A cut inside a sequence falls on a
+// 64-token chunk boundary of that sequence, so each piece runs exactly the chunks the whole call
+// would.  Sequence n takes part in the piece where it starts (an empty one at the very end, in the
+// last piece) and in every piece it continues into.
+bool plan_pieces(const int32_t *cu, int32_t N, int64_t T, int64_t piece, std::vector<HostPiece> &out) {
+    out.clear();
+    int64_t a = 0;
+    do {
+        int64_t e = std::min<int64_t>(a + piece, T);
+        if (e < T) {   // move the cut down to a chunk boundary of the sequence containing token e
+            int32_t m = 0;
+            while (m < N && cu[m + 1] <= e) ++m;
+            if (m >= N) return false;
+            e = cu[m] + ((e - cu[m]) / kda::kChunk) * kda::kChunk;
+            if (e <= a) return false;   // not reached for piece >= 64: a is a boundary of its own
+        }
+        int32_t lo = 0;   // first sequence not finished before a (empty ones starting at a included)
+        while (lo < N && cu[lo + 1] <= a && cu[lo] < a) ++lo;
+        int32_t hi = lo;  // last sequence starting before e (every remaining one in the last piece)
+        while (hi + 1 < N && (e == T || cu[hi + 1] < e)) ++hi;
+        if (lo >= N) return false;
+        out.push_back({a, e, lo, hi, e < T && cu[hi + 1] > e});
+        a = e;
+    } while (a < T);
+    return true;
+}
+
+struct HostLayout {
+    size_t in_bytes, out_bytes, slot_bytes, ws_bytes, cu_bytes, state_bytes, total;
+    int64_t max_tokens;
+};
+
+HostLayout host_layout(const std::vector<HostPiece> &pieces, int32_t N, int32_t H, int d_k, int d_v, bool f32_out) {
+    HostLayout L{};
+    int64_t max_tok = 0;
+    size_t ws = 0, cu_count = 0;
+    for (const HostPiece &pc : pieces) {
+        max_tok = std::max(max_tok, pc.e - pc.a);
+        ws = std::max(ws, kda_chunk_fwd_workspace_min(pc.e - pc.a, pc.n_hi - pc.n_lo + 1, 0, H, d_k, d_v));
+        cu_count += (size_t)(pc.n_hi - pc.n_lo + 2);
+    }
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t th = (size_t)max_tok * H;
+    // q, k, a, v, gate (bf16), beta (fp32): each region rounded up so every pointer stays aligned
+    L.in_bytes = 3 * up(th * d_k * 2) + 2 * up(th * d_v * 2) + up(th * 4);
+    L.out_bytes = up(th * d_v * (f32_out ? 4 : 2));
+    L.slot_bytes = L.in_bytes + L.out_bytes;
+    L.ws_bytes = up(ws);
+    L.cu_bytes = up(cu_count * 4 + (size_t)H * 4);
+    L.state_bytes = up((size_t)N * H * d_k * d_v * 4);
+    L.total = kHostSlots * L.slot_bytes + L.ws_bytes + L.cu_bytes + 2 * L.state_bytes;
+    L.max_tokens = max_tok;
+    return L;
+}
+
+}  // namespace
+
+size_t kda_chunk_fwd_host_buffer_size(const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                      int32_t d_k, int32_t d_v, kda_dtype out_dtype, int64_t piece_tokens) {
+    if (!cu_seqlens || num_seqs <= 0 || total_tokens < 0 || H <= 0 || !supported_dim(d_k) || !supported_dim(d_v))
+        return 0;
+    if (piece_tokens == 0) piece_tokens = kHostPieceDefault;
+    if (piece_tokens < kda::kChunk) return 0;
+    std::vector<HostPiece> pieces;
+    if (!plan_pieces(cu_seqlens, num_seqs, total_tokens, piece_tokens, pieces)) return 0;
+    return host_layout(pieces, num_seqs, H, d_k, d_v, out_dtype == KDA_DTYPE_F32).total;
+}
+
+kda_status kda_chunk_fwd_host(const void *q, const void *k, const void *v, const void *a, const float *beta,
+                              const void *gate, const float *A_log, const int32_t *cu_seqlens, int32_t num_seqs,
+                              int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                              const float *initial_state, float *final_state, void *out, kda_dtype out_dtype,
+                              int64_t piece_tokens, void *device_buffer, size_t device_buffer_bytes, void *stream) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: negative size or H <= 0");
+    if (!supported_dim(d_k) || !supported_dim(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_host: d_k and d_v must be 64 or 128");
+    if (num_seqs == 0) {
+        if (total_tokens != 0) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: tokens without sequences");
+        return KDA_OK;
+    }
+    if (!cu_seqlens || !A_log) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: NULL cu_seqlens or A_log");
+    if (total_tokens > 0 && (!q || !k || !v || !a || !beta || !out))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: NULL q/k/v/a/beta/out");
+    if (out_dtype != KDA_DTYPE_BF16 && out_dtype != KDA_DTYPE_F32)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: out_dtype must be KDA_DTYPE_BF16 or KDA_DTYPE_F32");
+    if (piece_tokens == 0) piece_tokens = kHostPieceDefault;
+    if (piece_tokens < kda::kChunk) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: piece_tokens below 64");
+    // cu_seqlens is read here on the host: it must be well formed
+    if (cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != total_tokens)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: cu_seqlens must run from 0 to total_tokens");
+    for (int32_t n = 0; n < num_seqs; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: cu_seqlens not monotone");
+    std::vector<HostPiece> pieces;
+    if (!plan_pieces(cu_seqlens, num_seqs, total_tokens, piece_tokens, pieces))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: could not cut the batch into pieces");
+    const bool f32_out = out_dtype == KDA_DTYPE_F32;
+    const HostLayout L = host_layout(pieces, num_seqs, H, d_k, d_v, f32_out);
+    if (!device_buffer || device_buffer_bytes < L.total)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: device buffer missing or too small (need " +
+                                             std::to_string(L.total) + " bytes)");
+    if ((reinterpret_cast<uintptr_t>(device_buffer) & 255u) != 0)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_host: device buffer not 256-byte aligned");
+
+    // device buffer: [slot 0 | slot 1 | workspace | cu arrays + A_log | S in | S out]
+    char *base = static_cast<char *>(device_buffer);
+    char *ws = base + kHostSlots * L.slot_bytes;
+    int32_t *d_cu = reinterpret_cast<int32_t *>(ws + L.ws_bytes);
+    float *d_S = reinterpret_cast<float *>(ws + L.ws_bytes + L.cu_bytes);
+    float *d_T = reinterpret_cast<float *>(reinterpret_cast<char *>(d_S) + L.state_bytes);
+    // host copy of every piece's cu_seqlens, then A_log
+    std::vector<int32_t> h_cu;
+    std::vector<size_t> cu_off;
+    for (const HostPiece &pc : pieces) {
+        cu_off.push_back(h_cu.size());
+        for (int32_t n = pc.n_lo; n <= pc.n_hi + 1; ++n)
+            h_cu.push_back((int32_t)(std::min<int64_t>(std::max<int64_t>(cu_seqlens[n], pc.a), pc.e) - pc.a));
+    }
+    const size_t alog_off = h_cu.size();
+    h_cu.resize(h_cu.size() + H);
+    std::memcpy(h_cu.data() + alog_off, A_log, (size_t)H * 4);
+    const float *d_Alog = reinterpret_cast<const float *>(d_cu + alog_off);
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);   // compute (the caller's stream)
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_in[kHostSlots] = {}, ev_comp[kHostSlots] = {}, ev_out[kHostSlots] = {};
+    cudaError_t e = cudaSuccess;
+    auto cleanup = [&]() {
+        for (int i = 0; i < kHostSlots; ++i) {
+            if (ev_in[i]) cudaEventDestroy(ev_in[i]);
+            if (ev_comp[i]) cudaEventDestroy(ev_comp[i]);
+            if (ev_out[i]) cudaEventDestroy(ev_out[i]);
+        }
+        if (ev_start) cudaEventDestroy(ev_start);
+        if (s_in) cudaStreamDestroy(s_in);      // released once their work completes
+        if (s_out) cudaStreamDestroy(s_out);
+    };
+#define KDA_HOST_TRY(call, where)               \
+    do {                                        \
+        if ((e = (call)) != cudaSuccess) {      \
+            cleanup();                          \
+            return cuda_fail(e, where);         \
+        }                                       \
+    } while (0)
+    KDA_HOST_TRY(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking), "kda_chunk_fwd_host: stream");
+    KDA_HOST_TRY(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking), "kda_chunk_fwd_host: stream");
+    KDA_HOST_TRY(cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming), "kda_chunk_fwd_host: event");
+    for (int i = 0; i < kHostSlots; ++i) {
+        KDA_HOST_TRY(cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming), "kda_chunk_fwd_host: event");
+        KDA_HOST_TRY(cudaEventCreateWithFlags(&ev_comp[i], cudaEventDisableTiming), "kda_chunk_fwd_host: event");
+        KDA_HOST_TRY(cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming), "kda_chunk_fwd_host: event");
+    }
+    // everything after what the caller queued before this call
+    KDA_HOST_TRY(cudaEventRecord(ev_start, cs), "kda_chunk_fwd_host: record");
+    KDA_HOST_TRY(cudaStreamWaitEvent(s_in, ev_start, 0), "kda_chunk_fwd_host: wait");
+    KDA_HOST_TRY(cudaStreamWaitEvent(s_out, ev_start, 0), "kda_chunk_fwd_host: wait");
+    KDA_HOST_TRY(cudaMemcpyAsync(d_cu, h_cu.data(), h_cu.size() * 4, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: cu copy");
+    const size_t state_bytes = (size_t)num_seqs * H * d_k * d_v * 4;
+    if (initial_state)
+        KDA_HOST_TRY(cudaMemcpyAsync(d_S, initial_state, state_bytes, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: state copy");
+    else
+        KDA_HOST_TRY(cudaMemsetAsync(d_S, 0, state_bytes, s_in), "kda_chunk_fwd_host: state clear");
+
+    const size_t SZ = (size_t)d_k * d_v;
+    const size_t osz = f32_out ? 4 : 2;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t th_max = (size_t)L.max_tokens * H;
+    for (size_t pi = 0; pi < pieces.size(); ++pi) {
+        const HostPiece &pc = pieces[pi];
+        const int slot = (int)(pi % kHostSlots);
+        char *sb = base + slot * L.slot_bytes;
+        char *dq = sb, *dk = dq + up(th_max * d_k * 2), *da = dk + up(th_max * d_k * 2);
+        char *dv = da + up(th_max * d_k * 2), *dg = dv + up(th_max * d_v * 2);
+        char *db = dg + up(th_max * d_v * 2), *dout = sb + L.in_bytes;
+        const int64_t tok = pc.e - pc.a;
+        const size_t rk = (size_t)H * d_k * 2, rv = (size_t)H * d_v * 2;
+        // inputs of this piece into its slot, once the piece two back has consumed the slot
+        if (pi >= kHostSlots) KDA_HOST_TRY(cudaStreamWaitEvent(s_in, ev_comp[slot], 0), "kda_chunk_fwd_host: wait");
+        if (tok > 0) {
+            KDA_HOST_TRY(cudaMemcpyAsync(dq, static_cast<const char *>(q) + pc.a * rk, tok * rk, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: copy");
+            KDA_HOST_TRY(cudaMemcpyAsync(dk, static_cast<const char *>(k) + pc.a * rk, tok * rk, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: copy");
+            KDA_HOST_TRY(cudaMemcpyAsync(da, static_cast<const char *>(a) + pc.a * rk, tok * rk, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: copy");
+            KDA_HOST_TRY(cudaMemcpyAsync(dv, static_cast<const char *>(v) + pc.a * rv, tok * rv, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: copy");
+            if (gate)
+                KDA_HOST_TRY(cudaMemcpyAsync(dg, static_cast<const char *>(gate) + pc.a * rv, tok * rv, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: copy");
+            KDA_HOST_TRY(cudaMemcpyAsync(db, beta + pc.a * H, tok * H * 4, cudaMemcpyHostToDevice, s_in), "kda_chunk_fwd_host: copy");
+        }
+        KDA_HOST_TRY(cudaEventRecord(ev_in[slot], s_in), "kda_chunk_fwd_host: record");
+        // the prefill of the piece, once its inputs are in and the piece two back has been copied out
+        KDA_HOST_TRY(cudaStreamWaitEvent(cs, ev_in[slot], 0), "kda_chunk_fwd_host: wait");
+        if (pi >= kHostSlots) KDA_HOST_TRY(cudaStreamWaitEvent(cs, ev_out[slot], 0), "kda_chunk_fwd_host: wait");
+        const int32_t ns = pc.n_hi - pc.n_lo + 1;
+        const kda_status st = kda_chunk_fwd(dq, dk, dv, da, reinterpret_cast<const float *>(db), gate ? dg : nullptr, d_Alog,
+                                            d_cu + cu_off[pi], ns, tok, 0, H, d_k, d_v, scale, d_S + (size_t)pc.n_lo * H * SZ,
+                                            d_T + (size_t)pc.n_lo * H * SZ, dout, out_dtype, ws, L.ws_bytes, cs);
+        if (st != KDA_OK) {
+            cleanup();
+            return st;
+        }
+        if (pc.carry)   // the sequence continuing into the next piece starts there from this state
+            KDA_HOST_TRY(cudaMemcpyAsync(d_S + (size_t)pc.n_hi * H * SZ, d_T + (size_t)pc.n_hi * H * SZ, H * SZ * 4,
+                                         cudaMemcpyDeviceToDevice, cs), "kda_chunk_fwd_host: carry");
+        KDA_HOST_TRY(cudaEventRecord(ev_comp[slot], cs), "kda_chunk_fwd_host: record");
+        // the piece's outputs back to the host
+        KDA_HOST_TRY(cudaStreamWaitEvent(s_out, ev_comp[slot], 0), "kda_chunk_fwd_host: wait");
+        if (tok > 0)
+            KDA_HOST_TRY(cudaMemcpyAsync(static_cast<char *>(out) + pc.a * H * d_v * osz, dout, tok * H * d_v * osz,
+                                         cudaMemcpyDeviceToHost, s_out), "kda_chunk_fwd_host: copy out");
+        KDA_HOST_TRY(cudaEventRecord(ev_out[slot], s_out), "kda_chunk_fwd_host: record");
+    }
+    if (final_state) {
+        KDA_HOST_TRY(cudaStreamWaitEvent(s_out, ev_comp[(pieces.size() - 1) % kHostSlots], 0), "kda_chunk_fwd_host: wait");
+        KDA_HOST_TRY(cudaMemcpyAsync(final_state, d_T, state_bytes, cudaMemcpyDeviceToHost, s_out), "kda_chunk_fwd_host: state out");
+    }
+    // the caller's stream reaches the end of the call once the last copy out is done
+    KDA_HOST_TRY(cudaEventRecord(ev_out[0], s_out), "kda_chunk_fwd_host: record");
+    KDA_HOST_TRY(cudaStreamWaitEvent(cs, ev_out[0], 0), "kda_chunk_fwd_host: wait");
+#undef KDA_HOST_TRY
+    cleanup();
+    return KDA_OK;
+}

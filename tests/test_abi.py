@@ -167,3 +167,26 @@ def test_chunk_bwd_rejects_bad_arguments():
     assert bwd(q=8) == kda.KDA_ERR_INVALID_ARG                    # misaligned
     assert bwd(N=0, T=0) == kda.KDA_OK
     assert kda.kda_chunk_bwd_workspace_size(8192, 1, 32, 128, 128) == (8192 // 32 + 1 + 32) * 32 * 128 * 128 * 4
+
+
+def test_host_prefill_validates_on_the_host():
+    import ctypes
+    import torch
+    cu = torch.tensor([0, 100, 260], dtype=torch.int32)
+    size = kda.kda_chunk_fwd_host_buffer_size(cu, 4, 128, 128)
+    assert size > 0
+    assert kda.kda_chunk_fwd_host_buffer_size(cu, 4, 128, 96) == 0                 # d
+    assert kda.kda_chunk_fwd_host_buffer_size(cu, 4, 128, 128, piece_tokens=32) == 0   # piece < 64
+    H = lib.kda_chunk_fwd_host
+    cu_p = ctypes.c_void_p(cu.data_ptr())
+    alog = torch.zeros(4)
+    al_p = ctypes.c_void_p(alog.data_ptr())
+    bad = torch.tensor([0, 120, 100], dtype=torch.int32)                            # not monotone
+    args = lambda cup, T, piece, buf, nbytes: (16, 16, 16, 16, 16, None, al_p, cup, 2, T, 4, 128, 128, 1.0, None,
+                                               None, 16, 0, piece, buf, nbytes, None)
+    assert H(*args(ctypes.c_void_p(bad.data_ptr()), 100, 0, 256, 1 << 40)) == kda.KDA_ERR_INVALID_ARG
+    assert H(*args(cu_p, 250, 0, 256, 1 << 40)) == kda.KDA_ERR_INVALID_ARG          # cu does not end at T
+    assert H(*args(cu_p, 260, 32, 256, 1 << 40)) == kda.KDA_ERR_INVALID_ARG         # piece < 64
+    assert H(*args(cu_p, 260, 0, None, 0)) == kda.KDA_ERR_INVALID_ARG               # no device buffer
+    assert H(*args(cu_p, 260, 0, 256, size - 1)) == kda.KDA_ERR_INVALID_ARG         # buffer too small
+    assert H(*args(cu_p, 260, 0, 16, size)) == kda.KDA_ERR_INVALID_ARG              # not 256-byte aligned
