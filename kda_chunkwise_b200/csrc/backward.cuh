@@ -26,6 +26,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "mma_frag.cuh"
+#include "async_copy.cuh"
 
 namespace kda {
 

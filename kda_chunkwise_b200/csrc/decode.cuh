@@ -35,21 +35,6 @@ __device__ __forceinline__ float4 f4_fma(float s, float4 x, float4 acc) {
     return acc;
 }
 
-// The column sums r and p of the four columns of column quad cq: the RPP row-group partials added
-// in row-group order, starting from zero -- the order in which the decode step's column threads
-// add them, so the verify pass (which uses this) reproduces the decode step bit for bit.
-template <int RPP, int LPR>
-__device__ __forceinline__ void quad_col_sums(const float4 (&red)[2][RPP][LPR], int cq, float4 &rr, float4 &pp) {
-    rr = make_float4(0.f, 0.f, 0.f, 0.f);
-    pp = rr;
-#pragma unroll
-    for (int g = 0; g < RPP; ++g) {
-        const float4 a = red[0][g][cq], b = red[1][g][cq];
-        rr.x += a.x; rr.y += a.y; rr.z += a.z; rr.w += a.w;
-        pp.x += b.x; pp.y += b.y; pp.z += b.z; pp.w += b.w;
-    }
-}
-
 constexpr int kDecodeThreads = 256;
 
 template <int DK, int DV>

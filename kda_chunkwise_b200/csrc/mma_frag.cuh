@@ -161,11 +161,6 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, int s
                  : "memory");
 }
 
-// 4-byte asynchronous global->shared copy
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
-}
-
 // ---- mbarriers and the cluster ------------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
