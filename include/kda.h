@@ -220,7 +220,7 @@ KDA_API kda_status kda_decode_commit(const void *k, const void *a, const float *
  * optionally followed (l2norm != 0) by y_t[h] <- y_t[h] / sqrt(|y_t[h]|^2 + 1e-12).
  *   x, y  bf16 [total_tokens, H, d] (d = 64 or 128; y may not alias x)
  *   w     fp32 [H, d, width], 1 <= width <= 4
- *   cu_seqlens int32 [num_seqs + 1] (device), as for kda_chunk_fwd.  At most 2,097,120 tokens.
+ *   cu_seqlens int32 [num_seqs + 1] (device), as for kda_chunk_fwd.
  * Malformed cu_seqlens are reported through the error word.
  */
 KDA_API kda_status kda_short_conv(const void *x, const float *w, const int32_t *cu_seqlens, int32_t num_seqs,

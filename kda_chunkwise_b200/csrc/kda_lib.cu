@@ -442,15 +442,27 @@ kda_status kda_short_conv(const void *x, const float *w, const int32_t *cu_seqle
     p.H = H;
     p.width = width;
     p.l2norm = l2norm != 0;
-    const int64_t runs = (total_tokens + kda::kConvRun - 1) / kda::kConvRun;
-    if (runs > 65535) return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: more than 2,097,120 tokens per call");
     const int64_t groups = (int64_t)H * (d / 8);
-    const dim3 grid((unsigned)((groups + kda::kPrepThreads - 1) / kda::kPrepThreads), (unsigned)runs);
+    const int64_t cblocks = (groups + kda::kPrepThreads - 1) / kda::kPrepThreads;
+    if (cblocks > 65535) return fail(KDA_ERR_INVALID_ARG, "kda_short_conv: H * d too large");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (d == 128) kda::short_conv_kernel<128><<<grid, kda::kPrepThreads, 0, st>>>(p);
-    else kda::short_conv_kernel<64><<<grid, kda::kPrepThreads, 0, st>>>(p);
+    auto kern = d == 128 ? kda::short_conv_kernel<128> : kda::short_conv_kernel<64>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kda::kConvSmem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(short_conv)");
+    // one run of consecutive tokens per CTA, as many CTAs as the device holds at once
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kda::kPrepThreads, kda::kConvSmem)) != cudaSuccess)
+        return cuda_fail(e, "short_conv occupancy");
+    if (per_sm < 1) return fail(KDA_ERR_UNSUPPORTED, "kda_short_conv: kernel does not fit on an SM");
+    const int64_t want = std::max<int64_t>(1, (int64_t)sms * per_sm / cblocks);
+    const int64_t run_len = std::max<int64_t>(kda::kConvAhead, (total_tokens + want - 1) / want);
+    const int64_t runs = (total_tokens + run_len - 1) / run_len;
+    const dim3 grid((unsigned)runs, (unsigned)cblocks);
+    kern<<<grid, kda::kPrepThreads, kda::kConvSmem, st>>>(p, run_len);
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    const cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "short_conv launch");
 }
 

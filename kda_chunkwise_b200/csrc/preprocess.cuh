@@ -13,13 +13,14 @@
 #pragma once
 
 #include "common.cuh"
+#include "mma_frag.cuh"
 
 namespace kda {
 
 constexpr int kConvMaxWidth = 4;
-constexpr int kConvRun = 32;          // tokens per thread (history rows are re-read once per run)
-constexpr int kConvBatch = 4;         // rows loaded together
+constexpr int kConvAhead = 16;        // input rows in flight per thread (a power of two)
 constexpr int kPrepThreads = 256;
+constexpr int kConvSmem = kConvAhead * kPrepThreads * 16;
 
 struct ConvParams {
     const uint16_t *x;        // [T, H, d] bf16
@@ -59,99 +60,121 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
     return make_uint4(w4[0], w4[1], w4[2], w4[3]);
 }
 
-// grid: x = column groups of 8 channels (H d / 8 per row) / kPrepThreads, y = runs of kConvRun
-// tokens.  A thread keeps its 8 channels' taps in registers for the whole run and slides a window
-// of the last W - 1 input rows; the run's rows are loaded kConvBatch at a time so that several
-// loads are in flight.
+// grid: x = runs of consecutive tokens (as many as fill the device once), y = blocks of
+// kPrepThreads column groups (8 channels each, H d / 8 per token row).  A thread owns one column
+// group for the whole run: its 8 channels' taps and the last W - 1 input rows stay in registers
+// (each input is converted once), and its next kConvAhead input rows are always in flight --
+// asynchronous 16-byte copies into a ring in shared memory that only this thread reads, so no
+// barrier is needed and no registers are held for the rows in flight.
 template <int D>
-__global__ void __launch_bounds__(kPrepThreads) short_conv_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kPrepThreads) short_conv_kernel(const ConvParams p, int64_t run_len) {
+    extern __shared__ __align__(16) uint4 conv_ring[];   // [kConvAhead][kPrepThreads]
     constexpr int LPH = D / 8;                        // lanes per (token, head) row
     const int64_t groups = (int64_t)p.H * LPH;        // 8-channel groups per token row
-    const int64_t g = (int64_t)blockIdx.x * kPrepThreads + threadIdx.x;
+    const int64_t g = (int64_t)blockIdx.y * kPrepThreads + threadIdx.x;
     const bool active = g < groups;                   // whole (token, head) rows share a warp
     const int h = static_cast<int>(g / LPH);
     const int c0 = static_cast<int>(g % LPH) * 8;
-    const int64_t t_begin = (int64_t)blockIdx.y * kConvRun;
+    const int64_t t_begin = (int64_t)blockIdx.x * run_len;
     if (t_begin >= p.total_tokens) return;
-    const int64_t t_end = min64(t_begin + kConvRun, p.total_tokens);
+    const int64_t t_end = min64(t_begin + run_len, p.total_tokens);
     const int W = p.width;
+    const uint16_t *xcol = p.x + (int64_t)h * D + c0;   // row t at xcol + t H D
+    const int64_t rstride = (int64_t)p.H * D;
 
-    // taps on the history (zero beyond W - 1) and the tap on the current token
+    // the first kConvAhead rows of the run in flight (one commit group per row, empty past the end)
+    const uint32_t ring = smem_u32(conv_ring) + threadIdx.x * 16;
+#pragma unroll 1
+    for (int i = 0; i < kConvAhead; ++i) {
+        if (active && t_begin + i < t_end) cp_async_16(ring + i * kPrepThreads * 16, xcol + (t_begin + i) * rstride, 16);
+        cp_async_commit();
+    }
+
+    // taps: slot k of the window holds x_{t-3+k}; the tap of x_{t-(W-1)+j} sits on slot 4 - W + j
     float wt[8][kConvMaxWidth - 1], wcur[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const float *wc = p.w + ((int64_t)h * D + c0 + c) * W;
 #pragma unroll
-        for (int j = 0; j < kConvMaxWidth - 1; ++j) wt[c][j] = (active && j < W - 1) ? wc[j] : 0.f;
+        for (int k = 0; k < kConvMaxWidth - 1; ++k) {
+            const int j = k - (kConvMaxWidth - W);
+            wt[c][k] = (active && j >= 0) ? wc[j] : 0.f;
+        }
         wcur[c] = active ? wc[W - 1] : 0.f;
     }
+    const int k0 = kConvMaxWidth - W;   // first window slot with a tap
 
     int s = seq_of(p.cu, p.num_seqs, t_begin);
     int64_t s_start = p.cu[s], s_end = p.cu[s + 1];
-    // history window: hist[j] = x_{t - (W-1) + j} for j < W - 1 (zero before the sequence start)
-    float hist[kConvMaxWidth - 1][8];
+    // the window before the run: rows t_begin - 3 .. t_begin - 1 of the same sequence, else zero
+    float win[kConvMaxWidth - 1][8];
 #pragma unroll
-    for (int j = 0; j < kConvMaxWidth - 1; ++j) {
-        const int64_t tj = t_begin - (W - 1) + j;
+    for (int k = 0; k < kConvMaxWidth - 1; ++k) {
+        const int64_t tk = t_begin - (kConvMaxWidth - 1) + k;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) hist[j][c] = 0.f;
-        if (active && j < W - 1 && tj >= s_start) load8(p.x + (tj * p.H + h) * D + c0, hist[j]);
+        for (int c = 0; c < 8; ++c) win[k][c] = 0.f;
+        if (active && k >= k0 && tk >= s_start) load8(xcol + tk * rstride, win[k]);
     }
-    for (int64_t tb = t_begin; tb < t_end; tb += kConvBatch) {
-        float xs[kConvBatch][8];
+
+    const uint16_t *src = xcol + (t_begin + kConvAhead) * rstride;   // the next row to request
+    uint16_t *dst = p.y + t_begin * rstride + (int64_t)h * D + c0;
+    int slot = 0;
+#pragma unroll 4
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        cp_async_wait_group<kConvAhead - 1>();   // row t has landed
+        const uint4 u = conv_ring[slot * kPrepThreads + threadIdx.x];
+        // row t + kConvAhead into the slot just read (this thread's own slot: read, then refilled)
+        if (active && t + kConvAhead < t_end) cp_async_16(ring + slot * (kPrepThreads * 16), src, 16);
+        cp_async_commit();
+        src += rstride;
+        slot = (slot + 1) & (kConvAhead - 1);
+        if (t >= s_end) {   // a new sequence starts here: its history is zero
+            while (t >= s_end && s + 1 < p.num_seqs) { ++s; s_start = p.cu[s]; s_end = p.cu[s + 1]; }
+            if (t >= s_end && threadIdx.x == 0) atomicOr(&g_kda_error_word, kErrBadSeqlens);
 #pragma unroll
-        for (int u = 0; u < kConvBatch; ++u) {
+            for (int k = 0; k < kConvMaxWidth - 1; ++k)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) xs[u][c] = 0.f;
-            if (active && tb + u < t_end) load8(p.x + ((tb + u) * p.H + h) * D + c0, xs[u]);
+                for (int c = 0; c < 8; ++c) win[k][c] = 0.f;
         }
+        float xv[8];
+        {
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int u = 0; u < kConvBatch; ++u) {
-            const int64_t t = tb + u;
-            if (t >= t_end) break;   // the same for the whole block
-            if (t >= s_end) {        // a new sequence starts here: its history is zero
-                while (t >= s_end && s + 1 < p.num_seqs) { ++s; s_start = p.cu[s]; s_end = p.cu[s + 1]; }
-                if (t >= s_end && threadIdx.x == 0) atomicOr(&g_kda_error_word, kErrBadSeqlens);
-#pragma unroll
-                for (int j = 0; j < kConvMaxWidth - 1; ++j)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) hist[j][c] = 0.f;
-            }
-            float y[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float acc = wcur[c] * xs[u][c];
-#pragma unroll
-                for (int j = 0; j < kConvMaxWidth - 1; ++j) acc = fmaf(wt[c][j], hist[j][c], acc);
-                y[c] = acc;
-            }
-            if (p.l2norm) {
-                float ss = 0.f;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) ss = fmaf(y[c], y[c], ss);
-#pragma unroll
-                for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                const float inv = rsqrtf(ss + 1e-12f);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) y[c] *= inv;
-            }
-            if (active) *reinterpret_cast<uint4 *>(p.y + (t * p.H + h) * D + c0) = pack8_bf16(y);
-            // slide the window: hist[j] <- hist[j + 1], newest = x_t
-#pragma unroll
-            for (int j = 0; j < kConvMaxWidth - 2; ++j)
-                if (j < W - 2)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) hist[j][c] = hist[j + 1][c];
-            if (W >= 2) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (W == 2) hist[0][c] = xs[u][c];
-                    else if (W == 3) hist[1][c] = xs[u][c];
-                    else hist[2][c] = xs[u][c];
-                }
+            for (int q = 0; q < 4; ++q) {
+                xv[2 * q] = bf16_to_f32(static_cast<uint16_t>(w4[q] & 0xFFFFu));
+                xv[2 * q + 1] = bf16_to_f32(static_cast<uint16_t>(w4[q] >> 16));
             }
         }
+        float y[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            float acc = wcur[c] * xv[c];
+#pragma unroll
+            for (int k = 0; k < kConvMaxWidth - 1; ++k)
+                if (k >= k0) acc = fmaf(wt[c][k], win[k][c], acc);
+            y[c] = acc;
+        }
+        if (p.l2norm) {
+            float ss = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) ss = fmaf(y[c], y[c], ss);
+#pragma unroll
+            for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float inv = rsqrtf(ss + 1e-12f);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) y[c] *= inv;
+        }
+        if (active) *reinterpret_cast<uint4 *>(dst) = pack8_bf16(y);
+        dst += rstride;
+        // slide the window
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            win[0][c] = win[1][c];
+            win[1][c] = win[2][c];
+            win[2][c] = xv[c];
+        }
     }
+    cp_async_wait_all();   // nothing left in flight at exit
 }
 
 struct NormGateParams {
