@@ -44,7 +44,9 @@ NCU_TRAFFIC = {
     "decode_N256_H64_d128_512steps": {"bytes_per_launch": 2114315008, "src": "1c3a7d12c8610c04"},
     # one verify launch plus one commit launch (round 4 of the captured run; commit's bytes depend on
     # how many sequences accepted at least one token)
-    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1182260224 + 1765504000, "src": "089cfaaf3b46dbfe"},
+    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1208901160 + 1765829120, "src": "187088189b7c5759"},
+    # kda_chunk_bwd on the prefill workload (ncu prints these two counters to three digits)
+    "bwd_prefill_B1_H32_T8192_d128": {"bytes_per_launch": 1.30e9 + 2.55e9, "src": "733838d1f4904973"},
 }
 
 
@@ -116,6 +118,7 @@ KERNEL_SOURCES = {
     "prefill": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh"),
     "decode": ("common.cuh", "decode.cuh"),
     "speculative": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "speculative.cuh"),
+    "backward": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "backward.cuh"),
 }
 
 
@@ -401,7 +404,8 @@ def main():
         backward = {"value": whole_job_rate(w.total_tokens, world, bms), "unit": "tokens/s", "ms_per_step": bms,
                     "workload": w.name, "scope": "one kda_chunk_bwd call",
                     "roofline": {"bound": "latency (sequential token steps per unit)", "achieved": bach,
-                                 "peak": hbm, "unit": "GB/s", "frac": bach / hbm, "traffic": None,
+                                 "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
+                                 "traffic": ncu_traffic("bwd_" + w.name, "backward"),
                                  "peak_source": f"hbm_gbs of {peak_src}", "algorithmic_bytes": bbytes}}
         del dout, dST, bws
         torch.cuda.empty_cache()

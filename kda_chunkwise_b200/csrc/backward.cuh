@@ -97,6 +97,34 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
     return v;
 }
 
+// The recomputed states S' (the scratch) are written and read back within a chunk: they are kept in
+// L2 with an evict-last policy so that the streamed inputs and gradients do not push them out.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void st_keep(float4 *p, float4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;\n" ::"l"(p), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+
+__device__ __forceinline__ float4 ld_keep(const float4 *p, uint64_t pol) {
+    float4 v;
+    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;\n"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol)
+                 : "memory");
+    return v;
+}
+
+// drop a 128-byte line of scratch from L2 without writing it back (its contents are dead)
+__device__ __forceinline__ void l2_discard(const void *p) {
+    asm volatile("discard.global.L2 [%0], 128;\n" ::"l"(p) : "memory");
+}
+
 // streaming (evict-first) store of a gradient that is never read again here
 __device__ __forceinline__ void st_stream(float *p, float4 v) { __stcs(reinterpret_cast<float4 *>(p), v); }
 
@@ -156,6 +184,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
     const size_t SZ = (size_t)DK * DV, SL = (size_t)DK * DC;
     const int col0 = rank * DC + 4 * cq;   // first of this thread's four value columns
     float4 *scratch = reinterpret_cast<float4 *>(p.scratch + (size_t)unit * C * SZ + (size_t)rank * C * SL);
+    const uint64_t keep = l2_evict_last_policy();
     auto ck_ptr = [&](int c) {
         return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(ckbase + c) * H + h) * SZ + (size_t)rank * SL);
     };
@@ -249,7 +278,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
             const float al = sAl[i * DK + row];
             kk[m] = bf16_to_f32(sK[i * DK + row]);
             S[m].x *= al; S[m].y *= al; S[m].z *= al; S[m].w *= al;
-            if (save) save[m * NT + tid] = S[m];
+            if (save) st_keep(save + m * NT + tid, S[m], keep);
             r = f4_fma(kk[m], S[m], r);
         }
         r = warp_rows_sum(r);
@@ -310,8 +339,8 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
 #pragma unroll
         for (int m = 0; m < NR; ++m) {
             const float al = sAl[(L - 1) * DK + rg + 32 * m];
-            scratch[(size_t)((L - 1) * NR + m) * NT + tid] =
-                make_float4(al * S[m].x, al * S[m].y, al * S[m].z, al * S[m].w);
+            st_keep(scratch + (size_t)((L - 1) * NR + m) * NT + tid,
+                    make_float4(al * S[m].x, al * S[m].y, al * S[m].z, al * S[m].w), keep);
         }
         // undo the chunk's tokens in reverse order; S' and the row inputs of token i - 1 are fetched
         // while token i runs
@@ -320,7 +349,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
 #pragma unroll
         for (int m = 0; m < NR; ++m) {
             const int row = rg + 32 * m;
-            Spn[m] = scratch[(size_t)((L - 1) * NR + m) * NT + tid];
+            Spn[m] = ld_keep(scratch + (size_t)((L - 1) * NR + m) * NT + tid, keep);
             kkn[m] = bf16_to_f32(sK[(L - 1) * DK + row]);
             qqn[m] = p.scale * bf16_to_f32(sQ[(L - 1) * DK + row]);
             aln[m] = sAl[(L - 1) * DK + row];
@@ -334,7 +363,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
 #pragma unroll
                 for (int m = 0; m < NR; ++m) {
                     const int row = rg + 32 * m;
-                    Spn[m] = scratch[(size_t)((i - 1) * NR + m) * NT + tid];
+                    Spn[m] = ld_keep(scratch + (size_t)((i - 1) * NR + m) * NT + tid, keep);
                     kkn[m] = bf16_to_f32(sK[(i - 1) * DK + row]);
                     qqn[m] = p.scale * bf16_to_f32(sQ[(i - 1) * DK + row]);
                     aln[m] = sAl[(i - 1) * DK + row];
@@ -469,6 +498,12 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
             p.dbeta[(tc + i) * H + h] = db;
         }
         cluster_sync();   // every CTA is done reading the row sums before they are overwritten
+    }
+    // the scratch is dead: drop it from L2 rather than write it back (every read of it came before
+    // the last cluster barrier, which every thread of this CTA has passed)
+    if (nck > 0) {
+        const char *sc = reinterpret_cast<const char *>(scratch);
+        for (int i = tid; i < C * NR * NT * 16 / 128; i += NT) l2_discard(sc + (size_t)i * 128);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dA_acc += __shfl_xor_sync(0xffffffffu, dA_acc, o);
