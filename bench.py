@@ -117,7 +117,7 @@ def peaks():
 KERNEL_SOURCES = {
     "prefill": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh"),
     "decode": ("common.cuh", "decode.cuh"),
-    "speculative": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "speculative.cuh"),
+    "speculative": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "f32x2.cuh", "speculative.cuh"),
     "backward": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "backward.cuh"),
 }
 

@@ -23,6 +23,7 @@
 #include "decode.cuh"
 #include "mma_frag.cuh"
 #include "async_copy.cuh"
+#include "f32x2.cuh"
 
 namespace kda {
 
@@ -123,9 +124,9 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
         const int h = static_cast<int>(nh % p.H);
         cp_async_wait_all();
         __syncthreads();   // this unit's copies have landed (every thread's)
-        float4 S[NR];
+        ulonglong2 S[NR];   // this thread's four columns of each row, as two packed pairs
 #pragma unroll
-        for (int m = 0; m < NR; ++m) S[m] = sS[(rg + m * RPP) * LPR + cq];
+        for (int m = 0; m < NR; ++m) S[m] = reinterpret_cast<const ulonglong2 *>(sS)[(rg + m * RPP) * LPR + cq];
         const float expA = expf(p.A_log[h]);
         for (int e = tid; e < K * DK; e += kThreads) {
             s_alpha[e] = __expf(log_decay(bf16_to_f32(r_a[e]), expA));
@@ -150,18 +151,23 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
 
         for (int t = 0; t < K; ++t) {
             const int64_t tok = (n * K + t) * p.H + h;
-            float4 r = make_float4(0.f, 0.f, 0.f, 0.f), pq = r;
+            // the decode step's arithmetic, two columns per instruction (same roundings, same bits)
+            ulonglong2 r = make_ulonglong2(0ull, 0ull), pq = r;
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
                 const int row = rg + m * RPP;
-                const float al = s_alpha[t * DK + row];
-                S[m].x *= al; S[m].y *= al; S[m].z *= al; S[m].w *= al;
-                r = f4_fma(s_k[t * DK + row], S[m], r);
-                pq = f4_fma(s_q[t * DK + row], S[m], pq);
+                const f32x2 al = f2_splat(s_alpha[t * DK + row]);
+                const f32x2 kk = f2_splat(s_k[t * DK + row]), qq = f2_splat(s_q[t * DK + row]);
+                S[m].x = f2_mul(S[m].x, al);
+                S[m].y = f2_mul(S[m].y, al);
+                r.x = f2_fma(kk, S[m].x, r.x);
+                r.y = f2_fma(kk, S[m].y, r.y);
+                pq.x = f2_fma(qq, S[m].x, pq.x);
+                pq.y = f2_fma(qq, S[m].y, pq.y);
             }
             float4 (&red)[2][RPP][LPR] = s_red[t & 1];
-            red[0][rg][cq] = r;
-            red[1][rg][cq] = pq;
+            reinterpret_cast<ulonglong2 &>(red[0][rg][cq]) = r;
+            reinterpret_cast<ulonglong2 &>(red[1][rg][cq]) = pq;
             __syncthreads();   // (the k . q of every token is ready too)
             float4 rr, pp;
             quad_col_sums<RPP, LPR>(red, cq, rr, pp);
@@ -179,13 +185,12 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
 #pragma unroll
                 for (int c = 0; c < 4; ++c) store_out(p.out, tok * DV + 4 * cq + c, p.out_f32, o[c]);
             }
+            const f32x2 u01 = f2_pack(u4.x, u4.y), u23 = f2_pack(u4.z, u4.w);
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
-                const float kk = s_k[t * DK + rg + m * RPP];
-                S[m].x = fmaf(kk, u4.x, S[m].x);
-                S[m].y = fmaf(kk, u4.y, S[m].y);
-                S[m].z = fmaf(kk, u4.z, S[m].z);
-                S[m].w = fmaf(kk, u4.w, S[m].w);
+                const f32x2 kk = f2_splat(s_k[t * DK + rg + m * RPP]);
+                S[m].x = f2_fma(kk, u01, S[m].x);
+                S[m].y = f2_fma(kk, u23, S[m].y);
             }
         }
         __syncthreads();   // the derived inputs are read by every thread before the next unit's
