@@ -131,8 +131,9 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const voi
  *   device_buffer: caller-owned device memory, 256-byte aligned, of
  *     kda_chunk_fwd_host_buffer_size(...) bytes: two staging slots, the prefill workspace and the
  *     states.
- * The batch is cut into pieces along the packed token axis; a cut inside a sequence falls on a
- * 64-token chunk boundary of that sequence, so every piece runs the chunks the whole call would,
+ * The batch is cut into pieces along the packed token axis (the last piece cut again 3 : 1 so that
+ * little is left to copy out at the end); a cut inside a sequence falls on a 64-token chunk
+ * boundary of that sequence, so every piece runs the chunks the whole call would,
  * and a sequence that continues into the next piece hands its state over on the device.  The
  * host-to-device copy of piece i+1, the prefill of piece i (on `stream`) and the device-to-host
  * copy of piece i-1 run on three streams at once.  Asynchronous with respect to the host: the

@@ -630,26 +630,41 @@ struct HostPiece {
 // 64-token chunk boundary of that sequence, so each piece runs exactly the chunks the whole call
 // would.  Sequence n takes part in the piece where it starts (an empty one at the very end, in the
 // last piece) and in every piece it continues into.
+// A cut at or below token e (0 < e < T) on a 64-token chunk boundary of the sequence containing e;
+// -1 if cu_seqlens does not cover e.
+int64_t chunk_cut(const int32_t *cu, int32_t N, int64_t e) {
+    int32_t m = 0;
+    while (m < N && cu[m + 1] <= e) ++m;
+    if (m >= N) return -1;
+    return cu[m] + ((e - cu[m]) / kda::kChunk) * kda::kChunk;
+}
+
 bool plan_pieces(const int32_t *cu, int32_t N, int64_t T, int64_t piece, std::vector<HostPiece> &out) {
     out.clear();
-    int64_t a = 0;
-    do {
+    std::vector<int64_t> cuts{0};
+    for (int64_t a = 0; a < T;) {
         int64_t e = std::min<int64_t>(a + piece, T);
-        if (e < T) {   // move the cut down to a chunk boundary of the sequence containing token e
-            int32_t m = 0;
-            while (m < N && cu[m + 1] <= e) ++m;
-            if (m >= N) return false;
-            e = cu[m] + ((e - cu[m]) / kda::kChunk) * kda::kChunk;
+        if (e < T) {
+            e = chunk_cut(cu, N, e);
             if (e <= a) return false;   // not reached for piece >= 64: a is a boundary of its own
+        } else if (T - a >= 4 * kda::kChunk) {
+            // the last piece is cut 3 : 1, so that little is left to copy out after the last prefill
+            const int64_t m = chunk_cut(cu, N, a + 3 * (T - a) / 4);
+            if (m > a && m < T) cuts.push_back(m);
         }
+        cuts.push_back(e);
+        a = e;
+    }
+    if (T == 0) cuts.push_back(0);   // one empty piece: the zero-length sequences' states
+    for (size_t i = 0; i + 1 < cuts.size(); ++i) {
+        const int64_t a = cuts[i], e = cuts[i + 1];
         int32_t lo = 0;   // first sequence not finished before a (empty ones starting at a included)
         while (lo < N && cu[lo + 1] <= a && cu[lo] < a) ++lo;
         int32_t hi = lo;  // last sequence starting before e (every remaining one in the last piece)
         while (hi + 1 < N && (e == T || cu[hi + 1] < e)) ++hi;
         if (lo >= N) return false;
         out.push_back({a, e, lo, hi, e < T && cu[hi + 1] > e});
-        a = e;
-    } while (a < T);
+    }
     return true;
 }
 
