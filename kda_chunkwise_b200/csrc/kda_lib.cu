@@ -96,8 +96,22 @@ kda_status launch_decode(const kda::DecodeParams &p, int64_t units, cudaStream_t
 
 template <int DK, int DV>
 kda_status launch_spec(const kda::SpecParams &p, int64_t units, bool commit, cudaStream_t stream) {
-    if (commit) kda::spec_commit_kernel<DK, DV><<<(unsigned)units, kda::kSpecThreads, 0, stream>>>(p);
-    else {
+    if (commit) {
+        // persistent: as many CTAs as fit on the device at once (at most one per unit)
+        const size_t smem = kda::SpecCommitSmem<DK, DV>::bytes(p.K);
+        cudaError_t e = cudaFuncSetAttribute(kda::spec_commit_kernel<DK, DV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_commit)");
+        int dev = 0, sms = 0, per_sm = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda::spec_commit_kernel<DK, DV>,
+                                                               kda::kSpecThreads, smem)) != cudaSuccess)
+            return cuda_fail(e, "decode_commit occupancy");
+        if (per_sm < 1) return fail(KDA_ERR_UNSUPPORTED, "kda_decode_commit: kernel does not fit on an SM");
+        const int64_t grid = units < (int64_t)per_sm * sms ? units : (int64_t)per_sm * sms;
+        kda::spec_commit_kernel<DK, DV><<<(unsigned)grid, kda::kSpecThreads, smem, stream>>>(p, units);
+    } else {
         // persistent: as many CTAs as fit on the device at once (at most one per unit)
         const size_t smem = kda::SpecVerifySmem<DK, DV>::bytes(p.K);
         cudaError_t e = cudaFuncSetAttribute(kda::spec_verify_kernel<DK, DV>,

@@ -198,57 +198,111 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
     cp_async_wait_all();   // nothing is left in flight at exit
 }
 
+// Dynamic shared memory of the commit kernel: the next state (fp32, its global layout), the next
+// unit's raw inputs (bf16 a, k [K][DK]; fp32 write vectors u [K][DV]) and the current unit's alpha
+// and k [K][DK] and write vectors [K][DV] (fp32).
 template <int DK, int DV>
-__global__ void __launch_bounds__(kSpecThreads) spec_commit_kernel(const SpecParams p) {
+struct SpecCommitSmem {
+    __host__ __device__ static size_t raw_off() { return (size_t)DK * DV * 4; }
+    __host__ __device__ static size_t u_off(int K) { return raw_off() + (size_t)K * 2 * DK * 2; }
+    __host__ __device__ static size_t derived_off(int K) { return u_off(K) + (size_t)K * DV * 4; }
+    __host__ __device__ static size_t bytes(int K) { return derived_off(K) + (size_t)K * (2 * DK + DV) * 4; }
+};
+
+// Persistent, like the verify pass: while one state takes its accepted updates and is written
+// back, the next state that accepted anything (and its inputs) is copied into shared memory.
+// States whose sequence accepted nothing are neither read nor written.
+template <int DK, int DV>
+__global__ void __launch_bounds__(kSpecThreads) spec_commit_kernel(const SpecParams p, int64_t units) {
     constexpr int kThreads = kSpecThreads;
     constexpr int LPR = DV / 4;
     constexpr int RPP = kThreads / LPR;
     constexpr int NR = DK / RPP;
+    using SL = SpecCommitSmem<DK, DV>;
 
-    __shared__ float s_alpha[kSpecMaxTokens][DK], s_k[kSpecMaxTokens][DK];
-    __shared__ __align__(16) float s_uw[kSpecMaxTokens][DV];
+    extern __shared__ __align__(16) unsigned char spec_dyn[];
+    const int K = p.K;
+    const float4 *sS = reinterpret_cast<const float4 *>(spec_dyn);
+    const uint16_t *r_a = reinterpret_cast<const uint16_t *>(spec_dyn + SL::raw_off()), *r_k = r_a + K * DK;
+    const float *r_u = reinterpret_cast<const float *>(spec_dyn + SL::u_off(K));
+    float *s_alpha = reinterpret_cast<float *>(spec_dyn + SL::derived_off(K)), *s_k = s_alpha + K * DK;
+    float *s_u = s_k + K * DK;
 
-    const int64_t nh = blockIdx.x;
-    const int64_t n = nh / p.H;
-    const int h = static_cast<int>(nh % p.H);
     const int tid = threadIdx.x;
     const int cq = tid % LPR, rg = tid / LPR;
-
-    int j = p.accepted[n];
-    if (j < 0 || j > p.K) {
-        if (tid == 0 && h == 0) atomicOr(&g_kda_error_word, kErrBadAccepted);
-        j = j < 0 ? 0 : p.K;
-    }
-    if (j == 0) return;   // nothing accepted: the state stays as it is
-
-    // the state's loads are issued first so that they overlap the staging of the small inputs
-    float4 *St = reinterpret_cast<float4 *>(p.state + nh * (int64_t)(DK * DV));
-    float4 S[NR];
-#pragma unroll
-    for (int m = 0; m < NR; ++m) S[m] = __ldcs(St + (rg + m * RPP) * LPR + cq);
-    const float expA = expf(p.A_log[h]);
-    for (int e = tid; e < j * DK; e += kThreads) {
-        const int t = e / DK, i = e % DK;
-        const int64_t tok = (n * p.K + t) * p.H + h;
-        s_alpha[t][i] = __expf(log_decay(bf16_to_f32(p.a[tok * DK + i]), expA));
-        s_k[t][i] = bf16_to_f32(p.k[tok * DK + i]);
-    }
-    for (int e = tid; e < j * DV; e += kThreads) s_uw[e / DV][e % DV] = __ldcs(p.u + (nh * p.K + e / DV) * DV + e % DV);
-    __syncthreads();
-    for (int t = 0; t < j; ++t) {
-        const float4 u4 = reinterpret_cast<const float4 *>(s_uw[t])[cq];
-#pragma unroll
-        for (int m = 0; m < NR; ++m) {
-            const int row = rg + m * RPP;
-            const float al = s_alpha[t][row], kk = s_k[t][row];
-            S[m].x = fmaf(kk, u4.x, al * S[m].x);
-            S[m].y = fmaf(kk, u4.y, al * S[m].y);
-            S[m].z = fmaf(kk, u4.z, al * S[m].z);
-            S[m].w = fmaf(kk, u4.w, al * S[m].w);
+    auto accepted = [&](int64_t nh) {   // the accepted count of unit nh's sequence, clamped to [0, K]
+        const int64_t n = nh / p.H;
+        int j = p.accepted[n];
+        if (j < 0 || j > K) {
+            if (tid == 0 && nh % p.H == 0) atomicOr(&g_kda_error_word, kErrBadAccepted);
+            j = j < 0 ? 0 : K;
         }
-    }
+        return j;
+    };
+    auto issue = [&](int64_t nh, int j) {   // asynchronous copy of unit nh's state and first j tokens' inputs
+        const int64_t n = nh / p.H;
+        const int h = static_cast<int>(nh % p.H);
+        const uint32_t base = smem_u32(spec_dyn);
+        const float *St = p.state + nh * (int64_t)(DK * DV);
+        for (int e = tid; e < DK * DV / 4; e += kThreads) cp_async_16(base + e * 16, St + e * 4, 16);
+        const uint32_t raw = base + (uint32_t)SL::raw_off();
+        for (int e = tid; e < j * (2 * DK / 8); e += kThreads) {   // a, k rows: 16 bytes = 8 values
+            const int which = e / (j * DK / 8), r = e % (j * DK / 8), t = r / (DK / 8), c8 = r % (DK / 8);
+            const uint16_t *src = which == 0 ? p.a : p.k;
+            cp_async_16(raw + ((which * K + t) * DK + c8 * 8) * 2, src + ((n * K + t) * p.H + h) * DK + c8 * 8, 16);
+        }
+        const uint32_t ru = base + (uint32_t)SL::u_off(K);
+        for (int e = tid; e < j * (DV / 4); e += kThreads)
+            cp_async_16(ru + e * 16, p.u + (nh * K) * DV + e * 4, 16);
+        cp_async_commit();
+    };
+    auto next_unit = [&](int64_t nh, int &j) {   // the first unit from nh on that accepted anything
+        for (; nh < units; nh += gridDim.x)
+            if ((j = accepted(nh)) > 0) return nh;
+        return units;
+    };
+
+    int j = 0;
+    int64_t nh = next_unit(blockIdx.x, j);
+    if (nh < units) issue(nh, j);
+    while (nh < units) {
+        const int h = static_cast<int>(nh % p.H);
+        cp_async_wait_all();
+        __syncthreads();   // this unit's copies have landed (every thread's)
+        float4 S[NR];
 #pragma unroll
-    for (int m = 0; m < NR; ++m) __stcs(St + (rg + m * RPP) * LPR + cq, S[m]);
+        for (int m = 0; m < NR; ++m) S[m] = sS[(rg + m * RPP) * LPR + cq];
+        const float expA = expf(p.A_log[h]);
+        for (int e = tid; e < j * DK; e += kThreads) {
+            s_alpha[e] = __expf(log_decay(bf16_to_f32(r_a[e]), expA));
+            s_k[e] = bf16_to_f32(r_k[e]);
+        }
+        for (int e = tid; e < j * DV / 4; e += kThreads)
+            reinterpret_cast<float4 *>(s_u)[e] = reinterpret_cast<const float4 *>(r_u)[e];
+        __syncthreads();   // the state and raw buffers are free for the next unit
+        int j2 = 0;
+        const int64_t nh2 = next_unit(nh + gridDim.x, j2);
+        if (nh2 < units) issue(nh2, j2);
+        for (int t = 0; t < j; ++t) {
+            const float4 u4 = reinterpret_cast<const float4 *>(s_u + t * DV)[cq];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) {
+                const int row = rg + m * RPP;
+                const float al = s_alpha[t * DK + row], kk = s_k[t * DK + row];
+                S[m].x = fmaf(kk, u4.x, al * S[m].x);
+                S[m].y = fmaf(kk, u4.y, al * S[m].y);
+                S[m].z = fmaf(kk, u4.z, al * S[m].z);
+                S[m].w = fmaf(kk, u4.w, al * S[m].w);
+            }
+        }
+        float4 *St = reinterpret_cast<float4 *>(p.state + nh * (int64_t)(DK * DV));
+#pragma unroll
+        for (int m = 0; m < NR; ++m) __stcs(St + (rg + m * RPP) * LPR + cq, S[m]);
+        __syncthreads();   // alpha, k and u are read by every thread before the next unit's
+        nh = nh2;
+        j = j2;
+    }
+    cp_async_wait_all();   // nothing is left in flight at exit
 }
 
 }  // namespace kda
