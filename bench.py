@@ -44,8 +44,8 @@ NCU_TRAFFIC = {
     "decode_N256_H64_d128_512steps": {"bytes_per_launch": 2114315008, "src": "1c3a7d12c8610c04"},
     # one verify launch plus one commit launch (round 4 of the captured run; commit's bytes depend on
     # how many sequences accepted at least one token)
-    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1158002176 + 49377536 + 930625536 + 830890752,
-                              "src": "4b4ed810e0504490"},
+    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1158005248 + 49608192 + 930634752 + 830197504,
+                              "src": "1b85ba110de6be44"},
     # kda_chunk_bwd on the prefill workload (ncu prints these two counters to three digits)
     "bwd_prefill_B1_H32_T8192_d128": {"bytes_per_launch": 1.30e9 + 2.55e9, "src": "733838d1f4904973"},
 }
