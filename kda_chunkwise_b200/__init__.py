@@ -15,6 +15,8 @@ Entry points (same names as the C ABI):
   kda_segment_maps, kda_state_combine,                      context-parallel prefill: a sequence split
   kda_context_parallel_fwd                                  into segments over the ranks of a group
   kda_chunk_bwd                                             gradients of the prefill
+  chunk_kda(...)                                            the prefill as a torch.autograd function: its
+                                                            forward is kda_chunk_fwd, its backward kda_chunk_bwd
 """
 from __future__ import annotations
 
@@ -31,7 +33,7 @@ __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
            "kda_decode_verify", "kda_decode_commit", "kda_short_conv", "kda_output_norm_gate",
            "kda_state_combine", "kda_segment_maps", "context_parallel_states", "kda_context_parallel_fwd",
            "kda_chunk_bwd", "kda_chunk_bwd_workspace_size", "kda_chunk_fwd_host",
-           "kda_chunk_fwd_host_buffer_size",
+           "kda_chunk_fwd_host_buffer_size", "chunk_kda",
            "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
@@ -527,6 +529,39 @@ def kda_chunk_bwd(q, k, v, a, beta, A_log, cu_seqlens, dout, gate=None, initial_
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream, dev))
     _check(st, "kda_chunk_bwd")
     return g
+
+
+class _ChunkKDA(torch.autograd.Function):
+    """kda_chunk_fwd forward, kda_chunk_bwd backward (both through the C ABI); the gradients come
+    back in fp32 and are cast to each input's dtype."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, a, beta, A_log, gate, initial_state, cu_seqlens, scale, out_dtype):
+        out, S = kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=gate, initial_state=initial_state,
+                               scale=scale, out_dtype=out_dtype)
+        ctx.save_for_backward(q, k, v, a, beta, A_log, gate, initial_state, cu_seqlens)
+        ctx.scale = scale
+        return out, S
+
+    @staticmethod
+    def backward(ctx, dout, dS):
+        q, k, v, a, beta, A_log, gate, initial_state, cu_seqlens = ctx.saved_tensors
+        if dout is None:
+            dout = torch.zeros((q.shape[0], q.shape[1], v.shape[-1]), dtype=torch.float32, device=q.device)
+        g = kda_chunk_bwd(q, k, v, a, beta, A_log, cu_seqlens, dout.to(torch.float32).contiguous(), gate=gate,
+                          initial_state=initial_state, dfinal_state=None if dS is None else dS.contiguous(),
+                          scale=ctx.scale)
+        like = lambda x, ref: None if x is None or ref is None else x.to(ref.dtype)
+        return (like(g["dq"], q), like(g["dk"], k), like(g["dv"], v), like(g["da"], a), g["dbeta"], g["dA_log"],
+                like(g["dgate"], gate), g["dinitial_state"], None, None, None)
+
+
+def chunk_kda(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None, scale: float = 1.0,
+              out_dtype=torch.bfloat16):
+    """The prefill (kda_chunk_fwd) as a differentiable function of q, k, v, a, beta, A_log, gate and
+    initial_state.  Returns (out [T, H, d_v], final_state [N, H, d_k, d_v] fp32); a loss on either
+    or both reaches the inputs through kda_chunk_bwd."""
+    return _ChunkKDA.apply(q, k, v, a, beta, A_log, gate, initial_state, cu_seqlens, float(scale), out_dtype)
 
 
 def kda_launch_count() -> int:
