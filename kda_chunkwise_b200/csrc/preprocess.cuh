@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "mma_frag.cuh"
+#include "f32x2.cuh"
 
 namespace kda {
 
@@ -103,17 +104,26 @@ __global__ void __launch_bounds__(kPrepThreads) short_conv_kernel(const ConvPara
         wcur[c] = active ? wc[W - 1] : 0.f;
     }
     const int k0 = kConvMaxWidth - W;   // first window slot with a tap
+    // the same taps as channel pairs (2q, 2q + 1), for the paired fp32 instructions
+    f32x2 wt2[4][kConvMaxWidth - 1], wcur2[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        wcur2[q] = f2_pack(wcur[2 * q], wcur[2 * q + 1]);
+#pragma unroll
+        for (int k = 0; k < kConvMaxWidth - 1; ++k) wt2[q][k] = f2_pack(wt[2 * q][k], wt[2 * q + 1][k]);
+    }
 
     int s = seq_of(p.cu, p.num_seqs, t_begin);
     int64_t s_start = p.cu[s], s_end = p.cu[s + 1];
     // the window before the run: rows t_begin - 3 .. t_begin - 1 of the same sequence, else zero
-    float win[kConvMaxWidth - 1][8];
+    f32x2 win[kConvMaxWidth - 1][4];   // channel pairs
 #pragma unroll
     for (int k = 0; k < kConvMaxWidth - 1; ++k) {
         const int64_t tk = t_begin - (kConvMaxWidth - 1) + k;
+        float w8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (active && k >= k0 && tk >= s_start) load8(xcol + tk * rstride, w8);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) win[k][c] = 0.f;
-        if (active && k >= k0 && tk >= s_start) load8(xcol + tk * rstride, win[k]);
+        for (int q = 0; q < 4; ++q) win[k][q] = f2_pack(w8[2 * q], w8[2 * q + 1]);
     }
 
     const uint16_t *src = xcol + (t_begin + kConvAhead) * rstride;   // the next row to request
@@ -134,25 +144,24 @@ __global__ void __launch_bounds__(kPrepThreads) short_conv_kernel(const ConvPara
 #pragma unroll
             for (int k = 0; k < kConvMaxWidth - 1; ++k)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) win[k][c] = 0.f;
+                for (int q = 0; q < 4; ++q) win[k][q] = 0ull;
         }
-        float xv[8];
+        // the row's 8 channels as pairs (a bf16 pair widens to two fp32 by moving each half up)
+        f32x2 xv[4];
         {
             const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                xv[2 * q] = bf16_to_f32(static_cast<uint16_t>(w4[q] & 0xFFFFu));
-                xv[2 * q + 1] = bf16_to_f32(static_cast<uint16_t>(w4[q] >> 16));
-            }
+            for (int q = 0; q < 4; ++q) xv[q] = f2_pack(__uint_as_float(w4[q] << 16), __uint_as_float(w4[q] & 0xFFFF0000u));
         }
+        // y = w_cur x_t + sum of the window's taps, in the window's order (two channels per instruction)
         float y[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float acc = wcur[c] * xv[c];
+        for (int q = 0; q < 4; ++q) {
+            f32x2 acc = f2_mul(wcur2[q], xv[q]);
 #pragma unroll
             for (int k = 0; k < kConvMaxWidth - 1; ++k)
-                if (k >= k0) acc = fmaf(wt[c][k], win[k][c], acc);
-            y[c] = acc;
+                if (k >= k0) acc = f2_fma(wt2[q][k], win[k][q], acc);
+            f2_unpack(acc, y[2 * q], y[2 * q + 1]);
         }
         if (p.l2norm) {
             float ss = 0.f;
@@ -168,10 +177,10 @@ __global__ void __launch_bounds__(kPrepThreads) short_conv_kernel(const ConvPara
         dst += rstride;
         // slide the window
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            win[0][c] = win[1][c];
-            win[1][c] = win[2][c];
-            win[2][c] = xv[c];
+        for (int q = 0; q < 4; ++q) {
+            win[0][q] = win[1][q];
+            win[1][q] = win[2][q];
+            win[2][q] = xv[q];
         }
     }
     cp_async_wait_all();   // nothing left in flight at exit
