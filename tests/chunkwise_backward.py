@@ -11,8 +11,9 @@ carried between chunks (dS0 = Q^T dO + Diag(Gamma_C) dS_C - W^T dU, dU = A^T dO 
 rest is chunk-local products, the derivative of the inverse (dL = -X^T dX X^T on the strict lower
 triangle, X = (I + L)^-1), and a reverse running sum that takes the gradient of b to that of g.
 Agreement with the token-by-token reverse-mode oracle (oracle/backward.py) to rounding checks the
-algebra a chunkwise backward kernel would follow.  e^b and 1/e^b are formed directly here (fp64,
-moderate decays); a kernel would rescale per 16-token tile as the forward does.
+algebra a chunkwise backward kernel would follow.  The forward here forms e^b and 1/e^b directly
+(fp64, moderate decays); with pairwise=True the key and query gradients are formed as a kernel
+would, every 1/e^b inside a pair e^{b_i - b_j} with i >= j (at most 1, so nothing overflows).
 """
 import numpy as np
 
@@ -21,7 +22,9 @@ def _sig(x):
     return 1.0 / (1.0 + np.exp(-x))
 
 
-def chunkwise_bwd(q, k, v, a, beta, A_log, dout, gate=None, S0=None, dS_T=None, scale=1.0, C=64):
+def chunkwise_bwd(q, k, v, a, beta, A_log, dout, gate=None, S0=None, dS_T=None, scale=1.0, C=64, pairwise=False):
+    """pairwise: form dq, dk and the gradient of b without any 1/e^b on its own, every such factor
+    inside a pair E_ijc = e^{b_ic - b_jc} with i >= j (so E <= 1), as a kernel would."""
     q, k, v, a, dout = (np.asarray(x, np.float64) for x in (q, k, v, a, dout))
     beta = np.asarray(beta, np.float64)
     T, d_k = q.shape
@@ -49,8 +52,8 @@ def chunkwise_bwd(q, k, v, a, beta, A_log, dout, gate=None, S0=None, dS_T=None, 
         W, Ut = Tp @ Kh, Tp @ vc
         U = Ut - W @ S
         O = Qh @ S + A @ U
-        chunks.append(dict(sl=sl, vc=vc, bc=bc, G=G, GC=GC, Qh=Qh, Kh=Kh, Kt=Kt, Kb=Kb, M=M, A=A, X=X, Tp=Tp,
-                           W=W, U=U, S0=S, O=O))
+        chunks.append(dict(sl=sl, vc=vc, bc=bc, b=b, G=G, GC=GC, Qh=Qh, Kh=Kh, Kt=Kt, Kb=Kb, M=M, A=A, X=X,
+                           Tp=Tp, W=W, U=U, S0=S, O=O))
         S = GC[:, None] * S + Kb.T @ U
 
     O_all = np.concatenate([c["O"] for c in chunks]) if chunks else np.zeros((0, d_v))
@@ -91,10 +94,24 @@ def chunkwise_bwd(q, k, v, a, beta, A_log, dout, gate=None, S0=None, dS_T=None, 
         dKh += dMm @ Kt
         dKt += dMm.T @ Kh
         # back to q, k and the running sum b of g
-        dq[sl] = scale * G * dQh
-        db = dQh * Qh + dKh * Kh - dKt * Kt - dKb * Kb
-        dk[sl] = G * dKh + dKt / G + (GC / G) * dKb
-        db[-1] += (dKb * Kb).sum(axis=0) + dGC * GC
+        if not pairwise:
+            dq[sl] = scale * G * dQh
+            db = dQh * Qh + dKh * Kh - dKt * Kt - dKb * Kb
+            dk[sl] = G * dKh + dKt / G + (GC / G) * dKb
+            db[-1] += (dKb * Kb).sum(axis=0) + dGC * GC
+        else:
+            kc, sq, b = k[sl], scale * q[sl], c["b"]
+            n = len(b)
+            incl = np.tril(np.ones((n, n), dtype=bool))
+            E = np.where(incl[:, :, None], np.exp(np.where(incl[:, :, None], b[:, None, :] - b[None, :, :], 0.0)), 0.0)
+            dAl, dMl = np.tril(dA), np.tril(dMm, -1)
+            dq[sl] = scale * (G * (dO @ S0c.T) + np.einsum("ij,jc,ijc->ic", dAl, kc, E))
+            P = G * (Tp.T @ dW) + np.einsum("ij,jc,ijc->ic", dMl, kc, E)
+            Qs = np.einsum("ij,ic,ijc->jc", dAl, sq, E) + np.einsum("ij,ic,ijc->jc", dMl, kc, E)
+            R = (GC / G) * dKb
+            dk[sl] = P + Qs + R
+            db = dq[sl] * q[sl] + (P - Qs - R) * kc
+            db[-1] += (R * kc).sum(axis=0) + dGC * GC
         dg[sl] = np.cumsum(db[::-1], axis=0)[::-1]
         dS = dS0
     sx = _sig(x)

@@ -35,3 +35,16 @@ def test_chunkwise_gradients_match_the_token_level_oracle(seed, T, C, gate, S0):
         err = np.abs(got[key] - ref[key]).max() / max(np.abs(ref[key]).max(), 1e-30)
         assert err <= 1e-9, f"{key}: relative max error {err:.2e}"
     assert abs(got["dA_log"] - ref["dA_log"]) <= 1e-9 * max(abs(ref["dA_log"]), 1.0)
+
+
+@pytest.mark.parametrize("seed,T,C", [(4, 150, 64), (5, 40, 16)])
+def test_overflow_free_pairwise_form_gives_the_same_gradients(seed, T, C):
+    # the form a kernel would use (no 1/e^b outside a pair e^{b_i - b_j}, i >= j) against the direct one
+    x = _unit(seed, T)
+    args = (x["q"], x["k"], x["v"], x["a"], x["beta"], x["A_log"], x["dout"])
+    kw = dict(gate=x["gate"], S0=x["S0"], dS_T=x["dS_T"], scale=0.7, C=C)
+    direct = chunkwise_bwd(*args, **kw)
+    pair = chunkwise_bwd(*args, pairwise=True, **kw)
+    for key in ("dq", "dk", "da", "dbeta", "dS0"):
+        err = np.abs(pair[key] - direct[key]).max() / max(np.abs(direct[key]).max(), 1e-30)
+        assert err <= 1e-10, f"{key}: relative max error {err:.2e}"
