@@ -278,6 +278,28 @@ KDA_API kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, co
                                  float *dbeta, float *dgate, float *dA_log, float *dinitial_state,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * kda_chunk_bwd_chunkwise — the same gradients as kda_chunk_bwd (same arguments and layouts), in
+ * chunkwise form: per 64-token chunk the forward operands, the states at the chunk starts (a pass
+ * over chunks), the state gradients at the chunk ends (a reverse pass over chunks) and the rest of
+ * the gradients chunk by chunk, all in fp32; T / 64 sequential steps per unit instead of 3 T.
+ * Workspace: kda_chunk_bwd_chunkwise_workspace_size(...) bytes, 16-byte aligned.
+ */
+KDA_API kda_status kda_chunk_bwd_chunkwise(const void *q, const void *k, const void *v, const void *a,
+                                           const float *beta, const void *gate, const float *A_log,
+                                           const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                           int32_t H, int32_t d_k, int32_t d_v, float scale,
+                                           const float *initial_state, const float *dout,
+                                           const float *dfinal_state, float *dq, float *dk, float *dv,
+                                           float *da, float *dbeta, float *dgate, float *dA_log,
+                                           float *dinitial_state, void *workspace, size_t workspace_bytes,
+                                           void *stream);
+
+/* Workspace of kda_chunk_bwd_chunkwise (host-only; 0 on invalid sizes): one record of the chunk's
+ * operands, states and state gradients per (64-token chunk, head). */
+KDA_API size_t kda_chunk_bwd_chunkwise_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H,
+                                                      int32_t d_k, int32_t d_v);
+
 /* Workspace kda_chunk_bwd needs (host-only; 0 on invalid sizes):
  * ((total_tokens / 32 + num_seqs) * H + num_seqs * H * 32) * d_k * d_v * 4 bytes. */
 KDA_API size_t kda_chunk_bwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k,

@@ -94,6 +94,10 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_bwd.restype = ctypes.c_int
     L.kda_chunk_bwd_workspace_size.argtypes = [i64, i32, i32, i32, i32]
     L.kda_chunk_bwd_workspace_size.restype = sz
+    L.kda_chunk_bwd_chunkwise.argtypes = L.kda_chunk_bwd.argtypes
+    L.kda_chunk_bwd_chunkwise.restype = ctypes.c_int
+    L.kda_chunk_bwd_chunkwise_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+    L.kda_chunk_bwd_chunkwise_workspace_size.restype = sz
     L.kda_chunk_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, f32, vp, vp, vp,
                                      ctypes.c_int, i64, vp, sz, vp]
     L.kda_chunk_fwd_host.restype = ctypes.c_int
@@ -489,8 +493,12 @@ def kda_chunk_bwd_workspace_size(total_tokens, num_seqs, H, d_k, d_v) -> int:
     return int(lib.kda_chunk_bwd_workspace_size(total_tokens, num_seqs, H, d_k, d_v))
 
 
+def kda_chunk_bwd_chunkwise_workspace_size(total_tokens, num_seqs, H, d_k, d_v) -> int:
+    return int(lib.kda_chunk_bwd_chunkwise_workspace_size(total_tokens, num_seqs, H, d_k, d_v))
+
+
 def kda_chunk_bwd(q, k, v, a, beta, A_log, cu_seqlens, dout, gate=None, initial_state=None,
-                  dfinal_state=None, scale: float = 1.0, workspace=None, stream=None):
+                  dfinal_state=None, scale: float = 1.0, workspace=None, stream=None, chunkwise: bool = False):
     """Gradients of kda_chunk_fwd's outputs (and final states) with respect to its inputs.
 
     dout fp32 [T, H, d_v]; dfinal_state fp32 [N, H, d_k, d_v] or None.  Returns a dict of fp32
@@ -519,15 +527,16 @@ def kda_chunk_bwd(q, k, v, a, beta, A_log, cu_seqlens, dout, gate=None, initial_
              dbeta=torch.empty((T, H), dtype=f32, device=dev), dA_log=torch.empty((H,), dtype=f32, device=dev),
              dgate=None if gate is None else torch.empty((T, H, d_v), dtype=f32, device=dev),
              dinitial_state=None if initial_state is None else torch.empty((N, H, d_k, d_v), dtype=f32, device=dev))
-    need = kda_chunk_bwd_workspace_size(T, N, H, d_k, d_v)
+    need = (kda_chunk_bwd_chunkwise_workspace_size if chunkwise else kda_chunk_bwd_workspace_size)(T, N, H, d_k, d_v)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    st = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate), _ptr(A_log),
+    fn = lib.kda_chunk_bwd_chunkwise if chunkwise else lib.kda_chunk_bwd
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(gate), _ptr(A_log),
                            _ptr(cu_seqlens), N, T, H, d_k, d_v, float(scale), _ptr(initial_state), _ptr(dout),
                            _ptr(dfinal_state), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["da"]),
                            _ptr(g["dbeta"]), _ptr(g["dgate"]), _ptr(g["dA_log"]), _ptr(g["dinitial_state"]),
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(stream, dev))
-    _check(st, "kda_chunk_bwd")
+    _check(st, "kda_chunk_bwd_chunkwise" if chunkwise else "kda_chunk_bwd")
     return g
 
 

@@ -18,6 +18,7 @@
 #include "preprocess.cuh"
 #include "state_map.cuh"
 #include "backward.cuh"
+#include "backward_chunk.cuh"
 
 namespace {
 
@@ -874,4 +875,105 @@ kda_status kda_chunk_fwd_host(const void *q, const void *k, const void *v, const
 #undef KDA_HOST_TRY
     cleanup();
     return KDA_OK;
+}
+
+// ---- the backward in chunkwise form ------------------------------------------------------------
+
+namespace {
+
+template <int DK, int DV>
+kda_status launch_bwd_chunkwise(const kda::BwdParams &p, int64_t units, int64_t records, cudaStream_t st) {
+    using SM = kda::BcSmem<DK, DV>;
+    constexpr int G = DV / kda::kBcCols;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kda::bc_prep_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kPrep)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(kda::bc_state_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kState)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(kda::bc_dstate_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kDState)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(kda::bc_grad_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kGrad)) != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute(chunk_bwd_chunkwise)");
+    kda::bc_prep_kernel<DK, DV><<<(unsigned)records, kda::kBcThreads, SM::kPrep, st>>>(p);
+    kda::bc_state_kernel<DK, DV><<<(unsigned)(units * G), kda::kBcThreads, SM::kState, st>>>(p);
+    kda::bc_dstate_kernel<DK, DV><<<(unsigned)(units * G), kda::kBcThreads, SM::kDState, st>>>(p);
+    kda::bc_grad_kernel<DK, DV><<<(unsigned)records, kda::kBcThreads, SM::kGrad, st>>>(p);
+    g_launches.fetch_add(4, std::memory_order_relaxed);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "chunk_bwd_chunkwise launch");
+}
+
+size_t bc_record_floats(int d_k, int d_v) {
+    if (d_k == 128 && d_v == 128) return kda::BcRec<128, 128>::kSize;
+    if (d_k == 128 && d_v == 64) return kda::BcRec<128, 64>::kSize;
+    if (d_k == 64 && d_v == 128) return kda::BcRec<64, 128>::kSize;
+    return kda::BcRec<64, 64>::kSize;
+}
+
+}  // namespace
+
+size_t kda_chunk_bwd_chunkwise_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k,
+                                              int32_t d_v) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || !supported_dim(d_k) || !supported_dim(d_v)) return 0;
+    const size_t records = (size_t)(total_tokens / kda::kBcChunk + num_seqs) * H;   // >= sum ceil(len / 64) H
+    return records * bc_record_floats(d_k, d_v) * 4;
+}
+
+kda_status kda_chunk_bwd_chunkwise(const void *q, const void *k, const void *v, const void *a, const float *beta,
+                                   const void *gate, const float *A_log, const int32_t *cu_seqlens, int32_t num_seqs,
+                                   int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                                   const float *initial_state, const float *dout, const float *dfinal_state,
+                                   float *dq, float *dk, float *dv, float *da, float *dbeta, float *dgate,
+                                   float *dA_log, float *dinitial_state, void *workspace, size_t workspace_bytes,
+                                   void *stream) {
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: negative size or H <= 0");
+    if (!supported_dim(d_k) || !supported_dim(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_bwd_chunkwise: d_k and d_v must be 64 or 128");
+    if (num_seqs == 0) {
+        if (total_tokens != 0) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: tokens without sequences");
+        return KDA_OK;
+    }
+    if (!cu_seqlens || !A_log || !dA_log) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: NULL cu_seqlens, A_log or dA_log");
+    if (total_tokens > 0 && (!q || !k || !v || !a || !beta || !dout || !dq || !dk || !dv || !da || !dbeta))
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: NULL input or gradient pointer");
+    if (gate && !dgate) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: gate given without dgate");
+    const void *ptrs[] = {q, k, v, a, gate, initial_state, dout, dfinal_state, dq, dk, dv, da, dgate,
+                          dinitial_state, workspace};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned(ptr, 16)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: tensor pointer not 16-byte aligned");
+    const void *ptrs4[] = {beta, A_log, cu_seqlens, dbeta, dA_log};
+    for (const void *ptr : ptrs4)
+        if (ptr && !aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: scalar array not 4-byte aligned");
+    const size_t need = kda_chunk_bwd_chunkwise_workspace_size(total_tokens, num_seqs, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: workspace missing or too small (need " + std::to_string(need) + " bytes)");
+    const int64_t units = (int64_t)num_seqs * H;
+    const int64_t records = (total_tokens / kda::kBcChunk + num_seqs) * (int64_t)H;
+    if (records > 0x7fffffffLL || units * (d_v / kda::kBcCols) > 0x7fffffffLL)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: too many chunks or units");
+    kda::BwdParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.a = static_cast<const uint16_t *>(a);
+    p.gate = static_cast<const uint16_t *>(gate);
+    p.beta = beta;
+    p.A_log = A_log;
+    p.cu = cu_seqlens;
+    p.S0 = initial_state;
+    p.dout = dout;
+    p.dS_T = dfinal_state;
+    p.dq = dq; p.dk = dk; p.dv = dv; p.da = da; p.dbeta = dbeta; p.dgate = dgate;
+    p.dA_log = dA_log;
+    p.dS0 = dinitial_state;
+    p.ckpt = static_cast<float *>(workspace);
+    p.scratch = nullptr;
+    p.total_tokens = total_tokens;
+    p.num_seqs = num_seqs;
+    p.H = H;
+    p.scale = scale;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(dA_log, 0, sizeof(float) * H, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dA_log)");
+    if (d_k == 128 && d_v == 128) return launch_bwd_chunkwise<128, 128>(p, units, records, st);
+    if (d_k == 128 && d_v == 64) return launch_bwd_chunkwise<128, 64>(p, units, records, st);
+    if (d_k == 64 && d_v == 128) return launch_bwd_chunkwise<64, 128>(p, units, records, st);
+    return launch_bwd_chunkwise<64, 64>(p, units, records, st);
 }

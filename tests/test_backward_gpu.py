@@ -57,9 +57,10 @@ def _check(kda, inp, dout, dST, g, units, scale=1.0):
     return dA_ref
 
 
+@pytest.mark.parametrize("chunkwise", [False, True])
 @pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
 @pytest.mark.parametrize("with_gate,with_state", [(True, True), (False, False)])
-def test_backward_matches_oracle(kda, dk, dv, with_gate, with_state):
+def test_backward_matches_oracle(kda, dk, dv, with_gate, with_state, chunkwise):
     w = KI.Workload("bwd", (70, 1, 130, 0, 64), 2, dk, dv, A_log="uniform", gate=with_gate,
                     init_state="normal_0.02" if with_state else "none", seed=31)
     inp = KI.make_inputs(w, "cuda")
@@ -68,7 +69,7 @@ def test_backward_matches_oracle(kda, dk, dv, with_gate, with_state):
     dST = torch.randn((w.num_seqs, w.H, dk, dv), generator=g_, device="cuda") if with_state else None
     g = kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
                           dout, gate=inp["gate"], initial_state=inp["initial_state"], dfinal_state=dST,
-                          scale=0.9)
+                          scale=0.9, chunkwise=chunkwise)
     kda.kda_sync_check()
     units = [(n, h) for n in range(w.num_seqs) for h in range(w.H)]
     dA_ref = _check(kda, inp, dout, dST, g, units, scale=0.9)
@@ -76,7 +77,8 @@ def test_backward_matches_oracle(kda, dk, dv, with_gate, with_state):
         assert abs(float(g["dA_log"][h]) - ref) <= 5e-3 * max(abs(ref), 1e-6), f"dA_log[{h}]"
 
 
-def test_backward_full_size_sampled(kda):
+@pytest.mark.parametrize("chunkwise", [False, True])
+def test_backward_full_size_sampled(kda, chunkwise):
     # the prefill workload (B=1, H=32, T=8192, d=128), three heads checked over all 8192 tokens
     w = KI.WORKLOADS["prefill_B1_H32_T8192_d128"]
     inp = KI.make_inputs(w, "cuda")
@@ -84,7 +86,8 @@ def test_backward_full_size_sampled(kda):
     dout = torch.randn((w.total_tokens, w.H, w.d_v), generator=g_, device="cuda") * 0.1
     dST = torch.randn((w.num_seqs, w.H, w.d_k, w.d_v), generator=g_, device="cuda") * 0.1
     g = kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
-                          dout, gate=inp["gate"], initial_state=inp["initial_state"], dfinal_state=dST)
+                          dout, gate=inp["gate"], initial_state=inp["initial_state"], dfinal_state=dST,
+                          chunkwise=chunkwise)
     kda.kda_sync_check()
     dA_ref = _check(kda, inp, dout, dST, g, [(0, 0), (0, 13), (0, 31)])
     for h, ref in dA_ref.items():
