@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kBcThreads) bc_prep_kernel(const BwdParams p) 
         float m = 0.f, a = 0.f;
         if (j <= i) {
             for (int ch = 0; ch < DK; ++ch) {
-                const float E = expf(sb[i * LK + ch] - sb[j * LK + ch]);
+                const float E = __expf(sb[i * LK + ch] - sb[j * LK + ch]);
                 const float kj = sk[j * LK + ch] * E;
                 a = fmaf(sq[i * LK + ch], kj, a);
                 m = fmaf(sk[i * LK + ch], kj, m);
@@ -226,10 +226,13 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(kBcThreads) bc_state_kernel(const BwdParams p) {
     constexpr int C = kBcChunk, NT = kBcThreads, DC = kBcCols, G = DV / DC;
     using R = BcRec<DK, DV>;
+    constexpr int LK = DK + 1;
     extern __shared__ __align__(16) float bcs[];
     float *sS = bcs;                 // [DK][DC]
     float *sU = sS + DK * DC;        // [C][DC]
     float *sT = sU + C * DC;         // [DK][DC]
+    float *sW = sT + DK * DC;        // [C][LK] W of the chunk
+    float *sKb = sW + C * LK;        // [C][LK] K- of the chunk
     const int64_t unit = blockIdx.x / G;
     const int slice = static_cast<int>(blockIdx.x % G);
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
@@ -253,14 +256,19 @@ __global__ void __launch_bounds__(kBcThreads) bc_state_kernel(const BwdParams p)
             const int i = e / DC, cc = e % DC;
             sU[e] = rec[R::kU + (size_t)i * DV + col0 + cc];
         }
+        for (int e = tid; e < C * DK; e += NT) {
+            const int i = e / DK, ch = e % DK;
+            sW[i * LK + ch] = rec[R::kW + e];
+            sKb[i * LK + ch] = rec[R::kKb + e];
+        }
         __syncthreads();
-        bc_gemm<C, DC, DK, false, false>(rec + R::kW, DK, sS, DC, sU, DC, -1.f, true);   // U = T'V - W S0
+        bc_gemm<C, DC, DK, false, false>(sW, LK, sS, DC, sU, DC, -1.f, true);   // U = T'V - W S0
         __syncthreads();
         for (int e = tid; e < C * DC; e += NT) {
             const int i = e / DC, cc = e % DC;
             rec[R::kU + (size_t)i * DV + col0 + cc] = sU[e];
         }
-        bc_gemm<DK, DC, C, true, false>(rec + R::kKb, DK, sU, DC, sT, DC, 1.f, false);   // K-^T U
+        bc_gemm<DK, DC, C, true, false>(sKb, LK, sU, DC, sT, DC, 1.f, false);   // K-^T U
         __syncthreads();
         for (int e = tid; e < DK * DC; e += NT) sS[e] = fmaf(rec[R::kGC + e / DC], sS[e], sT[e]);
         __syncthreads();
@@ -272,11 +280,16 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p) {
     constexpr int C = kBcChunk, NT = kBcThreads, DC = kBcCols, G = DV / DC;
     using R = BcRec<DK, DV>;
+    constexpr int LK = DK + 1, LC = C + 1;
     extern __shared__ __align__(16) float bcs[];
     float *sdS = bcs;                // [DK][DC]
     float *sO = sdS + DK * DC;       // [C][DC] O, then dO
     float *sdU = sO + C * DC;        // [C][DC]
     float *sT = sdU + C * DC;        // [DK][DC]
+    float *sQh = sT + DK * DC;       // [C][LK] the chunk's Q^, K-, W and A
+    float *sKb = sQh + C * LK;
+    float *sW = sKb + C * LK;
+    float *sA = sW + C * LK;         // [C][LC]
     const int64_t unit = blockIdx.x / G;
     const int slice = static_cast<int>(blockIdx.x % G);
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
@@ -295,10 +308,18 @@ __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p
         float *rec = p.ckpt + (size_t)((base + c) * H + h) * R::kSize;
         const int64_t t0 = s0 + (int64_t)c * C;
         const int L = static_cast<int>(min64(C, s1 - t0));
-        // O = Q^ S0 + A U (pre-gate outputs of this chunk's columns)
-        bc_gemm<C, DC, DK, false, false>(rec + R::kQh, DK, rec + R::kS0 + col0, DV, sO, DC, 1.f, false);
+        for (int e = tid; e < C * DK; e += NT) {
+            const int i = e / DK, ch = e % DK;
+            sQh[i * LK + ch] = rec[R::kQh + e];
+            sKb[i * LK + ch] = rec[R::kKb + e];
+            sW[i * LK + ch] = rec[R::kW + e];
+        }
+        for (int e = tid; e < C * C; e += NT) sA[(e / C) * LC + e % C] = rec[R::kA + e];
         __syncthreads();
-        bc_gemm<C, DC, C, false, false>(rec + R::kA, C, rec + R::kU + col0, DV, sO, DC, 1.f, true);
+        // O = Q^ S0 + A U (pre-gate outputs of this chunk's columns)
+        bc_gemm<C, DC, DK, false, false>(sQh, LK, rec + R::kS0 + col0, DV, sO, DC, 1.f, false);
+        __syncthreads();
+        bc_gemm<C, DC, C, false, false>(sA, LC, rec + R::kU + col0, DV, sO, DC, 1.f, true);
         __syncthreads();
         for (int e = tid; e < C * DC; e += NT) {   // dO = dout sigmoid(gate); dgate = dout O sigmoid'
             const int i = e / DC, cc = e % DC;
@@ -321,18 +342,18 @@ __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p
         }
         __syncthreads();
         // dU = A^T dO + K- dS_C
-        bc_gemm<C, DC, C, true, false>(rec + R::kA, C, sO, DC, sdU, DC, 1.f, false);
+        bc_gemm<C, DC, C, true, false>(sA, LC, sO, DC, sdU, DC, 1.f, false);
         __syncthreads();
-        bc_gemm<C, DC, DK, false, false>(rec + R::kKb, DK, sdS, DC, sdU, DC, 1.f, true);
+        bc_gemm<C, DC, DK, false, false>(sKb, LK, sdS, DC, sdU, DC, 1.f, true);
         __syncthreads();
         for (int e = tid; e < C * DC; e += NT) {
             const int i = e / DC, cc = e % DC;
             rec[R::kdU + (size_t)i * DV + col0 + cc] = sdU[e];
         }
         // dS0 = Q^T dO + Diag(Gamma_C) dS_C - W^T dU
-        bc_gemm<DK, DC, C, true, false>(rec + R::kQh, DK, sO, DC, sT, DC, 1.f, false);
+        bc_gemm<DK, DC, C, true, false>(sQh, LK, sO, DC, sT, DC, 1.f, false);
         __syncthreads();
-        bc_gemm<DK, DC, C, true, false>(rec + R::kW, DK, sdU, DC, sT, DC, -1.f, true);
+        bc_gemm<DK, DC, C, true, false>(sW, LK, sdU, DC, sT, DC, -1.f, true);
         __syncthreads();
         for (int e = tid; e < DK * DC; e += NT) sdS[e] = fmaf(rec[R::kGC + e / DC], sdS[e], sT[e]);
         __syncthreads();
@@ -457,17 +478,16 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
     }
     for (int i = tid; i < L; i += NT) p.dbeta[(t0 + i) * H + h] = sdb[i];
     __syncthreads();
-    // the pairwise sums, one key channel per thread (rows of each [C][DK] slot are strided by DK)
-    float dA_acc = 0.f;
-    for (int ch = tid; ch < DK; ch += NT) {
-        const float bC = sb[(C - 1) * LK + ch];
-        float lastR = 0.f;
-        for (int i = 0; i < C; ++i) {   // dq (over Q^'s slot) and P (over S0's slot)
+    // the pairwise sums: NT / DK threads per key channel, each taking every (NT / DK)-th row
+    constexpr int TPC = NT / DK;
+    {
+        const int ch = tid % DK, part = tid / DK;
+        for (int i = part; i < C; i += TPC) {   // dq (over Q^'s slot) and P (over S0's slot)
             const float bi = sb[i * LK + ch];
             float aq = expf(bi) * rec[R::kQh + (size_t)i * DK + ch];
             float ap = expf(bi) * rec[R::kS0 + (size_t)i * DK + ch];
             for (int j = 0; j <= i; ++j) {
-                const float E = expf(bi - sb[j * LK + ch]);
+                const float E = __expf(bi - sb[j * LK + ch]);
                 const float kE = sk[j * LK + ch] * E;
                 aq = fmaf(sdA[i * LC + j], kE, aq);
                 ap = fmaf(sM[i * LC + j], kE, ap);   // dM_ii = 0
@@ -475,15 +495,21 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
             rec[R::kQh + (size_t)i * DK + ch] = p.scale * aq;
             rec[R::kS0 + (size_t)i * DK + ch] = ap;
         }
-        for (int j = 0; j < C; ++j) {   // Q (over W's slot)
+        for (int j = part; j < C; j += TPC) {   // Q (over W's slot)
             const float bj = sb[j * LK + ch];
             float aQ = 0.f;
             for (int i = j; i < C; ++i) {
-                const float E = expf(sb[i * LK + ch] - bj);
+                const float E = __expf(sb[i * LK + ch] - bj);
                 aQ = fmaf(sdA[i * LC + j] * sq[i * LK + ch] + sM[i * LC + j] * sk[i * LK + ch], E, aQ);
             }
             rec[R::kW + (size_t)j * DK + ch] = aQ;
         }
+    }
+    __syncthreads();   // every row of dq, P and Q is in place
+    float dA_acc = 0.f;
+    for (int ch = tid; ch < DK; ch += NT) {
+        const float bC = sb[(C - 1) * LK + ch];
+        float lastR = 0.f;
         // dk = P + Q + R, db = dq q + (P - Q - R) k over K-'s slot (dK-), the last row's extra terms
         for (int r = 0; r < C; ++r) {
             const size_t o = (size_t)r * DK + ch;
@@ -528,8 +554,8 @@ template <int DK, int DV>
 struct BcSmem {
     static constexpr int C = kBcChunk, LK = DK + 1, LV = DV + 1, LC = C + 1;
     static constexpr int kPrep = (3 * C * LK + C * LV + 2 * C * LC + C) * 4;
-    static constexpr int kState = (2 * DK * kBcCols + C * kBcCols) * 4;
-    static constexpr int kDState = (2 * DK * kBcCols + 2 * C * kBcCols) * 4;
+    static constexpr int kState = (2 * DK * kBcCols + C * kBcCols + 2 * C * LK) * 4;
+    static constexpr int kDState = (2 * DK * kBcCols + 2 * C * kBcCols + 3 * C * LK + C * LC) * 4;
     static constexpr int kGrad = (4 * C * LK + 4 * C * LC + 2 * C + DK + kBcThreads / 32) * 4;
 };
 
