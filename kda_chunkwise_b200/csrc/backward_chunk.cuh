@@ -410,10 +410,12 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
         sM[i * LC + j] = rec[R::kM + e];
     }
     for (int i = tid; i < C; i += NT) sbeta[i] = i < L ? p.beta[(t0 + i) * H + h] : 0.f;
-    for (int ch = tid; ch < DK; ch += NT) {   // dGamma_C = rowsum(dS_C (.) S0)
+    for (int ch = tid >> 5; ch < DK; ch += NT / 32) {   // dGamma_C = rowsum(dS_C (.) S0), a warp per row
         float s = 0.f;
-        for (int v = 0; v < DV; ++v) s = fmaf(rec[R::kdS + (size_t)ch * DV + v], rec[R::kS0 + (size_t)ch * DV + v], s);
-        sdGC[ch] = s;
+        for (int v = tid & 31; v < DV; v += 32)
+            s = fmaf(rec[R::kdS + (size_t)ch * DV + v], rec[R::kS0 + (size_t)ch * DV + v], s);
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if ((tid & 31) == 0) sdGC[ch] = s;
     }
     __syncthreads();
     for (int e = tid; e < C * C; e += NT) {   // T' = X diag(beta)
