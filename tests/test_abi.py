@@ -148,8 +148,9 @@ def test_short_conv_and_norm_gate_reject_bad_arguments():
     assert NG(16, None, 16, 0, 2, 128, 1e-6, 32, 0, None) == kda.KDA_OK
 
 
-def test_chunk_bwd_rejects_bad_arguments():
-    B = lib.kda_chunk_bwd
+@pytest.mark.parametrize("entry", ["kda_chunk_bwd", "kda_chunk_bwd_chunkwise"])
+def test_chunk_bwd_rejects_bad_arguments(entry):
+    B = getattr(lib, entry)
     ok = dict(q=16, k=16, v=16, a=16, beta=16, gate=None, A_log=16, cu=16, N=1, T=64, H=2, dk=128, dv=128,
               S0=None, dout=16, dST=None, dq=16, dkk=16, dvv=16, da=16, db=16, dg=None, dA=16, dS0=None,
               ws=256, wsb=1 << 30)
@@ -167,6 +168,10 @@ def test_chunk_bwd_rejects_bad_arguments():
     assert bwd(q=8) == kda.KDA_ERR_INVALID_ARG                    # misaligned
     assert bwd(N=0, T=0) == kda.KDA_OK
     assert kda.kda_chunk_bwd_workspace_size(8192, 1, 32, 128, 128) == (8192 // 32 + 1 + 32) * 32 * 128 * 128 * 4
+    # one record per (64-token chunk, head): b, W, K-, Q^ [64][d_k]; T'V then U, dU, dO [64][d_v];
+    # A, X, M [64][64]; Gamma_C [d_k]; the incoming state and its gradient [d_k][d_v]
+    rec = 4 * 64 * 128 + 3 * 64 * 128 + 3 * 64 * 64 + 128 + 2 * 128 * 128
+    assert kda.kda_chunk_bwd_chunkwise_workspace_size(8192, 1, 32, 128, 128) == (8192 // 64 + 1) * 32 * rec * 4
 
 
 def test_host_prefill_validates_on_the_host():
