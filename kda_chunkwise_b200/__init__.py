@@ -14,7 +14,8 @@ Entry points (same names as the C ABI):
                                                             pre-gate normalisation + output gate
   kda_segment_maps, kda_state_combine,                      context-parallel prefill: a sequence split
   kda_context_parallel_fwd                                  into segments over the ranks of a group
-  kda_chunk_bwd                                             gradients of the prefill
+  kda_chunk_bwd                                             gradients of the prefill (chunkwise=True: the
+                                                            chunkwise form, kda_chunk_bwd_chunkwise)
   chunk_kda(...)                                            the prefill as a torch.autograd function: its
                                                             forward is kda_chunk_fwd, its backward kda_chunk_bwd
 """
@@ -504,6 +505,8 @@ def kda_chunk_bwd(q, k, v, a, beta, A_log, cu_seqlens, dout, gate=None, initial_
     dout fp32 [T, H, d_v]; dfinal_state fp32 [N, H, d_k, d_v] or None.  Returns a dict of fp32
     tensors: dq, dk, da [T, H, d_k]; dv, dgate [T, H, d_v] (dgate None without a gate); dbeta
     [T, H]; dA_log [H]; dinitial_state [N, H, d_k, d_v] (None without an initial state).
+    chunkwise: run kda_chunk_bwd_chunkwise (the chunkwise form) instead of the token-level kernel;
+    the gradients agree to rounding.
     """
     dev = q.device
     T, H, d_k = q.shape
