@@ -323,6 +323,26 @@ KDA_API const char *kda_last_error(void);
 KDA_API uint64_t kda_launch_count(void);
 
 /*
+ * kda_set_prefill_path — choose which of the two prefill kernels kda_chunk_fwd (and
+ * kda_chunk_fwd_noalloc, kda_chunk_fwd_host) run for d_k = d_v = 128.  (No counterpart in the pages:
+ * both kernels compute the same chunkwise form of "Kimi K3 · Lesson 3 of 14"; they differ only in how
+ * the work is spread over the GPU.)
+ *   path 0: chosen from the shapes (the default): one CTA per (sequence, head) unit when the units
+ *           are at least a third of the SM count, else the cluster kernel;
+ *   path 1: the cluster kernel (a unit's chunks spread over d_v/32 CTAs, chunk records in the
+ *           caller's workspace);
+ *   path 2: one CTA per unit, every intermediate on chip (no workspace).
+ * Other d_k, d_v always use the cluster kernel.  Process-wide; not synchronised with launches in
+ * flight on other threads.  Returns KDA_ERR_INVALID_ARG for any other value.  The workspace size
+ * (kda_chunk_fwd_workspace_size) follows the path in force when it is queried: 0 for path 2.
+ */
+KDA_API kda_status kda_set_prefill_path(int32_t path);
+
+/* kda_prefill_path — the kernel kda_chunk_fwd would run for num_units (sequence, head) units of
+ * this shape under the current setting: 1 (cluster kernel) or 2 (one CTA per unit). */
+KDA_API int32_t kda_prefill_path(int64_t num_units, int32_t d_k, int32_t d_v);
+
+/*
  * kda_inject_stall — failure injection for tests of the bounded waits.  (No counterpart in the
  * pages: the method has no inter-CTA waits; this exercises the library's own failure handling.)
  *

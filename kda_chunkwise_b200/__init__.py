@@ -106,6 +106,10 @@ def _load() -> ctypes.CDLL:
     L.kda_chunk_fwd_host_buffer_size.restype = sz
     L.kda_inject_stall.argtypes = [i32, ctypes.c_uint64]
     L.kda_inject_stall.restype = ctypes.c_int
+    L.kda_set_prefill_path.argtypes = [i32]
+    L.kda_set_prefill_path.restype = ctypes.c_int
+    L.kda_prefill_path.argtypes = [i64, i32, i32]
+    L.kda_prefill_path.restype = i32
     return L
 
 
@@ -579,6 +583,17 @@ def chunk_kda(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None
 def kda_launch_count() -> int:
     """Kernels launched through libkda by this process so far."""
     return int(lib.kda_launch_count())
+
+
+def kda_set_prefill_path(path: int) -> None:
+    """Which prefill kernel kda_chunk_fwd runs for d_k = d_v = 128: 0 chosen from the shapes,
+    1 the cluster kernel (chunk records in the workspace), 2 one CTA per (sequence, head)."""
+    _check(lib.kda_set_prefill_path(int(path)), "kda_set_prefill_path")
+
+
+def kda_prefill_path(num_units: int, d_k: int, d_v: int) -> int:
+    """The kernel kda_chunk_fwd would run now for num_units units: 1 (cluster) or 2 (per unit)."""
+    return int(lib.kda_prefill_path(int(num_units), int(d_k), int(d_v)))
 
 
 def kda_inject_stall(enable: bool, wait_limit_ns: int = 0) -> None:

@@ -69,6 +69,7 @@ struct BwdParams {
     const float *dout;                      // [T, H, d_v] fp32
     const float *dS_T;                      // [N, H, d_k, d_v] or null
     float *dq, *dk, *dv, *da, *dbeta, *dgate, *dA_log, *dS0;
+    int64_t ck_records;                     // chunk records per head the workspace holds
     float *ckpt;                            // [sum_n ceil(len_n / 32)][H][d_v / 32][d_k x 32 slice]
     float *scratch;                         // [N H][d_v / 32][32 tokens][d_k x 32 slice]
     int64_t total_tokens;
@@ -172,13 +173,16 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(const BwdParams p)
         if (tid == 0 && rank == 0) atomicOr(&g_kda_error_word, kErrBadSeqlens);
     }
     const int64_t len = s1 - s0;
-    const int nck = static_cast<int>((len + C - 1) / C);
     int64_t ckbase = 0;   // checkpoints of the sequences before this one
     for (int m = 0; m < n; ++m) {
         int64_t a0, a1;
         seq_span(p.cu, m, p.num_seqs, p.total_tokens, a0, a1);
         ckbase += (a1 - a0 + C - 1) / C;
     }
+    // Well-formed cu_seqlens never need more checkpoints than the workspace holds; malformed ones
+    // (flagged above) are cut short so that no checkpoint lands past it.
+    const int64_t ck_room = p.ck_records - ckbase > 0 ? p.ck_records - ckbase : 0;
+    const int nck = static_cast<int>(min64((len + C - 1) / C, ck_room));
     const int64_t H = p.H;
     const float expA = expf(p.A_log[h]);
     const size_t SZ = (size_t)DK * DV, SL = (size_t)DK * DC;

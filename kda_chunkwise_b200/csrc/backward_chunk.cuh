@@ -237,9 +237,12 @@ __global__ void __launch_bounds__(kBcThreads) bc_state_kernel(const BwdParams p)
     const int slice = static_cast<int>(blockIdx.x % G);
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
     int64_t s0, s1;
-    seq_span(p.cu, n, p.num_seqs, p.total_tokens, s0, s1);
-    const int nck = static_cast<int>((s1 - s0 + C - 1) / C);
+    if (!seq_span(p.cu, n, p.num_seqs, p.total_tokens, s0, s1) && threadIdx.x == 0 && slice == 0)
+        atomicOr(&g_kda_error_word, kErrBadSeqlens);
     const int64_t base = bc_chunk_base(p, n);
+    // malformed cu_seqlens (flagged above) are cut short: no record past the workspace's
+    const int64_t room = p.ck_records - base > 0 ? p.ck_records - base : 0;
+    const int nck = static_cast<int>(min64((s1 - s0 + C - 1) / C, room));
     const int tid = threadIdx.x, col0 = slice * DC;
     for (int e = tid; e < DK * DC; e += NT) {
         const int r = e / DC, cc = e % DC;
@@ -294,9 +297,12 @@ __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p
     const int slice = static_cast<int>(blockIdx.x % G);
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
     int64_t s0, s1;
-    seq_span(p.cu, n, p.num_seqs, p.total_tokens, s0, s1);
-    const int nck = static_cast<int>((s1 - s0 + C - 1) / C);
+    if (!seq_span(p.cu, n, p.num_seqs, p.total_tokens, s0, s1) && threadIdx.x == 0 && slice == 0)
+        atomicOr(&g_kda_error_word, kErrBadSeqlens);
     const int64_t base = bc_chunk_base(p, n);
+    // malformed cu_seqlens (flagged above) are cut short: no record past the workspace's
+    const int64_t room = p.ck_records - base > 0 ? p.ck_records - base : 0;
+    const int nck = static_cast<int>(min64((s1 - s0 + C - 1) / C, room));
     const int64_t H = p.H;
     const int tid = threadIdx.x, col0 = slice * DC;
     for (int e = tid; e < DK * DC; e += NT) {

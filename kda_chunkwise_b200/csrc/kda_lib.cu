@@ -1,6 +1,8 @@
 // libkda: C ABI entry points (declared in include/kda.h), argument validation and launches.
 // The whole library is this one translation unit; kernels live in the included headers.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <atomic>
@@ -14,6 +16,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_fused.cuh"
+#include "prefill_tc.cuh"
 #include "speculative.cuh"
 #include "preprocess.cuh"
 #include "state_map.cuh"
@@ -83,6 +86,76 @@ kda_status launch_prefill(const kda::FusedParams &p, int64_t units, cudaStream_t
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kda::kda_prefill_fused_kernel<DK, DV>, p);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return KDA_OK;
+}
+
+
+// ---- the per-unit tensor-core prefill (d_k = d_v = 128) -----------------------------------------
+
+// Which prefill kernel kda_chunk_fwd runs: 0 = chosen from the shapes, 1 = cluster kernel with the
+// L2 ring, 2 = one CTA per unit (set by kda_set_prefill_path; for tests and measurements).
+std::atomic<int> g_prefill_path{0};
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// 3-d map over a [T, H, 128] bf16 tensor: boxes of 64 channels x 1 head x 64 tokens, 128-byte
+// swizzle (the layout the kernel's shared-memory operands use); rows past T read as zeros.
+bool encode_thd(CUtensorMap *map, const void *ptr, int64_t T, int H) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return sms;
+}
+
+// The per-unit kernel keeps each unit on one SM (no workspace, no traffic between SMs); the
+// cluster kernel spreads a unit's chunks over four SMs.  With few units the cluster kernel's
+// extra SMs per unit win; once the units fill the device the per-unit kernel does.
+bool use_tc_prefill(int64_t units, int d_k, int d_v) {
+    if (d_k != 128 || d_v != 128) return false;
+    if (g_inject_stall.load(std::memory_order_relaxed)) return false;   // the injection targets the cluster kernel
+    const int forced = g_prefill_path.load(std::memory_order_relaxed);
+    if (forced) return forced == 2;
+    return units * 3 > device_sm_count();
+}
+
+kda_status launch_prefill_tc(const void *q, const void *k, const void *v, const void *a, const void *gate,
+                             const kda::tc::Params &p, int64_t units, cudaStream_t stream) {
+    kda::tc::Maps maps;
+    if (!encode_thd(&maps.q, q, p.total_tokens, p.H) || !encode_thd(&maps.k, k, p.total_tokens, p.H) ||
+        !encode_thd(&maps.v, v, p.total_tokens, p.H) || !encode_thd(&maps.a, a, p.total_tokens, p.H) ||
+        !encode_thd(&maps.gate, gate ? gate : q, p.total_tokens, p.H))
+        return fail(KDA_ERR_CUDA, "kda_chunk_fwd: cuTensorMapEncodeTiled failed");
+    cudaError_t e = cudaFuncSetAttribute(kda::tc::kda_prefill_tc_kernel<>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kda::tc::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
+    kda::tc::kda_prefill_tc_kernel<><<<(unsigned)units, kda::tc::kThreads, kda::tc::kSmemBytes, stream>>>(maps, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prefill_tc launch");
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return KDA_OK;
 }
@@ -219,6 +292,7 @@ size_t kda_chunk_fwd_workspace_min(int64_t total_tokens, int32_t num_seqs, int32
     if (!sizes_ok(total_tokens, num_seqs, max_seqlen, H) || !supported_dim(d_k) || !supported_dim(d_v))
         return 0;
     const int64_t units = (int64_t)num_seqs * H;
+    if (use_tc_prefill(units, d_k, d_v)) return 0;
     return ring_bytes(units, d_k, d_v);
 }
 
@@ -253,10 +327,10 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     const void *ptrs4[] = {beta, A_log, cu_seqlens};
     for (const void *ptr : ptrs4)
         if (ptr && !aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: beta/A_log/cu_seqlens not 4-byte aligned");
-    if (!workspace) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: NULL workspace");
+    const size_t need = kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
+    if (need > 0 && !workspace) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: NULL workspace");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: workspace not 256-byte aligned");
-    const size_t need = kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
     if (workspace_bytes < need)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: workspace too small (need " +
                                              std::to_string(need) + " bytes)");
@@ -264,6 +338,26 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     const int64_t units = (int64_t)num_seqs * H;
     if (units * (d_v / kda::kSlab) > 0x7fffffffLL)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: num_seqs * H too large");
+    if (total_tokens > 0x7fffffc0LL)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: total_tokens too large");
+    if (use_tc_prefill(units, d_k, d_v) && total_tokens > 0) {
+        kda::tc::Params tp{};
+        tp.beta = beta;
+        tp.A_log = A_log;
+        tp.cu = cu_seqlens;
+        tp.S_in = initial_state;
+        tp.S_out = final_state;
+        tp.out = out;
+        tp.total_tokens = total_tokens;
+        tp.num_seqs = num_seqs;
+        tp.H = H;
+        tp.max_seqlen = max_seqlen;
+        tp.scale = scale;
+        tp.out_f32 = out_dtype == KDA_DTYPE_F32;
+        tp.has_gate = gate != nullptr;
+        tp.wait_ns = kWaitNs;
+        return launch_prefill_tc(q, k, v, a, gate, tp, units, static_cast<cudaStream_t>(stream));
+    }
     char *ws = static_cast<char *>(workspace);
     kda::FusedParams p{};
     p.q = static_cast<const uint16_t *>(q);
@@ -351,6 +445,16 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     if (d_k == 128 && d_v == 64) return launch_decode<128, 64>(p, units, st);
     if (d_k == 64 && d_v == 128) return launch_decode<64, 128>(p, units, st);
     return launch_decode<64, 64>(p, units, st);
+}
+
+kda_status kda_set_prefill_path(int32_t path) {
+    if (path < 0 || path > 2) return fail(KDA_ERR_INVALID_ARG, "kda_set_prefill_path: path must be 0, 1 or 2");
+    g_prefill_path.store(path, std::memory_order_relaxed);
+    return KDA_OK;
+}
+
+int32_t kda_prefill_path(int64_t num_units, int32_t d_k, int32_t d_v) {
+    return use_tc_prefill(num_units, d_k, d_v) ? 2 : 1;
 }
 
 kda_status kda_inject_stall(int32_t enable, uint64_t wait_limit_ns) {
@@ -575,6 +679,7 @@ kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void
     const int64_t units = (int64_t)num_seqs * H;
     if (units * (d_v / kda::kBwdCols) > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd: num_seqs * H too large");
     kda::BwdParams p{};
+    p.ck_records = total_tokens / kda::kBwdChunk + num_seqs;
     p.q = static_cast<const uint16_t *>(q);
     p.k = static_cast<const uint16_t *>(k);
     p.v = static_cast<const uint16_t *>(v);
@@ -949,6 +1054,7 @@ kda_status kda_chunk_bwd_chunkwise(const void *q, const void *k, const void *v, 
     if (records > 0x7fffffffLL || units * (d_v / kda::kBcCols) > 0x7fffffffLL)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_chunkwise: too many chunks or units");
     kda::BwdParams p{};
+    p.ck_records = total_tokens / kda::kBcChunk + num_seqs;
     p.q = static_cast<const uint16_t *>(q);
     p.k = static_cast<const uint16_t *>(k);
     p.v = static_cast<const uint16_t *>(v);

@@ -1,0 +1,913 @@
+// Per-unit chunkwise prefill on the 5th-generation tensor cores: one CTA per (sequence, head).
+//
+// The chunkwise form ("Kimi K3 · Lesson 3 of 14", CHUNKWISE diagram; "The mapping that changed"):
+// per 64-token chunk with incoming state S, chunk-local cumulative log-decay b_r = sum_{i<=r} g_i
+// (per key channel) and Gamma_r = e^{b_r},
+//   Q^ = Gamma (.) (scale q)    K^ = Gamma (.) k    K- = (Gamma_C / Gamma) (.) k
+//   A_ij = sum_c q_ic k_jc e^{b_ic - b_jc} (j <= i)   L_ij = beta_i sum_c k_ic k_jc e^{b_ic - b_jc} (j < i)
+//   T' = (I + L)^-1 diag(beta),  W = T' K^,  U~ = T' V,  U = U~ - W S
+//   O = Q^ S + A U  (the pages' "(Gamma (.) Q) S + A V~"),   S <- Diag(Gamma_C) S + K-^T U,
+//   out = sigmoid(gate) (.) O.
+// Every chunk is dense tensor-core work; only S crosses chunk boundaries.
+//
+// The 1/Gamma rescale on 16-token tiles ("each key rescaled by the reciprocal of its accumulated
+// decay"): with r_p = b just before tile p, a token i of tile p carries the row factor
+// f_i = e^{b_i - r_p} in [e^-80, 1] (the g >= -5 floor caps a tile's decay at 80) and the key
+// factor 1/f_i in [1, e^80].  Gram block (p, q <= p) is sum_c (q_ic f_ic)(k_jc e^{r_p,c - b_jc}):
+//   - diagonal blocks (q = p): the key factor reaches e^80, beyond fp16, so these 16 x 16 x d_k
+//     products run on mma.sync m16n8k8 in tf32 (fp32 range, 11-bit significand), straight from the
+//     registers of the threads that computed the factors;
+//   - blocks below the diagonal: both factors are <= 1 and a factor that underflows belongs to a
+//     term below e^-87, so fp16 operands lose nothing: one tcgen05 MMA (M = 128: the row-scaled
+//     q and k rows of the four tiles, N = 96 rescaled keys, K = d_k) computes all of them.
+// Everything on the value path (T', K^, V, W, Q^, K-, A, S, U) is fp16 with fp32 accumulation; the
+// state's master copy is fp32 in tensor memory.
+//
+// Work per chunk (one CTA, 8 warps, the phases separated by CTA barriers):
+//   0. TMA: q, k, v, a, gate rows of the chunk (3-d tensor maps over [T, H, d], two 64-channel boxes
+//      per tensor, 128-byte swizzle), each issued as soon as its buffer is free; a is double buffered.
+//   1. pass 1 (thread = 2 channels x 16 tokens): g = -5 sigmoid(e^{A_h} a) in log2 units, the
+//      within-tile running sum l, tile totals; tables e^{r_p}, e^{b_C - r_p}, e^{r_p' - r_p}, Gamma_C.
+//   2. pass 2 (warp = tile x channel half, lane = the two rows and 16 channels an MMA fragment
+//      holds): f = 2^l, 1/f; the diagonal Gram blocks (mma.sync tf32); fp16 row-scaled q, k rows into
+//      TMEM (tcgen05.st 16x256b, the fragment layout); rescaled keys of later tiles (fp16) into shared
+//      memory; Q^, K^, K-, V converted in place over the input rows.
+//   3. off-diagonal Gram MMA; meanwhile the state is scaled by Gamma_C in TMEM and Q^ copied to TMEM.
+//   4. solve: 16 x 16 diagonal inverses by forward substitution, off-diagonal blocks of T' level by
+//      level (mma.sync); A assembled from the diagonal and off-diagonal Gram blocks.
+//   5. D[0:64] = [T'; 0] [K^ | V] = [W | U~]                         (tcgen05, N = 256, K = 64)
+//   6. -W -> TMEM, beside Q^ (rows 64-127)
+//   7. D[:, 128:256] += [-W; Q^] S   -> rows 0-63 U, rows 64-127 Q^ S  (tcgen05, A in TMEM)
+//   8. U -> shared memory (fp16)
+//   9. S += K-^T U  (S pre-scaled by Gamma_C);  D[:, 128:256] += [0; A] U  -> rows 64-127 O
+//  10. fp16 copy of the new S; out = sigmoid(gate) O, staged in shared memory, stored row by row.
+// Every wait on a TMA or MMA completion is bounded (%globaltimer); a timeout records kErrTimeout in
+// the device error word and every thread leaves the chunk loop at the next barrier.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "mma_frag.cuh"
+#include "umma.cuh"
+
+namespace kda {
+namespace tc {
+
+constexpr int kThreads = 256;
+constexpr int kD = 128;            // d_k = d_v of this kernel
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---- shared memory map (bytes; every operand tile 1024-aligned) ----------------------------------
+constexpr int kQ = 0;              // q -> Q^            SW128 [2 atoms][64 rows][128 B]
+constexpr int kK = 16384;          // k -> K^            ] together the B operand [K^ | V]
+constexpr int kV = 32768;          // v -> V (fp16)      ]   (four 64-channel atoms, 8 KB apart)
+constexpr int kA0 = 49152;         // a of even chunks -> K- (A operand of K-^T U, MN-major)
+constexpr int kA1 = 65536;         // a of odd chunks  -> K-
+constexpr int kG = 81920;          // gate
+constexpr int kL = 98304;          // fp32 [64][128] within-tile log2 cumsum l (pass 1 -> pass 2);
+                                   //   then U (fp16, 16 KB) and the output staging
+constexpr int kGB = 131072;        // fp16 rescaled keys of later tiles: K-major, no swizzle, 96 rows;
+                                   //   after the Gram, [T' | 0 | A]: three SW128 [64][64] fp16 tiles
+                                   //   (the zero tile is cleared again each chunk)
+constexpr int kT = kGB, kZ = kGB + 8192, kAm = kGB + 16384;
+constexpr int kS = 155648;         // fp16 S: B operand, MN-major, no swizzle (K = d_k, N = d_v)
+constexpr int kLD = 188416;        // fp16 [64][64] swizzled: -L below the diagonal blocks, D_p on them;
+                                   //   earlier the exchange of the diagonal Gram partial sums
+constexpr int kM = 196608;         // fp16 [4][16][64] block-product scratch of the solve
+constexpr int kLdf = 204800;       // fp32 [4][16][17] diagonal blocks of L
+constexpr int kTot = kLdf + 4 * 16 * 17 * 4;   // fp32 [4][128] tile totals of l
+constexpr int kTE = kTot + 2048;   // fp32 [4][128] 2^{r_p}
+constexpr int kTK = kTE + 2048;    // fp32 [4][128] 2^{b_C - r_p}
+constexpr int kTD = kTK + 2048;    // fp32 [6][128] 2^{r_p' - r_p}, p < p'
+constexpr int kGam = kTD + 3072;   // fp32 [128] Gamma_C
+constexpr int kBeta = kGam + 512;  // fp32 [64]
+constexpr int kBar = kBeta + 256;  // u64 mbarriers: q, kv, a0, a1, gate, mma
+constexpr int kMisc = kBar + 64;   // u32 TMEM base, int abort flag
+constexpr int kSmemBytes = kMisc + 16;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kGB + 3 * 8192 <= kS && kGB + 96 * 256 <= kS, "GB region");
+
+// ---- tensor memory columns -----------------------------------------------------------------------
+constexpr uint32_t cWU = 0;        // [W | U~] -> [. | U ; . | O]  (256 columns)
+constexpr uint32_t cGA = 0;        // fp16 row-scaled rows (A operand of the off-diagonal Gram), 64 cols
+constexpr uint32_t cGD = 64;       // off-diagonal Gram (fp32), 96 columns
+constexpr uint32_t cS = 256;       // fp32 state (128 columns)
+constexpr uint32_t cWQ = 384;      // fp16 [-W; Q^] (A operand of the state products), 64 columns
+
+// order of the off-diagonal key rows: tile p' uses rows off(p') .. off(p') + 16 p' - 1
+__host__ __device__ constexpr int gb_off(int pp) { return pp == 1 ? 0 : pp == 2 ? 16 : 48; }
+__host__ __device__ constexpr int td_index(int p, int pp) { return p == 0 ? pp - 1 : p == 1 ? pp + 1 : 5; }
+
+struct Params {
+    const float *beta, *A_log;
+    const int32_t *cu;
+    const float *S_in;
+    float *S_out;
+    void *out;
+    int64_t total_tokens;
+    int num_seqs, H;
+    int max_seqlen;
+    float scale;
+    bool out_f32, has_gate;
+    unsigned long long wait_ns;
+};
+
+struct Maps {
+    CUtensorMap q, k, v, a, gate;
+};
+
+// ---- small PTX helpers ---------------------------------------------------------------------------
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile("{\n.reg .pred P;\nelect.sync _|P, 0xffffffff;\nselp.u32 %0, 1, 0, P;\n}\n" : "=r"(p));
+    return p != 0;
+}
+
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, unsigned long long ns) {
+    if (mbar_try(bar, parity)) return true;
+    const unsigned long long t0 = gtimer();
+    while (!mbar_try(bar, parity))
+        if (gtimer() - t0 > ns) return false;
+    return true;
+}
+
+__device__ __forceinline__ void expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// one 64-channel x 64-token box of a [T, H, d] tensor (x = channel offset, 0 or 64)
+__device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap *map, int x, int h, int t, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// tcgen05.st 16x256b: lane (g, t) of the warp writes TMEM lanes base + g (r0, r1) and base + g + 8
+// (r2, r3), columns 2t and 2t + 1 of the 8-column block at taddr -- the m16n8 fragment layout.
+__device__ __forceinline__ void tmem_st_frag(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2),
+                 "r"(r3)
+                 : "memory");
+}
+
+// tcgen05.mma kind::f16 with both operands in shared memory, or A in tensor memory
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+                 "l"(a), "l"(b), "r"(idesc), "r"(acc)
+                 : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+                 "r"(a), "l"(b), "r"(idesc), "r"(acc)
+                 : "memory");
+}
+
+// shared-memory matrix descriptor: no swizzle (layout 0) or 128-byte swizzle (layout 2)
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+// instruction descriptor, kind::f16: fp16 A and B, fp32 D, A/B major (0 = K, 1 = MN)
+__host__ __device__ constexpr uint32_t idesc(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// byte offset of element (row, col) of a [rows][64]-element SW128 tile (2-byte elements)
+__device__ __forceinline__ uint32_t sw128(int row, int col) {
+    return row * 128 + ((((col >> 3) ^ row) & 7) << 4) + ((col & 7) << 1);
+}
+// element (token i, channel c) of a TMA-loaded [2 atoms][64][64] tile
+__device__ __forceinline__ uint32_t in_off(int i, int c) { return (c >> 6) * 8192 + sw128(i, c & 63); }
+// byte offset of element (k, n) of an MN-major, no-swizzle fp16 B operand with N = 128
+__device__ __forceinline__ uint32_t bmn_off(int k, int n) { return (((k >> 3) * 16 + (n >> 3)) << 7) + ((k & 7) << 4) + ((n & 7) << 1); }
+// fp32 l table [64][128] with its 16-byte chunks XOR-ed by 4 (row & 1): conflict-free for both passes
+__device__ __forceinline__ uint32_t l_off(int i, int c) { return i * 512 + ((((c >> 2) ^ ((i & 1) << 2))) << 4) + ((c & 3) << 2); }
+
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) { asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a), "r"(v)); }
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+    asm volatile("st.shared.v2.b32 [%0], {%1,%2};\n" ::"r"(a), "r"(x), "r"(y));
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+}
+
+__device__ __forceinline__ void bar_all() { named_bar(1, kThreads); }
+
+// ---------------------------------------------------------------------------------------------
+// The solve: T' = (I + L)^-1 diag(beta) from the fp32 diagonal blocks Ld[p] and the fp16 blocks
+// -L_pm (m < p) in LD.  (1) D_p = (I + L_pp)^-1 by column-oriented forward substitution, one column
+// per lane, written as fp16 into the diagonal blocks of LD and, times beta, of T'.  (2) level by
+// level d = p - q:  T'_pq = D_p sum_{m=q}^{p-1} (-L_pm) T'_mq  as 16 x 16 products; starting from
+// D_q diag(beta_q) yields T' directly.  T' is an SW128 [64][64] tile (the MMA's A operand).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
+    const uint32_t base = smem_u32(sm);
+    const float *Ld = reinterpret_cast<const float *>(sm + kLdf);
+    const float *sbeta = reinterpret_cast<const float *>(sm + kBeta);
+    const int g = lane >> 2, t4 = lane & 3;
+    if (warp < 4 && lane < 16) {
+        const int pb = warp, mcol = lane;
+        const float *L = Ld + pb * 16 * 17;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = i == mcol ? 1.f : 0.f;
+#pragma unroll
+        for (int j = 0; j < 15; ++j)
+#pragma unroll
+            for (int i = j + 1; i < 16; ++i) x[i] = fmaf(-L[i * 17 + j], x[j], x[i]);
+        const float bcol = sbeta[16 * pb + mcol];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 * pb + i, c = 16 * pb + mcol;
+            *reinterpret_cast<__half *>(sm + kLD + sw128(r, c)) = __float2half_rn(x[i]);
+            *reinterpret_cast<__half *>(sm + kT + sw128(r, c)) = __float2half_rn(x[i] * bcol);
+        }
+    } else if (warp >= 4) {   // zero the blocks of T' above the diagonal: (0,1..3), (1,2..3), (2,3)
+        for (int e = (warp - 4) * 32 + lane; e < 6 * 16 * 2; e += 128) {
+            const int ub = e / 32, rem = e % 32, r = rem >> 1, half = rem & 1;
+            const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
+            sts128(base + kT + sw128(16 * pb + r, 16 * qb + 8 * half), make_uint4(0, 0, 0, 0));
+        }
+    }
+    bar_all();
+#pragma unroll 1
+    for (int d = 1; d < 4; ++d) {
+        if (warp < 4 - d) {
+            const int qb = warp, pb = warp + d;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int mb = qb; mb < pb; ++mb) {
+                uint32_t af[4], bf[4];
+                ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * mb, lane));   // -L_pm
+                ldsm_x4_t(bf, ldsm_addr_bt<128>(base + kT, 16 * mb, 16 * qb, lane));  // T'_mq
+                mma_f16(acc[0], af, bf[0], bf[1]);
+                mma_f16(acc[1], af, bf[2], bf[3]);
+            }
+            const uint32_t aMw = base + kM + warp * 2048;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int cc = 8 * j + 2 * t4;
+                sts32(aMw + swz_elem<64>(g, cc), pack_f16(acc[j][0], acc[j][1]));
+                sts32(aMw + swz_elem<64>(g + 8, cc), pack_f16(acc[j][2], acc[j][3]));
+            }
+            __syncwarp();
+            float tq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            {
+                uint32_t af[4], bf[4];
+                ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * pb, lane));   // D_p
+                ldsm_x4_t(bf, ldsm_addr_bt<64>(aMw, 0, 0, lane));
+                mma_f16(tq[0], af, bf[0], bf[1]);
+                mma_f16(tq[1], af, bf[2], bf[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int cc = 16 * qb + 8 * j + 2 * t4;
+                sts32(base + kT + sw128(16 * pb + g, cc), pack_f16(tq[j][0], tq[j][1]));
+                sts32(base + kT + sw128(16 * pb + g + 8, cc), pack_f16(tq[j][2], tq[j][3]));
+            }
+        }
+        bar_all();
+    }
+}
+
+template <bool kSelfTest = false>
+__global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
+    extern __shared__ __align__(1024) unsigned char sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int unit = blockIdx.x;
+    const int n = unit / p.H, h = unit % p.H;
+    const uint32_t base = smem_u32(sm);
+    const uint32_t bQ = base + kBar, bKV = bQ + 8, bA0 = bQ + 16, bA1 = bQ + 24, bGt = bQ + 32, bMma = bQ + 40;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kMisc + 4);
+
+    int64_t s0, s1;
+    const bool well_formed = seq_span(p.cu, n, p.num_seqs, p.total_tokens, s0, s1);
+    if (h == 0 && tid == 0) {
+        if (!well_formed) atomicOr(&g_kda_error_word, kErrBadSeqlens);
+        if (p.max_seqlen > 0 && s1 - s0 > p.max_seqlen) atomicOr(&g_kda_error_word, kErrSeqTooLong);
+    }
+    const int nchunks = static_cast<int>((s1 - s0 + kChunk - 1) / kChunk);
+
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(bQ + 8 * i, 1);
+        *abort_flag = 0;
+        prefetch_map(&maps.q); prefetch_map(&maps.k); prefetch_map(&maps.v); prefetch_map(&maps.a);
+        if (p.has_gate) prefetch_map(&maps.gate);
+    }
+    if (warp == 0) tmem_alloc(base + kMisc, 512);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kMisc);
+
+    const float expA = expf(p.A_log[h]);
+    const int64_t H = p.H;
+    float *sbeta = reinterpret_cast<float *>(sm + kBeta);
+    // TMA issue (one elected lane of warp 0; `leader` is that lane)
+    const bool wq0 = warp == 0;
+    const bool leader = wq0 && elect_one();
+    uint32_t pend = 0, pend_par = 0;   // leader only: loads in flight per barrier and their wait parity
+    auto issued = [&](int i, uint32_t parity) { pend |= 1u << i; pend_par = (pend_par & ~(1u << i)) | (parity << i); };
+    auto load_pair = [&](const CUtensorMap *map, uint32_t dst, uint32_t bar, int cl) {
+        const int t = static_cast<int>(s0 + (int64_t)cl * kChunk);
+        tma_box(dst, map, 0, h, t, bar);
+        tma_box(dst + 8192, map, 64, h, t, bar);
+    };
+    if (leader && nchunks > 0) {
+        expect_tx(bA0, 16384); load_pair(&maps.a, base + kA0, bA0, 0); issued(2, 0);
+        expect_tx(bQ, 16384); load_pair(&maps.q, base + kQ, bQ, 0); issued(0, 0);
+        expect_tx(bKV, 32768); load_pair(&maps.k, base + kK, bKV, 0); load_pair(&maps.v, base + kV, bKV, 0); issued(1, 0);
+        if (p.has_gate) { expect_tx(bGt, 16384); load_pair(&maps.gate, base + kG, bGt, 0); issued(4, 0); }
+    }
+    auto load_beta = [&](int cl) -> float {
+        if (tid >= 64 || cl >= nchunks) return 0.f;
+        const int64_t tl = s0 + (int64_t)cl * kChunk;
+        return tid < s1 - tl ? __ldg(p.beta + (tl + tid) * H + h) : 0.f;
+    };
+    float beta_next = load_beta(0);
+
+    // epilogue mapping: TMEM lane quadrant q = warp % 4 (rows 32q + lane), column half hf = warp / 4
+    const int q4 = warp & 3, hf = warp >> 2, row = 32 * q4 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+
+    // initial state -> TMEM (fp32) and its fp16 copy (B operand)
+    {
+        const size_t st_base = ((size_t)n * H + h) * kD * kD;
+        float x[64];
+        if (p.S_in) {
+            const float4 *sp = reinterpret_cast<const float4 *>(p.S_in + st_base + (size_t)row * kD + 64 * hf);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float4 v = __ldg(sp + j);
+                x[4 * j] = v.x; x[4 * j + 1] = v.y; x[4 * j + 2] = v.z; x[4 * j + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) x[j] = 0.f;
+        }
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+            uint32_t v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(x[16 * part + e]);
+            tmem_st16(tq + cS + 64 * hf + 16 * part, v);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            sts128(base + kS + bmn_off(row, 64 * hf + 8 * j),
+                   make_uint4(pack_f16(x[8 * j], x[8 * j + 1]), pack_f16(x[8 * j + 2], x[8 * j + 3]),
+                              pack_f16(x[8 * j + 4], x[8 * j + 5]), pack_f16(x[8 * j + 6], x[8 * j + 7])));
+        tmem_wait_st();
+    }
+
+    uint32_t mma_phase = 0;
+    auto mma_wait = [&]() {   // every thread waits for the latest commit (bounded)
+        const bool ok = wait_bounded(bMma, mma_phase, p.wait_ns);
+        mma_phase ^= 1;
+        if (!ok) { atomicOr(&g_kda_error_word, kErrTimeout); *abort_flag = 1; }
+    };
+    auto mma_sync = [&]() {   // ... then a CTA barrier, after which the flag is read by everyone
+        mma_wait();
+        tc_fence_before();
+        bar_all();
+        tc_fence_after();
+    };
+    auto in_wait = [&](uint32_t bar, uint32_t parity) {
+        if (!wait_bounded(bar, parity, p.wait_ns)) { atomicOr(&g_kda_error_word, kErrTimeout); *abort_flag = 1; }
+        else pend &= ~(1u << ((bar - bQ) >> 3));
+    };
+    auto sync_tc = [&]() {   // shared-memory and TMEM writes visible to the tensor core and all threads
+        fence_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        bar_all();
+        tc_fence_after();
+    };
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int64_t t0 = s0 + (int64_t)c * kChunk;
+        const int L = static_cast<int>(min64(kChunk, s1 - t0));
+        const uint32_t aBuf = (c & 1) ? base + kA1 : base + kA0;
+        const uint32_t aBar = (c & 1) ? bA1 : bA0;
+        if (tid < 64) sbeta[tid] = beta_next;
+        beta_next = load_beta(c + 1);
+        // the next chunk's a goes into the other buffer (its K- of chunk c-1 is consumed)
+        if (leader && c + 1 < nchunks) {
+            fence_async_smem();
+            const uint32_t nb = (c & 1) ? base + kA0 : base + kA1, nbar = (c & 1) ? bA0 : bA1;
+            expect_tx(nbar, 16384);
+            load_pair(&maps.a, nb, nbar, c + 1);
+            issued((c & 1) ? 2 : 3, ((c + 1) >> 1) & 1);
+        }
+        in_wait(aBar, (c >> 1) & 1);
+
+        // ---- 1. pass 1: g, within-tile running sums, tile totals ---------------------------------
+        {
+            const int cp = tid & 63, pt = tid >> 6, c0 = 2 * cp;
+            float lx[16], ly[16];
+            float sx = 0.f, sy = 0.f;
+            constexpr float kG2 = kGMin * kLog2e;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int t = 16 * pt + i;
+                const float2 av = unpack_bf16(lds32(aBuf + in_off(t, c0)));
+                float gx = kG2 * sigmoid_fast(expA * av.x), gy = kG2 * sigmoid_fast(expA * av.y);
+                if (t >= L) gx = gy = 0.f;
+                sx += gx; sy += gy;
+                lx[i] = sx; ly[i] = sy;
+            }
+            float *tot = reinterpret_cast<float *>(sm + kTot);
+            *reinterpret_cast<float2 *>(tot + pt * 128 + c0) = make_float2(sx, sy);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int t = 16 * pt + i;
+                *reinterpret_cast<float2 *>(sm + kL + l_off(t, c0)) = make_float2(lx[i], ly[i]);
+            }
+            bar_all();
+            float2 tv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tv[q] = *reinterpret_cast<const float2 *>(tot + q * 128 + c0);
+            float2 R = make_float2(0.f, 0.f), BC = R;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (q < pt) { R.x += tv[q].x; R.y += tv[q].y; }
+                BC.x += tv[q].x; BC.y += tv[q].y;
+            }
+            *reinterpret_cast<float2 *>(sm + kTE + (pt * 128 + c0) * 4) = make_float2(ex2(R.x), ex2(R.y));
+            *reinterpret_cast<float2 *>(sm + kTK + (pt * 128 + c0) * 4) = make_float2(ex2(BC.x - R.x), ex2(BC.y - R.y));
+            float2 Rn = R;
+#pragma unroll
+            for (int pp = 1; pp < 4; ++pp) {
+                if (pp <= pt) continue;
+                Rn.x += tv[pp - 1].x; Rn.y += tv[pp - 1].y;
+                if (pp - 1 >= pt)
+                    *reinterpret_cast<float2 *>(sm + kTD + (td_index(pt, pp) * 128 + c0) * 4) =
+                        make_float2(ex2(Rn.x - R.x), ex2(Rn.y - R.y));
+            }
+            if (pt == 0) *reinterpret_cast<float2 *>(sm + kGam + c0 * 4) = make_float2(ex2(BC.x), ex2(BC.y));
+        }
+        in_wait(bQ, c & 1);
+        in_wait(bKV, c & 1);
+        bar_all();
+        if (*abort_flag) break;
+
+        // ---- 2. pass 2: operands and the diagonal Gram blocks -------------------------------------
+        float qk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float kk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const int pt = warp & 3, ch = warp >> 2;         // tile, channel half
+        const int g = lane >> 2, t4 = lane & 3;
+        {
+            const int i0 = 16 * pt + g, i1 = i0 + 8;
+            const bool in0 = i0 < L, in1 = i1 < L;
+#pragma unroll 1
+            for (int s = 0; s < 4; ++s) {
+                const int cb = 64 * ch + 16 * s + 4 * t4;     // this lane's 4 channels cb .. cb + 3
+                // inputs (bf16 x 4 per row), l (fp32 x 4 per row), tables
+                const uint32_t oq0 = in_off(i0, cb), oq1 = in_off(i1, cb);
+                uint2 qr0 = lds64(base + kQ + oq0), qr1 = lds64(base + kQ + oq1);
+                uint2 kr0 = lds64(base + kK + oq0), kr1 = lds64(base + kK + oq1);
+                uint2 vr0 = lds64(base + kV + oq0), vr1 = lds64(base + kV + oq1);
+                const float4 l0 = *reinterpret_cast<const float4 *>(sm + kL + l_off(i0, cb));
+                const float4 l1 = *reinterpret_cast<const float4 *>(sm + kL + l_off(i1, cb));
+                const float4 te = *reinterpret_cast<const float4 *>(sm + kTE + (pt * 128 + cb) * 4);
+                const float4 tk = *reinterpret_cast<const float4 *>(sm + kTK + (pt * 128 + cb) * 4);
+                float qv[2][4], kv[2][4], lv[2][4];
+                {
+                    const float2 a0 = unpack_bf16(qr0.x), a1 = unpack_bf16(qr0.y), b0 = unpack_bf16(qr1.x), b1 = unpack_bf16(qr1.y);
+                    qv[0][0] = a0.x; qv[0][1] = a0.y; qv[0][2] = a1.x; qv[0][3] = a1.y;
+                    qv[1][0] = b0.x; qv[1][1] = b0.y; qv[1][2] = b1.x; qv[1][3] = b1.y;
+                    const float2 c0 = unpack_bf16(kr0.x), c1 = unpack_bf16(kr0.y), d0 = unpack_bf16(kr1.x), d1 = unpack_bf16(kr1.y);
+                    kv[0][0] = c0.x; kv[0][1] = c0.y; kv[0][2] = c1.x; kv[0][3] = c1.y;
+                    kv[1][0] = d0.x; kv[1][1] = d0.y; kv[1][2] = d1.x; kv[1][3] = d1.y;
+                    lv[0][0] = l0.x; lv[0][1] = l0.y; lv[0][2] = l0.z; lv[0][3] = l0.w;
+                    lv[1][0] = l1.x; lv[1][1] = l1.y; lv[1][2] = l1.z; lv[1][3] = l1.w;
+                }
+                if (!in0) { qv[0][0] = qv[0][1] = qv[0][2] = qv[0][3] = 0.f; kv[0][0] = kv[0][1] = kv[0][2] = kv[0][3] = 0.f; vr0 = make_uint2(0, 0); }
+                if (!in1) { qv[1][0] = qv[1][1] = qv[1][2] = qv[1][3] = 0.f; kv[1][0] = kv[1][1] = kv[1][2] = kv[1][3] = 0.f; vr1 = make_uint2(0, 0); }
+                const float tev[4] = {te.x, te.y, te.z, te.w}, tkv[4] = {tk.x, tk.y, tk.z, tk.w};
+                float qr[2][4], kr[2][4], kt[2][4];   // row-scaled q, k (<= 1) and rescaled keys (>= 1)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float f = ex2(lv[r][e]), fi = ex2(-lv[r][e]);
+                        qr[r][e] = p.scale * qv[r][e] * f;
+                        kr[r][e] = kv[r][e] * f;
+                        kt[r][e] = kv[r][e] * fi;
+                    }
+                // diagonal Gram blocks, tf32: k-step u uses channels cb + 2u (slot t4) and cb + 2u + 1 (slot t4 + 4)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int e0 = 2 * u, e1 = 2 * u + 1;
+                    const uint32_t aq0 = to_tf32(qr[0][e0]), aq1 = to_tf32(qr[1][e0]), aq2 = to_tf32(qr[0][e1]), aq3 = to_tf32(qr[1][e1]);
+                    const uint32_t ak0 = to_tf32(kr[0][e0]), ak1 = to_tf32(kr[1][e0]), ak2 = to_tf32(kr[0][e1]), ak3 = to_tf32(kr[1][e1]);
+                    const uint32_t b00 = to_tf32(kt[0][e0]), b01 = to_tf32(kt[0][e1]), b10 = to_tf32(kt[1][e0]), b11 = to_tf32(kt[1][e1]);
+                    mma_tf32(qk[0], aq0, aq1, aq2, aq3, b00, b01);
+                    mma_tf32(qk[1], aq0, aq1, aq2, aq3, b10, b11);
+                    mma_tf32(kk[0], ak0, ak1, ak2, ak3, b00, b01);
+                    mma_tf32(kk[1], ak0, ak1, ak2, ak3, b10, b11);
+                }
+                // fp16 row-scaled q, k rows -> TMEM (Gram A operand; rows of tile pt: q at lanes 32pt..+15,
+                // k at 32pt + 16..+31; columns = channel pairs)
+                {
+                    const uint32_t col = tmem + cGA + (uint32_t)(32 * ch + 8 * s);
+                    tmem_st_frag(col + ((uint32_t)(32 * pt) << 16), pack_f16(qr[0][0], qr[0][1]), pack_f16(qr[0][2], qr[0][3]),
+                                 pack_f16(qr[1][0], qr[1][1]), pack_f16(qr[1][2], qr[1][3]));
+                    tmem_st_frag(col + ((uint32_t)(32 * pt + 16) << 16), pack_f16(kr[0][0], kr[0][1]), pack_f16(kr[0][2], kr[0][3]),
+                                 pack_f16(kr[1][0], kr[1][1]), pack_f16(kr[1][2], kr[1][3]));
+                }
+                // rescaled keys for the later tiles' off-diagonal blocks: row gb_off(pp) + i
+#pragma unroll
+                for (int pp = 1; pp < 4; ++pp) {
+                    if (pp <= pt) continue;
+                    const float4 td = *reinterpret_cast<const float4 *>(sm + kTD + (td_index(pt, pp) * 128 + cb) * 4);
+                    const float tdv[4] = {td.x, td.y, td.z, td.w};
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int nrow = gb_off(pp) + (r ? i1 : i0);
+                        const uint32_t o = kGB + (nrow >> 3) * 2048 + (cb >> 3) * 128 + (nrow & 7) * 16 + (cb & 7) * 2;
+                        sts64(base + o, pack_f16(kt[r][0] * tdv[0], kt[r][1] * tdv[1]), pack_f16(kt[r][2] * tdv[2], kt[r][3] * tdv[3]));
+                    }
+                }
+                // in place: Q^ = q^ e^{r_p}, K^ = k^ e^{r_p}, V -> fp16; K- = K~ e^{b_C - r_p} into the a buffer
+                sts64(base + kQ + oq0, pack_f16(qr[0][0] * tev[0], qr[0][1] * tev[1]), pack_f16(qr[0][2] * tev[2], qr[0][3] * tev[3]));
+                sts64(base + kQ + oq1, pack_f16(qr[1][0] * tev[0], qr[1][1] * tev[1]), pack_f16(qr[1][2] * tev[2], qr[1][3] * tev[3]));
+                sts64(base + kK + oq0, pack_f16(kr[0][0] * tev[0], kr[0][1] * tev[1]), pack_f16(kr[0][2] * tev[2], kr[0][3] * tev[3]));
+                sts64(base + kK + oq1, pack_f16(kr[1][0] * tev[0], kr[1][1] * tev[1]), pack_f16(kr[1][2] * tev[2], kr[1][3] * tev[3]));
+                sts64(aBuf + oq0, pack_f16(kt[0][0] * tkv[0], kt[0][1] * tkv[1]), pack_f16(kt[0][2] * tkv[2], kt[0][3] * tkv[3]));
+                sts64(aBuf + oq1, pack_f16(kt[1][0] * tkv[0], kt[1][1] * tkv[1]), pack_f16(kt[1][2] * tkv[2], kt[1][3] * tkv[3]));
+                sts64(base + kV + oq0, bf16x2_to_f16x2(vr0.x), bf16x2_to_f16x2(vr0.y));
+                sts64(base + kV + oq1, bf16x2_to_f16x2(vr1.x), bf16x2_to_f16x2(vr1.y));
+            }
+        }
+        // rescaled keys of the off-diagonal rows beyond what pass 2 wrote: none (every row is written)
+        // combine the two channel halves' diagonal partial sums in the warps of half 0
+        {
+            float *xch = reinterpret_cast<float *>(sm + kLD) + pt * 512;
+            if (ch == 1) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    xch[e * 32 + lane] = qk[e >> 2][e & 3];
+                    xch[(8 + e) * 32 + lane] = kk[e >> 2][e & 3];
+                }
+            }
+            sync_tc();
+            if (*abort_flag) break;
+            if (ch == 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    qk[e >> 2][e & 3] += xch[e * 32 + lane];
+                    kk[e >> 2][e & 3] += xch[(8 + e) * 32 + lane];
+                }
+            }
+        }
+
+        // ---- 3. off-diagonal Gram (TMEM A rows x rescaled keys) ----------------------------------
+        if (wq0) {
+            if (leader) {
+                constexpr uint32_t id = idesc(128, 96, 0, 0);
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k)
+                    mma_ts(tmem + cGD, tmem + cGA + 8 * k, sdesc(base + kGB + 256 * k, 128, 2048, 0), id, k > 0);
+                umma_commit(bMma);
+            }
+            __syncwarp();
+        }
+        // meanwhile: S <- Gamma_C S (fp32, in TMEM); Q^ -> TMEM rows 64-127 of [-W; Q^]
+        {
+            const float gam = reinterpret_cast<const float *>(sm + kGam)[row];
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                uint32_t v[16];
+                tmem_ld16(tq + cS + 64 * hf + 16 * part, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(gam * __uint_as_float(v[e]));
+                tmem_st16(tq + cS + 64 * hf + 16 * part, v);
+            }
+            if (q4 >= 2) {
+                const int i = row - 64;   // token row of Q^
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    uint32_t v[16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 x = lds128(base + kQ + in_off(i, 64 * hf + 32 * part + 8 * j));
+                        v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                    }
+                    tmem_st16(tq + cWQ + 32 * hf + 16 * part, v);
+                }
+            }
+        }
+        mma_wait();
+        tmem_wait_st();
+        tc_fence_before();
+        bar_all();
+        tc_fence_after();
+        if (*abort_flag) break;
+        // q buffer is free: the next chunk's q
+        if (leader && c + 1 < nchunks) {
+            fence_async_smem();
+            expect_tx(bQ, 16384);
+            load_pair(&maps.q, base + kQ, bQ, c + 1);
+            issued(0, (c + 1) & 1);
+        }
+
+        // ---- 4. solve inputs: A rows (tile pt) and -L rows from the Gram, diagonal blocks ----------
+        {
+            const float *sb = reinterpret_cast<const float *>(sm + kBeta);
+            if (ch == 0) {
+                // diagonal blocks from the fragments: A (j <= i) and L (j < i, times beta_i)
+                float *Ldp = reinterpret_cast<float *>(sm + kLdf) + pt * 16 * 17;
+                const float bi0 = sb[16 * pt + g], bi1 = sb[16 * pt + g + 8];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int j = 8 * nt + 2 * t4;   // column within the tile
+                    const int r0 = g, r1 = g + 8;
+                    sts32(base + kAm + sw128(16 * pt + r0, 16 * pt + j),
+                          pack_f16(j <= r0 ? qk[nt][0] : 0.f, j + 1 <= r0 ? qk[nt][1] : 0.f));
+                    sts32(base + kAm + sw128(16 * pt + r1, 16 * pt + j),
+                          pack_f16(j <= r1 ? qk[nt][2] : 0.f, j + 1 <= r1 ? qk[nt][3] : 0.f));
+                    Ldp[r0 * 17 + j] = j < r0 ? bi0 * kk[nt][0] : 0.f;
+                    Ldp[r0 * 17 + j + 1] = j + 1 < r0 ? bi0 * kk[nt][1] : 0.f;
+                    Ldp[r1 * 17 + j] = j < r1 ? bi1 * kk[nt][2] : 0.f;
+                    Ldp[r1 * 17 + j + 1] = j + 1 < r1 ? bi1 * kk[nt][3] : 0.f;
+                }
+            } else {
+                // off-diagonal rows from TMEM: lanes 32pt + r (q rows) and 32pt + 16 + r (k rows)
+                const int r = lane & 15;
+                const bool krow = lane >= 16;
+                const int i = 16 * pt + r;
+                const float bi = sb[i];
+                for (int blk = 0; blk < pt; ++blk) {   // 16 columns per block, all lanes of the warp
+                    uint32_t v[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * pt) << 16) + cGD + gb_off(pt) + 16 * blk, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint4 o;
+                        const float s = krow ? -bi : 1.f;
+                        o.x = pack_f16(s * __uint_as_float(v[8 * hh + 0]), s * __uint_as_float(v[8 * hh + 1]));
+                        o.y = pack_f16(s * __uint_as_float(v[8 * hh + 2]), s * __uint_as_float(v[8 * hh + 3]));
+                        o.z = pack_f16(s * __uint_as_float(v[8 * hh + 4]), s * __uint_as_float(v[8 * hh + 5]));
+                        o.w = pack_f16(s * __uint_as_float(v[8 * hh + 6]), s * __uint_as_float(v[8 * hh + 7]));
+                        sts128(base + (krow ? kLD : kAm) + sw128(i, 16 * blk + 8 * hh), o);
+                    }
+                }
+                if (!krow) {   // A: zeros right of the diagonal block
+                    for (int cc = 16 * (pt + 1); cc < 64; cc += 8) sts128(base + kAm + sw128(i, cc), make_uint4(0, 0, 0, 0));
+                }
+            }
+        }
+        // the zero block between T' and A shares its bytes with the rescaled keys of pass 2: clear it
+        for (int e = tid; e < 8192 / 16; e += kThreads) sts128(base + kZ + 16 * e, make_uint4(0, 0, 0, 0));
+        bar_all();
+        solve(sm, warp, lane);
+        sync_tc();   // T' visible to the tensor core
+
+        // ---- 5. [W | U~] = [T'; 0] [K^ | V] ---------------------------------------------------------
+        if (wq0) {
+            fence_async_smem();
+            if (leader) {
+                constexpr uint32_t id = idesc(128, 256, 0, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss(tmem + cWU, sdesc(base + kT + 32 * k, 16, 1024, 2), sdesc(base + kK + 2048 * k, 8192, 1024, 2), id, k > 0);
+                umma_commit(bMma);
+            }
+            __syncwarp();
+        }
+        mma_sync();
+        if (*abort_flag) break;
+        // k, v buffers are free: the next chunk's k, v
+        if (leader && c + 1 < nchunks) {
+            fence_async_smem();
+            expect_tx(bKV, 32768);
+            load_pair(&maps.k, base + kK, bKV, c + 1);
+            load_pair(&maps.v, base + kV, bKV, c + 1);
+            issued(1, (c + 1) & 1);
+        }
+        // ---- 6. -W -> TMEM rows 0-63 of [-W; Q^] ----------------------------------------------------
+        if (q4 < 2) {
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                uint32_t v[16];
+                tmem_ld16(tq + cWU + 64 * hf + 16 * part, v);
+                tmem_wait_ld();
+                uint32_t w[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) w[e] = pack_f16(-__uint_as_float(v[2 * e]), -__uint_as_float(v[2 * e + 1]));
+                asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(tq + cWQ + 32 * hf + 8 * part),
+                             "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                             : "memory");
+            }
+        }
+        sync_tc();
+        // ---- 7. D[:, 128:256] += [-W; Q^] S --------------------------------------------------------
+        if (wq0) {
+            if (leader) {
+                constexpr uint32_t id = idesc(128, 128, 0, 1);
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k)
+                    mma_ts(tmem + cWU + 128, tmem + cWQ + 8 * k, sdesc(base + kS + 4096 * k, 2048, 128, 0), id, 1);
+                umma_commit(bMma);
+            }
+            __syncwarp();
+        }
+        mma_sync();
+        if (*abort_flag) break;
+        // ---- 8. U (rows 0-63) -> shared memory (fp16, MN-major B operand) ---------------------------
+        if (q4 < 2) {
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                uint32_t v[16];
+                tmem_ld16(tq + cWU + 128 + 64 * hf + 16 * part, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+                    sts128(base + kL + bmn_off(row, 64 * hf + 16 * part + 8 * j),
+                           make_uint4(pack_f16(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                                      pack_f16(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                                      pack_f16(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                                      pack_f16(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]))));
+            }
+        }
+        sync_tc();
+        // ---- 9. S += K-^T U;  D[:, 128:256] += [0; A] U -------------------------------------------
+        if (wq0) {
+            if (leader) {
+                constexpr uint32_t id = idesc(128, 128, 1, 1), id2 = idesc(128, 128, 0, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss(tmem + cS, sdesc(aBuf + 2048 * k, 8192, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss(tmem + cWU + 128, sdesc(base + kZ + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);
+                umma_commit(bMma);
+            }
+            __syncwarp();
+        }
+        // the gate rows of this chunk must have arrived
+        if (p.has_gate) in_wait(bGt, c & 1);
+        mma_sync();
+        if (*abort_flag) break;
+        // ---- 10. new S (fp16 copy); gated output rows -----------------------------------------------
+        {
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                uint32_t v[16];
+                tmem_ld16(tq + cS + 64 * hf + 16 * part, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+                    sts128(base + kS + bmn_off(row, 64 * hf + 16 * part + 8 * j),
+                           make_uint4(pack_f16(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                                      pack_f16(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                                      pack_f16(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                                      pack_f16(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]))));
+            }
+            if (q4 >= 2) {
+                const int i = row - 64;
+#pragma unroll
+                for (int part = 0; part < 4; ++part) {
+                    uint32_t v[16];
+                    tmem_ld16(tq + cWU + 128 + 64 * hf + 16 * part, v);
+                    tmem_wait_ld();
+                    float o[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __uint_as_float(v[e]);
+                    const int cb = 64 * hf + 16 * part;
+                    if (p.has_gate) {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const uint4 gr = lds128(base + kG + in_off(i, cb + 8 * j));
+                            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 ga = unpack_bf16(gw[e]);
+                                o[8 * j + 2 * e] *= sigmoid_fast(ga.x);
+                                o[8 * j + 2 * e + 1] *= sigmoid_fast(ga.y);
+                            }
+                        }
+                    }
+                    if (p.out_f32) {   // staging fp32 [64][128], 16-byte chunks XOR-swizzled by row
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int chk = (cb >> 2) + j;
+                            sts128(base + kL + i * 512 + ((chk ^ (i & 7)) << 4),
+                                   make_uint4(__float_as_uint(o[4 * j]), __float_as_uint(o[4 * j + 1]), __float_as_uint(o[4 * j + 2]),
+                                              __float_as_uint(o[4 * j + 3])));
+                        }
+                    } else {           // staging bf16 [64][128]
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int chk = (cb >> 3) + j;
+                            sts128(base + kL + i * 256 + ((chk ^ (i & 7)) << 4),
+                                   make_uint4(pack_bf16(o[8 * j], o[8 * j + 1]), pack_bf16(o[8 * j + 2], o[8 * j + 3]),
+                                              pack_bf16(o[8 * j + 4], o[8 * j + 5]), pack_bf16(o[8 * j + 6], o[8 * j + 7])));
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        bar_all();
+        tc_fence_after();
+        // gate buffer free: the next chunk's gate
+        if (leader && c + 1 < nchunks && p.has_gate) {
+            fence_async_smem();
+            expect_tx(bGt, 16384);
+            load_pair(&maps.gate, base + kG, bGt, c + 1);
+            issued(4, (c + 1) & 1);
+        }
+        // rows < L of the staged output -> global, two rows per warp instruction
+        if (p.out_f32) {
+            float *outp = static_cast<float *>(p.out);
+            for (int e = tid; e < 64 * 32; e += kThreads) {
+                const int i = e >> 5, chk = e & 31;
+                if (i < L) {
+                    const uint4 x = lds128(base + kL + i * 512 + ((chk ^ (i & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(outp + ((t0 + i) * H + h) * kD + 4 * chk) = x;
+                }
+            }
+        } else {
+            uint16_t *outp = static_cast<uint16_t *>(p.out);
+            for (int e = tid; e < 64 * 16; e += kThreads) {
+                const int i = e >> 4, chk = e & 15;
+                if (i < L) {
+                    const uint4 x = lds128(base + kL + i * 256 + ((chk ^ (i & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(outp + ((t0 + i) * H + h) * kD + 8 * chk) = x;
+                }
+            }
+        }
+        bar_all();   // the staging area (kL) is rewritten by the next chunk's pass 1
+    }
+
+    if (*abort_flag && leader) {
+        // copies issued but never waited for complete before the CTA leaves (bounded)
+        for (int i = 0; i < 5; ++i)
+            if (pend >> i & 1) wait_bounded(bQ + 8 * i, pend_par >> i & 1, p.wait_ns);
+        wait_bounded(bMma, mma_phase ^ 1, p.wait_ns);
+    }
+    // final state (fp32, from TMEM)
+    if (p.S_out && !*abort_flag) {
+        const size_t st_base = ((size_t)n * H + h) * kD * kD;
+        float4 *sp = reinterpret_cast<float4 *>(p.S_out + st_base + (size_t)row * kD + 64 * hf);
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+            uint32_t v[16];
+            tmem_ld16(tq + cS + 64 * hf + 16 * part, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                sp[4 * part + j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
+                                               __uint_as_float(v[4 * j + 3]));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace tc
+}  // namespace kda

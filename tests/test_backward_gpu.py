@@ -92,3 +92,45 @@ def test_backward_full_size_sampled(kda, chunkwise):
     dA_ref = _check(kda, inp, dout, dST, g, [(0, 0), (0, 13), (0, 31)])
     for h, ref in dA_ref.items():
         assert abs(float(g["dA_log"][h]) - ref) <= 5e-3 * max(abs(ref), 1e-6), f"dA_log[{h}]"
+
+
+@pytest.mark.parametrize("chunkwise", [False, True])
+@pytest.mark.parametrize("a_mean,beta_lo", [(8.0, 0.9), (-8.0, 0.9)])
+def test_backward_saturated_and_nofade(kda, chunkwise, a_mean, beta_lo):
+    # a ~ N(8, 1): g = -5 in nearly every channel, a chunk decays by up to e^-320 (the pairwise form
+    # must keep every 1/e^b inside an e^{b_i - b_j}, i >= j); a ~ N(-8, 1): almost no fade.
+    w = KI.Workload("bwd_sat", (70, 130, 17), 2, 128, 128, a_mean=a_mean, beta="uniform_0.9_1" if beta_lo else "sigmoid_normal",
+                    gate=True, init_state="normal_0.02", seed=34)
+    inp = KI.make_inputs(w, "cuda")
+    g_ = torch.Generator(device="cuda").manual_seed(35)
+    dout = torch.randn((w.total_tokens, w.H, 128), generator=g_, device="cuda")
+    dST = torch.randn((w.num_seqs, w.H, 128, 128), generator=g_, device="cuda")
+    g = kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
+                          dout, gate=inp["gate"], initial_state=inp["initial_state"], dfinal_state=dST,
+                          chunkwise=chunkwise)
+    kda.kda_sync_check()
+    units = [(n, h) for n in range(w.num_seqs) for h in range(w.H)]
+    dA_ref = _check(kda, inp, dout, dST, g, units)
+    for h, ref in dA_ref.items():
+        assert abs(float(g["dA_log"][h]) - ref) <= 5e-3 * max(abs(ref), 1e-6), f"dA_log[{h}]"
+
+
+@pytest.mark.parametrize("chunkwise", [False, True])
+def test_backward_malformed_seqlens_stay_in_workspace(kda, chunkwise):
+    # cu_seqlens = [0, T, 0, T]: every offset in range but not monotone, so the spans add up to twice
+    # the tokens; the kernels must flag it and write nothing past the workspace they were given.
+    T, H = 640, 2
+    w = KI.Workload("bwd_bad", (T, 0, T), H, 128, 128, seed=36)
+    inp = KI.make_inputs(w, "cuda")
+    cu = torch.tensor([0, T, 0, T], dtype=torch.int32, device="cuda")
+    q, k, v, a = (inp[x][:T] for x in ("q", "k", "v", "a"))
+    beta = inp["beta"][:T]
+    dout = torch.randn((T, H, 128), device="cuda")
+    size = (kda.kda_chunk_bwd_chunkwise_workspace_size if chunkwise else kda.kda_chunk_bwd_workspace_size)(T, 3, H, 128, 128)
+    guard = 1 << 20
+    buf = torch.full((size + guard,), 0x5A, dtype=torch.uint8, device="cuda")
+    with pytest.raises(kda.KDAError):
+        kda.kda_chunk_bwd(q, k, v, a, beta, inp["A_log"], cu, dout, workspace=buf[:size], chunkwise=chunkwise)
+        kda.kda_sync_check()
+    torch.cuda.synchronize()
+    assert bool((buf[size:] == 0x5A).all()), "a kernel wrote past its workspace"
