@@ -150,10 +150,10 @@ kda_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
         !encode_thd(&maps.v, v, p.total_tokens, p.H) || !encode_thd(&maps.a, a, p.total_tokens, p.H) ||
         !encode_thd(&maps.gate, gate ? gate : q, p.total_tokens, p.H))
         return fail(KDA_ERR_CUDA, "kda_chunk_fwd: cuTensorMapEncodeTiled failed");
-    cudaError_t e = cudaFuncSetAttribute(kda::tc::kda_prefill_tc_kernel<>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kda::tc::kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kda::tc::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc)");
-    kda::tc::kda_prefill_tc_kernel<><<<(unsigned)units, kda::tc::kThreads, kda::tc::kSmemBytes, stream>>>(maps, p);
+    kda::tc::kda_prefill_tc_kernel<<<(unsigned)units, kda::tc::kThreads, kda::tc::kSmemBytes, stream>>>(maps, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill_tc launch");
     g_launches.fetch_add(1, std::memory_order_relaxed);

@@ -23,7 +23,7 @@
 // Everything on the value path (T', K^, V, W, Q^, K-, A, S, U) is fp16 with fp32 accumulation; the
 // state's master copy is fp32 in tensor memory.
 //
-// Work per chunk (one CTA, 8 warps, the phases separated by CTA barriers):
+// Work per chunk (one CTA, 16 warps, the phases separated by CTA barriers):
 //   0. TMA: q, k, v, a, gate rows of the chunk (3-d tensor maps over [T, H, d], two 64-channel boxes
 //      per tensor, 128-byte swizzle), each issued as soon as its buffer is free; a is double buffered.
 //   1. pass 1 (thread = 2 channels x 16 tokens): g = -5 sigmoid(e^{A_h} a) in log2 units, the
@@ -54,7 +54,7 @@
 namespace kda {
 namespace tc {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kD = 128;            // d_k = d_v of this kernel
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -66,18 +66,17 @@ constexpr int kA0 = 49152;         // a of even chunks -> K- (A operand of K-^T 
 constexpr int kA1 = 65536;         // a of odd chunks  -> K-
 constexpr int kG = 81920;          // gate
 constexpr int kL = 98304;          // fp32 [64][128] within-tile log2 cumsum l (pass 1 -> pass 2);
-                                   //   then U (fp16, 16 KB) and the output staging
-constexpr int kGB = 131072;        // fp16 rescaled keys of later tiles: K-major, no swizzle, 96 rows;
-                                   //   after the Gram, [T' | 0 | A]: three SW128 [64][64] fp16 tiles
-                                   //   (the zero tile is cleared again each chunk)
-constexpr int kT = kGB, kZ = kGB + 8192, kAm = kGB + 16384;
+                                   //   then U (fp16, 16 KB) and A'' (16 KB); then the output staging
+constexpr int kGB = 131072;        // fp16 rescaled keys of later tiles: K-major, no swizzle, 96 rows
+constexpr int kT = kGB;            // T'' (after the Gram): SW128 [128][64], rows in slot order (below)
+constexpr int kAm = kL + 16384;    // A'' (after pass 2): SW128 [128][64], rows in slot order
 constexpr int kS = 155648;         // fp16 S: B operand, MN-major, no swizzle (K = d_k, N = d_v)
 constexpr int kLD = 188416;        // fp16 [64][64] swizzled: -L below the diagonal blocks, D_p on them;
-                                   //   earlier the exchange of the diagonal Gram partial sums
-constexpr int kM = 196608;         // fp16 [4][16][64] block-product scratch of the solve
+                                   //   earlier (with kM) the exchange of the diagonal Gram partial sums
+constexpr int kM = 196608;         // fp16 [3][16][32] block-product scratch of the solve
 constexpr int kLdf = 204800;       // fp32 [4][16][17] diagonal blocks of L
-constexpr int kTot = kLdf + 4 * 16 * 17 * 4;   // fp32 [4][128] tile totals of l
-constexpr int kTE = kTot + 2048;   // fp32 [4][128] 2^{r_p}
+constexpr int kTot = kLdf + 4 * 16 * 17 * 4;   // fp32 [8][128] half-tile totals of l
+constexpr int kTE = kTot + 4096;   // fp32 [4][128] 2^{r_p}
 constexpr int kTK = kTE + 2048;    // fp32 [4][128] 2^{b_C - r_p}
 constexpr int kTD = kTK + 2048;    // fp32 [6][128] 2^{r_p' - r_p}, p < p'
 constexpr int kGam = kTD + 3072;   // fp32 [128] Gamma_C
@@ -88,12 +87,20 @@ constexpr int kSmemBytes = kMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(kGB + 3 * 8192 <= kS && kGB + 96 * 256 <= kS, "GB region");
 
+// ---- slot order of the 128 rows of the chunk's accumulators ---------------------------------------
+// Token row i of the chunk (tile p = i / 16, r = i % 16) has two rows: its query slot 32 p + r
+// (row-scaled q in the Gram, Q^ in the state products, the output O) and its key slot
+// 32 p + 16 + r (row-scaled k in the Gram, then W, U~, U).  Every TMEM lane quadrant thus holds
+// both slots of one tile, so the work on either kind of row is shared by all four schedulers.
+__host__ __device__ constexpr int qslot(int i) { return 32 * (i >> 4) + (i & 15); }
+__host__ __device__ constexpr int kslot(int i) { return 32 * (i >> 4) + 16 + (i & 15); }
+
 // ---- tensor memory columns -----------------------------------------------------------------------
-constexpr uint32_t cWU = 0;        // [W | U~] -> [. | U ; . | O]  (256 columns)
+constexpr uint32_t cWU = 0;        // [W | U~] -> [. | U] (key slots), [. | O] (query slots); 256 columns
 constexpr uint32_t cGA = 0;        // fp16 row-scaled rows (A operand of the off-diagonal Gram), 64 cols
 constexpr uint32_t cGD = 64;       // off-diagonal Gram (fp32), 96 columns
 constexpr uint32_t cS = 256;       // fp32 state (128 columns)
-constexpr uint32_t cWQ = 384;      // fp16 [-W; Q^] (A operand of the state products), 64 columns
+constexpr uint32_t cWQ = 384;      // fp16 -W (key slots) and Q^ (query slots), A operand of W S, Q^ S
 
 // order of the off-diagonal key rows: tile p' uses rows off(p') .. off(p') + 16 p' - 1
 __host__ __device__ constexpr int gb_off(int pp) { return pp == 1 ? 0 : pp == 2 ? 16 : 48; }
@@ -233,39 +240,20 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 __device__ __forceinline__ void bar_all() { named_bar(1, kThreads); }
 
 // ---------------------------------------------------------------------------------------------
-// The solve: T' = (I + L)^-1 diag(beta) from the fp32 diagonal blocks Ld[p] and the fp16 blocks
-// -L_pm (m < p) in LD.  (1) D_p = (I + L_pp)^-1 by column-oriented forward substitution, one column
-// per lane, written as fp16 into the diagonal blocks of LD and, times beta, of T'.  (2) level by
-// level d = p - q:  T'_pq = D_p sum_{m=q}^{p-1} (-L_pm) T'_mq  as 16 x 16 products; starting from
-// D_q diag(beta_q) yields T' directly.  T' is an SW128 [64][64] tile (the MMA's A operand).
+// The solve: T' = (I + L)^-1 diag(beta), given the diagonal inverses D_p = (I + L_pp)^-1 (fp16, on
+// the diagonal blocks of LD), T'_pp = D_p diag(beta_p) (on those of T') and the fp16 blocks -L_pm
+// (m < p) in LD: level by level d = p - q,  T'_pq = D_p sum_{m=q}^{p-1} (-L_pm) T'_mq  as 16 x 16
+// products; starting from D_q diag(beta_q) yields T' directly.  T' is an SW128 [64][64] tile (the
+// MMA's A operand); its rows are the key slots of a 128-row tile whose query slots are zero.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
     const uint32_t base = smem_u32(sm);
-    const float *Ld = reinterpret_cast<const float *>(sm + kLdf);
-    const float *sbeta = reinterpret_cast<const float *>(sm + kBeta);
     const int g = lane >> 2, t4 = lane & 3;
-    if (warp < 4 && lane < 16) {
-        const int pb = warp, mcol = lane;
-        const float *L = Ld + pb * 16 * 17;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = i == mcol ? 1.f : 0.f;
-#pragma unroll
-        for (int j = 0; j < 15; ++j)
-#pragma unroll
-            for (int i = j + 1; i < 16; ++i) x[i] = fmaf(-L[i * 17 + j], x[j], x[i]);
-        const float bcol = sbeta[16 * pb + mcol];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r = 16 * pb + i, c = 16 * pb + mcol;
-            *reinterpret_cast<__half *>(sm + kLD + sw128(r, c)) = __float2half_rn(x[i]);
-            *reinterpret_cast<__half *>(sm + kT + sw128(r, c)) = __float2half_rn(x[i] * bcol);
-        }
-    } else if (warp >= 4) {   // zero the blocks of T' above the diagonal: (0,1..3), (1,2..3), (2,3)
+    if (warp >= 4 && warp < 8) {   // zero the blocks of T' above the diagonal: (0,1..3), (1,2..3), (2,3)
         for (int e = (warp - 4) * 32 + lane; e < 6 * 16 * 2; e += 128) {
             const int ub = e / 32, rem = e % 32, r = rem >> 1, half = rem & 1;
             const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
-            sts128(base + kT + sw128(16 * pb + r, 16 * qb + 8 * half), make_uint4(0, 0, 0, 0));
+            sts128(base + kT + sw128(32 * pb + 16 + r, 16 * qb + 8 * half), make_uint4(0, 0, 0, 0));
         }
     }
     bar_all();
@@ -277,7 +265,7 @@ __device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
             for (int mb = qb; mb < pb; ++mb) {
                 uint32_t af[4], bf[4];
                 ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * mb, lane));   // -L_pm
-                ldsm_x4_t(bf, ldsm_addr_bt<128>(base + kT, 16 * mb, 16 * qb, lane));  // T'_mq
+                ldsm_x4_t(bf, ldsm_addr_bt<128>(base + kT, 32 * mb + 16, 16 * qb, lane));  // T'_mq
                 mma_f16(acc[0], af, bf[0], bf[1]);
                 mma_f16(acc[1], af, bf[2], bf[3]);
             }
@@ -300,15 +288,14 @@ __device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int cc = 16 * qb + 8 * j + 2 * t4;
-                sts32(base + kT + sw128(16 * pb + g, cc), pack_f16(tq[j][0], tq[j][1]));
-                sts32(base + kT + sw128(16 * pb + g + 8, cc), pack_f16(tq[j][2], tq[j][3]));
+                sts32(base + kT + sw128(32 * pb + 16 + g, cc), pack_f16(tq[j][0], tq[j][1]));
+                sts32(base + kT + sw128(32 * pb + 24 + g, cc), pack_f16(tq[j][2], tq[j][3]));
             }
         }
         bar_all();
     }
 }
 
-template <bool kSelfTest = false>
 __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
     extern __shared__ __align__(1024) unsigned char sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -365,45 +352,49 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     };
     float beta_next = load_beta(0);
 
-    // epilogue mapping: TMEM lane quadrant q = warp % 4 (rows 32q + lane), column half hf = warp / 4
-    const int q4 = warp & 3, hf = warp >> 2, row = 32 * q4 + lane;
+    // epilogue mapping: TMEM lane quadrant q4 = warp % 4 (rows 32 q4 + lane), column quarter
+    // cq = warp / 4 (columns 32 cq .. 32 cq + 31 of a 128-column matrix)
+    const int q4 = warp & 3, cq = warp >> 2, row = 32 * q4 + lane;
     const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
 
     // initial state -> TMEM (fp32) and its fp16 copy (B operand)
     {
         const size_t st_base = ((size_t)n * H + h) * kD * kD;
-        float x[64];
+        float x[32];
         if (p.S_in) {
-            const float4 *sp = reinterpret_cast<const float4 *>(p.S_in + st_base + (size_t)row * kD + 64 * hf);
+            const float4 *sp = reinterpret_cast<const float4 *>(p.S_in + st_base + (size_t)row * kD + 32 * cq);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 8; ++j) {
                 const float4 v = __ldg(sp + j);
                 x[4 * j] = v.x; x[4 * j + 1] = v.y; x[4 * j + 2] = v.z; x[4 * j + 3] = v.w;
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) x[j] = 0.f;
+            for (int j = 0; j < 32; ++j) x[j] = 0.f;
         }
 #pragma unroll
-        for (int part = 0; part < 4; ++part) {
+        for (int part = 0; part < 2; ++part) {
             uint32_t v[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(x[16 * part + e]);
-            tmem_st16(tq + cS + 64 * hf + 16 * part, v);
+            tmem_st16(tq + cS + 32 * cq + 16 * part, v);
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            sts128(base + kS + bmn_off(row, 64 * hf + 8 * j),
+        for (int j = 0; j < 4; ++j)
+            sts128(base + kS + bmn_off(row, 32 * cq + 8 * j),
                    make_uint4(pack_f16(x[8 * j], x[8 * j + 1]), pack_f16(x[8 * j + 2], x[8 * j + 3]),
                               pack_f16(x[8 * j + 4], x[8 * j + 5]), pack_f16(x[8 * j + 6], x[8 * j + 7])));
         tmem_wait_st();
     }
 
     uint32_t mma_phase = 0;
-    auto mma_wait = [&]() {   // every thread waits for the latest commit (bounded)
-        const bool ok = wait_bounded(bMma, mma_phase, p.wait_ns);
+    auto mma_wait = [&]() {   // the issuing thread waits for the latest commit (bounded); the CTA
+                              // barrier that follows every call releases the others
+        if (leader && !wait_bounded(bMma, mma_phase, p.wait_ns)) {
+            atomicOr(&g_kda_error_word, kErrTimeout);
+            *abort_flag = 1;
+        }
         mma_phase ^= 1;
-        if (!ok) { atomicOr(&g_kda_error_word, kErrTimeout); *abort_flag = 1; }
     };
     auto mma_sync = [&]() {   // ... then a CTA barrier, after which the flag is read by everyone
         mma_wait();
@@ -421,6 +412,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         tc_fence_before();
         bar_all();
         tc_fence_after();
+    };
+    // 32 consecutive fp32 TMEM columns of this thread's lane
+    auto tld32 = [&](uint32_t taddr, uint32_t (&v)[32]) {
+        uint32_t a[16], b[16];
+        tmem_ld16(taddr, a);
+        tmem_ld16(taddr + 16, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) { v[e] = a[e]; v[16 + e] = b[e]; }
+    };
+    // 32 fp32 values as fp16 into row k of an MN-major B operand (columns 32 cq ..)
+    auto store_b32 = [&](uint32_t region, int k, const uint32_t (&v)[32], float sgn) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            sts128(region + bmn_off(k, 32 * cq + 8 * j),
+                   make_uint4(pack_f16(sgn * __uint_as_float(v[8 * j]), sgn * __uint_as_float(v[8 * j + 1])),
+                              pack_f16(sgn * __uint_as_float(v[8 * j + 2]), sgn * __uint_as_float(v[8 * j + 3])),
+                              pack_f16(sgn * __uint_as_float(v[8 * j + 4]), sgn * __uint_as_float(v[8 * j + 5])),
+                              pack_f16(sgn * __uint_as_float(v[8 * j + 6]), sgn * __uint_as_float(v[8 * j + 7]))));
     };
 
     for (int c = 0; c < nchunks; ++c) {
@@ -441,49 +451,57 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         in_wait(aBar, (c >> 1) & 1);
 
         // ---- 1. pass 1: g, within-tile running sums, tile totals ---------------------------------
+        //      thread = channel pair cp (channels 2cp, 2cp + 1) x half tile part (8 tokens)
         {
-            const int cp = tid & 63, pt = tid >> 6, c0 = 2 * cp;
-            float lx[16], ly[16];
+            const int cp = tid & 63, part = tid >> 6, pt = part >> 1, c0 = 2 * cp;
+            float lx[8], ly[8];
             float sx = 0.f, sy = 0.f;
             constexpr float kG2 = kGMin * kLog2e;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = 16 * pt + i;
+            for (int i = 0; i < 8; ++i) {
+                const int t = 8 * part + i;
                 const float2 av = unpack_bf16(lds32(aBuf + in_off(t, c0)));
                 float gx = kG2 * sigmoid_fast(expA * av.x), gy = kG2 * sigmoid_fast(expA * av.y);
                 if (t >= L) gx = gy = 0.f;
                 sx += gx; sy += gy;
                 lx[i] = sx; ly[i] = sy;
             }
-            float *tot = reinterpret_cast<float *>(sm + kTot);
-            *reinterpret_cast<float2 *>(tot + pt * 128 + c0) = make_float2(sx, sy);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = 16 * pt + i;
-                *reinterpret_cast<float2 *>(sm + kL + l_off(t, c0)) = make_float2(lx[i], ly[i]);
-            }
+            float *tot = reinterpret_cast<float *>(sm + kTot);   // [8 half tiles][128]
+            *reinterpret_cast<float2 *>(tot + part * 128 + c0) = make_float2(sx, sy);
             bar_all();
-            float2 tv[4];
+            // within-tile running sum: the second half adds the first half's total
+            const float2 off = (part & 1) ? *reinterpret_cast<const float2 *>(tot + (part - 1) * 128 + c0) : make_float2(0.f, 0.f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) tv[q] = *reinterpret_cast<const float2 *>(tot + q * 128 + c0);
-            float2 R = make_float2(0.f, 0.f), BC = R;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (q < pt) { R.x += tv[q].x; R.y += tv[q].y; }
-                BC.x += tv[q].x; BC.y += tv[q].y;
+            for (int i = 0; i < 8; ++i) {
+                const int t = 8 * part + i;
+                *reinterpret_cast<float2 *>(sm + kL + l_off(t, c0)) = make_float2(lx[i] + off.x, ly[i] + off.y);
             }
-            *reinterpret_cast<float2 *>(sm + kTE + (pt * 128 + c0) * 4) = make_float2(ex2(R.x), ex2(R.y));
-            *reinterpret_cast<float2 *>(sm + kTK + (pt * 128 + c0) * 4) = make_float2(ex2(BC.x - R.x), ex2(BC.y - R.y));
-            float2 Rn = R;
+            if ((part & 1) == 0) {   // tables of tile pt, once per channel pair
+                float2 T4[4];
 #pragma unroll
-            for (int pp = 1; pp < 4; ++pp) {
-                if (pp <= pt) continue;
-                Rn.x += tv[pp - 1].x; Rn.y += tv[pp - 1].y;
-                if (pp - 1 >= pt)
+                for (int q = 0; q < 4; ++q) {
+                    const float2 x0 = *reinterpret_cast<const float2 *>(tot + (2 * q) * 128 + c0);
+                    const float2 x1 = *reinterpret_cast<const float2 *>(tot + (2 * q + 1) * 128 + c0);
+                    T4[q] = make_float2(x0.x + x1.x, x0.y + x1.y);
+                }
+                float2 R = make_float2(0.f, 0.f), BC = R;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (q < pt) { R.x += T4[q].x; R.y += T4[q].y; }
+                    BC.x += T4[q].x; BC.y += T4[q].y;
+                }
+                *reinterpret_cast<float2 *>(sm + kTE + (pt * 128 + c0) * 4) = make_float2(ex2(R.x), ex2(R.y));
+                *reinterpret_cast<float2 *>(sm + kTK + (pt * 128 + c0) * 4) = make_float2(ex2(BC.x - R.x), ex2(BC.y - R.y));
+                float2 Rn = R;
+#pragma unroll
+                for (int pp = 1; pp < 4; ++pp) {
+                    if (pp <= pt) continue;
+                    Rn.x += T4[pp - 1].x; Rn.y += T4[pp - 1].y;
                     *reinterpret_cast<float2 *>(sm + kTD + (td_index(pt, pp) * 128 + c0) * 4) =
                         make_float2(ex2(Rn.x - R.x), ex2(Rn.y - R.y));
+                }
+                if (pt == 0) *reinterpret_cast<float2 *>(sm + kGam + c0 * 4) = make_float2(ex2(BC.x), ex2(BC.y));
             }
-            if (pt == 0) *reinterpret_cast<float2 *>(sm + kGam + c0 * 4) = make_float2(ex2(BC.x), ex2(BC.y));
         }
         in_wait(bQ, c & 1);
         in_wait(bKV, c & 1);
@@ -491,23 +509,26 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (*abort_flag) break;
 
         // ---- 2. pass 2: operands and the diagonal Gram blocks -------------------------------------
+        //      warp = tile pt x channel quarter cq; lane (g, t4) = rows g, g + 8 of the tile and the
+        //      channels 32 cq + 16 s + 4 t4 .. + 3 (s = 0, 1), the layout of the MMA fragments
         float qk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         float kk[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        const int pt = warp & 3, ch = warp >> 2;         // tile, channel half
+        const int pt = warp & 3;                        // tile (= TMEM lane quadrant of this warp)
         const int g = lane >> 2, t4 = lane & 3;
         {
             const int i0 = 16 * pt + g, i1 = i0 + 8;
-            const bool in0 = i0 < L, in1 = i1 < L;
-#pragma unroll 1
-            for (int s = 0; s < 4; ++s) {
-                const int cb = 64 * ch + 16 * s + 4 * t4;     // this lane's 4 channels cb .. cb + 3
-                // inputs (bf16 x 4 per row), l (fp32 x 4 per row), tables
-                const uint32_t oq0 = in_off(i0, cb), oq1 = in_off(i1, cb);
+            const bool in0 = i0 < L, in1 = i1 < L, partial = L < kChunk;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const int cb = 32 * cq + 16 * s + 4 * t4;     // this lane's 4 channels cb .. cb + 3
+                // rows i0 and i1 = i0 + 8 share their low three bits: row i1 is 8 rows (1 KB of a
+                // swizzled input tile, 4 KB of the l table) after row i0
+                const uint32_t oq0 = in_off(i0, cb), oq1 = oq0 + 1024;
                 uint2 qr0 = lds64(base + kQ + oq0), qr1 = lds64(base + kQ + oq1);
                 uint2 kr0 = lds64(base + kK + oq0), kr1 = lds64(base + kK + oq1);
-                uint2 vr0 = lds64(base + kV + oq0), vr1 = lds64(base + kV + oq1);
-                const float4 l0 = *reinterpret_cast<const float4 *>(sm + kL + l_off(i0, cb));
-                const float4 l1 = *reinterpret_cast<const float4 *>(sm + kL + l_off(i1, cb));
+                const uint32_t ol0 = l_off(i0, cb);
+                const float4 l0 = *reinterpret_cast<const float4 *>(sm + kL + ol0);
+                const float4 l1 = *reinterpret_cast<const float4 *>(sm + kL + ol0 + 4096);
                 const float4 te = *reinterpret_cast<const float4 *>(sm + kTE + (pt * 128 + cb) * 4);
                 const float4 tk = *reinterpret_cast<const float4 *>(sm + kTK + (pt * 128 + cb) * 4);
                 float qv[2][4], kv[2][4], lv[2][4];
@@ -521,8 +542,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                     lv[0][0] = l0.x; lv[0][1] = l0.y; lv[0][2] = l0.z; lv[0][3] = l0.w;
                     lv[1][0] = l1.x; lv[1][1] = l1.y; lv[1][2] = l1.z; lv[1][3] = l1.w;
                 }
-                if (!in0) { qv[0][0] = qv[0][1] = qv[0][2] = qv[0][3] = 0.f; kv[0][0] = kv[0][1] = kv[0][2] = kv[0][3] = 0.f; vr0 = make_uint2(0, 0); }
-                if (!in1) { qv[1][0] = qv[1][1] = qv[1][2] = qv[1][3] = 0.f; kv[1][0] = kv[1][1] = kv[1][2] = kv[1][3] = 0.f; vr1 = make_uint2(0, 0); }
+                if (partial) {   // rows past the sequence's end are zero (warp-uniform branch)
+                    if (!in0) { qv[0][0] = qv[0][1] = qv[0][2] = qv[0][3] = 0.f; kv[0][0] = kv[0][1] = kv[0][2] = kv[0][3] = 0.f; }
+                    if (!in1) { qv[1][0] = qv[1][1] = qv[1][2] = qv[1][3] = 0.f; kv[1][0] = kv[1][1] = kv[1][2] = kv[1][3] = 0.f; }
+                }
                 const float tev[4] = {te.x, te.y, te.z, te.w}, tkv[4] = {tk.x, tk.y, tk.z, tk.w};
                 float qr[2][4], kr[2][4], kt[2][4];   // row-scaled q, k (<= 1) and rescaled keys (>= 1)
 #pragma unroll
@@ -547,9 +570,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                     mma_tf32(kk[1], ak0, ak1, ak2, ak3, b10, b11);
                 }
                 // fp16 row-scaled q, k rows -> TMEM (Gram A operand; rows of tile pt: q at lanes 32pt..+15,
-                // k at 32pt + 16..+31; columns = channel pairs)
+                // k at 32pt + 16..+31; column = channel pair)
                 {
-                    const uint32_t col = tmem + cGA + (uint32_t)(32 * ch + 8 * s);
+                    const uint32_t col = tmem + cGA + (uint32_t)(16 * cq + 8 * s);
                     tmem_st_frag(col + ((uint32_t)(32 * pt) << 16), pack_f16(qr[0][0], qr[0][1]), pack_f16(qr[0][2], qr[0][3]),
                                  pack_f16(qr[1][0], qr[1][1]), pack_f16(qr[1][2], qr[1][3]));
                     tmem_st_frag(col + ((uint32_t)(32 * pt + 16) << 16), pack_f16(kr[0][0], kr[0][1]), pack_f16(kr[0][2], kr[0][3]),
@@ -568,37 +591,65 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                         sts64(base + o, pack_f16(kt[r][0] * tdv[0], kt[r][1] * tdv[1]), pack_f16(kt[r][2] * tdv[2], kt[r][3] * tdv[3]));
                     }
                 }
-                // in place: Q^ = q^ e^{r_p}, K^ = k^ e^{r_p}, V -> fp16; K- = K~ e^{b_C - r_p} into the a buffer
-                sts64(base + kQ + oq0, pack_f16(qr[0][0] * tev[0], qr[0][1] * tev[1]), pack_f16(qr[0][2] * tev[2], qr[0][3] * tev[3]));
-                sts64(base + kQ + oq1, pack_f16(qr[1][0] * tev[0], qr[1][1] * tev[1]), pack_f16(qr[1][2] * tev[2], qr[1][3] * tev[3]));
+                // Q^ = q^ e^{r_p} (above, into TMEM); in place: K^ = k^ e^{r_p}, V -> fp16; K- = K~ e^{b_C - r_p}
+                // into the a buffer
+                tmem_st_frag(tmem + cWQ + (uint32_t)(16 * cq + 8 * s) + ((uint32_t)(32 * pt) << 16),
+                             pack_f16(qr[0][0] * tev[0], qr[0][1] * tev[1]), pack_f16(qr[0][2] * tev[2], qr[0][3] * tev[3]),
+                             pack_f16(qr[1][0] * tev[0], qr[1][1] * tev[1]), pack_f16(qr[1][2] * tev[2], qr[1][3] * tev[3]));
                 sts64(base + kK + oq0, pack_f16(kr[0][0] * tev[0], kr[0][1] * tev[1]), pack_f16(kr[0][2] * tev[2], kr[0][3] * tev[3]));
                 sts64(base + kK + oq1, pack_f16(kr[1][0] * tev[0], kr[1][1] * tev[1]), pack_f16(kr[1][2] * tev[2], kr[1][3] * tev[3]));
                 sts64(aBuf + oq0, pack_f16(kt[0][0] * tkv[0], kt[0][1] * tkv[1]), pack_f16(kt[0][2] * tkv[2], kt[0][3] * tkv[3]));
                 sts64(aBuf + oq1, pack_f16(kt[1][0] * tkv[0], kt[1][1] * tkv[1]), pack_f16(kt[1][2] * tkv[2], kt[1][3] * tkv[3]));
-                sts64(base + kV + oq0, bf16x2_to_f16x2(vr0.x), bf16x2_to_f16x2(vr0.y));
-                sts64(base + kV + oq1, bf16x2_to_f16x2(vr1.x), bf16x2_to_f16x2(vr1.y));
+                // V -> fp16 (rows past the end -> 0), by the warps of the last tile for all four tiles: they
+                // have no rescaled keys to write for later tiles, so this evens out the schedulers' work
+                if (pt == 3) {
+#pragma unroll
+                    for (int tb = 0; tb < 4; ++tb) {
+                        const uint32_t ov = oq0 - 3 * 2048 + tb * 2048;   // rows 16 tb + g and + 8
+                        uint2 v0 = lds64(base + kV + ov), v1 = lds64(base + kV + ov + 1024);
+                        if (partial) {
+                            if (16 * tb + g >= L) v0 = make_uint2(0, 0);
+                            if (16 * tb + g + 8 >= L) v1 = make_uint2(0, 0);
+                        }
+                        sts64(base + kV + ov, bf16x2_to_f16x2(v0.x), bf16x2_to_f16x2(v0.y));
+                        sts64(base + kV + ov + 1024, bf16x2_to_f16x2(v1.x), bf16x2_to_f16x2(v1.y));
+                    }
+                }
             }
         }
-        // rescaled keys of the off-diagonal rows beyond what pass 2 wrote: none (every row is written)
-        // combine the two channel halves' diagonal partial sums in the warps of half 0
+        // the four channel quarters' diagonal partial sums, added in a fixed order (cq 2, 3 -> 0, 1;
+        // then 1 -> 0) through 16 KB of the solve's scratch
         {
-            float *xch = reinterpret_cast<float *>(sm + kLD) + pt * 512;
-            if (ch == 1) {
+            float *xch = reinterpret_cast<float *>(sm + kLD);   // [2][4 tiles][16][32]
+            auto put = [&](int slot) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    xch[e * 32 + lane] = qk[e >> 2][e & 3];
-                    xch[(8 + e) * 32 + lane] = kk[e >> 2][e & 3];
+                    xch[((slot * 4 + pt) * 16 + e) * 32 + lane] = qk[e >> 2][e & 3];
+                    xch[((slot * 4 + pt) * 16 + 8 + e) * 32 + lane] = kk[e >> 2][e & 3];
                 }
-            }
+            };
+            auto add = [&](int slot) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    qk[e >> 2][e & 3] += xch[((slot * 4 + pt) * 16 + e) * 32 + lane];
+                    kk[e >> 2][e & 3] += xch[((slot * 4 + pt) * 16 + 8 + e) * 32 + lane];
+                }
+            };
+            if (cq >= 2) put(cq - 2);
             sync_tc();
             if (*abort_flag) break;
-            if (ch == 0) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    qk[e >> 2][e & 3] += xch[e * 32 + lane];
-                    kk[e >> 2][e & 3] += xch[(8 + e) * 32 + lane];
-                }
+            // every thread is past pass 2: the q buffer is free for the next chunk's q
+            if (leader && c + 1 < nchunks) {
+                fence_async_smem();
+                expect_tx(bQ, 16384);
+                load_pair(&maps.q, base + kQ, bQ, c + 1);
+                issued(0, (c + 1) & 1);
             }
+            if (cq < 2) add(cq);
+            bar_all();
+            if (cq == 1) put(0);
+            bar_all();
+            if (cq == 0) add(0);
         }
 
         // ---- 3. off-diagonal Gram (TMEM A rows x rescaled keys) ----------------------------------
@@ -612,30 +663,44 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
-        // meanwhile: S <- Gamma_C S (fp32, in TMEM); Q^ -> TMEM rows 64-127 of [-W; Q^]
+        // meanwhile: the diagonal blocks of L (fp32) and their inverses D_p = (I + L_pp)^-1, by
+        // column-oriented forward substitution, one column per lane of warp pt (kept in registers
+        // until the Gram MMA has released the tiles they are written to);
+        // S <- Gamma_C S (fp32, in TMEM)
+        float dinv[16];
+        if (cq == 0) {
+            const float *sb = reinterpret_cast<const float *>(sm + kBeta);
+            float *Ldp = reinterpret_cast<float *>(sm + kLdf) + pt * 16 * 17;
+            const float bi0 = sb[16 * pt + g], bi1 = sb[16 * pt + g + 8];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int j = 8 * nt + 2 * t4, r0 = g, r1 = g + 8;
+                Ldp[r0 * 17 + j] = j < r0 ? bi0 * kk[nt][0] : 0.f;
+                Ldp[r0 * 17 + j + 1] = j + 1 < r0 ? bi0 * kk[nt][1] : 0.f;
+                Ldp[r1 * 17 + j] = j < r1 ? bi1 * kk[nt][2] : 0.f;
+                Ldp[r1 * 17 + j + 1] = j + 1 < r1 ? bi1 * kk[nt][3] : 0.f;
+            }
+            __syncwarp();
+            const int mcol = lane & 15;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dinv[i] = i == mcol ? 1.f : 0.f;
+#pragma unroll
+            for (int j = 0; j < 15; ++j)
+#pragma unroll
+                for (int i = j + 1; i < 16; ++i) dinv[i] = fmaf(-Ldp[i * 17 + j], dinv[j], dinv[i]);
+        }
         {
             const float gam = reinterpret_cast<const float *>(sm + kGam)[row];
+            uint32_t v[32];
+            tld32(tq + cS + 32 * cq, v);
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
-                uint32_t v[16];
-                tmem_ld16(tq + cS + 64 * hf + 16 * part, v);
-                tmem_wait_ld();
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gam * __uint_as_float(v[e]));
+            {
+                uint32_t a[16], b[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(gam * __uint_as_float(v[e]));
-                tmem_st16(tq + cS + 64 * hf + 16 * part, v);
-            }
-            if (q4 >= 2) {
-                const int i = row - 64;   // token row of Q^
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    uint32_t v[16];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint4 x = lds128(base + kQ + in_off(i, 64 * hf + 32 * part + 8 * j));
-                        v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
-                    }
-                    tmem_st16(tq + cWQ + 32 * hf + 16 * part, v);
-                }
+                for (int e = 0; e < 16; ++e) { a[e] = v[e]; b[e] = v[16 + e]; }
+                tmem_st16(tq + cS + 32 * cq, a);
+                tmem_st16(tq + cS + 32 * cq + 16, b);
             }
         }
         mma_wait();
@@ -644,35 +709,31 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         bar_all();
         tc_fence_after();
         if (*abort_flag) break;
-        // q buffer is free: the next chunk's q
-        if (leader && c + 1 < nchunks) {
-            fence_async_smem();
-            expect_tx(bQ, 16384);
-            load_pair(&maps.q, base + kQ, bQ, c + 1);
-            issued(0, (c + 1) & 1);
+        if (cq == 0 && lane < 16) {   // D_p and T'_pp = D_p diag(beta_p) into their tiles
+            const float bcol = reinterpret_cast<const float *>(sm + kBeta)[16 * pt + lane];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * pt + i, cc = 16 * pt + lane;
+                *reinterpret_cast<__half *>(sm + kLD + sw128(r, cc)) = __float2half_rn(dinv[i]);
+                *reinterpret_cast<__half *>(sm + kT + sw128(kslot(r), cc)) = __float2half_rn(dinv[i] * bcol);
+            }
         }
 
         // ---- 4. solve inputs: A rows (tile pt) and -L rows from the Gram, diagonal blocks ----------
         {
             const float *sb = reinterpret_cast<const float *>(sm + kBeta);
-            if (ch == 0) {
-                // diagonal blocks from the fragments: A (j <= i) and L (j < i, times beta_i)
-                float *Ldp = reinterpret_cast<float *>(sm + kLdf) + pt * 16 * 17;
-                const float bi0 = sb[16 * pt + g], bi1 = sb[16 * pt + g + 8];
+            if (cq == 0) {
+                // diagonal blocks of A from the fragments (j <= i)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int j = 8 * nt + 2 * t4;   // column within the tile
                     const int r0 = g, r1 = g + 8;
-                    sts32(base + kAm + sw128(16 * pt + r0, 16 * pt + j),
+                    sts32(base + kAm + sw128(32 * pt + r0, 16 * pt + j),
                           pack_f16(j <= r0 ? qk[nt][0] : 0.f, j + 1 <= r0 ? qk[nt][1] : 0.f));
-                    sts32(base + kAm + sw128(16 * pt + r1, 16 * pt + j),
+                    sts32(base + kAm + sw128(32 * pt + r1, 16 * pt + j),
                           pack_f16(j <= r1 ? qk[nt][2] : 0.f, j + 1 <= r1 ? qk[nt][3] : 0.f));
-                    Ldp[r0 * 17 + j] = j < r0 ? bi0 * kk[nt][0] : 0.f;
-                    Ldp[r0 * 17 + j + 1] = j + 1 < r0 ? bi0 * kk[nt][1] : 0.f;
-                    Ldp[r1 * 17 + j] = j < r1 ? bi1 * kk[nt][2] : 0.f;
-                    Ldp[r1 * 17 + j + 1] = j + 1 < r1 ? bi1 * kk[nt][3] : 0.f;
                 }
-            } else {
+            } else if (cq == 1) {
                 // off-diagonal rows from TMEM: lanes 32pt + r (q rows) and 32pt + 16 + r (k rows)
                 const int r = lane & 15;
                 const bool krow = lane >= 16;
@@ -685,28 +746,30 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         uint4 o;
-                        const float s = krow ? -bi : 1.f;
-                        o.x = pack_f16(s * __uint_as_float(v[8 * hh + 0]), s * __uint_as_float(v[8 * hh + 1]));
-                        o.y = pack_f16(s * __uint_as_float(v[8 * hh + 2]), s * __uint_as_float(v[8 * hh + 3]));
-                        o.z = pack_f16(s * __uint_as_float(v[8 * hh + 4]), s * __uint_as_float(v[8 * hh + 5]));
-                        o.w = pack_f16(s * __uint_as_float(v[8 * hh + 6]), s * __uint_as_float(v[8 * hh + 7]));
-                        sts128(base + (krow ? kLD : kAm) + sw128(i, 16 * blk + 8 * hh), o);
+                        const float sg = krow ? -bi : 1.f;
+                        o.x = pack_f16(sg * __uint_as_float(v[8 * hh + 0]), sg * __uint_as_float(v[8 * hh + 1]));
+                        o.y = pack_f16(sg * __uint_as_float(v[8 * hh + 2]), sg * __uint_as_float(v[8 * hh + 3]));
+                        o.z = pack_f16(sg * __uint_as_float(v[8 * hh + 4]), sg * __uint_as_float(v[8 * hh + 5]));
+                        o.w = pack_f16(sg * __uint_as_float(v[8 * hh + 6]), sg * __uint_as_float(v[8 * hh + 7]));
+                        sts128(krow ? base + kLD + sw128(i, 16 * blk + 8 * hh) : base + kAm + sw128(qslot(i), 16 * blk + 8 * hh), o);
                     }
                 }
                 if (!krow) {   // A: zeros right of the diagonal block
-                    for (int cc = 16 * (pt + 1); cc < 64; cc += 8) sts128(base + kAm + sw128(i, cc), make_uint4(0, 0, 0, 0));
+                    for (int cc = 16 * (pt + 1); cc < 64; cc += 8) sts128(base + kAm + sw128(qslot(i), cc), make_uint4(0, 0, 0, 0));
                 }
             }
         }
-        // the zero block between T' and A shares its bytes with the rescaled keys of pass 2: clear it
-        for (int e = tid; e < 8192 / 16; e += kThreads) sts128(base + kZ + 16 * e, make_uint4(0, 0, 0, 0));
+        // the query slots of T'' are zero (their bytes held rescaled keys in pass 2)
+        {
+            const int e = tid;   // 512 chunks of 16 bytes: 4 tiles x 16 rows x 8 chunks
+            sts128(base + kT + (32 * (e >> 7) + ((e >> 3) & 15)) * 128 + 16 * (e & 7), make_uint4(0, 0, 0, 0));
+        }
         bar_all();
         solve(sm, warp, lane);
         sync_tc();   // T' visible to the tensor core
 
         // ---- 5. [W | U~] = [T'; 0] [K^ | V] ---------------------------------------------------------
         if (wq0) {
-            fence_async_smem();
             if (leader) {
                 constexpr uint32_t id = idesc(128, 256, 0, 1);
 #pragma unroll
@@ -727,19 +790,16 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             issued(1, (c + 1) & 1);
         }
         // ---- 6. -W -> TMEM rows 0-63 of [-W; Q^] ----------------------------------------------------
-        if (q4 < 2) {
+        {
+            uint32_t v[32], w[16];
+            tld32(tq + cWU + 32 * cq, v);
+            tmem_ld16(tq + cWQ + 16 * cq, w);
+            tmem_wait_ld();
+            if (lane >= 16) {   // key slot: -W;  query slot: Q^ stays
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
-                uint32_t v[16];
-                tmem_ld16(tq + cWU + 64 * hf + 16 * part, v);
-                tmem_wait_ld();
-                uint32_t w[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) w[e] = pack_f16(-__uint_as_float(v[2 * e]), -__uint_as_float(v[2 * e + 1]));
-                asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(tq + cWQ + 32 * hf + 8 * part),
-                             "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-                             : "memory");
+                for (int e = 0; e < 16; ++e) w[e] = pack_f16(-__uint_as_float(v[2 * e]), -__uint_as_float(v[2 * e + 1]));
             }
+            tmem_st16(tq + cWQ + 16 * cq, w);
         }
         sync_tc();
         // ---- 7. D[:, 128:256] += [-W; Q^] S --------------------------------------------------------
@@ -756,23 +816,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         mma_sync();
         if (*abort_flag) break;
         // ---- 8. U (rows 0-63) -> shared memory (fp16, MN-major B operand) ---------------------------
-        if (q4 < 2) {
-#pragma unroll
-            for (int part = 0; part < 4; ++part) {
-                uint32_t v[16];
-                tmem_ld16(tq + cWU + 128 + 64 * hf + 16 * part, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    sts128(base + kL + bmn_off(row, 64 * hf + 16 * part + 8 * j),
-                           make_uint4(pack_f16(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                                      pack_f16(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                                      pack_f16(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                                      pack_f16(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]))));
-            }
+        {
+            uint32_t v[32];
+            tld32(tq + cWU + 128 + 32 * cq, v);
+            if (lane >= 16) store_b32(base + kL, 16 * q4 + (lane - 16), v, 1.f);
         }
         sync_tc();
-        // ---- 9. S += K-^T U;  D[:, 128:256] += [0; A] U -------------------------------------------
+        // ---- 9. S += K-^T U;  D[:, 128:256] += A'' U  (the query slots become O) ---------------------
         if (wq0) {
             if (leader) {
                 constexpr uint32_t id = idesc(128, 128, 1, 1), id2 = idesc(128, 128, 0, 1);
@@ -781,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                     mma_ss(tmem + cS, sdesc(aBuf + 2048 * k, 8192, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_ss(tmem + cWU + 128, sdesc(base + kZ + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);
+                    mma_ss(tmem + cWU + 128, sdesc(base + kAm + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);
                 umma_commit(bMma);
             }
             __syncwarp();
@@ -792,58 +842,35 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (*abort_flag) break;
         // ---- 10. new S (fp16 copy); gated output rows -----------------------------------------------
         {
-#pragma unroll
-            for (int part = 0; part < 4; ++part) {
-                uint32_t v[16];
-                tmem_ld16(tq + cS + 64 * hf + 16 * part, v);
+            uint32_t v[32];
+            tld32(tq + cS + 32 * cq, v);
+            store_b32(base + kS, row, v, 1.f);
+            // query slots of quadrant q4: tokens 16 q4 + g and + 8 (lane (g, t4)), columns 32 cq + 8b + 2t4, + 1
+            {
+                uint32_t o16[16];
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+                    : "=r"(o16[0]), "=r"(o16[1]), "=r"(o16[2]), "=r"(o16[3]), "=r"(o16[4]), "=r"(o16[5]), "=r"(o16[6]), "=r"(o16[7]),
+                      "=r"(o16[8]), "=r"(o16[9]), "=r"(o16[10]), "=r"(o16[11]), "=r"(o16[12]), "=r"(o16[13]), "=r"(o16[14]), "=r"(o16[15])
+                    : "r"(tq + cWU + 128 + 32 * cq));
                 tmem_wait_ld();
+                const int gg = lane >> 2, tt = lane & 3;
 #pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    sts128(base + kS + bmn_off(row, 64 * hf + 16 * part + 8 * j),
-                           make_uint4(pack_f16(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
-                                      pack_f16(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
-                                      pack_f16(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
-                                      pack_f16(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]))));
-            }
-            if (q4 >= 2) {
-                const int i = row - 64;
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int i = 16 * q4 + gg + 8 * rr;
 #pragma unroll
-                for (int part = 0; part < 4; ++part) {
-                    uint32_t v[16];
-                    tmem_ld16(tq + cWU + 128 + 64 * hf + 16 * part, v);
-                    tmem_wait_ld();
-                    float o[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) o[e] = __uint_as_float(v[e]);
-                    const int cb = 64 * hf + 16 * part;
-                    if (p.has_gate) {
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const uint4 gr = lds128(base + kG + in_off(i, cb + 8 * j));
-                            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 ga = unpack_bf16(gw[e]);
-                                o[8 * j + 2 * e] *= sigmoid_fast(ga.x);
-                                o[8 * j + 2 * e + 1] *= sigmoid_fast(ga.y);
-                            }
+                    for (int b = 0; b < 4; ++b) {
+                        const int cc = 32 * cq + 8 * b + 2 * tt;
+                        float o0 = __uint_as_float(o16[4 * b + 2 * rr]), o1 = __uint_as_float(o16[4 * b + 2 * rr + 1]);
+                        if (p.has_gate) {
+                            const float2 ga = unpack_bf16(lds32(base + kG + in_off(i, cc)));
+                            o0 *= sigmoid_fast(ga.x);
+                            o1 *= sigmoid_fast(ga.y);
                         }
-                    }
-                    if (p.out_f32) {   // staging fp32 [64][128], 16-byte chunks XOR-swizzled by row
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int chk = (cb >> 2) + j;
-                            sts128(base + kL + i * 512 + ((chk ^ (i & 7)) << 4),
-                                   make_uint4(__float_as_uint(o[4 * j]), __float_as_uint(o[4 * j + 1]), __float_as_uint(o[4 * j + 2]),
-                                              __float_as_uint(o[4 * j + 3])));
-                        }
-                    } else {           // staging bf16 [64][128]
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const int chk = (cb >> 3) + j;
-                            sts128(base + kL + i * 256 + ((chk ^ (i & 7)) << 4),
-                                   make_uint4(pack_bf16(o[8 * j], o[8 * j + 1]), pack_bf16(o[8 * j + 2], o[8 * j + 3]),
-                                              pack_bf16(o[8 * j + 4], o[8 * j + 5]), pack_bf16(o[8 * j + 6], o[8 * j + 7])));
+                        if (p.out_f32) {   // staging fp32 [64][128], 16-byte chunks XOR-swizzled by row
+                            sts64(base + kL + i * 512 + ((((cc >> 2) ^ (i & 7))) << 4) + (cc & 3) * 4, __float_as_uint(o0), __float_as_uint(o1));
+                        } else {           // staging bf16 [64][128]
+                            sts32(base + kL + i * 256 + ((((cc >> 3) ^ (i & 7))) << 4) + (cc & 7) * 2, pack_bf16(o0, o1));
                         }
                     }
                 }
@@ -891,17 +918,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     // final state (fp32, from TMEM)
     if (p.S_out && !*abort_flag) {
         const size_t st_base = ((size_t)n * H + h) * kD * kD;
-        float4 *sp = reinterpret_cast<float4 *>(p.S_out + st_base + (size_t)row * kD + 64 * hf);
+        float4 *sp = reinterpret_cast<float4 *>(p.S_out + st_base + (size_t)row * kD + 32 * cq);
+        uint32_t v[32];
+        tld32(tq + cS + 32 * cq, v);
 #pragma unroll
-        for (int part = 0; part < 4; ++part) {
-            uint32_t v[16];
-            tmem_ld16(tq + cS + 64 * hf + 16 * part, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                sp[4 * part + j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
-                                               __uint_as_float(v[4 * j + 3]));
-        }
+        for (int j = 0; j < 8; ++j)
+            sp[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
+                                __uint_as_float(v[4 * j + 3]));
     }
     tc_fence_before();
     __syncthreads();
