@@ -3,13 +3,15 @@
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
-One step = one kda_chunk_fwd call over the prefill workload (B=1, H=32, T=8192, d=128; inputs
-resident in HBM).  The decode row (kda_decode_step over 256 sequences x 64 heads, 128x128 fp32
-states, 512 steps) is timed in the same run and reported under "decode", and rounds of speculative
-decode (kda_decode_verify of 4 proposed tokens + kda_decode_commit of the accepted prefix, same
-states) under "speculative".  Every rank runs its own
-independent batch (weak scaling, no collective on the data path); timing is on the device with
-CUDA events, max over ranks.  Rank 0 prints one JSON line.
+One step = one kda_chunk_fwd call over the packed variable-length prefill workload (64 sequences
+of U{512..32768} tokens, H=64, d=128: about 1.07 M tokens, 105 GB of inputs and outputs resident in
+HBM) -- the largest of the prefill workloads that fit one GPU.  Extra rows time the B=1, H=32,
+T=8192 prefill and the 1 M-token prefill; the backward and module rows run on the T=8192 workload;
+the decode row (kda_decode_step over 256 sequences x 64 heads, 128x128 fp32 states, 512 steps) and
+rounds of speculative decode (kda_decode_verify of 4 proposed tokens + kda_decode_commit of the
+accepted prefix, same states) are timed in the same run.  Every rank runs its own independent batch
+(weak scaling, no collective on the data path); timing is on the device with CUDA events, max over
+ranks.  Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this build) on the host cores.
 """
@@ -57,7 +59,11 @@ def parse_args():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="kda", choices=["kda", "reference"])
-    p.add_argument("--workload", default="prefill_B1_H32_T8192_d128")
+    p.add_argument("--workload", default="varlen_64seq_U512_32768_H64_d128")
+    p.add_argument("--extra-workloads", default="prefill_B1_H32_T8192_d128,long_B1_H32_T1048576_d128")
+    p.add_argument("--aux-workload", default="prefill_B1_H32_T8192_d128",
+                   help="workload of the backward and module rows")
+    p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--decode-steps", type=int, default=512)
     p.add_argument("--spec-rounds", type=int, default=64)
     p.add_argument("--no-decode", action="store_true")
@@ -116,7 +122,7 @@ def peaks():
 # source files each kernel is built from (a DRAM traffic figure is reported only while they are
 # unchanged since the ncu capture it came from)
 KERNEL_SOURCES = {
-    "prefill": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh"),
+    "prefill": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh", "prefill_tc.cuh"),
     "decode": ("common.cuh", "decode.cuh"),
     "speculative": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "f32x2.cuh", "speculative.cuh"),
     "backward": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "backward.cuh"),
@@ -219,9 +225,9 @@ class ClockSampler:
 def host_inputs_f64(inp, heads):
     import numpy as np
     h = lambda t: None if t is None else t[:, heads].detach().cpu().double().numpy()
-    S0 = inp["initial_state"]
+    S0 = inp.get("initial_state")
     return dict(q=h(inp["q"]), k=h(inp["k"]), v=h(inp["v"]), a=h(inp["a"]), beta=h(inp["beta"]),
-                gate=h(inp["gate"]), A_log=inp["A_log"][heads].cpu().double().numpy(),
+                gate=h(inp.get("gate")), A_log=inp["A_log"][heads].cpu().double().numpy(),
                 cu=inp["cu_seqlens"].cpu().numpy().astype(np.int64),
                 S0=None if S0 is None else S0[:, heads].cpu().double().numpy())
 
@@ -243,18 +249,47 @@ def oracle_sample(inp, w, target_s: float, threads: int):
     return list(range(heads)), per_head
 
 
-def cpu_baseline(inp, w, target_s=15.0):
+def sub_batch(inp, w, max_tokens: int):
+    """The first sequences of a packed batch, up to about max_tokens tokens (at least one), on the host."""
+    import numpy as np
+    import torch
+    cu = inp["cu_seqlens"].cpu().numpy().astype(np.int64)
+    n = 1
+    while n < w.num_seqs and cu[n + 1] <= max_tokens:
+        n += 1
+    T = int(cu[n])
+    sub = {k: (v[:T].cpu() if k in ("q", "k", "v", "a", "beta", "gate") and v is not None else v)
+           for k, v in inp.items()}
+    sub["cu_seqlens"] = torch.from_numpy(cu[: n + 1].astype(np.int32))
+    sub["initial_state"] = None if inp["initial_state"] is None else inp["initial_state"][:n].cpu()
+    sub["A_log"] = inp["A_log"].cpu()
+    return sub, w.replace(seqlens=tuple(int(x) for x in np.diff(cu[: n + 1])))
+
+
+def cpu_baseline(inp, w, target_s=15.0, max_tokens=65536):
+    """The fp64 oracle on the host cores over a bounded sample of the workload: its first sequences
+    (up to max_tokens tokens) and as many heads as take about target_s on all cores; plus the same
+    oracle single-threaded on one head of one sequence."""
     threads = len(os.sched_getaffinity(0))
-    heads, _ = oracle_sample(inp, w, target_s, threads)
-    x = host_inputs_f64(inp, heads)
-    used = min(threads, len(heads) * w.num_seqs)
+    sub, sw = sub_batch(inp, w, max_tokens)
+    heads, _ = oracle_sample(sub, sw, target_s, threads)
+    x = host_inputs_f64(sub, heads)
+    used = min(threads, len(heads) * sw.num_seqs)
     t0 = time.perf_counter()
     oracle_step(x, used)
     dt = time.perf_counter() - t0
-    tokens = w.total_tokens * len(heads) / w.H
+    tokens = sw.total_tokens * len(heads) / w.H
+    one, ow = sub_batch(inp, w, 1)
+    x1 = host_inputs_f64(one, [0])
+    t1 = time.perf_counter()
+    oracle_step(x1, 1)
+    dt1 = time.perf_counter() - t1
     return {"value": tokens / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
-            "sample": f"{len(heads)} of {w.H} heads x all {w.total_tokens} tokens of {w.name} "
-                      f"(fp64 token-by-token recurrence, {dt:.2f} s wall)"}
+            "single_thread": {"value": ow.total_tokens / w.H / dt1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"1 head x {ow.total_tokens} tokens (one sequence), {dt1:.2f} s"},
+            "sample": f"{len(heads)} of {w.H} heads x the first {sw.num_seqs} sequences ({sw.total_tokens} tokens) "
+                      f"of {w.name} (fp64 token-by-token recurrence, {dt:.2f} s wall); tokens/s counts whole "
+                      f"tokens of all {w.H} heads"}
 
 
 def run_reference(args):
@@ -265,21 +300,22 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = KI.WORKLOADS[args.workload]
-    inp = KI.make_inputs(w, "cpu")
+    small = w.replace(seqlens=w.seqlens[:2]) if w.num_seqs > 2 else w
+    inp, sw = sub_batch(KI.make_inputs(small, "cpu"), small, 32768)
     threads = len(os.sched_getaffinity(0))
-    heads, per_head = oracle_sample(inp, w, target_s=2.0, threads=threads)
+    heads, per_head = oracle_sample(inp, sw, target_s=1.0, threads=threads)
     x = host_inputs_f64(inp, heads)
-    used = min(threads, len(heads) * w.num_seqs)
+    used = min(threads, len(heads) * sw.num_seqs)
     for _ in range(args.warmup):
         oracle_step(x, used)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         oracle_step(x, used)
     dt = (time.perf_counter() - t0) / args.steps
-    tokens = w.total_tokens * len(heads) / w.H
+    tokens = sw.total_tokens * len(heads) / w.H
     value = tokens / dt
-    sample = (f"{len(heads)} of {w.H} heads x all {w.total_tokens} tokens of {w.name} per step "
-              f"(fp64 oracle; throughput scaled to whole tokens of all heads)")
+    sample = (f"{len(heads)} of {w.H} heads x the first {sw.num_seqs} sequences ({sw.total_tokens} tokens) "
+              f"of {w.name} per step (fp64 oracle; throughput counts whole tokens of all heads)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
@@ -296,6 +332,26 @@ def run_reference(args):
 
 
 # ---- the CUDA arm ------------------------------------------------------------------------------
+
+def time_calls(fn, steps: int, warmup: int, stream, world, dev, barrier, clocks=None):
+    """Milliseconds per call of fn (CUDA events on `stream`, after warm-up), max over ranks."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.active(True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.active(False)
+    barrier()
+    return max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+
 
 def main():
     args = parse_args()
@@ -322,133 +378,185 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    w = rank_workload(KI.WORKLOADS[args.workload], rank)
-    inp = KI.make_inputs(w, dev)
-    max_seqlen = max(w.seqlens)
-    ws_bytes = kda.kda_chunk_fwd_workspace_size(w.total_tokens, w.num_seqs, max_seqlen, w.H,
-                                                w.d_k, w.d_v)
-    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    out = torch.empty((w.total_tokens, w.H, w.d_v), dtype=torch.bfloat16, device=dev)
-    S_final = torch.empty((w.num_seqs, w.H, w.d_k, w.d_v), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-
-    def step():
-        kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"],
-                          inp["cu_seqlens"], gate=inp["gate"], initial_state=inp["initial_state"],
-                          out=out, final_state=S_final, max_seqlen=max_seqlen,
-                          workspace=workspace, stream=stream)
-
-    clocks = ClockSampler(dev)
-    for _ in range(args.warmup):
-        step()
-    kda.kda_sync_check()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = kda.kda_launch_count()
-    clocks.active(True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    clocks.active(False)
-    launches = kda.kda_launch_count() - launches0
-    barrier()
-    kda.kda_sync_check()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
-    value = whole_job_rate(w.total_tokens, world, ms)
-
     hbm, tf, tf_sus, peak_src = peaks()
-    bytes_step = prefill_bytes(w)
-    flops_step = prefill_flops(w)
-    achieved = bytes_step / (ms * 1e-3) / 1e9
-    src_hash = kernel_source_hash()
-    traffic_val = ncu_traffic(w.name, "prefill")
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": traffic_val,
+
+    def prefill_setup(w):
+        inp = KI.make_inputs(w, dev)
+        max_seqlen = max(w.seqlens)
+        ws_bytes = kda.kda_chunk_fwd_workspace_size(w.total_tokens, w.num_seqs, max_seqlen, w.H, w.d_k, w.d_v)
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        out = torch.empty((w.total_tokens, w.H, w.d_v), dtype=torch.bfloat16, device=dev)
+        S_final = torch.empty((w.num_seqs, w.H, w.d_k, w.d_v), dtype=torch.float32, device=dev)
+
+        def step():
+            kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"],
+                              inp["cu_seqlens"], gate=inp["gate"], initial_state=inp["initial_state"],
+                              out=out, final_state=S_final, max_seqlen=max_seqlen,
+                              workspace=workspace, stream=stream)
+        return inp, out, S_final, step
+
+    def prefill_roofline(w, ms, traffic_key):
+        bytes_step, flops_step = prefill_bytes(w), prefill_flops(w)
+        achieved = bytes_step / (ms * 1e-3) / 1e9
+        traffic = ncu_traffic(traffic_key, "prefill") if traffic_key else None
+        return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic,
+                "traffic_source": (f"dram__bytes_read.sum + dram__bytes_write.sum of an earlier ncu capture "
+                                   f"(profiles/), scaled to this workload; reported while the kernel sources "
+                                   f"are unchanged since" if traffic is not None else
+                                   "no current ncu capture of these kernel sources"),
                 "peak_source": f"hbm_gbs of {peak_src}",
                 "scope": "one kda_chunk_fwd call (all kernels of the prefill path)",
                 "algorithmic_bytes": bytes_step, "algorithmic_flops": flops_step,
                 "tensor_frac_of_bf16_peak": flops_step / (ms * 1e-3) / 1e12 / tf}
 
-    # backward row: kda_chunk_bwd on the prefill workload (gradients of every input)
+    # ---- headline: the packed variable-length prefill ----
+    w = rank_workload(KI.WORKLOADS[args.workload], rank)
+    inp, out, S_final, step = prefill_setup(w)
+    clocks = ClockSampler(dev)
+    for _ in range(args.warmup):
+        step()
+    kda.kda_sync_check()
+    launches0 = kda.kda_launch_count()
+    ms = time_calls(step, args.steps, 0, stream, world, dev, barrier, clocks)
+    launches = kda.kda_launch_count() - launches0
+    kda.kda_sync_check()
+    value = whole_job_rate(w.total_tokens, world, ms)
+    bytes_step = prefill_bytes(w)
+    roofline = prefill_roofline(w, ms, w.name)
+    path = kda.kda_prefill_path(w.num_seqs * w.H, w.d_k, w.d_v)
+    src_hash = kernel_source_hash()
+
+    # ---- end to end through the public API: kda_chunk_fwd_host on page-locked host tensors (the
+    #      copies to and from the device, piece by piece, overlapped with the prefill) ----
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k", "v", "a", "beta", "gate", "A_log", "cu_seqlens", "initial_state"]
+        host_in = {}
+        for n in names:   # straight into page-locked buffers (no pageable intermediate copy)
+            if inp[n] is not None:
+                host_in[n] = torch.empty(inp[n].shape, dtype=inp[n].dtype, pin_memory=True)
+                host_in[n].copy_(inp[n])
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        S_h = torch.empty(S_final.shape, dtype=S_final.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = out_h.numel() * out_h.element_size() + S_h.numel() * S_h.element_size()
+        del inp, out, S_final, step
+        torch.cuda.empty_cache()
+        hbuf = torch.empty(kda.kda_chunk_fwd_host_buffer_size(host_in["cu_seqlens"], w.H, w.d_k, w.d_v, torch.bfloat16),
+                           dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            kda.kda_chunk_fwd_host(host_in["q"], host_in["k"], host_in["v"], host_in["a"], host_in["beta"],
+                                   host_in["A_log"], host_in["cu_seqlens"], gate=host_in.get("gate"),
+                                   initial_state=host_in.get("initial_state"), out=out_h, final_state=S_h,
+                                   device_buffer=hbuf, stream=stream)
+
+        ems = time_calls(e2e_step, args.e2e_steps, 1, stream, world, dev, barrier)
+        kda.kda_sync_check()
+        e2e = {"value": whole_job_rate(w.total_tokens, world, ems), "unit": "tokens/s",
+               "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": args.e2e_steps, "workload": w.name,
+               "api": "kda_chunk_fwd_host (2048-token pieces; copies in, prefill, copies out on three streams)"}
+        cpu_src = {k: v for k, v in host_in.items()}
+        del hbuf, out_h, S_h
+        torch.cuda.empty_cache()
+    else:
+        cpu_src = inp
+        del out, S_final, step
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cpu_src, w)
+    del cpu_src
+    if not args.no_e2e:
+        del host_in
+    else:
+        del inp
+    torch.cuda.empty_cache()
+
+    # ---- extra prefill rows ----
+    extra = []
+    for name in [x for x in args.extra_workloads.split(",") if x]:
+        xw = rank_workload(KI.WORKLOADS[name], rank)
+        xinp, xout, xS, xstep = prefill_setup(xw)
+        xsteps = 3 if xw.total_tokens * xw.H > 8_000_000 else args.steps
+        xms = time_calls(xstep, xsteps, max(3, min(args.warmup, 3)), stream, world, dev, barrier, clocks)
+        kda.kda_sync_check()
+        extra.append({"workload": xw.name, "value": whole_job_rate(xw.total_tokens, world, xms), "unit": "tokens/s",
+                      "ms_per_step": xms, "steps": xsteps,
+                      "kernel": "per-unit" if kda.kda_prefill_path(xw.num_seqs * xw.H, xw.d_k, xw.d_v) == 2 else "cluster",
+                      "roofline": prefill_roofline(xw, xms, xw.name)})
+        del xinp, xout, xS, xstep
+        torch.cuda.empty_cache()
+
+    aw = rank_workload(KI.WORKLOADS[args.aux_workload], rank)
+    ainp = KI.make_inputs(aw, dev)
+    aout = torch.empty((aw.total_tokens, aw.H, aw.d_v), dtype=torch.bfloat16, device=dev)
+
+    # backward row: kda_chunk_bwd on the aux workload (gradients of every input)
     backward = None
     if not args.no_decode:
         gb = torch.Generator(device=dev).manual_seed(201 + rank)
-        dout = torch.randn((w.total_tokens, w.H, w.d_v), generator=gb, device=dev) * 0.1
-        dST = torch.randn((w.num_seqs, w.H, w.d_k, w.d_v), generator=gb, device=dev) * 0.1
-        bws = torch.empty(kda.kda_chunk_bwd_workspace_size(w.total_tokens, w.num_seqs, w.H, w.d_k, w.d_v),
+        dout = torch.randn((aw.total_tokens, aw.H, aw.d_v), generator=gb, device=dev) * 0.1
+        dST = torch.randn((aw.num_seqs, aw.H, aw.d_k, aw.d_v), generator=gb, device=dev) * 0.1
+        bws = torch.empty(kda.kda_chunk_bwd_workspace_size(aw.total_tokens, aw.num_seqs, aw.H, aw.d_k, aw.d_v),
                           dtype=torch.uint8, device=dev)
 
         def bstep():
-            return kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"],
-                                     inp["cu_seqlens"], dout, gate=inp["gate"], initial_state=inp["initial_state"],
+            return kda.kda_chunk_bwd(ainp["q"], ainp["k"], ainp["v"], ainp["a"], ainp["beta"], ainp["A_log"],
+                                     ainp["cu_seqlens"], dout, gate=ainp["gate"], initial_state=ainp["initial_state"],
                                      dfinal_state=dST, workspace=bws, stream=stream)
 
-        bstep()
-        barrier()
-        reps = 3
-        e0.record(stream)
-        for _ in range(reps):
-            bstep()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
+        bms = time_calls(bstep, 3, 1, stream, world, dev, barrier)
         kda.kda_sync_check()
-        bms = max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
-        th = w.total_tokens * w.H
+        th = aw.total_tokens * aw.H
         # inputs (as the forward) + dout (fp32) read; dq, dk, da, dv, dgate (fp32), dbeta written;
         # initial state and its gradient, final-state gradient
-        bbytes = th * (2 * (3 * w.d_k + 2 * w.d_v) + 4 + 4 * w.d_v + 4 * (3 * w.d_k + 2 * w.d_v) + 4) + \
-            3 * w.num_seqs * w.H * w.d_k * w.d_v * 4
+        bbytes = th * (2 * (3 * aw.d_k + 2 * aw.d_v) + 4 + 4 * aw.d_v + 4 * (3 * aw.d_k + 2 * aw.d_v) + 4) + \
+            3 * aw.num_seqs * aw.H * aw.d_k * aw.d_v * 4
         bach = bbytes / (bms * 1e-3) / 1e9
-        backward = {"value": whole_job_rate(w.total_tokens, world, bms), "unit": "tokens/s", "ms_per_step": bms,
-                    "workload": w.name, "scope": "one kda_chunk_bwd call",
+        backward = {"value": whole_job_rate(aw.total_tokens, world, bms), "unit": "tokens/s", "ms_per_step": bms,
+                    "workload": aw.name, "scope": "one kda_chunk_bwd call",
                     "roofline": {"bound": "latency (sequential token steps per unit)", "achieved": bach,
                                  "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
-                                 "traffic": ncu_traffic("bwd_" + w.name, "backward"),
+                                 "traffic": ncu_traffic("bwd_" + aw.name, "backward"),
                                  "peak_source": f"hbm_gbs of {peak_src}", "algorithmic_bytes": bbytes}}
         del dout, dST, bws
         torch.cuda.empty_cache()
 
     # module row: the short convolution of q, k, v (q, k L2-normalised) and the pre-gate
-    # normalisation + gate of one fp32 output, on the prefill workload's tensors
+    # normalisation + gate of one fp32 output, on the aux workload's tensors
     module = None
     if not args.no_decode:
         gm = torch.Generator(device=dev).manual_seed(101 + rank)
-        cw = torch.randn((w.H, w.d_k, 4), generator=gm, device=dev) * 0.5
-        nw = torch.rand((w.d_v,), generator=gm, device=dev) + 0.5
-        o32 = torch.randn((w.total_tokens, w.H, w.d_v), generator=gm, device=dev)
-        yq, yk, yv = (torch.empty_like(inp[key]) for key in ("q", "k", "v"))
+        cw = torch.randn((aw.H, aw.d_k, 4), generator=gm, device=dev) * 0.5
+        nw = torch.rand((aw.d_v,), generator=gm, device=dev) + 0.5
+        o32 = torch.randn((aw.total_tokens, aw.H, aw.d_v), generator=gm, device=dev)
+        yq, yk, yv = (torch.empty_like(ainp[key]) for key in ("q", "k", "v"))
 
         def mstep():
-            kda.kda_short_conv(inp["q"], cw, inp["cu_seqlens"], l2norm=True, out=yq, stream=stream)
-            kda.kda_short_conv(inp["k"], cw, inp["cu_seqlens"], l2norm=True, out=yk, stream=stream)
-            kda.kda_short_conv(inp["v"], cw, inp["cu_seqlens"], l2norm=False, out=yv, stream=stream)
-            kda.kda_output_norm_gate(o32, inp["gate"], nw, out=out, stream=stream)
+            kda.kda_short_conv(ainp["q"], cw, ainp["cu_seqlens"], l2norm=True, out=yq, stream=stream)
+            kda.kda_short_conv(ainp["k"], cw, ainp["cu_seqlens"], l2norm=True, out=yk, stream=stream)
+            kda.kda_short_conv(ainp["v"], cw, ainp["cu_seqlens"], l2norm=False, out=yv, stream=stream)
+            kda.kda_output_norm_gate(o32, ainp["gate"], nw, out=aout, stream=stream)
 
-        for _ in range(max(3, args.warmup)):
-            mstep()
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            mstep()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
+        mms = time_calls(mstep, args.steps, max(3, args.warmup), stream, world, dev, barrier)
         kda.kda_sync_check()
-        mms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
-        th = w.total_tokens * w.H
-        mbytes = 3 * 2 * th * w.d_k * 2 + th * w.d_v * (4 + 2 + 2)   # conv read + write x3; o, gate, out
+        th = aw.total_tokens * aw.H
+        mbytes = 3 * 2 * th * aw.d_k * 2 + th * aw.d_v * (4 + 2 + 2)   # conv read + write x3; o, gate, out
         mach = mbytes / (mms * 1e-3) / 1e9
-        module = {"value": whole_job_rate(w.total_tokens, world, mms), "unit": "tokens/s", "ms_per_step": mms,
-                  "workload": w.name, "scope": "3 kda_short_conv (width 4) + 1 kda_output_norm_gate",
+        module = {"value": whole_job_rate(aw.total_tokens, world, mms), "unit": "tokens/s", "ms_per_step": mms,
+                  "workload": aw.name, "scope": "3 kda_short_conv (width 4) + 1 kda_output_norm_gate",
                   "roofline": {"bound": "hbm", "achieved": mach, "peak": hbm, "unit": "GB/s",
                                "frac": mach / hbm, "traffic": None, "peak_source": f"hbm_gbs of {peak_src}",
                                "algorithmic_bytes": mbytes}}
         del o32, yq, yk, yv
-        torch.cuda.empty_cache()
+    del ainp, aout
+    torch.cuda.empty_cache()
 
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # decode row: 512 back-to-back steps over fixed states (each step reads and writes 1.07 GB)
     decode = None
     if not args.no_decode:
@@ -529,59 +637,23 @@ def main():
         del d, state, sout, su
         torch.cuda.empty_cache()
 
-    # end to end through the public API: kda_chunk_fwd_host on page-locked host tensors (the copies
-    # to and from the device, piece by piece, overlapped with the prefill)
-    e2e = None
-    if not args.no_e2e:
-        names = ["q", "k", "v", "a", "beta", "gate", "A_log", "cu_seqlens", "initial_state"]
-        host_in = {n: inp[n].cpu().pin_memory() for n in names if inp[n] is not None}
-        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        S_h = torch.empty(S_final.shape, dtype=S_final.dtype, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-        d2h = out_h.numel() * out_h.element_size() + S_h.numel() * S_h.element_size()
-        hbuf = torch.empty(kda.kda_chunk_fwd_host_buffer_size(host_in["cu_seqlens"], w.H, w.d_k, w.d_v, out.dtype),
-                           dtype=torch.uint8, device=dev)
-
-        def e2e_step():
-            kda.kda_chunk_fwd_host(host_in["q"], host_in["k"], host_in["v"], host_in["a"], host_in["beta"],
-                                   host_in["A_log"], host_in["cu_seqlens"], gate=host_in.get("gate"),
-                                   initial_state=host_in.get("initial_state"), out=out_h, final_state=S_h,
-                                   device_buffer=hbuf, stream=stream)
-
-        for _ in range(args.warmup):
-            e2e_step()
-        barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
-        e2e = {"value": whole_job_rate(w.total_tokens, world, ems), "unit": "tokens/s",
-               "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "kda_chunk_fwd_host (2048-token pieces; copies in, prefill, copies out on three streams)"}
-        del hbuf
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(inp, w)
-
     clk = clocks.summary()
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            # tensor-core operands are bf16 (Gram blocks, split hi + lo for Q K^T) and fp16 (value
-            # path); accumulation, the decay arithmetic and the carried state are fp32
-            "dtype": "bf16/fp16 mma, f32 accumulate",
+            # tensor-core operands: tf32 (diagonal Gram blocks), fp16 (off-diagonal Gram blocks and
+            # the value path); accumulation, the decay arithmetic and the carried state are fp32
+            "dtype": "tf32/fp16 mma, f32 accumulate",
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.num_seqs, "H": w.H, "T": w.total_tokens,
                        "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "tile": 16,
+                       "kernel": "per-unit" if path == 2 else "cluster",
                        "parallelism": f"independent batch per rank x{world}",
                        "l2": f"inputs larger than L2 ({bytes_step / 1e6:.0f} MB per step > 126 MB); no flush"},
-            "roofline": roofline, "backward": backward, "module": module, "decode": decode, "speculative": spec, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roofline, "prefill_rows": extra, "backward": backward, "module": module, "decode": decode,
+            "speculative": spec, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": launches, "clocks": clk, "kernel_src": src_hash,
         }
         print(json.dumps(line))

@@ -51,7 +51,9 @@ typedef enum kda_status {
     KDA_ERR_INVALID_ARG = 1, /* NULL required pointer, bad size, misaligned pointer, small workspace */
     KDA_ERR_UNSUPPORTED = 2, /* d_k or d_v outside {64, 128} */
     KDA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
-    KDA_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (reported by kda_sync_check) */
+    KDA_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (reported by kda_sync_check) */
+    KDA_ERR_RANGE = 5        /* a prefill state ended non-finite: an fp16 tensor-core operand
+                                (value, state, pseudo-value) left +-65504 (reported by kda_sync_check) */
 } kda_status;
 
 /* Storage type of the output o.  The recurrence itself is computed in fp32 either way. */
@@ -79,9 +81,18 @@ typedef enum kda_dtype {
  * max_seqlen: an upper bound on every sequence length, or 0 for none.  A sequence longer than a
  *   non-zero bound is reported through the error word (the result is still computed in full).
  * scale multiplies q.  workspace: device scratch of at least kda_chunk_fwd_workspace_min(...)
- *   bytes (equal to kda_chunk_fwd_workspace_size(...)), 256-byte aligned; it holds per-unit rings
- *   of chunk records (about 0.57 MiB per (sequence, head) at d = 128); its contents need no
- *   initialisation and it may be reused across calls on one stream.
+ *   bytes (equal to kda_chunk_fwd_workspace_size(...)), 256-byte aligned, or NULL when that size is
+ *   0; its contents need no initialisation and it may be reused across calls on one stream.
+ * Two kernels compute the same chunkwise form (kda_set_prefill_path below):
+ *   - with d_k = d_v = 128 and at least a third as many (sequence, head) units as the GPU has SMs,
+ *     one CTA per unit keeps every chunk intermediate on chip and needs no workspace (size 0);
+ *   - otherwise a unit's chunks are spread over d_v / 32 CTAs of a cluster, handing chunk records
+ *     to each other through per-unit rings in the workspace (about 0.57 MiB per unit at d = 128).
+ * Numerics: the decay arithmetic, the accumulation and the carried state are fp32; the tensor-core
+ *   operands are tf32 (the 16-token diagonal Gram blocks) and fp16 (everything else).  Values,
+ *   states and the chunk pseudo-values must therefore stay within +-65504 (unit-norm q and k and
+ *   O(1) values are far inside); a call that leaves that range ends with a non-finite state, which
+ *   kda_sync_check reports as KDA_ERR_RANGE.
  * A zero-length sequence copies its initial state (or zeros) to final_state.
  * total_tokens == 0 or num_seqs == 0 is valid and only writes final_state.
  */
@@ -103,11 +114,13 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, co
  * This entry point takes the same arguments as kda_chunk_fwd minus the workspace and instead uses
  * scratch memory built into the library: a 32 MiB device array that every GPU which loads
  * libkda holds until the process exits.  It calls no cudaMalloc or cudaFree.
- *   - The first call on a device looks up that array's device address (with that device current)
- *     and caches it; make that first call before any stream capture.
+ *   - Every call looks up that array's device address (with the calling thread's current device);
+ *     the first call on a device loads the library's device code there, so make it before any
+ *     stream capture.
  *   - Sizes whose scratch need (kda_chunk_fwd_workspace_min) exceeds 32 MiB are rejected with
- *     KDA_ERR_INVALID_ARG and a message in kda_last_error.  With d_k = d_v = 128 that allows
- *     56 (sequence, head) units per call, of any length.
+ *     KDA_ERR_INVALID_ARG and a message in kda_last_error.  With d_k = d_v = 128 the kernel chosen
+ *     by shape needs either no scratch (many units) or at most 49 units' rings (28 MiB), so no
+ *     such call is rejected; forcing the cluster kernel (kda_set_prefill_path(1)) allows 56 units.
  *   - Every call on a device shares the one array and nothing in it needs to start at zero, but
  *     calls that overlap on the GPU (different streams, or other threads) race on it: serialise
  *     them, for example by issuing them all on one stream.

@@ -39,7 +39,7 @@ __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
-KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_RANGE = range(6)
 KDA_DTYPE_BF16, KDA_DTYPE_F32 = 0, 1
 _OUT_DTYPES = {torch.bfloat16: KDA_DTYPE_BF16, torch.float32: KDA_DTYPE_F32}
 

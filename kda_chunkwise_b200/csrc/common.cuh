@@ -19,6 +19,8 @@ constexpr int kTilesPerChunk = kChunk / kTile;
 constexpr unsigned kErrBadSeqlens = 1u;   // cu_seqlens not monotone / not ending at total_tokens
 constexpr unsigned kErrSeqTooLong = 2u;   // a sequence longer than the max_seqlen given
 constexpr unsigned kErrTimeout = 4u;      // a bounded wait gave up
+constexpr unsigned kErrRange = 16u;       // a prefill state ended non-finite: some fp16 tensor-core
+                                          //   operand (state, pseudo-values, values) left +-65504
 
 __device__ __forceinline__ int64_t min64(int64_t x, int64_t y) { return x < y ? x : y; }
 

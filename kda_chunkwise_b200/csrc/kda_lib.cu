@@ -242,8 +242,6 @@ kda_status launch_bwd(const kda::BwdParams &p, int64_t units, cudaStream_t strea
 // cudaGetSymbolAddress, looked up once per device below.
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
 
 }  // namespace
 
@@ -257,14 +255,12 @@ kda_status static_scratch_address(void **ptr) {
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices)
         return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_noalloc: device ordinal out of range");
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_kda_static_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetSymbolAddress");
-        g_scratch_ptr[dev] = p;
-    }
-    *ptr = g_scratch_ptr[dev];
+    // Looked up on every call (it allocates nothing and is cheap), so a device reset or a new context
+    // on the device never leaves a stale address behind.
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_kda_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc: cudaGetSymbolAddress");
+    *ptr = p;
     return KDA_OK;
 }
 
@@ -279,6 +275,7 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_UNSUPPORTED: return "unsupported configuration";
         case KDA_ERR_CUDA: return "CUDA error";
         case KDA_ERR_TIMEOUT: return "device-side wait timed out";
+        case KDA_ERR_RANGE: return "value outside the fp16 operand range";
     }
     return "unknown status";
 }
@@ -728,6 +725,9 @@ kda_status kda_sync_check(void *stream) {
         return fail(KDA_ERR_INVALID_ARG, "a sequence is longer than max_seqlen");
     if (word & kda::kErrBadAccepted)
         return fail(KDA_ERR_INVALID_ARG, "an accepted count is outside [0, K] (it was clamped)");
+    if (word & kda::kErrRange)
+        return fail(KDA_ERR_RANGE, "a prefill state ended non-finite: a value, state or pseudo-value left the "
+                                   "+-65504 range of the fp16 tensor-core operands; outputs and final states are not valid");
     return KDA_OK;
 }
 

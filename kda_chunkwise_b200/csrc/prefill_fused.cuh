@@ -837,6 +837,14 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
 #pragma unroll
         for (int j = 0; j < 4; ++j) sp[j] = make_float4(S[4 * j], S[4 * j + 1], S[4 * j + 2], S[4 * j + 3]);
     }
+    // An fp16 operand that overflowed (state, pseudo-values, values beyond +-65504) becomes inf and
+    // reaches the fp32 state, where no fade can remove it: a non-finite final state flags the unit.
+    if (has_s) {
+        bool bad = false;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) bad |= !isfinite(S[j]);
+        if (bad) atomicOr(&g_kda_error_word, kErrRange);
+    }
 }
 
 template <int DK, int DV>

@@ -915,16 +915,24 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             if (pend >> i & 1) wait_bounded(bQ + 8 * i, pend_par >> i & 1, p.wait_ns);
         wait_bounded(bMma, mma_phase ^ 1, p.wait_ns);
     }
-    // final state (fp32, from TMEM)
-    if (p.S_out && !*abort_flag) {
-        const size_t st_base = ((size_t)n * H + h) * kD * kD;
-        float4 *sp = reinterpret_cast<float4 *>(p.S_out + st_base + (size_t)row * kD + 32 * cq);
+    // final state (fp32, from TMEM).  An fp16 operand that overflowed (state, pseudo-values, values
+    // beyond +-65504) becomes inf and reaches the fp32 state, where no fade can remove it: a
+    // non-finite final state flags the unit.
+    if (!*abort_flag) {
         uint32_t v[32];
         tld32(tq + cS + 32 * cq, v);
+        bool bad = false;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            sp[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
-                                __uint_as_float(v[4 * j + 3]));
+        for (int j = 0; j < 32; ++j) bad |= !isfinite(__uint_as_float(v[j]));
+        if (bad) atomicOr(&g_kda_error_word, kErrRange);
+        if (p.S_out) {
+            const size_t st_base = ((size_t)n * H + h) * kD * kD;
+            float4 *sp = reinterpret_cast<float4 *>(p.S_out + st_base + (size_t)row * kD + 32 * cq);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                sp[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
+                                    __uint_as_float(v[4 * j + 3]));
+        }
     }
     tc_fence_before();
     __syncthreads();

@@ -37,9 +37,10 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(5):
-        assert kda.kda_status_string(code)
+    for code in range(6):
+        assert kda.kda_status_string(code) != "unknown status"
     assert kda.kda_status_string(0) == "ok"
+    assert kda.kda_status_string(kda.KDA_ERR_RANGE) == "value outside the fp16 operand range"
 
 
 def test_workspace_sizes():

@@ -103,3 +103,25 @@ def test_per_unit_path_is_deterministic(kda):
     a = run(kda, inp, 2)
     b = run(kda, inp, 2)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_state_beyond_fp16_range_is_reported(kda, path):
+    # the state and the values reach the tensor cores as fp16: an initial state of 1e6 (beyond
+    # +-65504) cannot be represented; the call must end with KDA_ERR_RANGE, not with silent infs
+    w = KI.Workload("range", (100, 70), 2, 128, 128, init_state="normal_0.02", seed=14)
+    inp = KI.make_inputs(w, "cuda")
+    S0 = torch.full_like(inp["initial_state"], 1e6)
+    kda.kda_set_prefill_path(path)
+    try:
+        kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
+                          gate=inp["gate"], initial_state=S0)
+        with pytest.raises(kda.KDAError) as ei:
+            kda.kda_sync_check()
+        assert ei.value.status == kda.KDA_ERR_RANGE
+        # the error word is cleared: an in-range call afterwards is clean
+        kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
+                          gate=inp["gate"], initial_state=inp["initial_state"])
+        kda.kda_sync_check()
+    finally:
+        kda.kda_set_prefill_path(0)
