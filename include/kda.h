@@ -87,7 +87,7 @@ typedef enum kda_dtype {
  *   - with d_k = d_v = 128 and at least a third as many (sequence, head) units as the GPU has SMs,
  *     one CTA per unit keeps every chunk intermediate on chip and needs no workspace (size 0);
  *   - otherwise a unit's chunks are spread over d_v / 32 CTAs of a cluster, handing chunk records
- *     to each other through per-unit rings in the workspace (about 0.57 MiB per unit at d = 128).
+ *     to each other through per-unit rings in the workspace (about 0.63 MiB per unit at d = 128).
  * Numerics: the decay arithmetic, the accumulation and the carried state are fp32; the tensor-core
  *   operands are tf32 (the 16-token diagonal Gram blocks) and fp16 (everything else).  Values,
  *   states and the chunk pseudo-values must therefore stay within +-65504 (unit-norm q and k and
@@ -119,8 +119,8 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, co
  *     stream capture.
  *   - Sizes whose scratch need (kda_chunk_fwd_workspace_min) exceeds 32 MiB are rejected with
  *     KDA_ERR_INVALID_ARG and a message in kda_last_error.  With d_k = d_v = 128 the kernel chosen
- *     by shape needs either no scratch (many units) or at most 49 units' rings (28 MiB), so no
- *     such call is rejected; forcing the cluster kernel (kda_set_prefill_path(1)) allows 56 units.
+ *     by shape needs either no scratch (many units) or at most 49 units' rings (31 MiB), so no
+ *     such call is rejected; forcing the cluster kernel (kda_set_prefill_path(1)) allows 50 units.
  *   - Every call on a device shares the one array and nothing in it needs to start at zero, but
  *     calls that overlap on the GPU (different streams, or other threads) race on it: serialise
  *     them, for example by issuing them all on one stream.

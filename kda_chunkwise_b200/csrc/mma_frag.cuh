@@ -35,6 +35,11 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+__device__ __forceinline__ float2 unpack_f16(uint32_t v) {
+    const __half2 h = *reinterpret_cast<const __half2 *>(&v);
+    return __half22float2(h);
+}
+
 // bf16 pair -> fp16 pair (exact for values inside the fp16 range)
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     const float2 f = unpack_bf16(v);

@@ -69,7 +69,8 @@ struct RingLayout {
     static constexpr int kA1 = 0;                 // [W ; Q^]: lanes 0-63 W, 64-127 Q^ (K = d_k)
     static constexpr int kA2 = kA1 + DK / 8 * 128 * 16;  // K-^T: lanes = d_k rows (K = tokens)
     static constexpr int kA3 = kA2 + 8 * DK * 16;        // A: lanes 64-127 = token rows (K = tokens)
-    static constexpr int kU = kA3 + 8 * 64 * 16;  // U~: [slab][half][chunk 2][row 64][8 fp16]
+    static constexpr int kA4 = kA3 + 8 * 64 * 16;        // A - fp16(A), the same image
+    static constexpr int kU = kA4 + 8 * 64 * 16;  // U~: [slab][half][chunk 2][row 64][8 fp16]
     static constexpr int kGam = kU + G * 2 * 2 * 64 * 16;  // Gamma_C fp32 [DK]
     static constexpr int kBytes = ((kGam + DK * 4) + 1023) / 1024 * 1024;
 };
@@ -81,7 +82,8 @@ struct FusedSmem {
     // consumer (B operands of the tensor-core products: 8 x 8 fp16 core matrices, MN-major)
     static constexpr int kB1 = 0;                     // S_c: K = d_k rows, N = 32 columns
     static constexpr int kB2 = kB1 + DK * kSlab * 2;  // U:   K = 64 tokens, N = 32 columns
-    static constexpr int kFull = kB2 + 64 * kSlab * 2;  // u64 mbarrier [R]: chunk published
+    static constexpr int kB3 = kB2 + 64 * kSlab * 2;  // U - fp16(U), the same layout
+    static constexpr int kFull = kB3 + 64 * kSlab * 2;  // u64 mbarrier [R]: chunk published
     static constexpr int kEmpty = kFull + 8 * RL::R;  // u64 mbarrier [R]: chunk consumed (the
                                                       //   producing CTA's copy is the one used)
     static constexpr int kM1 = kEmpty + 8 * RL::R;    // u64 mbarrier: [W; Q^] S complete
@@ -152,10 +154,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity
     return true;
 }
 
-__device__ __forceinline__ float2 unpack_f16(uint32_t v) {
-    const __half2 h = *reinterpret_cast<const __half2 *>(&v);
-    return __half22float2(h);
-}
 
 // ---------------------------------------------------------------------------------------------
 // Producer: chunk-parallel work for chunks rank, rank + G, ... of one unit.
@@ -394,15 +392,25 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
             const int i0 = 16 * pb + g, i1 = i0 + 8;
             const bool diag = pb == qb;
             const float b0 = sbeta[i0], b1 = sbeta[i1];
-            uint32_t afr[4];
+            uint32_t afr[4], alo[4];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 const int jc = 16 * qb + 8 * nt + 2 * t4;
                 float aq[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) aq[e] = ahh[nt][e] + (ahl[nt][e] + alh[nt][e]);
-                afr[2 * nt] = pack_f16(!diag || jc <= i0 ? aq[0] : 0.f, !diag || jc + 1 <= i0 ? aq[1] : 0.f);
-                afr[2 * nt + 1] = pack_f16(!diag || jc <= i1 ? aq[2] : 0.f, !diag || jc + 1 <= i1 ? aq[3] : 0.f);
+                if (diag) {
+                    if (jc > i0) aq[0] = 0.f;
+                    if (jc + 1 > i0) aq[1] = 0.f;
+                    if (jc > i1) aq[2] = 0.f;
+                    if (jc + 1 > i1) aq[3] = 0.f;
+                }
+                // A as fp16 plus its fp16 rounding remainder (the output product uses both)
+                afr[2 * nt] = pack_f16(aq[0], aq[1]);
+                afr[2 * nt + 1] = pack_f16(aq[2], aq[3]);
+                const float2 h0 = unpack_f16(afr[2 * nt]), h1 = unpack_f16(afr[2 * nt + 1]);
+                alo[2 * nt] = pack_f16(aq[0] - h0.x, aq[1] - h0.y);
+                alo[2 * nt + 1] = pack_f16(aq[2] - h1.x, aq[3] - h1.y);
                 if (diag) {   // fp32 diagonal block for the 16x16 inverses
                     const int li = g, lj = 8 * nt + 2 * t4;
                     float *Ld = sLd + pb * 16 * 17;
@@ -421,12 +429,15 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
                 char *const b = slotp + RL::kA3 + ((2 * qb + nt) * 64 + i0) * 16 + t4 * 4;
                 st_u32(b, afr[2 * nt]);
                 st_u32(b + 8 * 16, afr[2 * nt + 1]);
+                st_u32(b + (RL::kA4 - RL::kA3), alo[2 * nt]);
+                st_u32(b + (RL::kA4 - RL::kA3) + 8 * 16, alo[2 * nt + 1]);
             }
         }
         if (warp >= 2) {   // zero blocks above the diagonal (the A image is read whole): one per warp
             const int ub = warp - 2;   // (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
             const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
             stg_v4(slotp + RL::kA3 + ((2 * qb + (lane >> 4)) * 64 + 16 * pb + (lane & 15)) * 16, make_uint4(0, 0, 0, 0));
+            stg_v4(slotp + RL::kA4 + ((2 * qb + (lane >> 4)) * 64 + 16 * pb + (lane & 15)) * 16, make_uint4(0, 0, 0, 0));
         }
         // 4b. K-^T and Q^ to the ring, by warps 2-7 (warps 0 and 1 take two Gram blocks each).
         //     K-^T tile (d_k tile md, token tile kt) as an A fragment: register e of a lane is row
@@ -577,7 +588,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
 // columns 16 half .. + 15; an fp16 copy in shared memory is the B operand):
 //   D  = [W ; Q^] S_c            (M = 128: rows 0-63 W S_c, rows 64-127 Q^ S_c)     TMEM
 //   U  = U~ - D[0:64]  -> shared memory (fp16, B operand)
-//   D3 = K-^T U,   D[64:128] += A U                                                  TMEM
+//   D3 = K-^T U,   D[64:128] += A U   (U and A each as fp16 value + fp16 remainder) TMEM
 //   S_{c+1} = Diag(Gamma_C) S_c + D3;   out = sigmoid(gate) D[64:128]
 // The A operands ([W; Q^], K-^T, A) of chunk c + 1 are fetched from the ring into registers while
 // chunk c's products run and then stored into the other of two TMEM buffers; the ring slot is
@@ -590,15 +601,15 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     using SM = FusedSmem<DK, DV>;
     constexpr int G = RL::G, R = RL::R;
     constexpr int A1C = DK / 2;                        // TMEM columns of one [W; Q^] buffer
-    constexpr uint32_t cD = 0, cD3 = 32, cA1 = 64, cA2 = cA1 + 2 * A1C, cA3 = cA2 + 64;
+    constexpr uint32_t cD = 0, cD3 = 32, cA1 = 64, cA2 = cA1 + 2 * A1C, cA3 = cA2 + 64, cA4 = cA3 + 64;
     constexpr uint32_t kIdesc = umma_idesc_f16(128, kSlab);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3, half = warp >> 2;
     const int row = 32 * q + lane;                     // this thread's TMEM lane
     const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
     const bool has_s = row < DK, has_u = row < 64, has_o = row >= 64;
-    unsigned char *const sB1 = sm + SM::kB1, *const sB2 = sm + SM::kB2;
-    const uint32_t aB1 = smem_u32(sB1), aB2 = smem_u32(sB2);
+    unsigned char *const sB1 = sm + SM::kB1, *const sB2 = sm + SM::kB2, *const sB3 = sm + SM::kB3;
+    const uint32_t aB1 = smem_u32(sB1), aB2 = smem_u32(sB2), aB3 = smem_u32(sB3);
     const uint32_t aFull = smem_u32(sm + SM::kFull), aEmpty = smem_u32(sm + SM::kEmpty);
     const uint32_t aM1 = smem_u32(sm + SM::kM1), aM2 = smem_u32(sm + SM::kM2);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(sm + SM::kCFlag);
@@ -643,6 +654,14 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         const uint32_t v[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
                                 x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
         tmem_st16(taddr, v);
+    };
+    // the remainder A - fp16(A) of chunk cl: straight from the ring into TMEM buffer b (has_o warps)
+    auto copy_a4 = [&](int cl, int b) {
+        const char *sp = slot_of(cl);
+        uint4 x4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x4[j] = ldg_cg_v4(sp + RL::kA4 + ((half * 4 + j) * 64 + row - 64) * 16);
+        st4(tq + cA4 + b * 32 + 16 * half, x4);
     };
     auto put_a = [&](int b, const uint4 (&x1)[NJ], const uint4 (&x2)[4], const uint4 (&x3)[4]) {
 #pragma unroll
@@ -692,6 +711,7 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
         wait_bar(aFull + 8 * 0, 0);
         fetch_a12(0, x1, x2);
         if (has_o) fetch_a3(0, x3);
+        if (has_o) copy_a4(0, 0);
         if (has_u) load_ut(0);
         if (has_s) gam = load_gam(0);
         if (has_o) load_gate(0);
@@ -733,7 +753,7 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             uint32_t d[16];
             tmem_ld16(tq + cD + 16 * half, d);
             tmem_wait_ld();
-            float u[16];
+            float u[16], ulo[16];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const uint32_t w4[4] = {ut[j].x, ut[j].y, ut[j].z, ut[j].w};
@@ -744,10 +764,19 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                     u[8 * j + 2 * e + 1] = t.y - __uint_as_float(d[8 * j + 2 * e + 1]);
                 }
             }
+            // U enters its products as fp16 U plus the fp16 rounding remainder U - fp16(U)
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+                const float2 hf = unpack_f16(pack_f16(u[e], u[e + 1]));
+                ulo[e] = u[e] - hf.x;
+                ulo[e + 1] = u[e + 1] - hf.y;
+            }
             store_b(sB2, row, u);
+            store_b(sB3, row, ulo);
             if (has_next) load_ut(c + 1);
         } else if (has_next) {
             fetch_a3(c + 1, x3);
+            copy_a4(c + 1, buf ^ 1);   // that TMEM buffer's last reader, chunk c - 1, is complete
         }
         fence_async_smem();
         tmem_wait_st();
@@ -762,7 +791,16 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                 umma_f16_ts(tmem + cD3, tmem + cA2 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, k > 0);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
+                umma_f16_ts(tmem + cD3, tmem + cA2 + buf * 32 + 8 * k, umma_desc(aB3 + 1024 * k, 512, 128), kIdesc, 1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
                 umma_f16_ts(tmem + cD, tmem + cA3 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, 1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                umma_f16_ts(tmem + cD, tmem + cA3 + buf * 32 + 8 * k, umma_desc(aB3 + 1024 * k, 512, 128), kIdesc, 1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                umma_f16_ts(tmem + cD, tmem + cA4 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, 1);
             umma_commit(aM2);
         }
         // 5. chunk c+1's A operands into the other TMEM buffer (its last user, chunk c-1, is done)
@@ -851,7 +889,7 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(kFusedThreads, 1) kda_prefill_fused_kernel(const FusedParams p) {
     using SM = FusedSmem<DK, DV>;
     constexpr int G = DV / kSlab;
-    constexpr uint32_t kTmemCols = DK == 128 ? 512 : 256;   // see the column map of the consumer
+    constexpr uint32_t kTmemCols = 512;   // see the column map of the consumer
     extern __shared__ __align__(1024) unsigned char fsmem[];
     const int unit = blockIdx.x / G, rank = blockIdx.x % G;
     const int n = unit / p.H, h = unit % p.H;

@@ -20,8 +20,10 @@
 //   - blocks below the diagonal: both factors are <= 1 and a factor that underflows belongs to a
 //     term below e^-87, so fp16 operands lose nothing: one tcgen05 MMA (M = 128: the row-scaled
 //     q and k rows of the four tiles, N = 96 rescaled keys, K = d_k) computes all of them.
-// Everything on the value path (T', K^, V, W, Q^, K-, A, S, U) is fp16 with fp32 accumulation; the
-// state's master copy is fp32 in tensor memory.
+// Everything on the value path (T', K^, V, W, Q^, K-, A, S, U) is fp16 with fp32 accumulation; U
+// and A, whose rounding shows most in the largest outputs, enter their products as an fp16 value
+// plus its fp16 rounding remainder (about 22 significant bits).  The state's master copy is fp32
+// in tensor memory.
 //
 // Work per chunk (one CTA, 16 warps, the phases separated by CTA barriers):
 //   0. TMA: q, k, v, a, gate rows of the chunk (3-d tensor maps over [T, H, d], two 64-channel boxes
@@ -68,8 +70,11 @@ constexpr int kG = 81920;          // gate
 constexpr int kL = 98304;          // fp32 [64][128] within-tile log2 cumsum l (pass 1 -> pass 2);
                                    //   then U (fp16, 16 KB) and A'' (16 KB); then the output staging
 constexpr int kGB = 131072;        // fp16 rescaled keys of later tiles: K-major, no swizzle, 96 rows
-constexpr int kT = kGB;            // T'' (after the Gram): SW128 [128][64], rows in slot order (below)
-constexpr int kAm = kL + 16384;    // A'' (after pass 2): SW128 [128][64], rows in slot order
+constexpr int kT = kGB;            // T'' (after the Gram): SW128 [128][64], rows in slot order (below);
+                                   //   after [W | U~], the remainder U - fp16(U) (B operand like U)
+constexpr int kUlo = kGB;
+constexpr int kAm = kL + 16384;    // A'' (after pass 2): SW128 [128][64]: fp16 A in the query slots, the
+                                   //   remainder A - fp16(A) in the key slots
 constexpr int kS = 155648;         // fp16 S: B operand, MN-major, no swizzle (K = d_k, N = d_v)
 constexpr int kLD = 188416;        // fp16 [64][64] swizzled: -L below the diagonal blocks, D_p on them;
                                    //   earlier (with kM) the exchange of the diagonal Gram partial sums
@@ -723,15 +728,21 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         {
             const float *sb = reinterpret_cast<const float *>(sm + kBeta);
             if (cq == 0) {
-                // diagonal blocks of A from the fragments (j <= i)
+                // diagonal blocks of A from the fragments (j <= i): fp16 A in the query slots, the
+                // rounding remainder A - fp16(A) (fp16) in the key slots, where the A_lo U product
+                // reads it through an operand that starts 16 rows later
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int j = 8 * nt + 2 * t4;   // column within the tile
-                    const int r0 = g, r1 = g + 8;
-                    sts32(base + kAm + sw128(32 * pt + r0, 16 * pt + j),
-                          pack_f16(j <= r0 ? qk[nt][0] : 0.f, j + 1 <= r0 ? qk[nt][1] : 0.f));
-                    sts32(base + kAm + sw128(32 * pt + r1, 16 * pt + j),
-                          pack_f16(j <= r1 ? qk[nt][2] : 0.f, j + 1 <= r1 ? qk[nt][3] : 0.f));
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int r = g + 8 * hh;
+                        const float x0 = j <= r ? qk[nt][2 * hh] : 0.f, x1 = j + 1 <= r ? qk[nt][2 * hh + 1] : 0.f;
+                        const uint32_t hi = pack_f16(x0, x1);
+                        const float2 hf = unpack_f16(hi);
+                        sts32(base + kAm + sw128(32 * pt + r, 16 * pt + j), hi);
+                        sts32(base + kAm + sw128(32 * pt + 16 + r, 16 * pt + j), pack_f16(x0 - hf.x, x1 - hf.y));
+                    }
                 }
             } else if (cq == 1) {
                 // off-diagonal rows from TMEM: lanes 32pt + r (q rows) and 32pt + 16 + r (k rows)
@@ -745,17 +756,28 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                     tmem_wait_ld();
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        uint4 o;
                         const float sg = krow ? -bi : 1.f;
-                        o.x = pack_f16(sg * __uint_as_float(v[8 * hh + 0]), sg * __uint_as_float(v[8 * hh + 1]));
-                        o.y = pack_f16(sg * __uint_as_float(v[8 * hh + 2]), sg * __uint_as_float(v[8 * hh + 3]));
-                        o.z = pack_f16(sg * __uint_as_float(v[8 * hh + 4]), sg * __uint_as_float(v[8 * hh + 5]));
-                        o.w = pack_f16(sg * __uint_as_float(v[8 * hh + 6]), sg * __uint_as_float(v[8 * hh + 7]));
-                        sts128(krow ? base + kLD + sw128(i, 16 * blk + 8 * hh) : base + kAm + sw128(qslot(i), 16 * blk + 8 * hh), o);
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x0 = sg * __uint_as_float(v[8 * hh + 2 * e]), x1 = sg * __uint_as_float(v[8 * hh + 2 * e + 1]);
+                            hi[e] = pack_f16(x0, x1);
+                            const float2 hf = unpack_f16(hi[e]);
+                            lo[e] = pack_f16(x0 - hf.x, x1 - hf.y);
+                        }
+                        if (krow) {
+                            sts128(base + kLD + sw128(i, 16 * blk + 8 * hh), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                        } else {
+                            sts128(base + kAm + sw128(qslot(i), 16 * blk + 8 * hh), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                            sts128(base + kAm + sw128(kslot(i), 16 * blk + 8 * hh), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                        }
                     }
                 }
-                if (!krow) {   // A: zeros right of the diagonal block
-                    for (int cc = 16 * (pt + 1); cc < 64; cc += 8) sts128(base + kAm + sw128(qslot(i), cc), make_uint4(0, 0, 0, 0));
+                if (!krow) {   // A and its remainder: zeros right of the diagonal block
+                    for (int cc = 16 * (pt + 1); cc < 64; cc += 8) {
+                        sts128(base + kAm + sw128(qslot(i), cc), make_uint4(0, 0, 0, 0));
+                        sts128(base + kAm + sw128(kslot(i), cc), make_uint4(0, 0, 0, 0));
+                    }
                 }
             }
         }
@@ -816,13 +838,32 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         mma_sync();
         if (*abort_flag) break;
         // ---- 8. U (rows 0-63) -> shared memory (fp16, MN-major B operand) ---------------------------
+        //      as fp16 U plus its rounding remainder U - fp16(U) (into the T'' tile, free since step 5)
         {
             uint32_t v[32];
             tld32(tq + cWU + 128 + 32 * cq, v);
-            if (lane >= 16) store_b32(base + kL, 16 * q4 + (lane - 16), v, 1.f);
+            if (lane >= 16) {
+                const int k = 16 * q4 + (lane - 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = __uint_as_float(v[8 * j + 2 * e]), x1 = __uint_as_float(v[8 * j + 2 * e + 1]);
+                        hi[e] = pack_f16(x0, x1);
+                        const float2 hf = unpack_f16(hi[e]);
+                        lo[e] = pack_f16(x0 - hf.x, x1 - hf.y);
+                    }
+                    const uint32_t o = bmn_off(k, 32 * cq + 8 * j);
+                    sts128(base + kL + o, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                    sts128(base + kUlo + o, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                }
+            }
         }
         sync_tc();
         // ---- 9. S += K-^T U;  D[:, 128:256] += A'' U  (the query slots become O) ---------------------
+        //      U and A each enter as fp16 value + fp16 remainder: S += K-^T (U_hi + U_lo),
+        //      O += A_hi (U_hi + U_lo) + A_lo U_hi
         if (wq0) {
             if (leader) {
                 constexpr uint32_t id = idesc(128, 128, 1, 1), id2 = idesc(128, 128, 0, 1);
@@ -831,7 +872,16 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                     mma_ss(tmem + cS, sdesc(aBuf + 2048 * k, 8192, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
+                    mma_ss(tmem + cS, sdesc(aBuf + 2048 * k, 8192, 1024, 2), sdesc(base + kUlo + 4096 * k, 2048, 128, 0), id, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
                     mma_ss(tmem + cWU + 128, sdesc(base + kAm + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss(tmem + cWU + 128, sdesc(base + kAm + 32 * k, 16, 1024, 2), sdesc(base + kUlo + 4096 * k, 2048, 128, 0), id2, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // A_lo: the key-slot rows of A'', 16 rows (2 KB) further on
+                    mma_ss(tmem + cWU + 128, sdesc(base + kAm + 2048 + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);
                 umma_commit(bMma);
             }
             __syncwarp();

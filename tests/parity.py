@@ -83,21 +83,25 @@ def assert_unit_ok(err, label=""):
         assert err["state_rel_l2"] <= REL_L2_TOL, f"{label} state rel L2 {err['state_rel_l2']:.3e}"
 
 
-def check_units(inp, out, final_state, units, scale=1.0, t_end=None):
-    """Oracle-check the listed (n, h) units of a GPU run; returns the worst errors seen."""
-    data = [gather_unit(inp, n, h, t_end) for n, h in units]
-    refs = run_oracle_units(data, scale)
+def check_units(inp, out, final_state, units, scale=1.0, t_end=None, batch=16):
+    """Oracle-check the listed (n, h) units of a GPU run, `batch` units at a time (the fp64 host
+    copies of long units are large); returns the worst errors seen."""
     worst = dict(out_rel_l2=0.0, state_rel_l2=0.0, out_max_abs_frac=0.0)
-    for (n, h), u, (o_ref, S_ref) in zip(units, data, refs):
-        s, e = u["span"]
-        o_gpu = host(out[s:e, h])
-        S_gpu = host(final_state[n, h]) if (final_state is not None and t_end is None) else None
-        err = unit_errors(o_gpu, o_ref, S_gpu, S_ref if S_gpu is not None else None,
-                          out_bf16=out.dtype == torch.bfloat16)
-        assert_unit_ok(err, f"unit (n={n}, h={h})")
-        worst["out_rel_l2"] = max(worst["out_rel_l2"], err["out_rel_l2"])
-        worst["state_rel_l2"] = max(worst["state_rel_l2"], err.get("state_rel_l2", 0.0))
-        if err["out_rms"] > 0:
-            worst["out_max_abs_frac"] = max(worst["out_max_abs_frac"],
-                                            err["out_max_abs"] / err["out_rms"])
+    for b0 in range(0, len(units), batch):
+        part = units[b0:b0 + batch]
+        data = [gather_unit(inp, n, h, t_end) for n, h in part]
+        refs = run_oracle_units(data, scale)
+        for (n, h), u, (o_ref, S_ref) in zip(part, data, refs):
+            s, e = u["span"]
+            o_gpu = host(out[s:e, h])
+            S_gpu = host(final_state[n, h]) if (final_state is not None and t_end is None) else None
+            err = unit_errors(o_gpu, o_ref, S_gpu, S_ref if S_gpu is not None else None,
+                              out_bf16=out.dtype == torch.bfloat16)
+            assert_unit_ok(err, f"unit (n={n}, h={h})")
+            worst["out_rel_l2"] = max(worst["out_rel_l2"], err["out_rel_l2"])
+            worst["state_rel_l2"] = max(worst["state_rel_l2"], err.get("state_rel_l2", 0.0))
+            if err["out_rms"] > 0:
+                worst["out_max_abs_frac"] = max(worst["out_max_abs_frac"],
+                                                err["out_max_abs"] / err["out_rms"])
+        del data, refs
     return worst

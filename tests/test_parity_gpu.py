@@ -243,48 +243,69 @@ def test_prefill_equals_decode_steps(kda):
     assert (S_p - state).norm() / state.norm() < 2e-3
 
 
-# ---- full-size workloads (sampled units) ---------------------------------------------------------
+# ---- full-size workloads ---------------------------------------------------------------------------
+# Outputs are stored in fp32 so that the max-|error| bound applies exactly as stated (2e-2 x rms of
+# the oracle's outputs, per unit), with no allowance for the bf16 output format.  Each test prints
+# its worst errors over the units it checks.
 
-@pytest.mark.parametrize("name,count", [("prefill_B1_H32_T8192_d128", 8),
-                                        ("saturated_B2_H32_T16384_d128", 4),
-                                        ("nofade_B2_H32_T16384_d128", 4)])
-def test_full_size_prefill(kda, name, count):
+def _report(name, worst):
+    print(f"\n[full-size parity] {name}: worst out rel L2 {worst['out_rel_l2']:.2e}, "
+          f"state rel L2 {worst['state_rel_l2']:.2e}, max|err|/rms {worst['out_max_abs_frac']:.2e}")
+
+
+@pytest.mark.parametrize("name,count,path", [
+    ("prefill_B1_H32_T8192_d128", 32, 0),      # 32 units: the cluster kernel
+    ("prefill_B1_H32_T8192_d128", 32, 2),      # the per-unit kernel forced
+    ("saturated_B2_H32_T16384_d128", 16, 0),   # 64 units: the per-unit kernel
+    ("saturated_B2_H32_T16384_d128", 16, 1),   # the cluster kernel forced
+    ("nofade_B2_H32_T16384_d128", 16, 0),
+    ("nofade_B2_H32_T16384_d128", 16, 1),
+])
+def test_full_size_prefill(kda, name, count, path):
     w = KI.WORKLOADS[name]
     inp = KI.make_inputs(w, "cuda")
-    out, S = run(kda, inp)
-    kda.kda_sync_check()
+    kda.kda_set_prefill_path(path)
+    try:
+        out, S = run(kda, inp, out_dtype=F32)
+        kda.kda_sync_check()
+    finally:
+        kda.kda_set_prefill_path(0)
     assert torch.isfinite(S).all()
-    check_units(inp, out, S, sampled_units(w, count))
+    _report(f"{name} path {path}", check_units(inp, out, S, sampled_units(w, count)))
 
 
 def test_full_size_varlen(kda):
     w = KI.VARLEN
     inp = KI.make_inputs(w, "cuda")
-    out, S = run(kda, inp)
+    out, S = run(kda, inp, out_dtype=F32)
     kda.kda_sync_check()
     lens = np.array(w.seqlens)
     # the longest and the shortest sequence, plus random ones
-    units = [(int(lens.argmax()), 0), (int(lens.argmin()), w.H - 1)] + sampled_units(w, 4, seed=1)
-    check_units(inp, out, S, units)
+    units = [(int(lens.argmax()), 0), (int(lens.argmin()), w.H - 1)] + sampled_units(w, 14, seed=1)
+    _report(w.name, check_units(inp, out, S, units))
     del inp, out, S
 
 
 def test_full_size_long_prefill(kda):
+    # every head of the 1 M-token sequence, eight at a time (fp64 copies of 1 M tokens x 128 channels)
     w = KI.LONG_1M
     inp = KI.make_inputs(w, "cuda")
-    out, S = run(kda, inp)
+    out, S = run(kda, inp, out_dtype=F32)
     kda.kda_sync_check()
     assert torch.isfinite(S).all()
-    check_units(inp, out, S, [(0, 0), (0, w.H - 1)])
+    _report(w.name, check_units(inp, out, S, [(0, h) for h in range(w.H)], batch=8))
 
 
 def test_full_size_decode(kda):
     w = KI.DECODE
     inp = KI.make_decode_inputs(w, "cuda")
-    outs, state = decode_run(kda, inp, w.steps)
+    outs, state = decode_run(kda, inp, w.steps, out_dtype=F32)
     r = np.random.default_rng(0)
-    for _ in range(6):
+    worst = 0.0
+    for _ in range(16):
         n, h = int(r.integers(w.N)), int(r.integers(w.H))
         o_ref, S_ref = oracle_unit(decode_unit(inp, n, h, w.steps))
-        err = unit_errors(host(outs[:, n, h]), o_ref, host(state[n, h]), S_ref, out_bf16=True)
+        err = unit_errors(host(outs[:, n, h]), o_ref, host(state[n, h]), S_ref)
         assert_unit_ok(err, f"decode unit ({n},{h})")
+        worst = max(worst, err["out_max_abs"] / max(err["out_rms"], 1e-30))
+    print(f"\n[full-size parity] {w.name}: worst max|err|/rms {worst:.2e}")
