@@ -468,10 +468,15 @@ def context_parallel_states(M, B, S0, group=None, combine=None):
         return S
     rank = dist.get_rank(group)
 
+    # NCCL gathers device tensors directly; gloo (CPU ranks, or ranks sharing one GPU) goes through
+    # host copies
+    via_host = M.is_cuda and dist.get_backend(group) == "gloo"
+
     def gather(x):   # every rank's x, stacked in rank order
-        x = x.contiguous()
-        flat = torch.empty((world * x.shape[0],) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
-        dist.all_gather_into_tensor(flat, x, group=group)
+        src = x.contiguous().cpu() if via_host else x.contiguous()
+        flat = torch.empty((world * src.shape[0],) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+        dist.all_gather_into_tensor(flat, src, group=group)
+        flat = flat.to(x.device) if via_host else flat
         return flat.view((world,) + tuple(x.shape))
 
     Ms, Bs = gather(M), gather(B)

@@ -588,7 +588,7 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
 // columns 16 half .. + 15; an fp16 copy in shared memory is the B operand):
 //   D  = [W ; Q^] S_c            (M = 128: rows 0-63 W S_c, rows 64-127 Q^ S_c)     TMEM
 //   U  = U~ - D[0:64]  -> shared memory (fp16, B operand)
-//   D3 = K-^T U,   D[64:128] += A U   (U and A each as fp16 value + fp16 remainder) TMEM
+//   D3 = K-^T U,   D[64:128] += A U   (there U and A each as fp16 value + remainder) TMEM
 //   S_{c+1} = Diag(Gamma_C) S_c + D3;   out = sigmoid(gate) D[64:128]
 // The A operands ([W; Q^], K-^T, A) of chunk c + 1 are fetched from the ring into registers while
 // chunk c's products run and then stored into the other of two TMEM buffers; the ring slot is
@@ -764,7 +764,7 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                     u[8 * j + 2 * e + 1] = t.y - __uint_as_float(d[8 * j + 2 * e + 1]);
                 }
             }
-            // U enters its products as fp16 U plus the fp16 rounding remainder U - fp16(U)
+            // U enters the output product as fp16 U plus the fp16 rounding remainder U - fp16(U)
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
                 const float2 hf = unpack_f16(pack_f16(u[e], u[e + 1]));
@@ -789,9 +789,6 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 umma_f16_ts(tmem + cD3, tmem + cA2 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, k > 0);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                umma_f16_ts(tmem + cD3, tmem + cA2 + buf * 32 + 8 * k, umma_desc(aB3 + 1024 * k, 512, 128), kIdesc, 1);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 umma_f16_ts(tmem + cD, tmem + cA3 + buf * 32 + 8 * k, umma_desc(aB2 + 1024 * k, 512, 128), kIdesc, 1);

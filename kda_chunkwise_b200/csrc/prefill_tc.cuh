@@ -21,8 +21,8 @@
 //     term below e^-87, so fp16 operands lose nothing: one tcgen05 MMA (M = 128: the row-scaled
 //     q and k rows of the four tiles, N = 96 rescaled keys, K = d_k) computes all of them.
 // Everything on the value path (T', K^, V, W, Q^, K-, A, S, U) is fp16 with fp32 accumulation; U
-// and A, whose rounding shows most in the largest outputs, enter their products as an fp16 value
-// plus its fp16 rounding remainder (about 22 significant bits).  The state's master copy is fp32
+// and A, whose rounding shows most in the largest outputs, enter the output product A U as an fp16
+// value plus its fp16 rounding remainder (about 22 significant bits).  The state's master copy is fp32
 // in tensor memory.
 //
 // Work per chunk (one CTA, 16 warps, the phases separated by CTA barriers):
@@ -862,17 +862,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         }
         sync_tc();
         // ---- 9. S += K-^T U;  D[:, 128:256] += A'' U  (the query slots become O) ---------------------
-        //      U and A each enter as fp16 value + fp16 remainder: S += K-^T (U_hi + U_lo),
-        //      O += A_hi (U_hi + U_lo) + A_lo U_hi
+        //      U and A each enter the output as fp16 value + fp16 remainder: O += A_hi (U_hi + U_lo)
+        //      + A_lo U_hi (the state's K-^T U takes U_hi only: its rounding there does not show)
         if (wq0) {
             if (leader) {
                 constexpr uint32_t id = idesc(128, 128, 1, 1), id2 = idesc(128, 128, 0, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_ss(tmem + cS, sdesc(aBuf + 2048 * k, 8192, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id, 1);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_ss(tmem + cS, sdesc(aBuf + 2048 * k, 8192, 1024, 2), sdesc(base + kUlo + 4096 * k, 2048, 128, 0), id, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_ss(tmem + cWU + 128, sdesc(base + kAm + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);

@@ -156,3 +156,45 @@ def test_context_parallel_prefill_matches_the_unsplit_oracle():
         S_prev = S
     kda.kda_sync_check()
     check_units(inp, out, S_out, [(n, h) for n in range(w.num_seqs) for h in range(w.H)])
+
+
+def _cp_gpu_rank(rank, world, port, out_dir):
+    """Rank `rank` of a gloo group whose ranks share one GPU: it holds segment `rank` of every
+    sequence and calls kda_context_parallel_fwd itself (the maps are exchanged over gloo through
+    host copies; no rank's kernel waits on another's)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import kda_chunkwise_b200 as kda
+        w = KI.Workload("cp_api", (300, 190), 2, 128, 128, A_log="uniform", init_state="normal_0.02", seed=22)
+        inp = KI.make_inputs(w, "cuda")
+        cu = inp["cu_seqlens"].cpu().tolist()
+        seg_bounds = [[(0, 70), (70, 200), (200, 300)], [(0, 64), (64, 100), (100, 190)]]
+        p = _split(inp, cu, seg_bounds)[rank]
+        out, S = kda.kda_context_parallel_fwd(p["q"], p["k"], p["v"], p["a"], p["beta"], inp["A_log"], p["cu_seqlens"],
+                                              gate=p["gate"], initial_state=inp["initial_state"],
+                                              out_dtype=torch.float32)
+        kda.kda_sync_check()
+        np.savez(os.path.join(out_dir, f"cpgpu{rank}.npz"), out=out.cpu().numpy(), S=S.cpu().numpy(),
+                 idx=p["idx"].cpu().numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_context_parallel_entry_point_over_three_ranks_matches_the_unsplit_oracle(tmp_path):
+    """kda_context_parallel_fwd as shipped (segment maps, all-gather, kda_state_combine fold,
+    corrected pass) on three ranks, against the oracle run over the unsplit sequences: the
+    outputs of every segment and, from the last rank, the final states."""
+    from parity import check_units
+    world = 3
+    mp.spawn(_cp_gpu_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    w = KI.Workload("cp_api", (300, 190), 2, 128, 128, A_log="uniform", init_state="normal_0.02", seed=22)
+    inp = KI.make_inputs(w, "cuda")
+    out = torch.empty((w.total_tokens, w.H, w.d_v), dtype=torch.float32)
+    for r in range(world):
+        z = np.load(tmp_path / f"cpgpu{r}.npz")
+        out[torch.from_numpy(z["idx"])] = torch.from_numpy(z["out"])
+    S_last = torch.from_numpy(np.load(tmp_path / f"cpgpu{world - 1}.npz")["S"])
+    check_units(inp, out, S_last, [(n, h) for n in range(w.num_seqs) for h in range(w.H)])
