@@ -41,8 +41,16 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture of each
 # kernel (profiles/ gives the commands), keyed by workload, with the hash of the kernel's sources at
 # capture time.  Reported only while the sources are unchanged.
+# DRAM bytes of one prefill launch per kernel (kda_prefill_path: 1 cluster, 2 per-unit), captured on
+# the named workload; a prefill row scales it by its own algorithmic bytes (both kernels move
+# traffic in proportion to the token-heads and units they process)
+PREFILL_TRAFFIC = {
+    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 339158528 + 57549824, "src": "2b02c5b4b703dc98"},
+    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1347348000 + 257897216,
+        "src": "2b02c5b4b703dc98"},
+}
+
 NCU_TRAFFIC = {
-    "prefill_B1_H32_T8192_d128": {"bytes_per_launch": 396773376, "src": "ce2389bee8082413"},
     "decode_N256_H64_d128_512steps": {"bytes_per_launch": 2114315008, "src": "1c3a7d12c8610c04"},
     # one verify launch plus one commit launch (round 4 of the captured run; commit's bytes depend on
     # how many sequences accepted at least one token)
@@ -137,6 +145,17 @@ def kernel_source_hash(kernel: str | None = None) -> str:
         if name.endswith((".cu", ".cuh")):
             h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
+
+
+def prefill_traffic(w, path: int):
+    """DRAM bytes of one prefill launch on w, scaled from the committed capture of the same kernel."""
+    import kda_inputs as KI
+    t = PREFILL_TRAFFIC.get(path)
+    if not t or t["src"] != kernel_source_hash("prefill"):
+        return None, None
+    cw = KI.WORKLOADS[t["workload"]]
+    scale = prefill_bytes(w) / prefill_bytes(cw)
+    return t["bytes_per_launch"] * scale, t["workload"]
 
 
 def ncu_traffic(key: str, kernel: str):
@@ -396,16 +415,16 @@ def main():
                               workspace=workspace, stream=stream)
         return inp, out, S_final, step
 
-    def prefill_roofline(w, ms, traffic_key):
+    def prefill_roofline(w, ms):
         bytes_step, flops_step = prefill_bytes(w), prefill_flops(w)
         achieved = bytes_step / (ms * 1e-3) / 1e9
-        traffic = ncu_traffic(traffic_key, "prefill") if traffic_key else None
+        traffic, captured = prefill_traffic(w, kda.kda_prefill_path(w.num_seqs * w.H, w.d_k, w.d_v))
         return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic,
-                "traffic_source": (f"dram__bytes_read.sum + dram__bytes_write.sum of an earlier ncu capture "
-                                   f"(profiles/), scaled to this workload; reported while the kernel sources "
-                                   f"are unchanged since" if traffic is not None else
-                                   "no current ncu capture of these kernel sources"),
+                "traffic_source": (f"dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of the same "
+                                   f"kernel on {captured} (profiles/), scaled by algorithmic bytes to this "
+                                   f"workload; reported while the kernel sources are unchanged since"
+                                   if traffic is not None else "no current ncu capture of these kernel sources"),
                 "peak_source": f"hbm_gbs of {peak_src}",
                 "scope": "one kda_chunk_fwd call (all kernels of the prefill path)",
                 "algorithmic_bytes": bytes_step, "algorithmic_flops": flops_step,
@@ -424,7 +443,7 @@ def main():
     kda.kda_sync_check()
     value = whole_job_rate(w.total_tokens, world, ms)
     bytes_step = prefill_bytes(w)
-    roofline = prefill_roofline(w, ms, w.name)
+    roofline = prefill_roofline(w, ms)
     path = kda.kda_prefill_path(w.num_seqs * w.H, w.d_k, w.d_v)
     src_hash = kernel_source_hash()
 
@@ -487,7 +506,7 @@ def main():
         extra.append({"workload": xw.name, "value": whole_job_rate(xw.total_tokens, world, xms), "unit": "tokens/s",
                       "ms_per_step": xms, "steps": xsteps,
                       "kernel": "per-unit" if kda.kda_prefill_path(xw.num_seqs * xw.H, xw.d_k, xw.d_v) == 2 else "cluster",
-                      "roofline": prefill_roofline(xw, xms, xw.name)})
+                      "roofline": prefill_roofline(xw, xms)})
         del xinp, xout, xS, xstep
         torch.cuda.empty_cache()
 

@@ -143,12 +143,11 @@ bool use_tc_prefill(int64_t units, int d_k, int d_v) {
     return units * 3 > device_sm_count();
 }
 
-kda_status launch_prefill_tc(const void *q, const void *k, const void *v, const void *a, const void *gate,
+kda_status launch_prefill_tc(const void *q, const void *k, const void *v, const void *a,
                              const kda::tc::Params &p, int64_t units, cudaStream_t stream) {
     kda::tc::Maps maps;
     if (!encode_thd(&maps.q, q, p.total_tokens, p.H) || !encode_thd(&maps.k, k, p.total_tokens, p.H) ||
-        !encode_thd(&maps.v, v, p.total_tokens, p.H) || !encode_thd(&maps.a, a, p.total_tokens, p.H) ||
-        !encode_thd(&maps.gate, gate ? gate : q, p.total_tokens, p.H))
+        !encode_thd(&maps.v, v, p.total_tokens, p.H) || !encode_thd(&maps.a, a, p.total_tokens, p.H))
         return fail(KDA_ERR_CUDA, "kda_chunk_fwd: cuTensorMapEncodeTiled failed");
     cudaError_t e = cudaFuncSetAttribute(kda::tc::kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kda::tc::kSmemBytes);
@@ -352,8 +351,9 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
         tp.scale = scale;
         tp.out_f32 = out_dtype == KDA_DTYPE_F32;
         tp.has_gate = gate != nullptr;
+        tp.gate = static_cast<const uint16_t *>(gate);
         tp.wait_ns = kWaitNs;
-        return launch_prefill_tc(q, k, v, a, gate, tp, units, static_cast<cudaStream_t>(stream));
+        return launch_prefill_tc(q, k, v, a, tp, units, static_cast<cudaStream_t>(stream));
     }
     char *ws = static_cast<char *>(workspace);
     kda::FusedParams p{};

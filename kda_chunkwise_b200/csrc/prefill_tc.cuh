@@ -26,10 +26,11 @@
 // in tensor memory.
 //
 // Work per chunk (one CTA, 16 warps, the phases separated by CTA barriers):
-//   0. TMA: q, k, v, a, gate rows of the chunk (3-d tensor maps over [T, H, d], two 64-channel boxes
-//      per tensor, 128-byte swizzle), each issued as soon as its buffer is free; a is double buffered.
-//   1. pass 1 (thread = 2 channels x 16 tokens): g = -5 sigmoid(e^{A_h} a) in log2 units, the
+//   0. TMA: q, k, v, a rows of the chunk (3-d tensor maps over [T, H, d], two 64-channel boxes per
+//      tensor, 128-byte swizzle), each issued as soon as its buffer is free; a is double buffered.
+//   1. pass 1 (thread = 2 channels x 8 tokens): g = -5 sigmoid(e^{A_h} a) in log2 units, the
 //      within-tile running sum l, tile totals; tables e^{r_p}, e^{b_C - r_p}, e^{r_p' - r_p}, Gamma_C.
+//      Chunk c + 1's pass 1 runs during chunk c's steps 5 and 7 (while the tensor cores work).
 //   2. pass 2 (warp = tile x channel half, lane = the two rows and 16 channels an MMA fragment
 //      holds): f = 2^l, 1/f; the diagonal Gram blocks (mma.sync tf32); fp16 row-scaled q, k rows into
 //      TMEM (tcgen05.st 16x256b, the fragment layout); rescaled keys of later tiles (fp16) into shared
@@ -42,7 +43,8 @@
 //   7. D[:, 128:256] += [-W; Q^] S   -> rows 0-63 U, rows 64-127 Q^ S  (tcgen05, A in TMEM)
 //   8. U -> shared memory (fp16)
 //   9. S += K-^T U  (S pre-scaled by Gamma_C);  D[:, 128:256] += [0; A] U  -> rows 64-127 O
-//  10. fp16 copy of the new S; out = sigmoid(gate) O, staged in shared memory, stored row by row.
+//  10. fp16 copy of the new S; out = sigmoid(gate) O (gate logits read from global memory during
+//      step 9), staged in shared memory, stored row by row.
 // Every wait on a TMA or MMA completion is bounded (%globaltimer); a timeout records kErrTimeout in
 // the device error word and every thread leaves the chunk loop at the next barrier.
 #pragma once
@@ -66,9 +68,8 @@ constexpr int kK = 16384;          // k -> K^            ] together the B operan
 constexpr int kV = 32768;          // v -> V (fp16)      ]   (four 64-channel atoms, 8 KB apart)
 constexpr int kA0 = 49152;         // a of even chunks -> K- (A operand of K-^T U, MN-major)
 constexpr int kA1 = 65536;         // a of odd chunks  -> K-
-constexpr int kG = 81920;          // gate
-constexpr int kL = 98304;          // fp32 [64][128] within-tile log2 cumsum l (pass 1 -> pass 2);
-                                   //   then U (fp16, 16 KB) and A'' (16 KB); then the output staging
+constexpr int kLT0 = 81920;        // fp32 l table, rows 0-31 (16 KB): pass 1 -> pass 2
+constexpr int kL = 98304;          // U (fp16, 16 KB) and A'' (16 KB); then the output staging
 constexpr int kGB = 131072;        // fp16 rescaled keys of later tiles: K-major, no swizzle, 96 rows
 constexpr int kT = kGB;            // T'' (after the Gram): SW128 [128][64], rows in slot order (below);
                                    //   after [W | U~], the remainder U - fp16(U) (B operand like U)
@@ -77,7 +78,9 @@ constexpr int kAm = kL + 16384;    // A'' (after pass 2): SW128 [128][64]: fp16 
                                    //   remainder A - fp16(A) in the key slots
 constexpr int kS = 155648;         // fp16 S: B operand, MN-major, no swizzle (K = d_k, N = d_v)
 constexpr int kLD = 188416;        // fp16 [64][64] swizzled: -L below the diagonal blocks, D_p on them;
-                                   //   earlier (with kM) the exchange of the diagonal Gram partial sums
+                                   //   earlier (with kM) the exchange of the diagonal Gram partial sums,
+                                   //   and before that rows 32-63 of the l table
+constexpr int kLT1 = kLD;          // fp32 l table, rows 32-63 (16 KB, over kLD and kM)
 constexpr int kM = 196608;         // fp16 [3][16][32] block-product scratch of the solve
 constexpr int kLdf = 204800;       // fp32 [4][16][17] diagonal blocks of L
 constexpr int kTot = kLdf + 4 * 16 * 17 * 4;   // fp32 [8][128] half-tile totals of l
@@ -112,6 +115,7 @@ __host__ __device__ constexpr int gb_off(int pp) { return pp == 1 ? 0 : pp == 2 
 __host__ __device__ constexpr int td_index(int p, int pp) { return p == 0 ? pp - 1 : p == 1 ? pp + 1 : 5; }
 
 struct Params {
+    const uint16_t *gate;            // [T, H, 128] bf16 gate logits, or null
     const float *beta, *A_log;
     const int32_t *cu;
     const float *S_in;
@@ -126,7 +130,7 @@ struct Params {
 };
 
 struct Maps {
-    CUtensorMap q, k, v, a, gate;
+    CUtensorMap q, k, v, a;
 };
 
 // ---- small PTX helpers ---------------------------------------------------------------------------
@@ -216,8 +220,10 @@ __device__ __forceinline__ uint32_t sw128(int row, int col) {
 __device__ __forceinline__ uint32_t in_off(int i, int c) { return (c >> 6) * 8192 + sw128(i, c & 63); }
 // byte offset of element (k, n) of an MN-major, no-swizzle fp16 B operand with N = 128
 __device__ __forceinline__ uint32_t bmn_off(int k, int n) { return (((k >> 3) * 16 + (n >> 3)) << 7) + ((k & 7) << 4) + ((n & 7) << 1); }
-// fp32 l table [64][128] with its 16-byte chunks XOR-ed by 4 (row & 1): conflict-free for both passes
+// fp32 l table [64][128] with its 16-byte chunks XOR-ed by 4 (row & 1): conflict-free for both passes;
+// rows 0-31 at kLT0, rows 32-63 at kLT1
 __device__ __forceinline__ uint32_t l_off(int i, int c) { return i * 512 + ((((c >> 2) ^ ((i & 1) << 2))) << 4) + ((c & 3) << 2); }
+__device__ __forceinline__ uint32_t lt_addr(int i, int c) { return (i < 32 ? kLT0 : kLT1 - 32 * 512) + l_off(i, c); }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     uint32_t v;
@@ -307,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     const int unit = blockIdx.x;
     const int n = unit / p.H, h = unit % p.H;
     const uint32_t base = smem_u32(sm);
-    const uint32_t bQ = base + kBar, bKV = bQ + 8, bA0 = bQ + 16, bA1 = bQ + 24, bGt = bQ + 32, bMma = bQ + 40;
+    const uint32_t bQ = base + kBar, bKV = bQ + 8, bA0 = bQ + 16, bA1 = bQ + 24, bMma = bQ + 40;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kMisc + 4);
 
     int64_t s0, s1;
@@ -322,7 +328,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         for (int i = 0; i < 6; ++i) mbar_init(bQ + 8 * i, 1);
         *abort_flag = 0;
         prefetch_map(&maps.q); prefetch_map(&maps.k); prefetch_map(&maps.v); prefetch_map(&maps.a);
-        if (p.has_gate) prefetch_map(&maps.gate);
     }
     if (warp == 0) tmem_alloc(base + kMisc, 512);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     // TMA issue (one elected lane of warp 0; `leader` is that lane)
     const bool wq0 = warp == 0;
     const bool leader = wq0 && elect_one();
-    uint32_t pend = 0, pend_par = 0;   // leader only: loads in flight per barrier and their wait parity
+    uint32_t pend = 0, pend_par = 0;   // leader only: loads in flight per barrier (q, kv, a0, a1) and their wait parity
     auto issued = [&](int i, uint32_t parity) { pend |= 1u << i; pend_par = (pend_par & ~(1u << i)) | (parity << i); };
     auto load_pair = [&](const CUtensorMap *map, uint32_t dst, uint32_t bar, int cl) {
         const int t = static_cast<int>(s0 + (int64_t)cl * kChunk);
@@ -348,7 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         expect_tx(bA0, 16384); load_pair(&maps.a, base + kA0, bA0, 0); issued(2, 0);
         expect_tx(bQ, 16384); load_pair(&maps.q, base + kQ, bQ, 0); issued(0, 0);
         expect_tx(bKV, 32768); load_pair(&maps.k, base + kK, bKV, 0); load_pair(&maps.v, base + kV, bKV, 0); issued(1, 0);
-        if (p.has_gate) { expect_tx(bGt, 16384); load_pair(&maps.gate, base + kG, bGt, 0); issued(4, 0); }
     }
     auto load_beta = [&](int cl) -> float {
         if (tid >= 64 || cl >= nchunks) return 0.f;
@@ -438,11 +442,80 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                               pack_f16(sgn * __uint_as_float(v[8 * j + 6]), sgn * __uint_as_float(v[8 * j + 7]))));
     };
 
+    // ---- 1. pass 1 of chunk cl, in two halves with a CTA barrier between them -----------------------
+    //      thread = channel pair cp (channels 2cp, 2cp + 1) x half tile part (8 tokens).
+    //      (a) g = -5 sigmoid(e^{A_h} a) in log2 units and the running sum over the part's 8 tokens;
+    //          part totals to shared memory;  (b) the within-tile running sums l (the l table) and
+    //      the tables of the tile references.  Chunk 0's pass 1 runs before the chunk loop; that of
+    //      chunk c + 1 runs inside chunk c, while the tensor cores work on chunk c's products.
+    const int p1_cp = tid & 63, p1_part = tid >> 6, p1_pt = p1_part >> 1, p1_c0 = 2 * p1_cp;
+    float p1_lx[8], p1_ly[8];
+    auto pass1a = [&](int cl) {
+        const int64_t tl = s0 + (int64_t)cl * kChunk;
+        const int Ll = static_cast<int>(min64(kChunk, s1 - tl));
+        const uint32_t ab = (cl & 1) ? base + kA1 : base + kA0;
+        in_wait((cl & 1) ? bA1 : bA0, (cl >> 1) & 1);
+        float sx = 0.f, sy = 0.f;
+        constexpr float kG2 = kGMin * kLog2e;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * p1_part + i;
+            const float2 av = unpack_bf16(lds32(ab + in_off(t, p1_c0)));
+            float gx = kG2 * sigmoid_fast(expA * av.x), gy = kG2 * sigmoid_fast(expA * av.y);
+            if (t >= Ll) gx = gy = 0.f;
+            sx += gx; sy += gy;
+            p1_lx[i] = sx; p1_ly[i] = sy;
+        }
+        float *tot = reinterpret_cast<float *>(sm + kTot);   // [8 half tiles][128]
+        *reinterpret_cast<float2 *>(tot + p1_part * 128 + p1_c0) = make_float2(sx, sy);
+    };
+    auto pass1b = [&]() {
+        const float *tot = reinterpret_cast<const float *>(sm + kTot);
+        const int part = p1_part, pt = p1_pt, c0 = p1_c0;
+        // within-tile running sum: the second half adds the first half's total
+        const float2 off = (part & 1) ? *reinterpret_cast<const float2 *>(tot + (part - 1) * 128 + c0) : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * part + i;
+            *reinterpret_cast<float2 *>(sm + lt_addr(t, c0)) = make_float2(p1_lx[i] + off.x, p1_ly[i] + off.y);
+        }
+        if ((part & 1) == 0) {   // tables of tile pt, once per channel pair
+            float2 T4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 x0 = *reinterpret_cast<const float2 *>(tot + (2 * q) * 128 + c0);
+                const float2 x1 = *reinterpret_cast<const float2 *>(tot + (2 * q + 1) * 128 + c0);
+                T4[q] = make_float2(x0.x + x1.x, x0.y + x1.y);
+            }
+            float2 R = make_float2(0.f, 0.f), BC = R;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (q < pt) { R.x += T4[q].x; R.y += T4[q].y; }
+                BC.x += T4[q].x; BC.y += T4[q].y;
+            }
+            *reinterpret_cast<float2 *>(sm + kTE + (pt * 128 + c0) * 4) = make_float2(ex2(R.x), ex2(R.y));
+            *reinterpret_cast<float2 *>(sm + kTK + (pt * 128 + c0) * 4) = make_float2(ex2(BC.x - R.x), ex2(BC.y - R.y));
+            float2 Rn = R;
+#pragma unroll
+            for (int pp = 1; pp < 4; ++pp) {
+                if (pp <= pt) continue;
+                Rn.x += T4[pp - 1].x; Rn.y += T4[pp - 1].y;
+                *reinterpret_cast<float2 *>(sm + kTD + (td_index(pt, pp) * 128 + c0) * 4) =
+                    make_float2(ex2(Rn.x - R.x), ex2(Rn.y - R.y));
+            }
+            if (pt == 0) *reinterpret_cast<float2 *>(sm + kGam + c0 * 4) = make_float2(ex2(BC.x), ex2(BC.y));
+        }
+    };
+    if (nchunks > 0) {
+        pass1a(0);
+        bar_all();
+        pass1b();
+    }
+
     for (int c = 0; c < nchunks; ++c) {
         const int64_t t0 = s0 + (int64_t)c * kChunk;
         const int L = static_cast<int>(min64(kChunk, s1 - t0));
         const uint32_t aBuf = (c & 1) ? base + kA1 : base + kA0;
-        const uint32_t aBar = (c & 1) ? bA1 : bA0;
         if (tid < 64) sbeta[tid] = beta_next;
         beta_next = load_beta(c + 1);
         // the next chunk's a goes into the other buffer (its K- of chunk c-1 is consumed)
@@ -452,61 +525,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             expect_tx(nbar, 16384);
             load_pair(&maps.a, nb, nbar, c + 1);
             issued((c & 1) ? 2 : 3, ((c + 1) >> 1) & 1);
-        }
-        in_wait(aBar, (c >> 1) & 1);
-
-        // ---- 1. pass 1: g, within-tile running sums, tile totals ---------------------------------
-        //      thread = channel pair cp (channels 2cp, 2cp + 1) x half tile part (8 tokens)
-        {
-            const int cp = tid & 63, part = tid >> 6, pt = part >> 1, c0 = 2 * cp;
-            float lx[8], ly[8];
-            float sx = 0.f, sy = 0.f;
-            constexpr float kG2 = kGMin * kLog2e;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int t = 8 * part + i;
-                const float2 av = unpack_bf16(lds32(aBuf + in_off(t, c0)));
-                float gx = kG2 * sigmoid_fast(expA * av.x), gy = kG2 * sigmoid_fast(expA * av.y);
-                if (t >= L) gx = gy = 0.f;
-                sx += gx; sy += gy;
-                lx[i] = sx; ly[i] = sy;
-            }
-            float *tot = reinterpret_cast<float *>(sm + kTot);   // [8 half tiles][128]
-            *reinterpret_cast<float2 *>(tot + part * 128 + c0) = make_float2(sx, sy);
-            bar_all();
-            // within-tile running sum: the second half adds the first half's total
-            const float2 off = (part & 1) ? *reinterpret_cast<const float2 *>(tot + (part - 1) * 128 + c0) : make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int t = 8 * part + i;
-                *reinterpret_cast<float2 *>(sm + kL + l_off(t, c0)) = make_float2(lx[i] + off.x, ly[i] + off.y);
-            }
-            if ((part & 1) == 0) {   // tables of tile pt, once per channel pair
-                float2 T4[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 x0 = *reinterpret_cast<const float2 *>(tot + (2 * q) * 128 + c0);
-                    const float2 x1 = *reinterpret_cast<const float2 *>(tot + (2 * q + 1) * 128 + c0);
-                    T4[q] = make_float2(x0.x + x1.x, x0.y + x1.y);
-                }
-                float2 R = make_float2(0.f, 0.f), BC = R;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (q < pt) { R.x += T4[q].x; R.y += T4[q].y; }
-                    BC.x += T4[q].x; BC.y += T4[q].y;
-                }
-                *reinterpret_cast<float2 *>(sm + kTE + (pt * 128 + c0) * 4) = make_float2(ex2(R.x), ex2(R.y));
-                *reinterpret_cast<float2 *>(sm + kTK + (pt * 128 + c0) * 4) = make_float2(ex2(BC.x - R.x), ex2(BC.y - R.y));
-                float2 Rn = R;
-#pragma unroll
-                for (int pp = 1; pp < 4; ++pp) {
-                    if (pp <= pt) continue;
-                    Rn.x += T4[pp - 1].x; Rn.y += T4[pp - 1].y;
-                    *reinterpret_cast<float2 *>(sm + kTD + (td_index(pt, pp) * 128 + c0) * 4) =
-                        make_float2(ex2(Rn.x - R.x), ex2(Rn.y - R.y));
-                }
-                if (pt == 0) *reinterpret_cast<float2 *>(sm + kGam + c0 * 4) = make_float2(ex2(BC.x), ex2(BC.y));
-            }
         }
         in_wait(bQ, c & 1);
         in_wait(bKV, c & 1);
@@ -531,9 +549,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 const uint32_t oq0 = in_off(i0, cb), oq1 = oq0 + 1024;
                 uint2 qr0 = lds64(base + kQ + oq0), qr1 = lds64(base + kQ + oq1);
                 uint2 kr0 = lds64(base + kK + oq0), kr1 = lds64(base + kK + oq1);
-                const uint32_t ol0 = l_off(i0, cb);
-                const float4 l0 = *reinterpret_cast<const float4 *>(sm + kL + ol0);
-                const float4 l1 = *reinterpret_cast<const float4 *>(sm + kL + ol0 + 4096);
+                const uint32_t ol0 = lt_addr(i0, cb);   // rows i0 and i0 + 8 lie in the same half
+                const float4 l0 = *reinterpret_cast<const float4 *>(sm + ol0);
+                const float4 l1 = *reinterpret_cast<const float4 *>(sm + ol0 + 4096);
                 const float4 te = *reinterpret_cast<const float4 *>(sm + kTE + (pt * 128 + cb) * 4);
                 const float4 tk = *reinterpret_cast<const float4 *>(sm + kTK + (pt * 128 + cb) * 4);
                 float qv[2][4], kv[2][4], lv[2][4];
@@ -640,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                     kk[e >> 2][e & 3] += xch[((slot * 4 + pt) * 16 + 8 + e) * 32 + lane];
                 }
             };
+            bar_all();   // every warp is past its reads of the l table, whose rows 32-63 the exchange reuses
             if (cq >= 2) put(cq - 2);
             sync_tc();
             if (*abort_flag) break;
@@ -801,6 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
+        if (c + 1 < nchunks) pass1a(c + 1);   // the next chunk's pass 1, first half
         mma_sync();
         if (*abort_flag) break;
         // k, v buffers are free: the next chunk's k, v
@@ -835,6 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
+        if (c + 1 < nchunks) pass1b();         // the next chunk's pass 1, second half
         mma_sync();
         if (*abort_flag) break;
         // ---- 8. U (rows 0-63) -> shared memory (fp16, MN-major B operand) ---------------------------
@@ -883,8 +904,20 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
-        // the gate rows of this chunk must have arrived
-        if (p.has_gate) in_wait(bGt, c & 1);
+        // meanwhile: this thread's gate logits (rows 16 q4 + g and + 8, column pairs 32 cq + 8b + 2t4)
+        uint32_t gpre[8];
+        {
+            const int gg = lane >> 2, tt = lane & 3;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int i = 16 * q4 + gg + 8 * rr;
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    gpre[4 * rr + b] = (p.has_gate && i < L)
+                        ? __ldg(reinterpret_cast<const uint32_t *>(p.gate + ((t0 + i) * H + h) * kD + 32 * cq + 8 * b + 2 * tt))
+                        : 0u;
+            }
+        }
         mma_sync();
         if (*abort_flag) break;
         // ---- 10. new S (fp16 copy); gated output rows -----------------------------------------------
@@ -910,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                         const int cc = 32 * cq + 8 * b + 2 * tt;
                         float o0 = __uint_as_float(o16[4 * b + 2 * rr]), o1 = __uint_as_float(o16[4 * b + 2 * rr + 1]);
                         if (p.has_gate) {
-                            const float2 ga = unpack_bf16(lds32(base + kG + in_off(i, cc)));
+                            const float2 ga = unpack_bf16(gpre[4 * rr + b]);
                             o0 *= sigmoid_fast(ga.x);
                             o1 *= sigmoid_fast(ga.y);
                         }
@@ -926,13 +959,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         tc_fence_before();
         bar_all();
         tc_fence_after();
-        // gate buffer free: the next chunk's gate
-        if (leader && c + 1 < nchunks && p.has_gate) {
-            fence_async_smem();
-            expect_tx(bGt, 16384);
-            load_pair(&maps.gate, base + kG, bGt, c + 1);
-            issued(4, (c + 1) & 1);
-        }
         // rows < L of the staged output -> global, two rows per warp instruction
         if (p.out_f32) {
             float *outp = static_cast<float *>(p.out);
@@ -953,12 +979,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 }
             }
         }
-        bar_all();   // the staging area (kL) is rewritten by the next chunk's pass 1
+        bar_all();   // the staging area (kL) is rewritten by the next chunk's step 8
     }
 
     if (*abort_flag && leader) {
         // copies issued but never waited for complete before the CTA leaves (bounded)
-        for (int i = 0; i < 5; ++i)
+        for (int i = 0; i < 4; ++i)
             if (pend >> i & 1) wait_bounded(bQ + 8 * i, pend_par >> i & 1, p.wait_ns);
         wait_bounded(bMma, mma_phase ^ 1, p.wait_ns);
     }
