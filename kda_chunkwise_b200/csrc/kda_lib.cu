@@ -111,16 +111,19 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 3-d map over a [T, H, 128] bf16 tensor: boxes of 64 channels x 1 head x 64 tokens, 128-byte
-// swizzle (the layout the kernel's shared-memory operands use); rows past T read as zeros.
-bool encode_thd(CUtensorMap *map, const void *ptr, int64_t T, int H) {
+// 3-d map over a [T, H, 128] bf16 (or fp32) tensor: boxes of 128 bytes of channels (64 bf16, 32
+// fp32) x 1 head x 64 tokens, 128-byte swizzle (the layout of the kernel's shared-memory tiles);
+// loaded rows past T read as zeros, stored rows past T are dropped.
+bool encode_thd(CUtensorMap *map, const void *ptr, int64_t T, int H, bool f32 = false) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
+    const cuuint64_t es = f32 ? 4 : 2;
     const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
-    const cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
-    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint64_t strides[2] = {128 * es, (cuuint64_t)H * 128 * es};
+    const cuuint32_t box[3] = {(cuuint32_t)(128 / es), 1, 64};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+    return enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr),
+               dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -147,7 +150,8 @@ kda_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
                              const kda::tc::Params &p, int64_t units, cudaStream_t stream) {
     kda::tc::Maps maps;
     if (!encode_thd(&maps.q, q, p.total_tokens, p.H) || !encode_thd(&maps.k, k, p.total_tokens, p.H) ||
-        !encode_thd(&maps.v, v, p.total_tokens, p.H) || !encode_thd(&maps.a, a, p.total_tokens, p.H))
+        !encode_thd(&maps.v, v, p.total_tokens, p.H) || !encode_thd(&maps.a, a, p.total_tokens, p.H) ||
+        !encode_thd(&maps.out, p.out, p.total_tokens, p.H, p.out_f32))
         return fail(KDA_ERR_CUDA, "kda_chunk_fwd: cuTensorMapEncodeTiled failed");
     cudaError_t e = cudaFuncSetAttribute(kda::tc::kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kda::tc::kSmemBytes);

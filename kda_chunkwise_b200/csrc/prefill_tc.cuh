@@ -41,10 +41,10 @@
 //   5. D[0:64] = [T'; 0] [K^ | V] = [W | U~]                         (tcgen05, N = 256, K = 64)
 //   6. -W -> TMEM, beside Q^ (rows 64-127)
 //   7. D[:, 128:256] += [-W; Q^] S   -> rows 0-63 U, rows 64-127 Q^ S  (tcgen05, A in TMEM)
-//   8. U -> shared memory (fp16)
-//   9. S += K-^T U  (S pre-scaled by Gamma_C);  D[:, 128:256] += [0; A] U  -> rows 64-127 O
+//   8. U -> shared memory (fp16 value and remainder); its TMEM rows zeroed
+//   9. S += K-^T U  (S pre-scaled by Gamma_C);  D[:, 128:256] += [A_hi; A_lo] U -> O in two parts
 //  10. fp16 copy of the new S; out = sigmoid(gate) O (gate logits read from global memory during
-//      step 9), staged in shared memory, stored row by row.
+//      step 9), staged in shared memory, stored by TMA (row by row for a sequence's last chunk).
 // Every wait on a TMA or MMA completion is bounded (%globaltimer); a timeout records kErrTimeout in
 // the device error word and every thread leaves the chunk loop at the next barrier.
 #pragma once
@@ -131,6 +131,7 @@ struct Params {
 
 struct Maps {
     CUtensorMap q, k, v, a;
+    CUtensorMap out;   // [T, H, 128] output: bf16 boxes of 64 channels, or fp32 boxes of 32 channels
 };
 
 // ---- small PTX helpers ---------------------------------------------------------------------------
@@ -166,6 +167,18 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap *map, in
         : "memory");
 }
 
+// one box of the staged output tile -> global (bulk-group completion)
+__device__ __forceinline__ void tma_store_box(const CUtensorMap *map, uint32_t src, int x, int h, int t) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(h), "r"(t)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// the shared-memory source of every committed store has been read / every store is complete
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -188,6 +201,23 @@ __device__ __forceinline__ void tmem_st_frag(uint32_t taddr, uint32_t r0, uint32
     asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2),
                  "r"(r3)
                  : "memory");
+}
+
+// tcgen05.ld / st 16x256b.x4: lane (g, t) of the warp holds TMEM lanes base + g (v[4b], v[4b + 1]) and
+// base + g + 8 (v[4b + 2], v[4b + 3]), columns 8b + 2t and 8b + 2t + 1, b = 0..3
+__device__ __forceinline__ void tmem_ld_frag4(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_frag4(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
 }
 
 // tcgen05.mma kind::f16 with both operands in shared memory, or A in tensor memory
@@ -216,8 +246,12 @@ __host__ __device__ constexpr uint32_t idesc(int M, int N, int a_mn, int b_mn) {
 __device__ __forceinline__ uint32_t sw128(int row, int col) {
     return row * 128 + ((((col >> 3) ^ row) & 7) << 4) + ((col & 7) << 1);
 }
-// element (token i, channel c) of a TMA-loaded [2 atoms][64][64] tile
+// element (token i, channel c) of a TMA-loaded [2 atoms][64][64] tile (also the bf16 output staging)
 __device__ __forceinline__ uint32_t in_off(int i, int c) { return (c >> 6) * 8192 + sw128(i, c & 63); }
+// element (token i, channel c) of the fp32 output staging: [4 atoms of 32 channels][64][128 B], SW128
+__device__ __forceinline__ uint32_t out_off_f32(int i, int c) {
+    return (c >> 5) * 8192 + i * 128 + ((((c >> 2) & 7) ^ (i & 7)) << 4) + ((c & 3) << 2);
+}
 // byte offset of element (k, n) of an MN-major, no-swizzle fp16 B operand with N = 128
 __device__ __forceinline__ uint32_t bmn_off(int k, int n) { return (((k >> 3) * 16 + (n >> 3)) << 7) + ((k & 7) << 4) + ((n & 7) << 1); }
 // fp32 l table [64][128] with its 16-byte chunks XOR-ed by 4 (row & 1): conflict-free for both passes;
@@ -253,57 +287,46 @@ __device__ __forceinline__ void bar_all() { named_bar(1, kThreads); }
 // ---------------------------------------------------------------------------------------------
 // The solve: T' = (I + L)^-1 diag(beta), given the diagonal inverses D_p = (I + L_pp)^-1 (fp16, on
 // the diagonal blocks of LD), T'_pp = D_p diag(beta_p) (on those of T') and the fp16 blocks -L_pm
-// (m < p) in LD: level by level d = p - q,  T'_pq = D_p sum_{m=q}^{p-1} (-L_pm) T'_mq  as 16 x 16
-// products; starting from D_q diag(beta_q) yields T' directly.  T' is an SW128 [64][64] tile (the
-// MMA's A operand); its rows are the key slots of a 128-row tile whose query slots are zero.
+// (m < p) in LD:  T'_pq = D_p sum_{m=q}^{p-1} (-L_pm) T'_mq  for p = q + 1, q + 2, ... as 16 x 16
+// products; starting from D_q diag(beta_q) yields T' directly.  Column block q of T' needs only
+// column block q, so warp (q, half) computes its 8 columns of blocks (q + 1, q) .. (3, q) in turn
+// with no barrier.  T' is an SW128 [64][64] tile (the MMA's A operand); its rows are the key slots
+// of a 128-row tile whose query slots are zero.
 // ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+
 __device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
+    if (warp >= 6) return;
     const uint32_t base = smem_u32(sm);
     const int g = lane >> 2, t4 = lane & 3;
-    if (warp >= 4 && warp < 8) {   // zero the blocks of T' above the diagonal: (0,1..3), (1,2..3), (2,3)
-        for (int e = (warp - 4) * 32 + lane; e < 6 * 16 * 2; e += 128) {
-            const int ub = e / 32, rem = e % 32, r = rem >> 1, half = rem & 1;
-            const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
-            sts128(base + kT + sw128(32 * pb + 16 + r, 16 * qb + 8 * half), make_uint4(0, 0, 0, 0));
-        }
-    }
-    bar_all();
+    const int qb = warp >> 1, half = warp & 1;
+    const uint32_t scr = base + kM + warp * 256;   // [16][8] fp16 product, 16-byte rows
 #pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-        if (warp < 4 - d) {
-            const int qb = warp, pb = warp + d;
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int mb = qb; mb < pb; ++mb) {
-                uint32_t af[4], bf[4];
-                ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * mb, lane));   // -L_pm
-                ldsm_x4_t(bf, ldsm_addr_bt<128>(base + kT, 32 * mb + 16, 16 * qb, lane));  // T'_mq
-                mma_f16(acc[0], af, bf[0], bf[1]);
-                mma_f16(acc[1], af, bf[2], bf[3]);
-            }
-            const uint32_t aMw = base + kM + warp * 2048;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int cc = 8 * j + 2 * t4;
-                sts32(aMw + swz_elem<64>(g, cc), pack_f16(acc[j][0], acc[j][1]));
-                sts32(aMw + swz_elem<64>(g + 8, cc), pack_f16(acc[j][2], acc[j][3]));
-            }
-            __syncwarp();
-            float tq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            {
-                uint32_t af[4], bf[4];
-                ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * pb, lane));   // D_p
-                ldsm_x4_t(bf, ldsm_addr_bt<64>(aMw, 0, 0, lane));
-                mma_f16(tq[0], af, bf[0], bf[1]);
-                mma_f16(tq[1], af, bf[2], bf[3]);
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int cc = 16 * qb + 8 * j + 2 * t4;
-                sts32(base + kT + sw128(32 * pb + 16 + g, cc), pack_f16(tq[j][0], tq[j][1]));
-                sts32(base + kT + sw128(32 * pb + 24 + g, cc), pack_f16(tq[j][2], tq[j][3]));
-            }
+    for (int pb = qb + 1; pb < 4; ++pb) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int mb = qb; mb < pb; ++mb) {
+            uint32_t af[4], bf[2];
+            ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * mb, lane));                        // -L_pm
+            ldsm_x2_t(bf, base + kT + swz<128>(32 * mb + 16 + (lane & 15), 2 * qb + half));          // T'_mq, 8 columns
+            mma_f16(acc, af, bf[0], bf[1]);
         }
-        bar_all();
+        sts32(scr + 16 * g + 4 * t4, pack_f16(acc[0], acc[1]));
+        sts32(scr + 16 * (g + 8) + 4 * t4, pack_f16(acc[2], acc[3]));
+        __syncwarp();
+        float tq[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            uint32_t af[4], bf[2];
+            ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * pb, lane));   // D_p
+            ldsm_x2_t(bf, scr + 16 * (lane & 15));
+            mma_f16(tq, af, bf[0], bf[1]);
+        }
+        const int cc = 16 * qb + 8 * half + 2 * t4;
+        sts32(base + kT + sw128(32 * pb + 16 + g, cc), pack_f16(tq[0], tq[1]));
+        sts32(base + kT + sw128(32 * pb + 24 + g, cc), pack_f16(tq[2], tq[3]));
+        __syncwarp();
     }
 }
 
@@ -327,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(bQ + 8 * i, 1);
         *abort_flag = 0;
-        prefetch_map(&maps.q); prefetch_map(&maps.k); prefetch_map(&maps.v); prefetch_map(&maps.a);
+        prefetch_map(&maps.q); prefetch_map(&maps.k); prefetch_map(&maps.v); prefetch_map(&maps.a); prefetch_map(&maps.out);
     }
     if (warp == 0) tmem_alloc(base + kMisc, 512);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -528,6 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         }
         in_wait(bQ, c & 1);
         in_wait(bKV, c & 1);
+        if (leader) bulk_wait_read();   // the previous chunk's output stores have read the staging area
         bar_all();
         if (*abort_flag) break;
 
@@ -640,40 +664,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 }
             }
         }
-        // the four channel quarters' diagonal partial sums, added in a fixed order (cq 2, 3 -> 0, 1;
-        // then 1 -> 0) through 16 KB of the solve's scratch
-        {
-            float *xch = reinterpret_cast<float *>(sm + kLD);   // [2][4 tiles][16][32]
-            auto put = [&](int slot) {
+        // the four channel quarters' diagonal partial sums: quarters 1-3 put theirs into the output
+        // staging area (free from the end of the previous chunk to step 8), quarter 0 adds them in a
+        // fixed order, (x0 + x2) + (x1 + x3)
+        float *xch = reinterpret_cast<float *>(sm + kL);   // [3][4 tiles][16][32]
+        if (cq >= 1) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    xch[((slot * 4 + pt) * 16 + e) * 32 + lane] = qk[e >> 2][e & 3];
-                    xch[((slot * 4 + pt) * 16 + 8 + e) * 32 + lane] = kk[e >> 2][e & 3];
-                }
-            };
-            auto add = [&](int slot) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    qk[e >> 2][e & 3] += xch[((slot * 4 + pt) * 16 + e) * 32 + lane];
-                    kk[e >> 2][e & 3] += xch[((slot * 4 + pt) * 16 + 8 + e) * 32 + lane];
-                }
-            };
-            bar_all();   // every warp is past its reads of the l table, whose rows 32-63 the exchange reuses
-            if (cq >= 2) put(cq - 2);
-            sync_tc();
-            if (*abort_flag) break;
-            // every thread is past pass 2: the q buffer is free for the next chunk's q
-            if (leader && c + 1 < nchunks) {
-                fence_async_smem();
-                expect_tx(bQ, 16384);
-                load_pair(&maps.q, base + kQ, bQ, c + 1);
-                issued(0, (c + 1) & 1);
+            for (int e = 0; e < 8; ++e) {
+                xch[(((cq - 1) * 4 + pt) * 16 + e) * 32 + lane] = qk[e >> 2][e & 3];
+                xch[(((cq - 1) * 4 + pt) * 16 + 8 + e) * 32 + lane] = kk[e >> 2][e & 3];
             }
-            if (cq < 2) add(cq);
-            bar_all();
-            if (cq == 1) put(0);
-            bar_all();
-            if (cq == 0) add(0);
+        }
+        sync_tc();
+        if (*abort_flag) break;
+        // every thread is past pass 2: the q buffer is free for the next chunk's q
+        if (leader && c + 1 < nchunks) {
+            fence_async_smem();
+            expect_tx(bQ, 16384);
+            load_pair(&maps.q, base + kQ, bQ, c + 1);
+            issued(0, (c + 1) & 1);
         }
 
         // ---- 3. off-diagonal Gram (TMEM A rows x rescaled keys) ----------------------------------
@@ -686,6 +695,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 umma_commit(bMma);
             }
             __syncwarp();
+        }
+        if (cq == 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int i0 = ((0 * 4 + pt) * 16 + e) * 32 + lane, i1 = i0 + 4 * 16 * 32, i2 = i1 + 4 * 16 * 32;
+                qk[e >> 2][e & 3] = (qk[e >> 2][e & 3] + xch[i1]) + (xch[i0] + xch[i2]);
+                kk[e >> 2][e & 3] = (kk[e >> 2][e & 3] + xch[i1 + 256]) + (xch[i0 + 256] + xch[i2 + 256]);
+            }
         }
         // meanwhile: the diagonal blocks of L (fp32) and their inverses D_p = (I + L_pp)^-1, by
         // column-oriented forward substitution, one column per lane of warp pt (kept in registers
@@ -798,12 +815,20 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                         sts128(base + kAm + sw128(kslot(i), cc), make_uint4(0, 0, 0, 0));
                     }
                 }
+            } else {
+                // T'' (over the rescaled keys, consumed by the Gram): zero query slots (4 tiles x 16
+                // rows x 8 chunks of 16 bytes) and zero blocks above the diagonal in the key slots,
+                // (0, 1..3), (1, 2..3), (2, 3) (16 rows x 2 chunks each)
+                for (int e = tid - 256; e < 512 + 192; e += 256) {
+                    if (e < 512) {
+                        sts128(base + kT + (32 * (e >> 7) + ((e >> 3) & 15)) * 128 + 16 * (e & 7), make_uint4(0, 0, 0, 0));
+                    } else {
+                        const int ub = (e - 512) >> 5, r = ((e - 512) >> 1) & 15, hh = e & 1;
+                        const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
+                        sts128(base + kT + sw128(32 * pb + 16 + r, 16 * qb + 8 * hh), make_uint4(0, 0, 0, 0));
+                    }
+                }
             }
-        }
-        // the query slots of T'' are zero (their bytes held rescaled keys in pass 2)
-        {
-            const int e = tid;   // 512 chunks of 16 bytes: 4 tiles x 16 rows x 8 chunks
-            sts128(base + kT + (32 * (e >> 7) + ((e >> 3) & 15)) * 128 + 16 * (e & 7), make_uint4(0, 0, 0, 0));
         }
         bar_all();
         solve(sm, warp, lane);
@@ -858,33 +883,39 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (c + 1 < nchunks) pass1b();         // the next chunk's pass 1, second half
         mma_sync();
         if (*abort_flag) break;
-        // ---- 8. U (rows 0-63) -> shared memory (fp16, MN-major B operand) ---------------------------
-        //      as fp16 U plus its rounding remainder U - fp16(U) (into the T'' tile, free since step 5)
+        // ---- 8. U (key slots) -> shared memory (fp16, MN-major B operand) ----------------------------
+        //      as fp16 U plus its rounding remainder U - fp16(U) (into the T'' tile, free since step 5);
+        //      lane (g, t4) holds tokens 16 q4 + g, + 8 and columns 32 cq + 8 b + 2 t4, + 1 (16x256b).
+        //      The key slots are then zeroed: step 9 accumulates A_lo U there.
         {
-            uint32_t v[32];
-            tld32(tq + cWU + 128 + 32 * cq, v);
-            if (lane >= 16) {
-                const int k = 16 * q4 + (lane - 16);
+            const uint32_t ta = tq + (16u << 16) + cWU + 128 + 32 * cq;
+            uint32_t u16[16];
+            tmem_ld_frag4(ta, u16);
+            tmem_wait_ld();
+            {
+                uint32_t z[16];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t hi[4], lo[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x0 = __uint_as_float(v[8 * j + 2 * e]), x1 = __uint_as_float(v[8 * j + 2 * e + 1]);
-                        hi[e] = pack_f16(x0, x1);
-                        const float2 hf = unpack_f16(hi[e]);
-                        lo[e] = pack_f16(x0 - hf.x, x1 - hf.y);
-                    }
-                    const uint32_t o = bmn_off(k, 32 * cq + 8 * j);
-                    sts128(base + kL + o, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                    sts128(base + kUlo + o, make_uint4(lo[0], lo[1], lo[2], lo[3]));
-                }
+                for (int e = 0; e < 16; ++e) z[e] = 0u;
+                tmem_st_frag4(ta, z);
             }
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const float x0 = __uint_as_float(u16[4 * b + 2 * rr]), x1 = __uint_as_float(u16[4 * b + 2 * rr + 1]);
+                    const uint32_t hi = pack_f16(x0, x1);
+                    const float2 hf = unpack_f16(hi);
+                    const uint32_t o = bmn_off(16 * q4 + g + 8 * rr, 32 * cq + 8 * b + 2 * t4);
+                    sts32(base + kL + o, hi);
+                    sts32(base + kUlo + o, pack_f16(x0 - hf.x, x1 - hf.y));
+                }
         }
         sync_tc();
         // ---- 9. S += K-^T U;  D[:, 128:256] += A'' U  (the query slots become O) ---------------------
-        //      U and A each enter the output as fp16 value + fp16 remainder: O += A_hi (U_hi + U_lo)
-        //      + A_lo U_hi (the state's K-^T U takes U_hi only: its rounding there does not show)
+        //      U and A each enter the output as fp16 value + fp16 remainder: A'' holds A_hi in the
+        //      query slots and A_lo in the key slots, so A'' (U_hi + U_lo) leaves Q^ S + A_hi U in the
+        //      query slots and A_lo U in the (zeroed) key slots; the epilogue adds the two (the
+        //      state's K-^T U takes U_hi only: its rounding there does not show)
         if (wq0) {
             if (leader) {
                 constexpr uint32_t id = idesc(128, 128, 1, 1), id2 = idesc(128, 128, 0, 1);
@@ -897,9 +928,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_ss(tmem + cWU + 128, sdesc(base + kAm + 32 * k, 16, 1024, 2), sdesc(base + kUlo + 4096 * k, 2048, 128, 0), id2, 1);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)   // A_lo: the key-slot rows of A'', 16 rows (2 KB) further on
-                    mma_ss(tmem + cWU + 128, sdesc(base + kAm + 2048 + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);
                 umma_commit(bMma);
             }
             __syncwarp();
@@ -925,63 +953,69 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             uint32_t v[32];
             tld32(tq + cS + 32 * cq, v);
             store_b32(base + kS, row, v, 1.f);
-            // query slots of quadrant q4: tokens 16 q4 + g and + 8 (lane (g, t4)), columns 32 cq + 8b + 2t4, + 1
-            {
-                uint32_t o16[16];
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-                    : "=r"(o16[0]), "=r"(o16[1]), "=r"(o16[2]), "=r"(o16[3]), "=r"(o16[4]), "=r"(o16[5]), "=r"(o16[6]), "=r"(o16[7]),
-                      "=r"(o16[8]), "=r"(o16[9]), "=r"(o16[10]), "=r"(o16[11]), "=r"(o16[12]), "=r"(o16[13]), "=r"(o16[14]), "=r"(o16[15])
-                    : "r"(tq + cWU + 128 + 32 * cq));
-                tmem_wait_ld();
-                const int gg = lane >> 2, tt = lane & 3;
+            // tokens 16 q4 + g and + 8 (lane (g, t4)), columns 32 cq + 8b + 2t4, + 1: query slots
+            // (Q^ S + A_hi U) plus key slots (A_lo U)
+            uint32_t oq[16], ok[16];
+            tmem_ld_frag4(tq + cWU + 128 + 32 * cq, oq);
+            tmem_ld_frag4(tq + (16u << 16) + cWU + 128 + 32 * cq, ok);
+            tmem_wait_ld();
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int i = 16 * q4 + gg + 8 * rr;
+            for (int rr = 0; rr < 2; ++rr) {
+                const int i = 16 * q4 + g + 8 * rr;
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const int cc = 32 * cq + 8 * b + 2 * tt;
-                        float o0 = __uint_as_float(o16[4 * b + 2 * rr]), o1 = __uint_as_float(o16[4 * b + 2 * rr + 1]);
-                        if (p.has_gate) {
-                            const float2 ga = unpack_bf16(gpre[4 * rr + b]);
-                            o0 *= sigmoid_fast(ga.x);
-                            o1 *= sigmoid_fast(ga.y);
-                        }
-                        if (p.out_f32) {   // staging fp32 [64][128], 16-byte chunks XOR-swizzled by row
-                            sts64(base + kL + i * 512 + ((((cc >> 2) ^ (i & 7))) << 4) + (cc & 3) * 4, __float_as_uint(o0), __float_as_uint(o1));
-                        } else {           // staging bf16 [64][128]
-                            sts32(base + kL + i * 256 + ((((cc >> 3) ^ (i & 7))) << 4) + (cc & 7) * 2, pack_bf16(o0, o1));
-                        }
+                for (int b = 0; b < 4; ++b) {
+                    const int cc = 32 * cq + 8 * b + 2 * t4;
+                    float o0 = __uint_as_float(oq[4 * b + 2 * rr]) + __uint_as_float(ok[4 * b + 2 * rr]);
+                    float o1 = __uint_as_float(oq[4 * b + 2 * rr + 1]) + __uint_as_float(ok[4 * b + 2 * rr + 1]);
+                    if (p.has_gate) {
+                        const float2 ga = unpack_bf16(gpre[4 * rr + b]);
+                        o0 *= sigmoid_fast(ga.x);
+                        o1 *= sigmoid_fast(ga.y);
                     }
+                    if (p.out_f32) sts64(base + kL + out_off_f32(i, cc), __float_as_uint(o0), __float_as_uint(o1));
+                    else sts32(base + kL + in_off(i, cc), pack_bf16(o0, o1));
                 }
             }
         }
+        fence_async_smem();
         tc_fence_before();
         bar_all();
         tc_fence_after();
-        // rows < L of the staged output -> global, two rows per warp instruction
-        if (p.out_f32) {
-            float *outp = static_cast<float *>(p.out);
-            for (int e = tid; e < 64 * 32; e += kThreads) {
-                const int i = e >> 5, chk = e & 31;
-                if (i < L) {
-                    const uint4 x = lds128(base + kL + i * 512 + ((chk ^ (i & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(outp + ((t0 + i) * H + h) * kD + 4 * chk) = x;
+        if (L == kChunk) {
+            // a whole chunk: TMA stores of the staged tile (the staging area is next written in the
+            // next chunk's pass 2, after the issuing thread has waited for these reads)
+            if (leader) {
+                if (p.out_f32) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) tma_store_box(&maps.out, base + kL + 8192 * j, 32 * j, h, (int)t0);
+                } else {
+                    tma_store_box(&maps.out, base + kL, 0, h, (int)t0);
+                    tma_store_box(&maps.out, base + kL + 8192, 64, h, (int)t0);
                 }
+                bulk_commit();
             }
         } else {
-            uint16_t *outp = static_cast<uint16_t *>(p.out);
-            for (int e = tid; e < 64 * 16; e += kThreads) {
-                const int i = e >> 4, chk = e & 15;
-                if (i < L) {
-                    const uint4 x = lds128(base + kL + i * 256 + ((chk ^ (i & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(outp + ((t0 + i) * H + h) * kD + 8 * chk) = x;
+            // rows < L of the staged output -> global, 16 bytes per thread and step
+            if (p.out_f32) {
+                float *outp = static_cast<float *>(p.out);
+                for (int e = tid; e < 64 * 32; e += kThreads) {
+                    const int i = e >> 5, chk = e & 31;
+                    if (i < L)
+                        *reinterpret_cast<uint4 *>(outp + ((t0 + i) * H + h) * kD + 4 * chk) = lds128(base + kL + out_off_f32(i, 4 * chk));
+                }
+            } else {
+                uint16_t *outp = static_cast<uint16_t *>(p.out);
+                for (int e = tid; e < 64 * 16; e += kThreads) {
+                    const int i = e >> 4, chk = e & 15;
+                    if (i < L)
+                        *reinterpret_cast<uint4 *>(outp + ((t0 + i) * H + h) * kD + 8 * chk) = lds128(base + kL + in_off(i, 8 * chk));
                 }
             }
+            bar_all();   // the staging area is next written in the next chunk's pass 2
         }
-        bar_all();   // the staging area (kL) is rewritten by the next chunk's step 8
     }
 
+    if (leader) bulk_wait_all();
     if (*abort_flag && leader) {
         // copies issued but never waited for complete before the CTA leaves (bounded)
         for (int i = 0; i < 4; ++i)
