@@ -103,6 +103,12 @@ static_assert(kGB + 3 * 8192 <= kS && kGB + 96 * 256 <= kS, "GB region");
 __host__ __device__ constexpr int qslot(int i) { return 32 * (i >> 4) + (i & 15); }
 __host__ __device__ constexpr int kslot(int i) { return 32 * (i >> 4) + 16 + (i & 15); }
 
+// ---- value-channel order of every N = d_v operand and accumulator (V, U~, U, S, O) ---------------
+// Within each block of 32 value channels, column n = 8b + 2t + e (b, t < 4, e < 2) holds channel
+// 8t + 2b + e.  A 16x256b TMEM load gives lane (g, t) the columns 8b + 2t + e, b = 0..3: eight
+// consecutive channels 8t .. 8t + 7, so the gate is read and the output written 16 bytes at a time.
+__host__ __device__ constexpr int vperm(int n) { return 8 * ((n >> 1) & 3) + 2 * ((n >> 3) & 3) + (n & 1); }
+
 // ---- tensor memory columns -----------------------------------------------------------------------
 constexpr uint32_t cWU = 0;        // [W | U~] -> [. | U] (key slots), [. | O] (query slots); 256 columns
 constexpr uint32_t cGA = 0;        // fp16 row-scaled rows (A operand of the off-diagonal Gram), 64 cols
@@ -404,18 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
 #pragma unroll
             for (int j = 0; j < 32; ++j) x[j] = 0.f;
         }
+        float xp[32];   // in the column order of the value channels
+#pragma unroll
+        for (int j = 0; j < 32; ++j) xp[j] = x[vperm(j)];
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
             uint32_t v[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(x[16 * part + e]);
+            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(xp[16 * part + e]);
             tmem_st16(tq + cS + 32 * cq + 16 * part, v);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             sts128(base + kS + bmn_off(row, 32 * cq + 8 * j),
-                   make_uint4(pack_f16(x[8 * j], x[8 * j + 1]), pack_f16(x[8 * j + 2], x[8 * j + 3]),
-                              pack_f16(x[8 * j + 4], x[8 * j + 5]), pack_f16(x[8 * j + 6], x[8 * j + 7])));
+                   make_uint4(pack_f16(xp[8 * j], xp[8 * j + 1]), pack_f16(xp[8 * j + 2], xp[8 * j + 3]),
+                              pack_f16(xp[8 * j + 4], xp[8 * j + 5]), pack_f16(xp[8 * j + 6], xp[8 * j + 7])));
         tmem_wait_st();
     }
 
@@ -647,19 +656,30 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 sts64(base + kK + oq1, pack_f16(kr[1][0] * tev[0], kr[1][1] * tev[1]), pack_f16(kr[1][2] * tev[2], kr[1][3] * tev[3]));
                 sts64(aBuf + oq0, pack_f16(kt[0][0] * tkv[0], kt[0][1] * tkv[1]), pack_f16(kt[0][2] * tkv[2], kt[0][3] * tkv[3]));
                 sts64(aBuf + oq1, pack_f16(kt[1][0] * tkv[0], kt[1][1] * tkv[1]), pack_f16(kt[1][2] * tkv[2], kt[1][3] * tkv[3]));
-                // V -> fp16 (rows past the end -> 0), by the warps of the last tile for all four tiles: they
-                // have no rescaled keys to write for later tiles, so this evens out the schedulers' work
-                if (pt == 3) {
+            }
+            // V -> fp16 in the value-channel column order (rows past the end -> 0), by the warps of
+            // the last tile: they have no rescaled keys to write for later tiles, so this evens out the
+            // schedulers' work.  Lane = rows lane and lane + 32 of channel block cq; output chunk b
+            // (columns 8b .. 8b + 7) takes word b of each of the four source chunks.
+            if (pt == 3) {
 #pragma unroll
-                    for (int tb = 0; tb < 4; ++tb) {
-                        const uint32_t ov = oq0 - 3 * 2048 + tb * 2048;   // rows 16 tb + g and + 8
-                        uint2 v0 = lds64(base + kV + ov), v1 = lds64(base + kV + ov + 1024);
-                        if (partial) {
-                            if (16 * tb + g >= L) v0 = make_uint2(0, 0);
-                            if (16 * tb + g + 8 >= L) v1 = make_uint2(0, 0);
-                        }
-                        sts64(base + kV + ov, bf16x2_to_f16x2(v0.x), bf16x2_to_f16x2(v0.y));
-                        sts64(base + kV + ov + 1024, bf16x2_to_f16x2(v1.x), bf16x2_to_f16x2(v1.y));
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int i = lane + 32 * rr;
+                    uint4 src[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) src[j] = lds128(base + kV + in_off(i, 32 * cq + 8 * j));
+                    if (partial && i >= L) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) src[j] = make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const uint32_t w0 = b == 0 ? src[0].x : b == 1 ? src[0].y : b == 2 ? src[0].z : src[0].w;
+                        const uint32_t w1 = b == 0 ? src[1].x : b == 1 ? src[1].y : b == 2 ? src[1].z : src[1].w;
+                        const uint32_t w2 = b == 0 ? src[2].x : b == 1 ? src[2].y : b == 2 ? src[2].z : src[2].w;
+                        const uint32_t w3 = b == 0 ? src[3].x : b == 1 ? src[3].y : b == 2 ? src[3].z : src[3].w;
+                        sts128(base + kV + in_off(i, 32 * cq + 8 * b),
+                               make_uint4(bf16x2_to_f16x2(w0), bf16x2_to_f16x2(w1), bf16x2_to_f16x2(w2), bf16x2_to_f16x2(w3)));
                     }
                 }
             }
@@ -932,19 +952,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
-        // meanwhile: this thread's gate logits (rows 16 q4 + g and + 8, column pairs 32 cq + 8b + 2t4)
-        uint32_t gpre[8];
-        {
-            const int gg = lane >> 2, tt = lane & 3;
+        // meanwhile: this thread's gate logits, tokens 16 q4 + g and + 8, channels 32 cq + 8 t4 .. + 7
+        uint4 gpre[2];
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int i = 16 * q4 + gg + 8 * rr;
-#pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    gpre[4 * rr + b] = (p.has_gate && i < L)
-                        ? __ldg(reinterpret_cast<const uint32_t *>(p.gate + ((t0 + i) * H + h) * kD + 32 * cq + 8 * b + 2 * tt))
-                        : 0u;
-            }
+        for (int rr = 0; rr < 2; ++rr) {
+            const int i = 16 * q4 + g + 8 * rr;
+            gpre[rr] = (p.has_gate && i < L)
+                ? __ldg(reinterpret_cast<const uint4 *>(p.gate + ((t0 + i) * H + h) * kD + 32 * cq + 8 * t4))
+                : make_uint4(0, 0, 0, 0);
         }
         mma_sync();
         if (*abort_flag) break;
@@ -953,27 +968,35 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             uint32_t v[32];
             tld32(tq + cS + 32 * cq, v);
             store_b32(base + kS, row, v, 1.f);
-            // tokens 16 q4 + g and + 8 (lane (g, t4)), columns 32 cq + 8b + 2t4, + 1: query slots
-            // (Q^ S + A_hi U) plus key slots (A_lo U)
+            // tokens 16 q4 + g and + 8 (lane (g, t4)), columns 32 cq + 8b + 2t4 + e = channels
+            // 32 cq + 8 t4 + 2b + e: query slots (Q^ S + A_hi U) plus key slots (A_lo U)
             uint32_t oq[16], ok[16];
             tmem_ld_frag4(tq + cWU + 128 + 32 * cq, oq);
             tmem_ld_frag4(tq + (16u << 16) + cWU + 128 + 32 * cq, ok);
             tmem_wait_ld();
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
-                const int i = 16 * q4 + g + 8 * rr;
+                const int i = 16 * q4 + g + 8 * rr, cc = 32 * cq + 8 * t4;
+                const uint32_t gw[4] = {gpre[rr].x, gpre[rr].y, gpre[rr].z, gpre[rr].w};
+                float o[8];
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
-                    const int cc = 32 * cq + 8 * b + 2 * t4;
-                    float o0 = __uint_as_float(oq[4 * b + 2 * rr]) + __uint_as_float(ok[4 * b + 2 * rr]);
-                    float o1 = __uint_as_float(oq[4 * b + 2 * rr + 1]) + __uint_as_float(ok[4 * b + 2 * rr + 1]);
+                    o[2 * b] = __uint_as_float(oq[4 * b + 2 * rr]) + __uint_as_float(ok[4 * b + 2 * rr]);
+                    o[2 * b + 1] = __uint_as_float(oq[4 * b + 2 * rr + 1]) + __uint_as_float(ok[4 * b + 2 * rr + 1]);
                     if (p.has_gate) {
-                        const float2 ga = unpack_bf16(gpre[4 * rr + b]);
-                        o0 *= sigmoid_fast(ga.x);
-                        o1 *= sigmoid_fast(ga.y);
+                        const float2 ga = unpack_bf16(gw[b]);
+                        o[2 * b] *= sigmoid_fast(ga.x);
+                        o[2 * b + 1] *= sigmoid_fast(ga.y);
                     }
-                    if (p.out_f32) sts64(base + kL + out_off_f32(i, cc), __float_as_uint(o0), __float_as_uint(o1));
-                    else sts32(base + kL + in_off(i, cc), pack_bf16(o0, o1));
+                }
+                if (p.out_f32) {
+                    sts128(base + kL + out_off_f32(i, cc), make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]),
+                                                                      __float_as_uint(o[2]), __float_as_uint(o[3])));
+                    sts128(base + kL + out_off_f32(i, cc + 4), make_uint4(__float_as_uint(o[4]), __float_as_uint(o[5]),
+                                                                          __float_as_uint(o[6]), __float_as_uint(o[7])));
+                } else {
+                    sts128(base + kL + in_off(i, cc), make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
+                                                                 pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7])));
                 }
             }
         }
@@ -1034,11 +1057,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (bad) atomicOr(&g_kda_error_word, kErrRange);
         if (p.S_out) {
             const size_t st_base = ((size_t)n * H + h) * kD * kD;
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[vperm(j)] = __uint_as_float(v[j]);
             float4 *sp = reinterpret_cast<float4 *>(p.S_out + st_base + (size_t)row * kD + 32 * cq);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                sp[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]), __uint_as_float(v[4 * j + 2]),
-                                    __uint_as_float(v[4 * j + 3]));
+            for (int j = 0; j < 8; ++j) sp[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
         }
     }
     tc_fence_before();
