@@ -117,10 +117,12 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, co
  *   - Every call looks up that array's device address (with the calling thread's current device);
  *     the first call on a device loads the library's device code there, so make it before any
  *     stream capture.
- *   - Sizes whose scratch need (kda_chunk_fwd_workspace_min) exceeds 32 MiB are rejected with
- *     KDA_ERR_INVALID_ARG and a message in kda_last_error.  With d_k = d_v = 128 the kernel chosen
- *     by shape needs either no scratch (many units) or at most 49 units' rings (31 MiB), so no
- *     such call is rejected; forcing the cluster kernel (kda_set_prefill_path(1)) allows 50 units.
+ *   - With d_k = d_v = 128 and the kernel left to the shapes (kda_set_prefill_path(0)), a call
+ *     whose cluster-kernel records would exceed 32 MiB (more than 50 units) runs the per-unit
+ *     kernel, which needs no scratch, so no such call is rejected.  Otherwise sizes whose scratch
+ *     need (kda_chunk_fwd_workspace_min) exceeds 32 MiB are rejected with KDA_ERR_INVALID_ARG and a
+ *     message in kda_last_error (forcing the cluster kernel, kda_set_prefill_path(1), allows 50
+ *     units of d = 128).
  *   - Every call on a device shares the one array and nothing in it needs to start at zero, but
  *     calls that overlap on the GPU (different streams, or other threads) race on it: serialise
  *     them, for example by issuing them all on one stream.
@@ -341,7 +343,7 @@ KDA_API uint64_t kda_launch_count(void);
  * both kernels compute the same chunkwise form of "Kimi K3 · Lesson 3 of 14"; they differ only in how
  * the work is spread over the GPU.)
  *   path 0: chosen from the shapes (the default): one CTA per (sequence, head) unit when the units
- *           are at least a third of the SM count, else the cluster kernel;
+ *           are more than three quarters of the SM count, else the cluster kernel;
  *   path 1: the cluster kernel (a unit's chunks spread over d_v/32 CTAs, chunk records in the
  *           caller's workspace);
  *   path 2: one CTA per unit, every intermediate on chip (no workspace).

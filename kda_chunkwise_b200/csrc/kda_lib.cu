@@ -136,14 +136,16 @@ int device_sm_count() {
 }
 
 // The per-unit kernel keeps each unit on one SM (no workspace, no traffic between SMs); the
-// cluster kernel spreads a unit's chunks over four SMs.  With few units the cluster kernel's
-// extra SMs per unit win; once the units fill the device the per-unit kernel does.
-bool use_tc_prefill(int64_t units, int d_k, int d_v) {
+// cluster kernel spreads a unit's chunks over four SMs and runs a unit about 3.2 times faster, but
+// does about 0.8 times the work per SM.  So the cluster kernel wins while it needs at most three
+// waves of four-SM units (units <= 3/4 of the SMs), the per-unit kernel from there on.
+// `path` overrides the process-wide setting when non-zero.
+bool use_tc_prefill(int64_t units, int d_k, int d_v, int path = 0) {
     if (d_k != 128 || d_v != 128) return false;
     if (g_inject_stall.load(std::memory_order_relaxed)) return false;   // the injection targets the cluster kernel
-    const int forced = g_prefill_path.load(std::memory_order_relaxed);
+    const int forced = path ? path : g_prefill_path.load(std::memory_order_relaxed);
     if (forced) return forced == 2;
-    return units * 3 > device_sm_count();
+    return units * 4 > (int64_t)device_sm_count() * 3;
 }
 
 kda_status launch_prefill_tc(const void *q, const void *k, const void *v, const void *a,
@@ -301,13 +303,18 @@ size_t kda_chunk_fwd_workspace_size(int64_t total_tokens, int32_t num_seqs, int3
     return kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
 }
 
-kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *a,
-                         const float *beta, const void *gate, const float *A_log,
-                         const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
-                         int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v, float scale,
-                         const float *initial_state, float *final_state, void *out,
-                         kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
-                         void *stream) {
+}  // extern "C"
+
+namespace {
+
+// kda_chunk_fwd with an optional choice of prefill kernel (0: the process-wide setting)
+kda_status chunk_fwd_impl(const void *q, const void *k, const void *v, const void *a,
+                          const float *beta, const void *gate, const float *A_log,
+                          const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                          int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                          const float *initial_state, float *final_state, void *out,
+                          kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                          void *stream, int path) {
     if (!sizes_ok(total_tokens, num_seqs, max_seqlen, H))
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: negative size or H <= 0");
     if (!supported_dim(d_k) || !supported_dim(d_v))
@@ -327,7 +334,7 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     const void *ptrs4[] = {beta, A_log, cu_seqlens};
     for (const void *ptr : ptrs4)
         if (ptr && !aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: beta/A_log/cu_seqlens not 4-byte aligned");
-    const size_t need = kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
+    const size_t need = use_tc_prefill((int64_t)num_seqs * H, d_k, d_v, path) ? 0 : ring_bytes((int64_t)num_seqs * H, d_k, d_v);
     if (need > 0 && !workspace) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: NULL workspace");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: workspace not 256-byte aligned");
@@ -340,7 +347,7 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: num_seqs * H too large");
     if (total_tokens > 0x7fffffc0LL)
         return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd: total_tokens too large");
-    if (use_tc_prefill(units, d_k, d_v) && total_tokens > 0) {
+    if (use_tc_prefill(units, d_k, d_v, path) && total_tokens > 0) {
         kda::tc::Params tp{};
         tp.beta = beta;
         tp.A_log = A_log;
@@ -388,13 +395,38 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void
     return launch_prefill<64, 64>(p, units, st);
 }
 
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v, const void *a,
+                         const float *beta, const void *gate, const float *A_log,
+                         const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                         int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                         const float *initial_state, float *final_state, void *out,
+                         kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+    return chunk_fwd_impl(q, k, v, a, beta, gate, A_log, cu_seqlens, num_seqs, total_tokens, max_seqlen, H, d_k, d_v,
+                          scale, initial_state, final_state, out, out_dtype, workspace, workspace_bytes, stream, 0);
+}
+
 kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *a,
                                  const float *beta, const void *gate, const float *A_log,
                                  const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                                  int32_t max_seqlen, int32_t H, int32_t d_k, int32_t d_v,
                                  float scale, const float *initial_state, float *final_state,
                                  void *out, kda_dtype out_dtype, void *stream) {
-    const size_t need = kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
+    // With the kernel left to the shapes, sizes whose cluster-kernel records would not fit run the
+    // per-unit kernel, which needs no scratch (d_k = d_v = 128); any other need beyond the array is
+    // rejected.
+    int path = 0;
+    if (g_prefill_path.load(std::memory_order_relaxed) == 0 && sizes_ok(total_tokens, num_seqs, max_seqlen, H) &&
+        kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v) > kStaticScratchBytes &&
+        use_tc_prefill((int64_t)num_seqs * H, d_k, d_v, 2))
+        path = 2;
+    const size_t need = use_tc_prefill((int64_t)num_seqs * H, d_k, d_v, path) || !sizes_ok(total_tokens, num_seqs, max_seqlen, H)
+                            ? 0
+                            : kda_chunk_fwd_workspace_min(total_tokens, num_seqs, max_seqlen, H, d_k, d_v);
     if (need > kStaticScratchBytes)
         return fail(KDA_ERR_INVALID_ARG,
                     "kda_chunk_fwd_noalloc: these sizes need " + std::to_string(need) +
@@ -403,9 +435,8 @@ kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, co
     void *scratch = nullptr;
     const kda_status st = static_scratch_address(&scratch);
     if (st != KDA_OK) return st;
-    return kda_chunk_fwd(q, k, v, a, beta, gate, A_log, cu_seqlens, num_seqs, total_tokens,
-                         max_seqlen, H, d_k, d_v, scale, initial_state, final_state, out,
-                         out_dtype, scratch, kStaticScratchBytes, stream);
+    return chunk_fwd_impl(q, k, v, a, beta, gate, A_log, cu_seqlens, num_seqs, total_tokens, max_seqlen, H, d_k, d_v,
+                          scale, initial_state, final_state, out, out_dtype, scratch, kStaticScratchBytes, stream, path);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *a,

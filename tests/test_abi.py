@@ -55,6 +55,23 @@ def test_workspace_sizes():
     assert small == kda.kda_chunk_fwd_workspace_min(64, 1, 64, 2, 64, 64)
 
 
+def test_prefill_kernel_choice_by_units():
+    # The cluster kernel (1) while the units are at most 3/4 of the SM count, the per-unit kernel (2)
+    # beyond; 148 SMs on B200, and the library assumes 148 when it cannot query a device.
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+    edge = sms * 3 // 4
+    assert kda.kda_prefill_path(edge, 128, 128) == 1
+    assert kda.kda_prefill_path(edge + 1, 128, 128) == 2
+    assert kda.kda_prefill_path(4096, 64, 128) == 1      # other head sizes: the cluster kernel only
+    kda.kda_set_prefill_path(2)
+    try:
+        assert kda.kda_prefill_path(1, 128, 128) == 2
+        assert kda.kda_chunk_fwd_workspace_min(8192, 1, 8192, 32, 128, 128) == 0
+    finally:
+        kda.kda_set_prefill_path(0)
+
+
 def _fwd(**over):
     base = dict(q=16, k=16, v=16, a=16, beta=16, gate=None, A_log=16, cu=16, N=1, T=64,
                 max_seqlen=64, H=2, dk=64, dv=64, scale=1.0, S0=None, SF=None, out=16,

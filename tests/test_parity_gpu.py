@@ -256,10 +256,10 @@ def _report(name, worst):
 @pytest.mark.parametrize("name,count,path", [
     ("prefill_B1_H32_T8192_d128", 32, 0),      # 32 units: the cluster kernel
     ("prefill_B1_H32_T8192_d128", 32, 2),      # the per-unit kernel forced
-    ("saturated_B2_H32_T16384_d128", 16, 0),   # 64 units: the per-unit kernel
-    ("saturated_B2_H32_T16384_d128", 16, 1),   # the cluster kernel forced
+    ("saturated_B2_H32_T16384_d128", 16, 0),   # 64 units: the cluster kernel
+    ("saturated_B2_H32_T16384_d128", 16, 2),   # the per-unit kernel forced
     ("nofade_B2_H32_T16384_d128", 16, 0),
-    ("nofade_B2_H32_T16384_d128", 16, 1),
+    ("nofade_B2_H32_T16384_d128", 16, 2),
 ])
 def test_full_size_prefill(kda, name, count, path):
     w = KI.WORKLOADS[name]

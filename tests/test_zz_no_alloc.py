@@ -57,3 +57,28 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     msg = kda.lib.kda_last_error().decode()
     assert "scratch" in msg and "kda_chunk_fwd" in msg
     assert kda.kda_chunk_fwd_workspace_min(64 * 512, 64, 512, 64, 128, 128) == 0
+
+
+def test_noalloc_runs_the_per_unit_kernel_when_cluster_records_would_not_fit():
+    # 2 sequences x 40 heads = 80 units: by shape the cluster kernel (at most 3/4 of the SM count),
+    # whose records (80 x 648 KiB) exceed the 32 MiB array; with the kernel left to the shapes the
+    # call runs the per-unit kernel instead, so it must equal kda_chunk_fwd on that kernel bit for bit.
+    import kda_chunkwise_b200 as kda
+    w = KI.Workload("noalloc80", (200, 131), 40, 128, 128, A_log="uniform", init_state="normal_0.02", seed=22)
+    inp = KI.make_inputs(w, "cuda")
+    args = (inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"])
+    assert kda.kda_prefill_path(w.num_seqs * w.H, 128, 128) == 1
+    assert kda.kda_chunk_fwd_workspace_min(w.total_tokens, w.num_seqs, 200, w.H, 128, 128) > 32 << 20
+    kda.kda_set_prefill_path(2)
+    try:
+        ref_out, ref_S = kda.kda_chunk_fwd(*args, gate=inp["gate"], initial_state=inp["initial_state"],
+                                           out_dtype=torch.float32)
+        kda.kda_sync_check()
+    finally:
+        kda.kda_set_prefill_path(0)
+    out = torch.full_like(ref_out, float("nan"))
+    S = torch.full_like(ref_S, float("nan"))
+    kda.kda_chunk_fwd_noalloc(*args, max_seqlen=max(w.seqlens), gate=inp["gate"], initial_state=inp["initial_state"],
+                              out=out, final_state=S)
+    kda.kda_sync_check()
+    assert torch.equal(out, ref_out) and torch.equal(S, ref_S)
