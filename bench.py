@@ -45,9 +45,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # the named workload; a prefill row scales it by its own algorithmic bytes (both kernels move
 # traffic in proportion to the token-heads and units they process)
 PREFILL_TRAFFIC = {
-    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 339158528 + 57549824, "src": "2b02c5b4b703dc98"},
-    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1347348000 + 257897216,
-        "src": "2b02c5b4b703dc98"},
+    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 339158528 + 57549824, "src": "0b922cae9af2ce3e"},
+    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1347348000 + 257897216, "src": "@unit"},
 }
 
 NCU_TRAFFIC = {
@@ -77,6 +76,8 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--prefill-path", type=int, default=0, choices=[0, 1, 2],
+                   help="prefill kernel: 0 chosen from the shapes, 1 cluster kernel, 2 per-unit kernel")
     return p.parse_args()
 
 
@@ -131,6 +132,8 @@ def peaks():
 # unchanged since the ncu capture it came from)
 KERNEL_SOURCES = {
     "prefill": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh", "prefill_tc.cuh"),
+    "prefill_cluster": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh"),
+    "prefill_unit": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_tc.cuh"),
     "decode": ("common.cuh", "decode.cuh"),
     "speculative": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "f32x2.cuh", "speculative.cuh"),
     "backward": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "backward.cuh"),
@@ -151,7 +154,7 @@ def prefill_traffic(w, path: int):
     """DRAM bytes of one prefill launch on w, scaled from the committed capture of the same kernel."""
     import kda_inputs as KI
     t = PREFILL_TRAFFIC.get(path)
-    if not t or t["src"] != kernel_source_hash("prefill"):
+    if not t or t["src"] != kernel_source_hash("prefill_cluster" if path == 1 else "prefill_unit"):
         return None, None
     cw = KI.WORKLOADS[t["workload"]]
     scale = prefill_bytes(w) / prefill_bytes(cw)
@@ -391,6 +394,8 @@ def main():
 
     import kda_chunkwise_b200 as kda
     import kda_inputs as KI
+    if args.prefill_path:
+        kda.kda_set_prefill_path(args.prefill_path)
 
     def barrier():
         if world > 1:
