@@ -59,6 +59,7 @@ namespace kda {
 namespace tc {
 
 constexpr int kThreads = 512;
+constexpr int kRankMax = 128;      // batches of at most this many sequences run longest first
 constexpr int kD = 128;            // d_k = d_v of this kernel
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -339,8 +340,25 @@ __device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
 __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __grid_constant__ Maps maps, const Params p) {
     extern __shared__ __align__(1024) unsigned char sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int unit = blockIdx.x;
-    const int n = unit / p.H, h = unit % p.H;
+    // Units in order of decreasing sequence length (ties by index) when the batch is small enough to
+    // rank here: blocks start in index order, so the longest units start first and the last wave
+    // holds the shortest.  Larger batches keep the packed order.
+    const int h = blockIdx.x % p.H;
+    int n = blockIdx.x / p.H;
+    if (p.num_seqs <= kRankMax) {
+        int64_t *len = reinterpret_cast<int64_t *>(sm + kL);
+        int *pick = reinterpret_cast<int *>(sm + kL + 8 * kRankMax);
+        if (tid < p.num_seqs) len[tid] = (int64_t)__ldg(p.cu + tid + 1) - __ldg(p.cu + tid);
+        __syncthreads();
+        if (tid < p.num_seqs) {
+            const int64_t li = len[tid];
+            int r = 0;
+            for (int j = 0; j < p.num_seqs; ++j) r += (len[j] > li) || (len[j] == li && j < tid);
+            if (r == n) *pick = tid;
+        }
+        __syncthreads();
+        n = *pick;
+    }
     const uint32_t base = smem_u32(sm);
     const uint32_t bQ = base + kBar, bKV = bQ + 8, bA0 = bQ + 16, bA1 = bQ + 24, bMma = bQ + 40;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kMisc + 4);
