@@ -30,7 +30,7 @@
 //      tensor, 128-byte swizzle), each issued as soon as its buffer is free; a is double buffered.
 //   1. pass 1 (thread = 2 channels x 8 tokens): g = -5 sigmoid(e^{A_h} a) in log2 units, the
 //      within-tile running sum l, tile totals; tables e^{r_p}, e^{b_C - r_p}, e^{r_p' - r_p}, Gamma_C.
-//      Chunk c + 1's pass 1 runs during chunk c's steps 5 and 7 (while the tensor cores work).
+//      Chunk c + 1's pass 1 runs during chunk c's steps 7 and 9 (while the tensor cores work).
 //   2. pass 2 (warp = tile x channel half, lane = the two rows and 16 channels an MMA fragment
 //      holds): f = 2^l, 1/f; the diagonal Gram blocks (mma.sync tf32); fp16 row-scaled q, k rows into
 //      TMEM (tcgen05.st 16x256b, the fragment layout); rescaled keys of later tiles (fp16) into shared
@@ -715,13 +715,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         }
         sync_tc();
         if (*abort_flag) break;
-        // every thread is past pass 2: the q buffer is free for the next chunk's q
-        if (leader && c + 1 < nchunks) {
-            fence_async_smem();
-            expect_tx(bQ, 16384);
-            load_pair(&maps.q, base + kQ, bQ, c + 1);
-            issued(0, (c + 1) & 1);
-        }
 
         // ---- 3. off-diagonal Gram (TMEM A rows x rescaled keys) ----------------------------------
         if (wq0) {
@@ -731,6 +724,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 for (int k = 0; k < kD / 16; ++k)
                     mma_ts(tmem + cGD, tmem + cGA + 8 * k, sdesc(base + kGB + 256 * k, 128, 2048, 0), id, k > 0);
                 umma_commit(bMma);
+                // every thread is past pass 2: the q buffer is free for the next chunk's q
+                if (c + 1 < nchunks) {
+                    fence_async_smem();
+                    expect_tx(bQ, 16384);
+                    load_pair(&maps.q, base + kQ, bQ, c + 1);
+                    issued(0, (c + 1) & 1);
+                }
             }
             __syncwarp();
         }
@@ -883,17 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
-        if (c + 1 < nchunks) pass1a(c + 1);   // the next chunk's pass 1, first half
         mma_sync();
         if (*abort_flag) break;
-        // k, v buffers are free: the next chunk's k, v
-        if (leader && c + 1 < nchunks) {
-            fence_async_smem();
-            expect_tx(bKV, 32768);
-            load_pair(&maps.k, base + kK, bKV, c + 1);
-            load_pair(&maps.v, base + kV, bKV, c + 1);
-            issued(1, (c + 1) & 1);
-        }
         // ---- 6. -W -> TMEM rows 0-63 of [-W; Q^] ----------------------------------------------------
         {
             uint32_t v[32], w[16];
@@ -915,10 +906,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 for (int k = 0; k < kD / 16; ++k)
                     mma_ts(tmem + cWU + 128, tmem + cWQ + 8 * k, sdesc(base + kS + 4096 * k, 2048, 128, 0), id, 1);
                 umma_commit(bMma);
+                // the k, v buffers were read by step 5 (complete): the next chunk's k, v
+                if (c + 1 < nchunks) {
+                    fence_async_smem();
+                    expect_tx(bKV, 32768);
+                    load_pair(&maps.k, base + kK, bKV, c + 1);
+                    load_pair(&maps.v, base + kV, bKV, c + 1);
+                    issued(1, (c + 1) & 1);
+                }
             }
             __syncwarp();
         }
-        if (c + 1 < nchunks) pass1b();         // the next chunk's pass 1, second half
+        if (c + 1 < nchunks) pass1a(c + 1);   // the next chunk's pass 1, first half
         mma_sync();
         if (*abort_flag) break;
         // ---- 8. U (key slots) -> shared memory (fp16, MN-major B operand) ----------------------------
@@ -970,6 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
+        if (c + 1 < nchunks) pass1b();         // the next chunk's pass 1, second half
         // meanwhile: this thread's gate logits, tokens 16 q4 + g and + 8, channels 32 cq + 8 t4 .. + 7
         uint4 gpre[2];
 #pragma unroll
