@@ -27,21 +27,6 @@
 
 namespace kda {
 
-// The column sums r and p of the four columns of column quad cq: the RPP row-group partials added
-// in row-group order, starting from zero -- the order in which the decode step's column threads
-// add them, so the verify pass (which uses this) reproduces the decode step bit for bit.
-template <int RPP, int LPR>
-__device__ __forceinline__ void quad_col_sums(const float4 (&red)[2][RPP][LPR], int cq, float4 &rr, float4 &pp) {
-    rr = make_float4(0.f, 0.f, 0.f, 0.f);
-    pp = rr;
-#pragma unroll
-    for (int g = 0; g < RPP; ++g) {
-        const float4 a = red[0][g][cq], b = red[1][g][cq];
-        rr.x += a.x; rr.y += a.y; rr.z += a.z; rr.w += a.w;
-        pp.x += b.x; pp.y += b.y; pp.z += b.z; pp.w += b.w;
-    }
-}
-
 constexpr int kSpecMaxTokens = 16;
 constexpr int kSpecThreads = kDecodeThreads;   // the same reduction order as the decode step
 constexpr unsigned kErrBadAccepted = 8u;   // error-word bit: an accepted count outside [0, K]
@@ -60,14 +45,14 @@ struct SpecParams {
 
 // Dynamic shared memory of the verify kernel: the next state (fp32, its global layout), the next
 // unit's raw inputs (bf16 a, k, q [K][DK], v, gate [K][DV]; fp32 beta [K]) and the current unit's
-// derived inputs (alpha, k, scale q [K][DK], v, sigmoid(gate) [K][DV], beta [K], k . scale q [K],
-// fp32).
+// derived inputs ({alpha, k, scale q, 0} [K][DK] as float4, v, sigmoid(gate) [K][DV], beta [K],
+// k . scale q [K], fp32).
 template <int DK, int DV>
 struct SpecVerifySmem {
     __host__ __device__ static size_t raw_off() { return (size_t)DK * DV * 4; }
     __host__ __device__ static size_t beta_off(int K) { return raw_off() + (size_t)K * (3 * DK + 2 * DV) * 2; }
     __host__ __device__ static size_t derived_off(int K) { return beta_off(K) + (size_t)((K + 3) & ~3) * 4; }
-    __host__ __device__ static size_t bytes(int K) { return derived_off(K) + (size_t)K * (3 * DK + 2 * DV + 2) * 4; }
+    __host__ __device__ static size_t bytes(int K) { return derived_off(K) + (size_t)K * (4 * DK + 2 * DV + 2) * 4; }
 };
 
 // Persistent: a CTA takes units blockIdx.x, blockIdx.x + gridDim.x, ...; while it runs the K token
@@ -87,10 +72,12 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
     const uint16_t *r_a = reinterpret_cast<const uint16_t *>(spec_dyn + SL::raw_off());
     const uint16_t *r_k = r_a + K * DK, *r_q = r_k + K * DK, *r_v = r_q + K * DK, *r_g = r_v + K * DV;
     const float *r_beta = reinterpret_cast<const float *>(spec_dyn + SL::beta_off(K));
-    float *s_alpha = reinterpret_cast<float *>(spec_dyn + SL::derived_off(K));
-    float *s_k = s_alpha + K * DK, *s_q = s_k + K * DK, *s_v = s_q + K * DK, *s_sg = s_v + K * DV;
+    float4 *s_akq = reinterpret_cast<float4 *>(spec_dyn + SL::derived_off(K));   // {alpha, k, scale q, 0}
+    float *s_v = reinterpret_cast<float *>(s_akq + K * DK), *s_sg = s_v + K * DV;
     float *s_b = s_sg + K * DV, *s_kqt = s_b + K;
-    __shared__ float4 s_red[2][2][RPP][LPR];   // two buffers: consecutive tokens alternate
+    // per token: the row groups' partial column sums, then the sums ([r or p][column quad])
+    __shared__ float4 s_red[2][RPP][LPR];
+    __shared__ float4 s_sum[2][LPR];
 
     const int tid = threadIdx.x;
     const int cq = tid % LPR, rg = tid / LPR;
@@ -128,11 +115,9 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
 #pragma unroll
         for (int m = 0; m < NR; ++m) S[m] = reinterpret_cast<const ulonglong2 *>(sS)[(rg + m * RPP) * LPR + cq];
         const float expA = expf(p.A_log[h]);
-        for (int e = tid; e < K * DK; e += kThreads) {
-            s_alpha[e] = __expf(log_decay(bf16_to_f32(r_a[e]), expA));
-            s_k[e] = bf16_to_f32(r_k[e]);
-            s_q[e] = p.scale * bf16_to_f32(r_q[e]);
-        }
+        for (int e = tid; e < K * DK; e += kThreads)
+            s_akq[e] = make_float4(__expf(log_decay(bf16_to_f32(r_a[e]), expA)), bf16_to_f32(r_k[e]),
+                                   p.scale * bf16_to_f32(r_q[e]), 0.f);
         for (int e = tid; e < K * DV; e += kThreads) {
             s_v[e] = bf16_to_f32(r_v[e]);
             if (p.gate) s_sg[e] = sigmoid_fast(bf16_to_f32(r_g[e]));
@@ -142,7 +127,10 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
         for (int t = tid >> 5; t < K; t += kThreads / 32) {   // k . scale q per token, as the decode step
             const int lane = tid & 31;
             float acc = 0.f;
-            for (int i = lane; i < DK; i += 32) acc = fmaf(s_k[t * DK + i], s_q[t * DK + i], acc);
+            for (int i = lane; i < DK; i += 32) {
+                const float4 akq = s_akq[t * DK + i];
+                acc = fmaf(akq.y, akq.z, acc);
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
             if (lane == 0) s_kqt[t] = acc;
@@ -156,8 +144,8 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
                 const int row = rg + m * RPP;
-                const f32x2 al = f2_splat(s_alpha[t * DK + row]);
-                const f32x2 kk = f2_splat(s_k[t * DK + row]), qq = f2_splat(s_q[t * DK + row]);
+                const float4 akq = s_akq[t * DK + row];
+                const f32x2 al = f2_splat(akq.x), kk = f2_splat(akq.y), qq = f2_splat(akq.z);
                 S[m].x = f2_mul(S[m].x, al);
                 S[m].y = f2_mul(S[m].y, al);
                 r.x = f2_fma(kk, S[m].x, r.x);
@@ -165,12 +153,23 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
                 pq.x = f2_fma(qq, S[m].x, pq.x);
                 pq.y = f2_fma(qq, S[m].y, pq.y);
             }
-            float4 (&red)[2][RPP][LPR] = s_red[t & 1];
-            reinterpret_cast<ulonglong2 &>(red[0][rg][cq]) = r;
-            reinterpret_cast<ulonglong2 &>(red[1][rg][cq]) = pq;
+            reinterpret_cast<ulonglong2 &>(s_red[0][rg][cq]) = r;
+            reinterpret_cast<ulonglong2 &>(s_red[1][rg][cq]) = pq;
             __syncthreads();   // (the k . q of every token is ready too)
-            float4 rr, pp;
-            quad_col_sums<RPP, LPR>(red, cq, rr, pp);
+            // the column sums, once per column quad (2 x LPR threads), in row-group order from zero
+            // as the decode step adds them; then every thread reads its own
+            if (tid < 2 * LPR) {
+                const int w = tid / LPR, c4 = tid % LPR;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int g = 0; g < RPP; ++g) {
+                    const float4 x = s_red[w][g][c4];
+                    acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+                }
+                s_sum[w][c4] = acc;
+            }
+            __syncthreads();
+            const float4 rr = s_sum[0][cq], pp = s_sum[1][cq];
             const float bt = s_b[t];
             const float4 v4 = reinterpret_cast<const float4 *>(s_v + t * DV)[cq];
             const float4 u4 = make_float4(bt * (v4.x - rr.x), bt * (v4.y - rr.y), bt * (v4.z - rr.z), bt * (v4.w - rr.w));
@@ -188,7 +187,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
             const f32x2 u01 = f2_pack(u4.x, u4.y), u23 = f2_pack(u4.z, u4.w);
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
-                const f32x2 kk = f2_splat(s_k[t * DK + rg + m * RPP]);
+                const f32x2 kk = f2_splat(s_akq[t * DK + rg + m * RPP].y);
                 S[m].x = f2_fma(kk, u01, S[m].x);
                 S[m].y = f2_fma(kk, u23, S[m].y);
             }
