@@ -30,7 +30,7 @@
 //      tensor, 128-byte swizzle), each issued as soon as its buffer is free; a is double buffered.
 //   1. pass 1 (thread = 2 channels x 8 tokens): g = -5 sigmoid(e^{A_h} a) in log2 units, the
 //      within-tile running sum l, tile totals; tables e^{r_p}, e^{b_C - r_p}, e^{r_p' - r_p}, Gamma_C.
-//      Chunk c + 1's pass 1 runs during chunk c's steps 7 and 9 (while the tensor cores work).
+//      Chunk c + 1's pass 1 runs during chunk c's steps 5, 7 and 9 (while the tensor cores work).
 //   2. pass 2 (warp = tile x channel half, lane = the two rows and 16 channels an MMA fragment
 //      holds): f = 2^l, 1/f; the diagonal Gram blocks (mma.sync tf32); fp16 row-scaled q, k rows into
 //      TMEM (tcgen05.st 16x256b, the fragment layout); rescaled keys of later tiles (fp16) into shared
@@ -511,25 +511,31 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     //      the tables of the tile references.  Chunk 0's pass 1 runs before the chunk loop; that of
     //      chunk c + 1 runs inside chunk c, while the tensor cores work on chunk c's products.
     const int p1_cp = tid & 63, p1_part = tid >> 6, p1_pt = p1_part >> 1, p1_c0 = 2 * p1_cp;
-    float p1_lx[8], p1_ly[8];
-    auto pass1a = [&](int cl) {
+    float p1_lx[8], p1_ly[8], p1_sx = 0.f, p1_sy = 0.f;
+    // (a) in two halves of four tokens (half 0 waits for the a tile), so that each half fits under
+    // one tensor-core step
+    auto pass1a = [&](int cl, int half) {
         const int64_t tl = s0 + (int64_t)cl * kChunk;
         const int Ll = static_cast<int>(min64(kChunk, s1 - tl));
         const uint32_t ab = (cl & 1) ? base + kA1 : base + kA0;
-        in_wait((cl & 1) ? bA1 : bA0, (cl >> 1) & 1);
-        float sx = 0.f, sy = 0.f;
+        if (half == 0) {
+            in_wait((cl & 1) ? bA1 : bA0, (cl >> 1) & 1);
+            p1_sx = p1_sy = 0.f;
+        }
         constexpr float kG2 = kGMin * kLog2e;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 4 * half; i < 4 * half + 4; ++i) {
             const int t = 8 * p1_part + i;
             const float2 av = unpack_bf16(lds32(ab + in_off(t, p1_c0)));
             float gx = kG2 * sigmoid_fast(expA * av.x), gy = kG2 * sigmoid_fast(expA * av.y);
             if (t >= Ll) gx = gy = 0.f;
-            sx += gx; sy += gy;
-            p1_lx[i] = sx; p1_ly[i] = sy;
+            p1_sx += gx; p1_sy += gy;
+            p1_lx[i] = p1_sx; p1_ly[i] = p1_sy;
         }
-        float *tot = reinterpret_cast<float *>(sm + kTot);   // [8 half tiles][128]
-        *reinterpret_cast<float2 *>(tot + p1_part * 128 + p1_c0) = make_float2(sx, sy);
+        if (half == 1) {
+            float *tot = reinterpret_cast<float *>(sm + kTot);   // [8 half tiles][128]
+            *reinterpret_cast<float2 *>(tot + p1_part * 128 + p1_c0) = make_float2(p1_sx, p1_sy);
+        }
     };
     auto pass1b = [&]() {
         const float *tot = reinterpret_cast<const float *>(sm + kTot);
@@ -569,7 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         }
     };
     if (nchunks > 0) {
-        pass1a(0);
+        pass1a(0, 0);
+        pass1a(0, 1);
         bar_all();
         pass1b();
     }
@@ -582,7 +589,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         beta_next = load_beta(c + 1);
         // the next chunk's a goes into the other buffer (its K- of chunk c-1 is consumed)
         if (leader && c + 1 < nchunks) {
-            fence_async_smem();
             const uint32_t nb = (c & 1) ? base + kA0 : base + kA1, nbar = (c & 1) ? bA0 : bA1;
             expect_tx(nbar, 16384);
             load_pair(&maps.a, nb, nbar, c + 1);
@@ -738,7 +744,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 umma_commit(bMma);
                 // every thread is past pass 2: the q buffer is free for the next chunk's q
                 if (c + 1 < nchunks) {
-                    fence_async_smem();
                     expect_tx(bQ, 16384);
                     load_pair(&maps.q, base + kQ, bQ, c + 1);
                     issued(0, (c + 1) & 1);
@@ -895,6 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
+        if (c + 1 < nchunks) pass1a(c + 1, 0);   // the next chunk's pass 1 (a), first four tokens
         mma_sync();
         if (*abort_flag) break;
         // ---- 6. -W -> TMEM rows 0-63 of [-W; Q^] ----------------------------------------------------
@@ -920,7 +926,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 umma_commit(bMma);
                 // the k, v buffers were read by step 5 (complete): the next chunk's k, v
                 if (c + 1 < nchunks) {
-                    fence_async_smem();
                     expect_tx(bKV, 32768);
                     load_pair(&maps.k, base + kK, bKV, c + 1);
                     load_pair(&maps.v, base + kV, bKV, c + 1);
@@ -929,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             }
             __syncwarp();
         }
-        if (c + 1 < nchunks) pass1a(c + 1);   // the next chunk's pass 1, first half
+        if (c + 1 < nchunks) pass1a(c + 1, 1);   // the next chunk's pass 1 (a), last four tokens
         mma_sync();
         if (*abort_flag) break;
         // ---- 8. U (key slots) -> shared memory (fp16, MN-major B operand) ----------------------------
