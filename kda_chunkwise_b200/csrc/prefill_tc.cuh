@@ -35,7 +35,8 @@
 //      holds): f = 2^l, 1/f; the diagonal Gram blocks (mma.sync tf32); fp16 row-scaled q, k rows into
 //      TMEM (tcgen05.st 16x256b, the fragment layout); rescaled keys of later tiles (fp16) into shared
 //      memory; Q^, K^, K-, V converted in place over the input rows.
-//   3. off-diagonal Gram MMA; meanwhile the state is scaled by Gamma_C in TMEM and Q^ copied to TMEM.
+//   3. off-diagonal Gram MMA; meanwhile the fp16 copy of the state is written (B operand of step 7)
+//      and the state scaled by Gamma_C in TMEM.
 //   4. solve: 16 x 16 diagonal inverses by forward substitution, off-diagonal blocks of T' level by
 //      level (mma.sync); A assembled from the diagonal and off-diagonal Gram blocks.
 //   5. D[0:64] = [T'; 0] [K^ | V] = [W | U~]                         (tcgen05, N = 256, K = 64)
@@ -43,8 +44,8 @@
 //   7. D[:, 128:256] += [-W; Q^] S   -> rows 0-63 U, rows 64-127 Q^ S  (tcgen05, A in TMEM)
 //   8. U -> shared memory (fp16 value and remainder); its TMEM rows zeroed
 //   9. S += K-^T U  (S pre-scaled by Gamma_C);  D[:, 128:256] += [A_hi; A_lo] U -> O in two parts
-//  10. fp16 copy of the new S; out = sigmoid(gate) O (gate logits read from global memory during
-//      step 9), staged in shared memory, stored by TMA (row by row for a sequence's last chunk).
+//  10. out = sigmoid(gate) O (gate logits read from global memory during step 9), staged in shared
+//      memory, stored by TMA (row by row for a sequence's last chunk).
 // Every wait on a TMA or MMA completion is bounded (%globaltimer); a timeout records kErrTimeout in
 // the device error word and every thread leaves the chunk loop at the next barrier.
 #pragma once
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     const int q4 = warp & 3, cq = warp >> 2, row = 32 * q4 + lane;
     const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
 
-    // initial state -> TMEM (fp32) and its fp16 copy (B operand)
+    // initial state -> TMEM (fp32; step 3 writes its fp16 copy)
     {
         const size_t st_base = ((size_t)n * H + h) * kD * kD;
         float x[32];
@@ -450,11 +451,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(xp[16 * part + e]);
             tmem_st16(tq + cS + 32 * cq + 16 * part, v);
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            sts128(base + kS + bmn_off(row, 32 * cq + 8 * j),
-                   make_uint4(pack_f16(xp[8 * j], xp[8 * j + 1]), pack_f16(xp[8 * j + 2], xp[8 * j + 3]),
-                              pack_f16(xp[8 * j + 4], xp[8 * j + 5]), pack_f16(xp[8 * j + 6], xp[8 * j + 7])));
         tmem_wait_st();
     }
 
@@ -789,6 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             const float gam = reinterpret_cast<const float *>(sm + kGam)[row];
             uint32_t v[32];
             tld32(tq + cS + 32 * cq, v);
+            store_b32(base + kS, row, v, 1.f);   // fp16 S_c: the B operand of step 7
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gam * __uint_as_float(v[e]));
             {
@@ -1000,9 +997,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (*abort_flag) break;
         // ---- 10. new S (fp16 copy); gated output rows -----------------------------------------------
         {
-            uint32_t v[32];
-            tld32(tq + cS + 32 * cq, v);
-            store_b32(base + kS, row, v, 1.f);
             // tokens 16 q4 + g and + 8 (lane (g, t4)), columns 32 cq + 8b + 2t4 + e = channels
             // 32 cq + 8 t4 + 2b + e: query slots (Q^ S + A_hi U) plus key slots (A_lo U)
             uint32_t oq[16], ok[16];
