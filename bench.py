@@ -46,7 +46,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # traffic in proportion to the token-heads and units they process)
 PREFILL_TRAFFIC = {
     1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 339158528 + 57549824, "src": "0b922cae9af2ce3e"},
-    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1347348000 + 257897216, "src": "@unit"},
+    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346657000 + 261571584, "src": "96b83a3ec9646b8a"},
 }
 
 NCU_TRAFFIC = {
