@@ -61,6 +61,8 @@ namespace tc {
 
 constexpr int kThreads = 512;
 constexpr int kRankMax = 128;      // batches of at most this many sequences run longest first
+constexpr int kMmaWarp = 6;        // tile 2 (pass 2), channel quarter 1 (Gram step), idle in the solve
+constexpr int kTmaWarp = 10;       // tile 2 (pass 2), channel quarter 2 (Gram step), idle in the solve
 constexpr int kD = 128;            // d_k = d_v of this kernel
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -399,17 +401,19 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     const float expA = expf(p.A_log[h]);
     const int64_t H = p.H;
     float *sbeta = reinterpret_cast<float *>(sm + kBeta);
-    // TMA issue (one elected lane of warp 0; `leader` is that lane)
-    const bool wq0 = warp == 0;
-    const bool leader = wq0 && elect_one();
-    uint32_t pend = 0, pend_par = 0;   // leader only: loads in flight per barrier (q, kv, a0, a1) and their wait parity
+    // One elected lane of warp kMmaWarp issues (and waits for) the tensor-core products, one of warp
+    // kTmaWarp the TMA copies: warps with the least work of their own in pass 2, the Gram step and
+    // the solve, so that the serial issue does not hold up a CTA barrier.
+    const bool mma_lead = warp == kMmaWarp && elect_one();
+    const bool tma_lead = warp == kTmaWarp && elect_one();
+    uint32_t pend = 0, pend_par = 0;   // tma_lead only: loads in flight per barrier (q, kv, a0, a1) and their wait parity
     auto issued = [&](int i, uint32_t parity) { pend |= 1u << i; pend_par = (pend_par & ~(1u << i)) | (parity << i); };
     auto load_pair = [&](const CUtensorMap *map, uint32_t dst, uint32_t bar, int cl) {
         const int t = static_cast<int>(s0 + (int64_t)cl * kChunk);
         tma_box(dst, map, 0, h, t, bar);
         tma_box(dst + 8192, map, 64, h, t, bar);
     };
-    if (leader && nchunks > 0) {
+    if (tma_lead && nchunks > 0) {
         expect_tx(bA0, 16384); load_pair(&maps.a, base + kA0, bA0, 0); issued(2, 0);
         expect_tx(bQ, 16384); load_pair(&maps.q, base + kQ, bQ, 0); issued(0, 0);
         expect_tx(bKV, 32768); load_pair(&maps.k, base + kK, bKV, 0); load_pair(&maps.v, base + kV, bKV, 0); issued(1, 0);
@@ -457,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
     uint32_t mma_phase = 0;
     auto mma_wait = [&]() {   // the issuing thread waits for the latest commit (bounded); the CTA
                               // barrier that follows every call releases the others
-        if (leader && !wait_bounded(bMma, mma_phase, p.wait_ns)) {
+        if (mma_lead && !wait_bounded(bMma, mma_phase, p.wait_ns)) {
             atomicOr(&g_kda_error_word, kErrTimeout);
             *abort_flag = 1;
         }
@@ -584,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (tid < 64) sbeta[tid] = beta_next;
         beta_next = load_beta(c + 1);
         // the next chunk's a goes into the other buffer (its K- of chunk c-1 is consumed)
-        if (leader && c + 1 < nchunks) {
+        if (tma_lead && c + 1 < nchunks) {
             const uint32_t nb = (c & 1) ? base + kA0 : base + kA1, nbar = (c & 1) ? bA0 : bA1;
             expect_tx(nbar, 16384);
             load_pair(&maps.a, nb, nbar, c + 1);
@@ -592,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         }
         in_wait(bQ, c & 1);
         in_wait(bKV, c & 1);
-        if (leader) bulk_wait_read();   // the previous chunk's output stores have read the staging area
+        if (tma_lead) bulk_wait_read();   // the previous chunk's output stores have read the staging area
         bar_all();
         if (*abort_flag) break;
 
@@ -731,21 +735,21 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (*abort_flag) break;
 
         // ---- 3. off-diagonal Gram (TMEM A rows x rescaled keys) ----------------------------------
-        if (wq0) {
-            if (leader) {
+        if (warp == kMmaWarp) {
+            if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 96, 0, 0);
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k)
                     mma_ts(tmem + cGD, tmem + cGA + 8 * k, sdesc(base + kGB + 256 * k, 128, 2048, 0), id, k > 0);
                 umma_commit(bMma);
-                // every thread is past pass 2: the q buffer is free for the next chunk's q
-                if (c + 1 < nchunks) {
-                    expect_tx(bQ, 16384);
-                    load_pair(&maps.q, base + kQ, bQ, c + 1);
-                    issued(0, (c + 1) & 1);
-                }
             }
             __syncwarp();
+        }
+        // every thread is past pass 2: the q buffer is free for the next chunk's q
+        if (tma_lead && c + 1 < nchunks) {
+            expect_tx(bQ, 16384);
+            load_pair(&maps.q, base + kQ, bQ, c + 1);
+            issued(0, (c + 1) & 1);
         }
         if (cq == 0) {
 #pragma unroll
@@ -887,8 +891,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         sync_tc();   // T' visible to the tensor core
 
         // ---- 5. [W | U~] = [T'; 0] [K^ | V] ---------------------------------------------------------
-        if (wq0) {
-            if (leader) {
+        if (warp == kMmaWarp) {
+            if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 256, 0, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
@@ -914,22 +918,22 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         }
         sync_tc();
         // ---- 7. D[:, 128:256] += [-W; Q^] S --------------------------------------------------------
-        if (wq0) {
-            if (leader) {
+        if (warp == kMmaWarp) {
+            if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 128, 0, 1);
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k)
                     mma_ts(tmem + cWU + 128, tmem + cWQ + 8 * k, sdesc(base + kS + 4096 * k, 2048, 128, 0), id, 1);
                 umma_commit(bMma);
-                // the k, v buffers were read by step 5 (complete): the next chunk's k, v
-                if (c + 1 < nchunks) {
-                    expect_tx(bKV, 32768);
-                    load_pair(&maps.k, base + kK, bKV, c + 1);
-                    load_pair(&maps.v, base + kV, bKV, c + 1);
-                    issued(1, (c + 1) & 1);
-                }
             }
             __syncwarp();
+        }
+        // the k, v buffers were read by step 5 (complete): the next chunk's k, v
+        if (tma_lead && c + 1 < nchunks) {
+            expect_tx(bKV, 32768);
+            load_pair(&maps.k, base + kK, bKV, c + 1);
+            load_pair(&maps.v, base + kV, bKV, c + 1);
+            issued(1, (c + 1) & 1);
         }
         if (c + 1 < nchunks) pass1a(c + 1, 1);   // the next chunk's pass 1 (a), last four tokens
         mma_sync();
@@ -967,8 +971,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         //      query slots and A_lo in the key slots, so A'' (U_hi + U_lo) leaves Q^ S + A_hi U in the
         //      query slots and A_lo U in the (zeroed) key slots; the epilogue adds the two (the
         //      state's K-^T U takes U_hi only: its rounding there does not show)
-        if (wq0) {
-            if (leader) {
+        if (warp == kMmaWarp) {
+            if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 128, 1, 1), id2 = idesc(128, 128, 0, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
@@ -1036,7 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (L == kChunk) {
             // a whole chunk: TMA stores of the staged tile (the staging area is next written in the
             // next chunk's pass 2, after the issuing thread has waited for these reads)
-            if (leader) {
+            if (tma_lead) {
                 if (p.out_f32) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) tma_store_box(&maps.out, base + kL + 8192 * j, 32 * j, h, (int)t0);
@@ -1067,13 +1071,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         }
     }
 
-    if (leader) bulk_wait_all();
-    if (*abort_flag && leader) {
-        // copies issued but never waited for complete before the CTA leaves (bounded)
+    if (tma_lead) bulk_wait_all();
+    // copies and products issued but never waited for complete before the CTA leaves (bounded)
+    if (*abort_flag && tma_lead) {
         for (int i = 0; i < 4; ++i)
             if (pend >> i & 1) wait_bounded(bQ + 8 * i, pend_par >> i & 1, p.wait_ns);
-        wait_bounded(bMma, mma_phase ^ 1, p.wait_ns);
     }
+    if (*abort_flag && mma_lead) wait_bounded(bMma, mma_phase ^ 1, p.wait_ns);
     // final state (fp32, from TMEM).  An fp16 operand that overflowed (state, pseudo-values, values
     // beyond +-65504) becomes inf and reaches the fp32 state, where no fade can remove it: a
     // non-finite final state flags the unit.
