@@ -311,7 +311,11 @@ KDA_API kda_status kda_chunk_bwd_chunkwise(const void *q, const void *k, const v
                                            void *stream);
 
 /* Workspace of kda_chunk_bwd_chunkwise (host-only; 0 on invalid sizes): one record of the chunk's
- * operands, states and state gradients per (64-token chunk, head). */
+ * operands, states and state gradients per (64-token chunk, head), (total_tokens / 64 + num_seqs)
+ * x H records of 410,112 bytes at d_k = d_v = 128 (196,864 at 64): 1.69 GB for 8192 tokens x 32
+ * heads, 215 GB for one 1 M-token sequence x 32 heads, more than one B200 holds -- use kda_chunk_bwd
+ * (66 KiB per 32 tokens and head) for long sequences.  Deterministic except dA_log, which is summed
+ * with float atomics over chunks, so its last bits can vary between runs. */
 KDA_API size_t kda_chunk_bwd_chunkwise_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H,
                                                       int32_t d_k, int32_t d_v);
 
