@@ -1,4 +1,5 @@
-// Backward pass of the KDA recurrence in chunkwise form (64-token chunks), fp32 on the CUDA cores.
+// Backward pass of the KDA recurrence in chunkwise form (64-token chunks): the products on the tensor
+// cores (tf32 with hi/lo operand splits, fp32-accurate), the rest in fp32 on the CUDA cores.
 //
 // Per chunk with incoming state S0, b the chunk-local running sum of g, Gamma = e^b, Gamma_C its last
 // row, the forward is  Q^ = Gamma (.) scale q, K^ = Gamma (.) k, K- = (Gamma_C / Gamma) (.) k,
@@ -49,46 +50,100 @@ struct BcRec {
     static constexpr size_t kSize = kdO + C * DV;
 };
 
-// C (M x N, row stride ldc) = alpha opA (M x K) opB (K x N) [+ C], by the whole CTA: a 16 x 16 grid
-// of threads, thread (ti, tj) holding rows ti + 16 x and columns tj + 16 y.
+// Shared-memory staging of bc_gemm: a k-slice of 16 of opA ([M][16 + 4]) and of opB ([16][N + 8]),
+// padded so that the fragment reads below are free of bank conflicts.
+constexpr int kBcKs = 16;
+constexpr int kBcStageFloats = 128 * (kBcKs + 4) + kBcKs * (128 + 8);
+
+__device__ __forceinline__ uint32_t bc_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void bc_mma_tf32(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// C (M x N, row stride ldc) = alpha opA (M x K) opB (K x N) [+ C], by the whole CTA (8 warps) on the
+// tensor cores: mma.sync m16n8k8 in tf32 on operands split as x = hi + lo (both tf32), summing
+// lo*hi + hi*lo + hi*hi, which keeps fp32's accuracy to about 2^-21 of each product.  The operands
+// (global or shared memory, any row strides) are staged 16 values of K at a time in `stage`
+// (kBcStageFloats floats of shared memory) with coalesced loads.  Warp w takes row block
+// w / (8 / (M / 16)) and a run of N / 8 / (8 / (M / 16)) column blocks of 8.
 // opA(i, k) = TA ? A[k lda + i] : A[i lda + k];  opB(k, j) = TB ? B[j ldb + k] : B[k ldb + j].
+// Contains CTA barriers: every thread calls it, and it begins with one, so the operands' writers
+// need no barrier of their own before the call (the caller still needs one after it before C is
+// read by other threads).
 template <int M, int N, int K, bool TA, bool TB>
 __device__ __forceinline__ void bc_gemm(const float *A, int lda, const float *B, int ldb, float *Cm, int ldc,
-                                        float alpha, bool accumulate) {
-    constexpr int RM = M / 16, RN = N / 16;
-    static_assert(M % 16 == 0 && N % 16 == 0, "tile");
-    const int ti = threadIdx.x / 16, tj = threadIdx.x % 16;
-    float c[RM][RN];
+                                        float alpha, bool accumulate, float *stage) {
+    constexpr int LA = kBcKs + 4, LB = N + 8;
+    constexpr int TM = M / 16, TN = N / 8, WPM = 8 / TM, NPW = TN / WPM;
+    static_assert(M % 16 == 0 && N % 8 == 0 && K % kBcKs == 0 && TM <= 8 && 8 % TM == 0 && TN % WPM == 0, "shape");
+    static_assert(M * LA + kBcKs * LB <= kBcStageFloats, "stage");
+    float *As = stage, *Bs = stage + M * LA;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
+    const int mt = warp / WPM, nt0 = (warp % WPM) * NPW;
+    float acc[NPW][4];
 #pragma unroll
-    for (int x = 0; x < RM; ++x)
-#pragma unroll
-        for (int y = 0; y < RN; ++y) c[x][y] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < K; ++k) {
-        float av[RM], bv[RN];
-#pragma unroll
-        for (int x = 0; x < RM; ++x) {
-            const int i = ti + 16 * x;
-            av[x] = TA ? A[(size_t)k * lda + i] : A[(size_t)i * lda + k];
+    for (int u = 0; u < NPW; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+    for (int k0 = 0; k0 < K; k0 += kBcKs) {
+        __syncthreads();   // the previous slice is consumed; on entry, the operands are written
+        for (int e = threadIdx.x; e < M * kBcKs; e += kBcThreads) {
+            if (TA) {
+                const int kk = e / M, i = e % M;
+                As[i * LA + kk] = A[(size_t)(k0 + kk) * lda + i];
+            } else {
+                const int i = e / kBcKs, kk = e % kBcKs;
+                As[i * LA + kk] = A[(size_t)i * lda + k0 + kk];
+            }
         }
-#pragma unroll
-        for (int y = 0; y < RN; ++y) {
-            const int j = tj + 16 * y;
-            bv[y] = TB ? B[(size_t)j * ldb + k] : B[(size_t)k * ldb + j];
+        for (int e = threadIdx.x; e < kBcKs * N; e += kBcThreads) {
+            if (TB) {
+                const int j = e / kBcKs, kk = e % kBcKs;
+                Bs[kk * LB + j] = B[(size_t)j * ldb + k0 + kk];
+            } else {
+                const int kk = e / N, j = e % N;
+                Bs[kk * LB + j] = B[(size_t)(k0 + kk) * ldb + j];
+            }
         }
+        __syncthreads();
 #pragma unroll
-        for (int x = 0; x < RM; ++x)
+        for (int ks = 0; ks < kBcKs; ks += 8) {
+            uint32_t ah[4], al[4];
+            {
+                const float *a = As + (16 * mt + g) * LA + ks + t4;
+                const float av[4] = {a[0], a[8 * LA], a[4], a[8 * LA + 4]};
 #pragma unroll
-            for (int y = 0; y < RN; ++y) c[x][y] = fmaf(av[x], bv[y], c[x][y]);
+                for (int r = 0; r < 4; ++r) {
+                    ah[r] = bc_tf32(av[r]);
+                    al[r] = bc_tf32(av[r] - __uint_as_float(ah[r]));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < NPW; ++u) {
+                const float *b = Bs + (ks + t4) * LB + 8 * (nt0 + u) + g;
+                const float b0 = b[0], b1 = b[4 * LB];
+                const uint32_t bh0 = bc_tf32(b0), bh1 = bc_tf32(b1);
+                const uint32_t bl0 = bc_tf32(b0 - __uint_as_float(bh0)), bl1 = bc_tf32(b1 - __uint_as_float(bh1));
+                bc_mma_tf32(acc[u], al, bh0, bh1);
+                bc_mma_tf32(acc[u], ah, bl0, bl1);
+                bc_mma_tf32(acc[u], ah, bh0, bh1);
+            }
+        }
     }
 #pragma unroll
-    for (int x = 0; x < RM; ++x)
+    for (int u = 0; u < NPW; ++u) {
+        const int r0 = 16 * mt + g, c0 = 8 * (nt0 + u) + 2 * t4;
 #pragma unroll
-        for (int y = 0; y < RN; ++y) {
-            const size_t o = (size_t)(ti + 16 * x) * ldc + tj + 16 * y;
-            const float r = alpha * c[x][y];
+        for (int q = 0; q < 4; ++q) {
+            const size_t o = (size_t)(r0 + 8 * (q >> 1)) * ldc + c0 + (q & 1);
+            const float r = alpha * acc[u][q];
             Cm[o] = accumulate ? Cm[o] + r : r;
         }
+    }
 }
 
 // The chunk with global index gc (over every sequence's chunks, in order): its sequence n, index c
@@ -123,7 +178,7 @@ __device__ __forceinline__ int64_t bc_chunk_base(const BwdParams &p, int n) {
 
 // ---- 1. per chunk: the forward operands ------------------------------------------------------
 template <int DK, int DV>
-__global__ void __launch_bounds__(kBcThreads) bc_prep_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kBcThreads, 1) bc_prep_kernel(const BwdParams p) {
     constexpr int C = kBcChunk, NT = kBcThreads, LK = DK + 1, LV = DV + 1, LC = C + 1;
     using R = BcRec<DK, DV>;
     extern __shared__ __align__(16) float bcs[];
@@ -134,6 +189,7 @@ __global__ void __launch_bounds__(kBcThreads) bc_prep_kernel(const BwdParams p) 
     float *sX = sv + C * LV;         // [C][LC] X
     float *sL = sX + C * LC;         // [C][LC] M, then L, then T'
     float *sbeta = sL + C * LC;      // [C]
+    float *sstage = sbeta + C;       // bc_gemm staging
     const int64_t gc = blockIdx.x / p.H;
     const int h = static_cast<int>(blockIdx.x % p.H);
     int n, c, L;
@@ -217,13 +273,13 @@ __global__ void __launch_bounds__(kBcThreads) bc_prep_kernel(const BwdParams p) 
         sk[i * LK + ch] *= expf(sb[i * LK + ch]);
     }
     __syncthreads();
-    bc_gemm<C, DK, C, false, false>(sL, LC, sk, LK, rec + R::kW, DK, 1.f, false);   // W = T' K^
-    bc_gemm<C, DV, C, false, false>(sL, LC, sv, LV, rec + R::kU, DV, 1.f, false);   // T' V
+    bc_gemm<C, DK, C, false, false>(sL, LC, sk, LK, rec + R::kW, DK, 1.f, false, sstage);   // W = T' K^
+    bc_gemm<C, DV, C, false, false>(sL, LC, sv, LV, rec + R::kU, DV, 1.f, false, sstage);   // T' V
 }
 
 // ---- 2. per unit and 32 value columns: the state at every chunk start, and U -----------------
 template <int DK, int DV>
-__global__ void __launch_bounds__(kBcThreads) bc_state_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kBcThreads, 1) bc_state_kernel(const BwdParams p) {
     constexpr int C = kBcChunk, NT = kBcThreads, DC = kBcCols, G = DV / DC;
     using R = BcRec<DK, DV>;
     constexpr int LK = DK + 1;
@@ -233,6 +289,7 @@ __global__ void __launch_bounds__(kBcThreads) bc_state_kernel(const BwdParams p)
     float *sT = sU + C * DC;         // [DK][DC]
     float *sW = sT + DK * DC;        // [C][LK] W of the chunk
     float *sKb = sW + C * LK;        // [C][LK] K- of the chunk
+    float *sstage = sKb + C * LK;    // bc_gemm staging
     const int64_t unit = blockIdx.x / G;
     const int slice = static_cast<int>(blockIdx.x % G);
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
@@ -265,13 +322,13 @@ __global__ void __launch_bounds__(kBcThreads) bc_state_kernel(const BwdParams p)
             sKb[i * LK + ch] = rec[R::kKb + e];
         }
         __syncthreads();
-        bc_gemm<C, DC, DK, false, false>(sW, LK, sS, DC, sU, DC, -1.f, true);   // U = T'V - W S0
+        bc_gemm<C, DC, DK, false, false>(sW, LK, sS, DC, sU, DC, -1.f, true, sstage);   // U = T'V - W S0
         __syncthreads();
         for (int e = tid; e < C * DC; e += NT) {
             const int i = e / DC, cc = e % DC;
             rec[R::kU + (size_t)i * DV + col0 + cc] = sU[e];
         }
-        bc_gemm<DK, DC, C, true, false>(sKb, LK, sU, DC, sT, DC, 1.f, false);   // K-^T U
+        bc_gemm<DK, DC, C, true, false>(sKb, LK, sU, DC, sT, DC, 1.f, false, sstage);   // K-^T U
         __syncthreads();
         for (int e = tid; e < DK * DC; e += NT) sS[e] = fmaf(rec[R::kGC + e / DC], sS[e], sT[e]);
         __syncthreads();
@@ -280,7 +337,7 @@ __global__ void __launch_bounds__(kBcThreads) bc_state_kernel(const BwdParams p)
 
 // ---- 3. per unit and 32 value columns, in reverse: the outputs' gate, dU and the state gradients
 template <int DK, int DV>
-__global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kBcThreads, 1) bc_dstate_kernel(const BwdParams p) {
     constexpr int C = kBcChunk, NT = kBcThreads, DC = kBcCols, G = DV / DC;
     using R = BcRec<DK, DV>;
     constexpr int LK = DK + 1, LC = C + 1;
@@ -293,6 +350,7 @@ __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p
     float *sKb = sQh + C * LK;
     float *sW = sKb + C * LK;
     float *sA = sW + C * LK;         // [C][LC]
+    float *sstage = sA + C * LC;     // bc_gemm staging
     const int64_t unit = blockIdx.x / G;
     const int slice = static_cast<int>(blockIdx.x % G);
     const int n = static_cast<int>(unit / p.H), h = static_cast<int>(unit % p.H);
@@ -323,9 +381,9 @@ __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p
         for (int e = tid; e < C * C; e += NT) sA[(e / C) * LC + e % C] = rec[R::kA + e];
         __syncthreads();
         // O = Q^ S0 + A U (pre-gate outputs of this chunk's columns)
-        bc_gemm<C, DC, DK, false, false>(sQh, LK, rec + R::kS0 + col0, DV, sO, DC, 1.f, false);
+        bc_gemm<C, DC, DK, false, false>(sQh, LK, rec + R::kS0 + col0, DV, sO, DC, 1.f, false, sstage);
         __syncthreads();
-        bc_gemm<C, DC, C, false, false>(sA, LC, rec + R::kU + col0, DV, sO, DC, 1.f, true);
+        bc_gemm<C, DC, C, false, false>(sA, LC, rec + R::kU + col0, DV, sO, DC, 1.f, true, sstage);
         __syncthreads();
         for (int e = tid; e < C * DC; e += NT) {   // dO = dout sigmoid(gate); dgate = dout O sigmoid'
             const int i = e / DC, cc = e % DC;
@@ -348,18 +406,18 @@ __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p
         }
         __syncthreads();
         // dU = A^T dO + K- dS_C
-        bc_gemm<C, DC, C, true, false>(sA, LC, sO, DC, sdU, DC, 1.f, false);
+        bc_gemm<C, DC, C, true, false>(sA, LC, sO, DC, sdU, DC, 1.f, false, sstage);
         __syncthreads();
-        bc_gemm<C, DC, DK, false, false>(sKb, LK, sdS, DC, sdU, DC, 1.f, true);
+        bc_gemm<C, DC, DK, false, false>(sKb, LK, sdS, DC, sdU, DC, 1.f, true, sstage);
         __syncthreads();
         for (int e = tid; e < C * DC; e += NT) {
             const int i = e / DC, cc = e % DC;
             rec[R::kdU + (size_t)i * DV + col0 + cc] = sdU[e];
         }
         // dS0 = Q^T dO + Diag(Gamma_C) dS_C - W^T dU
-        bc_gemm<DK, DC, C, true, false>(sQh, LK, sO, DC, sT, DC, 1.f, false);
+        bc_gemm<DK, DC, C, true, false>(sQh, LK, sO, DC, sT, DC, 1.f, false, sstage);
         __syncthreads();
-        bc_gemm<DK, DC, C, true, false>(sW, LK, sdU, DC, sT, DC, -1.f, true);
+        bc_gemm<DK, DC, C, true, false>(sW, LK, sdU, DC, sT, DC, -1.f, true, sstage);
         __syncthreads();
         for (int e = tid; e < DK * DC; e += NT) sdS[e] = fmaf(rec[R::kGC + e / DC], sdS[e], sT[e]);
         __syncthreads();
@@ -374,7 +432,7 @@ __global__ void __launch_bounds__(kBcThreads) bc_dstate_kernel(const BwdParams p
 
 // ---- 4. per chunk: every input's gradient ------------------------------------------------------
 template <int DK, int DV>
-__global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kBcThreads, 1) bc_grad_kernel(const BwdParams p) {
     constexpr int C = kBcChunk, NT = kBcThreads, LK = DK + 1, LC = C + 1;
     using R = BcRec<DK, DV>;
     extern __shared__ __align__(16) float bcs[];
@@ -390,6 +448,7 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
     float *sdb = sbeta + C;          // [C] dbeta
     float *sdGC = sdb + C;           // [DK]
     float *sred = sdGC + DK;         // [NT / 32]
+    float *sstage = sred + NT / 32;  // bc_gemm staging
     const int64_t gc = blockIdx.x / p.H;
     const int h = static_cast<int>(blockIdx.x % p.H);
     int n, c, L;
@@ -429,10 +488,10 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
         sT[i * LC + j] = sX[i * LC + j] * sbeta[j];
     }
     // dA = lower_incl(dO U^T);  dO S0^T over Q^;  dK- = U dS_C^T over K-;  dW = -dU S0^T over W
-    bc_gemm<C, C, DV, false, true>(rec + R::kdO, DV, rec + R::kU, DV, sdA, LC, 1.f, false);
-    bc_gemm<C, DK, DV, false, true>(rec + R::kdO, DV, rec + R::kS0, DV, rec + R::kQh, DK, 1.f, false);
-    bc_gemm<C, DK, DV, false, true>(rec + R::kU, DV, rec + R::kdS, DV, rec + R::kKb, DK, 1.f, false);
-    bc_gemm<C, DK, DV, false, true>(rec + R::kdU, DV, rec + R::kS0, DV, rec + R::kW, DK, -1.f, false);
+    bc_gemm<C, C, DV, false, true>(rec + R::kdO, DV, rec + R::kU, DV, sdA, LC, 1.f, false, sstage);
+    bc_gemm<C, DK, DV, false, true>(rec + R::kdO, DV, rec + R::kS0, DV, rec + R::kQh, DK, 1.f, false, sstage);
+    bc_gemm<C, DK, DV, false, true>(rec + R::kU, DV, rec + R::kdS, DV, rec + R::kKb, DK, 1.f, false, sstage);
+    bc_gemm<C, DK, DV, false, true>(rec + R::kdU, DV, rec + R::kS0, DV, rec + R::kW, DK, -1.f, false, sstage);
     __syncthreads();
     for (int e = tid; e < C * C; e += NT) {
         const int i = e / C, j = e % C;
@@ -444,17 +503,17 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
     }
     __syncthreads();
     // T'^T dW over S0 (no longer needed);  dv = T'^T dU over U
-    bc_gemm<C, DK, C, true, false>(sT, LC, rec + R::kW, DK, rec + R::kS0, DK, 1.f, false);
-    bc_gemm<C, DV, C, true, false>(sT, LC, rec + R::kdU, DV, rec + R::kU, DV, 1.f, false);
+    bc_gemm<C, DK, C, true, false>(sT, LC, rec + R::kW, DK, rec + R::kS0, DK, 1.f, false, sstage);
+    bc_gemm<C, DV, C, true, false>(sT, LC, rec + R::kdU, DV, rec + R::kU, DV, 1.f, false, sstage);
     __syncthreads();
     for (int e = tid; e < C * DV; e += NT) {
         const int i = e / DV, ch = e % DV;
         if (i < L) p.dv[((t0 + i) * H + h) * DV + ch] = rec[R::kU + e];
     }
     // dT' = dW K^T + dU V^T (over T', after the transposed use above)
-    bc_gemm<C, C, DK, false, true>(rec + R::kW, DK, sKh, LK, sT, LC, 1.f, false);
+    bc_gemm<C, C, DK, false, true>(rec + R::kW, DK, sKh, LK, sT, LC, 1.f, false, sstage);
     __syncthreads();
-    bc_gemm<C, C, DV, false, true>(rec + R::kdU, DV, rec + R::kdO, DV, sT, LC, 1.f, true);
+    bc_gemm<C, C, DV, false, true>(rec + R::kdU, DV, rec + R::kdO, DV, sT, LC, 1.f, true, sstage);
     __syncthreads();
     // dbeta_j = sum_i dT'_ij X_ij;  dX = dT' diag(beta)
     for (int j = tid; j < C; j += NT) {
@@ -469,9 +528,9 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
     }
     __syncthreads();
     // dL = strict_lower(-X^T dX X^T): Y = X^T dX over A (no longer needed), then dL = -Y X^T over dX
-    bc_gemm<C, C, C, true, false>(sX, LC, sT, LC, rec + R::kA, C, 1.f, false);
+    bc_gemm<C, C, C, true, false>(sX, LC, sT, LC, rec + R::kA, C, 1.f, false, sstage);
     __syncthreads();
-    bc_gemm<C, C, C, false, true>(rec + R::kA, C, sX, LC, sT, LC, -1.f, false);
+    bc_gemm<C, C, C, false, true>(rec + R::kA, C, sX, LC, sT, LC, -1.f, false, sstage);
     __syncthreads();
     // dbeta_i += sum_{j<i} dL_ij M_ij;  dM = diag(beta) dL (strict lower)
     for (int i = tid; i < C; i += NT) {
@@ -561,10 +620,10 @@ __global__ void __launch_bounds__(kBcThreads) bc_grad_kernel(const BwdParams p) 
 template <int DK, int DV>
 struct BcSmem {
     static constexpr int C = kBcChunk, LK = DK + 1, LV = DV + 1, LC = C + 1;
-    static constexpr int kPrep = (3 * C * LK + C * LV + 2 * C * LC + C) * 4;
-    static constexpr int kState = (2 * DK * kBcCols + C * kBcCols + 2 * C * LK) * 4;
-    static constexpr int kDState = (2 * DK * kBcCols + 2 * C * kBcCols + 3 * C * LK + C * LC) * 4;
-    static constexpr int kGrad = (4 * C * LK + 4 * C * LC + 2 * C + DK + kBcThreads / 32) * 4;
+    static constexpr int kPrep = (3 * C * LK + C * LV + 2 * C * LC + C + kBcStageFloats) * 4;
+    static constexpr int kState = (2 * DK * kBcCols + C * kBcCols + 2 * C * LK + kBcStageFloats) * 4;
+    static constexpr int kDState = (2 * DK * kBcCols + 2 * C * kBcCols + 3 * C * LK + C * LC + kBcStageFloats) * 4;
+    static constexpr int kGrad = (4 * C * LK + 4 * C * LC + 2 * C + DK + kBcThreads / 32 + kBcStageFloats) * 4;
 };
 
 }  // namespace kda
