@@ -38,9 +38,6 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture of each
-# kernel (profiles/ gives the commands), keyed by workload, with the hash of the kernel's sources at
-# capture time.  Reported only while the sources are unchanged.
 # DRAM bytes of one prefill launch per kernel (kda_prefill_path: 1 cluster, 2 per-unit), captured on
 # the named workload; a prefill row scales it by its own algorithmic bytes (both kernels move
 # traffic in proportion to the token-heads and units they process)
@@ -49,14 +46,17 @@ PREFILL_TRAFFIC = {
     2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346657000 + 261571584, "src": "96b83a3ec9646b8a"},
 }
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture of each
+# kernel (profiles/ gives the commands), keyed by workload, with the hash of the kernel's sources at
+# capture time.  Reported only while the sources are unchanged.
 NCU_TRAFFIC = {
-    "decode_N256_H64_d128_512steps": {"bytes_per_launch": 2114315008, "src": "1c3a7d12c8610c04"},
-    # one verify launch plus one commit launch (round 4 of the captured run; commit's bytes depend on
-    # how many sequences accepted at least one token)
-    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1158005248 + 49608192 + 930634752 + 830197504,
-                              "src": "1b85ba110de6be44"},
-    # kda_chunk_bwd on the prefill workload (ncu prints these two counters to three digits)
-    "bwd_prefill_B1_H32_T8192_d128": {"bytes_per_launch": 1.30e9 + 2.55e9, "src": "733838d1f4904973"},
+    "decode_N256_H64_d128_512steps": {"bytes_per_launch": 1094800000 + 1016000000, "src": "6184bb076c425fa7"},
+    # one verify launch plus one commit launch: the mean of the timed rounds of the captured run
+    # (commit's bytes depend on how many sequences accepted at least one token)
+    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1160200000 + 47250000 + 892350000 + 794300000,
+                              "src": "eb388ca15bf43403"},
+    # kda_chunk_bwd on the prefill workload (ncu prints these two counters to five digits)
+    "bwd_prefill_B1_H32_T8192_d128": {"bytes_per_launch": 1.2989e9 + 2.5685e9, "src": "9ec2178bcf630624"},
 }
 
 
