@@ -547,7 +547,25 @@ def main():
                                  "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
                                  "traffic": ncu_traffic("bwd_" + aw.name, "backward"),
                                  "peak_source": f"hbm_gbs of {peak_src}", "algorithmic_bytes": bbytes}}
-        del dout, dST, bws
+        del bws
+        torch.cuda.empty_cache()
+        # the same gradients in chunkwise form (kda_chunk_bwd_chunkwise: four launches, the products
+        # on the tensor cores), timed beside the token-level kernel that kda_chunk_bwd runs by default
+        cws = torch.empty(kda.kda_chunk_bwd_chunkwise_workspace_size(aw.total_tokens, aw.num_seqs, aw.H, aw.d_k, aw.d_v),
+                          dtype=torch.uint8, device=dev)
+
+        def cstep():
+            return kda.kda_chunk_bwd(ainp["q"], ainp["k"], ainp["v"], ainp["a"], ainp["beta"], ainp["A_log"],
+                                     ainp["cu_seqlens"], dout, gate=ainp["gate"], initial_state=ainp["initial_state"],
+                                     dfinal_state=dST, workspace=cws, stream=stream, chunkwise=True)
+
+        cms = time_calls(cstep, 3, 1, stream, world, dev, barrier)
+        kda.kda_sync_check()
+        backward["chunkwise"] = {"value": whole_job_rate(aw.total_tokens, world, cms), "unit": "tokens/s",
+                                 "ms_per_step": cms, "frac_of_hbm_peak": bbytes / (cms * 1e-3) / 1e9 / hbm,
+                                 "scope": "one kda_chunk_bwd(chunkwise=True) call: bc_prep, bc_state, bc_dstate, "
+                                          "bc_grad"}
+        del dout, dST, cws
         torch.cuda.empty_cache()
 
     # module row: the short convolution of q, k, v (q, k L2-normalised) and the pre-gate
