@@ -146,6 +146,13 @@ __device__ __forceinline__ void bc_gemm(const float *A, int lda, const float *B,
     }
 }
 
+// Bulk prefetch of [ptr, ptr + bytes) into L2 (ptr and bytes multiples of 16), issued by one thread:
+// the chunk records were written by an earlier kernel and have mostly left L2 by the time they are
+// read, and the passes over chunks know which record comes next.
+__device__ __forceinline__ void bc_prefetch_l2(const void *ptr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
 // The chunk with global index gc (over every sequence's chunks, in order): its sequence n, index c
 // within the sequence and token span; false past the last chunk.
 __device__ __forceinline__ bool bc_find(const BwdParams &p, int64_t gc, int &n, int &c, int64_t &t0, int &L) {
@@ -308,6 +315,12 @@ __global__ void __launch_bounds__(kBcThreads, 1) bc_state_kernel(const BwdParams
     __syncthreads();
     for (int c = 0; c < nck; ++c) {
         float *rec = p.ckpt + (size_t)((base + c) * p.H + h) * R::kSize;
+        if (tid == 0 && c + 1 < nck) {   // the next chunk's W and T'V (adjacent), K- and Gamma_C
+            const float *nx = rec + (size_t)p.H * R::kSize;
+            bc_prefetch_l2(nx + R::kW, (uint32_t)(C * (DK + DV) * 4));
+            bc_prefetch_l2(nx + R::kKb, (uint32_t)(C * DK * 4));
+            bc_prefetch_l2(nx + R::kGC, (uint32_t)(DK * 4));
+        }
         for (int e = tid; e < DK * DC; e += NT) {
             const int r = e / DC, cc = e % DC;
             rec[R::kS0 + (size_t)r * DV + col0 + cc] = sS[e];
@@ -370,6 +383,12 @@ __global__ void __launch_bounds__(kBcThreads, 1) bc_dstate_kernel(const BwdParam
     __syncthreads();
     for (int c = nck - 1; c >= 0; --c) {
         float *rec = p.ckpt + (size_t)((base + c) * H + h) * R::kSize;
+        if (tid == 0 && c > 0) {   // the next chunk in reverse: W and U, K-, Q^ and A, Gamma_C and S0
+            const float *nx = rec - (size_t)H * R::kSize;
+            bc_prefetch_l2(nx + R::kW, (uint32_t)(C * (DK + DV) * 4));
+            bc_prefetch_l2(nx + R::kKb, (uint32_t)((2 * C * DK + C * C) * 4));
+            bc_prefetch_l2(nx + R::kGC, (uint32_t)((DK + DK * DV) * 4));
+        }
         const int64_t t0 = s0 + (int64_t)c * C;
         const int L = static_cast<int>(min64(C, s1 - t0));
         for (int e = tid; e < C * DK; e += NT) {
@@ -457,6 +476,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) bc_grad_kernel(const BwdParams 
     float *rec = p.ckpt + (size_t)blockIdx.x * R::kSize;
     const int tid = threadIdx.x;
     const int64_t H = p.H;
+    if (tid == 0) bc_prefetch_l2(rec, (uint32_t)(R::kSize * 4));   // every slot of it is read below
     const float expA = expf(p.A_log[h]);
     for (int e = tid; e < C * DK; e += NT) {
         const int i = e / DK, ch = e % DK;
