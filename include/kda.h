@@ -269,6 +269,28 @@ KDA_API kda_status kda_state_combine(const float *M, const float *S_in, const fl
                                      int32_t units, int32_t d_k, int32_t d_v, void *stream);
 
 /*
+ * kda_segment_maps — the affine map S -> M S + B of every (sequence, head) unit over the tokens
+ * given (the maps kda_state_combine folds), in one pass: the recurrence is linear in (v, S) column
+ * by column, so [M | B] is the final state of one run over the value columns [0 | v] from the
+ * initial state [I | 0], and the chunk-local work (decays, Gram blocks, triangular solve, W) is
+ * shared by both maps.  (Context-parallel prefill; "Kimi K3 · Lesson 3 of 14", CHUNKWISE diagram:
+ * the state passes from chunk to chunk, here from segment to segment.)
+ *   q, k, a, v bf16 [total_tokens, H, d] (d_k = d_v = d, 64 or 128); beta fp32 [total_tokens, H];
+ *   A_log fp32 [H]; cu_seqlens int32 [num_seqs + 1] on the device, as kda_chunk_fwd;
+ *   M, B fp32 [num_seqs, H, d, d] (written; caller-owned).
+ *   workspace: kda_segment_maps_workspace_size(...) bytes, 256-byte aligned, caller-owned.
+ * Runs the cluster prefill kernel with 2d value columns (no outputs, no gate), then two strided
+ * device copies.  Errors as kda_chunk_fwd; KDA_ERR_UNSUPPORTED for other d.
+ */
+KDA_API kda_status kda_segment_maps(const void *q, const void *k, const void *v, const void *a, const float *beta,
+                                    const float *A_log, const int32_t *cu_seqlens, int32_t num_seqs,
+                                    int64_t total_tokens, int32_t max_seqlen, int32_t H, int32_t d, float scale,
+                                    float *M, float *B, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace of kda_segment_maps (host-only; 0 on invalid sizes or unsupported d). */
+KDA_API size_t kda_segment_maps_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d);
+
+/*
  * kda_chunk_bwd — gradients of the prefill (kda_chunk_fwd with the same inputs) with respect to
  * q, k, v, the decay logits a, beta, the gate logits, A_log and the initial state, given dout (the
  * gradient of the outputs) and optionally dfinal_state (the gradient of the final states).  The

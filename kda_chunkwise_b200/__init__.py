@@ -110,6 +110,10 @@ def _load() -> ctypes.CDLL:
     L.kda_set_prefill_path.restype = ctypes.c_int
     L.kda_prefill_path.argtypes = [i64, i32, i32]
     L.kda_prefill_path.restype = i32
+    L.kda_segment_maps.argtypes = [vp, vp, vp, vp, fp, fp, vp, i32, i64, i32, i32, i32, f32, fp, fp, vp, sz, vp]
+    L.kda_segment_maps.restype = ctypes.c_int
+    L.kda_segment_maps_workspace_size.argtypes = [i64, i32, i32, i32]
+    L.kda_segment_maps_workspace_size.restype = sz
     return L
 
 
@@ -441,12 +445,40 @@ def kda_state_combine(M, S_in, B, out=None, stream=None):
     return out
 
 
-def kda_segment_maps(q, k, v, a, beta, A_log, cu_seqlens, scale: float = 1.0, max_seqlen=None, stream=None):
+def kda_segment_maps(q, k, v, a, beta, A_log, cu_seqlens, scale: float = 1.0, max_seqlen=None, stream=None,
+                     single_pass: bool | None = None):
     """The affine map S -> M S + B of each (sequence, head) over the tokens given: B is the final
-    state from S = 0, M the final state of the homogeneous recurrence (v = 0) from S = I.  Two
-    kda_chunk_fwd calls; returns (M [N, H, d_k, d_k], B [N, H, d_k, d_v])."""
+    state from S = 0, M the final state of the homogeneous recurrence (v = 0) from S = I.  Returns
+    (M [N, H, d_k, d_k], B [N, H, d_k, d_v]).
+
+    single_pass: one pass of the cluster kernel over value columns [0 | v] from [I | 0]
+    (kda_segment_maps; d_k = d_v only), which shares the chunk-local work of both maps but needs
+    2 d / 32 CTAs per unit; or two kda_chunk_fwd calls.  None: one pass when every unit's cluster
+    fits the GPU at once (then it takes the time of one of the two calls), else two calls (the same
+    SM time, and with many units kda_chunk_fwd's per-unit kernel is the faster one)."""
     N = cu_seqlens.numel() - 1
     T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    dev = q.device
+    if single_pass is None:
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count if dev.type == "cuda" else 0
+        single_pass = N * H * (2 * d_k // 32) <= sms
+    if single_pass and d_k == d_v:
+        for name, t in (("q", q), ("k", k), ("v", v), ("a", a)):
+            _need(t, name, torch.bfloat16, (T, H, d_k), dev)
+        _need(beta, "beta", torch.float32, (T, H), dev)
+        _need(A_log, "A_log", torch.float32, (H,), dev)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+        if max_seqlen is None:
+            max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if N > 0 else 0
+        M = torch.empty((N, H, d_k, d_k), dtype=torch.float32, device=dev)
+        B = torch.empty((N, H, d_k, d_k), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(int(lib.kda_segment_maps_workspace_size(T, N, H, d_k)), 1), dtype=torch.uint8, device=dev)
+        st = lib.kda_segment_maps(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(beta), _ptr(A_log), _ptr(cu_seqlens), N, T,
+                                  max_seqlen, H, d_k, scale, _ptr(M), _ptr(B), _ptr(ws), ws.numel(),
+                                  _stream_handle(stream, dev))
+        _check(st, "kda_segment_maps")
+        return M, B
     _, B = kda_chunk_fwd(q, k, v, a, beta, A_log, cu_seqlens, gate=None, initial_state=None, scale=scale,
                          max_seqlen=max_seqlen, stream=stream, out_dtype=torch.bfloat16)
     v0 = torch.zeros((T, H, d_k), dtype=torch.bfloat16, device=q.device)

@@ -647,6 +647,75 @@ kda_status kda_output_norm_gate(const float *o, const void *gate, const float *w
     return e == cudaSuccess ? KDA_OK : cuda_fail(e, "norm_gate launch");
 }
 
+size_t kda_segment_maps_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d) {
+    if (!sizes_ok(total_tokens, num_seqs, 0, H) || !supported_dim(d)) return 0;
+    const int64_t units = (int64_t)num_seqs * H;
+    const size_t slot = d == 128 ? kda::RingLayout<128, 256>::kBytes : kda::RingLayout<64, 128>::kBytes;
+    const size_t ring = ((size_t)units * ring_slots(2 * d) * slot + 255) / 256 * 256;
+    return ring + (size_t)units * d * 2 * d * 4;   // then the final states [M | B]
+}
+
+kda_status kda_segment_maps(const void *q, const void *k, const void *v, const void *a, const float *beta,
+                            const float *A_log, const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                            int32_t max_seqlen, int32_t H, int32_t d, float scale, float *M, float *B,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+    if (!sizes_ok(total_tokens, num_seqs, max_seqlen, H))
+        return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: negative size or H <= 0");
+    if (!supported_dim(d)) return fail(KDA_ERR_UNSUPPORTED, "kda_segment_maps: d must be 64 or 128");
+    if (num_seqs == 0) {
+        if (total_tokens != 0) return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: tokens without sequences");
+        return KDA_OK;
+    }
+    if (!cu_seqlens || !A_log || !M || !B || !workspace)
+        return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: NULL cu_seqlens, A_log, M, B or workspace");
+    if (total_tokens > 0 && (!q || !k || !v || !a || !beta))
+        return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: NULL q/k/v/a/beta");
+    const void *ptrs[] = {q, k, v, a, M, B};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned(ptr, 16)) return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: tensor pointer not 16-byte aligned");
+    const void *ptrs4[] = {beta, A_log, cu_seqlens};
+    for (const void *ptr : ptrs4)
+        if (ptr && !aligned(ptr, 4)) return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: beta/A_log/cu_seqlens not 4-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: workspace not 256-byte aligned");
+    const size_t need = kda_segment_maps_workspace_size(total_tokens, num_seqs, H, d);
+    if (workspace_bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: workspace too small (need " + std::to_string(need) + " bytes)");
+    const int64_t units = (int64_t)num_seqs * H;
+    if (units * (2 * d / kda::kSlab) > 0x7fffffffLL) return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: num_seqs * H too large");
+    if (total_tokens > 0x7fffffc0LL) return fail(KDA_ERR_INVALID_ARG, "kda_segment_maps: total_tokens too large");
+    // one pass of the cluster kernel over value columns [0 | v] from [I | 0]: the final state is [M | B]
+    const size_t slot = d == 128 ? kda::RingLayout<128, 256>::kBytes : kda::RingLayout<64, 128>::kBytes;
+    const size_t ring = ((size_t)units * ring_slots(2 * d) * slot + 255) / 256 * 256;
+    char *ws = static_cast<char *>(workspace);
+    float *SMB = reinterpret_cast<float *>(ws + ring);
+    kda::FusedParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k = static_cast<const uint16_t *>(k);
+    p.v = static_cast<const uint16_t *>(v);
+    p.a = static_cast<const uint16_t *>(a);
+    p.beta = beta;
+    p.A_log = A_log;
+    p.cu = cu_seqlens;
+    p.S_out = SMB;
+    p.ring = ws;
+    p.total_tokens = total_tokens;
+    p.num_seqs = num_seqs;
+    p.H = H;
+    p.max_seqlen = max_seqlen;
+    p.scale = scale;
+    p.wait_ns = kWaitNs;
+    p.maps_cols = d;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const kda_status s = d == 128 ? launch_prefill<128, 256>(p, units, st) : launch_prefill<64, 128>(p, units, st);
+    if (s != KDA_OK) return s;
+    // [M | B] rows -> M and B
+    const size_t rows = (size_t)units * d, wb = (size_t)d * 4;
+    cudaError_t e = cudaMemcpy2DAsync(M, wb, SMB, 2 * wb, wb, rows, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(B, wb, SMB + d, 2 * wb, wb, rows, cudaMemcpyDeviceToDevice, st);
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e, "kda_segment_maps: copy of the maps");
+}
+
 kda_status kda_state_combine(const float *M, const float *S_in, const float *B, float *S_out, int32_t units,
                              int32_t d_k, int32_t d_v, void *stream) {
     if (units < 0) return fail(KDA_ERR_INVALID_ARG, "kda_state_combine: units < 0");

@@ -135,6 +135,10 @@ struct FusedParams {
     bool out_f32;
     int stall_first_chunk;       // failure injection: never publish chunk 0
     unsigned long long wait_ns;  // bound of every wait
+    // Segment maps (0: off).  Value columns [0, maps_cols) run the homogeneous recurrence from the
+    // identity (v = 0, S_in = I, read from nowhere); columns [maps_cols, DV) take v from p.v, a
+    // [T, H, DV - maps_cols] tensor, from S_in = 0.  The final state is then [M | B] of the tokens.
+    int maps_cols;
 };
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
@@ -217,8 +221,9 @@ __device__ __forceinline__ void fused_producer(const FusedParams &p, unsigned ch
         for (int it = 0; it < 64 * CPRV / kRoleThreads; ++it) {
             const int e = tid + it * kRoleThreads;
             const int row = e / CPRV, ch = e % CPRV;
-            const bool in = row < Ll;
-            const int64_t off = ((tl + (in ? row : 0)) * H + h) * DV + ch * 8;
+            const bool in = row < Ll && ch * 8 >= p.maps_cols;   // the maps' homogeneous columns read 0
+            const int vd = DV - p.maps_cols;                    // row length of p.v
+            const int64_t off = in ? ((tl + row) * H + h) * vd + ch * 8 - p.maps_cols : 0;
             cp_async_16(aV + swz<RBV>(row, ch), p.v + off, in ? 16 : 0);
         }
         cp_async_commit();
@@ -696,7 +701,10 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
     float S[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) S[j] = 0.f;
-    if (has_s && p.S_in) {
+    if (has_s && p.maps_cols) {   // [I | 0]
+#pragma unroll
+        for (int j = 0; j < 16; ++j) S[j] = (col0 + j < p.maps_cols && col0 + j == row) ? 1.f : 0.f;
+    } else if (has_s && p.S_in) {
         const float4 *sp = reinterpret_cast<const float4 *>(p.S_in + st_base + (size_t)row * DV + col0);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -836,7 +844,9 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                     }
                 }
                 const int64_t off = ((t0 + i) * H + h) * DV + col0;
-                if (p.out_f32) {
+                if (!p.out) {
+                    // no outputs wanted (the segment maps)
+                } else if (p.out_f32) {
                     float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) op[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);

@@ -213,3 +213,22 @@ def test_host_prefill_validates_on_the_host():
     assert H(*args(cu_p, 260, 0, None, 0)) == kda.KDA_ERR_INVALID_ARG               # no device buffer
     assert H(*args(cu_p, 260, 0, 256, size - 1)) == kda.KDA_ERR_INVALID_ARG         # buffer too small
     assert H(*args(cu_p, 260, 0, 16, size)) == kda.KDA_ERR_INVALID_ARG              # not 256-byte aligned
+
+
+def test_segment_maps_validate_on_the_host():
+    fake = 256
+    assert kda.lib.kda_segment_maps_workspace_size(1024, 2, 4, 96) == 0          # unsupported d
+    assert kda.lib.kda_segment_maps_workspace_size(-1, 2, 4, 128) == 0
+    need = kda.lib.kda_segment_maps_workspace_size(1024, 2, 4, 128)
+    assert need > 0 and need % 256 == 0
+    f = kda.lib.kda_segment_maps
+    args = lambda **o: dict(dict(q=fake, k=fake, v=fake, a=fake, beta=fake, A_log=fake, cu=fake, N=2, T=1024, ms=512,
+                                 H=4, d=128, scale=1.0, M=fake, B=fake, ws=fake, wsb=need, st=None), **o)
+    call = lambda a: f(a["q"], a["k"], a["v"], a["a"], a["beta"], a["A_log"], a["cu"], a["N"], a["T"], a["ms"], a["H"],
+                       a["d"], a["scale"], a["M"], a["B"], a["ws"], a["wsb"], a["st"])
+    assert call(args(d=96)) == kda.KDA_ERR_UNSUPPORTED
+    assert call(args(M=None)) == kda.KDA_ERR_INVALID_ARG
+    assert call(args(wsb=need - 1)) == kda.KDA_ERR_INVALID_ARG
+    assert call(args(ws=fake + 16)) == kda.KDA_ERR_INVALID_ARG             # workspace not 256-byte aligned
+    assert call(args(q=fake + 8)) == kda.KDA_ERR_INVALID_ARG               # misaligned tensor
+    assert call(args(N=0, T=0)) == kda.KDA_OK                              # nothing to do

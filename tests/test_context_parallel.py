@@ -198,3 +198,37 @@ def test_context_parallel_entry_point_over_three_ranks_matches_the_unsplit_oracl
         out[torch.from_numpy(z["idx"])] = torch.from_numpy(z["out"])
     S_last = torch.from_numpy(np.load(tmp_path / f"cpgpu{world - 1}.npz")["S"])
     check_units(inp, out, S_last, [(n, h) for n in range(w.num_seqs) for h in range(w.H)])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("a_mean", [0.0, -8.0])
+def test_one_pass_segment_maps_match_the_oracle_and_the_two_pass_maps(d, a_mean):
+    # kda_segment_maps in one pass ([0 | v] from [I | 0]) against the oracle's maps of each unit
+    # (B from S = 0, M from S = I with v = 0) and against the two-call form, on ragged sequences.
+    # With fading decays (a ~ N(0, 1)) M shrinks towards zero (as e^{b}), so errors are also bounded
+    # against the scale of the identity (1e-4 sqrt(d)); with almost no fade (a ~ N(-8, 1)) M stays
+    # of the identity's size.
+    import kda_chunkwise_b200 as kda
+    w = KI.Workload("maps", (300, 77, 129), 2, d, d, A_log="uniform", a_mean=a_mean, seed=23)
+    inp = KI.make_inputs(w, "cuda")
+    M1, B1 = kda.kda_segment_maps(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"])
+    M2, B2 = kda.kda_segment_maps(inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"],
+                                  single_pass=False)
+    kda.kda_sync_check()
+    floor = 1e-4 * d ** 0.5
+    for x, y in ((M1, M2), (B1, B2)):
+        assert float((x - y).norm()) <= 2e-3 * float(y.norm()) + floor
+    cu = inp["cu_seqlens"].cpu().tolist()
+    A_log = host(inp["A_log"])
+    for n in range(w.num_seqs):
+        s, e = cu[n], cu[n + 1]
+        for h in range(w.H):
+            q, k, v = (host(inp[x][s:e, h]) for x in ("q", "k", "v"))
+            g = oracle.gate_log_decay(host(inp["a"][s:e, h]), float(A_log[h]))
+            beta = host(inp["beta"][s:e, h])
+            _, B_ref = oracle.recurrence_g(q, k, v, g, beta, S0=np.zeros((d, d)))
+            _, M_ref = oracle.recurrence_g(q, k, np.zeros((e - s, d)), g, beta, S0=np.eye(d))
+            for got, ref, name in ((host(M1[n, h]), M_ref, "M"), (host(B1[n, h]), B_ref, "B")):
+                err = np.linalg.norm(got - ref)
+                assert err <= 5e-3 * np.linalg.norm(ref) + floor, f"unit ({n},{h}) {name}: |err| {err:.2e}"
