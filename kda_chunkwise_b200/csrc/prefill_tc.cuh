@@ -784,6 +784,17 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
             for (int j = 0; j < 15; ++j)
 #pragma unroll
                 for (int i = j + 1; i < 16; ++i) dinv[i] = fmaf(-Ldp[i * 17 + j], dinv[j], dinv[i]);
+            // D_p into its tile (free since pass 2); T'_pp = D_p diag(beta_p) in fp32 over L_pp, for
+            // step 4 to round into T'' (the Gram product still reads the rescaled keys under T'')
+            __syncwarp();
+            if (lane < 16) {
+                const float bcol = sb[16 * pt + lane];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    *reinterpret_cast<__half *>(sm + kLD + sw128(16 * pt + i, 16 * pt + lane)) = __float2half_rn(dinv[i]);
+                    Ldp[i * 17 + lane] = dinv[i] * bcol;
+                }
+            }
         }
         {
             const float gam = reinterpret_cast<const float *>(sm + kGam)[row];
@@ -806,15 +817,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         bar_all();
         tc_fence_after();
         if (*abort_flag) break;
-        if (cq == 0 && lane < 16) {   // D_p and T'_pp = D_p diag(beta_p) into their tiles
-            const float bcol = reinterpret_cast<const float *>(sm + kBeta)[16 * pt + lane];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * pt + i, cc = 16 * pt + lane;
-                *reinterpret_cast<__half *>(sm + kLD + sw128(r, cc)) = __float2half_rn(dinv[i]);
-                *reinterpret_cast<__half *>(sm + kT + sw128(kslot(r), cc)) = __float2half_rn(dinv[i] * bcol);
-            }
-        }
 
         // ---- 4. solve inputs: A rows (tile pt) and -L rows from the Gram, diagonal blocks ----------
         {
@@ -883,6 +885,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                         const int pb = ub < 3 ? 0 : ub < 5 ? 1 : 2, qb = ub < 3 ? ub + 1 : ub < 5 ? ub - 1 : 3;
                         sts128(base + kT + sw128(32 * pb + 16 + r, 16 * qb + 8 * hh), make_uint4(0, 0, 0, 0));
                     }
+                }
+                // the diagonal blocks T'_pp (fp32 from step 3) rounded into their key slots
+                const float *Ldf = reinterpret_cast<const float *>(sm + kLdf);
+                for (int e = tid - 256; e < 4 * 256; e += 256) {
+                    const int pb = e >> 8, i = (e >> 4) & 15, j = e & 15;
+                    *reinterpret_cast<__half *>(sm + kT + sw128(kslot(16 * pb + i), 16 * pb + j)) =
+                        __float2half_rn(Ldf[(pb * 16 + i) * 17 + j]);
                 }
             }
         }
