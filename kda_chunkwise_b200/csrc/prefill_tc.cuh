@@ -821,10 +821,38 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         // ---- 4. solve inputs: A rows (tile pt) and -L rows from the Gram, diagonal blocks ----------
         {
             const float *sb = reinterpret_cast<const float *>(sm + kBeta);
+            // off-diagonal block blk (< pt) of tile pt's rows from TMEM: lanes 32pt + r (q rows: A and
+            // its remainder) and 32pt + 16 + r (k rows: -L), all lanes of the warp
+            auto offdiag = [&](int blk) {
+                const int r = lane & 15;
+                const bool krow = lane >= 16;
+                const int i = 16 * pt + r;
+                const float sg = krow ? -sb[i] : 1.f;
+                uint32_t v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * pt) << 16) + cGD + gb_off(pt) + 16 * blk, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = sg * __uint_as_float(v[8 * hh + 2 * e]), x1 = sg * __uint_as_float(v[8 * hh + 2 * e + 1]);
+                        hi[e] = pack_f16(x0, x1);
+                        const float2 hf = unpack_f16(hi[e]);
+                        lo[e] = pack_f16(x0 - hf.x, x1 - hf.y);
+                    }
+                    if (krow) {
+                        sts128(base + kLD + sw128(i, 16 * blk + 8 * hh), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                    } else {
+                        sts128(base + kAm + sw128(qslot(i), 16 * blk + 8 * hh), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+                        sts128(base + kAm + sw128(kslot(i), 16 * blk + 8 * hh), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+                    }
+                }
+            };
+            const int split = (pt + 1) >> 1;   // quarter 1 takes blocks [0, split), quarter 0 the rest
             if (cq == 0) {
                 // diagonal blocks of A from the fragments (j <= i): fp16 A in the query slots, the
-                // rounding remainder A - fp16(A) (fp16) in the key slots, where the A_lo U product
-                // reads it through an operand that starts 16 rows later
+                // rounding remainder A - fp16(A) (fp16) in the key slots
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int j = 8 * nt + 2 * t4;   // column within the tile
@@ -838,36 +866,11 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                         sts32(base + kAm + sw128(32 * pt + 16 + r, 16 * pt + j), pack_f16(x0 - hf.x, x1 - hf.y));
                     }
                 }
+                for (int blk = split; blk < pt; ++blk) offdiag(blk);
             } else if (cq == 1) {
-                // off-diagonal rows from TMEM: lanes 32pt + r (q rows) and 32pt + 16 + r (k rows)
-                const int r = lane & 15;
-                const bool krow = lane >= 16;
-                const int i = 16 * pt + r;
-                const float bi = sb[i];
-                for (int blk = 0; blk < pt; ++blk) {   // 16 columns per block, all lanes of the warp
-                    uint32_t v[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * pt) << 16) + cGD + gb_off(pt) + 16 * blk, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const float sg = krow ? -bi : 1.f;
-                        uint32_t hi[4], lo[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float x0 = sg * __uint_as_float(v[8 * hh + 2 * e]), x1 = sg * __uint_as_float(v[8 * hh + 2 * e + 1]);
-                            hi[e] = pack_f16(x0, x1);
-                            const float2 hf = unpack_f16(hi[e]);
-                            lo[e] = pack_f16(x0 - hf.x, x1 - hf.y);
-                        }
-                        if (krow) {
-                            sts128(base + kLD + sw128(i, 16 * blk + 8 * hh), make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                        } else {
-                            sts128(base + kAm + sw128(qslot(i), 16 * blk + 8 * hh), make_uint4(hi[0], hi[1], hi[2], hi[3]));
-                            sts128(base + kAm + sw128(kslot(i), 16 * blk + 8 * hh), make_uint4(lo[0], lo[1], lo[2], lo[3]));
-                        }
-                    }
-                }
-                if (!krow) {   // A and its remainder: zeros right of the diagonal block
+                for (int blk = 0; blk < split; ++blk) offdiag(blk);
+                if (lane < 16) {   // A and its remainder: zeros right of the diagonal block
+                    const int i = 16 * pt + lane;
                     for (int cc = 16 * (pt + 1); cc < 64; cc += 8) {
                         sts128(base + kAm + sw128(qslot(i), cc), make_uint4(0, 0, 0, 0));
                         sts128(base + kAm + sw128(kslot(i), cc), make_uint4(0, 0, 0, 0));
