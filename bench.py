@@ -42,8 +42,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # the named workload; a prefill row scales it by its own algorithmic bytes (both kernels move
 # traffic in proportion to the token-heads and units they process)
 PREFILL_TRAFFIC = {
-    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 339158528 + 57549824, "src": "0b922cae9af2ce3e"},
-    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346657000 + 261571584, "src": "96b83a3ec9646b8a"},
+    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 338911744 + 58136576, "src": "cf63d7ad652decde"},
+    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346485000 + 257883904, "src": "5847da13fc9cef6f"},
 }
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture of each
