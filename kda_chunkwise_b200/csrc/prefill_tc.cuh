@@ -493,15 +493,15 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
 #pragma unroll
         for (int e = 0; e < 16; ++e) { v[e] = a[e]; v[16 + e] = b[e]; }
     };
-    // 32 fp32 values as fp16 into row k of an MN-major B operand (columns 32 cq ..)
-    auto store_b32 = [&](uint32_t region, int k, const uint32_t (&v)[32], float sgn) {
+    // 32 fp32 values as fp16 into row k of an MN-major B operand (columns 32 cb ..)
+    auto store_b32 = [&](uint32_t region, int k, int cb, const uint32_t (&v)[32]) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            sts128(region + bmn_off(k, 32 * cq + 8 * j),
-                   make_uint4(pack_f16(sgn * __uint_as_float(v[8 * j]), sgn * __uint_as_float(v[8 * j + 1])),
-                              pack_f16(sgn * __uint_as_float(v[8 * j + 2]), sgn * __uint_as_float(v[8 * j + 3])),
-                              pack_f16(sgn * __uint_as_float(v[8 * j + 4]), sgn * __uint_as_float(v[8 * j + 5])),
-                              pack_f16(sgn * __uint_as_float(v[8 * j + 6]), sgn * __uint_as_float(v[8 * j + 7]))));
+            sts128(region + bmn_off(k, 32 * cb + 8 * j),
+                   make_uint4(pack_f16(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                              pack_f16(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                              pack_f16(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                              pack_f16(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]))));
     };
 
     // ---- 1. pass 1 of chunk cl, in two halves with a CTA barrier between them -----------------------
@@ -796,19 +796,22 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                 }
             }
         }
-        {
+        // the state, 32 columns at a time: fp16 copy of S_c (the B operand of step 7), then
+        // S <- Gamma_C S; quarter 1 also takes quarter 0's columns (those warps invert)
+        if (cq != 0) {
             const float gam = reinterpret_cast<const float *>(sm + kGam)[row];
-            uint32_t v[32];
-            tld32(tq + cS + 32 * cq, v);
-            store_b32(base + kS, row, v, 1.f);   // fp16 S_c: the B operand of step 7
+#pragma unroll 1
+            for (int cb = cq == 1 ? 0 : cq; cb <= cq; ++cb) {
+                uint32_t v[32];
+                tld32(tq + cS + 32 * cb, v);
+                store_b32(base + kS, row, cb, v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gam * __uint_as_float(v[e]));
-            {
+                for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gam * __uint_as_float(v[e]));
                 uint32_t a[16], b[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) { a[e] = v[e]; b[e] = v[16 + e]; }
-                tmem_st16(tq + cS + 32 * cq, a);
-                tmem_st16(tq + cS + 32 * cq + 16, b);
+                tmem_st16(tq + cS + 32 * cb, a);
+                tmem_st16(tq + cS + 32 * cb + 16, b);
             }
         }
         mma_wait();
