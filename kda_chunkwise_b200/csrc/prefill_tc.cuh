@@ -738,9 +738,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (warp == kMmaWarp) {
             if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 96, 0, 0);
+                const uint64_t dg = sdesc(base + kGB, 128, 2048, 0);
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k)
-                    mma_ts(tmem + cGD, tmem + cGA + 8 * k, sdesc(base + kGB + 256 * k, 128, 2048, 0), id, k > 0);
+                    mma_ts(tmem + cGD, tmem + cGA + 8 * k, dg + 16 * k, id, k > 0);
                 umma_commit(bMma);
             }
             __syncwarp();
@@ -909,9 +910,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (warp == kMmaWarp) {
             if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 256, 0, 1);
+                // descriptors advance along K by adding the 16-byte start offset (no carry: every
+                // shared-memory address here is below 2^18)
+                const uint64_t dt = sdesc(base + kT, 16, 1024, 2), dk = sdesc(base + kK, 8192, 1024, 2);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_ss(tmem + cWU, sdesc(base + kT + 32 * k, 16, 1024, 2), sdesc(base + kK + 2048 * k, 8192, 1024, 2), id, k > 0);
+                    mma_ss(tmem + cWU, dt + 2 * k, dk + 128 * k, id, k > 0);
                 umma_commit(bMma);
             }
             __syncwarp();
@@ -936,9 +940,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (warp == kMmaWarp) {
             if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 128, 0, 1);
+                const uint64_t ds = sdesc(base + kS, 2048, 128, 0);
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k)
-                    mma_ts(tmem + cWU + 128, tmem + cWQ + 8 * k, sdesc(base + kS + 4096 * k, 2048, 128, 0), id, 1);
+                    mma_ts(tmem + cWU + 128, tmem + cWQ + 8 * k, ds + 256 * k, id, 1);
                 umma_commit(bMma);
             }
             __syncwarp();
@@ -989,15 +994,17 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
         if (warp == kMmaWarp) {
             if (mma_lead) {
                 constexpr uint32_t id = idesc(128, 128, 1, 1), id2 = idesc(128, 128, 0, 1);
+                const uint64_t da = sdesc(aBuf, 8192, 1024, 2), du = sdesc(base + kL, 2048, 128, 0);
+                const uint64_t dm = sdesc(base + kAm, 16, 1024, 2), dl = sdesc(base + kUlo, 2048, 128, 0);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_ss(tmem + cS, sdesc(aBuf + 2048 * k, 8192, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id, 1);
+                    mma_ss(tmem + cS, da + 128 * k, du + 256 * k, id, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_ss(tmem + cWU + 128, sdesc(base + kAm + 32 * k, 16, 1024, 2), sdesc(base + kL + 4096 * k, 2048, 128, 0), id2, 1);
+                    mma_ss(tmem + cWU + 128, dm + 2 * k, du + 256 * k, id2, 1);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_ss(tmem + cWU + 128, sdesc(base + kAm + 32 * k, 16, 1024, 2), sdesc(base + kUlo + 4096 * k, 2048, 128, 0), id2, 1);
+                    mma_ss(tmem + cWU + 128, dm + 2 * k, dl + 256 * k, id2, 1);
                 umma_commit(bMma);
             }
             __syncwarp();
