@@ -46,6 +46,18 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     return pack_f16(f.x, f.y);
 }
 
+// sigmoid of a pair of bf16 gate logits as 1/2 + tanh(x/2)/2, the tanh on the fp16x2 unit: one
+// MUFU operation per pair instead of four (exp2 and reciprocal per value).  Absolute error at most
+// 2.5e-4 over all bf16 logits, far below the bf16 rounding of the gated output; x beyond the fp16
+// range saturates to 0 or 1 as the sigmoid does.
+__device__ __forceinline__ float2 gate_sigmoid2(uint32_t g) {
+    const float2 x = unpack_bf16(g);
+    uint32_t t;
+    asm("tanh.approx.f16x2 %0, %1;\n" : "=r"(t) : "r"(pack_f16(0.5f * x.x, 0.5f * x.y)));
+    const float2 tf = unpack_f16(t);
+    return make_float2(fmaf(0.5f, tf.x, 0.5f), fmaf(0.5f, tf.y, 0.5f));
+}
+
 // Split x into bf16 hi + lo with hi + lo = x to about 2^-16 relative.
 __device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t &hi, uint32_t &lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);

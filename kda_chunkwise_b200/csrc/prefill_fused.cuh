@@ -835,9 +835,9 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                     for (int e = 0; e < 4; ++e) {
                         float o0 = __uint_as_float(d[8 * j + 2 * e]), o1 = __uint_as_float(d[8 * j + 2 * e + 1]);
                         if (p.gate) {
-                            const float2 ga = unpack_bf16(g4[e]);
-                            o0 *= sigmoid_fast(ga.x);
-                            o1 *= sigmoid_fast(ga.y);
+                            const float2 sg = gate_sigmoid2(g4[e]);
+                            o0 *= sg.x;
+                            o1 *= sg.y;
                         }
                         o[8 * j + 2 * e] = o0;
                         o[8 * j + 2 * e + 1] = o1;

@@ -294,18 +294,6 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 
 __device__ __forceinline__ void bar_all() { named_bar(1, kThreads); }
 
-// sigmoid of a pair of bf16 gate logits as 1/2 + tanh(x/2)/2, the tanh on the fp16x2 unit: one
-// MUFU operation per pair instead of four (exp2 and reciprocal per value).  Absolute error about
-// 3e-4, far below the bf16 rounding of the gated output; x beyond the fp16 range saturates to
-// 0 or 1 as the sigmoid does.
-__device__ __forceinline__ float2 gate_sigmoid2(uint32_t g) {
-    const float2 x = unpack_bf16(g);
-    uint32_t t;
-    asm("tanh.approx.f16x2 %0, %1;\n" : "=r"(t) : "r"(pack_f16(0.5f * x.x, 0.5f * x.y)));
-    const float2 tf = unpack_f16(t);
-    return make_float2(fmaf(0.5f, tf.x, 0.5f), fmaf(0.5f, tf.y, 0.5f));
-}
-
 // ---------------------------------------------------------------------------------------------
 // The solve: T' = (I + L)^-1 diag(beta), given the diagonal inverses D_p = (I + L_pp)^-1 (fp16, on
 // the diagonal blocks of LD), T'_pp = D_p diag(beta_p) (on those of T') and the fp16 blocks -L_pm
