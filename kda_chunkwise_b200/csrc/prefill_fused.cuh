@@ -835,7 +835,7 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                     for (int e = 0; e < 4; ++e) {
                         float o0 = __uint_as_float(d[8 * j + 2 * e]), o1 = __uint_as_float(d[8 * j + 2 * e + 1]);
                         if (p.gate) {
-                            const float2 sg = gate_sigmoid2(g4[e]);
+                            const float2 sg = p.out_f32 ? gate_sigmoid2_f32(g4[e]) : gate_sigmoid2(g4[e]);
                             o0 *= sg.x;
                             o1 *= sg.y;
                         }

@@ -82,10 +82,8 @@ constexpr int kAm = kL + 16384;    // A'' (after pass 2): SW128 [128][64]: fp16 
                                    //   remainder A - fp16(A) in the key slots
 constexpr int kS = 155648;         // fp16 S: B operand, MN-major, no swizzle (K = d_k, N = d_v)
 constexpr int kLD = 188416;        // fp16 [64][64] swizzled: -L below the diagonal blocks, D_p on them;
-                                   //   earlier (with kM) the exchange of the diagonal Gram partial sums,
-                                   //   and before that rows 32-63 of the l table
-constexpr int kLT1 = kLD;          // fp32 l table, rows 32-63 (16 KB, over kLD and kM)
-constexpr int kM = 196608;         // fp16 [3][16][32] block-product scratch of the solve
+                                   //   before that rows 32-63 of the l table
+constexpr int kLT1 = kLD;          // fp32 l table, rows 32-63 (16 KB, up to kLdf)
 constexpr int kLdf = 204800;       // fp32 [4][16][17] diagonal blocks of L
 constexpr int kTot = kLdf + 4 * 16 * 17 * 4;   // fp32 [8][128] half-tile totals of l
 constexpr int kTE = kTot + 4096;   // fp32 [4][128] 2^{r_p}
@@ -300,43 +298,63 @@ __device__ __forceinline__ void bar_all() { named_bar(1, kThreads); }
 // (m < p) in LD:  T'_pq = D_p sum_{m=q}^{p-1} (-L_pm) T'_mq  for p = q + 1, q + 2, ... as 16 x 16
 // products; starting from D_q diag(beta_q) yields T' directly.  Column block q of T' needs only
 // column block q, so warp (q, half) computes its 8 columns of blocks (q + 1, q) .. (3, q) in turn
-// with no barrier.  T' is an SW128 [64][64] tile (the MMA's A operand); its rows are the key slots
-// of a 128-row tile whose query slots are zero.
+// with no barrier.  The chain stays in registers: every -L_pm and D_p fragment is loaded up front,
+// and a product's accumulator (rows g, g + 8, columns 2 t4, 2 t4 + 1) becomes the B fragment of the
+// next product (rows 2 t4, 2 t4 + 1, column g) by an 8 x 8 register transpose.  T' is an SW128
+// [64][64] tile (the MMA's A operand); its rows are the key slots of a 128-row tile whose query
+// slots are zero.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
 }
 
-__device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
-    if (warp >= 6) return;
-    const uint32_t base = smem_u32(sm);
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+
+template <int QB>
+__device__ __forceinline__ void solve_column(uint32_t base, int half, int lane) {
+    constexpr int NP = 3 - QB;   // blocks below the diagonal in column block QB
     const int g = lane >> 2, t4 = lane & 3;
-    const int qb = warp >> 1, half = warp & 1;
-    const uint32_t scr = base + kM + warp * 256;   // [16][8] fp16 product, 16-byte rows
-#pragma unroll 1
-    for (int pb = qb + 1; pb < 4; ++pb) {
+    uint32_t lf[NP][NP][4], df[NP][4];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        const int pb = QB + 1 + p;
+#pragma unroll
+        for (int m = 0; m <= p; ++m) ldsm_x4(lf[p][m], ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * (QB + m), lane));   // -L_pm
+        ldsm_x4(df[p], ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * pb, lane));                                          // D_p
+    }
+    uint32_t tf[NP + 1][2];   // B fragments of T'_mq, m = QB .. 3 (this warp's 8 columns)
+    ldsm_x2_t(tf[0], base + kT + swz<128>(32 * QB + 16 + (lane & 15), 2 * QB + half));
+    const int cc = 16 * QB + 8 * half + 2 * t4;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        const int pb = QB + 1 + p;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int mb = qb; mb < pb; ++mb) {
-            uint32_t af[4], bf[2];
-            ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * mb, lane));                        // -L_pm
-            ldsm_x2_t(bf, base + kT + swz<128>(32 * mb + 16 + (lane & 15), 2 * qb + half));          // T'_mq, 8 columns
-            mma_f16(acc, af, bf[0], bf[1]);
-        }
-        sts32(scr + 16 * g + 4 * t4, pack_f16(acc[0], acc[1]));
-        sts32(scr + 16 * (g + 8) + 4 * t4, pack_f16(acc[2], acc[3]));
-        __syncwarp();
+#pragma unroll
+        for (int m = 0; m <= p; ++m) mma_f16(acc, lf[p][m], tf[m][0], tf[m][1]);
         float tq[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-            uint32_t af[4], bf[2];
-            ldsm_x4(af, ldsm_addr_a<128>(base + kLD, 16 * pb, 16 * pb, lane));   // D_p
-            ldsm_x2_t(bf, scr + 16 * (lane & 15));
-            mma_f16(tq, af, bf[0], bf[1]);
+        mma_f16(tq, df[p], transpose8x8(pack_f16(acc[0], acc[1])), transpose8x8(pack_f16(acc[2], acc[3])));
+        const uint32_t t0 = pack_f16(tq[0], tq[1]), t1 = pack_f16(tq[2], tq[3]);
+        sts32(base + kT + sw128(32 * pb + 16 + g, cc), t0);
+        sts32(base + kT + sw128(32 * pb + 24 + g, cc), t1);
+        if (p + 1 < NP) {
+            tf[p + 1][0] = transpose8x8(t0);
+            tf[p + 1][1] = transpose8x8(t1);
         }
-        const int cc = 16 * qb + 8 * half + 2 * t4;
-        sts32(base + kT + sw128(32 * pb + 16 + g, cc), pack_f16(tq[0], tq[1]));
-        sts32(base + kT + sw128(32 * pb + 24 + g, cc), pack_f16(tq[2], tq[3]));
-        __syncwarp();
+    }
+}
+
+__device__ __forceinline__ void solve(unsigned char *sm, int warp, int lane) {
+    const uint32_t base = smem_u32(sm);
+    const int half = warp & 1;
+    switch (warp >> 1) {
+        case 0: solve_column<0>(base, half, lane); break;
+        case 1: solve_column<1>(base, half, lane); break;
+        case 2: solve_column<2>(base, half, lane); break;
+        default: break;
     }
 }
 
@@ -1027,7 +1045,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_tc_kernel(const __gri
                     o[2 * b] = __uint_as_float(oq[4 * b + 2 * rr]) + __uint_as_float(ok[4 * b + 2 * rr]);
                     o[2 * b + 1] = __uint_as_float(oq[4 * b + 2 * rr + 1]) + __uint_as_float(ok[4 * b + 2 * rr + 1]);
                     if (p.has_gate) {
-                        const float2 sg = gate_sigmoid2(gw[b]);
+                        const float2 sg = p.out_f32 ? gate_sigmoid2_f32(gw[b]) : gate_sigmoid2(gw[b]);
                         o[2 * b] *= sg.x;
                         o[2 * b + 1] *= sg.y;
                     }
