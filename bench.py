@@ -131,9 +131,9 @@ def peaks():
 # source files each kernel is built from (a DRAM traffic figure is reported only while they are
 # unchanged since the ncu capture it came from)
 KERNEL_SOURCES = {
-    "prefill": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh", "prefill_tc.cuh"),
-    "prefill_cluster": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_fused.cuh"),
-    "prefill_unit": ("common.cuh", "mma_frag.cuh", "umma.cuh", "prefill_tc.cuh"),
+    "prefill": ("common.cuh", "mma_frag.cuh", "gate_sigmoid.cuh", "umma.cuh", "prefill_fused.cuh", "prefill_tc.cuh"),
+    "prefill_cluster": ("common.cuh", "mma_frag.cuh", "gate_sigmoid.cuh", "umma.cuh", "prefill_fused.cuh"),
+    "prefill_unit": ("common.cuh", "mma_frag.cuh", "gate_sigmoid.cuh", "umma.cuh", "prefill_tc.cuh"),
     "decode": ("common.cuh", "decode.cuh"),
     "speculative": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "f32x2.cuh", "speculative.cuh"),
     "backward": ("common.cuh", "decode.cuh", "mma_frag.cuh", "async_copy.cuh", "backward.cuh"),

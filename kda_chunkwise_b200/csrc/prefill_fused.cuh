@@ -46,6 +46,7 @@
 
 #include "common.cuh"
 #include "mma_frag.cuh"
+#include "gate_sigmoid.cuh"
 #include "umma.cuh"
 
 namespace kda {

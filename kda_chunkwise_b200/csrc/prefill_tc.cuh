@@ -54,6 +54,7 @@
 
 #include "common.cuh"
 #include "mma_frag.cuh"
+#include "gate_sigmoid.cuh"
 #include "umma.cuh"
 
 namespace kda {
