@@ -43,7 +43,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # traffic in proportion to the token-heads and units they process)
 PREFILL_TRAFFIC = {
     1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 338911744 + 58136576, "src": "cf63d7ad652decde"},
-    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346485000 + 257883904, "src": "5847da13fc9cef6f"},
+    2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346526000 + 257653760, "src": "9a662f478223b97e"},
 }
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture of each

@@ -830,18 +830,23 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             if (i < L) {
                 float o[16];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint32_t g4[4] = {gt[j].x, gt[j].y, gt[j].z, gt[j].w};
+                for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(d[j]);
+                if (p.gate) {   // one branch around each whole loop: the two sigmoids are never both live
+                    const uint32_t gw[8] = {gt[0].x, gt[0].y, gt[0].z, gt[0].w, gt[1].x, gt[1].y, gt[1].z, gt[1].w};
+                    if (p.out_f32) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float o0 = __uint_as_float(d[8 * j + 2 * e]), o1 = __uint_as_float(d[8 * j + 2 * e + 1]);
-                        if (p.gate) {
-                            const float2 sg = p.out_f32 ? gate_sigmoid2_f32(g4[e]) : gate_sigmoid2(g4[e]);
-                            o0 *= sg.x;
-                            o1 *= sg.y;
+                        for (int e = 0; e < 8; ++e) {
+                            const float2 sg = gate_sigmoid2_f32(gw[e]);
+                            o[2 * e] *= sg.x;
+                            o[2 * e + 1] *= sg.y;
                         }
-                        o[8 * j + 2 * e] = o0;
-                        o[8 * j + 2 * e + 1] = o1;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float2 sg = gate_sigmoid2(gw[e]);
+                            o[2 * e] *= sg.x;
+                            o[2 * e + 1] *= sg.y;
+                        }
                     }
                 }
                 const int64_t off = ((t0 + i) * H + h) * DV + col0;
