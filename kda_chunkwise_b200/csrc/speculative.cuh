@@ -45,14 +45,15 @@ struct SpecParams {
 
 // Dynamic shared memory of the verify kernel: the next state (fp32, its global layout), the next
 // unit's raw inputs (bf16 a, k, q [K][DK], v, gate [K][DV]; fp32 beta [K]) and the current unit's
-// derived inputs ({alpha, k, scale q, 0} [K][DK] as float4, v, sigmoid(gate) [K][DV], beta [K],
+// derived inputs ({alpha, alpha, k, k} [K][DK] as float4 and {scale q, scale q} [K][DK] as float2,
+// each pair one operand of the paired fp32 instructions; v, sigmoid(gate) [K][DV], beta [K],
 // k . scale q [K], fp32).
 template <int DK, int DV>
 struct SpecVerifySmem {
     __host__ __device__ static size_t raw_off() { return (size_t)DK * DV * 4; }
     __host__ __device__ static size_t beta_off(int K) { return raw_off() + (size_t)K * (3 * DK + 2 * DV) * 2; }
     __host__ __device__ static size_t derived_off(int K) { return beta_off(K) + (size_t)((K + 3) & ~3) * 4; }
-    __host__ __device__ static size_t bytes(int K) { return derived_off(K) + (size_t)K * (4 * DK + 2 * DV + 2) * 4; }
+    __host__ __device__ static size_t bytes(int K) { return derived_off(K) + (size_t)K * (6 * DK + 2 * DV + 2) * 4; }
 };
 
 // Persistent: a CTA takes units blockIdx.x, blockIdx.x + gridDim.x, ...; while it runs the K token
@@ -72,8 +73,9 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
     const uint16_t *r_a = reinterpret_cast<const uint16_t *>(spec_dyn + SL::raw_off());
     const uint16_t *r_k = r_a + K * DK, *r_q = r_k + K * DK, *r_v = r_q + K * DK, *r_g = r_v + K * DV;
     const float *r_beta = reinterpret_cast<const float *>(spec_dyn + SL::beta_off(K));
-    float4 *s_akq = reinterpret_cast<float4 *>(spec_dyn + SL::derived_off(K));   // {alpha, k, scale q, 0}
-    float *s_v = reinterpret_cast<float *>(s_akq + K * DK), *s_sg = s_v + K * DV;
+    float4 *s_ak = reinterpret_cast<float4 *>(spec_dyn + SL::derived_off(K));   // {alpha, alpha, k, k}
+    float2 *s_qq = reinterpret_cast<float2 *>(s_ak + K * DK);                   // {scale q, scale q}
+    float *s_v = reinterpret_cast<float *>(s_qq + K * DK), *s_sg = s_v + K * DV;
     float *s_b = s_sg + K * DV, *s_kqt = s_b + K;
     // per token: the row groups' partial column sums, then the sums ([r or p][column quad])
     __shared__ float4 s_red[2][RPP][LPR];
@@ -115,9 +117,12 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
 #pragma unroll
         for (int m = 0; m < NR; ++m) S[m] = reinterpret_cast<const ulonglong2 *>(sS)[(rg + m * RPP) * LPR + cq];
         const float expA = expf(p.A_log[h]);
-        for (int e = tid; e < K * DK; e += kThreads)
-            s_akq[e] = make_float4(__expf(log_decay(bf16_to_f32(r_a[e]), expA)), bf16_to_f32(r_k[e]),
-                                   p.scale * bf16_to_f32(r_q[e]), 0.f);
+        for (int e = tid; e < K * DK; e += kThreads) {
+            const float al = __expf(log_decay(bf16_to_f32(r_a[e]), expA)), kv = bf16_to_f32(r_k[e]);
+            const float qv = p.scale * bf16_to_f32(r_q[e]);
+            s_ak[e] = make_float4(al, al, kv, kv);
+            s_qq[e] = make_float2(qv, qv);
+        }
         for (int e = tid; e < K * DV; e += kThreads) {
             s_v[e] = bf16_to_f32(r_v[e]);
             if (p.gate) s_sg[e] = sigmoid_fast(bf16_to_f32(r_g[e]));
@@ -127,10 +132,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
         for (int t = tid >> 5; t < K; t += kThreads / 32) {   // k . scale q per token, as the decode step
             const int lane = tid & 31;
             float acc = 0.f;
-            for (int i = lane; i < DK; i += 32) {
-                const float4 akq = s_akq[t * DK + i];
-                acc = fmaf(akq.y, akq.z, acc);
-            }
+            for (int i = lane; i < DK; i += 32) acc = fmaf(s_ak[t * DK + i].z, s_qq[t * DK + i].x, acc);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
             if (lane == 0) s_kqt[t] = acc;
@@ -144,12 +146,12 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
                 const int row = rg + m * RPP;
-                const float4 akq = s_akq[t * DK + row];
-                const f32x2 al = f2_splat(akq.x), kk = f2_splat(akq.y), qq = f2_splat(akq.z);
-                S[m].x = f2_mul(S[m].x, al);
-                S[m].y = f2_mul(S[m].y, al);
-                r.x = f2_fma(kk, S[m].x, r.x);
-                r.y = f2_fma(kk, S[m].y, r.y);
+                const ulonglong2 ak = reinterpret_cast<const ulonglong2 *>(s_ak)[t * DK + row];   // (alpha, alpha), (k, k)
+                const f32x2 qq = reinterpret_cast<const f32x2 *>(s_qq)[t * DK + row];
+                S[m].x = f2_mul(S[m].x, ak.x);
+                S[m].y = f2_mul(S[m].y, ak.x);
+                r.x = f2_fma(ak.y, S[m].x, r.x);
+                r.y = f2_fma(ak.y, S[m].y, r.y);
                 pq.x = f2_fma(qq, S[m].x, pq.x);
                 pq.y = f2_fma(qq, S[m].y, pq.y);
             }
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_verify_kernel(const SpecPar
             const f32x2 u01 = f2_pack(u4.x, u4.y), u23 = f2_pack(u4.z, u4.w);
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
-                const f32x2 kk = f2_splat(s_akq[t * DK + rg + m * RPP].y);
+                const f32x2 kk = reinterpret_cast<const f32x2 *>(s_ak)[2 * (t * DK + rg + m * RPP) + 1];   // (k, k)
                 S[m].x = f2_fma(kk, u01, S[m].x);
                 S[m].y = f2_fma(kk, u23, S[m].y);
             }
