@@ -42,7 +42,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # the named workload; a prefill row scales it by its own algorithmic bytes (both kernels move
 # traffic in proportion to the token-heads and units they process)
 PREFILL_TRAFFIC = {
-    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 338911744 + 58136576, "src": "cf63d7ad652decde"},
+    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 338926080 + 56687616, "src": "c6f030b6473ca358"},
     2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346526000 + 257653760, "src": "9a662f478223b97e"},
 }
 
@@ -51,10 +51,10 @@ PREFILL_TRAFFIC = {
 # capture time.  Reported only while the sources are unchanged.
 NCU_TRAFFIC = {
     "decode_N256_H64_d128_512steps": {"bytes_per_launch": 1094800000 + 1016000000, "src": "6184bb076c425fa7"},
-    # one verify launch plus one commit launch: the mean of the timed rounds of the captured run
-    # (commit's bytes depend on how many sequences accepted at least one token)
-    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1160200000 + 47250000 + 892350000 + 794300000,
-                              "src": "eb388ca15bf43403"},
+    # one verify launch plus one commit launch (the fourth round of the captured run; commit's
+    # bytes depend on how many sequences accepted at least one token)
+    "spec_N256_H64_d128_K4": {"bytes_per_launch": 1158062080 + 49587456 + 930634496 + 830093568,
+                              "src": "75fe6eba2414bb31"},
     # kda_chunk_bwd on the prefill workload (ncu prints these two counters to five digits)
     "bwd_prefill_B1_H32_T8192_d128": {"bytes_per_launch": 1.2989e9 + 2.5685e9, "src": "9ec2178bcf630624"},
 }

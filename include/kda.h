@@ -369,7 +369,9 @@ KDA_API uint64_t kda_launch_count(void);
  * both kernels compute the same chunkwise form of "Kimi K3 · Lesson 3 of 14"; they differ only in how
  * the work is spread over the GPU.)
  *   path 0: chosen from the shapes (the default): one CTA per (sequence, head) unit when the units
- *           are more than three quarters of the SM count, else the cluster kernel;
+ *           are more than twice the clusters of the cluster kernel that fit on the device at once
+ *           (queried once with cudaOccupancyMaxActiveClusters: 32 on a 148-SM B200, so more than
+ *           64 units), else the cluster kernel;
  *   path 1: the cluster kernel (a unit's chunks spread over d_v/32 CTAs, chunk records in the
  *           caller's workspace);
  *   path 2: one CTA per unit, every intermediate on chip (no workspace).

@@ -135,17 +135,50 @@ int device_sm_count() {
     return sms;
 }
 
+// Clusters of the d = 128 cluster kernel (four CTAs each) that fit on the device at once: 32 on a
+// 148-SM B200, where a cluster must sit inside one GPC.  Queried once; without a device (or if the
+// query fails) the B200 figure scaled by the SM count.
+int64_t prefill_cluster_capacity() {
+    static std::atomic<int> cached{0};
+    int c = cached.load(std::memory_order_relaxed);
+    if (c > 0) return c;
+    constexpr int G = 128 / kda::kSlab;
+    const int smem = kda::FusedSmem<128, 128>::kBytes;
+    int n = 0;
+    if (cudaFuncSetAttribute(kda::kda_prefill_fused_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(G);
+        cfg.blockDim = dim3(kda::kFusedThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = G;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kda::kda_prefill_fused_kernel<128, 128>, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();   // a failed query leaves no sticky error behind
+    if (n <= 0) n = std::max(1, device_sm_count() * 32 / 148);
+    cached.store(n, std::memory_order_relaxed);
+    return n;
+}
+
 // The per-unit kernel keeps each unit on one SM (no workspace, no traffic between SMs); the
-// cluster kernel spreads a unit's chunks over four SMs and runs a unit about 3.2 times faster, but
-// does about 0.8 times the work per SM.  So the cluster kernel wins while it needs at most three
-// waves of four-SM units (units <= 3/4 of the SMs), the per-unit kernel from there on.
-// `path` overrides the process-wide setting when non-zero.
+// cluster kernel spreads a unit's chunks over four SMs and runs a unit about 2.4 times faster
+// (B200, d = 128: ~3.4 against ~8.3 us per 64-token chunk), but only C units run at once (C =
+// prefill_cluster_capacity(), 32 on B200) against one unit per SM for the per-unit kernel.  So the
+// cluster kernel wins while its units need at most two waves (units <= 2 C), the per-unit kernel
+// from there on (measured on equal-length batches: 64 units 0.44 against 0.54 ms, 74 units 0.65
+// against 0.54 ms).  `path` overrides the process-wide setting when non-zero.
 bool use_tc_prefill(int64_t units, int d_k, int d_v, int path = 0) {
     if (d_k != 128 || d_v != 128) return false;
     if (g_inject_stall.load(std::memory_order_relaxed)) return false;   // the injection targets the cluster kernel
     const int forced = path ? path : g_prefill_path.load(std::memory_order_relaxed);
     if (forced) return forced == 2;
-    return units * 4 > (int64_t)device_sm_count() * 3;
+    return units > 2 * prefill_cluster_capacity();
 }
 
 kda_status launch_prefill_tc(const void *q, const void *k, const void *v, const void *a,

@@ -56,13 +56,17 @@ def test_workspace_sizes():
 
 
 def test_prefill_kernel_choice_by_units():
-    # The cluster kernel (1) while the units are at most 3/4 of the SM count, the per-unit kernel (2)
-    # beyond; 148 SMs on B200, and the library assumes 148 when it cannot query a device.
+    # The cluster kernel (1) while its units need at most two waves of four-CTA clusters, the
+    # per-unit kernel (2) beyond.  A 148-SM B200 holds 32 such clusters at once (the library's
+    # figure for 148 SMs when it cannot query a device), so the edge is 64 units; other devices
+    # get their own figure from the occupancy query.
     import torch
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
-    edge = sms * 3 // 4
-    assert kda.kda_prefill_path(edge, 128, 128) == 1
-    assert kda.kda_prefill_path(edge + 1, 128, 128) == 2
+    if sms == 148:
+        assert kda.kda_prefill_path(64, 128, 128) == 1
+        assert kda.kda_prefill_path(65, 128, 128) == 2
+    assert kda.kda_prefill_path(1, 128, 128) == 1
+    assert kda.kda_prefill_path(4 * sms, 128, 128) == 2
     assert kda.kda_prefill_path(4096, 64, 128) == 1      # other head sizes: the cluster kernel only
     kda.kda_set_prefill_path(2)
     try:

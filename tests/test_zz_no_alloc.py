@@ -60,11 +60,11 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
 
 
 def test_noalloc_runs_the_per_unit_kernel_when_cluster_records_would_not_fit():
-    # 2 sequences x 40 heads = 80 units: by shape the cluster kernel (at most 3/4 of the SM count),
-    # whose records (80 x 648 KiB) exceed the 32 MiB array; with the kernel left to the shapes the
+    # 2 sequences x 28 heads = 56 units: by shape the cluster kernel (at most 64 units on B200),
+    # whose records (56 x 648 KiB) exceed the 32 MiB array; with the kernel left to the shapes the
     # call runs the per-unit kernel instead, so it must equal kda_chunk_fwd on that kernel bit for bit.
     import kda_chunkwise_b200 as kda
-    w = KI.Workload("noalloc80", (200, 131), 40, 128, 128, A_log="uniform", init_state="normal_0.02", seed=22)
+    w = KI.Workload("noalloc56", (200, 131), 28, 128, 128, A_log="uniform", init_state="normal_0.02", seed=22)
     inp = KI.make_inputs(w, "cuda")
     args = (inp["q"], inp["k"], inp["v"], inp["a"], inp["beta"], inp["A_log"], inp["cu_seqlens"])
     assert kda.kda_prefill_path(w.num_seqs * w.H, 128, 128) == 1
