@@ -370,8 +370,8 @@ KDA_API uint64_t kda_launch_count(void);
  * the work is spread over the GPU.)
  *   path 0: chosen from the shapes (the default): one CTA per (sequence, head) unit when the units
  *           are more than twice the clusters of the cluster kernel that fit on the device at once
- *           (queried once with cudaOccupancyMaxActiveClusters: 32 on a 148-SM B200, so more than
- *           64 units), else the cluster kernel;
+ *           (queried once with cudaOccupancyMaxActiveClusters: 33 on a 148-SM B200, so more than
+ *           66 units), else the cluster kernel;
  *   path 1: the cluster kernel (a unit's chunks spread over d_v/32 CTAs, chunk records in the
  *           caller's workspace);
  *   path 2: one CTA per unit, every intermediate on chip (no workspace).

@@ -135,9 +135,10 @@ int device_sm_count() {
     return sms;
 }
 
-// Clusters of the d = 128 cluster kernel (four CTAs each) that fit on the device at once: 32 on a
-// 148-SM B200, where a cluster must sit inside one GPC.  Queried once; without a device (or if the
-// query fails) the B200 figure scaled by the SM count.
+// Clusters of the d = 128 cluster kernel (four CTAs each) that fit on the device at once: 33 on a
+// 148-SM B200 (a cluster must sit inside one GPC; a probe launch confirms 33 run together and 36
+// take two waves).  Queried once; without a device (or if the query fails) the B200 figure scaled
+// by the SM count.
 int64_t prefill_cluster_capacity() {
     static std::atomic<int> cached{0};
     int c = cached.load(std::memory_order_relaxed);
@@ -161,7 +162,7 @@ int64_t prefill_cluster_capacity() {
         if (cudaOccupancyMaxActiveClusters(&n, kda::kda_prefill_fused_kernel<128, 128>, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();   // a failed query leaves no sticky error behind
-    if (n <= 0) n = std::max(1, device_sm_count() * 32 / 148);
+    if (n <= 0) n = std::max(1, device_sm_count() * 33 / 148);
     cached.store(n, std::memory_order_relaxed);
     return n;
 }
@@ -169,7 +170,7 @@ int64_t prefill_cluster_capacity() {
 // The per-unit kernel keeps each unit on one SM (no workspace, no traffic between SMs); the
 // cluster kernel spreads a unit's chunks over four SMs and runs a unit about 2.4 times faster
 // (B200, d = 128: ~3.4 against ~8.3 us per 64-token chunk), but only C units run at once (C =
-// prefill_cluster_capacity(), 32 on B200) against one unit per SM for the per-unit kernel.  So the
+// prefill_cluster_capacity(), 33 on B200) against one unit per SM for the per-unit kernel.  So the
 // cluster kernel wins while its units need at most two waves (units <= 2 C), the per-unit kernel
 // from there on (measured on equal-length batches: 64 units 0.44 against 0.54 ms, 74 units 0.65
 // against 0.54 ms).  `path` overrides the process-wide setting when non-zero.

@@ -57,16 +57,18 @@ def test_workspace_sizes():
 
 def test_prefill_kernel_choice_by_units():
     # The cluster kernel (1) while its units need at most two waves of four-CTA clusters, the
-    # per-unit kernel (2) beyond.  A 148-SM B200 holds 32 such clusters at once (the library's
-    # figure for 148 SMs when it cannot query a device), so the edge is 64 units; other devices
-    # get their own figure from the occupancy query.
+    # per-unit kernel (2) beyond: one switch, at twice the clusters that fit at once.  A 148-SM
+    # B200 holds 33 (the occupancy query; 33 is also the library's figure for 148 SMs when it
+    # cannot query a device), so the switch is after 66 units; a cluster must sit inside one GPC,
+    # so the figure lies below a quarter of the SM count.
     import torch
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
-    if sms == 148:
-        assert kda.kda_prefill_path(64, 128, 128) == 1
-        assert kda.kda_prefill_path(65, 128, 128) == 2
-    assert kda.kda_prefill_path(1, 128, 128) == 1
-    assert kda.kda_prefill_path(4 * sms, 128, 128) == 2
+    paths = [kda.kda_prefill_path(u, 128, 128) for u in range(1, 4 * sms + 1)]
+    edge = paths.index(2)   # units <= edge run the cluster kernel
+    assert set(paths[:edge]) == {1} and set(paths[edge:]) == {2}
+    assert edge % 2 == 0 and 2 <= edge <= 2 * (sms // 4)
+    if not torch.cuda.is_available():
+        assert edge == 66
     assert kda.kda_prefill_path(4096, 64, 128) == 1      # other head sizes: the cluster kernel only
     kda.kda_set_prefill_path(2)
     try:

@@ -60,7 +60,7 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
 
 
 def test_noalloc_runs_the_per_unit_kernel_when_cluster_records_would_not_fit():
-    # 2 sequences x 28 heads = 56 units: by shape the cluster kernel (at most 64 units on B200),
+    # 2 sequences x 28 heads = 56 units: by shape the cluster kernel (at most 66 units on B200),
     # whose records (56 x 648 KiB) exceed the 32 MiB array; with the kernel left to the shapes the
     # call runs the per-unit kernel instead, so it must equal kda_chunk_fwd on that kernel bit for bit.
     import kda_chunkwise_b200 as kda
