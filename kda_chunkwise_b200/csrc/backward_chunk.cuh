@@ -89,27 +89,48 @@ __device__ __forceinline__ void bc_gemm(const float *A, int lda, const float *B,
     float acc[NPW][4];
 #pragma unroll
     for (int u = 0; u < NPW; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+    // the next k-slice is read into registers while the current one is multiplied, so the global
+    // (L2) latency of the operands overlaps the products
+    constexpr int EA = M * kBcKs, EB = kBcKs * N;
+    constexpr int NA = (EA + kBcThreads - 1) / kBcThreads, NB = (EB + kBcThreads - 1) / kBcThreads;
+    float ra[NA], rb[NB];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int q = 0; q < NA; ++q) {
+            const int e = threadIdx.x + q * kBcThreads;
+            if (e < EA) ra[q] = TA ? A[(size_t)(k0 + e / M) * lda + e % M] : A[(size_t)(e / kBcKs) * lda + k0 + e % kBcKs];
+        }
+#pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            const int e = threadIdx.x + q * kBcThreads;
+            if (e < EB) rb[q] = TB ? B[(size_t)(e / kBcKs) * ldb + k0 + e % kBcKs] : B[(size_t)(k0 + e / N) * ldb + e % N];
+        }
+    };
+    auto stage_slice = [&]() {
+#pragma unroll
+        for (int q = 0; q < NA; ++q) {
+            const int e = threadIdx.x + q * kBcThreads;
+            if (e < EA) {
+                if (TA) As[(e % M) * LA + e / M] = ra[q];
+                else As[(e / kBcKs) * LA + e % kBcKs] = ra[q];
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            const int e = threadIdx.x + q * kBcThreads;
+            if (e < EB) {
+                if (TB) Bs[(e % kBcKs) * LB + e / kBcKs] = rb[q];
+                else Bs[(e / N) * LB + e % N] = rb[q];
+            }
+        }
+    };
+    __syncthreads();   // on entry: the operands are written
+    fetch(0);
     for (int k0 = 0; k0 < K; k0 += kBcKs) {
-        __syncthreads();   // the previous slice is consumed; on entry, the operands are written
-        for (int e = threadIdx.x; e < M * kBcKs; e += kBcThreads) {
-            if (TA) {
-                const int kk = e / M, i = e % M;
-                As[i * LA + kk] = A[(size_t)(k0 + kk) * lda + i];
-            } else {
-                const int i = e / kBcKs, kk = e % kBcKs;
-                As[i * LA + kk] = A[(size_t)i * lda + k0 + kk];
-            }
-        }
-        for (int e = threadIdx.x; e < kBcKs * N; e += kBcThreads) {
-            if (TB) {
-                const int j = e / kBcKs, kk = e % kBcKs;
-                Bs[kk * LB + j] = B[(size_t)j * ldb + k0 + kk];
-            } else {
-                const int kk = e / N, j = e % N;
-                Bs[kk * LB + j] = B[(size_t)(k0 + kk) * ldb + j];
-            }
-        }
+        if (k0 > 0) __syncthreads();   // the previous slice is consumed
+        stage_slice();
         __syncthreads();
+        if (k0 + kBcKs < K) fetch(k0 + kBcKs);
 #pragma unroll
         for (int ks = 0; ks < kBcKs; ks += 8) {
             uint32_t ah[4], al[4];
