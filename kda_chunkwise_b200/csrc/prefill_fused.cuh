@@ -44,6 +44,8 @@
 // CTA leaves while another may still arrive on its barriers.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "mma_frag.cuh"
 #include "gate_sigmoid.cuh"
@@ -827,32 +829,24 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
             tmem_ld16(tq + cD + 16 * half, d);
             tmem_wait_ld();
             const int i = row - 64;
-            if (i < L) {
+            // gate and store, one copy per output type (the two never share registers)
+            auto emit = [&](auto f32_tag) {
+                constexpr bool F32 = decltype(f32_tag)::value;
                 float o[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(d[j]);
-                if (p.gate) {   // one branch around each whole loop: the two sigmoids are never both live
+                if (p.gate) {
                     const uint32_t gw[8] = {gt[0].x, gt[0].y, gt[0].z, gt[0].w, gt[1].x, gt[1].y, gt[1].z, gt[1].w};
-                    if (p.out_f32) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float2 sg = gate_sigmoid2_f32(gw[e]);
-                            o[2 * e] *= sg.x;
-                            o[2 * e + 1] *= sg.y;
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float2 sg = gate_sigmoid2(gw[e]);
-                            o[2 * e] *= sg.x;
-                            o[2 * e + 1] *= sg.y;
-                        }
+                    for (int e = 0; e < 8; ++e) {
+                        const float2 sg = F32 ? gate_sigmoid2_f32(gw[e]) : gate_sigmoid2(gw[e]);
+                        o[2 * e] *= sg.x;
+                        o[2 * e + 1] *= sg.y;
                     }
                 }
+                if (!p.out) return;   // no outputs wanted (the segment maps)
                 const int64_t off = ((t0 + i) * H + h) * DV + col0;
-                if (!p.out) {
-                    // no outputs wanted (the segment maps)
-                } else if (p.out_f32) {
+                if constexpr (F32) {
                     float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) op[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
@@ -863,6 +857,10 @@ __device__ __forceinline__ void fused_consumer(const FusedParams &p, unsigned ch
                         op[j] = make_uint4(pack_bf16(o[8 * j], o[8 * j + 1]), pack_bf16(o[8 * j + 2], o[8 * j + 3]),
                                            pack_bf16(o[8 * j + 4], o[8 * j + 5]), pack_bf16(o[8 * j + 6], o[8 * j + 7]));
                 }
+            };
+            if (i < L) {
+                if (p.out_f32) emit(std::true_type{});
+                else emit(std::false_type{});
             }
             if (has_next) load_gate(c + 1);
         }
