@@ -42,7 +42,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # the named workload; a prefill row scales it by its own algorithmic bytes (both kernels move
 # traffic in proportion to the token-heads and units they process)
 PREFILL_TRAFFIC = {
-    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 338926080 + 56687616, "src": "c6f030b6473ca358"},
+    1: {"workload": "prefill_B1_H32_T8192_d128", "bytes_per_launch": 338915584 + 56528384, "src": "c98d8e5f0ae92cd4"},
     2: {"workload": "saturated_B2_H32_T16384_d128", "bytes_per_launch": 1346526000 + 257653760, "src": "9a662f478223b97e"},
 }
 
