@@ -137,8 +137,9 @@ int device_sm_count() {
 
 // Clusters of the d = 128 cluster kernel (four CTAs each) that fit on the device at once: 33 on a
 // 148-SM B200 (a cluster must sit inside one GPC; a probe launch confirms 33 run together and 36
-// take two waves).  Queried once; without a device (or if the query fails) the B200 figure scaled
-// by the SM count.
+// take two waves).  Queried once per process, on the device current at the first call (the GPUs of
+// one node are alike); without a device (or if the query fails) the B200 figure scaled by the SM
+// count.
 int64_t prefill_cluster_capacity() {
     static std::atomic<int> cached{0};
     int c = cached.load(std::memory_order_relaxed);
